@@ -1,0 +1,408 @@
+"""Pins for the float64 oracle: each check ties an oracle function to something
+other than itself -- a closed form, an invariant, a hand-derived fixture, an
+independent brute force or a library routine -- so that a dropped term, a wrong
+sign or index or a transposed operand fails here.  CPU only."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- a1 PE
+
+def test_pe1d_closed_forms():
+    L, F = 64, 8
+    pe = oracle.pe1d(L, F, True)
+    assert pe.shape == (L, 1 + 2 * F)
+    # t = 0: [0, cos 0 = 1 (F times), sin 0 = 0 (F times)]
+    np.testing.assert_array_equal(pe[0], np.r_[0.0, np.ones(F), np.zeros(F)])
+    # t = L/4: angle pi*j/2 -> cos: 0,-1,0,1,...; sin: 1,0,-1,0,...
+    j = np.arange(1, F + 1)
+    cos_q = np.array([[1, 0, -1, 0][k % 4] for k in j], float)
+    sin_q = np.array([[0, 1, 0, -1][k % 4] for k in j], float)
+    np.testing.assert_allclose(pe[L // 4], np.r_[0.25, cos_q, sin_q], atol=1e-15)
+    # all t against numpy's cos/sin of the unreduced angle
+    t = np.arange(L)[:, None]
+    ang = 2 * np.pi * j[None, :] * t / L
+    np.testing.assert_allclose(pe[:, 1:1 + F], np.cos(ang), atol=1e-13)
+    np.testing.assert_allclose(pe[:, 1 + F:], np.sin(ang), atol=1e-13)
+    np.testing.assert_array_equal(pe[:, 0], np.arange(L) / L)
+    assert oracle.pe1d(L, F, False).shape == (L, 2 * F)
+
+
+# ---------------------------------------------------------------- a2 filter MLP
+
+def _np_mlp(x, Ws, bs, gamma=None, beta=None):
+    a = x
+    for l, (W, b) in enumerate(zip(Ws, bs)):
+        a = a @ np.asarray(W, np.float64).T + np.asarray(b, np.float64)
+        if l < len(Ws) - 1:
+            if l == 0 and gamma is not None:
+                a = (1.0 + gamma) * a + beta
+            a = a / (1.0 + np.exp(-a))
+    return a
+
+
+def test_filter_gen_constant_output():
+    L, F, nout = 32, 4, 5
+    rng = np.random.default_rng(0)
+    Ws = [rng.standard_normal((16, 9)), np.zeros((nout, 16))]
+    c = rng.standard_normal(nout)
+    bs = [rng.standard_normal(16), c]
+    h0 = oracle.filter_gen_1d(L, F, True, Ws, bs, np.zeros(nout))
+    np.testing.assert_array_equal(h0, np.repeat(c[:, None], L, axis=1))
+    alpha = np.array([0.0, 0.5, 1.0, 2.0, 3.0])
+    h = oracle.filter_gen_1d(L, F, True, Ws, bs, alpha)
+    expect = c[:, None] * np.exp(-alpha[:, None] * np.arange(L)[None, :] / L)
+    np.testing.assert_allclose(h, expect, rtol=1e-15, atol=0)
+
+
+@pytest.mark.parametrize("hidden", [[32], [64, 64]])
+def test_filter_gen_vs_numpy_mlp(hidden):
+    L, F, nout = 128, 8, 24
+    rng = np.random.default_rng(1)
+    widths = [1 + 2 * F] + hidden + [nout]
+    Ws = [rng.uniform(-.5, .5, (widths[i + 1], widths[i])) for i in range(len(widths) - 1)]
+    bs = [rng.uniform(-.5, .5, widths[i + 1]) for i in range(len(widths) - 1)]
+    alpha = rng.uniform(0.3, 5, nout)
+    h = oracle.filter_gen_1d(L, F, True, Ws, bs, alpha)
+    t = np.arange(L)
+    j = np.arange(1, F + 1)
+    pe = np.concatenate([(t / L)[:, None], np.cos(2 * np.pi * np.outer(t, j) / L),
+                         np.sin(2 * np.pi * np.outer(t, j) / L)], axis=1)
+    ref = _np_mlp(pe, Ws, bs) * np.exp(-np.outer(t, alpha) / L)
+    np.testing.assert_allclose(h, ref.T, rtol=1e-12, atol=1e-13)
+
+
+def test_filter_gen_3d_points():
+    g, F, nout = 4, 4, 6
+    S = 2 * g
+    rng = np.random.default_rng(2)
+    widths = [6 * F, 16, nout]
+    Ws = [rng.uniform(-.5, .5, (widths[i + 1], widths[i])) for i in range(2)]
+    bs = [rng.uniform(-.5, .5, widths[i + 1]) for i in range(2)]
+    gamma, beta = 0.1 * rng.standard_normal(16), 0.1 * rng.standard_normal(16)
+    alpha = rng.uniform(0.5, 3, nout)
+    idx = np.arange(S ** 3)
+    out = oracle.filter_gen_3d_points(g, False, F, Ws, bs, gamma, beta, alpha, idx)
+    ix, iy, iz = idx // (S * S), (idx // S) % S, idx % S
+    r = np.stack([np.where(a < S // 2, a, a - S) for a in (ix, iy, iz)], axis=1)
+    inside = np.all(np.abs(r) <= g - 1, axis=1)
+    # the index S/2 on any axis (offset -g) is outside the support
+    assert not inside[(ix == S // 2) | (iy == S // 2) | (iz == S // 2)].any()
+    jj = np.arange(1, F + 1)
+    feats = []
+    for a in range(3):
+        ang = np.pi * np.outer(r[:, a], jj) / g
+        feats += [np.cos(ang), np.sin(ang)]
+    pe = np.concatenate(feats, axis=1)
+    rn = np.sqrt((r.astype(float) ** 2).sum(1)) / g
+    ref = _np_mlp(pe, Ws, bs, gamma, beta) * np.exp(-np.outer(rn, alpha))
+    ref[~inside] = 0
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-13)
+    # circular grid: every index is in the support
+    outc = oracle.filter_gen_3d_points(g, True, F, Ws, bs, gamma, beta, alpha, np.arange(g ** 3))
+    assert np.all(np.abs(outc).sum(1) > 0)
+
+
+# ---------------------------------------------------------------- a3 spectrum
+
+def test_dft_real_rows():
+    L, n = 16, 32
+    h = np.zeros((3, L))
+    h[0, 0] = 1.0
+    h[1, 5] = 2.0
+    h[2] = np.random.default_rng(3).standard_normal(L)
+    H = oracle.dft_real_rows(h, n)
+    k = np.arange(n // 2 + 1)
+    np.testing.assert_allclose(H[0], np.ones(n // 2 + 1), atol=1e-15)
+    np.testing.assert_allclose(H[1], 2 * np.exp(-2j * np.pi * k * 5 / n), atol=1e-14)
+    np.testing.assert_allclose(H, np.fft.rfft(h, n=n, axis=-1), atol=1e-12)
+
+
+# ---------------------------------------------------------------- a4-a7 causal conv
+
+def test_causal_conv_delta_and_skip():
+    u = np.random.default_rng(4).standard_normal(50)
+    h = np.zeros(50); h[0] = 1.0
+    np.testing.assert_array_equal(oracle.causal_conv(h, u), u)
+    np.testing.assert_allclose(oracle.causal_conv(h, u, 0.25), 1.25 * u, rtol=1e-15)
+
+
+def test_causal_conv_geometric_closed_form():
+    L = 300
+    rho = math.exp(-2.0 / L)
+    h = rho ** np.arange(L)
+    c = oracle.causal_conv(h, np.ones(L))
+    t = np.arange(L)
+    np.testing.assert_allclose(c, (1 - rho ** (t + 1)) / (1 - rho), rtol=1e-12)
+    # first-order recurrence for any input
+    u = np.random.default_rng(5).standard_normal(L)
+    c = oracle.causal_conv(h, u)
+    np.testing.assert_allclose(c[1:], rho * c[:-1] + u[1:], rtol=1e-10, atol=1e-12)
+    assert c[0] == u[0]
+
+
+def test_causal_conv_linearity_and_shift():
+    rng = np.random.default_rng(6)
+    L = 64
+    h, h2, u1, u2 = rng.standard_normal((4, L))
+    a, b = 1.5, -0.75
+    np.testing.assert_allclose(oracle.causal_conv(h, a * u1 + b * u2),
+                               a * oracle.causal_conv(h, u1) + b * oracle.causal_conv(h, u2),
+                               atol=1e-12)
+    np.testing.assert_allclose(oracle.causal_conv(a * h + b * h2, u1),
+                               a * oracle.causal_conv(h, u1) + b * oracle.causal_conv(h2, u1),
+                               atol=1e-12)
+    s = 7
+    us = np.r_[np.zeros(s), u1[:-s]]
+    np.testing.assert_allclose(oracle.causal_conv(h, us)[s:], oracle.causal_conv(h, u1)[:-s],
+                               atol=1e-12)
+    assert np.all(oracle.causal_conv(h, us)[:s] == 0)
+
+
+@pytest.mark.parametrize("L", [1, 2, 5, 16, 33, 64])
+def test_causal_conv_bruteforce_toeplitz(L):
+    rng = np.random.default_rng(L)
+    h = rng.integers(-4, 5, L).astype(float)
+    u = rng.integers(-4, 5, L).astype(float)
+    T = np.zeros((L, L))
+    for i in range(L):
+        for j in range(i + 1):
+            T[i, j] = h[i - j]
+    np.testing.assert_array_equal(oracle.causal_conv(h, u, 3.0), T @ u + 3.0 * u)
+
+
+def test_golden_causal_conv_gate():
+    gd = _golden("causal_conv_gate_L4.json")
+    c = oracle.causal_conv(gd["h"], gd["v"], gd["D"])
+    np.testing.assert_array_equal(c, gd["c"])
+    v = np.array(gd["v"], float).reshape(1, 1, 4)
+    x1 = np.array(gd["x1"], float).reshape(1, 1, 4)
+    h = np.array(gd["h"], float).reshape(1, 1, 4)
+    y = oracle.hyena_rows(v, [x1], h, np.array([[gd["D"]]]))
+    np.testing.assert_array_equal(y[0], gd["y"])
+
+
+def test_chain_reductions():
+    rng = np.random.default_rng(7)
+    B, D, L = 2, 3, 40
+    v = rng.standard_normal((B, D, L))
+    h = rng.standard_normal((2, D, L))
+    Dk = rng.standard_normal((2, D))
+    ones = np.ones((B, D, L))
+    # order 2 with x1 = 1 is the convolution plus skip
+    y = oracle.hyena_rows(v, [ones], h[:1], Dk[:1])
+    for b in range(B):
+        for d in range(D):
+            np.testing.assert_allclose(y[b * D + d], oracle.causal_conv(h[0, d], v[b, d], Dk[0, d]),
+                                       rtol=0, atol=0)
+    # order 3 with a delta filter at order 2: y = x2 * (1 + D_2) * z1
+    x1 = rng.standard_normal((B, D, L)); x2 = rng.standard_normal((B, D, L))
+    hd = h.copy(); hd[1] = 0; hd[1, :, 0] = 1
+    z1 = oracle.hyena_rows(v, [x1], h[:1], Dk[:1]).reshape(B, D, L)
+    y3 = oracle.hyena_rows(v, [x1, x2], hd, Dk).reshape(B, D, L)
+    np.testing.assert_allclose(y3, x2 * (1 + Dk[1][None, :, None]) * z1, rtol=1e-14, atol=1e-14)
+    # no skip at all
+    y0 = oracle.hyena_rows(v, [ones], h[:1], None)
+    np.testing.assert_array_equal(y0[0], oracle.causal_conv(h[0, 0], v[0, 0]))
+    # a prefix of the chain depends only on prefixes
+    yp = oracle.hyena_rows(v, [x1, x2], h, Dk, rows=[4], T=17)
+    np.testing.assert_array_equal(yp[0], oracle.hyena_rows(v, [x1, x2], h, Dk)[4, :17])
+
+
+@pytest.mark.parametrize("L", [3, 16, 64])
+def test_chain_bruteforce(L):
+    rng = np.random.default_rng(100 + L)
+    K, D = 3, 2
+    ints = lambda *s: rng.integers(-2, 3, s).astype(float)
+    v, xs, h, Dk = ints(1, D, L), [ints(1, D, L) for _ in range(K)], ints(K, D, L), ints(K, D)
+    y = oracle.hyena_rows(v, xs, h, Dk)
+    for d in range(D):
+        z = v[0, d]
+        for k in range(K):
+            T = np.array([[h[k, d, i - j] if j <= i else 0.0 for j in range(L)] for i in range(L)])
+            z = xs[k][0, d] * (T @ z + Dk[k, d] * z)
+        np.testing.assert_array_equal(y[d], z)
+
+
+def test_conv_gate_samples_match_rows():
+    rng = np.random.default_rng(8)
+    L = 200
+    h, u, x = rng.standard_normal((3, L))
+    ts = np.array([0, 1, 57, 199])
+    s = oracle.conv_gate_samples(h, u, x, 0.3, ts)
+    full = oracle.hyena_rows(u.reshape(1, 1, L), [x.reshape(1, 1, L)], h.reshape(1, 1, L), np.array([[0.3]]))
+    np.testing.assert_allclose(s, full[0, ts], rtol=0, atol=0)
+
+
+# ---------------------------------------------------------------- a9 N-D
+
+def _nd_brute(K, v, circular):
+    g = v.shape
+    S = g if circular else tuple(2 * a for a in g)
+    c = np.zeros(g)
+    for p in np.ndindex(*g):
+        s = 0.0
+        for q in np.ndindex(*g):
+            s += K[tuple((p[a] - q[a]) % S[a] for a in range(3))] * v[q]
+        c[p] = s
+    return c
+
+
+def test_golden_nd():
+    gd = _golden("nd_conv_2cube.json")
+    g = tuple(gd["g"])
+    K = np.zeros(tuple(2 * a for a in g))
+    for i, j, l, val in gd["kernel_entries"]:
+        K[int(i), int(j), int(l)] = val
+    v = np.array(gd["v"], float)
+    pts = np.arange(int(np.prod(g)))
+    c = oracle.nd_conv_points(K, v, None, 0.0, pts).reshape(g)
+    np.testing.assert_array_equal(c, gd["c"])
+
+
+@pytest.mark.parametrize("circular", [False, True])
+def test_nd_bruteforce_and_delta(circular):
+    rng = np.random.default_rng(9)
+    g = (3, 4, 2)
+    S = g if circular else tuple(2 * a for a in g)
+    K = rng.standard_normal(S)
+    v, x1 = rng.standard_normal((2,) + g)
+    pts = np.arange(int(np.prod(g)))
+    y = oracle.nd_conv_points(K, v, x1, 0.5, pts, circular).reshape(g)
+    np.testing.assert_allclose(y, x1 * (_nd_brute(K, v, circular) + 0.5 * v), rtol=1e-13, atol=1e-13)
+    Kd = np.zeros(S); Kd[0, 0, 0] = 1
+    np.testing.assert_array_equal(oracle.nd_conv_points(Kd, v, x1, 0.0, pts, circular).reshape(g), x1 * v)
+
+
+def test_nd_separable():
+    rng = np.random.default_rng(10)
+    g = 5
+    S = 2 * g
+    ks = [rng.standard_normal(2 * g - 1) for _ in range(3)]   # offsets -(g-1)..(g-1)
+    vs = [rng.standard_normal(g) for _ in range(3)]
+    K = np.zeros((S, S, S))
+    for a in range(-(g - 1), g):
+        for b in range(-(g - 1), g):
+            for c in range(-(g - 1), g):
+                K[a % S, b % S, c % S] = ks[0][a + g - 1] * ks[1][b + g - 1] * ks[2][c + g - 1]
+    v = np.einsum("i,j,k->ijk", *vs)
+    y = oracle.nd_conv_points(K, v, None, 0.0, np.arange(g ** 3)).reshape(g, g, g)
+    one_d = [np.convolve(ks[a], vs[a])[g - 1: 2 * g - 1] for a in range(3)]
+    np.testing.assert_allclose(y, np.einsum("i,j,k->ijk", *one_d), rtol=1e-12, atol=1e-12)
+
+
+def test_nd_shift_equivariance():
+    rng = np.random.default_rng(11)
+    g = (6, 6, 6)
+    K = rng.standard_normal((12, 12, 12))
+    v = np.zeros(g); v[:4, :4, :4] = rng.standard_normal((4, 4, 4))
+    vs = np.zeros(g); vs[2:, 1:5, 2:] = v[:4, :4, :4]
+    pts = np.arange(216)
+    a = oracle.nd_conv_points(K, v, None, 0.0, pts).reshape(g)
+    b = oracle.nd_conv_points(K, vs, None, 0.0, pts).reshape(g)
+    np.testing.assert_allclose(b[2:, 1:, 2:], a[:4, :5, :4], rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- a10 spectral gate
+
+def test_golden_spectral_gate():
+    gd = _golden("spectral_gate_n4.json")
+    g = np.array(gd["g_re"]) + 1j * np.array(gd["g_im"])
+    kap = oracle.gate_kernel(g)
+    mixed = oracle.circular_conv_samples(kap, gd["x1"], None, np.arange(4))
+    np.testing.assert_allclose(mixed, gd["mixed"], atol=1e-14)
+    y = oracle.circular_conv_samples(kap, gd["x1"], gd["x2"], np.arange(4))
+    np.testing.assert_allclose(y, gd["y"], atol=1e-14)
+
+
+def test_gate_kernel_special_cases():
+    n = 64
+    nb = n // 2 + 1
+    k = np.arange(nb)
+    kap = oracle.gate_kernel(np.ones(nb))
+    np.testing.assert_allclose(kap, np.r_[1.0, np.zeros(n - 1)], atol=1e-14)
+    for s in (1, 5, 32, 63):
+        kap = oracle.gate_kernel(np.exp(-2j * np.pi * k * s / n))
+        e = np.zeros(n); e[s] = 1
+        np.testing.assert_allclose(kap, e, atol=1e-13)
+    kap = oracle.gate_kernel(np.full(nb, -1.75 + 0j))
+    np.testing.assert_allclose(kap, np.r_[-1.75, np.zeros(n - 1)], atol=1e-14)
+    rng = np.random.default_rng(12)
+    g = rng.standard_normal(nb) + 1j * rng.standard_normal(nb)
+    np.testing.assert_allclose(oracle.gate_kernel(g), np.fft.irfft(g, n=n), atol=1e-13)
+
+
+def test_circular_conv_shift_parseval_library():
+    rng = np.random.default_rng(13)
+    n = 32
+    x1 = rng.standard_normal(n)
+    s = 3
+    e = np.zeros(n); e[s] = 1
+    y = oracle.circular_conv_samples(e, x1, None, np.arange(n))
+    np.testing.assert_array_equal(y, np.roll(x1, s))
+    kap = rng.standard_normal(n)
+    y = oracle.circular_conv_samples(kap, x1, None, np.arange(n))
+    G, X = np.fft.fft(kap), np.fft.fft(x1)
+    np.testing.assert_allclose(np.sum(y ** 2), np.sum(np.abs(G * X) ** 2) / n, rtol=1e-12)
+    np.testing.assert_allclose(y, np.real(np.fft.ifft(G * X)), atol=1e-12)
+    rows = oracle.circular_conv_rows(np.stack([kap, e]), [1, 0], np.stack([x1, x1]), None)
+    np.testing.assert_array_equal(rows[0], np.roll(x1, s))
+    np.testing.assert_allclose(rows[1], y, atol=1e-13)
+
+
+# ---------------------------------------------------------------- FFT-route references
+
+def test_fft_hyena_rows_matches_direct():
+    rng = np.random.default_rng(14)
+    B, D, L = 2, 3, 100            # L not a power of two: padded transform 256
+    v = rng.standard_normal((B, D, L))
+    xs = [rng.standard_normal((B, D, L)) for _ in range(2)]
+    h = rng.standard_normal((2, D, L)) * np.exp(-np.arange(L) / 30)
+    Dk = rng.standard_normal((2, D))
+    a = oracle.fft_hyena_rows(v, xs, h, Dk)
+    b = oracle.hyena_rows(v, xs, h, Dk)
+    np.testing.assert_allclose(a, b, rtol=1e-10, atol=1e-11)
+    assert oracle.transform_len(100) == 256 and oracle.transform_len(128) == 256
+
+
+def test_fft_nd_matches_direct():
+    rng = np.random.default_rng(15)
+    g = (4, 6, 8)
+    for circular in (False, True):
+        S = g if circular else tuple(2 * a for a in g)
+        K = rng.standard_normal(S)
+        v, x1 = rng.standard_normal((2,) + g)
+        a = oracle.fft_nd_conv(K, v, x1, 0.2, circular)
+        b = oracle.nd_conv_points(K, v, x1, 0.2, np.arange(int(np.prod(g))), circular).reshape(g)
+        np.testing.assert_allclose(a, b, rtol=1e-11, atol=1e-11)
+
+
+def test_fft_spectral_gate_matches_direct():
+    rng = np.random.default_rng(16)
+    n, R = 64, 3
+    g = rng.standard_normal((2, n // 2 + 1)) + 1j * rng.standard_normal((2, n // 2 + 1))
+    x1, x2 = rng.standard_normal((2, R, n))
+    kidx = np.array([0, 1, 1])
+    a = oracle.fft_spectral_gate_rows(g[kidx], x1, x2)
+    kap = np.stack([oracle.gate_kernel(gg) for gg in g])
+    b = oracle.circular_conv_rows(kap, kidx, x1, x2)
+    np.testing.assert_allclose(a, b, rtol=1e-11, atol=1e-12)
+
+
+def test_fft_spectrum_matches_direct():
+    rng = np.random.default_rng(17)
+    h = rng.standard_normal((4, 40))
+    np.testing.assert_allclose(oracle.fft_spectrum(h), oracle.dft_real_rows(h, 128), atol=1e-11)

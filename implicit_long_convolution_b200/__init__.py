@@ -1,0 +1,211 @@
+"""Python binding of libhyena_b200.so -- the Hyena implicit long-convolution
+hot path on B200 (sm_100a).
+
+This module only marshals arguments: every step of the path runs in the CUDA
+kernels behind the C ABI declared in ``include/hyena.h``.  PyTorch supplies
+device memory and the current stream.  If the shared library is missing the
+import of this package still works, but every call raises
+``HyenaLibraryMissing`` -- there is no CPU fallback.
+
+Functions mirror the C entry points (same names, same semantics):
+``hyena_filter_gen``, ``hyena_filter_spectrum``, ``hyena_fftconv``,
+``hyena_operator``, ``hyena_nd_conv``, ``spectral_gate``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+__all__ = [
+    "HyenaError", "HyenaLibraryMissing", "LIB_PATH", "lib", "spectrum_bins",
+    "hyena_filter_gen", "hyena_filter_spectrum", "filter_spectrum_workspace",
+    "hyena_fftconv", "hyena_operator", "operator_workspace", "hyena_nd_conv",
+    "nd_conv_workspace", "spectral_gate", "STATUS",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhyena_b200.so")
+
+STATUS = {0: "HY_OK", 1: "HY_ERR_INVALID_ARG", 2: "HY_ERR_UNSUPPORTED", 3: "HY_ERR_WORKSPACE",
+          4: "HY_ERR_CUDA", 5: "HY_ERR_TIMEOUT"}
+HY_F32, HY_BF16 = 0, 1
+HY_ACT_SILU, HY_ACT_IDENTITY = 0, 1
+
+
+class HyenaLibraryMissing(RuntimeError):
+    pass
+
+
+class HyenaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        self.status = status
+        self.status_name = STATUS.get(status, str(status))
+        super().__init__("%s: %s" % (self.status_name, message))
+
+
+class FilterDesc(ctypes.Structure):
+    _fields_ = [
+        ("ndim", ctypes.c_int), ("L", ctypes.c_int), ("grid", ctypes.c_int),
+        ("circular", ctypes.c_int), ("n_freq", ctypes.c_int), ("include_t", ctypes.c_int),
+        ("n_layers", ctypes.c_int), ("widths", ctypes.POINTER(ctypes.c_int)),
+        ("W", ctypes.POINTER(ctypes.c_void_p)), ("b", ctypes.POINTER(ctypes.c_void_p)),
+        ("act", ctypes.c_int), ("film_gamma", ctypes.c_void_p), ("film_beta", ctypes.c_void_p),
+        ("alpha", ctypes.c_void_p), ("n_sets", ctypes.c_int),
+    ]
+
+
+_lib = None
+_VP = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+
+
+def lib():
+    """The loaded shared library (raises HyenaLibraryMissing if not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise HyenaLibraryMissing(
+            "libhyena_b200.so is not built (run implicit_long_convolution_b200/build.py); "
+            "there is no fallback path")
+    L = ctypes.CDLL(LIB_PATH)
+    sig = {
+        "hyena_abi_version": (_I, []),
+        "hyena_status_string": (ctypes.c_char_p, [_I]),
+        "hyena_last_error": (ctypes.c_char_p, []),
+        "hyena_init": (_I, []),
+        "hyena_spectrum_bins": (_I64, [_I64]),
+        "hyena_filter_gen": (_I, [ctypes.POINTER(FilterDesc), _VP, _VP]),
+        "hyena_filter_spectrum_workspace": (_SZ, [_I64, _I, ctypes.POINTER(_I), _I]),
+        "hyena_filter_spectrum": (_I, [_I64, _I, ctypes.POINTER(_I), _I, _VP, _VP, _VP, _SZ, _VP]),
+        "hyena_fftconv": (_I, [_I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+        "hyena_operator_workspace": (_SZ, [_I, _I, _I, _I, _I]),
+        "hyena_operator": (_I, [_I, _I, _I, _I, _I, _VP, ctypes.POINTER(_VP), ctypes.POINTER(_VP),
+                                ctypes.POINTER(_VP), _VP, _VP, _SZ, _VP]),
+        "hyena_nd_conv_workspace": (_SZ, [_I, ctypes.POINTER(_I), _I, _I, _I]),
+        "hyena_nd_conv": (_I, [_I, ctypes.POINTER(_I), _I, _I, _I, _VP, _VP, _I64, _VP, _VP, _VP,
+                               _VP, _SZ, _VP]),
+        "spectral_gate": (_I, [_I, _I, _I, _I, _I, _VP, _VP, _I64, _VP, _VP, _VP]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = L
+    return L
+
+
+def _check(status: int):
+    if status != 0:
+        msg = lib().hyena_last_error()
+        raise HyenaError(status, msg.decode() if msg else "")
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is not None:
+        return stream if isinstance(stream, int) else stream.cuda_stream
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _dt(t) -> int:
+    import torch
+    if t.dtype == torch.float32:
+        return HY_F32
+    if t.dtype == torch.bfloat16:
+        return HY_BF16
+    raise HyenaError(1, "dtype %s not supported (float32 or bfloat16)" % t.dtype)
+
+
+def _ints(seq):
+    return (_I * len(seq))(*seq)
+
+
+def _ptrs(seq):
+    return (_VP * len(seq))(*[_ptr(t) for t in seq])
+
+
+def spectrum_bins(L: int) -> int:
+    """Bins of one causal filter spectrum row: M + 1, M = max(16, next pow2 >= L)."""
+    return int(lib().hyena_spectrum_bins(L))
+
+
+def hyena_filter_gen(h_out, *, ndim: int, Ws: Sequence, bs: Sequence, alpha, n_freq: int,
+                     L: int = 0, include_t: bool = True, grid: int = 0, circular: bool = False,
+                     film_gamma=None, film_beta=None, n_sets: int = 1, act: int = HY_ACT_SILU,
+                     stream=None):
+    """Fill h_out (fp32, device) with implicit filters; see hyena.h."""
+    widths = [int(Ws[0].shape[1])] + [int(w.shape[0]) for w in Ws]
+    keep = (_ints(widths), _ptrs(Ws), _ptrs(bs))
+    d = FilterDesc(ndim, L, grid, int(circular), n_freq, int(include_t), len(Ws),
+                   keep[0], keep[1], keep[2], act, _ptr(film_gamma), _ptr(film_beta),
+                   _ptr(alpha), n_sets)
+    _check(lib().hyena_filter_gen(ctypes.byref(d), _ptr(h_out), _stream(stream)))
+    return h_out
+
+
+def filter_spectrum_workspace(rows: int, ndim: int, dims: Sequence[int], circular: bool = False) -> int:
+    return int(lib().hyena_filter_spectrum_workspace(rows, ndim, _ints(dims), int(circular)))
+
+
+def hyena_filter_spectrum(h, H_out, *, rows: int, ndim: int, dims: Sequence[int],
+                          circular: bool = False, ws=None, stream=None):
+    wsb = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib().hyena_filter_spectrum(rows, ndim, _ints(dims), int(circular), _ptr(h), _ptr(H_out),
+                                       _ptr(ws), wsb, _stream(stream)))
+    return H_out
+
+
+def hyena_fftconv(u, H, y, *, Dskip=None, gate=None, ws=None, stream=None):
+    B, D, L = u.shape
+    wsb = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib().hyena_fftconv(B, D, L, _dt(u), _ptr(u), _ptr(H), _ptr(Dskip), _ptr(gate), _ptr(y),
+                               _ptr(ws), wsb, _stream(stream)))
+    return y
+
+
+def operator_workspace(order: int, B: int, D: int, L: int, dtype_code: int = HY_F32) -> int:
+    return int(lib().hyena_operator_workspace(order, B, D, L, dtype_code))
+
+
+def hyena_operator(v, xs: Sequence, Hs: Sequence, y, *, Dskips: Optional[Sequence] = None,
+                   ws=None, stream=None):
+    B, D, L = v.shape
+    order = len(xs) + 1
+    dsk = _ptrs(Dskips) if Dskips is not None else None
+    wsb = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib().hyena_operator(order, B, D, L, _dt(v), _ptr(v), _ptrs(xs), _ptrs(Hs), dsk, _ptr(y),
+                                _ptr(ws), wsb, _stream(stream)))
+    return y
+
+
+def nd_conv_workspace(dims: Sequence[int], B: int, D: int, circular: bool = False) -> int:
+    return int(lib().hyena_nd_conv_workspace(3, _ints(dims), B, D, int(circular)))
+
+
+def hyena_nd_conv(u, H, y, *, H_batch_stride: int = 0, circular: bool = False, Dskip=None,
+                  gate=None, ws=None, stream=None):
+    B, D = u.shape[:2]
+    dims = list(u.shape[2:])
+    wsb = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib().hyena_nd_conv(len(dims), _ints(dims), B, D, int(circular), _ptr(u), _ptr(H),
+                               H_batch_stride, _ptr(Dskip), _ptr(gate), _ptr(y), _ptr(ws), wsb,
+                               _stream(stream)))
+    return y
+
+
+def spectral_gate(x, g, y, *, x2=None, g_batch_stride: int = 0, stream=None):
+    B, Hh, Dh, L = x.shape
+    _check(lib().spectral_gate(B, Hh, Dh, L, _dt(x), _ptr(x), _ptr(g), g_batch_stride, _ptr(x2),
+                               _ptr(y), _stream(stream)))
+    return y

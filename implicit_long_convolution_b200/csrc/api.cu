@@ -1,0 +1,360 @@
+// api.cu -- the extern "C" entry points of libhyena_b200.so: argument
+// validation, path selection and launch.  See include/hyena.h for semantics.
+#include <cstdint>
+#include <cstring>
+
+#include "kernels.h"
+#include "resident.cuh"
+#include "status.h"
+#include "twiddle.h"
+
+using namespace hy;
+
+namespace {
+
+constexpr int kMaxResidentLogM = 14;   // M = 16384 complex points on chip
+
+bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
+int ilog2(int64_t x) {
+    int r = 0;
+    while ((int64_t(1) << r) < x) ++r;
+    return r;
+}
+int64_t spectrum_m(int64_t L) {
+    int64_t m = 16;
+    while (m < L) m *= 2;
+    return m;
+}
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+size_t dt_size(hy_dtype dt) { return dt == HY_BF16 ? 2 : 4; }
+bool overlap(const void *a, size_t na, const void *b, size_t nb) {
+    if (!a || !b) return false;
+    const char *pa = (const char *)a, *pb = (const char *)b;
+    return pa < pb + nb && pb < pa + na;
+}
+
+hy_status prologue(cudaStream_t) {
+    clear_error();
+    return tw_ensure_device();
+}
+
+// Shared body of hyena_fftconv / hyena_operator (1-D, causal).
+hy_status run_chain(int K, int B, int D, int L, hy_dtype dt, const void *v, const void *const *gates,
+                    const hy_c32 *const *H, const float *const *Dskip, void *y, void *ws,
+                    size_t ws_bytes, cudaStream_t stream, const char *who) {
+    if (B < 1 || D < 1 || L < 1) return set_error(HY_ERR_INVALID_ARG, "%s: B, D, L must be >= 1", who);
+    if (dt != HY_F32 && dt != HY_BF16) return set_error(HY_ERR_INVALID_ARG, "%s: unknown dtype", who);
+    if (!v || !y) return set_error(HY_ERR_INVALID_ARG, "%s: null signal pointer", who);
+    const size_t esz = dt_size(dt);
+    const size_t nbytes = (size_t)B * D * L * esz;
+    const size_t al = (L % 2 == 0) ? 2 * esz : esz;
+    if (!aligned(v, al) || !aligned(y, al))
+        return set_error(HY_ERR_INVALID_ARG, "%s: signals must be %zu-byte aligned", who, al);
+    if (overlap(v, nbytes, y, nbytes)) return set_error(HY_ERR_INVALID_ARG, "%s: y aliases the input", who);
+    const int64_t M = spectrum_m(L);
+    for (int k = 0; k < K; ++k) {
+        if (!H[k]) return set_error(HY_ERR_INVALID_ARG, "%s: spectrum %d is null", who, k);
+        if (!aligned(H[k], 8)) return set_error(HY_ERR_INVALID_ARG, "%s: spectrum %d misaligned", who, k);
+        if (gates[k]) {
+            if (!aligned(gates[k], al)) return set_error(HY_ERR_INVALID_ARG, "%s: gate %d misaligned", who, k);
+            if (overlap(gates[k], nbytes, y, nbytes))
+                return set_error(HY_ERR_INVALID_ARG, "%s: y aliases gate %d", who, k);
+        }
+        if (Dskip && Dskip[k] && overlap(Dskip[k], (size_t)D * 4, y, nbytes))
+            return set_error(HY_ERR_INVALID_ARG, "%s: y aliases Dskip %d", who, k);
+    }
+    const int log_m = ilog2(M);
+    if (log_m <= kMaxResidentLogM) {
+        hy_status st = prologue(stream);
+        if (st != HY_OK) return st;
+        ResidentParams p{};
+        p.n_rows = (int64_t)B * D;
+        p.L = L;
+        p.K = K;
+        p.B = B;
+        p.D = D;
+        p.remap = 1;
+        p.u = v;
+        for (int k = 0; k < K; ++k) {
+            p.gate[k] = gates[k];
+            p.spec[k] = reinterpret_cast<const float2 *>(H[k]);
+            p.skip[k] = Dskip ? Dskip[k] : nullptr;
+        }
+        p.spec_row_stride = M + 1;
+        p.sdiv = 1;
+        p.smod = D;
+        p.spec_batch_stride = 0;
+        p.y = y;
+        p.scale = (float)(1.0 / (4.0 * (double)M));
+        return launch_resident_conv(p, log_m, dt, false, stream);
+    }
+    // long sequences: multi-pass path
+    LongConvArgs a{};
+    a.K = K;
+    a.B = B;
+    a.D = D;
+    a.L = L;
+    a.log_mc = log_m;
+    a.dt = dt;
+    a.u = v;
+    for (int k = 0; k < K; ++k) {
+        a.gate[k] = gates[k];
+        a.spec[k] = reinterpret_cast<const float2 *>(H[k]);
+        a.skip[k] = Dskip ? Dskip[k] : nullptr;
+    }
+    a.y = y;
+    a.ws = ws;
+    a.ws_bytes = ws_bytes;
+    const size_t need = long_conv_workspace(B, D, log_m, K);
+    if (need == 0) return set_error(HY_ERR_UNSUPPORTED, "%s: L=%d is beyond the supported length", who, L);
+    if (!ws || ws_bytes < need)
+        return set_error(HY_ERR_WORKSPACE, "%s: needs %zu workspace bytes, got %zu", who, need, ws ? ws_bytes : (size_t)0);
+    if (!aligned(ws, 256)) return set_error(HY_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", who);
+    hy_status st = prologue(stream);
+    if (st != HY_OK) return st;
+    return launch_long_conv(a, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+int hyena_abi_version(void) { return HYENA_ABI_VERSION; }
+
+const char *hyena_status_string(hy_status s) {
+    switch (s) {
+        case HY_OK: return "HY_OK";
+        case HY_ERR_INVALID_ARG: return "HY_ERR_INVALID_ARG";
+        case HY_ERR_UNSUPPORTED: return "HY_ERR_UNSUPPORTED";
+        case HY_ERR_WORKSPACE: return "HY_ERR_WORKSPACE";
+        case HY_ERR_CUDA: return "HY_ERR_CUDA";
+        case HY_ERR_TIMEOUT: return "HY_ERR_TIMEOUT";
+    }
+    return "unknown status";
+}
+
+hy_status hyena_init(void) {
+    clear_error();
+    return tw_ensure_device();
+}
+
+int64_t hyena_spectrum_bins(int64_t L) {
+    if (L < 1) return 0;
+    return spectrum_m(L) + 1;
+}
+
+hy_status hyena_filter_gen(const hy_filter_desc *d, float *h, void *stream) {
+    clear_error();
+    if (!d || !h) return set_error(HY_ERR_INVALID_ARG, "hyena_filter_gen: null desc or output");
+    if (d->ndim != 1 && d->ndim != 3) return set_error(HY_ERR_INVALID_ARG, "hyena_filter_gen: ndim must be 1 or 3");
+    if (d->n_layers < 1 || d->n_layers > 4) return set_error(HY_ERR_UNSUPPORTED, "hyena_filter_gen: n_layers must be 1..4");
+    if (!d->widths || !d->W || !d->b || !d->alpha) return set_error(HY_ERR_INVALID_ARG, "hyena_filter_gen: null parameter array");
+    if (d->n_freq < 0 || d->n_sets < 1) return set_error(HY_ERR_INVALID_ARG, "hyena_filter_gen: bad n_freq or n_sets");
+    if (d->act != HY_ACT_SILU && d->act != HY_ACT_IDENTITY) return set_error(HY_ERR_INVALID_ARG, "hyena_filter_gen: bad activation");
+    if ((d->film_gamma == nullptr) != (d->film_beta == nullptr))
+        return set_error(HY_ERR_INVALID_ARG, "hyena_filter_gen: film_gamma and film_beta go together");
+    if (d->film_gamma && d->n_layers < 2) return set_error(HY_ERR_INVALID_ARG, "hyena_filter_gen: FiLM needs a hidden layer");
+    if (!d->film_gamma && d->n_sets != 1) return set_error(HY_ERR_INVALID_ARG, "hyena_filter_gen: n_sets > 1 needs FiLM");
+    for (int l = 0; l <= d->n_layers; ++l)
+        if (d->widths[l] < 1) return set_error(HY_ERR_INVALID_ARG, "hyena_filter_gen: width %d < 1", l);
+    for (int l = 0; l < d->n_layers; ++l)
+        if (!d->W[l] || !d->b[l]) return set_error(HY_ERR_INVALID_ARG, "hyena_filter_gen: null weight of layer %d", l);
+    if (d->ndim == 1) {
+        if (d->L < 1) return set_error(HY_ERR_INVALID_ARG, "hyena_filter_gen: L must be >= 1");
+        if (d->widths[0] != (d->include_t ? 1 : 0) + 2 * d->n_freq)
+            return set_error(HY_ERR_INVALID_ARG, "hyena_filter_gen: widths[0] must equal include_t + 2F");
+        if (d->n_freq < 1 && !d->include_t) return set_error(HY_ERR_INVALID_ARG, "hyena_filter_gen: empty encoding");
+    } else {
+        if (!is_pow2(d->grid) || d->grid < 2 || d->grid > 64)
+            return set_error(HY_ERR_UNSUPPORTED, "hyena_filter_gen: grid must be a power of two in [2, 64]");
+        if (d->widths[0] != 6 * d->n_freq || d->n_freq < 1)
+            return set_error(HY_ERR_INVALID_ARG, "hyena_filter_gen: widths[0] must equal 6F (F >= 1)");
+    }
+    hy_status st = tw_ensure_device();
+    if (st != HY_OK) return st;
+    return launch_filter_gen(*d, h, (cudaStream_t)stream);
+}
+
+size_t hyena_filter_spectrum_workspace(int64_t rows, int ndim, const int *dims, int circular) {
+    if (rows < 1 || !dims) return 0;
+    if (ndim == 1) {
+        if (circular) return 0;
+        const int log_m = ilog2(spectrum_m(dims[0]));
+        return log_m <= kMaxResidentLogM ? 0 : long_spectrum_workspace(rows, log_m);
+    }
+    if (ndim == 3) {
+        int S[3];
+        for (int a = 0; a < 3; ++a) S[a] = circular ? dims[a] : 2 * dims[a];
+        return nd_spectrum_workspace(rows, S);
+    }
+    return 0;
+}
+
+hy_status hyena_filter_spectrum(int64_t rows, int ndim, const int *dims, int circular, const float *h,
+                                hy_c32 *H, void *ws, size_t ws_bytes, void *stream) {
+    clear_error();
+    if (rows < 1 || !dims || !h || !H) return set_error(HY_ERR_INVALID_ARG, "hyena_filter_spectrum: bad rows or null pointer");
+    if (!aligned(h, 8) || !aligned(H, 8)) return set_error(HY_ERR_INVALID_ARG, "hyena_filter_spectrum: pointers must be 8-byte aligned");
+    cudaStream_t s = (cudaStream_t)stream;
+    if (ndim == 1) {
+        const int64_t L = dims[0];
+        if (L < 1) return set_error(HY_ERR_INVALID_ARG, "hyena_filter_spectrum: L must be >= 1");
+        if (overlap(h, (size_t)rows * L * 4, H, (size_t)rows * (L + 2) * 8))
+            return set_error(HY_ERR_INVALID_ARG, "hyena_filter_spectrum: H aliases h");
+        if (circular) {
+            if (!is_pow2(L) || L < 32 || L > 32768)
+                return set_error(HY_ERR_UNSUPPORTED, "hyena_filter_spectrum: circular L must be a power of two in [32, 32768]");
+            hy_status st = prologue(s);
+            if (st != HY_OK) return st;
+            return launch_spectrum_1d(rows, (int)L, ilog2(L / 2), true, h, reinterpret_cast<float2 *>(H), s);
+        }
+        const int log_m = ilog2(spectrum_m(L));
+        if (log_m <= kMaxResidentLogM) {
+            hy_status st = prologue(s);
+            if (st != HY_OK) return st;
+            return launch_spectrum_1d(rows, (int)L, log_m, false, h, reinterpret_cast<float2 *>(H), s);
+        }
+        const size_t need = long_spectrum_workspace(rows, log_m);
+        if (need == 0) return set_error(HY_ERR_UNSUPPORTED, "hyena_filter_spectrum: L=%lld beyond the supported length", (long long)L);
+        if (!ws || ws_bytes < need)
+            return set_error(HY_ERR_WORKSPACE, "hyena_filter_spectrum: needs %zu workspace bytes", need);
+        if (!aligned(ws, 256)) return set_error(HY_ERR_INVALID_ARG, "hyena_filter_spectrum: workspace must be 256-byte aligned");
+        hy_status st = prologue(s);
+        if (st != HY_OK) return st;
+        return launch_long_spectrum(rows, L, log_m, h, reinterpret_cast<float2 *>(H), ws, ws_bytes, s);
+    }
+    if (ndim == 3) {
+        int S[3];
+        for (int a = 0; a < 3; ++a) {
+            if (!is_pow2(dims[a]) || dims[a] < 4 || dims[a] > 128)
+                return set_error(HY_ERR_UNSUPPORTED, "hyena_filter_spectrum: grid edges must be powers of two in [4, 128]");
+            S[a] = circular ? dims[a] : 2 * dims[a];
+            if (S[a] > 128) return set_error(HY_ERR_UNSUPPORTED, "hyena_filter_spectrum: transform edge %d > 128", S[a]);
+        }
+        const size_t need = nd_spectrum_workspace(rows, S);
+        if (need > 0 && (!ws || ws_bytes < need))
+            return set_error(HY_ERR_WORKSPACE, "hyena_filter_spectrum: needs %zu workspace bytes", need);
+        hy_status st = prologue(s);
+        if (st != HY_OK) return st;
+        return launch_nd_spectrum(rows, S, h, reinterpret_cast<float2 *>(H), ws, ws_bytes, s);
+    }
+    return set_error(HY_ERR_INVALID_ARG, "hyena_filter_spectrum: ndim must be 1 or 3");
+}
+
+hy_status hyena_fftconv(int B, int D, int L, hy_dtype dt, const void *u, const hy_c32 *H, const float *Dskip,
+                        const void *gate, void *y, void *ws, size_t ws_bytes, void *stream) {
+    clear_error();
+    const void *gates[1] = {gate};
+    const hy_c32 *Hs[1] = {H};
+    const float *sk[1] = {Dskip};
+    return run_chain(1, B, D, L, dt, u, gates, Hs, sk, y, ws, ws_bytes, (cudaStream_t)stream, "hyena_fftconv");
+}
+
+size_t hyena_operator_workspace(int order, int B, int D, int L, hy_dtype dt) {
+    (void)dt;
+    if (order < 2 || order - 1 > kMaxOrders || B < 1 || D < 1 || L < 1) return 0;
+    const int log_m = ilog2(spectrum_m(L));
+    if (log_m <= kMaxResidentLogM) return 0;
+    return long_conv_workspace(B, D, log_m, order - 1);
+}
+
+hy_status hyena_operator(int order, int B, int D, int L, hy_dtype dt, const void *v, const void *const *x,
+                         const hy_c32 *const *H, const float *const *Dskip, void *y, void *ws, size_t ws_bytes,
+                         void *stream) {
+    clear_error();
+    if (order < 2 || order - 1 > kMaxOrders)
+        return set_error(HY_ERR_UNSUPPORTED, "hyena_operator: order must be 2..%d", kMaxOrders + 1);
+    if (!x || !H) return set_error(HY_ERR_INVALID_ARG, "hyena_operator: null x or H array");
+    for (int k = 0; k < order - 1; ++k)
+        if (!x[k]) return set_error(HY_ERR_INVALID_ARG, "hyena_operator: x[%d] is null", k);
+    return run_chain(order - 1, B, D, L, dt, v, x, H, Dskip, y, ws, ws_bytes, (cudaStream_t)stream, "hyena_operator");
+}
+
+size_t hyena_nd_conv_workspace(int ndim, const int *dims, int B, int D, int circular) {
+    if (ndim != 3 || !dims || B < 1 || D < 1) return 0;
+    int g[3] = {dims[0], dims[1], dims[2]};
+    return nd_conv_workspace(g, circular, B, D);
+}
+
+hy_status hyena_nd_conv(int ndim, const int *dims, int B, int D, int circular, const float *u, const hy_c32 *H,
+                        int64_t H_batch_stride, const float *Dskip, const float *gate, float *y, void *ws,
+                        size_t ws_bytes, void *stream) {
+    clear_error();
+    if (ndim != 3) return set_error(HY_ERR_UNSUPPORTED, "hyena_nd_conv: only ndim = 3 is built");
+    if (!dims || !u || !H || !y) return set_error(HY_ERR_INVALID_ARG, "hyena_nd_conv: null pointer");
+    if (B < 1 || D < 1 || H_batch_stride < 0) return set_error(HY_ERR_INVALID_ARG, "hyena_nd_conv: bad B, D or stride");
+    NDArgs a{};
+    for (int i = 0; i < 3; ++i) {
+        if (!is_pow2(dims[i]) || dims[i] < 4 || dims[i] > 128)
+            return set_error(HY_ERR_UNSUPPORTED, "hyena_nd_conv: grid edges must be powers of two in [4, 128]");
+        a.g[i] = dims[i];
+        a.S[i] = circular ? dims[i] : 2 * dims[i];
+        if (a.S[i] > 128) return set_error(HY_ERR_UNSUPPORTED, "hyena_nd_conv: transform edge %d > 128", a.S[i]);
+    }
+    const size_t vox = (size_t)dims[0] * dims[1] * dims[2];
+    const size_t nbytes = (size_t)B * D * vox * 4;
+    if (!aligned(u, 16) || !aligned(y, 16) || (gate && !aligned(gate, 16)) || !aligned(H, 8))
+        return set_error(HY_ERR_INVALID_ARG, "hyena_nd_conv: signals must be 16-byte aligned");
+    if (overlap(u, nbytes, y, nbytes) || overlap(gate, nbytes, y, nbytes))
+        return set_error(HY_ERR_INVALID_ARG, "hyena_nd_conv: y aliases an input");
+    a.circular = circular ? 1 : 0;
+    a.B = B;
+    a.D = D;
+    a.u = u;
+    a.H = reinterpret_cast<const float2 *>(H);
+    a.H_batch_stride = H_batch_stride;
+    a.skip = Dskip;
+    a.gate = gate;
+    a.y = y;
+    a.ws = ws;
+    a.ws_bytes = ws_bytes;
+    const size_t need = nd_conv_workspace(a.g, a.circular, B, D);
+    if (need > 0 && (!ws || ws_bytes < need))
+        return set_error(HY_ERR_WORKSPACE, "hyena_nd_conv: needs %zu workspace bytes, got %zu", need, ws ? ws_bytes : (size_t)0);
+    if (ws && !aligned(ws, 256)) return set_error(HY_ERR_INVALID_ARG, "hyena_nd_conv: workspace must be 256-byte aligned");
+    hy_status st = prologue((cudaStream_t)stream);
+    if (st != HY_OK) return st;
+    return launch_nd_conv(a, (cudaStream_t)stream);
+}
+
+hy_status spectral_gate(int B, int H, int Dh, int L, hy_dtype dt, const void *x, const hy_c32 *g,
+                        int64_t g_batch_stride, const void *x2, void *y, void *stream) {
+    clear_error();
+    if (B < 1 || H < 1 || Dh < 1) return set_error(HY_ERR_INVALID_ARG, "spectral_gate: B, H, Dh must be >= 1");
+    if (dt != HY_F32 && dt != HY_BF16) return set_error(HY_ERR_INVALID_ARG, "spectral_gate: unknown dtype");
+    if (!is_pow2(L) || L < 32 || L > 32768)
+        return set_error(HY_ERR_UNSUPPORTED, "spectral_gate: L must be a power of two in [32, 32768]");
+    if (!x || !g || !y) return set_error(HY_ERR_INVALID_ARG, "spectral_gate: null pointer");
+    if (g_batch_stride < 0) return set_error(HY_ERR_INVALID_ARG, "spectral_gate: negative gate stride");
+    const size_t esz = dt_size(dt);
+    const size_t nbytes = (size_t)B * H * Dh * L * esz;
+    if (!aligned(x, 2 * esz) || !aligned(y, 2 * esz) || (x2 && !aligned(x2, 2 * esz)) || !aligned(g, 8))
+        return set_error(HY_ERR_INVALID_ARG, "spectral_gate: misaligned pointer");
+    if (overlap(x, nbytes, y, nbytes) || overlap(x2, nbytes, y, nbytes))
+        return set_error(HY_ERR_INVALID_ARG, "spectral_gate: y aliases an input");
+    const int64_t rows = (int64_t)B * H * Dh;
+    if (rows > 0x7fffffffLL) return set_error(HY_ERR_UNSUPPORTED, "spectral_gate: too many rows");
+    hy_status st = prologue((cudaStream_t)stream);
+    if (st != HY_OK) return st;
+    const int M = L / 2;
+    ResidentParams p{};
+    p.n_rows = rows;
+    p.L = L;
+    p.K = 1;
+    p.B = 1;
+    p.D = 1;
+    p.remap = 0;
+    p.u = x;
+    p.gate[0] = x2;
+    p.spec[0] = reinterpret_cast<const float2 *>(g);
+    p.skip[0] = nullptr;
+    p.spec_row_stride = M + 1;
+    p.sdiv = Dh;
+    p.smod = H;
+    p.spec_batch_stride = g_batch_stride;
+    p.y = y;
+    p.scale = (float)(1.0 / (2.0 * (double)L));
+    return launch_resident_conv(p, ilog2(M), dt, true, (cudaStream_t)stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,250 @@
+// fft_core.cuh -- register/shared-memory FFT building blocks for sm_100a.
+//
+// A complex FFT of size M is computed by T = M / P cooperating threads; thread
+// t owns the P elements t + T*m (m = 0..P-1) in registers.  The transform is a
+// self-sorting (Stockham) sequence of radix-R stages.  Stage s with radix R and
+// p = product of the earlier radices takes butterfly i = t + q*T, reads its
+// inputs x_r = in[i + r*M/R] -- always the thread's own registers q + r*P/R --
+// multiplies x_r by W_{pR}^{k r} (k = i mod p), does a radix-R DFT in
+// registers and writes output r to (i - k)*R + k + r*p.  Between stages the
+// outputs go through shared memory; the last stage's outputs land exactly in
+// the thread's own slots, so a size-M FFT needs (stages - 1) exchanges and
+// leaves natural-order results in registers.
+//
+// The radix-R DFT is a decimation-in-frequency network fully unrolled at
+// compile time; its internal twiddles are compile-time constants and trivial
+// ones (±1, ±i, (±1±i)/√2) cost no multiply.
+#pragma once
+#include "common.cuh"
+
+namespace hy {
+
+// ----------------------------------------------------------------------------
+// Radix-R DFT (R = 2^p <= 64) in registers, DIF, bit-reversed output:
+// after dft_dif<R>(a), a[j] holds X[bitrev_R(j)].
+// ----------------------------------------------------------------------------
+template <int DIR, int SPAN, int J>
+__device__ __forceinline__ void bfly_dif(float2 &u, float2 &v) {
+    float2 s = cadd(u, v);
+    float2 d = csub(u, v);
+    u = s;
+    v = rot<DIR, 2 * SPAN, J>(d);
+}
+
+template <int DIR, int SPAN, int... J>
+__device__ __forceinline__ void dif_block(float2 *a, std::integer_sequence<int, J...>) {
+    (bfly_dif<DIR, SPAN, J>(a[J], a[J + SPAN]), ...);
+}
+
+// first layer when the upper half of the inputs is known to be zero:
+// (u, 0) -> (u, u * W)
+template <int DIR, int SPAN, int J>
+__device__ __forceinline__ void bfly_dif_zero(float2 &u, float2 &v) {
+    v = rot<DIR, 2 * SPAN, J>(u);
+}
+template <int DIR, int SPAN, int... J>
+__device__ __forceinline__ void dif_block_zero(float2 *a, std::integer_sequence<int, J...>) {
+    (bfly_dif_zero<DIR, SPAN, J>(a[J], a[J + SPAN]), ...);
+}
+
+template <int R, int DIR, int SPAN>
+__device__ __forceinline__ void dif_layers(float2 *a) {
+#pragma unroll
+    for (int start = 0; start < R; start += 2 * SPAN)
+        dif_block<DIR, SPAN>(a + start, std::make_integer_sequence<int, SPAN>{});
+    if constexpr (SPAN > 1) dif_layers<R, DIR, SPAN / 2>(a);
+}
+
+template <int R, int DIR, bool UPPER_ZERO = false>
+__device__ __forceinline__ void dft_dif(float2 *a) {
+    static_assert(R >= 1 && (R & (R - 1)) == 0, "radix must be a power of two");
+    if constexpr (R == 1) {
+        return;
+    } else if constexpr (UPPER_ZERO) {
+        dif_block_zero<DIR, R / 2>(a, std::make_integer_sequence<int, R / 2>{});
+        if constexpr (R > 2) dif_layers<R, DIR, R / 4>(a);
+    } else {
+        dif_layers<R, DIR, R / 2>(a);
+    }
+}
+
+__host__ __device__ constexpr int ct_log2(int x) { return x <= 1 ? 0 : 1 + ct_log2(x >> 1); }
+__host__ __device__ constexpr int bitrev(int j, int bits) {
+    int r = 0;
+    for (int b = 0; b < bits; ++b) r |= ((j >> b) & 1) << (bits - 1 - b);
+    return r;
+}
+
+// ----------------------------------------------------------------------------
+// Radix plan: stage 0 has radix P (its inputs need no twiddle); the remaining
+// log2(M/P) bits are split over as few stages as radix <= P allows, as evenly
+// as possible (larger radices first).  Shared by the device code and the
+// host-side twiddle-table builder.
+// ----------------------------------------------------------------------------
+__host__ __device__ constexpr int plan_stages(int log_m, int log_p) {
+    return 1 + (log_m - log_p + log_p - 1) / log_p;
+}
+__host__ __device__ constexpr int plan_log_radix(int log_m, int log_p, int s) {
+    if (s == 0) return log_p;
+    const int rest = log_m - log_p;
+    const int n = plan_stages(log_m, log_p) - 1;
+    const int base = rest / n, extra = rest % n;
+    return base + ((s - 1) < extra ? 1 : 0);
+}
+__host__ __device__ constexpr int plan_log_p(int log_m, int log_p, int s) {
+    int acc = 0;
+    for (int i = 0; i < s; ++i) acc += plan_log_radix(log_m, log_p, i);
+    return acc;
+}
+// twiddle entries of stage s: (R - 1) * p (none for stage 0)
+__host__ __device__ constexpr int plan_tw_count(int log_m, int log_p, int s) {
+    return s == 0 ? 0 : ((1 << plan_log_radix(log_m, log_p, s)) - 1) * (1 << plan_log_p(log_m, log_p, s));
+}
+__host__ __device__ constexpr int plan_tw_offset(int log_m, int log_p, int s) {
+    int acc = 0;
+    for (int i = 0; i < s; ++i) acc += plan_tw_count(log_m, log_p, i);
+    return acc;
+}
+__host__ __device__ constexpr int plan_tw_total(int log_m, int log_p) {
+    return plan_tw_offset(log_m, log_p, plan_stages(log_m, log_p));
+}
+
+// Shared-memory slot of complex element e: one pad slot every 32 elements
+// keeps the stride-R writes of the first stage conflict-free.
+__device__ __forceinline__ int spad(int e) { return e + (e >> 5); }
+__host__ __device__ constexpr int spad_size(int m) { return m + (m >> 5) + 1; }
+
+// x[m] = element t + m*T of a padded shared buffer (linear addressing when
+// T is a multiple of 32).
+template <int LOG_M, int LOG_P>
+__device__ __forceinline__ void load_own(float2 (&x)[1 << LOG_P], const float2 *sbuf, int t) {
+    constexpr int P = 1 << LOG_P;
+    constexpr int T = (1 << LOG_M) / P;
+    if constexpr (T % 32 == 0) {
+        const float2 *src = sbuf + spad(t);
+        constexpr int STEP = T + T / 32;
+#pragma unroll
+        for (int m = 0; m < P; ++m) x[m] = src[m * STEP];
+    } else {
+#pragma unroll
+        for (int m = 0; m < P; ++m) x[m] = sbuf[spad(t + m * T)];
+    }
+}
+template <int LOG_M, int LOG_P>
+__device__ __forceinline__ void store_own(const float2 (&x)[1 << LOG_P], float2 *sbuf, int t) {
+    constexpr int P = 1 << LOG_P;
+    constexpr int T = (1 << LOG_M) / P;
+    if constexpr (T % 32 == 0) {
+        float2 *dst = sbuf + spad(t);
+        constexpr int STEP = T + T / 32;
+#pragma unroll
+        for (int m = 0; m < P; ++m) dst[m * STEP] = x[m];
+    } else {
+#pragma unroll
+        for (int m = 0; m < P; ++m) sbuf[spad(t + m * T)] = x[m];
+    }
+}
+// Padded slot of the thread's own element t + m*T.
+template <int LOG_M, int LOG_P>
+__device__ __forceinline__ int own_slot(int t, int m) {
+    constexpr int T = (1 << LOG_M) >> LOG_P;
+    if constexpr (T % 32 == 0) return spad(t) + m * (T + T / 32);
+    else return spad(t + m * T);
+}
+// Address of padded element M - (t + m*T) for m = 0: the partner bins of the
+// real-FFT split walk down from here in steps of -(T + T/32).
+template <int LOG_M, int LOG_P>
+__device__ __forceinline__ int partner_slot(int t, int m) {
+    constexpr int M = 1 << LOG_M;
+    constexpr int T = M >> LOG_P;
+    if constexpr (T % 32 == 0) return spad(M - t) - m * (T + T / 32);
+    else return spad(M - t - m * T);
+}
+
+// Synchronisation of the threads that share one FFT.
+struct SyncBlock {
+    __device__ __forceinline__ void operator()() const { __syncthreads(); }
+};
+struct SyncWarp {
+    __device__ __forceinline__ void operator()() const { __syncwarp(); }
+};
+
+// ----------------------------------------------------------------------------
+// One Stockham stage.  x: the thread's P registers.  If LAST, outputs are left
+// in registers (natural order); otherwise written to sbuf and read back.
+// tw: this stage's table, layout [(r-1) * p + k] = W_{pR}^{k r} (forward).
+// ----------------------------------------------------------------------------
+template <int LOG_M, int LOG_P, int S, int DIR, bool UPPER_ZERO, typename Sync>
+__device__ __forceinline__ void fft_stage(float2 (&x)[1 << LOG_P], float2 *sbuf, int t,
+                                          const float2 *__restrict__ tw, Sync sync) {
+    constexpr int M = 1 << LOG_M;
+    constexpr int P = 1 << LOG_P;
+    constexpr int T = M / P;
+    constexpr int LR = plan_log_radix(LOG_M, LOG_P, S);
+    constexpr int R = 1 << LR;
+    constexpr int LPS = plan_log_p(LOG_M, LOG_P, S);
+    constexpr int PS = 1 << LPS;
+    constexpr int NB = P / R;                  // butterflies per thread
+    constexpr bool LAST = (S == plan_stages(LOG_M, LOG_P) - 1);
+
+    float2 y[NB][R];
+#pragma unroll
+    for (int q = 0; q < NB; ++q) {
+        const int i = t + q * T;
+        const int k = i & (PS - 1);
+#pragma unroll
+        for (int r = 0; r < R; ++r) y[q][r] = x[q + r * NB];
+        if constexpr (S > 0) {
+#pragma unroll
+            for (int r = 1; r < R; ++r) y[q][r] = cmul_dir<DIR>(y[q][r], __ldg(tw + (r - 1) * PS + k));
+        }
+        dft_dif<R, DIR, UPPER_ZERO>(y[q]);
+    }
+    if constexpr (LAST) {
+#pragma unroll
+        for (int q = 0; q < NB; ++q)
+#pragma unroll
+            for (int r = 0; r < R; ++r) x[q + r * NB] = y[q][bitrev(r, LR)];
+    } else {
+#pragma unroll
+        for (int q = 0; q < NB; ++q) {
+            const int i = t + q * T;
+            const int k = i & (PS - 1);
+            const int base = (i - k) * R + k;
+            if constexpr (PS % 32 == 0 || (PS == 1 && R <= 32)) {
+                // padded address is linear in r here: one base, constant steps
+                float2 *dst = sbuf + spad(base);
+                constexpr int STEP = PS + PS / 32;
+#pragma unroll
+                for (int r = 0; r < R; ++r) dst[r * STEP] = y[q][bitrev(r, LR)];
+            } else {
+#pragma unroll
+                for (int r = 0; r < R; ++r) sbuf[spad(base + r * PS)] = y[q][bitrev(r, LR)];
+            }
+        }
+        sync();
+        load_own<LOG_M, LOG_P>(x, sbuf, t);
+        sync();
+    }
+}
+
+template <int LOG_M, int LOG_P, int S, int DIR, bool UPPER_ZERO, typename Sync>
+__device__ __forceinline__ void fft_stages_from(float2 (&x)[1 << LOG_P], float2 *sbuf, int t,
+                                                const float2 *__restrict__ tw, Sync sync) {
+    constexpr int NS = plan_stages(LOG_M, LOG_P);
+    if constexpr (S < NS) {
+        fft_stage<LOG_M, LOG_P, S, DIR, (S == 0) && UPPER_ZERO>(x, sbuf, t, tw + plan_tw_offset(LOG_M, LOG_P, S), sync);
+        fft_stages_from<LOG_M, LOG_P, S + 1, DIR, UPPER_ZERO>(x, sbuf, t, tw, sync);
+    }
+}
+
+// Full complex FFT of size 2^LOG_M (unnormalised).  DIR = -1: forward
+// (e^{-2πi/M}); +1: inverse.  UPPER_ZERO: elements M/2..M-1 of the input are
+// zero (zero-padded rows) and are not read.
+template <int LOG_M, int LOG_P, int DIR, bool UPPER_ZERO = false, typename Sync = SyncBlock>
+__device__ __forceinline__ void block_fft(float2 (&x)[1 << LOG_P], float2 *sbuf, int t,
+                                          const float2 *__restrict__ tw, Sync sync = Sync{}) {
+    fft_stages_from<LOG_M, LOG_P, 0, DIR, UPPER_ZERO>(x, sbuf, t, tw, sync);
+}
+
+}  // namespace hy

@@ -1,0 +1,61 @@
+// kernels.h -- internal launcher declarations (host side).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/hyena.h"
+
+namespace hy {
+
+struct ResidentParams;
+
+hy_status launch_resident_conv(const ResidentParams &p, int log_m, hy_dtype dt, bool circular,
+                               cudaStream_t s);
+hy_status launch_spectrum_1d(int64_t rows, int L, int log_m, bool circular, const float *h, float2 *H,
+                             cudaStream_t s);
+
+// filter generator (filter_gen.cu); desc validated by the caller
+hy_status launch_filter_gen(const hy_filter_desc &d, float *h, cudaStream_t s);
+
+// multi-pass (four-step) path for long sequences (fourstep.cu)
+struct LongConvArgs {
+    int K;                         // orders
+    int64_t B, D, L;               // rows are (B, D), length L
+    int log_mc;                    // complex transform length M = 2^log_mc (n = 2M)
+    hy_dtype dt;
+    const void *u;
+    const void *gate[8];
+    const float2 *spec[8];         // (D, M+1) per order
+    const float *skip[8];
+    void *y;
+    void *ws;
+    size_t ws_bytes;
+};
+size_t long_conv_workspace(int64_t B, int64_t D, int log_mc, int K);
+hy_status launch_long_conv(const LongConvArgs &a, cudaStream_t s);
+size_t long_spectrum_workspace(int64_t rows, int log_mc);
+hy_status launch_long_spectrum(int64_t rows, int64_t L, int log_mc, const float *h, float2 *H, void *ws,
+                               size_t ws_bytes, cudaStream_t s);
+
+// N-D path (ndconv.cu)
+struct NDArgs {
+    int g[3];                      // grid
+    int S[3];                      // transform grid
+    int circular;
+    int64_t B, D;
+    const float *u;
+    const float2 *H;
+    int64_t H_batch_stride;
+    const float *skip;
+    const float *gate;
+    float *y;
+    void *ws;
+    size_t ws_bytes;
+};
+size_t nd_conv_workspace(const int g[3], int circular, int64_t B, int64_t D);
+hy_status launch_nd_conv(const NDArgs &a, cudaStream_t s);
+size_t nd_spectrum_workspace(int64_t rows, const int S[3]);
+hy_status launch_nd_spectrum(int64_t rows, const int S[3], const float *h, float2 *H, void *ws,
+                             size_t ws_bytes, cudaStream_t s);
+
+}  // namespace hy

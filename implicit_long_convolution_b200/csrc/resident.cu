@@ -1,0 +1,55 @@
+// resident.cu -- entry to the on-chip path: variant selection for the
+// FFT convolution and the 1-D filter-spectrum kernels.
+#include "resident_launch.cuh"
+
+namespace hy {
+
+namespace {
+
+template <int LOG_M, bool CIRC>
+hy_status launch_spectrum_t(int64_t rows, int L, const float *h, float2 *H, cudaStream_t s) {
+    constexpr int LOG_P = resident_log_p(LOG_M);
+    constexpr int M = 1 << LOG_M;
+    constexpr int T = M >> LOG_P;
+    const float2 *tw = tw_stages(LOG_M, LOG_P);
+    const float2 *tws = tw_split(LOG_M);
+    if (!tw || !tws) return set_error(HY_ERR_CUDA, "twiddle tables missing for M=2^%d", LOG_M);
+    const size_t smem = sizeof(float2) * (size_t)spad_size(M);
+    auto kernel = spectrum_rows_kernel<LOG_M, CIRC>;
+    hy_status st = set_smem_limit(kernel, smem, "spectrum smem attribute");
+    if (st != HY_OK) return st;
+    kernel<<<(unsigned)rows, T, smem, s>>>(rows, L, h, H, tw, tws);
+    return check_launch("spectrum launch");
+}
+
+}  // namespace
+
+hy_status launch_resident_conv(const ResidentParams &p, int log_m, hy_dtype dt, bool circular,
+                               cudaStream_t s) {
+    if (p.n_rows <= 0) return HY_OK;
+    if (p.n_rows > 0x7fffffffLL) return set_error(HY_ERR_UNSUPPORTED, "too many rows (%lld)", (long long)p.n_rows);
+    const bool chain = p.K > 1;
+    if (dt == HY_F32) {
+        if (circular) return dispatch_conv<float, true, false>(log_m, p, s);
+        return chain ? dispatch_conv<float, false, true>(log_m, p, s) : dispatch_conv<float, false, false>(log_m, p, s);
+    }
+    if (circular) return dispatch_conv<__nv_bfloat16, true, false>(log_m, p, s);
+    return chain ? dispatch_conv<__nv_bfloat16, false, true>(log_m, p, s)
+                 : dispatch_conv<__nv_bfloat16, false, false>(log_m, p, s);
+}
+
+hy_status launch_spectrum_1d(int64_t rows, int L, int log_m, bool circular, const float *h, float2 *H,
+                             cudaStream_t s) {
+    if (rows <= 0) return HY_OK;
+    if (rows > 0x7fffffffLL) return set_error(HY_ERR_UNSUPPORTED, "too many rows (%lld)", (long long)rows);
+    switch (log_m) {
+#define HY_CASE(LM) \
+    case LM: return circular ? launch_spectrum_t<LM, true>(rows, L, h, H, s) : launch_spectrum_t<LM, false>(rows, L, h, H, s);
+        HY_CASE(4) HY_CASE(5) HY_CASE(6) HY_CASE(7) HY_CASE(8) HY_CASE(9) HY_CASE(10)
+        HY_CASE(11) HY_CASE(12) HY_CASE(13) HY_CASE(14)
+#undef HY_CASE
+        default: return set_error(HY_ERR_UNSUPPORTED, "resident transform 2^%d not built", log_m);
+    }
+}
+
+}  // namespace hy

@@ -1,0 +1,271 @@
+// resident.cuh -- single-launch FFT convolution with gating, one sequence row
+// per CTA held on chip (registers + shared memory) across all orders.
+//
+// Per row (a real sequence of L samples, transform length n = 2M):
+//   pack      z[m] = s[2m] + i s[2m+1], m < M (rows zero-padded to n)
+//   forward   Z = FFT_M(z)                       (block_fft, registers + smem)
+//   split     X[k] = ½(Z[k] + Z*[M-k]) - ½ i W_n^k (Z[k] - Z*[M-k]),  k = 0..M
+//   multiply  Y[k] = X[k] · H[k]                 (filter spectrum or gate)
+//   merge     Z'[k] = (Y[k] + Y*[M-k]) + i W_n^{-k} (Y[k] - Y*[M-k])
+//   inverse   z' = IFFT_M(Z') / n ;  c[2m] = Re z'[m], c[2m+1] = Im z'[m]
+//   epilogue  z_k = x_k ⊙ (c + D_k · z_{k-1})   (next order starts from z_k)
+// Split and merge of bins k and M-k are done together by the thread owning
+// k < M/2; the partner value crosses shared memory.  Only the first L
+// samples of each order are kept (the rest of the padded row restarts at 0),
+// which makes every order a linear, causal convolution.  In the circular
+// variant (spectral gate) n = L and nothing is padded.
+#pragma once
+#include "fft_core.cuh"
+
+namespace hy {
+
+constexpr int kMaxOrders = 8;   // filters per operator call (order <= 9)
+
+
+__host__ __device__ constexpr int resident_log_p(int log_m) {
+    return log_m - 5 < 2 ? 2 : (log_m - 5 > 5 ? 5 : log_m - 5);
+}
+
+struct ResidentParams {
+    int64_t n_rows;
+    int L;                       // valid samples per row
+    int K;                       // orders (filters) chained in this launch
+    int B, D;                    // CTA c -> row (c % B) * D + c / B when remap
+    int remap;
+    const void *u;               // z_0 rows (IO dtype), row stride L
+    const void *gate[kMaxOrders];
+    const float2 *spec[kMaxOrders];
+    const float *skip[kMaxOrders];
+    int64_t spec_row_stride;     // complex elements between spectrum rows
+    int64_t sdiv, smod;          // spectrum channel of row r: (r / sdiv) % smod
+    int64_t spec_batch_stride;   // per sample r / (sdiv * smod); 0 = shared
+    void *y;
+    float scale;                 // 1 / (2n): folds the halving of split and the 1/n
+    const float2 *tw_fft;
+    const float2 *tw_split;
+};
+
+template <int LOG_M, int LOG_P>
+__device__ __forceinline__ void split_multiply_merge(float2 (&x)[1 << LOG_P], float2 *sbuf, int t,
+                                                     const float2 *__restrict__ H,
+                                                     const float2 *__restrict__ tws) {
+    constexpr int M = 1 << LOG_M;
+    constexpr int P = 1 << LOG_P;
+    constexpr int T = M / P;
+    store_own<LOG_M, LOG_P>(x, sbuf, t);
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < P / 2; ++m) {
+        const int k = t + m * T;
+        if (k == 0) {
+            // DC and Nyquist: X[0] = Re Z0 + Im Z0, X[M] = Re Z0 - Im Z0 (both
+            // real, doubled here); only the real part of the product is kept.
+            const float2 z0 = x[0];
+            const float y0 = 2.f * (z0.x + z0.y) * ldv(&H[0].x);
+            const float yM = 2.f * (z0.x - z0.y) * ldv(&H[M].x);
+            x[0] = make_float2(y0 + yM, y0 - yM);
+        } else {
+            const float2 zk = x[m];
+            const float2 zn = sbuf[partner_slot<LOG_M, LOG_P>(t, m)];
+            const float2 A = make_float2(zk.x + zn.x, zk.y - zn.y);   // Z[k] + Z*[M-k]
+            const float2 Bv = make_float2(zk.x - zn.x, zk.y + zn.y);  // Z[k] - Z*[M-k]
+            const float2 w = ldv(tws + k);                          // W_n^k
+            const float2 wB = cmul(Bv, w);
+            const float2 C = make_float2(wB.y, -wB.x);                // -i W B
+            const float2 Xk = cadd(A, C);                             // 2 X[k]
+            const float2 Xn = cconj(csub(A, C));                      // 2 X[M-k]
+            const float2 Yk = cmul(Xk, ldv(H + k));
+            const float2 Yn = cmul(Xn, ldv(H + (M - k)));
+            const float2 A2 = make_float2(Yk.x + Yn.x, Yk.y - Yn.y);
+            const float2 B2 = make_float2(Yk.x - Yn.x, Yk.y + Yn.y);
+            const float2 cB = cmulc(B2, w);
+            const float2 C2 = make_float2(-cB.y, cB.x);               // i W^-1 B'
+            x[m] = cadd(A2, C2);
+            sbuf[partner_slot<LOG_M, LOG_P>(t, m)] = cconj(csub(A2, C2));
+        }
+    }
+    if (t == 0) {
+        // k = M/2 pairs with itself: Z'[M/2] = 4 Z[M/2] conj(H[M/2]) (doubled scale)
+        const float2 z = x[P / 2];
+        const float2 hm = ldv(H + M / 2);
+        const float2 r = cmulc(z, hm);
+        x[P / 2] = make_float2(4.f * r.x, 4.f * r.y);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int m = P / 2; m < P; ++m)
+        if (!(t == 0 && m == P / 2)) x[m] = sbuf[own_slot<LOG_M, LOG_P>(t, m)];
+    __syncthreads();
+}
+
+// CTAs per SM the register budget is sized for (128 registers per thread at
+// 256 threads): two CTAs overlap one's barriers with the other's arithmetic.
+__host__ __device__ constexpr int resident_min_blocks(int log_m) {
+    return ((1 << log_m) >> resident_log_p(log_m)) <= 256 ? 2 : 1;
+}
+
+// CHAIN = false: exactly one order (K = 1): order-2 operator, single gated
+// convolution, spectral gate.  CHAIN = true: K >= 1 orders in a runtime loop
+// (the loop costs registers, so the single-order case has its own build).
+template <int LOG_M, typename IO, bool CIRC, bool CHAIN>
+__global__ void __launch_bounds__((1 << LOG_M) >> resident_log_p(LOG_M), resident_min_blocks(LOG_M))
+resident_conv_kernel(const ResidentParams p) {
+    constexpr int LOG_P = resident_log_p(LOG_M);
+    constexpr int M = 1 << LOG_M;
+    constexpr int P = 1 << LOG_P;
+    constexpr int T = M / P;
+    constexpr int PIN = CIRC ? P : P / 2;   // registers carrying samples
+    using IOT = IOTraits<IO>;
+
+    extern __shared__ float2 smem[];
+    float2 *sbuf = smem;
+    float2 *ustash = smem + spad_size(M);   // z_{k-1} for orders >= 2
+
+    const int t = threadIdx.x;
+    const int64_t c = blockIdx.x;
+    const int64_t row = p.remap ? (c % p.B) * (int64_t)p.D + c / p.B : c;
+    const int64_t ch = (row / p.sdiv) % p.smod;
+    const int64_t smp = row / (p.sdiv * p.smod);
+    const int L = p.L;
+    const bool pairs = (L & 1) == 0;
+    const IO *u = reinterpret_cast<const IO *>(p.u) + row * (int64_t)L;
+
+    float2 x[P];
+#pragma unroll
+    for (int m = 0; m < P; ++m) {
+        x[m] = make_float2(0.f, 0.f);
+        if (m < PIN) {
+            const int i0 = 2 * (t + m * T);
+            if (pairs) {
+                if (i0 < L) x[m] = IOT::load2(u + i0);
+            } else {
+                if (i0 < L) x[m].x = IOT::load(u + i0);
+                if (i0 + 1 < L) x[m].y = IOT::load(u + i0 + 1);
+            }
+        }
+    }
+
+    auto one_order = [&](const int k, const bool last) {
+        block_fft<LOG_M, LOG_P, -1, !CIRC>(x, sbuf, t, p.tw_fft);
+        const float2 *H = p.spec[k] + smp * p.spec_batch_stride + ch * p.spec_row_stride;
+        split_multiply_merge<LOG_M, LOG_P>(x, sbuf, t, H, p.tw_split);
+        block_fft<LOG_M, LOG_P, +1, false>(x, sbuf, t, p.tw_fft);
+
+        const float dk = p.skip[k] ? ldv(p.skip[k] + ch) : 0.f;
+        const IO *g = reinterpret_cast<const IO *>(p.gate[k]);
+        IO *yout = reinterpret_cast<IO *>(p.y) + row * (int64_t)L;
+#pragma unroll
+        for (int m = 0; m < P; ++m) {
+            if (m >= PIN) {
+                x[m] = make_float2(0.f, 0.f);
+                continue;
+            }
+            const int e = t + m * T;
+            const int i0 = 2 * e;
+            float2 prev = make_float2(0.f, 0.f);
+            if (k == 0) {
+                if (dk != 0.f) {
+                    if (pairs) {
+                        if (i0 < L) prev = IOT::load2(u + i0);
+                    } else {
+                        if (i0 < L) prev.x = IOT::load(u + i0);
+                        if (i0 + 1 < L) prev.y = IOT::load(u + i0 + 1);
+                    }
+                }
+            } else {
+                prev = ustash[e];
+            }
+            float2 z = make_float2(fmaf(x[m].x, p.scale, dk * prev.x), fmaf(x[m].y, p.scale, dk * prev.y));
+            if (g) {
+                float2 gv = make_float2(0.f, 0.f);
+                if (pairs) {
+                    if (i0 < L) gv = IOT::load2(g + row * (int64_t)L + i0);
+                } else {
+                    if (i0 < L) gv.x = IOT::load(g + row * (int64_t)L + i0);
+                    if (i0 + 1 < L) gv.y = IOT::load(g + row * (int64_t)L + i0 + 1);
+                }
+                z = make_float2(z.x * gv.x, z.y * gv.y);
+            }
+            if (i0 >= L) z.x = 0.f;
+            if (i0 + 1 >= L) z.y = 0.f;
+            if (last) {
+                if (pairs) {
+                    if (i0 < L) IOT::store2(yout + i0, z);
+                } else {
+                    if (i0 < L) IOT::store(yout + i0, z.x);
+                    if (i0 + 1 < L) IOT::store(yout + i0 + 1, z.y);
+                }
+            } else {
+                ustash[e] = z;
+                x[m] = z;
+            }
+        }
+    };
+
+    if constexpr (CHAIN) {
+        for (int k = 0; k < p.K; ++k) one_order(k, k == p.K - 1);
+    } else {
+        one_order(0, true);
+    }
+}
+
+// Filter spectrum rows: H[r, k] = Σ_t h[r, t] W_n^{kt}, k = 0..M, for rows of
+// L fp32 samples (zero-padded to n = 2M, or exactly n = L when circular).
+template <int LOG_M, bool CIRC>
+__global__ void __launch_bounds__((1 << LOG_M) >> resident_log_p(LOG_M))
+spectrum_rows_kernel(int64_t n_rows, int L, const float *__restrict__ h, float2 *__restrict__ Hout,
+                     const float2 *__restrict__ tw_fft, const float2 *__restrict__ tws) {
+    constexpr int LOG_P = resident_log_p(LOG_M);
+    constexpr int M = 1 << LOG_M;
+    constexpr int P = 1 << LOG_P;
+    constexpr int T = M / P;
+    constexpr int PIN = CIRC ? P : P / 2;
+    extern __shared__ float2 smem[];
+    float2 *sbuf = smem;
+    const int t = threadIdx.x;
+    const int64_t row = blockIdx.x;
+    const float *hr = h + row * (int64_t)L;
+    float2 *Hr = Hout + row * (int64_t)(M + 1);
+    const bool pairs = (L & 1) == 0;
+
+    float2 x[P];
+#pragma unroll
+    for (int m = 0; m < P; ++m) {
+        x[m] = make_float2(0.f, 0.f);
+        if (m < PIN) {
+            const int i0 = 2 * (t + m * T);
+            if (pairs) {
+                if (i0 < L) x[m] = __ldg(reinterpret_cast<const float2 *>(hr + i0));
+            } else {
+                if (i0 < L) x[m].x = __ldg(hr + i0);
+                if (i0 + 1 < L) x[m].y = __ldg(hr + i0 + 1);
+            }
+        }
+    }
+    block_fft<LOG_M, LOG_P, -1, !CIRC>(x, sbuf, t, tw_fft);
+    store_own<LOG_M, LOG_P>(x, sbuf, t);
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < P / 2; ++m) {
+        const int k = t + m * T;
+        if (k == 0) {
+            const float2 z0 = x[0];
+            Hr[0] = make_float2(z0.x + z0.y, 0.f);
+            Hr[M] = make_float2(z0.x - z0.y, 0.f);
+        } else {
+            const float2 zk = x[m];
+            const float2 zn = sbuf[partner_slot<LOG_M, LOG_P>(t, m)];
+            const float2 A = make_float2(zk.x + zn.x, zk.y - zn.y);
+            const float2 Bv = make_float2(zk.x - zn.x, zk.y + zn.y);
+            const float2 wB = cmul(Bv, __ldg(tws + k));
+            const float2 C = make_float2(wB.y, -wB.x);
+            const float2 Xk = cadd(A, C);
+            const float2 Xn = cconj(csub(A, C));
+            Hr[k] = make_float2(0.5f * Xk.x, 0.5f * Xk.y);
+            Hr[M - k] = make_float2(0.5f * Xn.x, 0.5f * Xn.y);
+        }
+    }
+    if (t == 0) Hr[M / 2] = cconj(x[P / 2]);
+}
+
+}  // namespace hy

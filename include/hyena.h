@@ -1,0 +1,207 @@
+/*
+ * hyena.h -- C ABI of libhyena_b200.so: the Hyena implicit long-convolution
+ * hot path on NVIDIA B200 (sm_100a).
+ *
+ * Pages cited (title, section):
+ *   [HN] "Hyena: 암묵적 장거리 컨볼루션으로 어텐션을 완전 대체한 서브-이차 모델" --
+ *        아키텍처 상세: step 2 (h(t) = FFN(pos_enc(t))·w(t), w(t) = e^{-αt}),
+ *        step 3 (y = x_{N-1} ⊙ (h_{N-1} * (x_{N-2} ⊙ (h_{N-2} * (…))))), and the
+ *        ImplicitFilter / hyena_operator code sketch.
+ *   [ES] "4. Hyena 상세" -- 어떻게 동작하나요? (filter generator: small MLP with
+ *        sinusoidal features and an exponential decay window; FFT convolution:
+ *        FFT -> pointwise product -> inverse FFT, O(N log N)).
+ *   [ND] "Native Multi-Dimensional Subquadratic Operators via Input Dependent
+ *        Long Convolutions" -- 방법론: HyenaND (네이티브 ND 합성곱 via the N-D FFT;
+ *        레지스터 및 FiLM; 경계 처리: circular, or non-circular by zero-padding
+ *        each axis to double).
+ *   [SP] "FFT의 반격: Self-Attention의 효율적 대안" -- 토큰 믹서 구성과 생성 지원
+ *        (real FFT -> gate on the n/2+1 bins -> inverse FFT).
+ *
+ * Conventions for every call:
+ *   - Pointers named as device pointers must point to device memory (or
+ *     memory the device can address) owned by the caller; the library never
+ *     takes ownership and never frees.  Host arrays of device pointers
+ *     (x[], H[], Dskip[], W[], b[]) are read during the call only.
+ *   - Signals are contiguous, channel-major with unit stride along the
+ *     sequence (or the last grid axis): (B, D, L) or (B, D, g0, g1, g2).
+ *     bf16 means IEEE bfloat16 bits (uint16); all arithmetic is fp32.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream) and never synchronises the host, except the
+ *     first call on each device (see hyena_init).
+ *   - Arguments are checked on the host before anything is launched; a
+ *     rejected call returns a status other than HY_OK, launches nothing and
+ *     leaves a message for hyena_last_error().  Launch failures are returned
+ *     as HY_ERR_CUDA.  Outputs must not alias inputs.
+ *   - No C++ exception crosses this boundary.
+ */
+#ifndef HYENA_B200_H
+#define HYENA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define HYENA_ABI_VERSION 1
+
+typedef enum hy_status {
+    HY_OK = 0,
+    HY_ERR_INVALID_ARG = 1,   /* a null pointer, a bad size, aliasing, ... */
+    HY_ERR_UNSUPPORTED = 2,   /* a valid request outside what is built    */
+    HY_ERR_WORKSPACE = 3,     /* workspace missing or too small           */
+    HY_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed      */
+    HY_ERR_TIMEOUT = 5        /* reserved: a bounded device wait gave up   */
+} hy_status;
+
+typedef enum hy_dtype { HY_F32 = 0, HY_BF16 = 1 } hy_dtype;
+
+typedef enum hy_act { HY_ACT_SILU = 0, HY_ACT_IDENTITY = 1 } hy_act;
+
+/* Interleaved single-precision complex (same bytes as float2 / complex64). */
+typedef struct hy_c32 { float re; float im; } hy_c32;
+
+/* Transform length used for a causal (zero-padded) 1-D convolution of
+ * length L: n = 2M with M = max(16, next power of two >= L).  Zero-padding to
+ * n >= 2L makes the FFT product a linear convolution ([HN] fft_conv, [ND]
+ * 경계 처리).  A filter spectrum row therefore has M + 1 bins; for L a power of
+ * two >= 16 that is L + 1. */
+int64_t hyena_spectrum_bins(int64_t L);
+
+/* ------------------------------------------------------------------------
+ * Filter generator  ([HN] step 2 and ImplicitFilter; [ES]; [ND] FiLM)
+ *
+ *   1-D:  h[s, o, t] = MLP(PE(t))[o] · exp(-alpha[o] · t / L)
+ *         PE(t) = [t/L (if include_t), cos(2π j t/L) j=1..F, sin(2π j t/L) j=1..F]
+ *   3-D:  h[s, o, p] = MLP_s(PE3(r(p)))[o] · exp(-alpha[o] · |r(p)| / g)
+ *         on the transform grid of edge S (S = 2g, or g when circular); r(p)
+ *         is the signed offset of grid index p per axis (i < S/2 -> i, else
+ *         i - S); PE3 = per axis (x, y, z): cos(π j r_a/g), sin(π j r_a/g),
+ *         j = 1..F.  Non-circular kernels are zero outside |r_a| <= g - 1.
+ *   MLP: layer l maps widths[l] -> widths[l+1], y = W_l x + b_l (W_l row-major
+ *   out x in); every layer but the last is followed by `act`; when
+ *   film_gamma is set, the first hidden layer is modulated per filter set s
+ *   before the activation: y <- (1 + gamma[s]) ⊙ y + beta[s].
+ * ---------------------------------------------------------------------- */
+typedef struct hy_filter_desc {
+    int ndim;                /* 1 or 3 */
+    int L;                   /* ndim = 1: filter length */
+    int grid;                /* ndim = 3: unpadded cube edge g (power of two, 4..64) */
+    int circular;            /* ndim = 3: 1 = kernel on the g^3 grid */
+    int n_freq;              /* F >= 0 */
+    int include_t;           /* ndim = 1: prepend t/L to the encoding */
+    int n_layers;            /* 1..4 */
+    const int *widths;       /* host, n_layers + 1 entries; widths[0] = input width; hidden <= 128 */
+    const float *const *W;   /* host array of n_layers device pointers */
+    const float *const *b;   /* host array of n_layers device pointers */
+    int act;                 /* hy_act for hidden layers */
+    const float *film_gamma; /* device (n_sets, widths[1]) or NULL */
+    const float *film_beta;  /* device (n_sets, widths[1]) or NULL (with gamma) */
+    const float *alpha;      /* device (widths[n_layers]); >= 0 */
+    int n_sets;              /* filter sets s (1 unless FiLM-conditioned) */
+} hy_filter_desc;
+
+/* Writes h (device, fp32): 1-D (n_sets, n_out, L); 3-D (n_sets, n_out, S, S, S). */
+hy_status hyena_filter_gen(const hy_filter_desc *desc, float *h, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Filter spectrum  ([HN] fft_conv; [ES] FFT convolution; [ND] N-D FFT)
+ *
+ *   ndim = 1: dims[0] = L.  Each of `rows` filter rows h[r, 0..L) is
+ *             zero-padded to n = 2·M (hyena_spectrum_bins) and
+ *             H[r, k] = Σ_t h[r, t] e^{-2πi k t / n}, k = 0..M.
+ *             (circular = 1: rows of length L = n, a power of two >= 32,
+ *             no padding; L/2 + 1 bins.)
+ *   ndim = 3: dims = (g0, g1, g2) unpadded grid; rows are kernels on the
+ *             transform grid S_a = 2 g_a (or g_a when circular), row-major;
+ *             H[r] = rFFT3(h[r]) with shape (S0, S1, S2/2 + 1).
+ *   ws: device workspace of at least hyena_filter_spectrum_workspace() bytes
+ *   (may be NULL when that is 0).
+ * ---------------------------------------------------------------------- */
+size_t hyena_filter_spectrum_workspace(int64_t rows, int ndim, const int *dims, int circular);
+hy_status hyena_filter_spectrum(int64_t rows, int ndim, const int *dims, int circular,
+                                const float *h, hy_c32 *H, void *ws, size_t ws_bytes,
+                                void *stream);
+
+/* ------------------------------------------------------------------------
+ * One gated long convolution  ([HN] step 3 for one order; skip term D·u)
+ *
+ *   y[b,d,t] = gate[b,d,t] · ( Σ_{s<=t} h_d[t-s] u[b,d,s] + Dskip[d] · u[b,d,t] )
+ *
+ *   u, gate, y: (B, D, L) of dtype dt.  gate may be NULL (no gate), Dskip
+ *   may be NULL (no skip).  H: (D, hyena_spectrum_bins(L)) spectra of h_d,
+ *   shared across the batch.  ws as for hyena_operator with order 2.
+ * ---------------------------------------------------------------------- */
+hy_status hyena_fftconv(int B, int D, int L, hy_dtype dt, const void *u, const hy_c32 *H,
+                        const float *Dskip, const void *gate, void *y, void *ws,
+                        size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
+ * The order-N Hyena operator  ([HN] step 3 gating equation and the
+ * hyena_operator sketch; D·u skip inside each order)
+ *
+ *   z_0 = v;  z_k = x_k ⊙ (h_k * z_{k-1} + D_k ⊙ z_{k-1}),  k = 1..order-1;
+ *   y = z_{order-1}.   Each h_k * is causal over the whole sequence.
+ *
+ *   v, x[k], y: (B, D, L) of dtype dt; x is a host array of order-1 device
+ *   pointers; H a host array of order-1 device pointers to (D, bins) spectra;
+ *   Dskip a host array of order-1 device pointers to (D) fp32 (the array, or
+ *   any entry, may be NULL for no skip).  Intermediate z_k stay fp32.
+ *   Sequences with hyena_spectrum_bins(L) - 1 <= 16384 run on chip in one
+ *   launch with no workspace; longer ones use the multi-pass path, which
+ *   needs hyena_operator_workspace() bytes of device workspace.
+ * ---------------------------------------------------------------------- */
+size_t hyena_operator_workspace(int order, int B, int D, int L, hy_dtype dt);
+hy_status hyena_operator(int order, int B, int D, int L, hy_dtype dt, const void *v,
+                         const void *const *x, const hy_c32 *const *H,
+                         const float *const *Dskip, void *y, void *ws, size_t ws_bytes,
+                         void *stream);
+
+/* ------------------------------------------------------------------------
+ * N-D global convolution with gating  ([ND] 네이티브 ND 합성곱, 경계 처리)
+ *
+ *   y[b,d,p] = gate[b,d,p] · ( Σ_q K_{b,d}[(p - q) mod S] u[b,d,q]
+ *                              + Dskip[d] · u[b,d,p] ),  p, q in the grid
+ *   ndim = 3, dims = (g0, g1, g2) powers of two (4..128); S = 2g per axis
+ *   (circular = 0: linear convolution) or S = g (circular = 1).
+ *   u, gate, y: (B, D, g0, g1, g2) fp32; H: spectra (rFFT3 of K) of shape
+ *   (S0, S1, S2/2 + 1) per (sample, channel), sample b at H + b·H_batch_stride
+ *   (in hy_c32 units; 0 = shared across samples), channel d at
+ *   + d·S0·S1·(S2/2+1).  gate / Dskip may be NULL.
+ * ---------------------------------------------------------------------- */
+size_t hyena_nd_conv_workspace(int ndim, const int *dims, int B, int D, int circular);
+hy_status hyena_nd_conv(int ndim, const int *dims, int B, int D, int circular, const float *u,
+                        const hy_c32 *H, int64_t H_batch_stride, const float *Dskip,
+                        const float *gate, float *y, void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Spectral-gating token mixer  ([SP] real FFT -> diagonal gate on n/2+1
+ * bins -> inverse FFT; circular)
+ *
+ *   y[b,h,c,:] = x2[b,h,c,:] ⊙ irFFT_L( g_{b,h} ⊙ rFFT_L(x[b,h,c,:]) )
+ *   x, x2, y: (B, H, Dh, L) of dtype dt, L a power of two in [32, 32768];
+ *   g: (H, L/2 + 1) complex per sample, sample b at g + b·g_batch_stride
+ *   (0 = shared).  At the DC and Nyquist bins only the real part of the
+ *   gated product is kept (the inverse of a real transform).  x2 may be NULL.
+ * ---------------------------------------------------------------------- */
+hy_status spectral_gate(int B, int H, int Dh, int L, hy_dtype dt, const void *x,
+                        const hy_c32 *g, int64_t g_batch_stride, const void *x2, void *y,
+                        void *stream);
+
+/* ------------------------------------------------------------------------
+ * Library state and errors
+ * ---------------------------------------------------------------------- */
+/* Uploads the constant twiddle tables to the current device.  Called
+ * implicitly by the first call on each device; that first call blocks the
+ * host briefly and must not be made while a stream is being captured.  */
+hy_status hyena_init(void);
+/* Message for the last non-OK status returned on this host thread. */
+const char *hyena_last_error(void);
+const char *hyena_status_string(hy_status s);
+int hyena_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HYENA_B200_H */

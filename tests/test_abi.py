@@ -1,0 +1,116 @@
+"""The C-ABI library loads, exports every function include/hyena.h declares,
+and rejects bad arguments on the host with the documented status -- all
+without a GPU (validation happens before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import implicit_long_convolution_b200 as hy
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hyena.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(\w+)\s*\(", src, flags=re.M)
+    return sorted(set(n for n in names if n not in ("defined",)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(hy.LIB_PATH):
+        pytest.fail("libhyena_b200.so is not built; run __graft_entry__.build()")
+    return hy.lib()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert "hyena_operator" in names and "spectral_gate" in names and "hyena_filter_gen" in names
+    for n in names:
+        assert hasattr(lib, n), "missing export %s" % n
+
+
+def test_version_and_strings(lib):
+    assert lib.hyena_abi_version() == 1
+    assert lib.hyena_status_string(3) == b"HY_ERR_WORKSPACE"
+    assert lib.hyena_spectrum_bins(8192) == 8193
+    assert lib.hyena_spectrum_bins(1000) == 1025
+    assert lib.hyena_spectrum_bins(1) == 17
+    assert lib.hyena_spectrum_bins(0) == 0
+
+
+def _err(lib, status, substring):
+    msg = lib.hyena_last_error().decode()
+    assert status != 0 and substring in msg, (status, msg)
+    return status
+
+
+FAKE = 0x10000  # a non-null, aligned pointer value; never dereferenced: calls fail validation first
+
+
+def test_operator_validation(lib):
+    X = (ctypes.c_void_p * 1)(FAKE)
+    H = (ctypes.c_void_p * 1)(FAKE)
+    # order out of range
+    assert _err(lib, lib.hyena_operator(1, 1, 1, 64, 0, FAKE, X, H, None, FAKE * 2, None, 0, None), "order") == 2
+    # null x array
+    assert _err(lib, lib.hyena_operator(2, 1, 1, 64, 0, FAKE, None, H, None, FAKE * 2, None, 0, None), "null") == 1
+    # bad sizes
+    assert lib.hyena_operator(2, 0, 1, 64, 0, FAKE, X, H, None, FAKE * 2, None, 0, None) == 1
+    assert lib.hyena_operator(2, 1, 1, 0, 0, FAKE, X, H, None, FAKE * 2, None, 0, None) == 1
+    # unknown dtype
+    assert lib.hyena_operator(2, 1, 1, 64, 7, FAKE, X, H, None, FAKE * 2, None, 0, None) == 1
+    # output aliases input
+    assert _err(lib, lib.hyena_operator(2, 1, 4, 64, 0, FAKE, X, H, None, FAKE + 64, None, 0, None), "alias") == 1
+    # misaligned signal
+    assert lib.hyena_operator(2, 1, 1, 64, 0, FAKE + 4, X, H, None, FAKE * 4, None, 0, None) == 1
+    # long sequence without workspace
+    big = 1 << 20
+    need = lib.hyena_operator_workspace(3, 1, 2, big, 0)
+    assert need > 0
+    X2 = (ctypes.c_void_p * 2)(FAKE * 64, FAKE * 128)
+    H2 = (ctypes.c_void_p * 2)(FAKE, FAKE)
+    st = lib.hyena_operator(3, 1, 2, big, 0, FAKE * 16, X2, H2, None, FAKE * 256, None, 0, None)
+    assert _err(lib, st, "workspace") == 3
+    assert lib.hyena_operator_workspace(2, 1, 1, 8192, 1) == 0
+
+
+def test_fftconv_and_gate_validation(lib):
+    assert lib.hyena_fftconv(1, 1, 64, 0, None, FAKE, None, None, FAKE, None, 0, None) == 1
+    assert lib.hyena_fftconv(1, 1, 64, 0, FAKE, None, None, None, FAKE * 2, None, 0, None) == 1
+    # spectral gate: L must be a power of two in [32, 32768]
+    assert lib.spectral_gate(1, 1, 1, 100, 1, FAKE, FAKE, 0, None, FAKE * 2, None) == 2
+    assert lib.spectral_gate(1, 1, 1, 65536, 1, FAKE, FAKE, 0, None, FAKE * 2, None) == 2
+    assert lib.spectral_gate(1, 1, 1, 64, 1, FAKE, None, 0, None, FAKE * 2, None) == 1
+    assert lib.spectral_gate(1, 1, 1, 64, 1, FAKE, FAKE, -1, None, FAKE * 2, None) == 1
+    assert _err(lib, lib.spectral_gate(1, 2, 2, 64, 1, FAKE, FAKE, 0, None, FAKE + 64, None), "alias") == 1
+
+
+def test_filter_and_nd_validation(lib):
+    dims = (ctypes.c_int * 3)(64, 64, 64)
+    assert lib.hyena_nd_conv(2, dims, 1, 1, 0, FAKE, FAKE, 0, None, None, FAKE * 2, None, 0, None) == 2
+    bad = (ctypes.c_int * 3)(64, 48, 64)
+    assert lib.hyena_nd_conv(3, bad, 1, 1, 0, FAKE, FAKE, 0, None, None, FAKE * 2, None, 0, None) == 2
+    assert lib.hyena_nd_conv(3, dims, 1, 1, 0, FAKE, FAKE, -5, None, None, FAKE * 2, None, 0, None) == 1
+    one = (ctypes.c_int * 1)(64)
+    assert lib.hyena_filter_spectrum(0, 1, one, 0, FAKE, FAKE * 2, None, 0, None) == 1
+    assert lib.hyena_filter_spectrum(4, 2, one, 0, FAKE, FAKE * 2, None, 0, None) == 1
+    assert lib.hyena_filter_spectrum(4, 1, (ctypes.c_int * 1)(100), 1, FAKE, FAKE * 2, None, 0, None) == 2
+    assert lib.hyena_filter_gen(None, FAKE, None) == 1
+    # widths[0] inconsistent with the encoding
+    widths = (ctypes.c_int * 3)(16, 32, 16)
+    W = (ctypes.c_void_p * 2)(FAKE, FAKE)
+    d = hy.FilterDesc(1, 1024, 0, 0, 8, 1, 2, widths, W, W, 0, None, None, FAKE, 1)
+    assert _err(lib, lib.hyena_filter_gen(ctypes.byref(d), FAKE * 2, None), "include_t + 2F") == 1
+    d = hy.FilterDesc(3, 0, 48, 0, 4, 0, 2, (ctypes.c_int * 3)(24, 64, 8), W, W, 0, None, None, FAKE, 1)
+    assert lib.hyena_filter_gen(ctypes.byref(d), FAKE * 2, None) == 2
+
+
+def test_binding_raises_named_errors(lib):
+    with pytest.raises(hy.HyenaError) as ei:
+        hy._check(lib.spectral_gate(1, 1, 1, 100, 1, FAKE, FAKE, 0, None, FAKE * 2, None))
+    assert ei.value.status_name == "HY_ERR_UNSUPPORTED"

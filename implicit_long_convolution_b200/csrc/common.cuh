@@ -101,24 +101,32 @@ __device__ __forceinline__ float2 rot(float2 v) {
 // would hold a register per in-flight value through the transform) nor
 // speculates it out of the branch that guards it.
 // ----------------------------------------------------------------------------
+// Streaming data (signals, spectra) is read once per SM: L1::no_allocate keeps
+// it from evicting the twiddle tables, which every row re-reads.
 __device__ __forceinline__ float ldv(const float *p) {
     float v;
-    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    asm volatile("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(v) : "l"(p));
     return v;
 }
 __device__ __forceinline__ float2 ldv(const float2 *p) {
     float2 v;
-    asm volatile("ld.global.nc.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p));
+    asm volatile("ld.global.nc.L1::no_allocate.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p));
     return v;
 }
 __device__ __forceinline__ uint32_t ldv_u16(const void *p) {
     unsigned short v;
-    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+    asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
     return v;
 }
 __device__ __forceinline__ uint32_t ldv_u32(const void *p) {
     uint32_t v;
-    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+// L1-cached ordered load (small tables shared by all rows)
+__device__ __forceinline__ float2 ldc(const float2 *p) {
+    float2 v;
+    asm volatile("ld.global.nc.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p));
     return v;
 }
 

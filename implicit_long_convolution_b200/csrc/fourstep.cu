@@ -1,26 +1,465 @@
-// fourstep.cu -- multi-pass path for sequences too long for one CTA (stub).
+// fourstep.cu -- multi-pass FFT convolution for sequences too long for one
+// CTA ([HN] step 3 chain and [ES] FFT convolution at HyenaDNA-scale length).
+//
+// A row of n = 2M real samples is packed into M = N1*N2 complex points
+// z[m] = s[2m] + i s[2m+1] (zero for m >= M/2: the causal zero-padding).  With
+// input index m = n1 + N1*n2 and bin index k = k2 + N2*k1:
+//
+//   Z[k2 + N2 k1] = Σ_n1 W_N1^{n1 k1} · W_M^{n1 k2} · Σ_n2 z[n1 + N1 n2] W_N2^{n2 k2}
+//
+//   pass A (columns): for each n1, FFT over n2, times W_M^{n1 k2}, stored at
+//                     n1 + N1*k2 (the input layout).
+//   pass B (rows):    for each k2 the N1 values are contiguous: FFT over n1
+//                     gives Z at bins k2 + N2*k1.  Bin k pairs with M - k,
+//                     which lives in row N2 - k2 (row 0 and row N2/2 pair with
+//                     themselves), so a CTA holds 4 rows and their 4 mirrors
+//                     and does the real-FFT split, the spectrum product and
+//                     the merge there, then the inverse row FFT and
+//                     W_M^{-n1 k2}.
+//   pass C (columns): inverse FFT over k2, first half of the outputs only,
+//                     then skip term and gate; when another order follows,
+//                     its pass A runs in the same kernel on the same columns.
+//
+// Each column or row FFT (N1, N2 <= 1024) is done by one warp (block_fft with
+// warp synchronisation); columns are staged through shared memory so global
+// accesses stay coalesced.  Rows are processed in chunks whose intermediates
+// (8 bytes per complex point) stay resident in the 126 MB L2 between passes.
 #include "kernels.h"
+#include "fft_core.cuh"
 #include "status.h"
+#include "twiddle.h"
 
 namespace hy {
-// Rows are processed in chunks small enough for their intermediates to stay
-// in the 126 MB L2 between passes.  Per row in flight: one complex buffer of
-// M points and one fp32 stash of M samples (z_{k-1} for the skip term).
-static int64_t chunk_rows(int64_t rows, int log_mc) {
+
+namespace {
+
+constexpr int WARPS = 8;          // columns or rows per CTA
+constexpr int NT = WARPS * 32;
+
+__host__ __device__ constexpr int fs_log_p(int log_n) { return log_n - 5; }   // per-lane points
+
+// W_N^e from a two-level table: tab[0..2^lo) = W_N^j, tab[2^lo + j] = W_N^{j 2^lo}
+__device__ __forceinline__ float2 tw2(const float2 *__restrict__ tab, int lo, uint32_t e) {
+    const float2 a = __ldg(tab + (e & ((1u << lo) - 1)));
+    const float2 b = __ldg(tab + (1u << lo) + (e >> lo));
+    return cmul(a, b);
+}
+
+struct FsParams {
+    int64_t row0;                 // first row of this chunk (flat b*D + d)
+    int64_t D;
+    int L;                        // valid real samples per row
+    int K, k;                     // orders, current order
+    const void *u;                // z_0 rows (IO)
+    const void *gate_k;           // x_k of the current order (pass C), IO
+    const float *skip_k;          // D_k (pass C)
+    const float2 *spec;           // H of the current order (pass B)
+    float2 *buf;                  // ws: complex buffer, chunk_rows x M
+    float *stash;                 // ws: fp32 z_{k} of the chunk, chunk_rows x M
+    void *y;                      // output (IO)
+    float scale;                  // 1 / (2n)
+    const float2 *tw_n1;          // block FFT tables (size N1, per-lane 2^(log N1 - 5))
+    const float2 *tw_n2;
+    const float2 *tw_m;           // two-level W_M
+    int lo_m;
+    const float2 *tw_2m;          // two-level W_{2M}
+    int lo_2m;
+    float2 *Hout;                 // spectrum mode: output bins (rows x (M+1))
+};
+
+// ----------------------------------------------------------------------------
+// Column pass: A (forward), C (inverse + epilogue), or C followed by A.
+// Block (blockIdx.x = column block of 8, blockIdx.y = row in chunk).
+// ----------------------------------------------------------------------------
+template <int LOG_N1, int LOG_N2, typename IO, bool INV, bool FWD, bool SPEC_INPUT>
+__global__ void __launch_bounds__(NT) colpass_kernel(const FsParams p) {
+    constexpr int N1 = 1 << LOG_N1;
+    constexpr int N2 = 1 << LOG_N2;
+    constexpr int M = N1 * N2;
+    constexpr int LP = fs_log_p(LOG_N2);
+    constexpr int P = 1 << LP;
+    constexpr int CS = spad_size(N2);           // column stride in the tile
+    using IOT = IOTraits<IO>;
+
+    extern __shared__ float2 tile[];            // WARPS columns x CS
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n1_0 = blockIdx.x * WARPS;
+    const int64_t row = p.row0 + blockIdx.y;
+    const int64_t rl = blockIdx.y;              // row within chunk
+    float2 *buf = p.buf + rl * (int64_t)M;
+    float *stash = p.stash + rl * (int64_t)M;
+    const int L = p.L;
+    float2 *col = tile + warp * CS;
+    float2 x[P];
+
+    if constexpr (INV) {
+        // ---- load all N2 rows of the 8 columns (coalesced float4 = 2 complex)
+        for (int e = tid; e < N2 * (WARPS / 2); e += NT) {
+            const int r = e / (WARPS / 2), c2 = (e % (WARPS / 2)) * 2;
+            const float4 v = __ldcg(reinterpret_cast<const float4 *>(buf + n1_0 + c2 + (int64_t)N1 * r));
+            tile[c2 * CS + spad(r)] = make_float2(v.x, v.y);
+            tile[(c2 + 1) * CS + spad(r)] = make_float2(v.z, v.w);
+        }
+        __syncthreads();
+        load_own<LOG_N2, LP>(x, col, lane);
+        __syncwarp();
+        block_fft<LOG_N2, LP, +1, false, SyncWarp>(x, col, lane, p.tw_n2, SyncWarp{});
+        // keep the first half (n2 < N2/2): samples 2m, 2m+1 with m < M/2
+#pragma unroll
+        for (int m = 0; m < P / 2; ++m) col[spad(lane + 32 * m)] = x[m];
+        __syncthreads();
+        // ---- epilogue: 8 columns x N2/2 rows; each thread handles 2 complex
+        //      = 4 consecutive real samples at 2*(n1_0 + c2 + N1*r)
+        const float dk = p.skip_k ? __ldg(p.skip_k + row % p.D) : 0.f;
+        const IO *g = reinterpret_cast<const IO *>(p.gate_k);
+        const IO *uin = reinterpret_cast<const IO *>(p.u) + row * (int64_t)L;
+        const bool last = (p.k == p.K - 1);
+        IO *yout = reinterpret_cast<IO *>(p.y) + row * (int64_t)L;
+        for (int e = tid; e < (N2 / 2) * (WARPS / 2); e += NT) {
+            const int r = e / (WARPS / 2), c2 = (e % (WARPS / 2)) * 2;
+            const int64_t s0 = 2 * ((int64_t)n1_0 + c2 + (int64_t)N1 * r);   // first real sample
+            float2 a = tile[c2 * CS + spad(r)], b = tile[(c2 + 1) * CS + spad(r)];
+            float v[4] = {a.x * p.scale, a.y * p.scale, b.x * p.scale, b.y * p.scale};
+            float pv[4] = {0.f, 0.f, 0.f, 0.f}, gv[4] = {1.f, 1.f, 1.f, 1.f};
+            if (dk != 0.f) {
+                if (p.k == 0) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        if (s0 + q < L) pv[q] = IOT::load(uin + s0 + q);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        if (s0 + q < L) pv[q] = __ldcg(stash + s0 + q);
+                }
+            }
+            if (g) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (s0 + q < L) gv[q] = IOT::load(g + row * (int64_t)L + s0 + q);
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                v[q] = gv[q] * fmaf(dk, pv[q], v[q]);
+                if (s0 + q >= L) v[q] = 0.f;
+            }
+            if (last) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (s0 + q < L) IOT::store(yout + s0 + q, v[q]);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (s0 + q < L) __stcg(stash + s0 + q, v[q]);
+                tile[c2 * CS + spad(r)] = make_float2(v[0], v[1]);
+                tile[(c2 + 1) * CS + spad(r)] = make_float2(v[2], v[3]);
+            }
+        }
+        if (last || !FWD) return;
+        __syncthreads();
+    } else {
+        // ---- first order: packed input rows n2 < N2/2 of the 8 columns
+        const float *hin = reinterpret_cast<const float *>(p.u);
+        const IO *uin = reinterpret_cast<const IO *>(p.u) + row * (int64_t)L;
+        for (int e = tid; e < (N2 / 2) * (WARPS / 2); e += NT) {
+            const int r = e / (WARPS / 2), c2 = (e % (WARPS / 2)) * 2;
+            const int64_t s0 = 2 * ((int64_t)n1_0 + c2 + (int64_t)N1 * r);
+            float v[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if constexpr (SPEC_INPUT) v[q] = (s0 + q < L) ? __ldg(hin + row * (int64_t)L + s0 + q) : 0.f;
+                else v[q] = (s0 + q < L) ? IOT::load(uin + s0 + q) : 0.f;
+            }
+            tile[c2 * CS + spad(r)] = make_float2(v[0], v[1]);
+            tile[(c2 + 1) * CS + spad(r)] = make_float2(v[2], v[3]);
+        }
+        __syncthreads();
+    }
+    if constexpr (FWD) {
+        // ---- forward column FFT (upper half zero) and W_M^{n1 k2}
+        load_own<LOG_N2, LP>(x, col, lane);
+        __syncwarp();
+        block_fft<LOG_N2, LP, -1, true, SyncWarp>(x, col, lane, p.tw_n2, SyncWarp{});
+        const uint32_t n1 = n1_0 + warp;
+#pragma unroll
+        for (int m = 0; m < P; ++m) {
+            const uint32_t k2 = lane + 32 * m;
+            x[m] = cmul(x[m], tw2(p.tw_m, p.lo_m, (n1 * k2) & (M - 1)));
+            col[spad(k2)] = x[m];
+        }
+        __syncthreads();
+        for (int e = tid; e < N2 * (WARPS / 2); e += NT) {
+            const int r = e / (WARPS / 2), c2 = (e % (WARPS / 2)) * 2;
+            const float2 a = tile[c2 * CS + spad(r)], b = tile[(c2 + 1) * CS + spad(r)];
+            __stcg(reinterpret_cast<float4 *>(buf + n1_0 + c2 + (int64_t)N1 * r), make_float4(a.x, a.y, b.x, b.y));
+        }
+    }
+}
+
+// ----------------------------------------------------------------------------
+// Row pass (B): 8 rows per CTA -- 4 low rows k2 and their mirrors N2 - k2
+// (group 0: rows 0..3, N2/2, N2-1..N2-3).  SPEC: write the half spectrum of
+// the rows instead of multiplying (long filter spectra).
+// ----------------------------------------------------------------------------
+enum { OWN_ALL = 0, OWN_NONE = 1, OWN_SELF0 = 2, OWN_SELFH = 3 };
+
+template <int LOG_N1, int LOG_N2, bool SPEC>
+__global__ void __launch_bounds__(NT) rowpass_kernel(const FsParams p) {
+    constexpr int N1 = 1 << LOG_N1;
+    constexpr int N2 = 1 << LOG_N2;
+    constexpr int M = N1 * N2;
+    constexpr int LP = fs_log_p(LOG_N1);
+    constexpr int P = 1 << LP;
+    constexpr int RS = spad_size(N1);
+    extern __shared__ float2 rows_s[];        // WARPS rows x RS
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = blockIdx.x;
+    const int64_t row = p.row0 + blockIdx.y;
+    const int64_t rl = blockIdx.y;
+    float2 *buf = p.buf + rl * (int64_t)M;
+
+    // rows of this CTA and the pairing of warp w
+    int k2, partner, mode;
+    if (warp < 4) {
+        k2 = 4 * g + warp;
+        if (g == 0 && warp == 0) { mode = OWN_SELF0; partner = warp; }
+        else { mode = OWN_ALL; partner = warp + 4; }
+    } else {
+        if (g == 0 && warp == 4) { k2 = N2 / 2; mode = OWN_SELFH; partner = warp; }
+        else { k2 = N2 - (4 * g + warp - 4); mode = OWN_NONE; partner = warp - 4; }
+    }
+    float2 *own = rows_s + warp * RS;
+    float2 *oth = rows_s + partner * RS;
+
+    // ---- load the row (contiguous) and forward FFT over n1 -> bins k2 + N2 k1
+    float2 x[P];
+    const float2 *src = buf + (int64_t)N1 * k2;
+#pragma unroll
+    for (int m = 0; m < P; ++m) x[m] = __ldcg(src + lane + 32 * m);
+    block_fft<LOG_N1, LP, -1, false, SyncWarp>(x, own, lane, p.tw_n1, SyncWarp{});
+#pragma unroll
+    for (int m = 0; m < P; ++m) own[spad(lane + 32 * m)] = x[m];
+    __syncthreads();
+
+    const int64_t d = row % p.D;
+    const float2 *H = SPEC ? nullptr : p.spec + d * (int64_t)(M + 1);
+    float2 *Ho = SPEC ? p.Hout + row * (int64_t)(M + 1) : nullptr;
+
+    // element (own k1) pairs with partner element pk1 of row partner_k2
+#pragma unroll
+    for (int m = 0; m < P; ++m) {
+        const int k1 = lane + 32 * m;
+        bool owner;
+        int pk1;
+        if (mode == OWN_ALL) { owner = true; pk1 = N1 - 1 - k1; }
+        else if (mode == OWN_NONE) { owner = false; pk1 = 0; }
+        else if (mode == OWN_SELF0) { owner = k1 < N1 / 2; pk1 = (N1 - k1) & (N1 - 1); }
+        else { owner = k1 < N1 / 2; pk1 = N1 - 1 - k1; }
+        if (!owner) continue;
+        const uint32_t k = (uint32_t)k2 + (uint32_t)N2 * k1;
+        const float2 zk = x[m];
+        if (mode == OWN_SELF0 && k1 == 0) {
+            // DC (bin 0) and Nyquist (bin M): both real
+            if constexpr (SPEC) {
+                Ho[0] = make_float2(zk.x + zk.y, 0.f);
+                Ho[M] = make_float2(zk.x - zk.y, 0.f);
+            } else {
+                const float y0 = 2.f * (zk.x + zk.y) * __ldg(&H[0].x);
+                const float yM = 2.f * (zk.x - zk.y) * __ldg(&H[M].x);
+                x[m] = make_float2(y0 + yM, y0 - yM);
+            }
+            continue;
+        }
+        const float2 zn = oth[spad(pk1)];
+        const float2 A = make_float2(zk.x + zn.x, zk.y - zn.y);
+        const float2 Bv = make_float2(zk.x - zn.x, zk.y + zn.y);
+        const float2 w = tw2(p.tw_2m, p.lo_2m, k);                   // W_{2M}^k
+        const float2 wB = cmul(Bv, w);
+        const float2 C = make_float2(wB.y, -wB.x);
+        const float2 Xk = cadd(A, C);                                 // 2 X[k]
+        const float2 Xn = cconj(csub(A, C));                          // 2 X[M-k]
+        if constexpr (SPEC) {
+            Ho[k] = make_float2(0.5f * Xk.x, 0.5f * Xk.y);
+            Ho[M - k] = make_float2(0.5f * Xn.x, 0.5f * Xn.y);
+        } else {
+            const float2 Yk = cmul(Xk, __ldg(H + k));
+            const float2 Yn = cmul(Xn, __ldg(H + (M - k)));
+            const float2 A2 = make_float2(Yk.x + Yn.x, Yk.y - Yn.y);
+            const float2 B2 = make_float2(Yk.x - Yn.x, Yk.y + Yn.y);
+            const float2 cB = cmulc(B2, w);
+            const float2 C2 = make_float2(-cB.y, cB.x);
+            x[m] = cadd(A2, C2);
+            oth[spad(pk1)] = cconj(csub(A2, C2));
+        }
+    }
+    if constexpr (SPEC) {
+        // bin M/2 (row 0, k1 = N1/2) pairs with itself: X[M/2] = conj(Z[M/2])
+        if (mode == OWN_SELF0 && lane == 0) Ho[M / 2] = cconj(x[(N1 / 2) / 32]);
+        return;
+    }
+    // self-paired element of row 0: bin M/2 (k1 = N1/2)
+    if (mode == OWN_SELF0 && lane == 0) {
+        constexpr int mh = (N1 / 2) / 32;
+        const float2 r = cmulc(x[mh], __ldg(H + M / 2));
+        x[mh] = make_float2(4.f * r.x, 4.f * r.y);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < P; ++m) {
+        const int k1 = lane + 32 * m;
+        bool owner;
+        if (mode == OWN_ALL) owner = true;
+        else if (mode == OWN_NONE) owner = false;
+        else owner = k1 < N1 / 2 || (mode == OWN_SELF0 && k1 == N1 / 2);
+        if (!owner) x[m] = own[spad(k1)];
+    }
+    __syncwarp();
+    // ---- inverse FFT over k1 -> n1, times W_M^{-n1 k2}, back to the buffer
+    block_fft<LOG_N1, LP, +1, false, SyncWarp>(x, own, lane, p.tw_n1, SyncWarp{});
+    float2 *dst = buf + (int64_t)N1 * k2;
+#pragma unroll
+    for (int m = 0; m < P; ++m) {
+        const uint32_t n1 = lane + 32 * m;
+        __stcg(dst + n1, cmulc(x[m], tw2(p.tw_m, p.lo_m, (n1 * (uint32_t)k2) & (M - 1))));
+    }
+}
+
+int64_t chunk_rows_of(int64_t rows, int log_mc) {
     const int64_t per_row = (int64_t)12 << log_mc;
-    int64_t c = ((int64_t)64 << 20) / per_row;
+    int64_t c = ((int64_t)96 << 20) / per_row;
     if (c < 1) c = 1;
     return c < rows ? c : rows;
 }
+
+template <typename Kern>
+hy_status smem_attr(Kern k, size_t bytes) {
+    if (bytes > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+        if (e != cudaSuccess) return set_cuda_error("multi-pass smem attribute", e);
+    }
+    return HY_OK;
+}
+
+template <int LOG_N1, int LOG_N2, typename IO>
+hy_status run_conv(const LongConvArgs &a, cudaStream_t s) {
+    constexpr int N1 = 1 << LOG_N1, N2 = 1 << LOG_N2;
+    constexpr int LOG_MC = LOG_N1 + LOG_N2;
+    const int64_t rows = a.B * a.D;
+    const int64_t cr = chunk_rows_of(rows, LOG_MC);
+    FsParams p{};
+    p.D = a.D;
+    p.L = (int)a.L;
+    p.K = a.K;
+    p.u = a.u;
+    p.y = a.y;
+    p.buf = reinterpret_cast<float2 *>(a.ws);
+    p.stash = reinterpret_cast<float *>(reinterpret_cast<char *>(a.ws) + (size_t)cr * ((size_t)8 << LOG_MC));
+    p.scale = (float)(1.0 / (4.0 * (double)((int64_t)1 << LOG_MC)));
+    p.tw_n1 = tw_stages(LOG_N1, fs_log_p(LOG_N1));
+    p.tw_n2 = tw_stages(LOG_N2, fs_log_p(LOG_N2));
+    p.lo_m = LOG_MC / 2;
+    p.tw_m = tw_pow2(LOG_MC, p.lo_m);
+    p.lo_2m = (LOG_MC + 1) / 2;
+    p.tw_2m = tw_pow2(LOG_MC + 1, p.lo_2m);
+    if (!p.tw_n1 || !p.tw_n2 || !p.tw_m || !p.tw_2m) return set_error(HY_ERR_CUDA, "multi-pass twiddle tables missing");
+    const size_t smem_c = sizeof(float2) * WARPS * spad_size(N2);
+    const size_t smem_r = sizeof(float2) * WARPS * spad_size(N1);
+    auto kA = colpass_kernel<LOG_N1, LOG_N2, IO, false, true, false>;
+    auto kCA = colpass_kernel<LOG_N1, LOG_N2, IO, true, true, false>;
+    auto kC = colpass_kernel<LOG_N1, LOG_N2, IO, true, false, false>;
+    auto kB = rowpass_kernel<LOG_N1, LOG_N2, false>;
+    hy_status st;
+    if ((st = smem_attr(kA, smem_c)) != HY_OK || (st = smem_attr(kCA, smem_c)) != HY_OK ||
+        (st = smem_attr(kC, smem_c)) != HY_OK || (st = smem_attr(kB, smem_r)) != HY_OK)
+        return st;
+    for (int64_t r0 = 0; r0 < rows; r0 += cr) {
+        const int64_t nr = (rows - r0) < cr ? (rows - r0) : cr;
+        p.row0 = r0;
+        dim3 gc(N1 / WARPS, (unsigned)nr), gr(N2 / 8, (unsigned)nr);
+        p.k = 0;
+        kA<<<gc, NT, smem_c, s>>>(p);
+        for (int k = 0; k < a.K; ++k) {
+            p.k = k;
+            p.spec = a.spec[k];
+            p.gate_k = a.gate[k];
+            p.skip_k = a.skip[k];
+            kB<<<gr, NT, smem_r, s>>>(p);
+            if (k + 1 < a.K) kCA<<<gc, NT, smem_c, s>>>(p);
+            else kC<<<gc, NT, smem_c, s>>>(p);
+        }
+        if ((st = check_launch("multi-pass conv launch")) != HY_OK) return st;
+    }
+    return HY_OK;
+}
+
+template <int LOG_N1, int LOG_N2>
+hy_status run_spectrum(int64_t rows, int64_t L, const float *h, float2 *H, void *ws, cudaStream_t s) {
+    constexpr int N1 = 1 << LOG_N1, N2 = 1 << LOG_N2;
+    constexpr int LOG_MC = LOG_N1 + LOG_N2;
+    const int64_t cr = chunk_rows_of(rows, LOG_MC);
+    FsParams p{};
+    p.D = 1;
+    p.L = (int)L;
+    p.K = 1;
+    p.u = h;
+    p.buf = reinterpret_cast<float2 *>(ws);
+    p.stash = nullptr;
+    p.Hout = H;
+    p.tw_n1 = tw_stages(LOG_N1, fs_log_p(LOG_N1));
+    p.tw_n2 = tw_stages(LOG_N2, fs_log_p(LOG_N2));
+    p.lo_m = LOG_MC / 2;
+    p.tw_m = tw_pow2(LOG_MC, p.lo_m);
+    p.lo_2m = (LOG_MC + 1) / 2;
+    p.tw_2m = tw_pow2(LOG_MC + 1, p.lo_2m);
+    if (!p.tw_n1 || !p.tw_n2 || !p.tw_m || !p.tw_2m) return set_error(HY_ERR_CUDA, "multi-pass twiddle tables missing");
+    const size_t smem_c = sizeof(float2) * WARPS * spad_size(N2);
+    const size_t smem_r = sizeof(float2) * WARPS * spad_size(N1);
+    auto kA = colpass_kernel<LOG_N1, LOG_N2, float, false, true, true>;
+    auto kB = rowpass_kernel<LOG_N1, LOG_N2, true>;
+    hy_status st;
+    if ((st = smem_attr(kA, smem_c)) != HY_OK || (st = smem_attr(kB, smem_r)) != HY_OK) return st;
+    for (int64_t r0 = 0; r0 < rows; r0 += cr) {
+        const int64_t nr = (rows - r0) < cr ? (rows - r0) : cr;
+        p.row0 = r0;
+        kA<<<dim3(N1 / WARPS, (unsigned)nr), NT, smem_c, s>>>(p);
+        kB<<<dim3(N2 / 8, (unsigned)nr), NT, smem_r, s>>>(p);
+        if ((st = check_launch("multi-pass spectrum launch")) != HY_OK) return st;
+    }
+    return HY_OK;
+}
+
+}  // namespace
+
 size_t long_conv_workspace(int64_t B, int64_t D, int log_mc, int) {
-    if (log_mc < 15 || log_mc > 22) return 0;
-    return (size_t)chunk_rows(B * D, log_mc) * ((size_t)12 << log_mc);
+    if (log_mc < 15 || log_mc > 20) return 0;
+    return (size_t)chunk_rows_of(B * D, log_mc) * ((size_t)12 << log_mc);
 }
-hy_status launch_long_conv(const LongConvArgs &, cudaStream_t) {
-    return set_error(HY_ERR_UNSUPPORTED, "multi-pass path not built");
+
+size_t long_spectrum_workspace(int64_t rows, int log_mc) {
+    if (log_mc < 15 || log_mc > 20) return 0;
+    return (size_t)chunk_rows_of(rows, log_mc) * ((size_t)12 << log_mc);
 }
-size_t long_spectrum_workspace(int64_t, int) { return 0; }
-hy_status launch_long_spectrum(int64_t, int64_t, int, const float *, float2 *, void *, size_t, cudaStream_t) {
-    return set_error(HY_ERR_UNSUPPORTED, "multi-pass path not built");
+
+hy_status launch_long_conv(const LongConvArgs &a, cudaStream_t s) {
+    const bool bf = a.dt == HY_BF16;
+    switch (a.log_mc) {
+#define HY_LC(LM, N1L, N2L) \
+    case LM: return bf ? run_conv<N1L, N2L, __nv_bfloat16>(a, s) : run_conv<N1L, N2L, float>(a, s);
+        HY_LC(15, 7, 8) HY_LC(16, 8, 8) HY_LC(17, 8, 9) HY_LC(18, 9, 9) HY_LC(19, 9, 10) HY_LC(20, 10, 10)
+#undef HY_LC
+        default: return set_error(HY_ERR_UNSUPPORTED, "multi-pass length 2^%d not built", a.log_mc);
+    }
 }
+
+hy_status launch_long_spectrum(int64_t rows, int64_t L, int log_mc, const float *h, float2 *H, void *ws,
+                               size_t ws_bytes, cudaStream_t s) {
+    (void)ws_bytes;
+    switch (log_mc) {
+#define HY_LS(LM, N1L, N2L) \
+    case LM: return run_spectrum<N1L, N2L>(rows, L, h, H, ws, s);
+        HY_LS(15, 7, 8) HY_LS(16, 8, 8) HY_LS(17, 8, 9) HY_LS(18, 9, 9) HY_LS(19, 9, 10) HY_LS(20, 10, 10)
+#undef HY_LS
+        default: return set_error(HY_ERR_UNSUPPORTED, "multi-pass length 2^%d not built", log_mc);
+    }
+}
+
 }  // namespace hy

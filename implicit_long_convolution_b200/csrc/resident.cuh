@@ -53,35 +53,51 @@ __device__ __forceinline__ void split_multiply_merge(float2 (&x)[1 << LOG_P], fl
     constexpr int P = 1 << LOG_P;
     constexpr int T = M / P;
     store_own<LOG_M, LOG_P>(x, sbuf, t);
+    // bins k = t + m*T (m < P/2) pair with M - k; the loads of a batch of
+    // pairs are issued together so their L2 round trips overlap
+    constexpr int BATCH = (P / 2) < 4 ? (P / 2) : 4;
     __syncthreads();
 #pragma unroll
-    for (int m = 0; m < P / 2; ++m) {
-        const int k = t + m * T;
-        if (k == 0) {
-            // DC and Nyquist: X[0] = Re Z0 + Im Z0, X[M] = Re Z0 - Im Z0 (both
-            // real, doubled here); only the real part of the product is kept.
-            const float2 z0 = x[0];
-            const float y0 = 2.f * (z0.x + z0.y) * ldv(&H[0].x);
-            const float yM = 2.f * (z0.x - z0.y) * ldv(&H[M].x);
-            x[0] = make_float2(y0 + yM, y0 - yM);
-        } else {
-            const float2 zk = x[m];
-            const float2 zn = sbuf[partner_slot<LOG_M, LOG_P>(t, m)];
-            const float2 A = make_float2(zk.x + zn.x, zk.y - zn.y);   // Z[k] + Z*[M-k]
-            const float2 Bv = make_float2(zk.x - zn.x, zk.y + zn.y);  // Z[k] - Z*[M-k]
-            const float2 w = ldv(tws + k);                          // W_n^k
-            const float2 wB = cmul(Bv, w);
-            const float2 C = make_float2(wB.y, -wB.x);                // -i W B
-            const float2 Xk = cadd(A, C);                             // 2 X[k]
-            const float2 Xn = cconj(csub(A, C));                      // 2 X[M-k]
-            const float2 Yk = cmul(Xk, ldv(H + k));
-            const float2 Yn = cmul(Xn, ldv(H + (M - k)));
-            const float2 A2 = make_float2(Yk.x + Yn.x, Yk.y - Yn.y);
-            const float2 B2 = make_float2(Yk.x - Yn.x, Yk.y + Yn.y);
-            const float2 cB = cmulc(B2, w);
-            const float2 C2 = make_float2(-cB.y, cB.x);               // i W^-1 B'
-            x[m] = cadd(A2, C2);
-            sbuf[partner_slot<LOG_M, LOG_P>(t, m)] = cconj(csub(A2, C2));
+    for (int m0 = 0; m0 < P / 2; m0 += BATCH) {
+        float2 hk[BATCH], hn[BATCH], wk[BATCH];
+#pragma unroll
+        for (int j = 0; j < BATCH; ++j) {
+            const int k = t + (m0 + j) * T;
+            hk[j] = ldv(H + k);
+            hn[j] = ldv(H + (M - k));
+            wk[j] = ldc(tws + k);
+        }
+#pragma unroll
+        for (int j = 0; j < BATCH; ++j) {
+            const int m = m0 + j;
+            const int k = t + m * T;
+            if (k == 0) {
+                // DC and Nyquist: X[0] = Re Z0 + Im Z0, X[M] = Re Z0 - Im Z0
+                // (both real, doubled here); only the real part of the product
+                // is kept.  H[M] = hn[j] at k = 0.
+                const float2 z0 = x[0];
+                const float y0 = 2.f * (z0.x + z0.y) * hk[j].x;
+                const float yM = 2.f * (z0.x - z0.y) * hn[j].x;
+                x[0] = make_float2(y0 + yM, y0 - yM);
+            } else {
+                const float2 zk = x[m];
+                const float2 zn = sbuf[partner_slot<LOG_M, LOG_P>(t, m)];
+                const float2 A = make_float2(zk.x + zn.x, zk.y - zn.y);   // Z[k] + Z*[M-k]
+                const float2 Bv = make_float2(zk.x - zn.x, zk.y + zn.y);  // Z[k] - Z*[M-k]
+                const float2 w = wk[j];                                   // W_n^k
+                const float2 wB = cmul(Bv, w);
+                const float2 C = make_float2(wB.y, -wB.x);                // -i W B
+                const float2 Xk = cadd(A, C);                             // 2 X[k]
+                const float2 Xn = cconj(csub(A, C));                      // 2 X[M-k]
+                const float2 Yk = cmul(Xk, hk[j]);
+                const float2 Yn = cmul(Xn, hn[j]);
+                const float2 A2 = make_float2(Yk.x + Yn.x, Yk.y - Yn.y);
+                const float2 B2 = make_float2(Yk.x - Yn.x, Yk.y + Yn.y);
+                const float2 cB = cmulc(B2, w);
+                const float2 C2 = make_float2(-cB.y, cB.x);               // i W^-1 B'
+                x[m] = cadd(A2, C2);
+                sbuf[partner_slot<LOG_M, LOG_P>(t, m)] = cconj(csub(A2, C2));
+            }
         }
     }
     if (t == 0) {
@@ -153,53 +169,64 @@ resident_conv_kernel(const ResidentParams p) {
 
         const float dk = p.skip[k] ? ldv(p.skip[k] + ch) : 0.f;
         const IO *g = reinterpret_cast<const IO *>(p.gate[k]);
+        const IO *grow = g ? g + row * (int64_t)L : nullptr;
         IO *yout = reinterpret_cast<IO *>(p.y) + row * (int64_t)L;
+        // batches of EB samples: issue the batch's gate / skip loads first
+        // (the output stores would otherwise order each load behind them)
+        constexpr int EB = (PIN < 8) ? PIN : 8;
 #pragma unroll
-        for (int m = 0; m < P; ++m) {
-            if (m >= PIN) {
-                x[m] = make_float2(0.f, 0.f);
-                continue;
-            }
-            const int e = t + m * T;
-            const int i0 = 2 * e;
-            float2 prev = make_float2(0.f, 0.f);
-            if (k == 0) {
-                if (dk != 0.f) {
+        for (int m0 = 0; m0 < PIN; m0 += EB) {
+            float2 gv[EB], pv[EB];
+#pragma unroll
+            for (int j = 0; j < EB; ++j) {
+                const int i0 = 2 * (t + (m0 + j) * T);
+                gv[j] = make_float2(1.f, 1.f);
+                pv[j] = make_float2(0.f, 0.f);
+                if (grow) {
                     if (pairs) {
-                        if (i0 < L) prev = IOT::load2(u + i0);
+                        if (i0 < L) gv[j] = IOT::load2(grow + i0);
                     } else {
-                        if (i0 < L) prev.x = IOT::load(u + i0);
-                        if (i0 + 1 < L) prev.y = IOT::load(u + i0 + 1);
+                        if (i0 < L) gv[j].x = IOT::load(grow + i0);
+                        if (i0 + 1 < L) gv[j].y = IOT::load(grow + i0 + 1);
                     }
                 }
-            } else {
-                prev = ustash[e];
-            }
-            float2 z = make_float2(fmaf(x[m].x, p.scale, dk * prev.x), fmaf(x[m].y, p.scale, dk * prev.y));
-            if (g) {
-                float2 gv = make_float2(0.f, 0.f);
-                if (pairs) {
-                    if (i0 < L) gv = IOT::load2(g + row * (int64_t)L + i0);
+                if (k == 0) {
+                    if (dk != 0.f) {
+                        if (pairs) {
+                            if (i0 < L) pv[j] = IOT::load2(u + i0);
+                        } else {
+                            if (i0 < L) pv[j].x = IOT::load(u + i0);
+                            if (i0 + 1 < L) pv[j].y = IOT::load(u + i0 + 1);
+                        }
+                    }
                 } else {
-                    if (i0 < L) gv.x = IOT::load(g + row * (int64_t)L + i0);
-                    if (i0 + 1 < L) gv.y = IOT::load(g + row * (int64_t)L + i0 + 1);
+                    pv[j] = ustash[t + (m0 + j) * T];
                 }
-                z = make_float2(z.x * gv.x, z.y * gv.y);
             }
-            if (i0 >= L) z.x = 0.f;
-            if (i0 + 1 >= L) z.y = 0.f;
-            if (last) {
-                if (pairs) {
-                    if (i0 < L) IOT::store2(yout + i0, z);
+#pragma unroll
+            for (int j = 0; j < EB; ++j) {
+                const int m = m0 + j;
+                const int e = t + m * T;
+                const int i0 = 2 * e;
+                float2 z = make_float2(fmaf(x[m].x, p.scale, dk * pv[j].x), fmaf(x[m].y, p.scale, dk * pv[j].y));
+                z = make_float2(z.x * gv[j].x, z.y * gv[j].y);
+                if (i0 >= L) z.x = 0.f;
+                if (i0 + 1 >= L) z.y = 0.f;
+                if (last) {
+                    if (pairs) {
+                        if (i0 < L) IOT::store2(yout + i0, z);
+                    } else {
+                        if (i0 < L) IOT::store(yout + i0, z.x);
+                        if (i0 + 1 < L) IOT::store(yout + i0 + 1, z.y);
+                    }
                 } else {
-                    if (i0 < L) IOT::store(yout + i0, z.x);
-                    if (i0 + 1 < L) IOT::store(yout + i0 + 1, z.y);
+                    ustash[e] = z;
+                    x[m] = z;
                 }
-            } else {
-                ustash[e] = z;
-                x[m] = z;
             }
         }
+#pragma unroll
+        for (int m = PIN; m < P; ++m) x[m] = make_float2(0.f, 0.f);
     };
 
     if constexpr (CHAIN) {

@@ -54,6 +54,25 @@ def check(a, ref, dtype, what=""):
     return r
 
 
+def check_part(a, ref, rms_full, dtype, what=""):
+    """The same tolerance for a slice of an output (a prefix, sampled
+    positions), with errors measured against the RMS of the whole output the
+    slice belongs to: RMS(err) <= 1e-5 * RMS_full and max-abs <= 1e-4 * RMS_full
+    for fp32; RMS(err) <= 1e-2 * RMS_full for bf16 I/O."""
+    a = np.asarray(a, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert a.shape == ref.shape
+    assert np.all(np.isfinite(a)), what + ": non-finite output"
+    err = a - ref
+    rms_err = float(np.sqrt(np.mean(err ** 2)))
+    tol = BF16_REL_L2 if dtype == "bf16" else F32_REL_L2
+    assert rms_err <= tol * rms_full, "%s: RMS err %.3e > %.0e * %.3e" % (what, rms_err, tol, rms_full)
+    if dtype != "bf16":
+        mx = float(np.max(np.abs(err)))
+        assert mx <= F32_MAXABS_OF_RMS * rms_full, "%s: max-abs %.3e" % (what, mx)
+    return rms_err / rms_full
+
+
 def bf16_ulp_diff(dev_bf16_tensor, ref64, floor_of_rms=1e-2):
     """Largest distance in bf16 units-in-the-last-place between the device's
     bf16 output and the float64 reference rounded to bf16, over elements whose

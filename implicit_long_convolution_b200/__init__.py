@@ -20,7 +20,7 @@ from typing import Optional, Sequence
 __all__ = [
     "HyenaError", "HyenaLibraryMissing", "LIB_PATH", "lib", "spectrum_bins",
     "hyena_filter_gen", "hyena_filter_spectrum", "filter_spectrum_workspace",
-    "hyena_fftconv", "hyena_operator", "operator_workspace", "hyena_nd_conv",
+    "hyena_fftconv", "hyena_operator", "operator_workspace", "hyena_operator_noalloc", "hyena_nd_conv",
     "nd_conv_workspace", "spectral_gate", "STATUS",
 ]
 
@@ -84,6 +84,8 @@ def lib():
         "hyena_operator_workspace": (_SZ, [_I, _I, _I, _I, _I]),
         "hyena_operator": (_I, [_I, _I, _I, _I, _I, _VP, ctypes.POINTER(_VP), ctypes.POINTER(_VP),
                                 ctypes.POINTER(_VP), _VP, _VP, _SZ, _VP]),
+        "hyena_operator_noalloc": (_I, [_I, _I, _I, _I, _I, _VP, ctypes.POINTER(_VP), ctypes.POINTER(_VP),
+                                        ctypes.POINTER(_VP), _VP, _VP]),
         "hyena_nd_conv_workspace": (_SZ, [_I, ctypes.POINTER(_I), _I, _I, _I]),
         "hyena_nd_conv": (_I, [_I, ctypes.POINTER(_I), _I, _I, _I, _VP, _VP, _I64, _VP, _VP, _VP,
                                _VP, _SZ, _VP]),
@@ -186,6 +188,18 @@ def hyena_operator(v, xs: Sequence, Hs: Sequence, y, *, Dskips: Optional[Sequenc
     wsb = ws.numel() * ws.element_size() if ws is not None else 0
     _check(lib().hyena_operator(order, B, D, L, _dt(v), _ptr(v), _ptrs(xs), _ptrs(Hs), dsk, _ptr(y),
                                 _ptr(ws), wsb, _stream(stream)))
+    return y
+
+
+def hyena_operator_noalloc(v, xs: Sequence, Hs: Sequence, y, *, Dskips: Optional[Sequence] = None,
+                           stream=None):
+    """hyena_operator for callers that cannot allocate device memory: long
+    sequences use the library's static device scratch (see hyena.h)."""
+    B, D, L = v.shape
+    order = len(xs) + 1
+    dsk = _ptrs(Dskips) if Dskips is not None else None
+    _check(lib().hyena_operator_noalloc(order, B, D, L, _dt(v), _ptr(v), _ptrs(xs), _ptrs(Hs), dsk,
+                                        _ptr(y), _stream(stream)))
     return y
 
 

@@ -358,3 +358,66 @@ hy_status spectral_gate(int B, int H, int Dh, int L, hy_dtype dt, const void *x,
 }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------------------
+// hyena_operator_noalloc: the operator for callers that cannot allocate device
+// memory (see include/hyena.h).  Sequences that fit on chip run exactly as in
+// hyena_operator; longer ones use the multi-pass kernels with their workspace
+// in the library's static device scratch instead of a caller buffer.
+// ----------------------------------------------------------------------------
+extern "C" hy_status hyena_operator_noalloc(int order, int B, int D, int L, hy_dtype dt, const void *v,
+                                            const void *const *x, const hy_c32 *const *H,
+                                            const float *const *Dskip, void *y, void *stream) {
+    clear_error();
+    const char *who = "hyena_operator_noalloc";
+    if (order < 2 || order - 1 > kMaxOrders)
+        return set_error(HY_ERR_UNSUPPORTED, "%s: order must be 2..%d", who, kMaxOrders + 1);
+    if (!x || !H) return set_error(HY_ERR_INVALID_ARG, "%s: null x or H array", who);
+    const int K = order - 1;
+    for (int k = 0; k < K; ++k)
+        if (!x[k]) return set_error(HY_ERR_INVALID_ARG, "%s: x[%d] is null", who, k);
+    if (B < 1 || D < 1 || L < 1) return set_error(HY_ERR_INVALID_ARG, "%s: B, D, L must be >= 1", who);
+    if (dt != HY_F32 && dt != HY_BF16) return set_error(HY_ERR_INVALID_ARG, "%s: unknown dtype", who);
+    if (!v || !y) return set_error(HY_ERR_INVALID_ARG, "%s: null signal pointer", who);
+    const size_t esz = dt_size(dt);
+    const size_t nbytes = (size_t)B * D * L * esz;
+    const size_t al = (L % 2 == 0) ? 2 * esz : esz;
+    if (!aligned(v, al) || !aligned(y, al))
+        return set_error(HY_ERR_INVALID_ARG, "%s: signals must be %zu-byte aligned", who, al);
+    if (overlap(v, nbytes, y, nbytes)) return set_error(HY_ERR_INVALID_ARG, "%s: y aliases the input", who);
+    const int64_t M = spectrum_m(L);
+    for (int k = 0; k < K; ++k) {
+        if (!H[k] || !aligned(H[k], 8)) return set_error(HY_ERR_INVALID_ARG, "%s: spectrum %d null or misaligned", who, k);
+        if (!aligned(x[k], al)) return set_error(HY_ERR_INVALID_ARG, "%s: gate %d misaligned", who, k);
+        if (overlap(x[k], nbytes, y, nbytes)) return set_error(HY_ERR_INVALID_ARG, "%s: y aliases gate %d", who, k);
+    }
+    const int log_m = ilog2(M);
+    if (log_m <= kMaxResidentLogM) {
+        // on chip: no workspace of any kind
+        const void *no_ws = nullptr;
+        return run_chain(K, B, D, L, dt, v, x, H, Dskip, y, const_cast<void *>(no_ws), 0,
+                         (cudaStream_t)stream, who);
+    }
+    // one row's intermediates (12 bytes per complex point) must fit the scratch
+    if ((size_t)12 * (size_t)M > noalloc_scratch_bytes())
+        return set_error(HY_ERR_WORKSPACE, "%s: L=%d needs %zu scratch bytes per row; the static scratch holds %zu",
+                         who, L, (size_t)12 * (size_t)M, noalloc_scratch_bytes());
+    if (log_m > 20) return set_error(HY_ERR_UNSUPPORTED, "%s: L=%d is beyond the supported length", who, L);
+    hy_status st = prologue((cudaStream_t)stream);
+    if (st != HY_OK) return st;
+    LongConvArgs a{};
+    a.K = K;
+    a.B = B;
+    a.D = D;
+    a.L = L;
+    a.log_mc = log_m;
+    a.dt = dt;
+    a.u = v;
+    for (int k = 0; k < K; ++k) {
+        a.gate[k] = x[k];
+        a.spec[k] = reinterpret_cast<const float2 *>(H[k]);
+        a.skip[k] = Dskip ? Dskip[k] : nullptr;
+    }
+    a.y = y;
+    return launch_long_conv_noalloc(a, (cudaStream_t)stream);
+}

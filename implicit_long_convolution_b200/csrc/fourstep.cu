@@ -24,6 +24,8 @@
 // warp synchronisation); columns are staged through shared memory so global
 // accesses stay coalesced.  Rows are processed in chunks whose intermediates
 // (8 bytes per complex point) stay resident in the 126 MB L2 between passes.
+#include <mutex>
+
 #include "kernels.h"
 #include "fft_core.cuh"
 #include "status.h"
@@ -459,6 +461,125 @@ hy_status launch_long_spectrum(int64_t rows, int64_t L, int log_mc, const float 
         HY_LS(15, 7, 8) HY_LS(16, 8, 8) HY_LS(17, 8, 9) HY_LS(18, 9, 9) HY_LS(19, 9, 10) HY_LS(20, 10, 10)
 #undef HY_LS
         default: return set_error(HY_ERR_UNSUPPORTED, "multi-pass length 2^%d not built", log_mc);
+    }
+}
+
+}  // namespace hy
+
+// ============================================================================
+// Allocation-free variant of the multi-pass operator.
+//
+// Some callers cannot call cudaMalloc at all: code running inside a custom
+// allocator or a memory-pool callback, plugins whose host framework owns every
+// device allocation, and real-time loops that must not touch the driver's
+// allocator.  For them the multi-pass workspace lives in a fixed static device
+// array instead of a caller buffer.  Rows are processed in chunks sized to
+// that array, with the same kernels as launch_long_conv.
+// ============================================================================
+namespace hy {
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = (size_t)32 << 20;   // 32 MiB per device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[64] = {nullptr};
+
+// Device address of the scratch array for the current device.  Host code
+// cannot use the array's name as a device address; it is resolved once per
+// device with cudaGetSymbolAddress while that device is current.
+hy_status noalloc_scratch(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return set_cuda_error("cudaGetDevice", e);
+    if (dev < 0 || dev >= 64) return set_error(HY_ERR_UNSUPPORTED, "device index %d >= 64", dev);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return set_cuda_error("cudaGetSymbolAddress(no-alloc scratch)", e);
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return HY_OK;
+}
+
+template <int LOG_N1, int LOG_N2, typename IO>
+hy_status run_conv_static(const LongConvArgs &a, void *scratch, cudaStream_t s) {
+    constexpr int N1 = 1 << LOG_N1, N2 = 1 << LOG_N2;
+    constexpr int LOG_MC = LOG_N1 + LOG_N2;
+    const int64_t rows = a.B * a.D;
+    const size_t per_row = (size_t)12 << LOG_MC;
+    int64_t cr = (int64_t)(kNoAllocScratchBytes / per_row);
+    if (cr < 1)
+        return set_error(HY_ERR_WORKSPACE, "hyena_operator_noalloc: one row needs %zu bytes, the static scratch holds %zu",
+                         per_row, kNoAllocScratchBytes);
+    if (cr > rows) cr = rows;
+    FsParams p{};
+    p.D = a.D;
+    p.L = (int)a.L;
+    p.K = a.K;
+    p.u = a.u;
+    p.y = a.y;
+    p.buf = reinterpret_cast<float2 *>(scratch);
+    p.stash = reinterpret_cast<float *>(reinterpret_cast<char *>(scratch) + (size_t)cr * ((size_t)8 << LOG_MC));
+    p.scale = (float)(1.0 / (4.0 * (double)((int64_t)1 << LOG_MC)));
+    p.tw_n1 = tw_stages(LOG_N1, fs_log_p(LOG_N1));
+    p.tw_n2 = tw_stages(LOG_N2, fs_log_p(LOG_N2));
+    p.lo_m = LOG_MC / 2;
+    p.tw_m = tw_pow2(LOG_MC, p.lo_m);
+    p.lo_2m = (LOG_MC + 1) / 2;
+    p.tw_2m = tw_pow2(LOG_MC + 1, p.lo_2m);
+    if (!p.tw_n1 || !p.tw_n2 || !p.tw_m || !p.tw_2m) return set_error(HY_ERR_CUDA, "multi-pass twiddle tables missing");
+    const size_t smem_c = sizeof(float2) * WARPS * spad_size(N2);
+    const size_t smem_r = sizeof(float2) * WARPS * spad_size(N1);
+    auto kA = colpass_kernel<LOG_N1, LOG_N2, IO, false, true, false>;
+    auto kCA = colpass_kernel<LOG_N1, LOG_N2, IO, true, true, false>;
+    auto kC = colpass_kernel<LOG_N1, LOG_N2, IO, true, false, false>;
+    auto kB = rowpass_kernel<LOG_N1, LOG_N2, false>;
+    hy_status st;
+    if ((st = smem_attr(kA, smem_c)) != HY_OK || (st = smem_attr(kCA, smem_c)) != HY_OK ||
+        (st = smem_attr(kC, smem_c)) != HY_OK || (st = smem_attr(kB, smem_r)) != HY_OK)
+        return st;
+    // Nothing in the scratch has to start at zero: pass A writes every complex
+    // point of a row before pass B reads it, and the fp32 stash is written by
+    // one order before the next order reads it.
+    for (int64_t r0 = 0; r0 < rows; r0 += cr) {
+        const int64_t nr = (rows - r0) < cr ? (rows - r0) : cr;
+        p.row0 = r0;
+        dim3 gc(N1 / WARPS, (unsigned)nr), gr(N2 / 8, (unsigned)nr);
+        p.k = 0;
+        kA<<<gc, NT, smem_c, s>>>(p);
+        for (int k = 0; k < a.K; ++k) {
+            p.k = k;
+            p.spec = a.spec[k];
+            p.gate_k = a.gate[k];
+            p.skip_k = a.skip[k];
+            kB<<<gr, NT, smem_r, s>>>(p);
+            if (k + 1 < a.K) kCA<<<gc, NT, smem_c, s>>>(p);
+            else kC<<<gc, NT, smem_c, s>>>(p);
+        }
+        if ((st = check_launch("no-alloc multi-pass launch")) != HY_OK) return st;
+    }
+    return HY_OK;
+}
+
+}  // namespace
+
+size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+hy_status launch_long_conv_noalloc(const LongConvArgs &a, cudaStream_t s) {
+    void *scratch = nullptr;
+    hy_status st = noalloc_scratch(&scratch);
+    if (st != HY_OK) return st;
+    const bool bf = a.dt == HY_BF16;
+    switch (a.log_mc) {
+#define HY_LC(LM, N1L, N2L) \
+    case LM: return bf ? run_conv_static<N1L, N2L, __nv_bfloat16>(a, scratch, s) : run_conv_static<N1L, N2L, float>(a, scratch, s);
+        HY_LC(15, 7, 8) HY_LC(16, 8, 8) HY_LC(17, 8, 9) HY_LC(18, 9, 9) HY_LC(19, 9, 10) HY_LC(20, 10, 10)
+#undef HY_LC
+        default: return set_error(HY_ERR_UNSUPPORTED, "hyena_operator_noalloc: length 2^%d beyond the static scratch", a.log_mc);
     }
 }
 

@@ -37,6 +37,11 @@ size_t long_spectrum_workspace(int64_t rows, int log_mc);
 hy_status launch_long_spectrum(int64_t rows, int64_t L, int log_mc, const float *h, float2 *H, void *ws,
                                size_t ws_bytes, cudaStream_t s);
 
+// Multi-pass operator with its workspace in a static device array
+// (fourstep.cu); no allocation by anyone.
+size_t noalloc_scratch_bytes();
+hy_status launch_long_conv_noalloc(const LongConvArgs &a, cudaStream_t s);
+
 // N-D path (ndconv.cu)
 struct NDArgs {
     int g[3];                      // grid

@@ -159,6 +159,37 @@ hy_status hyena_operator(int order, int B, int D, int L, hy_dtype dt, const void
                          void *stream);
 
 /* ------------------------------------------------------------------------
+ * hyena_operator_noalloc -- the operator above for callers that cannot
+ * allocate device memory.  (The pages have no counterpart: this is a
+ * deployment variant, not part of the method.)
+ *
+ * Who needs it: code that runs where cudaMalloc is off limits -- inside a
+ * custom allocator or a memory-pool callback, in a plugin whose host
+ * framework owns every device allocation, or in a real-time loop that must
+ * not enter the driver's allocator.  Such a caller cannot provide the
+ * workspace hyena_operator asks for on long sequences.
+ *
+ * Same arguments and results as hyena_operator, without ws / ws_bytes.
+ * Sequences with hyena_spectrum_bins(L) - 1 <= 16384 run on chip as in
+ * hyena_operator (no workspace at all).  Longer ones keep their intermediates
+ * in one static device array of 32 MiB that the library reserves on every
+ * GPU that loads it, until the process exits; one row needs 12 bytes per
+ * complex point, so L <= 1,048,576 (longer is rejected with
+ * HY_ERR_WORKSPACE or HY_ERR_UNSUPPORTED).  The call allocates nothing and
+ * calls no allocating routine.
+ *
+ * The first call on a device looks up the array's device address (and, like
+ * every entry point, uploads the twiddle tables); make that first call before
+ * any stream capture.  Every call shares the one array and leaves its
+ * contents behind; no part of it needs to start at zero.  Calls whose
+ * execution overlaps on the GPU (other streams, other host threads) race on
+ * the array: order them on one stream or serialise them.
+ * ---------------------------------------------------------------------- */
+hy_status hyena_operator_noalloc(int order, int B, int D, int L, hy_dtype dt, const void *v,
+                                 const void *const *x, const hy_c32 *const *H,
+                                 const float *const *Dskip, void *y, void *stream);
+
+/* ------------------------------------------------------------------------
  * N-D global convolution with gating  ([ND] 네이티브 ND 합성곱, 경계 처리)
  *
  *   y[b,d,p] = gate[b,d,p] · ( Σ_q K_{b,d}[(p - q) mod S] u[b,d,q]

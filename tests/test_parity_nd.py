@@ -1,0 +1,152 @@
+"""Parity of the HyenaND 3-D path (filter generator on the grid, 3-D filter
+spectrum, gated global convolution) against the float64 oracle: tiny grids on
+every voxel by the direct definition, shared and per-sample kernels, circular
+and zero-padded boundaries, skip and gate, and workload 4 at full size
+(B2 D128 64^3, FiLM-conditioned filters)."""
+import numpy as np
+import pytest
+
+import hyena_workloads as hw
+import oracle
+from _helpers import c64_dev, check, check_part, f32_dev, to_np
+
+pytestmark = pytest.mark.gpu
+torch = pytest.importorskip("torch")
+import implicit_long_convolution_b200 as hy  # noqa: E402
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.set_device(0)
+
+
+def gpu_spectrum3(Kern, circular=False):
+    """(R, S, S, S) float32 kernels -> device (R, S, S, S/2+1) via the library."""
+    R, S = Kern.shape[0], Kern.shape[1]
+    H = torch.empty((R, S, S, S // 2 + 1), dtype=torch.complex64, device="cuda")
+    g = S if circular else S // 2
+    wsb = hy.filter_spectrum_workspace(R, 3, [g, g, g], circular)
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device="cuda")
+    hy.hyena_filter_spectrum(f32_dev(Kern.reshape(R, -1)), H, rows=R, ndim=3, dims=[g, g, g],
+                             circular=circular, ws=ws)
+    return H
+
+
+def gpu_nd(u, H, *, circular, gate=None, skip=None, H_batch_stride=0):
+    B, D = u.shape[:2]
+    dims = list(u.shape[2:])
+    ws = torch.empty(max(hy.nd_conv_workspace(dims, B, D, circular), 1), dtype=torch.uint8, device="cuda")
+    y = torch.empty_like(u)
+    hy.hyena_nd_conv(u, H, y, H_batch_stride=H_batch_stride, circular=circular, Dskip=skip, gate=gate, ws=ws)
+    torch.cuda.synchronize()
+    return y
+
+
+@pytest.mark.parametrize("g,circular,per_sample,skip,gate", [
+    (4, False, False, True, True),
+    (8, False, True, True, True),
+    (8, True, False, False, True),
+    (16, True, True, True, False),
+])
+def test_nd_small_grids_direct(g, circular, per_sample, skip, gate):
+    rng = np.random.default_rng(g * 10 + circular)
+    B, D = 2, 3
+    S = g if circular else 2 * g
+    nk = B * D if per_sample else D
+    Kern = rng.standard_normal((nk, S, S, S)).astype(np.float32)
+    if not circular:   # offset -g is outside the non-circular support
+        Kern[:, S // 2] = 0
+        Kern[:, :, S // 2] = 0
+        Kern[:, :, :, S // 2] = 0
+    v = rng.standard_normal((B, D, g, g, g)).astype(np.float32)
+    x1 = rng.standard_normal((B, D, g, g, g)).astype(np.float32)
+    Dk = rng.standard_normal(D).astype(np.float32)
+    H = gpu_spectrum3(Kern, circular)
+    Href = np.fft.rfftn(Kern.astype(np.float64), axes=(1, 2, 3))
+    Hg = H.cpu().numpy().astype(np.complex128)
+    check(np.stack([Hg.real, Hg.imag]), np.stack([Href.real, Href.imag]), "f32", "3-D spectrum")
+    stride = D * S * S * (S // 2 + 1) if per_sample else 0
+    y = gpu_nd(f32_dev(v), H, circular=circular, gate=f32_dev(x1) if gate else None,
+               skip=f32_dev(Dk) if skip else None, H_batch_stride=stride)
+    got = to_np(y)
+    pts = np.arange(g ** 3)
+    for b in range(B):
+        for d in range(D):
+            kern = Kern[b * D + d] if per_sample else Kern[d]
+            ref = oracle.nd_conv_points(kern, v[b, d], x1[b, d] if gate else None,
+                                        float(Dk[d]) if skip else 0.0, pts, circular).reshape(g, g, g)
+            check(got[b, d], ref, "f32", "N-D g%d b%d d%d" % (g, b, d))
+
+
+def test_nd_delta_and_shift_kernels():
+    g, S = 8, 16
+    K = np.zeros((2, S, S, S), np.float32)
+    K[0, 0, 0, 0] = 1.0                      # identity
+    K[1, 1, 2, S - 3] = 1.0                  # shift by (+1, +2, -3)
+    H = gpu_spectrum3(K)
+    v = np.random.default_rng(1).standard_normal((1, 2, g, g, g)).astype(np.float32)
+    got = to_np(gpu_nd(f32_dev(v), H, circular=False))
+    np.testing.assert_allclose(got[0, 0], v[0, 0], atol=1e-5)
+    sh = np.zeros((g, g, g), np.float32)
+    sh[1:, 2:, :g - 3] = v[0, 1, :g - 1, :g - 2, 3:]
+    np.testing.assert_allclose(got[0, 1], sh, atol=1e-5)
+
+
+def test_nd_filter_gen_3d_vs_oracle():
+    g, F = 8, 4
+    w = hw.make("c4", seed=44, B=2, D=6, grid=(g, g, g), with_signals=False)
+    S = 2 * g
+    h = torch.empty((2, 6, S, S, S), device="cuda")
+    hy.hyena_filter_gen(h, ndim=3, grid=g, Ws=[f32_dev(a) for a in w.Ws], bs=[f32_dev(a) for a in w.bs],
+                        alpha=f32_dev(w.alpha), n_freq=F, film_gamma=f32_dev(w.film_gamma),
+                        film_beta=f32_dev(w.film_beta), n_sets=2)
+    torch.cuda.synchronize()
+    got = to_np(h)
+    idx = np.arange(S ** 3)
+    for b in range(2):
+        ref = oracle.filter_gen_3d_points(g, False, F, w.Ws, w.bs, w.film_gamma[b], w.film_beta[b], w.alpha, idx)
+        check(got[b].reshape(6, -1), ref.T, "f32", "3-D filters sample %d" % b)
+
+
+def test_c4_full_size():
+    """Workload 4 at full size: per-sample FiLM filters on the 128^3 transform
+    grid, their spectra and the gated convolution of B2 D128 64^3.  Four slabs
+    are checked on all voxels against the FFT-route reference and on 2048
+    voxels (plus the 8 corners) against the direct definition."""
+    w = hw.make("c4")
+    s = w.spec
+    B, D, g = s["B"], s["D"], s["grid"][0]
+    S = 2 * g
+    dev = "cuda"
+    h = torch.empty((B, D, S, S, S), device=dev)
+    hy.hyena_filter_gen(h, ndim=3, grid=g, Ws=[f32_dev(a) for a in w.Ws], bs=[f32_dev(a) for a in w.bs],
+                        alpha=f32_dev(w.alpha), n_freq=s["F"], film_gamma=f32_dev(w.film_gamma),
+                        film_beta=f32_dev(w.film_beta), n_sets=B)
+    H = torch.empty((B, D, S, S, S // 2 + 1), dtype=torch.complex64, device=dev)
+    ws = torch.empty(hy.filter_spectrum_workspace(B * D, 3, [g, g, g]), dtype=torch.uint8, device=dev)
+    hy.hyena_filter_spectrum(h, H, rows=B * D, ndim=3, dims=[g, g, g], ws=ws)
+    del ws
+    u = f32_dev(w.v.f32)
+    x1 = f32_dev(w.xs[0].f32)
+    y = gpu_nd(u, H, circular=False, gate=x1, H_batch_stride=D * S * S * (S // 2 + 1))
+    got = to_np(y)
+    assert np.all(np.isfinite(got))
+    slabs = [(0, 0), (0, 77), (1, 3), (1, 127)]
+    rng = np.random.default_rng(4)
+    pts = np.concatenate([rng.choice(g ** 3, 2048, replace=False),
+                          [0, g - 1, g * (g - 1), g * g - 1, g ** 3 - g * g, g ** 3 - g * (g - 1) - 1,
+                           g ** 3 - g, g ** 3 - 1]])
+    idx = np.arange(S ** 3)
+    for b, d in slabs:
+        Ws = list(w.Ws[:-1]) + [w.Ws[-1][[d]]]
+        bs = list(w.bs[:-1]) + [w.bs[-1][[d]]]
+        kern = oracle.filter_gen_3d_points(g, False, s["F"], Ws, bs, w.film_gamma[b], w.film_beta[b],
+                                           w.alpha[[d]], idx)[:, 0].reshape(S, S, S)
+        check(to_np(h[b, d]), kern, "f32", "c4 filter b%d d%d" % (b, d))
+        ref = oracle.fft_nd_conv(kern, w.v.f32[b, d], w.xs[0].f32[b, d])
+        check(got[b, d], ref, "f32", "c4 slab b%d d%d (FFT route)" % (b, d))
+        direct = oracle.nd_conv_points(kern, w.v.f32[b, d], w.xs[0].f32[b, d], 0.0, pts)
+        check_part(got[b, d].ravel()[pts], direct, float(np.sqrt(np.mean(ref ** 2))), "f32",
+                   "c4 slab b%d d%d voxels (direct)" % (b, d))

@@ -1,28 +1,34 @@
 """Benchmark of the Hyena hot path on B200.
 
-Workload: the order-2 Hyena operator at B=8, D=768, L=8192 with bf16 I/O and
-fp32 FFT math (implicit filters 65->64->64->768).  One step is one pass of the
-whole path over one batch: implicit filter generation (PE + MLP + decay),
-filter spectra (zero-padded rFFT), and the fused FFT convolution with skip
-term and gate -- three launches of this library's kernels.
+Default workload (the headline): the order-2 Hyena operator at B=8, D=768,
+L=8192 with bf16 I/O and fp32 FFT math (implicit filters 65->64->64->768).
+One step is one pass of the whole path over one batch: implicit filter
+generation (PE + MLP + decay), filter spectra (zero-padded rFFT), and the
+fused FFT convolution with skip term and gate -- all in this library's kernels.
 
-Metric: achieved GB/s of compulsory HBM traffic per step (the operator's
-inputs, output and filter spectra read once, plus the spectra written once by
-the filter path), with ms per step and the fraction of the measured HBM peak.
-Inputs stream 352 MB per step through a 126 MB L2, so no flush is needed.
+Other workloads (``--workload``): c1 (order 2, B1 D16 L1024 fp32), c3 (order 3,
+B1 D256 L=2^20 fp32, multi-pass), c4 (HyenaND 3-D, B2 D128 64^3 fp32,
+FiLM filters), c5 (spectral gate, B4 H32 Dh64 L32768 bf16).
+
+Metric: achieved GB/s of compulsory HBM traffic per step (inputs, outputs and
+filter spectra read once, plus the spectra written once by the filter path),
+with ms per step and, for the dominant kernel (the convolution), the fraction
+of the measured HBM peak.  Every workload but c1 streams more than the 126 MB
+L2 per step, so no flush is needed between steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload c1|c2|c3|c4|c5]
 
 Under torchrun (N > 1) every rank runs the same per-GPU workload on its own
 GPU (independent batches, no collective on the data path: weak scaling); the
 timed region is bracketed by barriers and the slowest rank's time counts.
-``--impl reference`` times the float64 CPU oracle on a bounded sample instead.
+``--impl reference`` times the float64 CPU oracle on a bounded sample.
 """
 from __future__ import annotations
 
 import argparse
+import datetime
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -37,24 +43,39 @@ sys.path.insert(0, ROOT)
 
 import hyena_workloads as hw  # noqa: E402
 
-WORKLOAD = "c2"
-L2_BYTES = 126 * 1024 * 1024
+DEFAULT_WORKLOAD = "c2"
+DESCR = {
+    "c1": "hyena order-2 operator B1 D16 L1024 fp32 (filters 17->32->16)",
+    "c2": "hyena order-2 operator B8 D768 L8192 bf16 (filters 65->64->64->768)",
+    "c3": "hyena order-3 operator B1 D256 L1048576 fp32 (filters 17->64->512)",
+    "c4": "hyenaND order-2 3-D conv B2 D128 64^3 fp32 (FiLM filters 24->64->128 on 128^3)",
+    "c5": "spectral gate B4 H32 Dh64 L32768 bf16",
+}
+
+
+def spectrum_bins(L):
+    m = 16
+    while m < L:
+        m *= 2
+    return m + 1
 
 
 def workload_bytes(spec):
-    """Compulsory bytes of one step and of one operator launch."""
-    B, D, L = spec["B"], spec["D"], spec["L"]
-    el = 2 if spec["dtype"] == "bf16" else 4
-    K = spec["order"] - 1
-    bins = 1
-    while bins < L:
-        bins *= 2
-    bins = max(bins, 16) + 1
-    sig = B * D * L * el
-    spectra = K * D * bins * 8
-    op = (1 + K) * sig + sig + spectra + K * D * 4          # v, x_k, y, H, Dskip
-    step = op + spectra                                       # + spectra written by the filter path
-    return step, op
+    """(compulsory bytes of one step, of the convolution launch(es))."""
+    sig = hw.signal_bytes(spec)
+    if spec["kind"] == "operator":
+        K, D = spec["order"] - 1, spec["D"]
+        spectra = K * D * spectrum_bins(spec["L"]) * 8
+        op = (1 + K) * sig + sig + spectra + K * D * 4
+        return op + spectra, op
+    if spec["kind"] == "nd":
+        S = 2 * spec["grid"][0]
+        spectra = spec["B"] * spec["D"] * S * S * (S // 2 + 1) * 8
+        op = 2 * sig + sig + spectra
+        return op + spectra, op
+    gate = spec["H"] * (spec["L"] // 2 + 1) * 8
+    op = 3 * sig + gate
+    return op, op
 
 
 def measured_peaks():
@@ -103,7 +124,6 @@ class ClockSampler:
                     continue
                 if t_begin is not None:
                     try:
-                        import datetime
                         ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
                     except ValueError:
                         ts = None
@@ -126,14 +146,11 @@ def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
     if world > 1:
-        import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(local)
     return world, rank, local
 
 
@@ -153,6 +170,121 @@ def max_over_ranks(x, world):
     return float(t.item())
 
 
+# ------------------------------------------------------------------ setups
+
+class Setup:
+    """Device state of one workload: spectra() runs the filter rows of the
+    path, op() the convolution; inputs (device, host signal) feed the
+    end-to-end run."""
+
+    def __init__(self):
+        self.inputs = []
+        self.output = None
+        self.launches = 0
+        self.kernel = ""
+
+
+def setup_operator(w, dev, hy, torch):
+    s = w.spec
+    B, D, L, K = s["B"], s["D"], s["L"], s["order"] - 1
+    f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dev)
+    if s["dtype"] == "bf16":
+        sig = lambda x: torch.from_numpy(x.bf16.view(np.int16)).view(torch.bfloat16).to(dev)
+        code = hy.HY_BF16
+    else:
+        sig = lambda x: torch.from_numpy(np.ascontiguousarray(x.f32)).to(dev)
+        code = hy.HY_F32
+    Ws, bs, alpha = [f32(a) for a in w.Ws], [f32(a) for a in w.bs], f32(w.alpha)
+    Dsk = [f32(w.Dskip[k]) for k in range(K)]
+    v, xs = sig(w.v), [sig(x) for x in w.xs]
+    y = torch.empty_like(v)
+    nb = hy.spectrum_bins(L)
+    h = torch.empty((K * D, L), device=dev)
+    H = torch.empty((K * D, nb), dtype=torch.complex64, device=dev)
+    Hs = [H[k * D:(k + 1) * D] for k in range(K)]
+    wsf = hy.filter_spectrum_workspace(K * D, 1, [L])
+    wso = hy.operator_workspace(K + 1, B, D, L, code)
+    ws = torch.empty(max(wsf, wso, 1), dtype=torch.uint8, device=dev)
+    st = Setup()
+
+    def spectra():
+        hy.hyena_filter_gen(h, ndim=1, L=L, Ws=Ws, bs=bs, alpha=alpha, n_freq=s["F"], include_t=True)
+        hy.hyena_filter_spectrum(h, H, rows=K * D, ndim=1, dims=[L], ws=ws if wsf else None)
+
+    def op():
+        hy.hyena_operator(v, xs, Hs, y, Dskips=Dsk, ws=ws if wso else None)
+
+    st.spectra, st.op = spectra, op
+    st.inputs = [(v, w.v)] + list(zip(xs, w.xs))
+    st.output = y
+    M = nb - 1
+    if wso:
+        rows_chunk = max(1, wso // (12 * M))
+        op_l = -(-(B * D) // rows_chunk) * (1 + 2 * K)
+        st.kernel = "multi-pass colpass/rowpass kernels (M=2^%d)" % (M.bit_length() - 1)
+    else:
+        op_l = 1
+        st.kernel = "resident_conv_kernel<M=2^%d>" % (M.bit_length() - 1)
+    spec_l = 2 * -(-(K * D) // max(1, wsf // (12 * M))) if wsf else 1
+    st.launches = 1 + spec_l + op_l
+    return st
+
+
+def setup_nd(w, dev, hy, torch):
+    s = w.spec
+    B, D, g = s["B"], s["D"], s["grid"][0]
+    S = 2 * g
+    f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dev)
+    Ws, bs, alpha = [f32(a) for a in w.Ws], [f32(a) for a in w.bs], f32(w.alpha)
+    gm, bt = f32(w.film_gamma), f32(w.film_beta)
+    u, x1 = f32(w.v.f32), f32(w.xs[0].f32)
+    y = torch.empty_like(u)
+    h = torch.empty((B, D, S, S, S), device=dev)
+    H = torch.empty((B, D, S, S, S // 2 + 1), dtype=torch.complex64, device=dev)
+    wsf = hy.filter_spectrum_workspace(B * D, 3, [g, g, g])
+    wsc = hy.nd_conv_workspace([g, g, g], B, D)
+    ws = torch.empty(max(wsf, wsc, 1), dtype=torch.uint8, device=dev)
+    st = Setup()
+
+    def spectra():
+        hy.hyena_filter_gen(h, ndim=3, grid=g, Ws=Ws, bs=bs, alpha=alpha, n_freq=s["F"],
+                            film_gamma=gm, film_beta=bt, n_sets=B)
+        hy.hyena_filter_spectrum(h, H, rows=B * D, ndim=3, dims=[g, g, g], ws=ws)
+
+    def op():
+        hy.hyena_nd_conv(u, H, y, H_batch_stride=D * S * S * (S // 2 + 1), gate=x1, ws=ws)
+
+    st.spectra, st.op = spectra, op
+    st.inputs = [(u, w.v), (x1, w.xs[0])]
+    st.output = y
+    per_c = g * S * (S // 2 + 1) * 8
+    per_s = S * S * (S // 2 + 1) * 8
+    st.launches = (1 + 2 * -(-(B * D) // max(1, wsf // per_s))
+                   + 3 * -(-(B * D) // max(1, wsc // per_c)))
+    st.kernel = "nd_fwd_plane/nd_xpass/nd_inv_plane<S=%d>" % S
+    return st
+
+
+def setup_gate(w, dev, hy, torch):
+    s = w.spec
+    sig = lambda x: torch.from_numpy(x.bf16.view(np.int16)).view(torch.bfloat16).to(dev)
+    x, x2 = sig(w.v), sig(w.xs[0])
+    g = torch.from_numpy(w.gate).to(dev)
+    y = torch.empty_like(x)
+    st = Setup()
+    st.spectra = lambda: None
+
+    def op():
+        hy.spectral_gate(x, g, y, x2=x2)
+
+    st.op = op
+    st.inputs = [(x, w.v), (x2, w.xs[0])]
+    st.output = y
+    st.launches = 1
+    st.kernel = "resident_conv_kernel<M=2^%d, circular>" % ((s["L"] // 2).bit_length() - 1)
+    return st
+
+
 # ------------------------------------------------------------------ our arm
 
 def run_ours(args):
@@ -160,38 +292,37 @@ def run_ours(args):
     import implicit_long_convolution_b200 as hy
 
     world, rank, local = dist_setup()
-    w = hw.make(WORKLOAD, seed=hw.SEEDS[WORKLOAD] + 1000 * rank)
+    name = args.workload
+    w = hw.make(name, seed=hw.SEEDS[name] + 1000 * rank)
     s = w.spec
-    B, D, L, K = s["B"], s["D"], s["L"], s["order"] - 1
     dev = torch.device("cuda", local)
-    f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dev)
-    bf = lambda sig: torch.from_numpy(sig.bf16.view(np.int16)).view(torch.bfloat16).to(dev)
-    Ws, bs, alpha = [f32(a) for a in w.Ws], [f32(a) for a in w.bs], f32(w.alpha)
-    Dsk = [f32(w.Dskip[k]) for k in range(K)]
-    v, xs = bf(w.v), [bf(x) for x in w.xs]
-    y = torch.empty_like(v)
-    nb = hy.spectrum_bins(L)
-    h = torch.empty((K * D, L), device=dev)
-    H = torch.empty((K * D, nb), dtype=torch.complex64, device=dev)
-    Hs = [H[k * D:(k + 1) * D] for k in range(K)]
+    setup = {"operator": setup_operator, "nd": setup_nd, "gate": setup_gate}[s["kind"]]
+    st = setup(w, dev, hy, torch)
     stream = torch.cuda.current_stream(dev)
     op_ev = []
 
     def step(record=False):
-        hy.hyena_filter_gen(h, ndim=1, L=L, Ws=Ws, bs=bs, alpha=alpha, n_freq=s["F"], include_t=True)
-        hy.hyena_filter_spectrum(h, H, rows=K * D, ndim=1, dims=[L])
+        st.spectra()
         if record:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-        hy.hyena_operator(v, xs, Hs, y, Dskips=Dsk)
+        st.op()
         if record:
             e1.record(stream)
             op_ev.append((e0, e1))
 
-    launches_per_step = 3
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    steps = args.steps
+    if steps <= 0:   # size the timed region to about one second
+        ta, tb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ta.record(stream)
+        step()
+        tb.record(stream)
+        torch.cuda.synchronize()
+        steps = int(max(10, min(5000, 1000.0 / max(ta.elapsed_time(tb), 1e-3))))
+        steps = int(max_over_ranks(steps, world))
     clocks = ClockSampler(local)
     barrier(world)
     torch.cuda.synchronize()
@@ -201,37 +332,40 @@ def run_ours(args):
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
-    for _ in range(args.steps):
+    for _ in range(steps):
         step(record=True)
     t1.record(stream)
     torch.cuda.synchronize()
     wall1 = time.time()
     barrier(world)
     ck = clocks.stop(wall0, wall1)
-    ms = t0.elapsed_time(t1)
+    ms = max_over_ranks(t0.elapsed_time(t1), world)
     op_ms = [a.elapsed_time(b) for a, b in op_ev]
-    ms = max_over_ranks(ms, world)
     op_avg = max_over_ranks(sum(op_ms) / len(op_ms), world)
 
     step_bytes, op_bytes = workload_bytes(s)
     sec = ms / 1e3
-    value = world * args.steps * step_bytes / sec / 1e9
+    value = world * steps * step_bytes / sec / 1e9
     peak, peak_kind = measured_peaks()
     achieved = op_bytes / (op_avg / 1e3) / 1e9
 
     # end to end through the public API with host buffers: H2D of the step's
-    # inputs from pinned memory, the path, D2H of the result
-    hv = torch.from_numpy(w.v.bf16.view(np.int16)).view(torch.bfloat16).pin_memory()
-    hx = [torch.from_numpy(x.bf16.view(np.int16)).view(torch.bfloat16).pin_memory() for x in w.xs]
-    hy_out = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-    e2e_steps = max(2, min(args.steps, 10))
+    # input signals from pinned memory, the whole step, D2H of the result
+    hosts = []
+    for dvc, sg in st.inputs:
+        if dvc.dtype == torch.bfloat16:
+            t = torch.from_numpy(np.ascontiguousarray(sg.bf16.view(np.int16))).view(torch.bfloat16)
+        else:
+            t = torch.from_numpy(np.ascontiguousarray(sg.f32))
+        hosts.append(t.pin_memory())
+    out_h = torch.empty(st.output.shape, dtype=st.output.dtype).pin_memory()
+    e2e_steps = max(2, min(steps, 10))
 
     def e2e_step():
-        v.copy_(hv, non_blocking=True)
-        for xd, xh in zip(xs, hx):
-            xd.copy_(xh, non_blocking=True)
+        for (dvc, _), hst in zip(st.inputs, hosts):
+            dvc.copy_(hst, non_blocking=True)
         step()
-        hy_out.copy_(y, non_blocking=True)
+        out_h.copy_(st.output, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize()
@@ -244,40 +378,44 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(a0.elapsed_time(a1) / e2e_steps, world)
-    h2d = hv.numel() * 2 + sum(x.numel() * 2 for x in hx)
-    d2h = hy_out.numel() * 2
+    h2d = sum(hh.numel() * hh.element_size() for hh in hosts)
+    d2h = out_h.numel() * out_h.element_size()
 
+    cfg = {"workload": DESCR[name]}
+    cfg.update({k: v for k, v in s.items() if k in ("B", "D", "L", "order", "H", "Dh", "grid")})
+    cfg.update({"step": ("filter_gen + filter_spectrum + convolution" if s["kind"] != "gate"
+                         else "spectral_gate"),
+                "step_bytes": step_bytes, "conv_bytes": op_bytes,
+                "l2": ("inputs larger than L2 (%.0f MB streamed per step vs 126 MB); no flush" % (op_bytes / 1e6)
+                       if op_bytes > 126e6 else "inputs smaller than L2 (no flush): launch-bound case"),
+                "parallelism": "independent replicas x%d (no data-path collective)" % world})
+    el = 2 if s["dtype"] == "bf16" else 4
     line = {
-        "metric": "Hyena op GB/s (order-2, B8 D768 L8192, bf16 I/O, fp32 FFT math)",
+        "metric": "Hyena op GB/s (%s)" % DESCR[name],
         "value": round(value, 2),
         "unit": "GB/s",
         "n_gpus": world,
-        "steps": args.steps,
+        "steps": steps,
         "warmup": args.warmup,
-        "ms_per_step": round(ms / args.steps, 4),
+        "ms_per_step": round(ms / steps, 4),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f32 math, bf16 I/O",
+        "dtype": "f32 math, %s I/O" % s["dtype"],
         "data": "synthetic (seeded N(0,1) signals, random-init filter MLP)",
-        "config": {"workload": "hyena order-2 operator B8 D768 L8192 bf16 (filters 65->64->64->768)",
-                   "B": B, "D": D, "L": L, "order": K + 1,
-                   "step": "filter_gen + filter_spectrum + hyena_operator",
-                   "step_bytes": step_bytes, "operator_bytes": op_bytes,
-                   "l2": "inputs larger than L2 (%.0f MB streamed per step vs 126 MB)" % (op_bytes / 1e6),
-                   "parallelism": "replicas x%d" % world},
-        "tokens_channels_per_s": round(world * args.steps * B * D * L / sec, 1),
-        "operator_ms": round(op_avg, 4),
-        "roofline": {"bound": "hbm", "kernel": "resident_conv_kernel<13,bf16>",
+        "config": cfg,
+        "tokens_channels_per_s": round(world * steps * (hw.signal_bytes(s) // el) / sec, 1),
+        "conv_ms": round(op_avg, 4),
+        "roofline": {"bound": "hbm", "kernel": st.kernel,
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
-                     "traffic": None},
+                     "frac": round(achieved / peak, 4), "peak_kind": peak_kind, "traffic": None},
         "e2e": {"value": round(world * step_bytes / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": st.launches * steps,
         "clocks": ck,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if (rank == 0 and world == 1 and not args.no_cpu_baseline and s["kind"] == "operator"
+            and s["L"] <= 16384):
         line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
     if world > 1:
         import torch.distributed as dist
@@ -292,7 +430,8 @@ def run_ours(args):
 def cpu_baseline(w, budget_s=12.0):
     """The float64 oracle as it stands on a bounded sample of the workload:
     the filter MLP for all L positions plus the direct O(L^2) gated chain on
-    as many rows as fit the time budget.  Value in the metric's unit."""
+    as many rows as fit the time budget; the value scales the sample to one
+    whole step (rows are independent, so row time scales linearly)."""
     import oracle
     s = w.spec
     B, D, L, K = s["B"], s["D"], s["L"], s["order"] - 1
@@ -302,23 +441,22 @@ def cpu_baseline(w, budget_s=12.0):
     h64 = oracle.filter_gen_1d(L, s["F"], True, w.Ws, w.bs, w.alpha)
     t_filter = time.perf_counter() - t0
     cores = oracle.threads()
-    probe = max(cores, 8)
+    probe = min(rows_total, max(cores, 8))
     t0 = time.perf_counter()
     oracle.hyena_rows(w.v.f32, [x.f32 for x in w.xs], h64.reshape(K, D, L), w.Dskip,
                       rows=np.arange(probe))
     t_probe = time.perf_counter() - t0
     n = int(max(probe, min(rows_total, probe * max(1.0, (budget_s - t_filter) / max(t_probe, 1e-3)))))
-    n = max(cores, (n // cores) * cores)
+    n = min(rows_total, max(probe, (n // cores) * cores))
     rows = np.random.default_rng(0).choice(rows_total, n, replace=False)
     t0 = time.perf_counter()
     oracle.hyena_rows(w.v.f32, [x.f32 for x in w.xs], h64.reshape(K, D, L), w.Dskip, rows=rows)
     t_rows = time.perf_counter() - t0
-    # scale: the whole step = filter path once + all rows
-    est_step = t_filter + t_rows * rows_total / n
+    est_step = t_filter + t_rows * rows_total / rows.size
     return {"value": round(step_bytes / est_step / 1e9, 6), "unit": "GB/s", "cores": cores,
             "kind": "oracle",
             "sample": "filter MLP on all %d positions + direct O(L^2) float64 chain on %d of %d rows "
-                      "(%.1f s); value scales the sample to one whole step" % (L, n, rows_total,
+                      "(%.1f s); value scales the sample to one whole step" % (L, rows.size, rows_total,
                                                                                t_filter + t_rows)}
 
 
@@ -327,7 +465,12 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    w = hw.make(WORKLOAD)
+    name = args.workload
+    w = hw.make(name)
+    if w.spec["kind"] != "operator" or w.spec["L"] > 16384:
+        print(json.dumps({"impl": "reference", "unavailable":
+                          "the oracle arm is timed on the on-chip operator workloads (c1, c2) only"}))
+        return
     budget = max(2.0, min(args.cpu_budget, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         cpu_baseline(w, budget_s=budget)
@@ -340,15 +483,15 @@ def run_reference(args):
     wall = time.perf_counter() - t0
     step_bytes, _ = workload_bytes(w.spec)
     value = statistics.median(vals)
+    s = w.spec
     line = {
         "impl": "reference",
-        "metric": "Hyena op GB/s (order-2, B8 D768 L8192, bf16 I/O, fp32 FFT math)",
+        "metric": "Hyena op GB/s (%s)" % DESCR[name],
         "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(step_bytes / (value * 1e9) * 1e3, 3) if value > 0 else None,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) signals, random-init filter MLP)",
-        "config": {"workload": "hyena order-2 operator B8 D768 L8192 bf16 (filters 65->64->64->768)",
-                   "B": 8, "D": 768, "L": 8192, "order": 2},
+        "config": {"workload": DESCR[name], "B": s["B"], "D": s["D"], "L": s["L"], "order": s["order"]},
         "cpu_baseline": last,
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "wall_s": round(wall, 1),
@@ -359,18 +502,21 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=0, help="timed steps (0: size the region to ~1 s)")
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(DESCR), default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
-    if args.warmup < 3 and args.impl == "ours":
-        args.warmup = 3
     if args.impl == "reference":
+        if args.steps <= 0:
+            args.steps = 3
         run_reference(args)
-    else:
-        run_ours(args)
+        return
+    if args.warmup < 3:
+        args.warmup = 3
+    run_ours(args)
 
 
 if __name__ == "__main__":

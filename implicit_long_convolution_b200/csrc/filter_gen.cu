@@ -5,12 +5,15 @@
 // exponential decay window; [ND] 방법론: HyenaND: coordinate MLP on the N-D
 // grid with FiLM conditioning per sample.
 //
-// One CTA evaluates TP = 64 positions of one filter set: it builds the
-// positional encoding in shared memory, runs every MLP layer as a small fp32
-// GEMM (register tile of 4 positions x 4 outputs per thread, weights staged
-// in shared memory 64 outputs at a time), applies FiLM and SiLU on hidden
+// One CTA evaluates TP = 32 positions of one filter set for one chunk of at
+// most OUT_CHUNK outputs of the last layer (grid z): it builds the positional
+// encoding in shared memory, runs every MLP layer as a small fp32 GEMM
+// (register tile of 4 positions x 4 outputs per thread, weights staged in
+// shared memory 128 outputs at a time), applies FiLM and SiLU on hidden
 // layers and the decay window on the last one, and writes the filter rows
-// with the position index fastest (coalesced).
+// with the position index fastest (coalesced).  The hidden layers are
+// recomputed per output chunk; they are a small part of the work when the
+// last layer is wide, and the chunks give the grid enough CTAs.
 #include "kernels.h"
 #include "status.h"
 
@@ -18,9 +21,10 @@ namespace hy {
 
 namespace {
 
-constexpr int TP = 64;          // positions per CTA
+constexpr int TP = 32;          // positions per CTA
 constexpr int NT = 256;         // threads
-constexpr int OC = 64;          // outputs per weight chunk
+constexpr int OC = 128;         // outputs per weight chunk
+constexpr int OUT_CHUNK = 256;  // last-layer outputs per CTA (grid z)
 constexpr int MAXW = 132;       // max layer width (input encoding or hidden), multiple of 4
 constexpr int MAXL = 4;
 
@@ -123,18 +127,20 @@ __global__ void __launch_bounds__(NT) filter_gen_kernel(const GenParams p) {
     __syncthreads();
 
     // ---- MLP layers (a2)
-    const int tx = tid % 16, ty = tid / 16;    // positions tx*4.., outputs ty*4..
+    const int tx = tid % (TP / 4), ty = tid / (TP / 4);   // positions tx*4.., outputs ty*4..
     float *cur = actA, *nxt = actB;
     for (int l = 0; l < p.nl; ++l) {
         const int win = p.widths[l], wout = p.widths[l + 1];
         const bool last = (l == p.nl - 1);
         const float *W = p.W[l];
         const float *bias = p.b[l];
-        for (int o0 = 0; o0 < wout; o0 += OC) {
+        const int obeg = last ? blockIdx.z * OUT_CHUNK : 0;
+        const int oend = last ? min(wout, obeg + OUT_CHUNK) : wout;
+        for (int o0 = obeg; o0 < oend; o0 += OC) {
             // stage W[o0 .. o0+OC)[0..win) transposed
             for (int idx = tid; idx < OC * win; idx += NT) {
                 const int oo = idx / win, i = idx % win;
-                wt[i * OC + oo] = (o0 + oo < wout) ? __ldg(W + (int64_t)(o0 + oo) * win + i) : 0.f;
+                wt[i * OC + oo] = (o0 + oo < oend) ? __ldg(W + (int64_t)(o0 + oo) * win + i) : 0.f;
             }
             __syncthreads();
             float acc[4][4];
@@ -155,7 +161,7 @@ __global__ void __launch_bounds__(NT) filter_gen_kernel(const GenParams p) {
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const int o = o0 + ty * 4 + c;
-                if (o >= wout) continue;
+                if (o >= oend) continue;
                 const float bo = __ldg(bias + o);
                 if (!last) {
                     float gm = 0.f, bt = 0.f;
@@ -226,7 +232,8 @@ hy_status launch_filter_gen(const hy_filter_desc &d, float *h, cudaStream_t s) {
     const size_t smem = sizeof(float) * (size_t)(2 * MAXW * TP + MAXW * OC);
     cudaError_t e = cudaFuncSetAttribute(filter_gen_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return set_cuda_error("filter_gen smem attribute", e);
-    dim3 grid((unsigned)nblk, (unsigned)d.n_sets);
+    const int nout = d.widths[d.n_layers];
+    dim3 grid((unsigned)nblk, (unsigned)d.n_sets, (unsigned)((nout + OUT_CHUNK - 1) / OUT_CHUNK));
     filter_gen_kernel<<<grid, NT, smem, s>>>(p);
     return check_launch("filter_gen launch");
 }

@@ -24,11 +24,38 @@ hy_status launch_spectrum_t(int64_t rows, int L, const float *h, float2 *H, cuda
 
 }  // namespace
 
+int device_sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+static bool aligned16(const void *q) { return ((uintptr_t)q & 15u) == 0; }
+
 hy_status launch_resident_conv(const ResidentParams &p, int log_m, hy_dtype dt, bool circular,
                                cudaStream_t s) {
     if (p.n_rows <= 0) return HY_OK;
     if (p.n_rows > 0x7fffffffLL) return set_error(HY_ERR_UNSUPPORTED, "too many rows (%lld)", (long long)p.n_rows);
     const bool chain = p.K > 1;
+    // one order over whole power-of-two rows, 16-byte aligned: the persistent
+    // streaming kernel (cp.async prefetch of inputs and gate)
+    const int64_t full = circular ? (int64_t)2 << log_m : (int64_t)1 << log_m;
+    const int esz = dt == HY_BF16 ? 2 : 4;
+    const bool fits = stream_smem_bytes(log_m, esz, circular, false) <= (size_t)227 * 1024;
+    if (!chain && fits && log_m >= 6 && p.L == full && aligned16(p.u) && aligned16(p.y) &&
+        (!p.gate[0] || aligned16(p.gate[0]))) {
+        if (dt == HY_F32)
+            return circular ? dispatch_stream<float, true>(log_m, p, s) : dispatch_stream<float, false>(log_m, p, s);
+        return circular ? dispatch_stream<__nv_bfloat16, true>(log_m, p, s)
+                        : dispatch_stream<__nv_bfloat16, false>(log_m, p, s);
+    }
     if (dt == HY_F32) {
         if (circular) return dispatch_conv<float, true, false>(log_m, p, s);
         return chain ? dispatch_conv<float, false, true>(log_m, p, s) : dispatch_conv<float, false, false>(log_m, p, s);

@@ -236,6 +236,154 @@ resident_conv_kernel(const ResidentParams p) {
     }
 }
 
+// ----------------------------------------------------------------------------
+// Streaming variant for one order (K = 1) with L = 2^LOG_M (causal) or
+// L = 2^(LOG_M+1) (circular) samples per row: a persistent CTA walks its rows
+// and overlaps HBM with the FFTs.  While row r is being transformed, cp.async
+// brings row r+1's input and row r's gate into shared memory (stage buffers
+// next to the FFT exchange buffer); the skip term reuses the input samples
+// kept packed in registers.  Without PF_GATE (when two stage buffers would not
+// fit) the gate is read from global memory in the epilogue.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+    const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <typename IO> struct Packed;              // one sample pair kept for the skip term
+template <> struct Packed<__nv_bfloat16> {
+    uint32_t v;
+    __device__ __forceinline__ void set(float2 f) {
+        v = (__float_as_uint(f.x) >> 16) | (__float_as_uint(f.y) & 0xffff0000u);
+    }
+    __device__ __forceinline__ float2 get() const {
+        return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+    }
+};
+template <> struct Packed<float> {
+    float2 v;
+    __device__ __forceinline__ void set(float2 f) { v = f; }
+    __device__ __forceinline__ float2 get() const { return v; }
+};
+
+// float2 slots before the stage buffers (even, so they start 16-byte aligned)
+__host__ __device__ constexpr int stream_stage_offset(int m) { return ((spad_size(m) + 1) / 2) * 2; }
+// dynamic shared memory of the streaming kernel
+__host__ __device__ constexpr size_t stream_smem_bytes(int log_m, int io_bytes, bool circ, bool pf_gate) {
+    return (size_t)stream_stage_offset(1 << log_m) * 8 +
+           (size_t)(circ ? 2 : 1) * (1 << log_m) * io_bytes * (pf_gate ? 2 : 1);
+}
+// prefetch the gate too when both stage buffers fit beside the CTAs per SM the
+// registers allow (about 113 KB each for two CTAs, 227 KB for one)
+__host__ __device__ constexpr bool stream_pf_gate(int log_m, int io_bytes, bool circ) {
+    return stream_smem_bytes(log_m, io_bytes, circ, true) <=
+           (resident_min_blocks(log_m) >= 2 ? (size_t)113 * 1024 : (size_t)227 * 1024);
+}
+
+template <int LOG_M, typename IO, bool CIRC, bool PF_GATE>
+__global__ void __launch_bounds__((1 << LOG_M) >> resident_log_p(LOG_M), resident_min_blocks(LOG_M))
+resident_stream_kernel(const ResidentParams p) {
+    constexpr int LOG_P = resident_log_p(LOG_M);
+    constexpr int M = 1 << LOG_M;
+    constexpr int P = 1 << LOG_P;
+    constexpr int T = M / P;
+    constexpr int PIN = CIRC ? P : P / 2;
+    constexpr int L = CIRC ? 2 * M : M;                  // samples per row
+    constexpr int CHUNKS = L * (int)sizeof(IO) / 16;     // 16-byte copies per row
+    using IOT = IOTraits<IO>;
+
+    extern __shared__ float2 smem[];
+    float2 *sbuf = smem;
+    IO *in_st = reinterpret_cast<IO *>(smem + stream_stage_offset(M));   // 16-byte aligned
+    IO *g_st = in_st + L;
+
+    const int t = threadIdx.x;
+    const IO *ubase = reinterpret_cast<const IO *>(p.u);
+    const IO *gbase = reinterpret_cast<const IO *>(p.gate[0]);
+    IO *ybase = reinterpret_cast<IO *>(p.y);
+    auto row_of = [&](int64_t c) { return p.remap ? (c % p.B) * (int64_t)p.D + c / p.B : c; };
+    auto copy_row = [&](IO *dst, const IO *src) {
+        for (int i = t; i < CHUNKS; i += T)
+            cp_async16(reinterpret_cast<char *>(dst) + 16 * i, reinterpret_cast<const char *>(src) + 16 * i);
+    };
+
+    int64_t c = blockIdx.x;
+    if (c < p.n_rows) copy_row(in_st, ubase + row_of(c) * L);
+    cp_async_commit();
+    const float dk_null = 0.f;
+    for (; c < p.n_rows; c += gridDim.x) {
+        const int64_t row = row_of(c);
+        const int64_t ch = (row / p.sdiv) % p.smod;
+        const int64_t smp = row / (p.sdiv * p.smod);
+        cp_async_wait<0>();
+        __syncthreads();
+        float2 x[P];
+        constexpr int NKEEP = CIRC ? 1 : PIN;             // the spectral gate has no skip term
+        Packed<IO> keep[NKEEP];
+#pragma unroll
+        for (int m = 0; m < P; ++m) {
+            x[m] = make_float2(0.f, 0.f);
+            if (m < PIN) {
+                const int i0 = 2 * (t + m * T);
+                if constexpr (sizeof(IO) == 2) {
+                    const uint32_t b = *reinterpret_cast<const uint32_t *>(in_st + i0);
+                    x[m] = make_float2(__uint_as_float(b << 16), __uint_as_float(b & 0xffff0000u));
+                } else {
+                    x[m] = *reinterpret_cast<const float2 *>(in_st + i0);
+                }
+                if constexpr (!CIRC) keep[m].set(x[m]);
+            }
+        }
+        __syncthreads();                                  // stage buffer free for the next row
+        if (PF_GATE && gbase) copy_row(g_st, gbase + row * L);
+        cp_async_commit();
+        if (c + gridDim.x < p.n_rows) copy_row(in_st, ubase + row_of(c + gridDim.x) * L);
+        cp_async_commit();
+
+        block_fft<LOG_M, LOG_P, -1, !CIRC>(x, sbuf, t, p.tw_fft);
+        const float2 *H = p.spec[0] + smp * p.spec_batch_stride + ch * p.spec_row_stride;
+        split_multiply_merge<LOG_M, LOG_P>(x, sbuf, t, H, p.tw_split);
+        block_fft<LOG_M, LOG_P, +1, false>(x, sbuf, t, p.tw_fft);
+
+        const float dk = p.skip[0] ? ldv(p.skip[0] + ch) : dk_null;
+        if constexpr (PF_GATE) {
+            cp_async_wait<1>();                           // the gate of this row has landed
+            __syncthreads();
+        }
+        IO *yout = ybase + row * (int64_t)L;
+#pragma unroll
+        for (int m = 0; m < PIN; ++m) {
+            const int i0 = 2 * (t + m * T);
+            float2 z;
+            if constexpr (CIRC) {
+                z = make_float2(x[m].x * p.scale, x[m].y * p.scale);
+            } else {
+                const float2 pv = keep[m].get();
+                z = make_float2(fmaf(x[m].x, p.scale, dk * pv.x), fmaf(x[m].y, p.scale, dk * pv.y));
+            }
+            if (gbase) {
+                float2 gv;
+                if constexpr (PF_GATE) {
+                    if constexpr (sizeof(IO) == 2) {
+                        const uint32_t b = *reinterpret_cast<const uint32_t *>(g_st + i0);
+                        gv = make_float2(__uint_as_float(b << 16), __uint_as_float(b & 0xffff0000u));
+                    } else {
+                        gv = *reinterpret_cast<const float2 *>(g_st + i0);
+                    }
+                } else {
+                    gv = IOT::load2(gbase + row * (int64_t)L + i0);
+                }
+                z = make_float2(z.x * gv.x, z.y * gv.y);
+            }
+            IOT::store2(yout + i0, z);
+        }
+    }
+    cp_async_wait<0>();
+}
+
 // Filter spectrum rows: H[r, k] = Σ_t h[r, t] W_n^{kt}, k = 0..M, for rows of
 // L fp32 samples (zero-padded to n = 2M, or exactly n = L when circular).
 template <int LOG_M, bool CIRC>

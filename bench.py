@@ -161,13 +161,25 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The slowest rank's value (used for every timed quantity)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cpu" if dist.get_backend() == "gloo" else "cuda"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(name, rank):
+    """Each rank draws its own batch of the same per-GPU workload."""
+    return hw.SEEDS[name] + 1000 * rank
+
+
+def job_value(world, steps, step_bytes, max_ms):
+    """Whole-job GB/s: the bytes of every rank's steps over the slowest rank's time."""
+    return world * steps * step_bytes / (max_ms / 1e3) / 1e9
 
 
 # ------------------------------------------------------------------ setups
@@ -293,7 +305,7 @@ def run_ours(args):
 
     world, rank, local = dist_setup()
     name = args.workload
-    w = hw.make(name, seed=hw.SEEDS[name] + 1000 * rank)
+    w = hw.make(name, seed=rank_seed(name, rank))
     s = w.spec
     dev = torch.device("cuda", local)
     setup = {"operator": setup_operator, "nd": setup_nd, "gate": setup_gate}[s["kind"]]
@@ -345,7 +357,7 @@ def run_ours(args):
 
     step_bytes, op_bytes = workload_bytes(s)
     sec = ms / 1e3
-    value = world * steps * step_bytes / sec / 1e9
+    value = job_value(world, steps, step_bytes, ms)
     peak, peak_kind = measured_peaks()
     achieved = op_bytes / (op_avg / 1e3) / 1e9
 

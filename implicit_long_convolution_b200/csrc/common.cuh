@@ -33,6 +33,12 @@ __device__ __forceinline__ float2 cmul_dir(float2 a, float2 w) {
     else return cmulc(a, w);
 }
 
+// f(integral_constant<int, I>) for I in the sequence, in order
+template <typename F, int... I>
+__device__ __forceinline__ void fold_seq(F &&f, std::integer_sequence<int, I...>) {
+    (f(std::integral_constant<int, I>{}), ...);
+}
+
 // ----------------------------------------------------------------------------
 // compile-time trig (Taylor series on |x| <= pi, evaluated in double)
 // ----------------------------------------------------------------------------

@@ -76,29 +76,35 @@ __host__ __device__ constexpr int bitrev(int j, int bits) {
 }
 
 // ----------------------------------------------------------------------------
-// Radix plan: stage 0 has radix P (its inputs need no twiddle); the remaining
-// log2(M/P) bits are split over as few stages as radix <= P allows, as evenly
-// as possible (larger radices first).  Shared by the device code and the
-// host-side twiddle-table builder.
+// Radix plan: radix P while it fits, then the remainder (e.g. 8192 points with
+// 32 per thread: 32 x 32 x 8).  Stage 0 needs no twiddles.  (A balanced plan,
+// 32 x 16 x 16, has two butterflies per thread in the twiddled stages and
+// needs more registers for the same instruction count.)  Shared by the device
+// code and the host-side twiddle-table builder.
 // ----------------------------------------------------------------------------
 __host__ __device__ constexpr int plan_stages(int log_m, int log_p) {
-    return 1 + (log_m - log_p + log_p - 1) / log_p;
+    return (log_m + log_p - 1) / log_p;
 }
 __host__ __device__ constexpr int plan_log_radix(int log_m, int log_p, int s) {
-    if (s == 0) return log_p;
-    const int rest = log_m - log_p;
-    const int n = plan_stages(log_m, log_p) - 1;
-    const int base = rest / n, extra = rest % n;
-    return base + ((s - 1) < extra ? 1 : 0);
+    return (s < plan_stages(log_m, log_p) - 1) ? log_p : (log_m - log_p * (plan_stages(log_m, log_p) - 1));
 }
 __host__ __device__ constexpr int plan_log_p(int log_m, int log_p, int s) {
     int acc = 0;
     for (int i = 0; i < s; ++i) acc += plan_log_radix(log_m, log_p, i);
     return acc;
 }
-// twiddle entries of stage s: (R - 1) * p (none for stage 0)
+// Columns of stage s's twiddle table.  Butterfly i = t + q*T of a stage with
+// p = 2^plan_log_p needs W_{pR}^{(i mod p) r}.  When p <= T that is the same
+// for every q (column i mod p).  When p > T (only the last stage, where
+// i < p) W^{(t + qT) r} = W^{t r} * W^{qT r}: the table keeps the T columns
+// W^{t r} and the second factor is a compile-time constant.
+__host__ __device__ constexpr int plan_tw_cols(int log_m, int log_p, int s) {
+    return (1 << plan_log_p(log_m, log_p, s)) < (1 << (log_m - log_p)) ? (1 << plan_log_p(log_m, log_p, s))
+                                                                         : (1 << (log_m - log_p));
+}
+// twiddle entries of stage s: (R - 1) * columns (none for stage 0)
 __host__ __device__ constexpr int plan_tw_count(int log_m, int log_p, int s) {
-    return s == 0 ? 0 : ((1 << plan_log_radix(log_m, log_p, s)) - 1) * (1 << plan_log_p(log_m, log_p, s));
+    return s == 0 ? 0 : ((1 << plan_log_radix(log_m, log_p, s)) - 1) * plan_tw_cols(log_m, log_p, s);
 }
 __host__ __device__ constexpr int plan_tw_offset(int log_m, int log_p, int s) {
     int acc = 0;
@@ -169,6 +175,27 @@ struct SyncWarp {
     __device__ __forceinline__ void operator()() const { __syncwarp(); }
 };
 
+// Butterfly Q of a wide last stage: y[r] = x[Q + r*NB] times the twiddle
+// wb[r] * W_N^{QT r} (forward; conjugated for DIR = +1), then the radix-R DFT.
+// QT = Q*T is a template constant, so W_N^{QT r} is a compile-time rotation
+// (free for Q = 0).
+template <int DIR, int N, int QT, int... J>
+__device__ __forceinline__ void tw_apply_q(float2 *y, const float2 *wb, std::integer_sequence<int, J...>) {
+    ((y[J + 1] = cmul_dir<DIR>(y[J + 1], rot<-1, N, QT * (J + 1)>(wb[J + 1]))), ...);
+}
+template <int R, int NB, int T, int N, int DIR, bool UPPER_ZERO, int P, int... Q>
+__device__ __forceinline__ void wide_last_stage(float2 (&x)[P], float2 (&y)[NB][R], const float2 *wb,
+                                                std::integer_sequence<int, Q...>) {
+    auto one = [&](auto qc) {
+        constexpr int q = decltype(qc)::value;
+#pragma unroll
+        for (int r = 0; r < R; ++r) y[q][r] = x[q + r * NB];
+        tw_apply_q<DIR, N, q * T>(y[q], wb, std::make_integer_sequence<int, R - 1>{});
+        dft_dif<R, DIR, UPPER_ZERO>(y[q]);
+    };
+    (one(std::integral_constant<int, Q>{}), ...);
+}
+
 // ----------------------------------------------------------------------------
 // One Stockham stage.  x: the thread's P registers.  If LAST, outputs are left
 // in registers (natural order); otherwise written to sbuf and read back.
@@ -188,6 +215,14 @@ __device__ __forceinline__ void fft_stage(float2 (&x)[1 << LOG_P], float2 *sbuf,
     constexpr bool LAST = (S == plan_stages(LOG_M, LOG_P) - 1);
 
     float2 y[NB][R];
+    if constexpr (S > 0 && PS > T) {
+        static_assert(LAST, "a stage wider than the thread count must be the last");
+        // W^{(t + qT) r} = W^{t r} * W^{qT r}; the second factor is constant
+        float2 wb[R];
+#pragma unroll
+        for (int r = 1; r < R; ++r) wb[r] = __ldg(tw + (r - 1) * T + t);
+        wide_last_stage<R, NB, T, PS * R, DIR, UPPER_ZERO>(x, y, wb, std::make_integer_sequence<int, NB>{});
+    } else {
 #pragma unroll
     for (int q = 0; q < NB; ++q) {
         const int i = t + q * T;
@@ -199,6 +234,7 @@ __device__ __forceinline__ void fft_stage(float2 (&x)[1 << LOG_P], float2 *sbuf,
             for (int r = 1; r < R; ++r) y[q][r] = cmul_dir<DIR>(y[q][r], __ldg(tw + (r - 1) * PS + k));
         }
         dft_dif<R, DIR, UPPER_ZERO>(y[q]);
+    }
     }
     if constexpr (LAST) {
 #pragma unroll

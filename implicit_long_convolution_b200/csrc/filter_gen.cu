@@ -25,6 +25,7 @@ constexpr int TP = 32;          // positions per CTA
 constexpr int NT = 256;         // threads
 constexpr int OC = 128;         // outputs per weight chunk
 constexpr int OUT_CHUNK = 256;  // last-layer outputs per CTA (grid z)
+constexpr int WS = OC + 1;      // row stride of the staged (transposed) weights
 constexpr int MAXW = 132;       // max layer width (input encoding or hidden), multiple of 4
 constexpr int MAXL = 4;
 
@@ -52,7 +53,7 @@ __global__ void __launch_bounds__(NT) filter_gen_kernel(const GenParams p) {
     extern __shared__ float sm[];
     float *actA = sm;                      // [MAXW][TP]
     float *actB = actA + MAXW * TP;        // [MAXW][TP]
-    float *wt = actB + MAXW * TP;          // [MAXW][OC] transposed weight chunk
+    float *wt = actB + MAXW * TP;          // [MAXW][WS] transposed weight chunk
     __shared__ float s_norm[TP];           // decay argument per position (t/L or |r|/g)
     __shared__ int s_valid[TP];
 
@@ -137,10 +138,16 @@ __global__ void __launch_bounds__(NT) filter_gen_kernel(const GenParams p) {
         const int obeg = last ? blockIdx.z * OUT_CHUNK : 0;
         const int oend = last ? min(wout, obeg + OUT_CHUNK) : wout;
         for (int o0 = obeg; o0 < oend; o0 += OC) {
-            // stage W[o0 .. o0+OC)[0..win) transposed
-            for (int idx = tid; idx < OC * win; idx += NT) {
-                const int oo = idx / win, i = idx % win;
-                wt[i * OC + oo] = (o0 + oo < oend) ? __ldg(W + (int64_t)(o0 + oo) * win + i) : 0.f;
+            // stage W[o0 .. o0+OC)[0..win) transposed with row stride OC+1:
+            // consecutive threads read consecutive inputs of one output row
+            // (coalesced) and their stores land in distinct banks
+            {
+                const int lane = tid & 31, wid = tid >> 5;
+                for (int oo = wid; oo < OC; oo += NT / 32) {
+                    const bool ok = o0 + oo < oend;
+                    const float *wrow = W + (int64_t)(o0 + oo) * win;
+                    for (int i = lane; i < win; i += 32) wt[i * WS + oo] = ok ? __ldg(wrow + i) : 0.f;
+                }
             }
             __syncthreads();
             float acc[4][4];
@@ -148,11 +155,12 @@ __global__ void __launch_bounds__(NT) filter_gen_kernel(const GenParams p) {
             for (int a = 0; a < 4; ++a)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
+#pragma unroll 4
             for (int i = 0; i < win; ++i) {
                 const float4 av = *reinterpret_cast<const float4 *>(cur + i * TP + tx * 4);
-                const float4 wv = *reinterpret_cast<const float4 *>(wt + i * OC + ty * 4);
+                const float *wr = wt + i * WS + ty * 4;
                 const float aa[4] = {av.x, av.y, av.z, av.w};
-                const float ww[4] = {wv.x, wv.y, wv.z, wv.w};
+                const float ww[4] = {wr[0], wr[1], wr[2], wr[3]};
 #pragma unroll
                 for (int a = 0; a < 4; ++a)
 #pragma unroll
@@ -178,20 +186,27 @@ __global__ void __launch_bounds__(NT) filter_gen_kernel(const GenParams p) {
                         nxt[o * TP + tx * 4 + a] = v;
                     }
                 } else {
+                    // last layer: decay window, staged in the free activation
+                    // buffer as [output][position] for coalesced row stores
                     const float al = __ldg(p.alpha + o);
-                    float *hrow = p.h + ((int64_t)set * wout + o) * p.npos + p0;
 #pragma unroll
                     for (int a = 0; a < 4; ++a) {
                         const int pos = tx * 4 + a;
-                        if (p0 + pos < p.npos) {
-                            float v = (acc[a][c] + bo) * expf(-al * s_norm[pos]);
-                            if (!s_valid[pos]) v = 0.f;
-                            hrow[pos] = v;
-                        }
+                        float v = (acc[a][c] + bo) * expf(-al * s_norm[pos]);
+                        if (!s_valid[pos]) v = 0.f;
+                        nxt[(o - o0) * TP + pos] = v;
                     }
                 }
             }
             __syncthreads();
+            if (last) {
+                const int nrow = min(OC, oend - o0);
+                for (int idx = tid; idx < nrow * TP; idx += NT) {
+                    const int ol = idx / TP, pos = idx % TP;
+                    if (p0 + pos < p.npos) p.h[((int64_t)set * wout + o0 + ol) * p.npos + p0 + pos] = nxt[ol * TP + pos];
+                }
+                __syncthreads();
+            }
         }
         float *tmp = cur;
         cur = nxt;
@@ -229,7 +244,7 @@ hy_status launch_filter_gen(const hy_filter_desc &d, float *h, cudaStream_t s) {
     p.h = h;
     const int64_t nblk = (p.npos + TP - 1) / TP;
     if (nblk > 0x7fffffffLL || d.n_sets > 65535) return set_error(HY_ERR_UNSUPPORTED, "filter grid too large");
-    const size_t smem = sizeof(float) * (size_t)(2 * MAXW * TP + MAXW * OC);
+    const size_t smem = sizeof(float) * (size_t)(2 * MAXW * TP + MAXW * WS);
     cudaError_t e = cudaFuncSetAttribute(filter_gen_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return set_cuda_error("filter_gen smem attribute", e);
     const int nout = d.widths[d.n_layers];

@@ -8,7 +8,8 @@
 //   multiply  Y[k] = X[k] · H[k]                 (filter spectrum or gate)
 //   merge     Z'[k] = (Y[k] + Y*[M-k]) + i W_n^{-k} (Y[k] - Y*[M-k])
 //   inverse   z' = IFFT_M(Z') / n ;  c[2m] = Re z'[m], c[2m+1] = Im z'[m]
-//   epilogue  z_k = x_k ⊙ (c + D_k · z_{k-1})   (next order starts from z_k)
+//   epilogue  z_k = x_k ⊙ c                    (next order starts from z_k)
+// The skip term D_k·z_{k-1} is applied in the spectrum (bins times H + D_k).
 // Split and merge of bins k and M-k are done together by the thread owning
 // k < M/2; the partner value crosses shared memory.  Only the first L
 // samples of each order are kept (the rest of the padded row restarts at 0),
@@ -45,31 +46,37 @@ struct ResidentParams {
     const float2 *tw_split;
 };
 
+// The skip term folds into the spectrum: h * u + D u = (h + D delta) * u, and
+// the spectrum of delta is 1 at every bin, so each bin is multiplied by H + D.
+// Bins k = t + m*T (m < P/2) pair with M - k; a batch of pairs issues its
+// spectrum loads together so their L2 round trips overlap.  The split twiddle
+// W_n^k (n = 2M) is W_n^t * W_{2P}^m: one table entry per thread times a
+// compile-time rotation.
 template <int LOG_M, int LOG_P>
 __device__ __forceinline__ void split_multiply_merge(float2 (&x)[1 << LOG_P], float2 *sbuf, int t,
                                                      const float2 *__restrict__ H,
-                                                     const float2 *__restrict__ tws) {
+                                                     const float2 *__restrict__ tws, float dk) {
     constexpr int M = 1 << LOG_M;
     constexpr int P = 1 << LOG_P;
     constexpr int T = M / P;
-    store_own<LOG_M, LOG_P>(x, sbuf, t);
-    // bins k = t + m*T (m < P/2) pair with M - k; the loads of a batch of
-    // pairs are issued together so their L2 round trips overlap
     constexpr int BATCH = (P / 2) < 4 ? (P / 2) : 4;
+    store_own<LOG_M, LOG_P>(x, sbuf, t);
+    const float2 wt0 = ldc(tws + t);
     __syncthreads();
-#pragma unroll
-    for (int m0 = 0; m0 < P / 2; m0 += BATCH) {
-        float2 hk[BATCH], hn[BATCH], wk[BATCH];
+    auto batch = [&](auto bc) {
+        constexpr int m0 = decltype(bc)::value * BATCH;
+        float2 hk[BATCH], hn[BATCH];
 #pragma unroll
         for (int j = 0; j < BATCH; ++j) {
             const int k = t + (m0 + j) * T;
             hk[j] = ldv(H + k);
             hn[j] = ldv(H + (M - k));
-            wk[j] = ldc(tws + k);
+            hk[j].x += dk;
+            hn[j].x += dk;
         }
-#pragma unroll
-        for (int j = 0; j < BATCH; ++j) {
-            const int m = m0 + j;
+        auto pair = [&](auto jc) {
+            constexpr int j = decltype(jc)::value;
+            constexpr int m = m0 + j;
             const int k = t + m * T;
             if (k == 0) {
                 // DC and Nyquist: X[0] = Re Z0 + Im Z0, X[M] = Re Z0 - Im Z0
@@ -84,7 +91,7 @@ __device__ __forceinline__ void split_multiply_merge(float2 (&x)[1 << LOG_P], fl
                 const float2 zn = sbuf[partner_slot<LOG_M, LOG_P>(t, m)];
                 const float2 A = make_float2(zk.x + zn.x, zk.y - zn.y);   // Z[k] + Z*[M-k]
                 const float2 Bv = make_float2(zk.x - zn.x, zk.y + zn.y);  // Z[k] - Z*[M-k]
-                const float2 w = wk[j];                                   // W_n^k
+                const float2 w = rot<-1, 2 * P, m>(wt0);                  // W_n^k
                 const float2 wB = cmul(Bv, w);
                 const float2 C = make_float2(wB.y, -wB.x);                // -i W B
                 const float2 Xk = cadd(A, C);                             // 2 X[k]
@@ -98,12 +105,15 @@ __device__ __forceinline__ void split_multiply_merge(float2 (&x)[1 << LOG_P], fl
                 x[m] = cadd(A2, C2);
                 sbuf[partner_slot<LOG_M, LOG_P>(t, m)] = cconj(csub(A2, C2));
             }
-        }
-    }
+        };
+        fold_seq(pair, std::make_integer_sequence<int, BATCH>{});
+    };
+    fold_seq(batch, std::make_integer_sequence<int, (P / 2) / BATCH>{});
     if (t == 0) {
-        // k = M/2 pairs with itself: Z'[M/2] = 4 Z[M/2] conj(H[M/2]) (doubled scale)
+        // k = M/2 pairs with itself: Z'[M/2] = 4 Z[M/2] conj(H[M/2] + D) (doubled scale)
         const float2 z = x[P / 2];
-        const float2 hm = ldv(H + M / 2);
+        float2 hm = ldv(H + M / 2);
+        hm.x += dk;
         const float2 r = cmulc(z, hm);
         x[P / 2] = make_float2(4.f * r.x, 4.f * r.y);
     }
@@ -135,7 +145,6 @@ resident_conv_kernel(const ResidentParams p) {
 
     extern __shared__ float2 smem[];
     float2 *sbuf = smem;
-    float2 *ustash = smem + spad_size(M);   // z_{k-1} for orders >= 2
 
     const int t = threadIdx.x;
     const int64_t c = blockIdx.x;
@@ -162,26 +171,29 @@ resident_conv_kernel(const ResidentParams p) {
     }
 
     auto one_order = [&](const int k, const bool last) {
+        // thread index re-read per order (volatile): addresses derived from it
+        // are formed inside the order loop instead of held across it
+        int t;
+        asm volatile("mov.u32 %0, %%tid.x;" : "=r"(t));
         block_fft<LOG_M, LOG_P, -1, !CIRC>(x, sbuf, t, p.tw_fft);
+        const float dk = p.skip[k] ? ldv(p.skip[k] + ch) : 0.f;
         const float2 *H = p.spec[k] + smp * p.spec_batch_stride + ch * p.spec_row_stride;
-        split_multiply_merge<LOG_M, LOG_P>(x, sbuf, t, H, p.tw_split);
+        split_multiply_merge<LOG_M, LOG_P>(x, sbuf, t, H, p.tw_split, dk);
         block_fft<LOG_M, LOG_P, +1, false>(x, sbuf, t, p.tw_fft);
 
-        const float dk = p.skip[k] ? ldv(p.skip[k] + ch) : 0.f;
         const IO *g = reinterpret_cast<const IO *>(p.gate[k]);
         const IO *grow = g ? g + row * (int64_t)L : nullptr;
         IO *yout = reinterpret_cast<IO *>(p.y) + row * (int64_t)L;
-        // batches of EB samples: issue the batch's gate / skip loads first
-        // (the output stores would otherwise order each load behind them)
+        // batches of EB samples: issue the batch's gate loads first (the
+        // output stores would otherwise order each load behind them)
         constexpr int EB = (PIN < 8) ? PIN : 8;
 #pragma unroll
         for (int m0 = 0; m0 < PIN; m0 += EB) {
-            float2 gv[EB], pv[EB];
+            float2 gv[EB];
 #pragma unroll
             for (int j = 0; j < EB; ++j) {
                 const int i0 = 2 * (t + (m0 + j) * T);
                 gv[j] = make_float2(1.f, 1.f);
-                pv[j] = make_float2(0.f, 0.f);
                 if (grow) {
                     if (pairs) {
                         if (i0 < L) gv[j] = IOT::load2(grow + i0);
@@ -190,26 +202,12 @@ resident_conv_kernel(const ResidentParams p) {
                         if (i0 + 1 < L) gv[j].y = IOT::load(grow + i0 + 1);
                     }
                 }
-                if (k == 0) {
-                    if (dk != 0.f) {
-                        if (pairs) {
-                            if (i0 < L) pv[j] = IOT::load2(u + i0);
-                        } else {
-                            if (i0 < L) pv[j].x = IOT::load(u + i0);
-                            if (i0 + 1 < L) pv[j].y = IOT::load(u + i0 + 1);
-                        }
-                    }
-                } else {
-                    pv[j] = ustash[t + (m0 + j) * T];
-                }
             }
 #pragma unroll
             for (int j = 0; j < EB; ++j) {
                 const int m = m0 + j;
-                const int e = t + m * T;
-                const int i0 = 2 * e;
-                float2 z = make_float2(fmaf(x[m].x, p.scale, dk * pv[j].x), fmaf(x[m].y, p.scale, dk * pv[j].y));
-                z = make_float2(z.x * gv[j].x, z.y * gv[j].y);
+                const int i0 = 2 * (t + m * T);
+                float2 z = make_float2(x[m].x * p.scale * gv[j].x, x[m].y * p.scale * gv[j].y);
                 if (i0 >= L) z.x = 0.f;
                 if (i0 + 1 >= L) z.y = 0.f;
                 if (last) {
@@ -220,7 +218,6 @@ resident_conv_kernel(const ResidentParams p) {
                         if (i0 + 1 < L) IOT::store(yout + i0 + 1, z.y);
                     }
                 } else {
-                    ustash[e] = z;
                     x[m] = z;
                 }
             }
@@ -241,8 +238,8 @@ resident_conv_kernel(const ResidentParams p) {
 // L = 2^(LOG_M+1) (circular) samples per row: a persistent CTA walks its rows
 // and overlaps HBM with the FFTs.  While row r is being transformed, cp.async
 // brings row r+1's input and row r's gate into shared memory (stage buffers
-// next to the FFT exchange buffer); the skip term reuses the input samples
-// kept packed in registers.  Without PF_GATE (when two stage buffers would not
+// next to the FFT exchange buffer); the skip term rides on the spectrum (see
+// split_multiply_merge).  Without PF_GATE (when two stage buffers would not
 // fit) the gate is read from global memory in the epilogue.
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
@@ -252,22 +249,6 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-template <typename IO> struct Packed;              // one sample pair kept for the skip term
-template <> struct Packed<__nv_bfloat16> {
-    uint32_t v;
-    __device__ __forceinline__ void set(float2 f) {
-        v = (__float_as_uint(f.x) >> 16) | (__float_as_uint(f.y) & 0xffff0000u);
-    }
-    __device__ __forceinline__ float2 get() const {
-        return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
-    }
-};
-template <> struct Packed<float> {
-    float2 v;
-    __device__ __forceinline__ void set(float2 f) { v = f; }
-    __device__ __forceinline__ float2 get() const { return v; }
-};
 
 // float2 slots before the stage buffers (even, so they start 16-byte aligned)
 __host__ __device__ constexpr int stream_stage_offset(int m) { return ((spad_size(m) + 1) / 2) * 2; }
@@ -313,16 +294,17 @@ resident_stream_kernel(const ResidentParams p) {
     int64_t c = blockIdx.x;
     if (c < p.n_rows) copy_row(in_st, ubase + row_of(c) * L);
     cp_async_commit();
-    const float dk_null = 0.f;
     for (; c < p.n_rows; c += gridDim.x) {
+        // the thread index re-read per row (volatile) so the addresses derived
+        // from it are formed inside the loop instead of held across it
+        int t;
+        asm volatile("mov.u32 %0, %%tid.x;" : "=r"(t));
         const int64_t row = row_of(c);
         const int64_t ch = (row / p.sdiv) % p.smod;
         const int64_t smp = row / (p.sdiv * p.smod);
         cp_async_wait<0>();
         __syncthreads();
         float2 x[P];
-        constexpr int NKEEP = CIRC ? 1 : PIN;             // the spectral gate has no skip term
-        Packed<IO> keep[NKEEP];
 #pragma unroll
         for (int m = 0; m < P; ++m) {
             x[m] = make_float2(0.f, 0.f);
@@ -334,7 +316,6 @@ resident_stream_kernel(const ResidentParams p) {
                 } else {
                     x[m] = *reinterpret_cast<const float2 *>(in_st + i0);
                 }
-                if constexpr (!CIRC) keep[m].set(x[m]);
             }
         }
         __syncthreads();                                  // stage buffer free for the next row
@@ -344,11 +325,11 @@ resident_stream_kernel(const ResidentParams p) {
         cp_async_commit();
 
         block_fft<LOG_M, LOG_P, -1, !CIRC>(x, sbuf, t, p.tw_fft);
+        const float dk = p.skip[0] ? ldv(p.skip[0] + ch) : 0.f;
         const float2 *H = p.spec[0] + smp * p.spec_batch_stride + ch * p.spec_row_stride;
-        split_multiply_merge<LOG_M, LOG_P>(x, sbuf, t, H, p.tw_split);
+        split_multiply_merge<LOG_M, LOG_P>(x, sbuf, t, H, p.tw_split, dk);
         block_fft<LOG_M, LOG_P, +1, false>(x, sbuf, t, p.tw_fft);
 
-        const float dk = p.skip[0] ? ldv(p.skip[0] + ch) : dk_null;
         if constexpr (PF_GATE) {
             cp_async_wait<1>();                           // the gate of this row has landed
             __syncthreads();
@@ -357,13 +338,7 @@ resident_stream_kernel(const ResidentParams p) {
 #pragma unroll
         for (int m = 0; m < PIN; ++m) {
             const int i0 = 2 * (t + m * T);
-            float2 z;
-            if constexpr (CIRC) {
-                z = make_float2(x[m].x * p.scale, x[m].y * p.scale);
-            } else {
-                const float2 pv = keep[m].get();
-                z = make_float2(fmaf(x[m].x, p.scale, dk * pv.x), fmaf(x[m].y, p.scale, dk * pv.y));
-            }
+            float2 z = make_float2(x[m].x * p.scale, x[m].y * p.scale);
             if (gbase) {
                 float2 gv;
                 if constexpr (PF_GATE) {

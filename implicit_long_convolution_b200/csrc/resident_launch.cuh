@@ -26,7 +26,7 @@ hy_status launch_conv_t(ResidentParams p, cudaStream_t s) {
     p.tw_fft = tw_stages(LOG_M, LOG_P);
     p.tw_split = tw_split(LOG_M);
     if (!p.tw_fft || !p.tw_split) return set_error(HY_ERR_CUDA, "twiddle tables missing for M=2^%d", LOG_M);
-    const size_t smem = sizeof(float2) * (size_t)(spad_size(M) + ((CHAIN && p.K > 1) ? M / 2 : 0));
+    const size_t smem = sizeof(float2) * (size_t)spad_size(M);
     auto kernel = resident_conv_kernel<LOG_M, IO, CIRC, CHAIN>;
     hy_status st = set_smem_limit(kernel, smem, "resident conv smem attribute");
     if (st != HY_OK) return st;

@@ -46,8 +46,9 @@ struct Registry {
         for (int s = 1; s < ns; ++s) {
             const int R = 1 << plan_log_radix(log_m, log_p, s);
             const int p = 1 << plan_log_p(log_m, log_p, s);
+            const int cols = plan_tw_cols(log_m, log_p, s);   // min(p, T): see fft_core.cuh
             for (int r = 1; r < R; ++r)
-                for (int k = 0; k < p; ++k) v.push_back(w_forward((int64_t)k * r, (int64_t)p * R));
+                for (int k = 0; k < cols; ++k) v.push_back(w_forward((int64_t)k * r, (int64_t)p * R));
         }
         if (v.empty()) v.push_back(make_float2(1.f, 0.f));
         add(key, v);

@@ -78,6 +78,33 @@ def workload_bytes(spec):
     return op, op
 
 
+CONV_SOURCES = ["common.cuh", "fft_core.cuh", "resident.cuh", "resident_launch.cuh", "resident.cu",
+                "resident_stream_bf16.cu", "resident_stream_f32.cu", "twiddle.cu", "twiddle.h"]
+
+
+def conv_sources_digest():
+    """sha256 over the sources of the on-chip convolution kernels."""
+    import hashlib
+    hsh = hashlib.sha256()
+    for f in CONV_SOURCES:
+        with open(os.path.join(ROOT, "implicit_long_convolution_b200", "csrc", f), "rb") as fh:
+            hsh.update(fh.read())
+    return hsh.hexdigest()
+
+
+def recorded_traffic(kernel_key):
+    """DRAM bytes per launch from the last ncu capture of this kernel, or None
+    when the kernel's sources changed since (profiles/dram_traffic.json)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel_key)
+    if not rec or rec.get("sources_sha256") != conv_sources_digest():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -420,7 +447,9 @@ def run_ours(args):
         "conv_ms": round(op_avg, 4),
         "roofline": {"bound": "hbm", "kernel": st.kernel,
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "peak_kind": peak_kind, "traffic": None},
+                     "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                     "traffic": recorded_traffic(name) if s["kind"] == "operator" and "resident" in st.kernel
+                     else None},
         "e2e": {"value": round(world * step_bytes / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": st.launches * steps,

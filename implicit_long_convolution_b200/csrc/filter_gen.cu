@@ -5,11 +5,11 @@
 // exponential decay window; [ND] 방법론: HyenaND: coordinate MLP on the N-D
 // grid with FiLM conditioning per sample.
 //
-// One CTA evaluates TP = 32 positions of one filter set for one chunk of at
-// most OUT_CHUNK outputs of the last layer (grid z): it builds the positional
+// One CTA evaluates TP = 64 positions of one filter set for one chunk of the
+// outputs of the last layer (grid z; only as many chunks as fill the GPU): it builds the positional
 // encoding in shared memory, runs every MLP layer as a small fp32 GEMM
 // (register tile of 4 positions x 4 outputs per thread, weights staged in
-// shared memory 128 outputs at a time), applies FiLM and SiLU on hidden
+// shared memory 64 outputs at a time), applies FiLM and SiLU on hidden
 // layers and the decay window on the last one, and writes the filter rows
 // with the position index fastest (coalesced).  The hidden layers are
 // recomputed per output chunk; they are a small part of the work when the
@@ -21,11 +21,10 @@ namespace hy {
 
 namespace {
 
-constexpr int TP = 32;          // positions per CTA
+constexpr int TP = 64;          // positions per CTA
 constexpr int NT = 256;         // threads
-constexpr int OC = 128;         // outputs per weight chunk
-constexpr int OUT_CHUNK = 256;  // last-layer outputs per CTA (grid z)
-constexpr int WS = OC + 1;      // row stride of the staged (transposed) weights
+constexpr int OC = 64;          // outputs per weight chunk
+constexpr int WS = OC + 4;      // row stride of the staged (transposed) weights (float4-aligned)
 constexpr int MAXW = 132;       // max layer width (input encoding or hidden), multiple of 4
 constexpr int MAXL = 4;
 
@@ -42,6 +41,7 @@ struct GenParams {
     const float *gamma, *beta;
     const float *alpha;
     int64_t npos;               // positions per set (L or S^3)
+    int out_chunk;              // last-layer outputs per CTA (grid z), multiple of OC
     float *h;
 };
 
@@ -135,12 +135,12 @@ __global__ void __launch_bounds__(NT) filter_gen_kernel(const GenParams p) {
         const bool last = (l == p.nl - 1);
         const float *W = p.W[l];
         const float *bias = p.b[l];
-        const int obeg = last ? blockIdx.z * OUT_CHUNK : 0;
-        const int oend = last ? min(wout, obeg + OUT_CHUNK) : wout;
+        const int obeg = last ? blockIdx.z * p.out_chunk : 0;
+        const int oend = last ? min(wout, obeg + p.out_chunk) : wout;
         for (int o0 = obeg; o0 < oend; o0 += OC) {
-            // stage W[o0 .. o0+OC)[0..win) transposed with row stride OC+1:
-            // consecutive threads read consecutive inputs of one output row
-            // (coalesced) and their stores land in distinct banks
+            // stage W[o0 .. o0+OC)[0..win) transposed (row stride OC+4 keeps
+            // the float4 reads aligned): consecutive threads read consecutive
+            // inputs of one output row (coalesced)
             {
                 const int lane = tid & 31, wid = tid >> 5;
                 for (int oo = wid; oo < OC; oo += NT / 32) {
@@ -158,9 +158,9 @@ __global__ void __launch_bounds__(NT) filter_gen_kernel(const GenParams p) {
 #pragma unroll 4
             for (int i = 0; i < win; ++i) {
                 const float4 av = *reinterpret_cast<const float4 *>(cur + i * TP + tx * 4);
-                const float *wr = wt + i * WS + ty * 4;
+                const float4 wv = *reinterpret_cast<const float4 *>(wt + i * WS + ty * 4);
                 const float aa[4] = {av.x, av.y, av.z, av.w};
-                const float ww[4] = {wr[0], wr[1], wr[2], wr[3]};
+                const float ww[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
                 for (int a = 0; a < 4; ++a)
 #pragma unroll
@@ -247,8 +247,23 @@ hy_status launch_filter_gen(const hy_filter_desc &d, float *h, cudaStream_t s) {
     const size_t smem = sizeof(float) * (size_t)(2 * MAXW * TP + MAXW * WS);
     cudaError_t e = cudaFuncSetAttribute(filter_gen_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return set_cuda_error("filter_gen smem attribute", e);
+    // split the last layer over grid z only as far as needed to fill the GPU
+    // (each split recomputes the hidden layers)
     const int nout = d.widths[d.n_layers];
-    dim3 grid((unsigned)nblk, (unsigned)d.n_sets, (unsigned)((nout + OUT_CHUNK - 1) / OUT_CHUNK));
+    const int64_t base = nblk * d.n_sets;
+    int sms = 148;
+    {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    const int max_chunks = (nout + OC - 1) / OC;
+    int chunks = (int)((2 * (int64_t)sms + base - 1) / base);
+    if (chunks < 1) chunks = 1;
+    if (chunks > max_chunks) chunks = max_chunks;
+    p.out_chunk = ((nout + chunks - 1) / chunks + OC - 1) / OC * OC;
+    chunks = (nout + p.out_chunk - 1) / p.out_chunk;
+    dim3 grid((unsigned)nblk, (unsigned)d.n_sets, (unsigned)chunks);
     filter_gen_kernel<<<grid, NT, smem, s>>>(p);
     return check_launch("filter_gen launch");
 }

@@ -2,6 +2,9 @@
 device results with the float64 oracle."""
 import numpy as np
 
+# measured errors of this session (written out by conftest when PARITY_LOG is set)
+RECORD = []
+
 # tolerances of the hot path (fp32 math): fp32 I/O and bf16 I/O
 F32_REL_L2 = 1e-5
 F32_MAXABS_OF_RMS = 1e-4
@@ -44,11 +47,12 @@ def check(a, ref, dtype, what=""):
     assert a.shape == ref.shape, (a.shape, ref.shape)
     assert np.all(np.isfinite(a)), what + ": non-finite output"
     r = rel_l2(a, ref)
+    rms = float(np.sqrt(np.mean(ref ** 2))) if ref.size else 0.0
+    mx = float(np.max(np.abs(a - ref))) if ref.size else 0.0
+    RECORD.append({"what": what, "dtype": dtype, "rel_l2": r, "maxabs_over_rms": mx / rms if rms else 0.0})
     if dtype == "bf16":
         assert r <= BF16_REL_L2, "%s: rel-L2 %.3e > %.0e" % (what, r, BF16_REL_L2)
     else:
-        rms = float(np.sqrt(np.mean(ref ** 2))) if ref.size else 0.0
-        mx = float(np.max(np.abs(a - ref))) if ref.size else 0.0
         assert r <= F32_REL_L2, "%s: rel-L2 %.3e > %.0e" % (what, r, F32_REL_L2)
         assert mx <= F32_MAXABS_OF_RMS * rms + 1e-30, "%s: max-abs %.3e > 1e-4*RMS %.3e" % (what, mx, rms)
     return r

@@ -9,3 +9,16 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running CPU oracle case")
+
+
+def pytest_sessionfinish(session, exitstatus):
+    path = os.environ.get("PARITY_LOG")
+    if not path:
+        return
+    try:
+        import json
+        import _helpers
+        with open(path, "w") as f:
+            json.dump(_helpers.RECORD, f, indent=1)
+    except Exception:
+        pass

@@ -332,7 +332,8 @@ def run_ours(args):
 
     world, rank, local = dist_setup()
     name = args.workload
-    w = hw.make(name, seed=rank_seed(name, rank))
+    over = {"D": args.channels} if args.channels else {}
+    w = hw.make(name, seed=rank_seed(name, rank), **over)
     s = w.spec
     dev = torch.device("cuda", local)
     setup = {"operator": setup_operator, "nd": setup_nd, "gate": setup_gate}[s["kind"]]
@@ -420,7 +421,7 @@ def run_ours(args):
     h2d = sum(hh.numel() * hh.element_size() for hh in hosts)
     d2h = out_h.numel() * out_h.element_size()
 
-    cfg = {"workload": DESCR[name]}
+    cfg = {"workload": DESCR[name] + (" [D=%d profiling case]" % s["D"] if over else "")}
     cfg.update({k: v for k, v in s.items() if k in ("B", "D", "L", "order", "H", "Dh", "grid")})
     cfg.update({"step": ("filter_gen + filter_spectrum + convolution" if s["kind"] != "gate"
                          else "spectral_gate"),
@@ -430,7 +431,7 @@ def run_ours(args):
                 "parallelism": "independent replicas x%d (no data-path collective)" % world})
     el = 2 if s["dtype"] == "bf16" else 4
     line = {
-        "metric": "Hyena op GB/s (%s)" % DESCR[name],
+        "metric": "Hyena op GB/s (%s)" % cfg["workload"],
         "value": round(value, 2),
         "unit": "GB/s",
         "n_gpus": world,
@@ -549,7 +550,11 @@ def main():
     ap.add_argument("--workload", choices=sorted(DESCR), default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--channels", type=int, default=0,
+                    help="override the channel count D (smaller cases for profiler captures)")
     args = ap.parse_args()
+    if args.channels and hw.WORKLOADS[args.workload]["kind"] == "gate":
+        ap.error("--channels applies to the operator and N-D workloads")
     if args.impl == "reference":
         if args.steps <= 0:
             args.steps = 3

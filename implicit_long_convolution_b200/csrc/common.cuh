@@ -129,6 +129,17 @@ __device__ __forceinline__ uint32_t ldv_u32(const void *p) {
     asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
     return v;
 }
+__device__ __forceinline__ float4 ldv4(const float *p) {
+    float4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint2 ldv_u64(const void *p) {
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return v;
+}
 // L1-cached ordered load (small tables shared by all rows)
 __device__ __forceinline__ float2 ldc(const float2 *p) {
     float2 v;
@@ -145,10 +156,13 @@ template <> struct IOTraits<float> {
     static __device__ __forceinline__ float2 load2(const float *p) {
         return ldv(reinterpret_cast<const float2 *>(p));
     }
+    // 4 consecutive elements; p 16-byte aligned
+    static __device__ __forceinline__ float4 load4(const float *p) { return ldv4(p); }
     static __device__ __forceinline__ void store(float *p, float v) { *p = v; }
     static __device__ __forceinline__ void store2(float *p, float2 v) {
         *reinterpret_cast<float2 *>(p) = v;
     }
+    static __device__ __forceinline__ void store4(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
 };
 // bf16 -> fp32 is the exact widening of the top 16 bits.
 template <> struct IOTraits<__nv_bfloat16> {
@@ -159,9 +173,22 @@ template <> struct IOTraits<__nv_bfloat16> {
         const uint32_t v = ldv_u32(p);
         return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
     }
+    // 4 consecutive elements; p 8-byte aligned
+    static __device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
+        const uint2 v = ldv_u64(p);
+        return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                           __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+    }
     static __device__ __forceinline__ void store(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
     static __device__ __forceinline__ void store2(__nv_bfloat16 *p, float2 v) {
         *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(v.x, v.y);
+    }
+    static __device__ __forceinline__ void store4(__nv_bfloat16 *p, float4 v) {
+        const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+        uint2 u;
+        u.x = *reinterpret_cast<const uint32_t *>(&a);
+        u.y = *reinterpret_cast<const uint32_t *>(&b);
+        *reinterpret_cast<uint2 *>(p) = u;
     }
 };
 

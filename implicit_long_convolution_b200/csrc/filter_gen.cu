@@ -5,15 +5,21 @@
 // exponential decay window; [ND] 방법론: HyenaND: coordinate MLP on the N-D
 // grid with FiLM conditioning per sample.
 //
-// One CTA evaluates TP = 64 positions of one filter set for one chunk of the
-// outputs of the last layer (grid z; only as many chunks as fill the GPU): it builds the positional
-// encoding in shared memory, runs every MLP layer as a small fp32 GEMM
-// (register tile of 4 positions x 4 outputs per thread, weights staged in
-// shared memory 64 outputs at a time), applies FiLM and SiLU on hidden
-// layers and the decay window on the last one, and writes the filter rows
-// with the position index fastest (coalesced).  The hidden layers are
-// recomputed per output chunk; they are a small part of the work when the
-// last layer is wide, and the chunks give the grid enough CTAs.
+// One CTA owns P = 64 consecutive positions of one filter set.  It builds
+// the positional encoding in shared memory, runs the hidden layers once
+// (64-output tiles) and then sweeps the last layer in 128-output tiles;
+// only when the grid has fewer CTAs than SMs is the last layer split over
+// grid z (each split recomputes the small hidden layers).  Every
+// layer is an fp32 GEMM over K = layer input width, accumulated as K outer
+// products into a 4-position x CPT-output register tile per thread:
+//   activations  act[k][pos]    (one float4 read: 4 positions)
+//   weights      wT[k][o]       (transposed while staged; CPT/4 float4 reads)
+// so each k costs 1 + CPT/4 shared loads for 4*CPT independent FMAs.  The
+// weight tile (with its bias, decay rates and FiLM rows) of the next tile is
+// copied with cp.async while the current one is computed (two buffers).
+// Hidden outputs get bias, FiLM and the activation and stay in shared
+// memory; last-layer outputs get bias and the decay window and go straight
+// to HBM as float4 row segments.
 #include "kernels.h"
 #include "status.h"
 
@@ -21,17 +27,20 @@ namespace hy {
 
 namespace {
 
-constexpr int TP = 64;          // positions per CTA
-constexpr int NT = 256;         // threads
-constexpr int OC = 64;          // outputs per weight chunk
-constexpr int WS = OC + 4;      // row stride of the staged (transposed) weights (float4-aligned)
-constexpr int MAXW = 132;       // max layer width (input encoding or hidden), multiple of 4
+constexpr int P = 64;           // positions per CTA
+constexpr int NT = 256;         // threads: 16 position groups x 16 output groups
+constexpr int CPT_H = 4;        // outputs per thread, hidden layers (64-output tiles)
+constexpr int CPT_L = 8;        // outputs per thread, last layer (128-output tiles)
+constexpr int OT_MAX = 16 * CPT_L;
+constexpr int OTS = OT_MAX + 4; // wT row stride: = 4 (mod 32) keeps the staging stores conflict-free
+constexpr int MAXW = 132;       // max layer input width
 constexpr int MAXL = 4;
+constexpr int NPAR = 4;         // per-output parameter rows staged with a tile: bias, alpha, gamma, beta
 
 struct GenParams {
     int ndim;
     int64_t L;                  // 1-D length
-    int g, S, circular;         // 3-D
+    int g, S, log_s, circular;  // 3-D
     int F, include_t;
     int nl;
     int widths[MAXL + 1];
@@ -41,7 +50,10 @@ struct GenParams {
     const float *gamma, *beta;
     const float *alpha;
     int64_t npos;               // positions per set (L or S^3)
-    int out_chunk;              // last-layer outputs per CTA (grid z), multiple of OC
+    int ka;                     // max layer input width (activation rows)
+    int wbuf;                   // floats per weight buffer
+    int out_chunk;              // last-layer outputs per grid-z slice (multiple of OT_MAX)
+    int vec_out;                // float4 stores of the output rows are aligned
     float *h;
 };
 
@@ -49,168 +61,266 @@ __device__ __forceinline__ float silu(float a) { return a / (1.f + expf(-a)); }
 
 __device__ __forceinline__ int signed_off(int i, int S) { return i < S / 2 ? i : i - S; }
 
-__global__ void __launch_bounds__(NT) filter_gen_kernel(const GenParams p) {
-    extern __shared__ float sm[];
-    float *actA = sm;                      // [MAXW][TP]
-    float *actB = actA + MAXW * TP;        // [MAXW][TP]
-    float *wt = actB + MAXW * TP;          // [MAXW][WS] transposed weight chunk
-    __shared__ float s_norm[TP];           // decay argument per position (t/L or |r|/g)
-    __shared__ int s_valid[TP];
+__device__ __forceinline__ void cpa4(float *smem, const float *g) {
+    const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sa), "l"(g) : "memory");
+}
+__device__ __forceinline__ void cpa_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cpa_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Stage outputs o0 .. o0+rows of layer l: wT[k][r] = W[o0 + r][k] (k < win)
+// and the per-output rows par[j][r] (bias; decay rate on the last layer;
+// FiLM gamma/beta of this set on the first hidden layer).  A warp copies
+// 4 weight rows x 8 consecutive k per instruction: 32-byte global segments,
+// and with the row stride = 4 (mod 32) the 32 shared stores hit 32 banks.
+// Rows at or past `end` are left as they are (their outputs are not used).
+__device__ __forceinline__ void stage_tile(const GenParams &p, int l, int o0, int rows, int end, int set,
+                                           float *wT) {
+    const int win = p.widths[l];
+    const float *W = p.W[l];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int rr = lane >> 3, kk = lane & 7;
+    for (int r0 = 4 * warp; r0 < rows; r0 += 4 * (NT / 32)) {
+        const int r = r0 + rr;
+        if (o0 + r >= end) continue;
+        const float *src = W + (int64_t)(o0 + r) * win;
+        for (int k0 = 0; k0 < win; k0 += 8) {
+            const int k = k0 + kk;
+            if (k < win) cpa4(wT + k * OTS + r, src + k);
+        }
+    }
+    float *par = wT + p.ka * OTS;
+    const bool last = l == p.nl - 1;
+    const bool film = l == 0 && !last && p.gamma;
+    const int wout = p.widths[l + 1];
+    for (int r = threadIdx.x; r < rows; r += NT) {
+        const int o = o0 + r;
+        if (o >= end) continue;
+        cpa4(par + r, p.b[l] + o);
+        if (last) cpa4(par + OT_MAX + r, p.alpha + o);
+        if (film) {
+            cpa4(par + 2 * OT_MAX + r, p.gamma + (int64_t)set * wout + o);
+            cpa4(par + 3 * OT_MAX + r, p.beta + (int64_t)set * wout + o);
+        }
+    }
+}
+
+// acc[a][c] = sum_k act[k][4tx + a] * wT[k][CPT*ty + c], k ascending.
+template <int CPT>
+__device__ __forceinline__ void tile_gemm(const float *act, const float *wT, int K, int tx, int ty,
+                                          float (&acc)[4][CPT]) {
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) acc[a][c] = 0.f;
+    const float *ap = act + 4 * tx;
+    const float *wp = wT + CPT * ty;
+#pragma unroll 4
+    for (int k = 0; k < K; ++k) {
+        const float4 av = *reinterpret_cast<const float4 *>(ap + k * P);
+        const float x[4] = {av.x, av.y, av.z, av.w};
+        float w[CPT];
+#pragma unroll
+        for (int c4 = 0; c4 < CPT / 4; ++c4) {
+            const float4 wv = *reinterpret_cast<const float4 *>(wp + k * OTS + 4 * c4);
+            w[4 * c4 + 0] = wv.x;
+            w[4 * c4 + 1] = wv.y;
+            w[4 * c4 + 2] = wv.z;
+            w[4 * c4 + 3] = wv.w;
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int c = 0; c < CPT; ++c) acc[a][c] = fmaf(w[c], x[a], acc[a][c]);
+    }
+}
+
+__global__ void __launch_bounds__(NT, 2) filter_gen_kernel(const GenParams p) {
+    extern __shared__ __align__(16) float sm[];
+    float *actA = sm;                          // [ka][P]
+    float *actB = actA + p.ka * P;             // [ka][P]
+    float *const wbase = actB + p.ka * P;      // two buffers: wT [ka][OTS], then NPAR x OT_MAX parameters
+    __shared__ float s_norm[P];                // decay argument per position (t/L or |r|/g)
+    __shared__ int s_valid[P];
 
     const int tid = threadIdx.x;
-    const int64_t p0 = (int64_t)blockIdx.x * TP;
+    const int tx = tid & 15, ty = tid >> 4;
+    const int64_t p0 = (int64_t)blockIdx.x * P;
     const int set = blockIdx.y;
+    const int nl = p.nl;
+    const int nout = p.widths[nl];
+    const int lbeg = blockIdx.z * p.out_chunk;
+    const int lend = min(nout, lbeg + p.out_chunk);
+
+    // tile sequence: hidden layers in 64-output tiles, then the last layer's
+    // slice in 128-output tiles
+    auto tile_rows = [&](int l) { return l == nl - 1 ? 16 * CPT_L : 16 * CPT_H; };
+    auto first_o = [&](int l) { return l == nl - 1 ? lbeg : 0; };
+    auto end_o = [&](int l) { return l == nl - 1 ? lend : p.widths[l + 1]; };
+
+    int l = 0, o0 = first_o(0);
+    stage_tile(p, l, o0, tile_rows(l), end_o(l), set, wbase);
+    cpa_commit();
 
     // ---- positional encoding (a1) into actA[feature][pos]
     const int w0 = p.widths[0];
-    for (int pos = tid; pos < TP; pos += NT) {
-        const int64_t q = p0 + pos;
-        s_valid[pos] = q < p.npos;
-        s_norm[pos] = 0.f;
-    }
     if (p.ndim == 1) {
-        for (int idx = tid; idx < TP * w0; idx += NT) {
-            const int pos = idx % TP, f = idx / TP;
+        // integer phase (j t) mod L, then the angle 2 pi r / L; below 2^24
+        // every integer involved is exact in float
+        const bool narrow = p.L * (int64_t)(p.F + 1) < (1LL << 31) && p.L <= (1 << 24);
+        const float Lf = (float)p.L;
+        for (int idx = tid; idx < P * w0; idx += NT) {
+            const int pos = idx & (P - 1), f = idx / P;
             const int64_t tt = p0 + pos;
             float v = 0.f;
             if (tt < p.npos) {
                 if (p.include_t && f == 0) {
-                    v = (float)((double)tt / (double)p.L);
+                    v = narrow ? __fdiv_rn((float)tt, Lf) : (float)((double)tt / (double)p.L);
                 } else {
                     const int ff = f - p.include_t;      // 0..2F-1
-                    const int j = (ff % p.F) + 1;
-                    const int64_t r = ((int64_t)j * tt) % p.L;
-                    float s, c;
-                    sincospif((float)(2.0 * (double)r / (double)p.L), &s, &c);
-                    v = (ff < p.F) ? c : s;
+                    const int j = (ff < p.F ? ff : ff - p.F) + 1;
+                    float arg;
+                    if (narrow) {
+                        const unsigned r = (unsigned)(j * (int)tt) % (unsigned)p.L;
+                        arg = __fdiv_rn((float)(2 * r), Lf);
+                    } else {
+                        const int64_t r = ((int64_t)j * tt) % p.L;
+                        arg = (float)(2.0 * (double)r / (double)p.L);
+                    }
+                    float sn, cs;
+                    sincospif(arg, &sn, &cs);
+                    v = (ff < p.F) ? cs : sn;
                 }
             }
-            actA[f * TP + pos] = v;
+            actA[f * P + pos] = v;
         }
-        for (int pos = tid; pos < TP; pos += NT) {
+        for (int pos = tid; pos < P; pos += NT) {
             const int64_t tt = p0 + pos;
-            s_norm[pos] = (float)((double)tt / (double)p.L);
+            s_valid[pos] = tt < p.npos;
+            s_norm[pos] = narrow ? __fdiv_rn((float)tt, Lf) : (float)((double)tt / (double)p.L);
         }
     } else {
-        const int S = p.S;
-        for (int idx = tid; idx < TP * w0; idx += NT) {
-            const int pos = idx % TP, f = idx / TP;
+        const int S = p.S, ls = p.log_s, twog_m = 2 * p.g - 1;
+        const float gf = (float)p.g;
+        for (int idx = tid; idx < P * w0; idx += NT) {
+            const int pos = idx & (P - 1), f = idx / P;
             const int64_t q = p0 + pos;
             float v = 0.f;
             if (q < p.npos) {
                 const int axis = f / (2 * p.F);
-                const int ff = f % (2 * p.F);
-                const int j = (ff % p.F) + 1;
-                const int ia = axis == 0 ? (int)(q / ((int64_t)S * S)) : (axis == 1 ? (int)((q / S) % S) : (int)(q % S));
-                const int ra = signed_off(ia, S);
-                const int twog = 2 * p.g;
-                int mm = (j * ra) % twog;
-                if (mm < 0) mm += twog;
-                float s, c;
-                sincospif((float)mm / (float)p.g, &s, &c);     // angle π j r / g
-                v = (ff < p.F) ? c : s;
+                const int ff = f - axis * 2 * p.F;
+                const int j = (ff < p.F ? ff : ff - p.F) + 1;
+                const int ia = (int)(q >> (ls * (2 - axis))) & (S - 1);
+                const int mm = (j * signed_off(ia, S)) & twog_m;   // (j r) mod 2g, 2g a power of two
+                float sn, cs;
+                sincospif((float)mm / gf, &sn, &cs);               // angle pi j r / g
+                v = (ff < p.F) ? cs : sn;
             }
-            actA[f * TP + pos] = v;
+            actA[f * P + pos] = v;
         }
-        for (int pos = tid; pos < TP; pos += NT) {
+        for (int pos = tid; pos < P; pos += NT) {
             const int64_t q = p0 + pos;
+            int valid = 0;
+            float nrm = 0.f;
             if (q < p.npos) {
-                const int r0 = signed_off((int)(q / ((int64_t)S * S)), S);
-                const int r1 = signed_off((int)((q / S) % S), S);
-                const int r2 = signed_off((int)(q % S), S);
-                bool inside = true;
-                if (!p.circular) inside = (abs(r0) < p.g) && (abs(r1) < p.g) && (abs(r2) < p.g);
-                s_valid[pos] = inside ? 1 : 0;
-                s_norm[pos] = sqrtf((float)(r0 * r0 + r1 * r1 + r2 * r2)) / (float)p.g;
+                const int r0 = signed_off((int)(q >> (2 * ls)) & (S - 1), S);
+                const int r1 = signed_off((int)(q >> ls) & (S - 1), S);
+                const int r2 = signed_off((int)q & (S - 1), S);
+                valid = p.circular || ((abs(r0) < p.g) && (abs(r1) < p.g) && (abs(r2) < p.g));
+                nrm = sqrtf((float)(r0 * r0 + r1 * r1 + r2 * r2)) / gf;
             }
+            s_valid[pos] = valid;
+            s_norm[pos] = nrm;
         }
     }
-    __syncthreads();
 
     // ---- MLP layers (a2)
-    const int tx = tid % (TP / 4), ty = tid / (TP / 4);   // positions tx*4.., outputs ty*4..
     float *cur = actA, *nxt = actB;
-    for (int l = 0; l < p.nl; ++l) {
-        const int win = p.widths[l], wout = p.widths[l + 1];
-        const bool last = (l == p.nl - 1);
-        const float *W = p.W[l];
-        const float *bias = p.b[l];
-        const int obeg = last ? blockIdx.z * p.out_chunk : 0;
-        const int oend = last ? min(wout, obeg + p.out_chunk) : wout;
-        for (int o0 = obeg; o0 < oend; o0 += OC) {
-            // stage W[o0 .. o0+OC)[0..win) transposed (row stride OC+4 keeps
-            // the float4 reads aligned): consecutive threads read consecutive
-            // inputs of one output row (coalesced)
-            {
-                const int lane = tid & 31, wid = tid >> 5;
-                for (int oo = wid; oo < OC; oo += NT / 32) {
-                    const bool ok = o0 + oo < oend;
-                    const float *wrow = W + (int64_t)(o0 + oo) * win;
-                    for (int i = lane; i < win; i += 32) wt[i * WS + oo] = ok ? __ldg(wrow + i) : 0.f;
+    int buf = 0;
+    while (l < nl) {
+        // next tile in the sequence, prefetched into the other buffer
+        int nl_l = l, nl_o = o0 + tile_rows(l);
+        if (nl_o >= end_o(l)) {
+            nl_l = l + 1;
+            nl_o = nl_l < nl ? first_o(nl_l) : 0;
+        }
+        if (nl_l < nl) {
+            stage_tile(p, nl_l, nl_o, tile_rows(nl_l), end_o(nl_l), set, wbase + (buf ^ 1) * p.wbuf);
+            cpa_commit();
+            cpa_wait<1>();
+        } else {
+            cpa_wait<0>();
+        }
+        __syncthreads();   // weight tile and the previous layer's activations visible
+
+        const float *wT = wbase + buf * p.wbuf;
+        const float *par = wT + p.ka * OTS;
+        const int K = p.widths[l];
+        if (l < nl - 1) {
+            float acc[4][CPT_H];
+            tile_gemm<CPT_H>(cur, wT, K, tx, ty, acc);
+            const int wout = p.widths[l + 1];
+            const bool film = (l == 0) && p.gamma;
+#pragma unroll
+            for (int c = 0; c < CPT_H; ++c) {
+                const int r = CPT_H * ty + c;
+                const int o = o0 + r;
+                if (o >= wout) continue;
+                const float bo = par[r];
+                const float gm = film ? par[2 * OT_MAX + r] : 0.f;
+                const float bt = film ? par[3 * OT_MAX + r] : 0.f;
+                float v[4];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    float x = acc[a][c] + bo;
+                    if (film) x = fmaf(1.f + gm, x, bt);
+                    if (p.act == HY_ACT_SILU) x = silu(x);
+                    v[a] = x;
                 }
+                *reinterpret_cast<float4 *>(nxt + o * P + 4 * tx) = make_float4(v[0], v[1], v[2], v[3]);
             }
-            __syncthreads();
-            float acc[4][4];
+        } else {
+            float acc[4][CPT_L];
+            tile_gemm<CPT_L>(cur, wT, K, tx, ty, acc);
+            float nrm[4];
+            bool ok[4];
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
-#pragma unroll 4
-            for (int i = 0; i < win; ++i) {
-                const float4 av = *reinterpret_cast<const float4 *>(cur + i * TP + tx * 4);
-                const float4 wv = *reinterpret_cast<const float4 *>(wt + i * WS + ty * 4);
-                const float aa[4] = {av.x, av.y, av.z, av.w};
-                const float ww[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-                for (int a = 0; a < 4; ++a)
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) acc[a][c] = fmaf(ww[c], aa[a], acc[a][c]);
+            for (int a = 0; a < 4; ++a) {
+                nrm[a] = s_norm[4 * tx + a];
+                ok[a] = s_valid[4 * tx + a] != 0;
             }
+            const int64_t q0 = p0 + 4 * tx;
+            const bool full = p.vec_out && q0 + 3 < p.npos;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int o = o0 + ty * 4 + c;
-                if (o >= oend) continue;
-                const float bo = __ldg(bias + o);
-                if (!last) {
-                    float gm = 0.f, bt = 0.f;
-                    const bool film = (l == 0) && p.gamma;
-                    if (film) {
-                        gm = __ldg(p.gamma + (int64_t)set * wout + o);
-                        bt = __ldg(p.beta + (int64_t)set * wout + o);
-                    }
+            for (int c = 0; c < CPT_L; ++c) {
+                const int r = CPT_L * ty + c;
+                const int o = o0 + r;
+                if (o >= lend) continue;
+                const float bo = par[r];
+                const float al = par[OT_MAX + r];
+                float v[4];
 #pragma unroll
-                    for (int a = 0; a < 4; ++a) {
-                        float v = acc[a][c] + bo;
-                        if (film) v = fmaf(1.f + gm, v, bt);
-                        if (p.act == HY_ACT_SILU) v = silu(v);
-                        nxt[o * TP + tx * 4 + a] = v;
-                    }
+                for (int a = 0; a < 4; ++a) v[a] = ok[a] ? (acc[a][c] + bo) * expf(-al * nrm[a]) : 0.f;
+                float *dst = p.h + ((int64_t)set * nout + o) * p.npos + q0;
+                if (full) {
+                    *reinterpret_cast<float4 *>(dst) = make_float4(v[0], v[1], v[2], v[3]);
                 } else {
-                    // last layer: decay window, staged in the free activation
-                    // buffer as [output][position] for coalesced row stores
-                    const float al = __ldg(p.alpha + o);
 #pragma unroll
-                    for (int a = 0; a < 4; ++a) {
-                        const int pos = tx * 4 + a;
-                        float v = (acc[a][c] + bo) * expf(-al * s_norm[pos]);
-                        if (!s_valid[pos]) v = 0.f;
-                        nxt[(o - o0) * TP + pos] = v;
-                    }
+                    for (int a = 0; a < 4; ++a)
+                        if (q0 + a < p.npos) dst[a] = v[a];
                 }
-            }
-            __syncthreads();
-            if (last) {
-                const int nrow = min(OC, oend - o0);
-                for (int idx = tid; idx < nrow * TP; idx += NT) {
-                    const int ol = idx / TP, pos = idx % TP;
-                    if (p0 + pos < p.npos) p.h[((int64_t)set * wout + o0 + ol) * p.npos + p0 + pos] = nxt[ol * TP + pos];
-                }
-                __syncthreads();
             }
         }
-        float *tmp = cur;
-        cur = nxt;
-        nxt = tmp;
+        __syncthreads();   // all reads of this weight buffer and of cur done
+        if (nl_l != l) {
+            float *t = cur;
+            cur = nxt;
+            nxt = t;
+        }
+        l = nl_l;
+        o0 = nl_o;
+        buf ^= 1;
     }
 }
 
@@ -223,14 +333,19 @@ hy_status launch_filter_gen(const hy_filter_desc &d, float *h, cudaStream_t s) {
     p.g = d.grid;
     p.circular = d.circular;
     p.S = d.circular ? d.grid : 2 * d.grid;
+    p.log_s = 0;
+    while ((1 << p.log_s) < p.S) ++p.log_s;
     p.F = d.n_freq;
     p.include_t = d.include_t;
     p.nl = d.n_layers;
     if (p.nl < 1 || p.nl > MAXL) return set_error(HY_ERR_UNSUPPORTED, "n_layers must be 1..%d", MAXL);
+    p.ka = 1;
     for (int l = 0; l <= p.nl; ++l) {
         p.widths[l] = d.widths[l];
-        if (l < p.nl && d.widths[l] > MAXW)
-            return set_error(HY_ERR_UNSUPPORTED, "layer input width %d > %d", d.widths[l], MAXW);
+        if (l < p.nl) {
+            if (d.widths[l] > MAXW) return set_error(HY_ERR_UNSUPPORTED, "layer input width %d > %d", d.widths[l], MAXW);
+            p.ka = d.widths[l] > p.ka ? d.widths[l] : p.ka;
+        }
     }
     for (int l = 0; l < p.nl; ++l) {
         p.W[l] = d.W[l];
@@ -241,14 +356,16 @@ hy_status launch_filter_gen(const hy_filter_desc &d, float *h, cudaStream_t s) {
     p.beta = d.film_beta;
     p.alpha = d.alpha;
     p.npos = d.ndim == 1 ? (int64_t)d.L : (int64_t)p.S * p.S * p.S;
+    p.vec_out = (p.npos % 4 == 0) && ((uintptr_t)h % 16 == 0);
     p.h = h;
-    const int64_t nblk = (p.npos + TP - 1) / TP;
+    p.wbuf = p.ka * OTS + NPAR * OT_MAX;       // a multiple of 4 floats: buffers stay 16-byte aligned
+    const int64_t nblk = (p.npos + P - 1) / P;
     if (nblk > 0x7fffffffLL || d.n_sets > 65535) return set_error(HY_ERR_UNSUPPORTED, "filter grid too large");
-    const size_t smem = sizeof(float) * (size_t)(2 * MAXW * TP + MAXW * WS);
+    const size_t smem = sizeof(float) * ((size_t)2 * p.ka * P + (size_t)2 * p.wbuf);
     cudaError_t e = cudaFuncSetAttribute(filter_gen_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return set_cuda_error("filter_gen smem attribute", e);
-    // split the last layer over grid z only as far as needed to fill the GPU
-    // (each split recomputes the hidden layers)
+    // split the last layer over grid z only when there are fewer CTAs than
+    // SMs (each split recomputes the hidden layers)
     const int nout = d.widths[d.n_layers];
     const int64_t base = nblk * d.n_sets;
     int sms = 148;
@@ -257,12 +374,13 @@ hy_status launch_filter_gen(const hy_filter_desc &d, float *h, cudaStream_t s) {
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     }
-    const int max_chunks = (nout + OC - 1) / OC;
-    int chunks = (int)((2 * (int64_t)sms + base - 1) / base);
-    if (chunks < 1) chunks = 1;
-    if (chunks > max_chunks) chunks = max_chunks;
-    p.out_chunk = ((nout + chunks - 1) / chunks + OC - 1) / OC * OC;
-    chunks = (nout + p.out_chunk - 1) / p.out_chunk;
+    const int ntile = (nout + OT_MAX - 1) / OT_MAX;
+    int chunks = 1;
+    if (base < (int64_t)sms) chunks = (int)((sms + base - 1) / base);
+    if (chunks > ntile) chunks = ntile;
+    const int per = (ntile + chunks - 1) / chunks;
+    p.out_chunk = per * OT_MAX;
+    chunks = (ntile + per - 1) / per;
     dim3 grid((unsigned)nblk, (unsigned)d.n_sets, (unsigned)chunks);
     filter_gen_kernel<<<grid, NT, smem, s>>>(p);
     return check_launch("filter_gen launch");

@@ -67,6 +67,7 @@ struct FsParams {
     const float2 *tw_2m;          // two-level W_{2M}
     int lo_2m;
     float2 *Hout;                 // spectrum mode: output bins (rows x (M+1))
+    int vec4;                     // rows of u, gates and y take 4-element vector accesses
 };
 
 // ----------------------------------------------------------------------------
@@ -94,13 +95,54 @@ __global__ void __launch_bounds__(NT) colpass_kernel(const FsParams p) {
     float2 *col = tile + warp * CS;
     float2 x[P];
 
+    // Each thread owns EIT groups of 4 consecutive real samples (2 complex
+    // points of neighbouring columns) in the first N2/2 rows.  Global loads
+    // are issued for all of a thread's groups before any of them is used.
+    constexpr int EIT = (N2 / 2) * (WARPS / 2) / NT;
+    static_assert(EIT * NT == (N2 / 2) * (WARPS / 2), "column tile does not divide evenly");
+    auto group_of = [&](int i, int &r, int &c2) {
+        const int e = tid + i * NT;
+        r = e / (WARPS / 2);
+        c2 = (e % (WARPS / 2)) * 2;
+    };
+    // 4 real samples at s0 of a row (zero past L)
+    auto load_row4 = [&](auto *src, int64_t s0, bool vec, auto loader1, auto loader4) {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (vec && s0 + 3 < L) {
+            v = loader4(src + s0);
+        } else {
+            if (s0 + 0 < L) v.x = loader1(src + s0 + 0);
+            if (s0 + 1 < L) v.y = loader1(src + s0 + 1);
+            if (s0 + 2 < L) v.z = loader1(src + s0 + 2);
+            if (s0 + 3 < L) v.w = loader1(src + s0 + 3);
+        }
+        return v;
+    };
+    auto io1 = [](const IO *q) { return IOT::load(q); };
+    auto io4 = [](const IO *q) { return IOT::load4(q); };
+    auto f1 = [](const float *q) { return __ldcg(q); };
+    auto f4 = [](const float *q) { return __ldcg(reinterpret_cast<const float4 *>(q)); };
+    auto h1 = [](const float *q) { return ldv(q); };
+    auto h4 = [](const float *q) { return ldv4(q); };
+
     if constexpr (INV) {
         // ---- load all N2 rows of the 8 columns (coalesced float4 = 2 complex)
-        for (int e = tid; e < N2 * (WARPS / 2); e += NT) {
-            const int r = e / (WARPS / 2), c2 = (e % (WARPS / 2)) * 2;
-            const float4 v = __ldcg(reinterpret_cast<const float4 *>(buf + n1_0 + c2 + (int64_t)N1 * r));
-            tile[c2 * CS + spad(r)] = make_float2(v.x, v.y);
-            tile[(c2 + 1) * CS + spad(r)] = make_float2(v.z, v.w);
+        {
+            constexpr int EL = N2 * (WARPS / 2) / NT;
+            float4 v[EL];
+#pragma unroll
+            for (int i = 0; i < EL; ++i) {
+                const int e = tid + i * NT;
+                const int r = e / (WARPS / 2), c2 = (e % (WARPS / 2)) * 2;
+                v[i] = __ldcg(reinterpret_cast<const float4 *>(buf + n1_0 + c2 + (int64_t)N1 * r));
+            }
+#pragma unroll
+            for (int i = 0; i < EL; ++i) {
+                const int e = tid + i * NT;
+                const int r = e / (WARPS / 2), c2 = (e % (WARPS / 2)) * 2;
+                tile[c2 * CS + spad(r)] = make_float2(v[i].x, v[i].y);
+                tile[(c2 + 1) * CS + spad(r)] = make_float2(v[i].z, v[i].w);
+            }
         }
         __syncthreads();
         load_own<LOG_N2, LP>(x, col, lane);
@@ -109,70 +151,92 @@ __global__ void __launch_bounds__(NT) colpass_kernel(const FsParams p) {
         // keep the first half (n2 < N2/2): samples 2m, 2m+1 with m < M/2
 #pragma unroll
         for (int m = 0; m < P / 2; ++m) col[spad(lane + 32 * m)] = x[m];
+        // ---- epilogue inputs (gate, skip source), all requested up front
+        const float dk = p.skip_k ? __ldg(p.skip_k + row % p.D) : 0.f;
+        const IO *g = reinterpret_cast<const IO *>(p.gate_k);
+        const IO *grow = g ? g + row * (int64_t)L : nullptr;
+        const IO *uin = reinterpret_cast<const IO *>(p.u) + row * (int64_t)L;
+        const bool vec = p.vec4 != 0;
+        float4 gv[EIT], pv[EIT];
+#pragma unroll
+        for (int i = 0; i < EIT; ++i) {
+            int r, c2;
+            group_of(i, r, c2);
+            const int64_t s0 = 2 * ((int64_t)n1_0 + c2 + (int64_t)N1 * r);
+            gv[i] = grow ? load_row4(grow, s0, vec, io1, io4) : make_float4(1.f, 1.f, 1.f, 1.f);
+            if (dk == 0.f) pv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            else if (p.k == 0) pv[i] = load_row4(uin, s0, vec, io1, io4);
+            else pv[i] = load_row4(stash, s0, true, f1, f4);
+        }
         __syncthreads();
         // ---- epilogue: 8 columns x N2/2 rows; each thread handles 2 complex
         //      = 4 consecutive real samples at 2*(n1_0 + c2 + N1*r)
-        const float dk = p.skip_k ? __ldg(p.skip_k + row % p.D) : 0.f;
-        const IO *g = reinterpret_cast<const IO *>(p.gate_k);
-        const IO *uin = reinterpret_cast<const IO *>(p.u) + row * (int64_t)L;
         const bool last = (p.k == p.K - 1);
         IO *yout = reinterpret_cast<IO *>(p.y) + row * (int64_t)L;
-        for (int e = tid; e < (N2 / 2) * (WARPS / 2); e += NT) {
-            const int r = e / (WARPS / 2), c2 = (e % (WARPS / 2)) * 2;
+#pragma unroll
+        for (int i = 0; i < EIT; ++i) {
+            int r, c2;
+            group_of(i, r, c2);
             const int64_t s0 = 2 * ((int64_t)n1_0 + c2 + (int64_t)N1 * r);   // first real sample
-            float2 a = tile[c2 * CS + spad(r)], b = tile[(c2 + 1) * CS + spad(r)];
-            float v[4] = {a.x * p.scale, a.y * p.scale, b.x * p.scale, b.y * p.scale};
-            float pv[4] = {0.f, 0.f, 0.f, 0.f}, gv[4] = {1.f, 1.f, 1.f, 1.f};
-            if (dk != 0.f) {
-                if (p.k == 0) {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        if (s0 + q < L) pv[q] = IOT::load(uin + s0 + q);
-                } else {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        if (s0 + q < L) pv[q] = __ldcg(stash + s0 + q);
-                }
-            }
-            if (g) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    if (s0 + q < L) gv[q] = IOT::load(g + row * (int64_t)L + s0 + q);
-            }
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                v[q] = gv[q] * fmaf(dk, pv[q], v[q]);
-                if (s0 + q >= L) v[q] = 0.f;
-            }
+            const float2 a = tile[c2 * CS + spad(r)], b = tile[(c2 + 1) * CS + spad(r)];
+            const float sc = p.scale;
+            float4 v = make_float4(gv[i].x * fmaf(dk, pv[i].x, a.x * sc), gv[i].y * fmaf(dk, pv[i].y, a.y * sc),
+                                   gv[i].z * fmaf(dk, pv[i].z, b.x * sc), gv[i].w * fmaf(dk, pv[i].w, b.y * sc));
+            if (s0 + 0 >= L) v.x = 0.f;
+            if (s0 + 1 >= L) v.y = 0.f;
+            if (s0 + 2 >= L) v.z = 0.f;
+            if (s0 + 3 >= L) v.w = 0.f;
+            const bool full = s0 + 3 < L;
             if (last) {
+                if (vec && full) {
+                    IOT::store4(yout + s0, v);
+                } else {
+                    const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    if (s0 + q < L) IOT::store(yout + s0 + q, v[q]);
+                    for (int q = 0; q < 4; ++q)
+                        if (s0 + q < L) IOT::store(yout + s0 + q, vv[q]);
+                }
             } else {
+                if (full) {
+                    __stcg(reinterpret_cast<float4 *>(stash + s0), v);
+                } else {
+                    const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    if (s0 + q < L) __stcg(stash + s0 + q, v[q]);
-                tile[c2 * CS + spad(r)] = make_float2(v[0], v[1]);
-                tile[(c2 + 1) * CS + spad(r)] = make_float2(v[2], v[3]);
+                    for (int q = 0; q < 4; ++q)
+                        if (s0 + q < L) __stcg(stash + s0 + q, vv[q]);
+                }
+                tile[c2 * CS + spad(r)] = make_float2(v.x, v.y);
+                tile[(c2 + 1) * CS + spad(r)] = make_float2(v.z, v.w);
             }
         }
         if (last || !FWD) return;
         __syncthreads();
     } else {
         // ---- first order: packed input rows n2 < N2/2 of the 8 columns
-        const float *hin = reinterpret_cast<const float *>(p.u);
-        const IO *uin = reinterpret_cast<const IO *>(p.u) + row * (int64_t)L;
-        for (int e = tid; e < (N2 / 2) * (WARPS / 2); e += NT) {
-            const int r = e / (WARPS / 2), c2 = (e % (WARPS / 2)) * 2;
-            const int64_t s0 = 2 * ((int64_t)n1_0 + c2 + (int64_t)N1 * r);
-            float v[4];
+        float4 v[EIT];
+        if constexpr (SPEC_INPUT) {
+            const float *hin = reinterpret_cast<const float *>(p.u) + row * (int64_t)L;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                if constexpr (SPEC_INPUT) v[q] = (s0 + q < L) ? __ldg(hin + row * (int64_t)L + s0 + q) : 0.f;
-                else v[q] = (s0 + q < L) ? IOT::load(uin + s0 + q) : 0.f;
+            for (int i = 0; i < EIT; ++i) {
+                int r, c2;
+                group_of(i, r, c2);
+                v[i] = load_row4(hin, 2 * ((int64_t)n1_0 + c2 + (int64_t)N1 * r), p.vec4 != 0, h1, h4);
             }
-            tile[c2 * CS + spad(r)] = make_float2(v[0], v[1]);
-            tile[(c2 + 1) * CS + spad(r)] = make_float2(v[2], v[3]);
+        } else {
+            const IO *uin = reinterpret_cast<const IO *>(p.u) + row * (int64_t)L;
+#pragma unroll
+            for (int i = 0; i < EIT; ++i) {
+                int r, c2;
+                group_of(i, r, c2);
+                v[i] = load_row4(uin, 2 * ((int64_t)n1_0 + c2 + (int64_t)N1 * r), p.vec4 != 0, io1, io4);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < EIT; ++i) {
+            int r, c2;
+            group_of(i, r, c2);
+            tile[c2 * CS + spad(r)] = make_float2(v[i].x, v[i].y);
+            tile[(c2 + 1) * CS + spad(r)] = make_float2(v[i].z, v[i].w);
         }
         __syncthreads();
     }
@@ -201,18 +265,47 @@ __global__ void __launch_bounds__(NT) colpass_kernel(const FsParams p) {
 // Row pass (B): 8 rows per CTA -- 4 low rows k2 and their mirrors N2 - k2
 // (group 0: rows 0..3, N2/2, N2-1..N2-3).  SPEC: write the half spectrum of
 // the rows instead of multiplying (long filter spectra).
+//
+// The bins of row k2 are k2 + N2*k1: one row alone touches one 8-byte value
+// per 32-byte sector of a natural-order spectrum.  The CTA's low rows are 4
+// consecutive k2 (and the mirrors 4 consecutive N2 - k2), so the spectrum
+// reads are staged in shared memory by all 256 threads with 4 neighbouring
+// lanes on 4 neighbouring bins (cp.async, double-buffered over 4 batches of
+// k1), and the SPEC outputs are collected in the row buffers and written 8
+// rows x 1 k1 per 8 lanes.
 // ----------------------------------------------------------------------------
 enum { OWN_ALL = 0, OWN_NONE = 1, OWN_SELF0 = 2, OWN_SELFH = 3 };
 
+constexpr int RP_BATCHES = 4;   // k1 batches of the spectrum staging
+
+__device__ __forceinline__ void cpa8(void *smem, const void *g) {
+    const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(sa), "l"(g) : "memory");
+}
+__device__ __forceinline__ void cpa_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cpa_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <int LOG_N1, bool SPEC>
+__host__ __device__ constexpr size_t rowpass_smem_bytes() {
+    // row buffers, then (conv) two staging buffers of [low/high][4 rows][N1/4 k1]
+    return sizeof(float2) * ((size_t)WARPS * spad_size(1 << LOG_N1) +
+                             (SPEC ? 0 : (size_t)2 * 2 * 4 * ((1 << LOG_N1) / RP_BATCHES)));
+}
+
 template <int LOG_N1, int LOG_N2, bool SPEC>
-__global__ void __launch_bounds__(NT) rowpass_kernel(const FsParams p) {
+__global__ void __launch_bounds__(NT, 2) rowpass_kernel(const FsParams p) {
     constexpr int N1 = 1 << LOG_N1;
     constexpr int N2 = 1 << LOG_N2;
     constexpr int M = N1 * N2;
     constexpr int LP = fs_log_p(LOG_N1);
     constexpr int P = 1 << LP;
     constexpr int RS = spad_size(N1);
-    extern __shared__ float2 rows_s[];        // WARPS rows x RS
+    constexpr int MB = P / RP_BATCHES;        // m values per staging batch
+    constexpr int BK = 32 * MB;               // k1 values per staging batch
+    static_assert(MB >= 1, "row too short for the staging batches");
+    extern __shared__ float2 rows_s[];        // WARPS rows x RS, then the staging buffers
+    float2 *hstage = rows_s + WARPS * RS;     // [2 buffers][2 low/high][4][BK]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = blockIdx.x;
     const int64_t row = p.row0 + blockIdx.y;
@@ -232,6 +325,31 @@ __global__ void __launch_bounds__(NT) rowpass_kernel(const FsParams p) {
     float2 *own = rows_s + warp * RS;
     float2 *oth = rows_s + partner * RS;
 
+    const int64_t d = row % p.D;
+    const float2 *H = SPEC ? nullptr : p.spec + d * (int64_t)(M + 1);
+    float2 *Ho = SPEC ? p.Hout + row * (int64_t)(M + 1) : nullptr;
+
+    // staging of batch b: [lh][j][kk] = H[k] (lh = 0) or H[M - k] (lh = 1)
+    // with k = 4g + j + N2 (b BK + kk), for the low rows j = 0..3
+    const uint32_t k_st = (uint32_t)(4 * g + (tid & 3)) + (uint32_t)N2 * (uint32_t)(tid >> 2);
+    const float2 *h_lo = SPEC ? nullptr : H + k_st;             // H[k], k = k_st + N2 * (b BK + i NT/4)
+    const float2 *h_hi = SPEC ? nullptr : H + (M - k_st);       // H[M - k]
+    const int s_off = (tid & 3) * BK + (tid >> 2);
+    auto stage = [&](int b, float2 *dst) {
+#pragma unroll
+        for (int i = 0; i < (BK + NT / 4 - 1) / (NT / 4); ++i) {
+            if ((tid >> 2) + i * (NT / 4) < BK) {
+                const int off = N2 * (b * BK + i * (NT / 4));
+                cpa8(dst + s_off + i * (NT / 4), h_lo + off);
+                cpa8(dst + 4 * BK + s_off + i * (NT / 4), h_hi - off);
+            }
+        }
+    };
+    if constexpr (!SPEC) {
+        stage(0, hstage);
+        cpa_commit();
+    }
+
     // ---- load the row (contiguous) and forward FFT over n1 -> bins k2 + N2 k1
     float2 x[P];
     const float2 *src = buf + (int64_t)N1 * k2;
@@ -242,60 +360,93 @@ __global__ void __launch_bounds__(NT) rowpass_kernel(const FsParams p) {
     for (int m = 0; m < P; ++m) own[spad(lane + 32 * m)] = x[m];
     __syncthreads();
 
-    const int64_t d = row % p.D;
-    const float2 *H = SPEC ? nullptr : p.spec + d * (int64_t)(M + 1);
-    float2 *Ho = SPEC ? p.Hout + row * (int64_t)(M + 1) : nullptr;
-
     // element (own k1) pairs with partner element pk1 of row partner_k2
 #pragma unroll
-    for (int m = 0; m < P; ++m) {
-        const int k1 = lane + 32 * m;
-        bool owner;
-        int pk1;
-        if (mode == OWN_ALL) { owner = true; pk1 = N1 - 1 - k1; }
-        else if (mode == OWN_NONE) { owner = false; pk1 = 0; }
-        else if (mode == OWN_SELF0) { owner = k1 < N1 / 2; pk1 = (N1 - k1) & (N1 - 1); }
-        else { owner = k1 < N1 / 2; pk1 = N1 - 1 - k1; }
-        if (!owner) continue;
-        const uint32_t k = (uint32_t)k2 + (uint32_t)N2 * k1;
-        const float2 zk = x[m];
-        if (mode == OWN_SELF0 && k1 == 0) {
-            // DC (bin 0) and Nyquist (bin M): both real
-            if constexpr (SPEC) {
-                Ho[0] = make_float2(zk.x + zk.y, 0.f);
-                Ho[M] = make_float2(zk.x - zk.y, 0.f);
+    for (int b = 0; b < RP_BATCHES; ++b) {
+        const float2 *hs = hstage + (b & 1) * (8 * BK);
+        if constexpr (!SPEC) {
+            if (b + 1 < RP_BATCHES) {
+                stage(b + 1, hstage + ((b + 1) & 1) * (8 * BK));
+                cpa_commit();
+                cpa_wait<1>();
             } else {
-                const float y0 = 2.f * (zk.x + zk.y) * __ldg(&H[0].x);
-                const float yM = 2.f * (zk.x - zk.y) * __ldg(&H[M].x);
-                x[m] = make_float2(y0 + yM, y0 - yM);
+                cpa_wait<0>();
             }
-            continue;
+            __syncthreads();
         }
-        const float2 zn = oth[spad(pk1)];
-        const float2 A = make_float2(zk.x + zn.x, zk.y - zn.y);
-        const float2 Bv = make_float2(zk.x - zn.x, zk.y + zn.y);
-        const float2 w = tw2(p.tw_2m, p.lo_2m, k);                   // W_{2M}^k
-        const float2 wB = cmul(Bv, w);
-        const float2 C = make_float2(wB.y, -wB.x);
-        const float2 Xk = cadd(A, C);                                 // 2 X[k]
-        const float2 Xn = cconj(csub(A, C));                          // 2 X[M-k]
-        if constexpr (SPEC) {
-            Ho[k] = make_float2(0.5f * Xk.x, 0.5f * Xk.y);
-            Ho[M - k] = make_float2(0.5f * Xn.x, 0.5f * Xn.y);
-        } else {
-            const float2 Yk = cmul(Xk, __ldg(H + k));
-            const float2 Yn = cmul(Xn, __ldg(H + (M - k)));
-            const float2 A2 = make_float2(Yk.x + Yn.x, Yk.y - Yn.y);
-            const float2 B2 = make_float2(Yk.x - Yn.x, Yk.y + Yn.y);
-            const float2 cB = cmulc(B2, w);
-            const float2 C2 = make_float2(-cB.y, cB.x);
-            x[m] = cadd(A2, C2);
-            oth[spad(pk1)] = cconj(csub(A2, C2));
+#pragma unroll
+        for (int mm = 0; mm < MB; ++mm) {
+            const int m = b * MB + mm;
+            const int k1 = lane + 32 * m;
+            bool owner;
+            int pk1;
+            if (mode == OWN_ALL) { owner = true; pk1 = N1 - 1 - k1; }
+            else if (mode == OWN_NONE) { owner = false; pk1 = 0; }
+            else if (mode == OWN_SELF0) { owner = k1 < N1 / 2; pk1 = (N1 - k1) & (N1 - 1); }
+            else { owner = k1 < N1 / 2; pk1 = N1 - 1 - k1; }
+            if (!owner) continue;
+            const uint32_t k = (uint32_t)k2 + (uint32_t)N2 * k1;
+            const float2 zk = x[m];
+            // spectrum bins k and M - k: staged for warps 0..3, direct for row N2/2
+            float2 hk = make_float2(0.f, 0.f), hn = make_float2(0.f, 0.f);
+            if constexpr (!SPEC) {
+                if (warp < 4) {
+                    hk = hs[warp * BK + lane + 32 * mm];
+                    hn = hs[(4 + warp) * BK + lane + 32 * mm];
+                } else {
+                    hk = __ldg(H + k);
+                    hn = __ldg(H + (M - k));
+                }
+            }
+            if (mode == OWN_SELF0 && k1 == 0) {
+                // DC (bin 0) and Nyquist (bin M): both real
+                if constexpr (SPEC) {
+                    own[spad(0)] = make_float2(zk.x + zk.y, 0.f);
+                    Ho[M] = make_float2(zk.x - zk.y, 0.f);
+                } else {
+                    const float y0 = 2.f * (zk.x + zk.y) * hk.x;
+                    const float yM = 2.f * (zk.x - zk.y) * hn.x;
+                    x[m] = make_float2(y0 + yM, y0 - yM);
+                }
+                continue;
+            }
+            const float2 zn = oth[spad(pk1)];
+            const float2 A = make_float2(zk.x + zn.x, zk.y - zn.y);
+            const float2 Bv = make_float2(zk.x - zn.x, zk.y + zn.y);
+            const float2 w = tw2(p.tw_2m, p.lo_2m, k);                   // W_{2M}^k
+            const float2 wB = cmul(Bv, w);
+            const float2 C = make_float2(wB.y, -wB.x);
+            const float2 Xk = cadd(A, C);                                 // 2 X[k]
+            const float2 Xn = cconj(csub(A, C));                          // 2 X[M-k]
+            if constexpr (SPEC) {
+                own[spad(k1)] = make_float2(0.5f * Xk.x, 0.5f * Xk.y);
+                oth[spad(pk1)] = make_float2(0.5f * Xn.x, 0.5f * Xn.y);
+            } else {
+                const float2 Yk = cmul(Xk, hk);
+                const float2 Yn = cmul(Xn, hn);
+                const float2 A2 = make_float2(Yk.x + Yn.x, Yk.y - Yn.y);
+                const float2 B2 = make_float2(Yk.x - Yn.x, Yk.y + Yn.y);
+                const float2 cB = cmulc(B2, w);
+                const float2 C2 = make_float2(-cB.y, cB.x);
+                x[m] = cadd(A2, C2);
+                oth[spad(pk1)] = cconj(csub(A2, C2));
+            }
         }
+        if constexpr (!SPEC) __syncthreads();   // staging buffer b & 1 is refilled next
     }
     if constexpr (SPEC) {
         // bin M/2 (row 0, k1 = N1/2) pairs with itself: X[M/2] = conj(Z[M/2])
-        if (mode == OWN_SELF0 && lane == 0) Ho[M / 2] = cconj(x[(N1 / 2) / 32]);
+        if (mode == OWN_SELF0 && lane == 0) own[spad(N1 / 2)] = cconj(x[(N1 / 2) / 32]);
+        __syncthreads();
+        // rows_s[w][k1] now holds bin k2_w + N2 k1 of every row of the CTA;
+        // 8 lanes store the 8 rows' bins of one k1
+        const int w = tid & 7;
+        int kw;
+        if (w < 4) kw = 4 * g + w;
+        else kw = (g == 0 && w == 4) ? N2 / 2 : N2 - (4 * g + w - 4);
+#pragma unroll 4
+        for (int k1 = tid >> 3; k1 < N1; k1 += NT / 8)
+            Ho[(uint32_t)kw + (uint32_t)N2 * (uint32_t)k1] = rows_s[w * RS + spad(k1)];
         return;
     }
     // self-paired element of row 0: bin M/2 (k1 = N1/2)
@@ -332,6 +483,15 @@ int64_t chunk_rows_of(int64_t rows, int log_mc) {
     return c < rows ? c : rows;
 }
 
+// Every row start of u, the gates and y is aligned for 4-element vectors.
+bool vec4_rows(const LongConvArgs &a, size_t el) {
+    const uintptr_t al = 4 * el;
+    if (a.L % 4 != 0 || (uintptr_t)a.u % al || (uintptr_t)a.y % al) return false;
+    for (int k = 0; k < a.K; ++k)
+        if (a.gate[k] && (uintptr_t)a.gate[k] % al) return false;
+    return true;
+}
+
 template <typename Kern>
 hy_status smem_attr(Kern k, size_t bytes) {
     if (bytes > 48 * 1024) {
@@ -356,6 +516,7 @@ hy_status run_conv(const LongConvArgs &a, cudaStream_t s) {
     p.buf = reinterpret_cast<float2 *>(a.ws);
     p.stash = reinterpret_cast<float *>(reinterpret_cast<char *>(a.ws) + (size_t)cr * ((size_t)8 << LOG_MC));
     p.scale = (float)(1.0 / (4.0 * (double)((int64_t)1 << LOG_MC)));
+    p.vec4 = vec4_rows(a, sizeof(IO));
     p.tw_n1 = tw_stages(LOG_N1, fs_log_p(LOG_N1));
     p.tw_n2 = tw_stages(LOG_N2, fs_log_p(LOG_N2));
     p.lo_m = LOG_MC / 2;
@@ -364,7 +525,7 @@ hy_status run_conv(const LongConvArgs &a, cudaStream_t s) {
     p.tw_2m = tw_pow2(LOG_MC + 1, p.lo_2m);
     if (!p.tw_n1 || !p.tw_n2 || !p.tw_m || !p.tw_2m) return set_error(HY_ERR_CUDA, "multi-pass twiddle tables missing");
     const size_t smem_c = sizeof(float2) * WARPS * spad_size(N2);
-    const size_t smem_r = sizeof(float2) * WARPS * spad_size(N1);
+    const size_t smem_r = rowpass_smem_bytes<LOG_N1, false>();
     auto kA = colpass_kernel<LOG_N1, LOG_N2, IO, false, true, false>;
     auto kCA = colpass_kernel<LOG_N1, LOG_N2, IO, true, true, false>;
     auto kC = colpass_kernel<LOG_N1, LOG_N2, IO, true, false, false>;
@@ -406,6 +567,7 @@ hy_status run_spectrum(int64_t rows, int64_t L, const float *h, float2 *H, void 
     p.buf = reinterpret_cast<float2 *>(ws);
     p.stash = nullptr;
     p.Hout = H;
+    p.vec4 = L % 4 == 0 && (uintptr_t)h % 16 == 0;
     p.tw_n1 = tw_stages(LOG_N1, fs_log_p(LOG_N1));
     p.tw_n2 = tw_stages(LOG_N2, fs_log_p(LOG_N2));
     p.lo_m = LOG_MC / 2;
@@ -414,7 +576,7 @@ hy_status run_spectrum(int64_t rows, int64_t L, const float *h, float2 *H, void 
     p.tw_2m = tw_pow2(LOG_MC + 1, p.lo_2m);
     if (!p.tw_n1 || !p.tw_n2 || !p.tw_m || !p.tw_2m) return set_error(HY_ERR_CUDA, "multi-pass twiddle tables missing");
     const size_t smem_c = sizeof(float2) * WARPS * spad_size(N2);
-    const size_t smem_r = sizeof(float2) * WARPS * spad_size(N1);
+    const size_t smem_r = rowpass_smem_bytes<LOG_N1, true>();
     auto kA = colpass_kernel<LOG_N1, LOG_N2, float, false, true, true>;
     auto kB = rowpass_kernel<LOG_N1, LOG_N2, true>;
     hy_status st;
@@ -525,6 +687,7 @@ hy_status run_conv_static(const LongConvArgs &a, void *scratch, cudaStream_t s) 
     p.buf = reinterpret_cast<float2 *>(scratch);
     p.stash = reinterpret_cast<float *>(reinterpret_cast<char *>(scratch) + (size_t)cr * ((size_t)8 << LOG_MC));
     p.scale = (float)(1.0 / (4.0 * (double)((int64_t)1 << LOG_MC)));
+    p.vec4 = vec4_rows(a, sizeof(IO));
     p.tw_n1 = tw_stages(LOG_N1, fs_log_p(LOG_N1));
     p.tw_n2 = tw_stages(LOG_N2, fs_log_p(LOG_N2));
     p.lo_m = LOG_MC / 2;
@@ -533,7 +696,7 @@ hy_status run_conv_static(const LongConvArgs &a, void *scratch, cudaStream_t s) 
     p.tw_2m = tw_pow2(LOG_MC + 1, p.lo_2m);
     if (!p.tw_n1 || !p.tw_n2 || !p.tw_m || !p.tw_2m) return set_error(HY_ERR_CUDA, "multi-pass twiddle tables missing");
     const size_t smem_c = sizeof(float2) * WARPS * spad_size(N2);
-    const size_t smem_r = sizeof(float2) * WARPS * spad_size(N1);
+    const size_t smem_r = rowpass_smem_bytes<LOG_N1, false>();
     auto kA = colpass_kernel<LOG_N1, LOG_N2, IO, false, true, false>;
     auto kCA = colpass_kernel<LOG_N1, LOG_N2, IO, true, true, false>;
     auto kC = colpass_kernel<LOG_N1, LOG_N2, IO, true, false, false>;

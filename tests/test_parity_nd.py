@@ -110,6 +110,33 @@ def test_nd_filter_gen_3d_vs_oracle():
         check(got[b].reshape(6, -1), ref.T, "f32", "3-D filters sample %d" % b)
 
 
+@pytest.mark.parametrize("g,circular,hidden,nout", [(2, True, [16], 5), (2, False, [24, 12], 3), (4, True, [64], 130)])
+def test_nd_filter_gen_small_grids(g, circular, hidden, nout):
+    """Grids smaller than one 64-position tile, several hidden layers and a
+    last layer wider than one 128-output tile, with FiLM on two sets."""
+    F = 3
+    rng = np.random.default_rng(g * 100 + nout)
+    widths = [6 * F] + hidden + [nout]
+    Ws, bs = [], []
+    for a, b in zip(widths[:-1], widths[1:]):
+        Ws.append(rng.uniform(-1 / np.sqrt(a), 1 / np.sqrt(a), (b, a)).astype(np.float32))
+        bs.append(rng.uniform(-1 / np.sqrt(a), 1 / np.sqrt(a), b).astype(np.float32))
+    alpha = rng.uniform(0.5, 3.0, nout).astype(np.float32)
+    gam = rng.normal(0, 0.1, (2, hidden[0])).astype(np.float32)
+    bet = rng.normal(0, 0.1, (2, hidden[0])).astype(np.float32)
+    S = g if circular else 2 * g
+    h = torch.empty((2, nout, S, S, S), device="cuda")
+    hy.hyena_filter_gen(h, ndim=3, grid=g, circular=circular, Ws=[f32_dev(a) for a in Ws],
+                        bs=[f32_dev(a) for a in bs], alpha=f32_dev(alpha), n_freq=F,
+                        film_gamma=f32_dev(gam), film_beta=f32_dev(bet), n_sets=2)
+    torch.cuda.synchronize()
+    got = to_np(h)
+    idx = np.arange(S ** 3)
+    for b in range(2):
+        ref = oracle.filter_gen_3d_points(g, circular, F, Ws, bs, gam[b], bet[b], alpha, idx)
+        check(got[b].reshape(nout, -1), ref.T, "f32", "3-D filters g%d circ%d set %d" % (g, circular, b))
+
+
 def test_c4_full_size():
     """Workload 4 at full size: per-sample FiLM filters on the 128^3 transform
     grid, their spectra and the gated convolution of B2 D128 64^3.  Four slabs

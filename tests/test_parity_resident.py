@@ -121,6 +121,38 @@ def test_filter_gen_1d_vs_oracle():
         check(to_np(h), ref, "f32", "filter_gen %s" % name)
 
 
+def _mlp(rng, widths):
+    Ws, bs = [], []
+    for a, b in zip(widths[:-1], widths[1:]):
+        lim = 1.0 / np.sqrt(a)
+        Ws.append(rng.uniform(-lim, lim, (b, a)).astype(np.float32))
+        bs.append(rng.uniform(-lim, lim, b).astype(np.float32))
+    return Ws, bs
+
+
+@pytest.mark.parametrize("L,F,include_t,hidden,nout,offset", [
+    (1, 2, True, [8], 3, 0),                 # one position
+    (777, 3, True, [33], 130, 0),            # ragged length, odd widths, two last-layer tiles
+    (1000, 5, False, [100, 20, 7], 300, 1),  # four layers, misaligned output rows
+    (4096, 16, True, [], 64, 0),             # single layer (encoding -> output)
+    (3000, 64, True, [128], 40, 0),          # widest encoding (129) and hidden (128)
+])
+def test_filter_gen_1d_shapes(L, F, include_t, hidden, nout, offset):
+    rng = np.random.default_rng(L + nout)
+    w0 = int(include_t) + 2 * F
+    Ws, bs = _mlp(rng, [w0] + hidden + [nout])
+    alpha = rng.uniform(0.1, 4.0, nout).astype(np.float32)
+    flat = torch.full((nout * L + offset,), float("nan"), device="cuda")
+    h = flat[offset:].view(nout, L)
+    hy.hyena_filter_gen(h, ndim=1, L=L, Ws=[f32_dev(a) for a in Ws], bs=[f32_dev(a) for a in bs],
+                        alpha=f32_dev(alpha), n_freq=F, include_t=include_t)
+    torch.cuda.synchronize()
+    ref = oracle.filter_gen_1d(L, F, include_t, Ws, bs, alpha)
+    check(to_np(h), ref, "f32", "filter_gen L%d widths %s" % (L, [w0] + hidden + [nout]))
+    if offset:
+        assert np.isnan(to_np(flat[:offset])).all()
+
+
 def test_c1_end_to_end():
     """Workload 1 exactly: MLP parameters -> filters -> spectra -> operator."""
     w = hw.make("c1")

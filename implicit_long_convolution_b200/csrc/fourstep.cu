@@ -266,17 +266,21 @@ __global__ void __launch_bounds__(NT) colpass_kernel(const FsParams p) {
 // (group 0: rows 0..3, N2/2, N2-1..N2-3).  SPEC: write the half spectrum of
 // the rows instead of multiplying (long filter spectra).
 //
-// The bins of row k2 are k2 + N2*k1: one row alone touches one 8-byte value
-// per 32-byte sector of a natural-order spectrum.  The CTA's low rows are 4
-// consecutive k2 (and the mirrors 4 consecutive N2 - k2), so the spectrum
-// reads are staged in shared memory by all 256 threads with 4 neighbouring
-// lanes on 4 neighbouring bins (cp.async, double-buffered over 4 batches of
-// k1), and the SPEC outputs are collected in the row buffers and written 8
-// rows x 1 k1 per 8 lanes.
+// Bin k = k2 + N2 k1 of a low row pairs with bin M - k = (N2 - k2) + N2 (N1 -
+// 1 - k1) of its mirror row, so every warp takes the pairs of its own bins
+// k1 < N1/2 (partner values read from the mirror row in shared memory); rows
+// 0 and N2/2 pair with themselves.
+//
+// One row alone touches one 8-byte value per 32-byte sector of a natural-
+// order spectrum.  The CTA's rows come in runs of 4 consecutive k2, so the
+// spectrum bins are staged in shared memory by all 256 threads with 4
+// neighbouring lanes on 4 neighbouring bins (cp.async, double-buffered over
+// batches of k1), and the SPEC outputs are collected in the row buffers and
+// written 8 rows x 1 k1 per 8 lanes.
 // ----------------------------------------------------------------------------
-enum { OWN_ALL = 0, OWN_NONE = 1, OWN_SELF0 = 2, OWN_SELFH = 3 };
+enum { PAIR = 0, SELF0 = 1, SELFH = 2 };
 
-constexpr int RP_BATCHES = 4;   // k1 batches of the spectrum staging
+__host__ __device__ constexpr int rp_batches(int log_n1) { return (1 << log_n1) / 64 >= 4 ? 4 : (1 << log_n1) / 64; }
 
 __device__ __forceinline__ void cpa8(void *smem, const void *g) {
     const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
@@ -288,9 +292,9 @@ __device__ __forceinline__ void cpa_wait() { asm volatile("cp.async.wait_group %
 
 template <int LOG_N1, bool SPEC>
 __host__ __device__ constexpr size_t rowpass_smem_bytes() {
-    // row buffers, then (conv) two staging buffers of [low/high][4 rows][N1/4 k1]
+    // row buffers, then (conv) two staging buffers of [8 rows][k, M-k][N1/2 / batches]
     return sizeof(float2) * ((size_t)WARPS * spad_size(1 << LOG_N1) +
-                             (SPEC ? 0 : (size_t)2 * 2 * 4 * ((1 << LOG_N1) / RP_BATCHES)));
+                             (SPEC ? 0 : (size_t)2 * WARPS * 2 * ((1 << LOG_N1) / 2 / rp_batches(LOG_N1))));
 }
 
 template <int LOG_N1, int LOG_N2, bool SPEC>
@@ -301,27 +305,26 @@ __global__ void __launch_bounds__(NT, 2) rowpass_kernel(const FsParams p) {
     constexpr int LP = fs_log_p(LOG_N1);
     constexpr int P = 1 << LP;
     constexpr int RS = spad_size(N1);
-    constexpr int MB = P / RP_BATCHES;        // m values per staging batch
-    constexpr int BK = 32 * MB;               // k1 values per staging batch
-    static_assert(MB >= 1, "row too short for the staging batches");
+    constexpr int NB = rp_batches(LOG_N1);    // staging batches over the owned k1 < N1/2
+    constexpr int MB = P / 2 / NB;            // m values per batch
+    constexpr int BK = 32 * MB;               // k1 values per batch
+    static_assert(NB >= 1 && MB >= 1 && MB * NB * 2 == P, "row pass batching");
     extern __shared__ float2 rows_s[];        // WARPS rows x RS, then the staging buffers
-    float2 *hstage = rows_s + WARPS * RS;     // [2 buffers][2 low/high][4][BK]
+    float2 *hstage = rows_s + WARPS * RS;     // [2 buffers][8 rows][k, M-k][BK]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = blockIdx.x;
     const int64_t row = p.row0 + blockIdx.y;
     const int64_t rl = blockIdx.y;
     float2 *buf = p.buf + rl * (int64_t)M;
 
-    // rows of this CTA and the pairing of warp w
-    int k2, partner, mode;
-    if (warp < 4) {
-        k2 = 4 * g + warp;
-        if (g == 0 && warp == 0) { mode = OWN_SELF0; partner = warp; }
-        else { mode = OWN_ALL; partner = warp + 4; }
-    } else {
-        if (g == 0 && warp == 4) { k2 = N2 / 2; mode = OWN_SELFH; partner = warp; }
-        else { k2 = N2 - (4 * g + warp - 4); mode = OWN_NONE; partner = warp - 4; }
-    }
+    // row of warp w (w < 4: low rows, w >= 4: their mirrors)
+    auto row_k2 = [&](int w) {
+        if (w < 4) return 4 * g + w;
+        return (g == 0 && w == 4) ? N2 / 2 : N2 - (4 * g + w - 4);
+    };
+    const int k2 = row_k2(warp);
+    const int mode = (g == 0 && warp == 0) ? SELF0 : ((g == 0 && warp == 4) ? SELFH : PAIR);
+    const int partner = mode == PAIR ? (warp ^ 4) : warp;
     float2 *own = rows_s + warp * RS;
     float2 *oth = rows_s + partner * RS;
 
@@ -329,19 +332,21 @@ __global__ void __launch_bounds__(NT, 2) rowpass_kernel(const FsParams p) {
     const float2 *H = SPEC ? nullptr : p.spec + d * (int64_t)(M + 1);
     float2 *Ho = SPEC ? p.Hout + row * (int64_t)(M + 1) : nullptr;
 
-    // staging of batch b: [lh][j][kk] = H[k] (lh = 0) or H[M - k] (lh = 1)
-    // with k = 4g + j + N2 (b BK + kk), for the low rows j = 0..3
-    const uint32_t k_st = (uint32_t)(4 * g + (tid & 3)) + (uint32_t)N2 * (uint32_t)(tid >> 2);
-    const float2 *h_lo = SPEC ? nullptr : H + k_st;             // H[k], k = k_st + N2 * (b BK + i NT/4)
-    const float2 *h_hi = SPEC ? nullptr : H + (M - k_st);       // H[M - k]
-    const int s_off = (tid & 3) * BK + (tid >> 2);
+    // staging of batch b: [w][0][kk] = H[k], [w][1][kk] = H[M - k] with
+    // k = k2_w + N2 (b BK + kk); thread: rows j and 4 + j, kk = tid/4 + 64 i
+    const int sj = tid & 3, skk = tid >> 2;
+    const uint32_t k_lo = (uint32_t)row_k2(sj) + (uint32_t)N2 * (uint32_t)skk;
+    const uint32_t k_hi = (uint32_t)row_k2(4 + sj) + (uint32_t)N2 * (uint32_t)skk;
     auto stage = [&](int b, float2 *dst) {
 #pragma unroll
         for (int i = 0; i < (BK + NT / 4 - 1) / (NT / 4); ++i) {
-            if ((tid >> 2) + i * (NT / 4) < BK) {
-                const int off = N2 * (b * BK + i * (NT / 4));
-                cpa8(dst + s_off + i * (NT / 4), h_lo + off);
-                cpa8(dst + 4 * BK + s_off + i * (NT / 4), h_hi - off);
+            const int kk = skk + i * (NT / 4);
+            if (kk < BK) {
+                const uint32_t off = (uint32_t)N2 * (uint32_t)(b * BK + i * (NT / 4));
+                cpa8(dst + (2 * sj + 0) * BK + kk, H + (k_lo + off));
+                cpa8(dst + (2 * sj + 1) * BK + kk, H + (M - (k_lo + off)));
+                cpa8(dst + (2 * (4 + sj) + 0) * BK + kk, H + (k_hi + off));
+                cpa8(dst + (2 * (4 + sj) + 1) * BK + kk, H + (M - (k_hi + off)));
             }
         }
     };
@@ -360,13 +365,13 @@ __global__ void __launch_bounds__(NT, 2) rowpass_kernel(const FsParams p) {
     for (int m = 0; m < P; ++m) own[spad(lane + 32 * m)] = x[m];
     __syncthreads();
 
-    // element (own k1) pairs with partner element pk1 of row partner_k2
+    // ---- pairs of the owned bins k1 = lane + 32 m < N1/2 (m < P/2)
 #pragma unroll
-    for (int b = 0; b < RP_BATCHES; ++b) {
-        const float2 *hs = hstage + (b & 1) * (8 * BK);
+    for (int b = 0; b < NB; ++b) {
+        const float2 *hs = hstage + (b & 1) * (WARPS * 2 * BK);
         if constexpr (!SPEC) {
-            if (b + 1 < RP_BATCHES) {
-                stage(b + 1, hstage + ((b + 1) & 1) * (8 * BK));
+            if (b + 1 < NB) {
+                stage(b + 1, hstage + ((b + 1) & 1) * (WARPS * 2 * BK));
                 cpa_commit();
                 cpa_wait<1>();
             } else {
@@ -378,27 +383,15 @@ __global__ void __launch_bounds__(NT, 2) rowpass_kernel(const FsParams p) {
         for (int mm = 0; mm < MB; ++mm) {
             const int m = b * MB + mm;
             const int k1 = lane + 32 * m;
-            bool owner;
-            int pk1;
-            if (mode == OWN_ALL) { owner = true; pk1 = N1 - 1 - k1; }
-            else if (mode == OWN_NONE) { owner = false; pk1 = 0; }
-            else if (mode == OWN_SELF0) { owner = k1 < N1 / 2; pk1 = (N1 - k1) & (N1 - 1); }
-            else { owner = k1 < N1 / 2; pk1 = N1 - 1 - k1; }
-            if (!owner) continue;
+            const int pk1 = mode == SELF0 ? ((N1 - k1) & (N1 - 1)) : (N1 - 1 - k1);
             const uint32_t k = (uint32_t)k2 + (uint32_t)N2 * k1;
             const float2 zk = x[m];
-            // spectrum bins k and M - k: staged for warps 0..3, direct for row N2/2
             float2 hk = make_float2(0.f, 0.f), hn = make_float2(0.f, 0.f);
             if constexpr (!SPEC) {
-                if (warp < 4) {
-                    hk = hs[warp * BK + lane + 32 * mm];
-                    hn = hs[(4 + warp) * BK + lane + 32 * mm];
-                } else {
-                    hk = __ldg(H + k);
-                    hn = __ldg(H + (M - k));
-                }
+                hk = hs[(2 * warp + 0) * BK + lane + 32 * mm];
+                hn = hs[(2 * warp + 1) * BK + lane + 32 * mm];
             }
-            if (mode == OWN_SELF0 && k1 == 0) {
+            if (mode == SELF0 && k1 == 0) {
                 // DC (bin 0) and Nyquist (bin M): both real
                 if constexpr (SPEC) {
                     own[spad(0)] = make_float2(zk.x + zk.y, 0.f);
@@ -436,34 +429,29 @@ __global__ void __launch_bounds__(NT, 2) rowpass_kernel(const FsParams p) {
     }
     if constexpr (SPEC) {
         // bin M/2 (row 0, k1 = N1/2) pairs with itself: X[M/2] = conj(Z[M/2])
-        if (mode == OWN_SELF0 && lane == 0) own[spad(N1 / 2)] = cconj(x[(N1 / 2) / 32]);
+        if (mode == SELF0 && lane == 0) own[spad(N1 / 2)] = cconj(x[(N1 / 2) / 32]);
         __syncthreads();
         // rows_s[w][k1] now holds bin k2_w + N2 k1 of every row of the CTA;
         // 8 lanes store the 8 rows' bins of one k1
         const int w = tid & 7;
-        int kw;
-        if (w < 4) kw = 4 * g + w;
-        else kw = (g == 0 && w == 4) ? N2 / 2 : N2 - (4 * g + w - 4);
+        const int kw = row_k2(w);
 #pragma unroll 4
         for (int k1 = tid >> 3; k1 < N1; k1 += NT / 8)
             Ho[(uint32_t)kw + (uint32_t)N2 * (uint32_t)k1] = rows_s[w * RS + spad(k1)];
         return;
     }
     // self-paired element of row 0: bin M/2 (k1 = N1/2)
-    if (mode == OWN_SELF0 && lane == 0) {
+    if (mode == SELF0 && lane == 0) {
         constexpr int mh = (N1 / 2) / 32;
         const float2 r = cmulc(x[mh], __ldg(H + M / 2));
         x[mh] = make_float2(4.f * r.x, 4.f * r.y);
     }
     __syncthreads();
+    // bins k1 >= N1/2 were produced by the partner warp (or this one)
 #pragma unroll
-    for (int m = 0; m < P; ++m) {
+    for (int m = P / 2; m < P; ++m) {
         const int k1 = lane + 32 * m;
-        bool owner;
-        if (mode == OWN_ALL) owner = true;
-        else if (mode == OWN_NONE) owner = false;
-        else owner = k1 < N1 / 2 || (mode == OWN_SELF0 && k1 == N1 / 2);
-        if (!owner) x[m] = own[spad(k1)];
+        if (!(mode == SELF0 && k1 == N1 / 2)) x[m] = own[spad(k1)];
     }
     __syncwarp();
     // ---- inverse FFT over k1 -> n1, times W_M^{-n1 k2}, back to the buffer

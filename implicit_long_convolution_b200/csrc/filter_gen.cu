@@ -57,7 +57,10 @@ struct GenParams {
     float *h;
 };
 
-__device__ __forceinline__ float silu(float a) { return a / (1.f + expf(-a)); }
+constexpr float kLog2e = 1.4426950408889634f;
+
+// x * sigmoid(x); exp(-x) as 2^(-x log2 e) (relative error ~1e-7 |x|)
+__device__ __forceinline__ float silu(float a) { return a * __frcp_rn(1.f + exp2f(-a * kLog2e)); }
 
 __device__ __forceinline__ int signed_off(int i, int S) { return i < S / 2 ? i : i - S; }
 
@@ -203,6 +206,16 @@ __global__ void __launch_bounds__(NT, 2) filter_gen_kernel(const GenParams p) {
     } else {
         const int S = p.S, ls = p.log_s, twog_m = 2 * p.g - 1;
         const float gf = (float)p.g;
+        // every feature is cos or sin of pi m / g for one of the 2g phases m
+        // = (j r) mod 2g: tabulate them once (in the second activation buffer,
+        // free until the first layer writes it)
+        float2 *phase = reinterpret_cast<float2 *>(actB);
+        for (int m = tid; m <= twog_m; m += NT) {
+            float sn, cs;
+            sincospif((float)m / gf, &sn, &cs);
+            phase[m] = make_float2(cs, sn);
+        }
+        __syncthreads();
         for (int idx = tid; idx < P * w0; idx += NT) {
             const int pos = idx & (P - 1), f = idx / P;
             const int64_t q = p0 + pos;
@@ -213,9 +226,8 @@ __global__ void __launch_bounds__(NT, 2) filter_gen_kernel(const GenParams p) {
                 const int j = (ff < p.F ? ff : ff - p.F) + 1;
                 const int ia = (int)(q >> (ls * (2 - axis))) & (S - 1);
                 const int mm = (j * signed_off(ia, S)) & twog_m;   // (j r) mod 2g, 2g a power of two
-                float sn, cs;
-                sincospif((float)mm / gf, &sn, &cs);               // angle pi j r / g
-                v = (ff < p.F) ? cs : sn;
+                const float2 cs = phase[mm];                       // angle pi j r / g
+                v = (ff < p.F) ? cs.x : cs.y;
             }
             actA[f * P + pos] = v;
         }
@@ -298,10 +310,10 @@ __global__ void __launch_bounds__(NT, 2) filter_gen_kernel(const GenParams p) {
                 const int o = o0 + r;
                 if (o >= lend) continue;
                 const float bo = par[r];
-                const float al = par[OT_MAX + r];
+                const float al = par[OT_MAX + r] * kLog2e;      // e^{-a n} = 2^{-a log2(e) n}
                 float v[4];
 #pragma unroll
-                for (int a = 0; a < 4; ++a) v[a] = ok[a] ? (acc[a][c] + bo) * expf(-al * nrm[a]) : 0.f;
+                for (int a = 0; a < 4; ++a) v[a] = ok[a] ? (acc[a][c] + bo) * exp2f(-al * nrm[a]) : 0.f;
                 float *dst = p.h + ((int64_t)set * nout + o) * p.npos + q0;
                 if (full) {
                     *reinterpret_cast<float4 *>(dst) = make_float4(v[0], v[1], v[2], v[3]);

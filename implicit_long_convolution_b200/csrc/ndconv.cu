@@ -90,16 +90,24 @@ __global__ void __launch_bounds__(NT) nd_fwd_plane(const NdParams p) {
     {
         const int g = tid / R::T, t = tid % R::T;
         float2 *xb = gbuf + g * spad_size(R::N);
+        // the next round's row is requested before this round's FFT
+        auto load_row = [&](int j, float2 (&v)[R::P]) {
+#pragma unroll
+            for (int m = 0; m < R::P; ++m) {
+                const int e = t + m * R::T;             // packed point
+                v[m] = make_float2(0.f, 0.f);
+                if (j < gI && e < PK) v[m] = __ldg(reinterpret_cast<const float2 *>(plane + (int64_t)j * gI) + e);
+            }
+        };
+        float2 xn[R::P];
+        load_row(g, xn);
         for (int j0 = 0; j0 < gI; j0 += R::G) {
             const int j = j0 + g;
             const bool act = j < gI;
             float2 x[R::P];
 #pragma unroll
-            for (int m = 0; m < R::P; ++m) {
-                const int e = t + m * R::T;             // packed point
-                x[m] = make_float2(0.f, 0.f);
-                if (act && e < PK) x[m] = __ldg(reinterpret_cast<const float2 *>(plane + (int64_t)j * gI) + e);
-            }
+            for (int m = 0; m < R::P; ++m) x[m] = xn[m];
+            if (j0 + R::G < gI) load_row(j + R::G, xn);
             block_fft<LOG_S - 1, R::LP, -1, PAD, SyncWarp>(x, xb, t, p.tw_r, SyncWarp{});
             store_own<LOG_S - 1, R::LP>(x, xb, t);
             __syncwarp();
@@ -149,7 +157,24 @@ __global__ void __launch_bounds__(NT) nd_fwd_plane(const NdParams p) {
 
 // ---------------------------------------------------------------------------
 // F2: along x for one y-bin: conv (times H, inverse, crop) or spectrum out.
+// The kernel spectrum H[kx, k1, kz] of this y-bin is S runs of S/2+1
+// contiguous bins; each round of G lines (kz) stages its S x G block through
+// shared memory (cp.async, two buffers), so HBM sees 128-byte runs instead of
+// one 8-byte value per line per kx.  Spectrum outputs go back through the
+// tile and leave as contiguous runs.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ void nd_cpa8(void *smem, const void *g) {
+    const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(sa), "l"(g) : "memory");
+}
+__device__ __forceinline__ void nd_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void nd_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// H staging block of one round: S rows (kx) x G lines, row stride G + 1
+template <int LOG_S>
+__host__ __device__ constexpr int xpass_hstride() { return NT / (1 << LOG_S) * 8 + 1; }
+
 template <int LOG_S, bool PAD, bool SPEC>
 __global__ void __launch_bounds__(NT) nd_xpass(const NdParams p) {
     constexpr int S = 1 << LOG_S;
@@ -157,27 +182,55 @@ __global__ void __launch_bounds__(NT) nd_xpass(const NdParams p) {
     constexpr int NB = H2 + 1;
     constexpr int gI = PAD ? S / 2 : S;
     using C = Grp<LOG_S>;
+    constexpr int G = C::G;                              // lines per round
+    constexpr int HS = xpass_hstride<LOG_S>();           // = G + 1
+    static_assert(HS == G + 1, "staging stride");
+    constexpr int NR = (NB + G - 1) / G;                 // rounds
     extern __shared__ float2 sm[];
     float2 *tile = sm;                                  // gI rows (x) x NB
     float2 *gbuf = sm + gI * NB;
+    float2 *hst = gbuf + NT / C::T * spad_size(C::N);   // conv: 2 x [S][HS]
     const int tid = threadIdx.x;
     const int64_t sl = blockIdx.y;                      // slab within chunk
     const int64_t slab = p.slab0 + sl;
     const int k1 = blockIdx.x;
     float2 *base = p.ws + sl * (int64_t)gI * S * NB + (int64_t)k1 * NB;
     for (int e = tid; e < gI * NB; e += NT) {
-        const int ii = e / NB, k = e % NB;
-        tile[e] = __ldcg(base + (int64_t)ii * S * NB + k);
+        const int ii = e / NB, k = e - ii * NB;
+        nd_cpa8(tile + e, base + (int64_t)ii * S * NB + k);
     }
-    __syncthreads();
+    nd_commit();
     const int64_t d = slab % p.D, b = slab / p.D;
-    const float2 *Hs = SPEC ? nullptr : p.H + b * p.H_batch_stride + d * (int64_t)S * S * NB;
-    float2 *Ho = SPEC ? p.Hout + slab * (int64_t)S * S * NB : nullptr;
+    const float2 *Hs = SPEC ? nullptr : p.H + b * p.H_batch_stride + d * (int64_t)S * S * NB + (int64_t)k1 * NB;
+    auto stage = [&](int r, float2 *dst) {
+        for (int e = tid; e < S * G; e += NT) {
+            const int kx = e / G, kk = e % G;
+            const int k = r * G + kk;
+            if (k < NB) nd_cpa8(dst + kx * HS + kk, Hs + (int64_t)kx * S * NB + k);
+        }
+    };
+    if constexpr (!SPEC) {
+        stage(0, hst);
+        nd_commit();
+    }
+    nd_wait<0>();
+    __syncthreads();
     const int g = tid / C::T, t = tid % C::T;
     float2 *xb = gbuf + g * spad_size(C::N);
-    for (int k0 = 0; k0 < NB; k0 += C::G) {
-        const int k = k0 + g;
+#pragma unroll 1
+    for (int r = 0; r < NR; ++r) {
+        const int k = r * G + g;
         const bool act = k < NB;
+        if constexpr (!SPEC) {
+            if (r + 1 < NR) {
+                stage(r + 1, hst + ((r + 1) & 1) * S * HS);
+                nd_commit();
+                nd_wait<1>();
+            } else {
+                nd_wait<0>();
+            }
+            __syncthreads();
+        }
         float2 x[C::P];
 #pragma unroll
         for (int m = 0; m < C::P; ++m) {
@@ -186,20 +239,22 @@ __global__ void __launch_bounds__(NT) nd_xpass(const NdParams p) {
         }
         block_fft<LOG_S, C::LP, -1, PAD, SyncWarp>(x, xb, t, p.tw_c, SyncWarp{});
         if constexpr (SPEC) {
+            // back into column k of the tile (gI = S here); the z split
+            // carries a factor 2 (folded into the conv scale)
+            __syncwarp();
             if (act) {
 #pragma unroll
                 for (int m = 0; m < C::P; ++m) {
                     const int kx = t + m * C::T;
-                    // the z split carries a factor 2 (folded into the conv scale)
-                    Ho[((int64_t)kx * S + k1) * NB + k] = make_float2(0.5f * x[m].x, 0.5f * x[m].y);
+                    tile[kx * NB + k] = make_float2(0.5f * x[m].x, 0.5f * x[m].y);
                 }
             }
         } else {
+            const float2 *hb = hst + (r & 1) * S * HS + g;
 #pragma unroll
             for (int m = 0; m < C::P; ++m) {
                 const int kx = t + m * C::T;
-                const float2 h = act ? __ldg(Hs + ((int64_t)kx * S + k1) * NB + k) : make_float2(0.f, 0.f);
-                x[m] = cmul(x[m], h);
+                x[m] = cmul(x[m], act ? hb[kx * HS] : make_float2(0.f, 0.f));
             }
             __syncwarp();
             block_fft<LOG_S, C::LP, +1, false, SyncWarp>(x, xb, t, p.tw_c, SyncWarp{});
@@ -211,12 +266,19 @@ __global__ void __launch_bounds__(NT) nd_xpass(const NdParams p) {
                     if (ii < gI) tile[ii * NB + k] = x[m];
                 }
             }
+            __syncthreads();   // staging buffer r & 1 is refilled next round
         }
     }
-    if constexpr (!SPEC) {
+    if constexpr (SPEC) {
         __syncthreads();
+        float2 *Ho = p.Hout + slab * (int64_t)S * S * NB + (int64_t)k1 * NB;
+        for (int e = tid; e < S * NB; e += NT) {
+            const int kx = e / NB, k = e - kx * NB;
+            Ho[(int64_t)kx * S * NB + k] = tile[e];
+        }
+    } else {
         for (int e = tid; e < gI * NB; e += NT) {
-            const int ii = e / NB, k = e % NB;
+            const int ii = e / NB, k = e - ii * NB;
             __stcg(base + (int64_t)ii * S * NB + k, tile[e]);
         }
     }
@@ -241,7 +303,9 @@ __global__ void __launch_bounds__(NT) nd_inv_plane(const NdParams p) {
     const int64_t slab = p.slab0 + sl;
     const int i = blockIdx.x;
     const float2 *src = p.ws + (sl * gI + i) * (int64_t)S * NB;
-    for (int e = tid; e < S * NB; e += NT) tile[e] = __ldcg(src + e);
+    for (int e = tid; e < S * NB; e += NT) nd_cpa8(tile + e, src + e);
+    nd_commit();
+    nd_wait<0>();
     __syncthreads();
     // ---- inverse along y (k1 -> j), keep j < gI
     {
@@ -276,6 +340,16 @@ __global__ void __launch_bounds__(NT) nd_inv_plane(const NdParams p) {
             const int j = j0 + g;
             const bool act = j < gI;
             const float2 *Y = tile + (act ? j : 0) * NB;
+            constexpr int PK = gI / 2;
+            const int64_t rb = pbase + (int64_t)(act ? j : 0) * gI;
+            float2 uu[R::P], gg[R::P];
+#pragma unroll
+            for (int m = 0; m < R::P; ++m) {
+                const int e = t + m * R::T;
+                const bool in = act && e < PK;
+                uu[m] = (in && dk != 0.f) ? __ldg(reinterpret_cast<const float2 *>(p.u + rb) + e) : make_float2(0.f, 0.f);
+                gg[m] = (in && p.gate) ? __ldg(reinterpret_cast<const float2 *>(p.gate + rb) + e) : make_float2(1.f, 1.f);
+            }
             float2 x[R::P];
 #pragma unroll
             for (int m = 0; m < R::P; ++m) {
@@ -292,22 +366,18 @@ __global__ void __launch_bounds__(NT) nd_inv_plane(const NdParams p) {
             }
             block_fft<LOG_S - 1, R::LP, +1, false, SyncWarp>(x, xb, t, p.tw_r, SyncWarp{});
             if (act) {
-                constexpr int PK = gI / 2;
-                const int64_t rb = pbase + (int64_t)j * gI;
 #pragma unroll
                 for (int m = 0; m < R::P; ++m) {
                     const int e = t + m * R::T;                 // packed output point
                     if (e < PK) {
                         float2 v = make_float2(x[m].x * p.scale, x[m].y * p.scale);
                         if (dk != 0.f) {
-                            const float2 uu = __ldg(reinterpret_cast<const float2 *>(p.u + rb) + e);
-                            v.x = fmaf(dk, uu.x, v.x);
-                            v.y = fmaf(dk, uu.y, v.y);
+                            v.x = fmaf(dk, uu[m].x, v.x);
+                            v.y = fmaf(dk, uu[m].y, v.y);
                         }
                         if (p.gate) {
-                            const float2 gg = __ldg(reinterpret_cast<const float2 *>(p.gate + rb) + e);
-                            v.x *= gg.x;
-                            v.y *= gg.y;
+                            v.x *= gg[m].x;
+                            v.y *= gg[m].y;
                         }
                         reinterpret_cast<float2 *>(p.y + rb)[e] = v;
                     }
@@ -354,13 +424,14 @@ hy_status run_nd(const NDArgs &a, NdParams p, cudaStream_t s, bool spec, int64_t
     const int64_t per_slab = (int64_t)gI * S * NB * 8;
     const int64_t cs = nd_chunk(slabs, per_slab);
     const size_t sm1 = sizeof(float2) * ((size_t)S * NB + gbuf_elems<LOG_S>());
-    const size_t sm2 = sizeof(float2) * ((size_t)gI * NB + gbuf_elems<LOG_S>());
+    const size_t sm2 = sizeof(float2) * ((size_t)gI * NB + (size_t)NT / Grp<LOG_S>::T * spad_size(Grp<LOG_S>::N));
+    const size_t sm2c = sm2 + sizeof(float2) * 2 * (size_t)S * xpass_hstride<LOG_S>();
     auto k1 = nd_fwd_plane<LOG_S, PAD>;
     auto k2c = nd_xpass<LOG_S, PAD, false>;
     auto k2s = nd_xpass<LOG_S, PAD, true>;
     auto k3 = nd_inv_plane<LOG_S, PAD>;
     hy_status st;
-    if ((st = nd_smem(k1, sm1)) != HY_OK || (st = nd_smem(k2c, sm2)) != HY_OK ||
+    if ((st = nd_smem(k1, sm1)) != HY_OK || (st = nd_smem(k2c, sm2c)) != HY_OK ||
         (st = nd_smem(k2s, sm2)) != HY_OK || (st = nd_smem(k3, sm1)) != HY_OK)
         return st;
     (void)a;
@@ -371,7 +442,7 @@ hy_status run_nd(const NDArgs &a, NdParams p, cudaStream_t s, bool spec, int64_t
         if (spec) {
             k2s<<<dim3(S, (unsigned)ns), NT, sm2, s>>>(p);
         } else {
-            k2c<<<dim3(S, (unsigned)ns), NT, sm2, s>>>(p);
+            k2c<<<dim3(S, (unsigned)ns), NT, sm2c, s>>>(p);
             k3<<<dim3(gI, (unsigned)ns), NT, sm1, s>>>(p);
         }
         if ((st = check_launch("N-D launch")) != HY_OK) return st;

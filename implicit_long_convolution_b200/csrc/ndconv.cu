@@ -173,7 +173,7 @@ __device__ __forceinline__ void nd_wait() { asm volatile("cp.async.wait_group %0
 
 // H staging block of one round: S rows (kx) x G lines, row stride G + 1
 template <int LOG_S>
-__host__ __device__ constexpr int xpass_hstride() { return NT / (1 << LOG_S) * 8 + 1; }
+__host__ __device__ constexpr int xpass_hstride() { return Grp<LOG_S>::G + 1; }
 
 template <int LOG_S, bool PAD, bool SPEC>
 __global__ void __launch_bounds__(NT) nd_xpass(const NdParams p) {

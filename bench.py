@@ -483,19 +483,23 @@ def cpu_baseline(w, budget_s=12.0):
     h64 = oracle.filter_gen_1d(L, s["F"], True, w.Ws, w.bs, w.alpha)
     t_filter = time.perf_counter() - t0
     cores = oracle.threads()
-    probe = min(rows_total, max(cores, 8))
-    # the first call also starts the oracle's thread pool: time the second
-    for _ in range(2):
+    # growing batches of distinct random rows until the sample has used about
+    # the budget (the rate of a small batch is not a good predictor)
+    order = np.random.default_rng(0).permutation(rows_total)
+    done, t_rows, n = 0, 0.0, min(rows_total, max(cores, 8))
+    while done < rows_total:
+        batch = order[done:done + n]
         t0 = time.perf_counter()
-        oracle.hyena_rows(w.v.f32, [x.f32 for x in w.xs], h64.reshape(K, D, L), w.Dskip,
-                          rows=np.arange(probe))
-        t_probe = time.perf_counter() - t0
-    n = int(max(probe, min(rows_total, probe * max(1.0, (budget_s - t_filter) / max(t_probe, 1e-3)))))
-    n = min(rows_total, max(probe, (n // cores) * cores))
-    rows = np.random.default_rng(0).choice(rows_total, n, replace=False)
-    t0 = time.perf_counter()
-    oracle.hyena_rows(w.v.f32, [x.f32 for x in w.xs], h64.reshape(K, D, L), w.Dskip, rows=rows)
-    t_rows = time.perf_counter() - t0
+        oracle.hyena_rows(w.v.f32, [x.f32 for x in w.xs], h64.reshape(K, D, L), w.Dskip, rows=batch)
+        dt = time.perf_counter() - t0
+        done += batch.size
+        t_rows += dt
+        left = budget_s - t_filter - t_rows
+        if left <= 0:
+            break
+        per_row = dt / batch.size
+        n = int(min(rows_total - done, max(cores, min(8 * batch.size, left / per_row))))
+    rows = order[:done]
     est_step = t_filter + t_rows * rows_total / rows.size
     return {"value": round(step_bytes / est_step / 1e9, 6), "unit": "GB/s", "cores": cores,
             "kind": "oracle",

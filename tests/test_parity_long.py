@@ -54,6 +54,8 @@ LONG = [
     (2, 1, 32768, 3, "f32", True),
     (1, 3, 40000, 2, "bf16", True),
     (1, 2, 65536, 2, "f32", False),
+    (1, 1, 30001, 2, "f32", True),      # odd length: scalar tails of the vector loads
+    (1, 1, 50002, 3, "bf16", True),     # L = 2 (mod 4)
 ]
 
 
@@ -74,6 +76,34 @@ def test_long_operator_vs_direct(B, D, L, order, dtype, skip):
     ref = oracle.hyena_rows(w.v.f32, [x.f32 for x in w.xs], h32.astype(np.float64),
                             w.Dskip if skip else None)
     check(to_np(y).reshape(B * D, L), ref, dtype, "long operator L%d order%d" % (L, order))
+
+
+def test_long_operator_misaligned_rows_bitwise():
+    """Signals that are 8- but not 16-byte aligned take the scalar load/store
+    path of the column passes; it must give bit-identical results to the
+    vector path on the same values."""
+    B, D, L, order = 1, 2, 36000, 3
+    w = hw.make("c3", seed=5, B=B, D=D, L=L, order=order)
+    h32 = _filters(np.random.default_rng(5), 2, D, L)
+    Hs, _ = _spectra(h32)
+    dsk = [f32_dev(w.Dskip[k]) for k in range(2)]
+
+    # 8 bytes past a 256-byte boundary: allowed (rows of even length need
+    # 8-byte alignment) but not 16-byte aligned
+    def shifted(a):
+        flat = torch.zeros(a.size + 2, device="cuda")
+        flat[2:] = torch.from_numpy(np.ascontiguousarray(a, np.float32).ravel()).cuda()
+        return flat[2:].view(a.shape)
+
+    y0 = _run(f32_dev(w.v.f32), [f32_dev(x.f32) for x in w.xs], Hs, dsk, L, B, D, order, 0)
+    v1 = shifted(w.v.f32)
+    xs1 = [shifted(x.f32) for x in w.xs]
+    y1 = torch.empty(B * D * L + 2, device="cuda")[2:].view(B, D, L)
+    wsb = hy.operator_workspace(order, B, D, L, 0)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    hy.hyena_operator(v1, xs1, Hs, y1, Dskips=dsk, ws=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y0, y1)
 
 
 def test_long_operator_2p18_fft_reference():
@@ -158,3 +188,13 @@ def test_long_spectrum_matches_reference():
     k = np.arange(L + 1)
     np.testing.assert_allclose(Hd[0], np.ones(L + 1), atol=1e-6)
     np.testing.assert_allclose(Hd[1], np.exp(-2j * np.pi * k * 12345 / (2 * L)), atol=2e-6)
+
+
+def test_long_spectrum_ragged_length():
+    """A filter length that is neither a power of two nor a multiple of 4."""
+    L = 70001
+    h32 = _filters(np.random.default_rng(6), 1, 2, L)
+    _, H = _spectra(h32)
+    ref = oracle.fft_spectrum(h32.reshape(2, L), n=2 * (hy.spectrum_bins(L) - 1))
+    Hg = H.cpu().numpy().astype(np.complex128)
+    check(np.stack([Hg.real, Hg.imag]), np.stack([ref.real, ref.imag]), "f32", "spectrum L=70001")

@@ -21,7 +21,8 @@ __all__ = [
     "HyenaError", "HyenaLibraryMissing", "LIB_PATH", "lib", "spectrum_bins",
     "hyena_filter_gen", "hyena_filter_spectrum", "filter_spectrum_workspace",
     "hyena_fftconv", "hyena_operator", "operator_workspace", "hyena_operator_noalloc", "hyena_nd_conv",
-    "nd_conv_workspace", "spectral_gate", "STATUS",
+    "nd_conv_workspace", "spectral_gate", "operator_host_workspace", "hyena_operator_host",
+    "spectral_gate_host_workspace", "spectral_gate_host", "STATUS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhyena_b200.so")
@@ -90,6 +91,11 @@ def lib():
         "hyena_nd_conv": (_I, [_I, ctypes.POINTER(_I), _I, _I, _I, _VP, _VP, _I64, _VP, _VP, _VP,
                                _VP, _SZ, _VP]),
         "spectral_gate": (_I, [_I, _I, _I, _I, _I, _VP, _VP, _I64, _VP, _VP, _VP]),
+        "hyena_operator_host_workspace": (_SZ, [_I, _I, _I, _I, _I]),
+        "hyena_operator_host": (_I, [_I, _I, _I, _I, _I, _VP, ctypes.POINTER(_VP), ctypes.POINTER(_VP),
+                                     ctypes.POINTER(_VP), _VP, _VP, _SZ, _VP]),
+        "spectral_gate_host_workspace": (_SZ, [_I, _I, _I, _I, _I]),
+        "spectral_gate_host": (_I, [_I, _I, _I, _I, _I, _VP, _VP, _I64, _VP, _VP, _VP, _SZ, _VP]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -222,4 +228,36 @@ def spectral_gate(x, g, y, *, x2=None, g_batch_stride: int = 0, stream=None):
     B, Hh, Dh, L = x.shape
     _check(lib().spectral_gate(B, Hh, Dh, L, _dt(x), _ptr(x), _ptr(g), g_batch_stride, _ptr(x2),
                                _ptr(y), _stream(stream)))
+    return y
+
+
+def operator_host_workspace(order: int, B: int, D: int, L: int, dtype_code: int) -> int:
+    return int(lib().hyena_operator_host_workspace(order, B, D, L, dtype_code))
+
+
+def hyena_operator_host(v, xs: Sequence, Hs: Sequence, y, *, Dskips: Optional[Sequence] = None,
+                        ws=None, stream=None):
+    """hyena_operator with v, xs and y in (page-locked) host memory; Hs,
+    Dskips and ws on the device.  Copies and compute overlap chunk by chunk;
+    y is valid once the stream is synchronised (see hyena.h)."""
+    B, D, L = v.shape
+    order = len(xs) + 1
+    dsk = _ptrs(Dskips) if Dskips is not None else None
+    wsb = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib().hyena_operator_host(order, B, D, L, _dt(v), _ptr(v), _ptrs(xs), _ptrs(Hs), dsk, _ptr(y),
+                                     _ptr(ws), wsb, _stream(stream)))
+    return y
+
+
+def spectral_gate_host_workspace(B: int, H: int, Dh: int, L: int, dtype_code: int) -> int:
+    return int(lib().spectral_gate_host_workspace(B, H, Dh, L, dtype_code))
+
+
+def spectral_gate_host(x, g, y, *, x2=None, g_batch_stride: int = 0, ws=None, stream=None):
+    """spectral_gate with x, x2 and y in (page-locked) host memory; g and ws
+    on the device (see hyena.h)."""
+    B, Hh, Dh, L = x.shape
+    wsb = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib().spectral_gate_host(B, Hh, Dh, L, _dt(x), _ptr(x), _ptr(g), g_batch_stride, _ptr(x2),
+                                    _ptr(y), _ptr(ws), wsb, _stream(stream)))
     return y

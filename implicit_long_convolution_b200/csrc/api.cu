@@ -4,6 +4,7 @@
 #include <cstring>
 
 #include "kernels.h"
+#include "host_pipeline.h"
 #include "resident.cuh"
 #include "status.h"
 #include "twiddle.h"
@@ -420,4 +421,179 @@ extern "C" hy_status hyena_operator_noalloc(int order, int B, int D, int L, hy_d
     }
     a.y = y;
     return launch_long_conv_noalloc(a, (cudaStream_t)stream);
+}
+
+// ----------------------------------------------------------------------------
+// Host-buffer entry points (see include/hyena.h and host_pipeline.h): the
+// operator and the spectral gate over signals in host memory, with the
+// host-to-device copies, the compute and the device-to-host copies of
+// successive row chunks overlapped.
+// ----------------------------------------------------------------------------
+namespace {
+
+// Chunks of a (B, G, row) signal: whole batches when one batch is at most the
+// target size, else runs of `ng` groups (channels or heads) within one batch.
+struct HostPlan {
+    bool whole;       // chunks are nb whole batches
+    int nb, ng;       // batches per chunk (whole) or groups per chunk
+    int per_batch;    // chunks per batch (!whole)
+    int nchunks;
+    int64_t max_groups;   // groups in the largest chunk
+};
+
+HostPlan host_plan(int B, int G, size_t group_bytes, int min_groups) {
+    HostPlan p{};
+    int64_t g = (int64_t)(kHostChunkBytes / (group_bytes ? group_bytes : 1));
+    if (g < min_groups) g = min_groups;
+    if (g < 1) g = 1;
+    if (g >= G) {
+        p.whole = true;
+        p.nb = (int)((g / G) < B ? (g / G) : B);
+        if (p.nb < 1) p.nb = 1;
+        p.ng = G;
+        p.nchunks = (B + p.nb - 1) / p.nb;
+        p.max_groups = (int64_t)p.nb * G;
+    } else {
+        p.whole = false;
+        p.nb = 1;
+        p.ng = (int)g;
+        p.per_batch = (G + p.ng - 1) / p.ng;
+        p.nchunks = B * p.per_batch;
+        p.max_groups = p.ng;
+    }
+    return p;
+}
+
+// chunk c of plan p: first batch b0, batches nbc, first group g0, groups ngc
+void host_chunk(const HostPlan &p, int B, int G, int c, int &b0, int &nbc, int &g0, int &ngc) {
+    if (p.whole) {
+        b0 = c * p.nb;
+        nbc = (B - b0) < p.nb ? (B - b0) : p.nb;
+        g0 = 0;
+        ngc = G;
+    } else {
+        b0 = c / p.per_batch;
+        nbc = 1;
+        g0 = (c % p.per_batch) * p.ng;
+        ngc = (G - g0) < p.ng ? (G - g0) : p.ng;
+    }
+}
+
+size_t host_ring_bytes(int n_in, size_t slot) { return (size_t)kHostSlots * ((size_t)n_in * round256(slot) + round256(slot)); }
+
+HostPlan operator_host_plan(int D, int B, int L, hy_dtype dt) {
+    const int log_m = ilog2(spectrum_m(L));
+    // multi-pass chunks of at least 8 rows keep its launches full
+    return host_plan(B, D, (size_t)L * dt_size(dt), log_m > kMaxResidentLogM ? 8 : 1);
+}
+
+}  // namespace
+
+extern "C" size_t hyena_operator_host_workspace(int order, int B, int D, int L, hy_dtype dt) {
+    if (order < 2 || order - 1 > kMaxOrders || B < 1 || D < 1 || L < 1 || (dt != HY_F32 && dt != HY_BF16)) return 0;
+    const HostPlan p = operator_host_plan(D, B, L, dt);
+    const size_t slot = (size_t)p.max_groups * L * dt_size(dt);
+    const size_t chain = hyena_operator_workspace(order, 1, (int)p.max_groups, L, dt);
+    return host_ring_bytes(order, slot) + round256(chain);
+}
+
+extern "C" hy_status hyena_operator_host(int order, int B, int D, int L, hy_dtype dt, const void *v,
+                                         const void *const *x, const hy_c32 *const *H,
+                                         const float *const *Dskip, void *y, void *ws, size_t ws_bytes,
+                                         void *stream) {
+    clear_error();
+    const char *who = "hyena_operator_host";
+    if (order < 2 || order - 1 > kMaxOrders)
+        return set_error(HY_ERR_UNSUPPORTED, "%s: order must be 2..%d", who, kMaxOrders + 1);
+    if (B < 1 || D < 1 || L < 1) return set_error(HY_ERR_INVALID_ARG, "%s: B, D, L must be >= 1", who);
+    if (dt != HY_F32 && dt != HY_BF16) return set_error(HY_ERR_INVALID_ARG, "%s: unknown dtype", who);
+    if (!x || !H) return set_error(HY_ERR_INVALID_ARG, "%s: null x or H array", who);
+    const int K = order - 1;
+    hy_status st;
+    if ((st = check_host_ptr(v, who, "v")) != HY_OK || (st = check_host_ptr(y, who, "y")) != HY_OK) return st;
+    for (int k = 0; k < K; ++k) {
+        if ((st = check_host_ptr(x[k], who, "x[k]")) != HY_OK) return st;
+        if (!H[k]) return set_error(HY_ERR_INVALID_ARG, "%s: H[%d] is null", who, k);
+    }
+    const size_t need = hyena_operator_host_workspace(order, B, D, L, dt);
+    if (!ws || ws_bytes < need)
+        return set_error(HY_ERR_WORKSPACE, "%s: needs %zu workspace bytes, got %zu", who, need, ws ? ws_bytes : (size_t)0);
+    if (!aligned(ws, 256)) return set_error(HY_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", who);
+    const size_t esz = dt_size(dt);
+    const HostPlan p = operator_host_plan(D, B, L, dt);
+    const size_t slot = (size_t)p.max_groups * L * esz;
+    char *ring = reinterpret_cast<char *>(ws);
+    char *chain_ws = ring + host_ring_bytes(order, slot);
+    const size_t chain_bytes = ws_bytes - host_ring_bytes(order, slot);
+    const int64_t M = spectrum_m(L);
+    auto describe = [&](int c, HostChunk &ch) {
+        int b0, nbc, g0, ngc;
+        host_chunk(p, B, D, c, b0, nbc, g0, ngc);
+        const size_t off = ((size_t)b0 * D + g0) * L * esz;
+        ch.in_bytes = (size_t)nbc * ngc * L * esz;
+        ch.src[0] = reinterpret_cast<const char *>(v) + off;
+        for (int k = 0; k < K; ++k) ch.src[1 + k] = reinterpret_cast<const char *>(x[k]) + off;
+        ch.dst = reinterpret_cast<char *>(y) + off;
+        ch.out_bytes = ch.in_bytes;
+    };
+    auto compute = [&](int c, const void *const *din, void *dout, cudaStream_t s) {
+        int b0, nbc, g0, ngc;
+        host_chunk(p, B, D, c, b0, nbc, g0, ngc);
+        const hy_c32 *Hc[kMaxOrders];
+        const float *Dc[kMaxOrders];
+        for (int k = 0; k < K; ++k) {
+            Hc[k] = H[k] + (size_t)g0 * (M + 1);
+            Dc[k] = (Dskip && Dskip[k]) ? Dskip[k] + g0 : nullptr;
+        }
+        return run_chain(K, nbc, ngc, L, dt, din[0], din + 1, Hc, Dskip ? Dc : nullptr, dout, chain_ws,
+                         chain_bytes, s, who);
+    };
+    return run_host_pipeline(order, p.nchunks, slot, slot, ring, (cudaStream_t)stream, describe, compute, who);
+}
+
+extern "C" size_t spectral_gate_host_workspace(int B, int H, int Dh, int L, hy_dtype dt) {
+    if (B < 1 || H < 1 || Dh < 1 || L < 1 || (dt != HY_F32 && dt != HY_BF16)) return 0;
+    const HostPlan p = host_plan(B, H, (size_t)Dh * L * dt_size(dt), 1);
+    return host_ring_bytes(2, (size_t)p.max_groups * Dh * L * dt_size(dt));
+}
+
+extern "C" hy_status spectral_gate_host(int B, int H, int Dh, int L, hy_dtype dt, const void *x, const hy_c32 *g,
+                                        int64_t g_batch_stride, const void *x2, void *y, void *ws, size_t ws_bytes,
+                                        void *stream) {
+    clear_error();
+    const char *who = "spectral_gate_host";
+    if (B < 1 || H < 1 || Dh < 1 || L < 1) return set_error(HY_ERR_INVALID_ARG, "%s: B, H, Dh, L must be >= 1", who);
+    if (dt != HY_F32 && dt != HY_BF16) return set_error(HY_ERR_INVALID_ARG, "%s: unknown dtype", who);
+    if (!g) return set_error(HY_ERR_INVALID_ARG, "%s: null gate", who);
+    if (g_batch_stride < 0) return set_error(HY_ERR_INVALID_ARG, "%s: negative gate stride", who);
+    hy_status st;
+    if ((st = check_host_ptr(x, who, "x")) != HY_OK || (st = check_host_ptr(y, who, "y")) != HY_OK) return st;
+    if (x2 && (st = check_host_ptr(x2, who, "x2")) != HY_OK) return st;
+    const size_t need = spectral_gate_host_workspace(B, H, Dh, L, dt);
+    if (!ws || ws_bytes < need)
+        return set_error(HY_ERR_WORKSPACE, "%s: needs %zu workspace bytes, got %zu", who, need, ws ? ws_bytes : (size_t)0);
+    if (!aligned(ws, 256)) return set_error(HY_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", who);
+    const size_t esz = dt_size(dt);
+    const HostPlan p = host_plan(B, H, (size_t)Dh * L * esz, 1);
+    const size_t slot = (size_t)p.max_groups * Dh * L * esz;
+    const int n_in = x2 ? 2 : 1;
+    const int64_t nbins = L / 2 + 1;
+    auto describe = [&](int c, HostChunk &ch) {
+        int b0, nbc, h0, nhc;
+        host_chunk(p, B, H, c, b0, nbc, h0, nhc);
+        const size_t off = (((size_t)b0 * H + h0) * Dh) * L * esz;
+        ch.in_bytes = (size_t)nbc * nhc * Dh * L * esz;
+        ch.src[0] = reinterpret_cast<const char *>(x) + off;
+        if (x2) ch.src[1] = reinterpret_cast<const char *>(x2) + off;
+        ch.dst = reinterpret_cast<char *>(y) + off;
+        ch.out_bytes = ch.in_bytes;
+    };
+    auto compute = [&](int c, const void *const *din, void *dout, cudaStream_t s) {
+        int b0, nbc, h0, nhc;
+        host_chunk(p, B, H, c, b0, nbc, h0, nhc);
+        const hy_c32 *gc = g + (size_t)b0 * g_batch_stride + (size_t)h0 * nbins;
+        return spectral_gate(nbc, nhc, Dh, L, dt, din[0], gc, g_batch_stride, x2 ? din[1] : nullptr, dout, s);
+    };
+    return run_host_pipeline(n_in, p.nchunks, slot, slot, reinterpret_cast<char *>(ws), (cudaStream_t)stream,
+                             describe, compute, who);
 }

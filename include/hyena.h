@@ -221,6 +221,44 @@ hy_status spectral_gate(int B, int H, int Dh, int L, hy_dtype dt, const void *x,
                         void *stream);
 
 /* ------------------------------------------------------------------------
+ * Host-buffer variants -- the operator and the spectral gate above with the
+ * signals in HOST memory.  (The pages have no counterpart: this is the I/O
+ * runtime around the method.)
+ *
+ *   v, x[k], y (operator) and x, x2, y (gate) are host pointers with the
+ *   layouts of the device entry points; H / g and Dskip stay device pointers.
+ *   Use page-locked host memory (cudaHostAlloc / cudaHostRegister): with
+ *   pageable memory the copies still work but do not overlap.  Device
+ *   pointers for the signals are rejected (HY_ERR_INVALID_ARG).
+ *
+ *   The rows are cut into chunks of about 16 MB per signal (whole batches,
+ *   or runs of channels / heads within one batch; at least 8 rows on the
+ *   multi-pass path).  Chunk c is copied in on a library-owned copy stream,
+ *   computed on `stream` by the same kernels as the device entry point, and
+ *   copied out on a second library-owned copy stream, in a ring of 3 device
+ *   slots inside ws -- so the copy in of chunk c+1, the compute of chunk c
+ *   and the copy out of chunk c-1 overlap.  Results equal the device entry
+ *   point's bit for bit.
+ *
+ *   ws: device workspace of at least *_host_workspace() bytes, 256-byte
+ *   aligned, owned by the caller and not to be touched until `stream` has
+ *   passed the call.  The call only enqueues work and returns; `stream`
+ *   waits for the last copy out, so y is valid once `stream` is
+ *   synchronised.  The host buffers must stay valid until then.  The call
+ *   creates a few CUDA events (and, on the first call on a device, the two
+ *   copy streams); do not call it during stream capture.
+ * ---------------------------------------------------------------------- */
+size_t hyena_operator_host_workspace(int order, int B, int D, int L, hy_dtype dt);
+hy_status hyena_operator_host(int order, int B, int D, int L, hy_dtype dt, const void *v,
+                              const void *const *x, const hy_c32 *const *H,
+                              const float *const *Dskip, void *y, void *ws, size_t ws_bytes,
+                              void *stream);
+size_t spectral_gate_host_workspace(int B, int H, int Dh, int L, hy_dtype dt);
+hy_status spectral_gate_host(int B, int H, int Dh, int L, hy_dtype dt, const void *x,
+                             const hy_c32 *g, int64_t g_batch_stride, const void *x2, void *y,
+                             void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
  * Library state and errors
  * ---------------------------------------------------------------------- */
 /* Uploads the constant twiddle tables to the current device.  Called

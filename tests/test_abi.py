@@ -110,6 +110,28 @@ def test_filter_and_nd_validation(lib):
     assert lib.hyena_filter_gen(ctypes.byref(d), FAKE * 2, None) == 2
 
 
+def test_host_entry_validation_and_workspace(lib):
+    X = (ctypes.c_void_p * 2)(FAKE, FAKE)
+    H = (ctypes.c_void_p * 2)(FAKE, FAKE)
+    assert _err(lib, lib.hyena_operator_host(1, 1, 1, 64, 0, FAKE, X, H, None, FAKE * 2, None, 0, None), "order") == 2
+    assert _err(lib, lib.hyena_operator_host(2, 0, 1, 64, 0, FAKE, X, H, None, FAKE * 2, None, 0, None), "B, D, L") == 1
+    assert _err(lib, lib.hyena_operator_host(2, 1, 1, 64, 0, None, X, H, None, FAKE * 2, None, 0, None), "v is null") == 1
+    assert _err(lib, lib.hyena_operator_host(2, 1, 1, 64, 0, FAKE, None, H, None, FAKE * 2, None, 0, None), "null x") == 1
+    assert _err(lib, lib.hyena_operator_host(2, 1, 1, 64, 0, FAKE, X, H, None, FAKE * 2, None, 0, None), "workspace") == 3
+    assert _err(lib, lib.spectral_gate_host(0, 1, 1, 64, 0, FAKE, FAKE, 0, None, FAKE * 2, None, 0, None), "B, H") == 1
+    assert _err(lib, lib.spectral_gate_host(1, 1, 1, 64, 0, FAKE, FAKE, -1, None, FAKE * 2, None, 0, None), "stride") == 1
+    assert _err(lib, lib.spectral_gate_host(1, 1, 1, 64, 0, FAKE, FAKE, 0, None, FAKE * 2, None, 0, None), "workspace") == 3
+    # ring of 3 slots x (inputs + output), chunks of about 16 MB per signal:
+    # the order-2 bf16 operator B8 D768 L8192 moves one batch (12.6 MB) per chunk
+    assert lib.hyena_operator_host_workspace(2, 8, 768, 8192, 1) == 3 * 3 * 768 * 8192 * 2
+    # the spectral gate B4 H32 Dh64 L32768 bf16 moves 4 heads (16 MB) per chunk
+    assert lib.spectral_gate_host_workspace(4, 32, 64, 32768, 1) == 3 * 3 * 4 * 64 * 32768 * 2
+    # multi-pass: chunks of 8 rows of 2^20 plus the multi-pass workspace of 8 rows
+    assert lib.hyena_operator_host_workspace(3, 1, 256, 1 << 20, 0) == \
+        3 * 4 * 8 * (1 << 20) * 4 + lib.hyena_operator_workspace(3, 1, 8, 1 << 20, 0)
+    assert lib.hyena_operator_host_workspace(1, 8, 768, 8192, 1) == 0
+
+
 def test_binding_raises_named_errors(lib):
     with pytest.raises(hy.HyenaError) as ei:
         hy._check(lib.spectral_gate(1, 1, 1, 100, 1, FAKE, FAKE, 0, None, FAKE * 2, None))

@@ -299,7 +299,12 @@ def setup_nd(w, dev, hy, torch):
     def op():
         hy.hyena_nd_conv(u, H, y, H_batch_stride=D * S * S * (S // 2 + 1), gate=x1, ws=ws)
 
-    st.spectra, st.op = spectra, op
+    wsh = torch.empty(hy.nd_conv_host_workspace([g, g, g], B, D), dtype=torch.uint8, device=dev)
+
+    def host_op(hosts, out_h):
+        hy.hyena_nd_conv_host(hosts[0], H, out_h, H_batch_stride=D * S * S * (S // 2 + 1), gate=hosts[1], ws=wsh)
+
+    st.spectra, st.op, st.host_op = spectra, op, host_op
     st.inputs = [(u, w.v), (x1, w.xs[0])]
     st.output = y
     per_c = g * S * (S // 2 + 1) * 8

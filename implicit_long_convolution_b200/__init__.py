@@ -22,7 +22,8 @@ __all__ = [
     "hyena_filter_gen", "hyena_filter_spectrum", "filter_spectrum_workspace",
     "hyena_fftconv", "hyena_operator", "operator_workspace", "hyena_operator_noalloc", "hyena_nd_conv",
     "nd_conv_workspace", "spectral_gate", "operator_host_workspace", "hyena_operator_host",
-    "spectral_gate_host_workspace", "spectral_gate_host", "STATUS",
+    "spectral_gate_host_workspace", "spectral_gate_host", "nd_conv_host_workspace", "hyena_nd_conv_host",
+    "STATUS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhyena_b200.so")
@@ -94,6 +95,9 @@ def lib():
         "hyena_operator_host_workspace": (_SZ, [_I, _I, _I, _I, _I]),
         "hyena_operator_host": (_I, [_I, _I, _I, _I, _I, _VP, ctypes.POINTER(_VP), ctypes.POINTER(_VP),
                                      ctypes.POINTER(_VP), _VP, _VP, _SZ, _VP]),
+        "hyena_nd_conv_host_workspace": (_SZ, [_I, ctypes.POINTER(_I), _I, _I, _I]),
+        "hyena_nd_conv_host": (_I, [_I, ctypes.POINTER(_I), _I, _I, _I, _VP, _VP, _I64, _VP, _VP, _VP,
+                                    _VP, _SZ, _VP]),
         "spectral_gate_host_workspace": (_SZ, [_I, _I, _I, _I, _I]),
         "spectral_gate_host": (_I, [_I, _I, _I, _I, _I, _VP, _VP, _I64, _VP, _VP, _VP, _SZ, _VP]),
     }
@@ -260,4 +264,21 @@ def spectral_gate_host(x, g, y, *, x2=None, g_batch_stride: int = 0, ws=None, st
     wsb = ws.numel() * ws.element_size() if ws is not None else 0
     _check(lib().spectral_gate_host(B, Hh, Dh, L, _dt(x), _ptr(x), _ptr(g), g_batch_stride, _ptr(x2),
                                     _ptr(y), _ptr(ws), wsb, _stream(stream)))
+    return y
+
+
+def nd_conv_host_workspace(dims: Sequence[int], B: int, D: int, circular: bool = False) -> int:
+    return int(lib().hyena_nd_conv_host_workspace(3, _ints(dims), B, D, int(circular)))
+
+
+def hyena_nd_conv_host(u, H, y, *, H_batch_stride: int = 0, circular: bool = False, Dskip=None,
+                       gate=None, ws=None, stream=None):
+    """hyena_nd_conv with u, gate and y in (page-locked) host memory; H,
+    Dskip and ws on the device (see hyena.h)."""
+    B, D = u.shape[:2]
+    dims = list(u.shape[2:])
+    wsb = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib().hyena_nd_conv_host(len(dims), _ints(dims), B, D, int(circular), _ptr(u), _ptr(H),
+                                    H_batch_stride, _ptr(Dskip), _ptr(gate), _ptr(y), _ptr(ws), wsb,
+                                    _stream(stream)))
     return y

@@ -597,3 +597,60 @@ extern "C" hy_status spectral_gate_host(int B, int H, int Dh, int L, hy_dtype dt
     return run_host_pipeline(n_in, p.nchunks, slot, slot, reinterpret_cast<char *>(ws), (cudaStream_t)stream,
                              describe, compute, who);
 }
+
+extern "C" size_t hyena_nd_conv_host_workspace(int ndim, const int *dims, int B, int D, int circular) {
+    if (ndim != 3 || !dims || B < 1 || D < 1 || dims[0] < 1 || dims[1] < 1 || dims[2] < 1) return 0;
+    const size_t vox = (size_t)dims[0] * dims[1] * dims[2];
+    const HostPlan p = host_plan(B, D, vox * 4, 1);
+    const size_t chain = hyena_nd_conv_workspace(ndim, dims, 1, (int)p.max_groups, circular);
+    return host_ring_bytes(2, (size_t)p.max_groups * vox * 4) + round256(chain);
+}
+
+extern "C" hy_status hyena_nd_conv_host(int ndim, const int *dims, int B, int D, int circular, const float *u,
+                                        const hy_c32 *H, int64_t H_batch_stride, const float *Dskip,
+                                        const float *gate, float *y, void *ws, size_t ws_bytes, void *stream) {
+    clear_error();
+    const char *who = "hyena_nd_conv_host";
+    if (ndim != 3) return set_error(HY_ERR_UNSUPPORTED, "%s: only ndim = 3 is built", who);
+    if (!dims || !H) return set_error(HY_ERR_INVALID_ARG, "%s: null pointer", who);
+    if (B < 1 || D < 1 || H_batch_stride < 0) return set_error(HY_ERR_INVALID_ARG, "%s: bad B, D or stride", who);
+    for (int i = 0; i < 3; ++i)
+        if (dims[i] < 1) return set_error(HY_ERR_INVALID_ARG, "%s: bad grid", who);
+    hy_status st;
+    if ((st = check_host_ptr(u, who, "u")) != HY_OK || (st = check_host_ptr(y, who, "y")) != HY_OK) return st;
+    if (gate && (st = check_host_ptr(gate, who, "gate")) != HY_OK) return st;
+    const size_t need = hyena_nd_conv_host_workspace(ndim, dims, B, D, circular);
+    if (!ws || ws_bytes < need)
+        return set_error(HY_ERR_WORKSPACE, "%s: needs %zu workspace bytes, got %zu", who, need, ws ? ws_bytes : (size_t)0);
+    if (!aligned(ws, 256)) return set_error(HY_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", who);
+    const size_t vox = (size_t)dims[0] * dims[1] * dims[2];
+    const HostPlan p = host_plan(B, D, vox * 4, 1);
+    const size_t slot = (size_t)p.max_groups * vox * 4;
+    const int n_in = gate ? 2 : 1;
+    char *ring = reinterpret_cast<char *>(ws);
+    char *chain_ws = ring + host_ring_bytes(2, slot);
+    const size_t chain_bytes = ws_bytes - host_ring_bytes(2, slot);
+    int S[3];
+    for (int i = 0; i < 3; ++i) S[i] = circular ? dims[i] : 2 * dims[i];
+    const size_t spec_per_channel = (size_t)S[0] * S[1] * (S[2] / 2 + 1);
+    auto describe = [&](int c, HostChunk &ch) {
+        int b0, nbc, d0, ndc;
+        host_chunk(p, B, D, c, b0, nbc, d0, ndc);
+        const size_t off = ((size_t)b0 * D + d0) * vox;
+        ch.in_bytes = (size_t)nbc * ndc * vox * 4;
+        ch.src[0] = u + off;
+        if (gate) ch.src[1] = gate + off;
+        ch.dst = y + off;
+        ch.out_bytes = ch.in_bytes;
+    };
+    auto compute = [&](int c, const void *const *din, void *dout, cudaStream_t s) {
+        int b0, nbc, d0, ndc;
+        host_chunk(p, B, D, c, b0, nbc, d0, ndc);
+        const hy_c32 *Hc = H + (size_t)b0 * H_batch_stride + (size_t)d0 * spec_per_channel;
+        return hyena_nd_conv(ndim, dims, nbc, ndc, circular, reinterpret_cast<const float *>(din[0]), Hc,
+                             H_batch_stride, Dskip ? Dskip + d0 : nullptr,
+                             gate ? reinterpret_cast<const float *>(din[1]) : nullptr,
+                             reinterpret_cast<float *>(dout), chain_bytes ? chain_ws : nullptr, chain_bytes, s);
+    };
+    return run_host_pipeline(n_in, p.nchunks, slot, slot, ring, (cudaStream_t)stream, describe, compute, who);
+}

@@ -221,19 +221,20 @@ hy_status spectral_gate(int B, int H, int Dh, int L, hy_dtype dt, const void *x,
                         void *stream);
 
 /* ------------------------------------------------------------------------
- * Host-buffer variants -- the operator and the spectral gate above with the
- * signals in HOST memory.  (The pages have no counterpart: this is the I/O
+ * Host-buffer variants -- the operator, the N-D convolution and the
+ * spectral gate above with the signals in HOST memory.  (The pages have no counterpart: this is the I/O
  * runtime around the method.)
  *
- *   v, x[k], y (operator) and x, x2, y (gate) are host pointers with the
- *   layouts of the device entry points; H / g and Dskip stay device pointers.
+ *   v, x[k], y (operator), u, gate, y (N-D) and x, x2, y (gate) are host
+ *   pointers with the layouts of the device entry points; H / g and Dskip
+ *   stay device pointers.
  *   Use page-locked host memory (cudaHostAlloc / cudaHostRegister): with
  *   pageable memory the copies still work but do not overlap.  Device
  *   pointers for the signals are rejected (HY_ERR_INVALID_ARG).
  *
- *   The rows are cut into chunks of about 16 MB per signal (whole batches,
- *   or runs of channels / heads within one batch; at least 8 rows on the
- *   multi-pass path).  Chunk c is copied in on a library-owned copy stream,
+ *   The rows (N-D: slabs) are cut into chunks of about 16 MB per signal
+ *   (whole batches, or runs of channels / heads within one batch; at least
+ *   8 rows on the multi-pass path).  Chunk c is copied in on a library-owned copy stream,
  *   computed on `stream` by the same kernels as the device entry point, and
  *   copied out on a second library-owned copy stream, in a ring of 3 device
  *   slots inside ws -- so the copy in of chunk c+1, the compute of chunk c
@@ -253,6 +254,11 @@ hy_status hyena_operator_host(int order, int B, int D, int L, hy_dtype dt, const
                               const void *const *x, const hy_c32 *const *H,
                               const float *const *Dskip, void *y, void *ws, size_t ws_bytes,
                               void *stream);
+size_t hyena_nd_conv_host_workspace(int ndim, const int *dims, int B, int D, int circular);
+hy_status hyena_nd_conv_host(int ndim, const int *dims, int B, int D, int circular,
+                             const float *u, const hy_c32 *H, int64_t H_batch_stride,
+                             const float *Dskip, const float *gate, float *y, void *ws,
+                             size_t ws_bytes, void *stream);
 size_t spectral_gate_host_workspace(int B, int H, int Dh, int L, hy_dtype dt);
 hy_status spectral_gate_host(int B, int H, int Dh, int L, hy_dtype dt, const void *x,
                              const hy_c32 *g, int64_t g_batch_stride, const void *x2, void *y,

@@ -130,6 +130,16 @@ def test_host_entry_validation_and_workspace(lib):
     assert lib.hyena_operator_host_workspace(3, 1, 256, 1 << 20, 0) == \
         3 * 4 * 8 * (1 << 20) * 4 + lib.hyena_operator_workspace(3, 1, 8, 1 << 20, 0)
     assert lib.hyena_operator_host_workspace(1, 8, 768, 8192, 1) == 0
+    dims = (ctypes.c_int * 3)(64, 64, 64)
+    # 3-D: 16 slabs of 64^3 fp32 per chunk, plus the N-D workspace of 16 slabs
+    assert lib.hyena_nd_conv_host_workspace(3, dims, 2, 128, 0) == \
+        3 * 3 * 16 * 64 ** 3 * 4 + lib.hyena_nd_conv_workspace(3, dims, 1, 16, 0)
+    assert _err(lib, lib.hyena_nd_conv_host(2, dims, 1, 1, 0, FAKE, FAKE, 0, None, None, FAKE * 2, None, 0, None),
+                "ndim") == 2
+    assert _err(lib, lib.hyena_nd_conv_host(3, dims, 1, 1, 0, FAKE, FAKE, -1, None, None, FAKE * 2, None, 0, None),
+                "stride") == 1
+    assert _err(lib, lib.hyena_nd_conv_host(3, dims, 1, 1, 0, FAKE, FAKE, 0, None, None, FAKE * 2, None, 0, None),
+                "workspace") == 3
 
 
 def test_binding_raises_named_errors(lib):

@@ -3,7 +3,7 @@ signals in page-locked host memory, copied in, computed and copied out chunk
 by chunk on three streams.  Each chunk runs the device entry point's kernels
 on a subset of rows, so the results must equal the device path bit for bit;
 the shapes make several chunks, more than the 3 ring slots, on the on-chip
-and the multi-pass operator and on the gate."""
+and the multi-pass operator, the N-D convolution and the gate."""
 import numpy as np
 import pytest
 
@@ -80,6 +80,45 @@ def test_spectral_gate_host_matches_device():
     yh = torch.empty(x.shape, dtype=x.dtype).pin_memory()
     ws = torch.empty(hy.spectral_gate_host_workspace(B, Hh, Dh, L, hy.HY_BF16), dtype=torch.uint8, device="cuda")
     hy.spectral_gate_host(xh, g, yh, x2=x2h, g_batch_stride=Hh * (M + 1), ws=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(yh, y_dev.cpu())
+
+
+def test_nd_conv_host_matches_device():
+    B, D, g = 2, 40, 32                    # 128 KB slabs: 128 per chunk would be whole batches
+    S = 2 * g
+    rng = np.random.default_rng(12)
+    nb = S // 2 + 1
+    H = torch.from_numpy((rng.standard_normal((B, D, S, S, nb)) + 1j * rng.standard_normal((B, D, S, S, nb)))
+                         .astype(np.complex64) * 1e-3).cuda()
+    u = torch.randn((B, D, g, g, g), device="cuda")
+    x1 = torch.randn_like(u)
+    dsk = f32_dev(rng.standard_normal(D).astype(np.float32))
+    stride = D * S * S * nb
+    y_dev = torch.empty_like(u)
+    wsd = torch.empty(hy.nd_conv_workspace([g, g, g], B, D), dtype=torch.uint8, device="cuda")
+    hy.hyena_nd_conv(u, H, y_dev, H_batch_stride=stride, Dskip=dsk, gate=x1, ws=wsd)
+    yh = torch.empty(u.shape).pin_memory()
+    ws = torch.empty(hy.nd_conv_host_workspace([g, g, g], B, D), dtype=torch.uint8, device="cuda")
+    hy.hyena_nd_conv_host(_pinned(u), H, yh, H_batch_stride=stride, Dskip=dsk, gate=_pinned(x1), ws=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(yh, y_dev.cpu())
+
+
+def test_nd_conv_host_channel_chunks():
+    B, D, g = 2, 24, 64                    # 1 MB slabs: 16 per chunk, 2 chunks per batch
+    S = 2 * g
+    rng = np.random.default_rng(13)
+    nb = S // 2 + 1
+    H = torch.from_numpy((rng.standard_normal((D, S, S, nb)) + 1j * rng.standard_normal((D, S, S, nb)))
+                         .astype(np.complex64) * 1e-3).cuda()
+    u = torch.randn((B, D, g, g, g), device="cuda")
+    y_dev = torch.empty_like(u)
+    wsd = torch.empty(hy.nd_conv_workspace([g, g, g], B, D), dtype=torch.uint8, device="cuda")
+    hy.hyena_nd_conv(u, H, y_dev, ws=wsd)
+    yh = torch.empty(u.shape).pin_memory()
+    ws = torch.empty(hy.nd_conv_host_workspace([g, g, g], B, D), dtype=torch.uint8, device="cuda")
+    hy.hyena_nd_conv_host(_pinned(u), H, yh, ws=ws)
     torch.cuda.synchronize()
     assert torch.equal(yh, y_dev.cpu())
 

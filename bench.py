@@ -570,6 +570,57 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_projection(args):
+    """The input projection at the operator workload's width (B8 L8192,
+    768 -> 2 x 768 channels, bf16): one bf16 GEMM per projection plus the
+    bias pass, timed with CUDA events; TFLOP/s against the measured bf16
+    GEMM peak (burst)."""
+    import torch
+    import implicit_long_convolution_b200 as hy
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    B, L, C, D, n_out = 8, 8192, 768, 768, 2
+    g = torch.Generator(device=dev)
+    g.manual_seed(rank_seed("c2", rank))
+    x = torch.randn((B, L, C), device=dev, generator=g).to(torch.bfloat16)
+    W = (torch.randn((n_out * D, C), device=dev, generator=g) / C ** 0.5).to(torch.bfloat16)
+    bias = torch.randn(n_out * D, device=dev, generator=g) * 0.1
+    outs = [torch.empty((B, D, L), dtype=torch.bfloat16, device=dev) for _ in range(n_out)]
+    ws = torch.empty(hy.projection_workspace(), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    run = lambda: hy.hyena_projection(x, W, outs, bias=bias, ws=ws)
+    for _ in range(max(3, args.warmup)):
+        run()
+    steps = args.steps if args.steps > 0 else 200
+    torch.cuda.synchronize()
+    barrier(world)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        run()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(t0.elapsed_time(t1), world) / steps
+    flops = 2.0 * B * L * C * n_out * D
+    tf = world * flops / (ms / 1e3) / 1e12
+    peak = None
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            peak = float(json.load(f)["bf16_tflops"])
+    if rank == 0:
+        print(json.dumps({
+            "metric": "input projection TFLOP/s (B8 L8192, 768 -> 2 x 768, bf16, channel-major outputs + bias)",
+            "value": round(tf, 1), "unit": "TFLOP/s", "n_gpus": world, "steps": steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16 (fp32 accumulate)", "data": "synthetic",
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(tf / world / peak, 4) if peak else None, "traffic": None},
+            "config": {"workload": "hyena input projection at the order-2 operator width",
+                       "B": B, "L": L, "C": C, "D": D, "n_out": n_out}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -579,6 +630,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(DESCR), default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--projection", action="store_true",
+                    help="time the input projection at the operator workload's width instead")
     ap.add_argument("--channels", type=int, default=0,
                     help="override the channel count D (smaller cases for profiler captures)")
     args = ap.parse_args()
@@ -591,6 +644,9 @@ def main():
         return
     if args.warmup < 3:
         args.warmup = 3
+    if args.projection:
+        run_projection(args)
+        return
     run_ours(args)
 
 

@@ -23,7 +23,7 @@ __all__ = [
     "hyena_fftconv", "hyena_operator", "operator_workspace", "hyena_operator_noalloc", "hyena_nd_conv",
     "nd_conv_workspace", "spectral_gate", "operator_host_workspace", "hyena_operator_host",
     "spectral_gate_host_workspace", "spectral_gate_host", "nd_conv_host_workspace", "hyena_nd_conv_host",
-    "STATUS",
+    "projection_workspace", "hyena_projection", "STATUS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhyena_b200.so")
@@ -95,6 +95,8 @@ def lib():
         "hyena_operator_host_workspace": (_SZ, [_I, _I, _I, _I, _I]),
         "hyena_operator_host": (_I, [_I, _I, _I, _I, _I, _VP, ctypes.POINTER(_VP), ctypes.POINTER(_VP),
                                      ctypes.POINTER(_VP), _VP, _VP, _SZ, _VP]),
+        "hyena_projection_workspace": (_SZ, []),
+        "hyena_projection": (_I, [_I, _I, _I, _I, _I, _I, _VP, _VP, _VP, ctypes.POINTER(_VP), _VP, _SZ, _VP]),
         "hyena_nd_conv_host_workspace": (_SZ, [_I, ctypes.POINTER(_I), _I, _I, _I]),
         "hyena_nd_conv_host": (_I, [_I, ctypes.POINTER(_I), _I, _I, _I, _VP, _VP, _I64, _VP, _VP, _VP,
                                     _VP, _SZ, _VP]),
@@ -282,3 +284,19 @@ def hyena_nd_conv_host(u, H, y, *, H_batch_stride: int = 0, circular: bool = Fal
                                     H_batch_stride, _ptr(Dskip), _ptr(gate), _ptr(y), _ptr(ws), wsb,
                                     _stream(stream)))
     return y
+
+
+def projection_workspace() -> int:
+    return int(lib().hyena_projection_workspace())
+
+
+def hyena_projection(x, W, outs: Sequence, *, bias=None, ws=None, stream=None):
+    """out_k[b, d, l] = bias[kD + d] + sum_c W[kD + d, c] x[b, l, c] for the
+    n_out = len(outs) projections (device tensors; see hyena.h)."""
+    B, L, C = x.shape
+    n_out = len(outs)
+    D = outs[0].shape[1]
+    wsb = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib().hyena_projection(B, L, C, D, n_out, _dt(x), _ptr(x), _ptr(W), _ptr(bias), _ptrs(outs),
+                                  _ptr(ws), wsb, _stream(stream)))
+    return outs

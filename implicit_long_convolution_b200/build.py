@@ -63,7 +63,7 @@ def build(force: bool = False, jobs: int | None = None) -> str:
         return LIB
     tmp = LIB + ".tmp.%d" % os.getpid()
     cmd = [_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared",
-           "-Xcompiler", "-fPIC", "-cudart", "static", *objs, "-o", tmp]
+           "-Xcompiler", "-fPIC", "-cudart", "static", *objs, "-ldl", "-o", tmp]
     subprocess.check_call(cmd)
     os.replace(tmp, LIB)
     return LIB

@@ -4,7 +4,7 @@
  *
  * Pages cited (title, section):
  *   [HN] "Hyena: 암묵적 장거리 컨볼루션으로 어텐션을 완전 대체한 서브-이차 모델" --
- *        아키텍처 상세: step 2 (h(t) = FFN(pos_enc(t))·w(t), w(t) = e^{-αt}),
+ *        아키텍처 상세: step 1 (v, x_1, …, x_{N-1} = split(W_proj·x)), step 2 (h(t) = FFN(pos_enc(t))·w(t), w(t) = e^{-αt}),
  *        step 3 (y = x_{N-1} ⊙ (h_{N-1} * (x_{N-2} ⊙ (h_{N-2} * (…))))), and the
  *        ImplicitFilter / hyena_operator code sketch.
  *   [ES] "4. Hyena 상세" -- 어떻게 동작하나요? (filter generator: small MLP with
@@ -219,6 +219,30 @@ hy_status hyena_nd_conv(int ndim, const int *dims, int B, int D, int circular, c
 hy_status spectral_gate(int B, int H, int Dh, int L, hy_dtype dt, const void *x,
                         const hy_c32 *g, int64_t g_batch_stride, const void *x2, void *y,
                         void *stream);
+
+/* ------------------------------------------------------------------------
+ * Input projection  ([HN] 아키텍처 상세, step 1: v, x_1, …, x_{N-1} =
+ * split(W_proj · x), a learnable linear map)
+ *
+ *   out_k[b, d, l] = bias[k·D + d] + Σ_c W[k·D + d, c] · x[b, l, c]
+ *   for k = 0 .. n_out-1 (n_out = N for an order-N operator: v, x_1, …),
+ *   d < D, l < L, c < C.
+ *   x: device (B, L, C) token-major activations; W: device (n_out·D, C)
+ *   row-major (the PyTorch Linear layout); bias: device fp32 (n_out·D) or
+ *   NULL; out: host array of n_out device pointers, each (B, D, L) -- the
+ *   channel-major layout hyena_operator reads, no transpose needed.
+ *   x, W, out share dt.  bf16: tensor-core GEMM with fp32 accumulation,
+ *   the product rounded to bf16, then the bias added (a second pass over
+ *   the outputs) and rounded again; fp32: fp32 arithmetic (no TF32).  The GEMM is cuBLASLt's, loaded on the first
+ *   call (HY_ERR_UNSUPPORTED if it cannot be loaded).
+ *   x, W, out 16-byte aligned and C·sizeof(dt) a multiple of 16;
+ *   ws: device workspace of hyena_projection_workspace() bytes, 256-byte
+ *   aligned.
+ * ---------------------------------------------------------------------- */
+size_t hyena_projection_workspace(void);
+hy_status hyena_projection(int B, int L, int C, int D, int n_out, hy_dtype dt, const void *x,
+                           const void *W, const float *bias, void *const *out, void *ws,
+                           size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
  * Host-buffer variants -- the operator, the N-D convolution and the

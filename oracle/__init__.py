@@ -17,7 +17,7 @@ Two layers:
 
 Pages cited (title, section):
   [HN] "Hyena: 암묵적 장거리 컨볼루션으로 어텐션을 완전 대체한 서브-이차 모델",
-       아키텍처 상세 (steps 2 and 3) and its ImplicitFilter / hyena_operator sketch.
+       아키텍처 상세 (steps 1, 2 and 3) and its ImplicitFilter / hyena_operator sketch.
   [ES] "4. Hyena 상세", 어떻게 동작하나요?.
   [ND] "Native Multi-Dimensional Subquadratic Operators via Input Dependent Long
        Convolutions", 방법론: HyenaND (네이티브 ND 합성곱, 경계 처리).
@@ -52,6 +52,7 @@ PINS = {
     "gate_kernel": "g=1 delta, shift gate, constant gate, numpy.fft.irfft",
     "circular_conv": "shift gate, Parseval, numpy.fft circular convolution",
     "fft_*": "matched against the direct functions above on sampled outputs",
+    "projection": "identity weights give the transposed input, zero weights the bias, linearity",
 }
 
 
@@ -108,6 +109,25 @@ def threads() -> int:
     """OpenMP threads the oracle uses (OMP_NUM_THREADS, else the affinity set)."""
     env = os.environ.get("OMP_NUM_THREADS")
     return int(env) if env else len(os.sched_getaffinity(0))
+
+
+# --------------------------------------------------------------------------
+# input projection ([HN] 아키텍처 상세, step 1: v, x_1, ... = split(W_proj x))
+# --------------------------------------------------------------------------
+
+def projection(x, W, bias, n_out: int) -> list:
+    """out_k[b, d, l] = bias[kD + d] + sum_c W[kD + d, c] x[b, l, c], float64.
+
+    x: (B, L, C); W: (n_out*D, C); bias: (n_out*D,) or None.  Returns the
+    n_out channel-major (B, D, L) arrays (the split of W_proj x)."""
+    x = np.asarray(x, np.float64)
+    W = np.asarray(W, np.float64)
+    D = W.shape[0] // n_out
+    assert W.shape[0] == n_out * D and W.shape[1] == x.shape[2]
+    full = np.matmul(x, W.T)                        # (B, L, n_out*D), a library matmul
+    if bias is not None:
+        full = full + np.asarray(bias, np.float64)[None, None, :]
+    return [np.ascontiguousarray(full[:, :, k * D:(k + 1) * D].transpose(0, 2, 1)) for k in range(n_out)]
 
 
 # --------------------------------------------------------------------------

@@ -406,3 +406,27 @@ def test_fft_spectrum_matches_direct():
     rng = np.random.default_rng(17)
     h = rng.standard_normal((4, 40))
     np.testing.assert_allclose(oracle.fft_spectrum(h), oracle.dft_real_rows(h, 128), atol=1e-11)
+
+
+def test_projection_identity_zero_and_linearity():
+    """Input projection: identity blocks return the input transposed to
+    channel-major (times the block's scale), zero weights return the bias on
+    every position, and the map is linear in x."""
+    rng = np.random.default_rng(18)
+    B, L, C = 2, 7, 5
+    x = rng.standard_normal((B, L, C))
+    W = np.concatenate([np.eye(C), 3.0 * np.eye(C)])          # n_out = 2, D = C
+    v, x1 = oracle.projection(x, W, None, 2)
+    assert v.shape == (B, C, L)
+    np.testing.assert_array_equal(v, x.transpose(0, 2, 1))
+    np.testing.assert_array_equal(x1, 3.0 * x.transpose(0, 2, 1))
+    bias = rng.standard_normal(3 * 4)
+    outs = oracle.projection(x, np.zeros((12, C)), bias, 3)
+    for k, o in enumerate(outs):
+        np.testing.assert_array_equal(o, np.broadcast_to(bias[4 * k:4 * k + 4][None, :, None], (B, 4, L)))
+    W2 = rng.standard_normal((8, C))
+    x2 = rng.standard_normal((B, L, C))
+    a = oracle.projection(x + 2 * x2, W2, None, 2)
+    b1, b2 = oracle.projection(x, W2, None, 2), oracle.projection(x2, W2, None, 2)
+    for k in range(2):
+        np.testing.assert_allclose(a[k], b1[k] + 2 * b2[k], rtol=1e-12, atol=1e-12)

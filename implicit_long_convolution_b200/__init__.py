@@ -23,7 +23,8 @@ __all__ = [
     "hyena_fftconv", "hyena_operator", "operator_workspace", "hyena_operator_noalloc", "hyena_nd_conv",
     "nd_conv_workspace", "spectral_gate", "operator_host_workspace", "hyena_operator_host",
     "spectral_gate_host_workspace", "spectral_gate_host", "nd_conv_host_workspace", "hyena_nd_conv_host",
-    "projection_workspace", "hyena_projection", "STATUS",
+    "projection_workspace", "hyena_projection", "operator_backward_workspace", "hyena_operator_backward",
+    "STATUS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhyena_b200.so")
@@ -95,6 +96,10 @@ def lib():
         "hyena_operator_host_workspace": (_SZ, [_I, _I, _I, _I, _I]),
         "hyena_operator_host": (_I, [_I, _I, _I, _I, _I, _VP, ctypes.POINTER(_VP), ctypes.POINTER(_VP),
                                      ctypes.POINTER(_VP), _VP, _VP, _SZ, _VP]),
+        "hyena_operator_backward_workspace": (_SZ, [_I, _I, _I, _I, _I]),
+        "hyena_operator_backward": (_I, [_I, _I, _I, _I, _I, _VP, ctypes.POINTER(_VP), ctypes.POINTER(_VP),
+                                         ctypes.POINTER(_VP), _VP, _VP, ctypes.POINTER(_VP), ctypes.POINTER(_VP),
+                                         ctypes.POINTER(_VP), _VP, _SZ, _VP]),
         "hyena_projection_workspace": (_SZ, []),
         "hyena_projection": (_I, [_I, _I, _I, _I, _I, _I, _VP, _VP, _VP, ctypes.POINTER(_VP), _VP, _SZ, _VP]),
         "hyena_nd_conv_host_workspace": (_SZ, [_I, ctypes.POINTER(_I), _I, _I, _I]),
@@ -300,3 +305,22 @@ def hyena_projection(x, W, outs: Sequence, *, bias=None, ws=None, stream=None):
     _check(lib().hyena_projection(B, L, C, D, n_out, _dt(x), _ptr(x), _ptr(W), _ptr(bias), _ptrs(outs),
                                   _ptr(ws), wsb, _stream(stream)))
     return outs
+
+
+def operator_backward_workspace(order: int, B: int, D: int, L: int, dtype_code: int) -> int:
+    return int(lib().hyena_operator_backward_workspace(order, B, D, L, dtype_code))
+
+
+def hyena_operator_backward(v, xs: Sequence, Hs: Sequence, dy, dv, dxs: Sequence, *,
+                            Dskips: Optional[Sequence] = None, dhs: Optional[Sequence] = None,
+                            dDs: Optional[Sequence] = None, ws=None, stream=None):
+    """Gradients of the operator (see hyena.h): dv, dxs[k] (like v), dhs[k]
+    (fp32 (D, L)) and dDs[k] (fp32 (D,)); dhs / dDs may be None."""
+    B, D, L = v.shape
+    order = len(xs) + 1
+    wsb = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib().hyena_operator_backward(
+        order, B, D, L, _dt(v), _ptr(v), _ptrs(xs), _ptrs(Hs), _ptrs(Dskips) if Dskips is not None else None,
+        _ptr(dy), _ptr(dv), _ptrs(dxs), _ptrs(dhs) if dhs is not None else None,
+        _ptrs(dDs) if dDs is not None else None, _ptr(ws), wsb, _stream(stream)))
+    return dv

@@ -654,3 +654,132 @@ extern "C" hy_status hyena_nd_conv_host(int ndim, const int *dims, int B, int D,
     };
     return run_host_pipeline(n_in, p.nchunks, slot, slot, ring, (cudaStream_t)stream, describe, compute, who);
 }
+
+// ----------------------------------------------------------------------------
+// Backward pass of the 1-D operator (see include/hyena.h and backward.cu):
+// forward recompute, then per order from the last: dx_k, the reversed e_k,
+// dD_k, dh_k (a convolution of z_{k-1} with per-row spectra of the reversed
+// e_k, summed over the batch) and the next gradient (a convolution of the
+// reversed e_k with h_k, read back reversed, plus D_k e_k).  Every
+// convolution is the forward path's (run_chain); intermediates are fp32 rows
+// in the workspace.
+// ----------------------------------------------------------------------------
+namespace {
+
+struct BwLayout {
+    size_t row;            // bytes of one fp32 signal (all rows)
+    size_t c, z, g, er, r, w, es, chain;   // offsets
+    size_t chain_bytes, total;
+};
+
+BwLayout bw_layout(int K, int B, int D, int L) {
+    BwLayout p{};
+    const int64_t R = (int64_t)B * D;
+    const int64_t M = spectrum_m(L);
+    p.row = round256((size_t)R * L * 4);
+    size_t o = 0;
+    p.c = o; o += (size_t)K * p.row;
+    p.z = o; o += (size_t)K * p.row;
+    p.g = o; o += p.row;
+    p.er = o; o += p.row;
+    p.r = o; o += p.row;
+    p.w = o; o += p.row;
+    p.es = o; o += round256((size_t)R * (M + 1) * 8);
+    const int Lc = L;
+    size_t ch = hyena_operator_workspace(2, B, D, L, HY_F32);
+    const size_t ch2 = hyena_operator_workspace(2, 1, (int)R, L, HY_F32);
+    const size_t ch3 = hyena_filter_spectrum_workspace(R, 1, &Lc, 0);
+    ch = ch > ch2 ? ch : ch2;
+    ch = ch > ch3 ? ch : ch3;
+    p.chain = o;
+    p.chain_bytes = round256(ch);
+    o += p.chain_bytes;
+    p.total = o;
+    return p;
+}
+
+}  // namespace
+
+extern "C" size_t hyena_operator_backward_workspace(int order, int B, int D, int L, hy_dtype dt) {
+    if (order < 2 || order - 1 > kMaxOrders || B < 1 || D < 1 || L < 1 || (dt != HY_F32 && dt != HY_BF16)) return 0;
+    if ((int64_t)B * D > 0x7fffffffLL) return 0;
+    return bw_layout(order - 1, B, D, L).total;
+}
+
+extern "C" hy_status hyena_operator_backward(int order, int B, int D, int L, hy_dtype dt, const void *v,
+                                             const void *const *x, const hy_c32 *const *H,
+                                             const float *const *Dskip, const void *dy, void *dv,
+                                             void *const *dx, float *const *dh, float *const *dD, void *ws,
+                                             size_t ws_bytes, void *stream) {
+    clear_error();
+    const char *who = "hyena_operator_backward";
+    if (order < 2 || order - 1 > kMaxOrders)
+        return set_error(HY_ERR_UNSUPPORTED, "%s: order must be 2..%d", who, kMaxOrders + 1);
+    if (B < 1 || D < 1 || L < 1) return set_error(HY_ERR_INVALID_ARG, "%s: B, D, L must be >= 1", who);
+    if (dt != HY_F32 && dt != HY_BF16) return set_error(HY_ERR_INVALID_ARG, "%s: unknown dtype", who);
+    if (!v || !dy || !dv || !x || !H || !dx) return set_error(HY_ERR_INVALID_ARG, "%s: null pointer", who);
+    const int K = order - 1;
+    const size_t esz = dt_size(dt);
+    const size_t al = (L % 2 == 0) ? 2 * esz : esz;
+    if (!aligned(v, al) || !aligned(dy, al) || !aligned(dv, al))
+        return set_error(HY_ERR_INVALID_ARG, "%s: signals must be %zu-byte aligned", who, al);
+    for (int k = 0; k < K; ++k) {
+        if (!x[k] || !H[k] || !dx[k]) return set_error(HY_ERR_INVALID_ARG, "%s: null x, H or dx of order %d", who, k);
+        if (!aligned(x[k], al) || !aligned(dx[k], al) || !aligned(H[k], 8))
+            return set_error(HY_ERR_INVALID_ARG, "%s: order %d misaligned", who, k);
+    }
+    if ((int64_t)B * D > 0x7fffffffLL) return set_error(HY_ERR_UNSUPPORTED, "%s: too many rows", who);
+    const BwLayout lay = bw_layout(K, B, D, L);
+    if (!ws || ws_bytes < lay.total)
+        return set_error(HY_ERR_WORKSPACE, "%s: needs %zu workspace bytes, got %zu", who, lay.total, ws ? ws_bytes : (size_t)0);
+    if (!aligned(ws, 256)) return set_error(HY_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", who);
+    cudaStream_t s = (cudaStream_t)stream;
+    char *base = reinterpret_cast<char *>(ws);
+    auto buf = [&](size_t off) { return reinterpret_cast<float *>(base + off); };
+    float *c[kMaxOrders], *z[kMaxOrders];
+    for (int k = 0; k < K; ++k) {
+        c[k] = buf(lay.c + (size_t)k * lay.row);
+        z[k] = buf(lay.z + (size_t)k * lay.row);
+    }
+    float *g = buf(lay.g), *er = buf(lay.er), *r = buf(lay.r), *w = buf(lay.w);
+    hy_c32 *es = reinterpret_cast<hy_c32 *>(base + lay.es);
+    void *chain = base + lay.chain;
+    const int64_t R = (int64_t)B * D;
+    const int64_t n = R * L;
+    hy_status st = prologue(s);
+    if (st != HY_OK) return st;
+    // ---- forward recompute: z_0 = v; c_k = h_k * z_{k-1} + D_k z_{k-1}; z_k = x_k ⊙ c_k
+    if ((st = bw_to_f32(v, dt, z[0], n, s)) != HY_OK) return st;
+    for (int k = 0; k < K; ++k) {
+        const void *nog[1] = {nullptr};
+        const hy_c32 *Hk[1] = {H[k]};
+        const float *Sk[1] = {Dskip ? Dskip[k] : nullptr};
+        if ((st = run_chain(1, B, D, L, HY_F32, z[k], nog, Hk, Sk, c[k], chain, lay.chain_bytes, s, who)) != HY_OK)
+            return st;
+        if (k + 1 < K && (st = bw_gate(x[k], dt, c[k], z[k + 1], n, s)) != HY_OK) return st;
+    }
+    // ---- backward from the last order
+    if ((st = bw_to_f32(dy, dt, g, n, s)) != HY_OK) return st;
+    for (int k = K - 1; k >= 0; --k) {
+        if (dD && dD[k] && (st = bw_dD(g, x[k], dt, z[k], dD[k], B, D, L, s)) != HY_OK) return st;
+        if ((st = bw_dx_e(g, c[k], x[k], dt, dx[k], er, R, L, s)) != HY_OK) return st;
+        const void *nog[1] = {nullptr};
+        const float *nos[1] = {nullptr};
+        if (dh && dh[k]) {
+            // w = z_{k-1} * reverse(e_k) with each row's own spectrum, then
+            // dh_k[d][τ] = Σ_b w[b, d][L-1-τ]
+            const int Lr = L;
+            if ((st = hyena_filter_spectrum(R, 1, &Lr, 0, er, es, chain, lay.chain_bytes, s)) != HY_OK) return st;
+            const hy_c32 *Es[1] = {es};
+            if ((st = run_chain(1, 1, (int)R, L, HY_F32, z[k], nog, Es, nos, w, chain, lay.chain_bytes, s, who)) != HY_OK)
+                return st;
+            if ((st = bw_dh(w, dh[k], B, D, L, s)) != HY_OK) return st;
+        }
+        // g_{k-1}[s] = (h_k * reverse(e_k))[L-1-s] + D_k e_k[s]
+        const hy_c32 *Hk[1] = {H[k]};
+        if ((st = run_chain(1, B, D, L, HY_F32, er, nog, Hk, nos, r, chain, lay.chain_bytes, s, who)) != HY_OK)
+            return st;
+        if ((st = bw_next_g(r, g, x[k], dt, Dskip ? Dskip[k] : nullptr, R, D, L, s)) != HY_OK) return st;
+    }
+    return bw_from_f32(g, dt, dv, n, s);
+}

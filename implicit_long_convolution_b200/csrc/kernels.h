@@ -42,6 +42,18 @@ hy_status launch_long_spectrum(int64_t rows, int64_t L, int log_mc, const float 
 size_t noalloc_scratch_bytes();
 hy_status launch_long_conv_noalloc(const LongConvArgs &a, cudaStream_t s);
 
+// backward-pass element-wise and reduction kernels (backward.cu)
+hy_status bw_to_f32(const void *src, hy_dtype dt, float *dst, int64_t n, cudaStream_t s);
+hy_status bw_from_f32(const float *src, hy_dtype dt, void *dst, int64_t n, cudaStream_t s);
+hy_status bw_gate(const void *x, hy_dtype dt, const float *c, float *z, int64_t n, cudaStream_t s);
+hy_status bw_dx_e(const float *g, const float *c, const void *x, hy_dtype dt, void *dx, float *er, int64_t rows, int L,
+                  cudaStream_t s);
+hy_status bw_next_g(const float *r, float *g, const void *x, hy_dtype dt, const float *Dk, int64_t rows, int D, int L,
+                    cudaStream_t s);
+hy_status bw_dh(const float *w, float *dh, int B, int D, int L, cudaStream_t s);
+hy_status bw_dD(const float *g, const void *x, hy_dtype dt, const float *z, float *dD, int B, int D, int L,
+                cudaStream_t s);
+
 // N-D path (ndconv.cu)
 struct NDArgs {
     int g[3];                      // grid

@@ -159,6 +159,35 @@ hy_status hyena_operator(int order, int B, int D, int L, hy_dtype dt, const void
                          void *stream);
 
 /* ------------------------------------------------------------------------
+ * Backward pass of the operator  ([HN] 아키텍처 상세, step 3, differentiated;
+ * the pages train the operator but print no gradient formulas -- these are
+ * the derivatives of the recurrence above.)
+ *
+ *   With z_0 = v, c_k = h_k * z_{k-1} + D_k z_{k-1} (causal), z_k = x_k ⊙ c_k,
+ *   y = z_K, and dy = dL/dy, from g_K = dy down to k = 1:
+ *     dx_k = g_k ⊙ c_k,   e_k = g_k ⊙ x_k,
+ *     g_{k-1}[s] = Σ_{t>=s} h_k[t-s] e_k[t] + D_k e_k[s],
+ *     dh_k[d, τ] = Σ_b Σ_{t>=τ} e_k[b,d,t] z_{k-1}[b,d,t-τ]   (τ < L),
+ *     dD_k[d]   = Σ_b Σ_t e_k[b,d,t] z_{k-1}[b,d,t],
+ *   and dv = g_0.
+ *   Inputs as hyena_operator (v, x[k], H[k] = spectra of h_k, Dskip may be
+ *   NULL) plus dy (dt, (B, D, L)).  Outputs: dv and dx[k] (dt, (B, D, L));
+ *   dh[k] (fp32, (D, L)) and dD[k] (fp32, (D)) -- either array or any entry
+ *   may be NULL to skip it.  All arithmetic fp32; the convolutions are the
+ *   forward path's (the sums over t >= s are causal convolutions of the
+ *   time-reversed e_k).  Deterministic (no atomics).
+ *   ws: device workspace of hyena_operator_backward_workspace() bytes,
+ *   256-byte aligned (fp32 intermediates: 2K + 4 signals and the per-row
+ *   spectra of e_k).
+ * ---------------------------------------------------------------------- */
+size_t hyena_operator_backward_workspace(int order, int B, int D, int L, hy_dtype dt);
+hy_status hyena_operator_backward(int order, int B, int D, int L, hy_dtype dt, const void *v,
+                                  const void *const *x, const hy_c32 *const *H,
+                                  const float *const *Dskip, const void *dy, void *dv,
+                                  void *const *dx, float *const *dh, float *const *dD, void *ws,
+                                  size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
  * hyena_operator_noalloc -- the operator above for callers that cannot
  * allocate device memory.  (The pages have no counterpart: this is a
  * deployment variant, not part of the method.)

@@ -53,6 +53,8 @@ PINS = {
     "circular_conv": "shift gate, Parseval, numpy.fft circular convolution",
     "fft_*": "matched against the direct functions above on sampled outputs",
     "projection": "identity weights give the transposed input, zero weights the bias, linearity",
+    "hyena_backward": "central finite differences of the direct forward (hyena_rows) for every input",
+    "hyena_backward_samples": "equals hyena_backward (order 2) at every index",
 }
 
 
@@ -240,6 +242,79 @@ def hyena_rows(v, xs, h, Dskip, rows=None, T=None) -> np.ndarray:
                            ctypes.c_int64(T), _dp(v), _ptr_array(xs), _dp(h), dsk,
                            ctypes.c_int64(rows.size), _ip(rows), _dp(y))
     return y
+
+
+def _causal_matrix(h: np.ndarray) -> np.ndarray:
+    """T[t, s] = h[t - s] for t >= s, else 0: c = T z is the causal convolution."""
+    L = h.shape[0]
+    idx = np.arange(L)[:, None] - np.arange(L)[None, :]
+    return np.where(idx >= 0, h[np.clip(idx, 0, L - 1)], 0.0)
+
+
+def hyena_backward(v, xs, h, Dskip, dy):
+    """Gradients of the order-N operator ([HN] 아키텍처 상세, step 3,
+    differentiated), float64, by explicit matrices: with T_k the causal
+    convolution matrix of h_k, c_k = T_k z_{k-1} + D_k z_{k-1}, so the
+    adjoint is g_{k-1} = T_k^T e_k + D_k e_k with e_k = g_k x_k; dx_k =
+    g_k c_k; dh_k[tau] = sum_b sum_t e_k[t] z_{k-1}[t - tau] (the matrix of
+    z_{k-1} transposed times e_k); dD_k = sum_b e_k . z_{k-1}.
+
+    v, xs[k], dy: (B, D, L); h: (K, D, L); Dskip: (K, D) or None.
+    Returns (dv, [dx_k], dh (K, D, L), dD (K, D))."""
+    v = np.asarray(v, np.float64)
+    dy = np.asarray(dy, np.float64)
+    xs = [np.asarray(x, np.float64) for x in xs]
+    h = np.asarray(h, np.float64)
+    K = h.shape[0]
+    B, D, L = v.shape
+    Dk = np.zeros((K, D)) if Dskip is None else np.asarray(Dskip, np.float64)
+    dv = np.empty_like(v)
+    dxs = [np.empty_like(v) for _ in range(K)]
+    dh = np.zeros((K, D, L))
+    dD = np.zeros((K, D))
+    for d in range(D):
+        T = [_causal_matrix(h[k, d]) for k in range(K)]
+        for b in range(B):
+            z = [v[b, d]]
+            c = []
+            for k in range(K):
+                c.append(T[k] @ z[k] + Dk[k, d] * z[k])
+                z.append(xs[k][b, d] * c[k])
+            g = dy[b, d]
+            for k in range(K - 1, -1, -1):
+                dxs[k][b, d] = g * c[k]
+                e = g * xs[k][b, d]
+                dh[k, d] += _causal_matrix(z[k]).T @ e
+                dD[k, d] += e @ z[k]
+                g = T[k].T @ e + Dk[k, d] * e
+            dv[b, d] = g
+    return dv, dxs, dh, dD
+
+
+def hyena_backward_samples(v, x1, h, Dk, dy, ts):
+    """Order-2 gradients by their direct sums at chosen indices, float64:
+    for each row (b, d) and s in ts
+      dv[s] = sum_{t>=s} h[t-s] e[t] + D e[s],  e = dy x1,
+      dx1[s] = dy[s] (sum_{u<=s} h[s-u] v[u] + D v[s]),
+    and for each lag tau in ts dh[d, tau] = sum_b sum_{t>=tau} e[t] v[t-tau];
+    dD[d] = sum_b e . v in full.  v, x1, dy: (B, D, L); h: (D, L); Dk: (D,)
+    or None.  Returns (dv (B, D, n), dx1 (B, D, n), dh (D, n), dD (D,))."""
+    v, x1, dy, h = (np.asarray(a, np.float64) for a in (v, x1, dy, h))
+    ts = np.asarray(ts, np.int64)
+    B, D, L = v.shape
+    Dk = np.zeros(D) if Dk is None else np.asarray(Dk, np.float64)
+    e = dy * x1
+    dv = np.empty((B, D, ts.size))
+    dx = np.empty((B, D, ts.size))
+    dh = np.zeros((D, ts.size))
+    for b in range(B):
+        for d in range(D):
+            for j, s in enumerate(ts):
+                dv[b, d, j] = float(h[d, :L - s] @ e[b, d, s:]) + Dk[d] * e[b, d, s]
+                dx[b, d, j] = dy[b, d, s] * (float(h[d, :s + 1][::-1] @ v[b, d, :s + 1]) + Dk[d] * v[b, d, s])
+                dh[d, j] += float(e[b, d, s:] @ v[b, d, :L - s])
+    dD = np.einsum("bdt,bdt->d", e, v)
+    return dv, dx, dh, dD
 
 
 def conv_gate_samples(h, u, x, Dk, ts) -> np.ndarray:

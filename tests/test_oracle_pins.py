@@ -430,3 +430,62 @@ def test_projection_identity_zero_and_linearity():
     b1, b2 = oracle.projection(x, W2, None, 2), oracle.projection(x2, W2, None, 2)
     for k in range(2):
         np.testing.assert_allclose(a[k], b1[k] + 2 * b2[k], rtol=1e-12, atol=1e-12)
+
+
+def test_backward_matches_finite_differences():
+    """Every gradient of the float64 backward equals the central difference of
+    the loss sum(dy * y), with y from the direct forward oracle (the C
+    hyena_rows, a separate code path), at a few elements of each input."""
+    rng = np.random.default_rng(19)
+    B, D, L, K = 2, 3, 11, 2
+    v = rng.standard_normal((B, D, L))
+    xs = [rng.standard_normal((B, D, L)) for _ in range(K)]
+    h = rng.standard_normal((K, D, L)) * 0.5
+    Dk = rng.standard_normal((K, D))
+    dy = rng.standard_normal((B, D, L))
+    dv, dxs, dh, dD = oracle.hyena_backward(v, xs, h, Dk, dy)
+
+    def loss(v_, xs_, h_, D_):
+        return float(np.sum(dy * oracle.hyena_rows(v_, xs_, h_, D_).reshape(B, D, L)))
+
+    eps = 1e-6
+
+    def fd(make):
+        return (loss(*make(eps)) - loss(*make(-eps))) / (2 * eps)
+
+    for i in [(0, 0, 0), (1, 2, 5), (0, 1, L - 1)]:
+        def mv(e, i=i):
+            a = v.copy(); a[i] += e
+            return a, xs, h, Dk
+        assert abs(fd(mv) - dv[i]) < 1e-6 * (1 + abs(dv[i]))
+        for k in range(K):
+            def mx(e, i=i, k=k):
+                a = [x.copy() for x in xs]; a[k][i] += e
+                return v, a, h, Dk
+            assert abs(fd(mx) - dxs[k][i]) < 1e-6 * (1 + abs(dxs[k][i]))
+    for k in range(K):
+        for j in [(0, 0), (2, 4), (1, L - 1)]:
+            def mh(e, j=j, k=k):
+                a = h.copy(); a[(k,) + j] += e
+                return v, xs, a, Dk
+            assert abs(fd(mh) - dh[(k,) + j]) < 1e-6 * (1 + abs(dh[(k,) + j]))
+        for d in range(D):
+            def md(e, d=d, k=k):
+                a = Dk.copy(); a[k, d] += e
+                return v, xs, h, a
+            assert abs(fd(md) - dD[k, d]) < 1e-6 * (1 + abs(dD[k, d]))
+
+
+def test_backward_samples_equal_full_backward():
+    rng = np.random.default_rng(20)
+    B, D, L = 2, 3, 40
+    v, x1, dy = rng.standard_normal((3, B, D, L))
+    h = rng.standard_normal((D, L))
+    Dk = rng.standard_normal(D)
+    dv, dxs, dh, dD = oracle.hyena_backward(v, [x1], h[None], Dk[None], dy)
+    ts = np.arange(L)
+    sv, sx, sh, sD = oracle.hyena_backward_samples(v, x1, h, Dk, dy, ts)
+    np.testing.assert_allclose(sv, dv, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(sx, dxs[0], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(sh, dh[0], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(sD, dD[0], rtol=1e-12, atol=1e-12)

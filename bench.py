@@ -621,6 +621,59 @@ def run_projection(args):
                        "B": B, "L": L, "C": C, "D": D, "n_out": n_out}}), flush=True)
 
 
+def run_backward(args):
+    """The operator's backward pass on the order-2 operator workload (B8 D768
+    L8192, bf16 signals): dv, dx_1, dh_1 and dD_1 from dy, with the forward
+    recomputed inside.  GB/s = compulsory bytes (v, x_1, dy and the spectra
+    read; dv, dx_1 and dh_1 written) / time."""
+    import torch
+    import implicit_long_convolution_b200 as hy
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    w = hw.make("c2", seed=rank_seed("c2", rank), with_signals=True)
+    s = w.spec
+    B, D, L = s["B"], s["D"], s["L"]
+    bf = lambda sig: torch.from_numpy(sig.bf16.view(np.int16)).view(torch.bfloat16).to(dev)
+    v, x1 = bf(w.v), bf(w.xs[0])
+    dy = torch.randn((B, D, L), device=dev).to(torch.bfloat16)
+    f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dev)
+    Ws, bs, alpha = [f32(a) for a in w.Ws], [f32(a) for a in w.bs], f32(w.alpha)
+    h = torch.empty((D, L), device=dev)
+    hy.hyena_filter_gen(h, ndim=1, L=L, Ws=Ws, bs=bs, alpha=alpha, n_freq=s["F"], include_t=True)
+    H = torch.empty((D, hy.spectrum_bins(L)), dtype=torch.complex64, device=dev)
+    hy.hyena_filter_spectrum(h, H, rows=D, ndim=1, dims=[L])
+    dsk = [f32(w.Dskip[0])]
+    dv, dx = torch.empty_like(v), [torch.empty_like(v)]
+    dh, dD = [torch.empty((D, L), device=dev)], [torch.empty(D, device=dev)]
+    ws = torch.empty(hy.operator_backward_workspace(2, B, D, L, hy.HY_BF16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    run = lambda: hy.hyena_operator_backward(v, [x1], [H], dy, dv, dx, Dskips=dsk, dhs=dh, dDs=dD, ws=ws)
+    for _ in range(max(3, args.warmup)):
+        run()
+    steps = args.steps if args.steps > 0 else 50
+    torch.cuda.synchronize()
+    barrier(world)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        run()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(t0.elapsed_time(t1), world) / steps
+    nb = hy.spectrum_bins(L)
+    sig_bytes = B * D * L * 2
+    step_bytes = 5 * sig_bytes + D * nb * 8 + D * L * 4 + D * 4
+    if rank == 0:
+        print(json.dumps({
+            "metric": "Hyena op backward GB/s (order-2 operator B8 D768 L8192 bf16: dv, dx1, dh1, dD1)",
+            "value": round(world * step_bytes / (ms / 1e3) / 1e9, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32 math, bf16 I/O", "data": "synthetic",
+            "config": {"workload": "hyena order-2 operator backward B8 D768 L8192 bf16", "B": B, "D": D, "L": L,
+                       "step_bytes": step_bytes}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -630,6 +683,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(DESCR), default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the operator's backward pass on the order-2 operator workload instead")
     ap.add_argument("--projection", action="store_true",
                     help="time the input projection at the operator workload's width instead")
     ap.add_argument("--channels", type=int, default=0,
@@ -646,6 +701,9 @@ def main():
         args.warmup = 3
     if args.projection:
         run_projection(args)
+        return
+    if args.backward:
+        run_backward(args)
         return
     run_ours(args)
 

@@ -24,6 +24,24 @@ __device__ __forceinline__ float ld_io(const __nv_bfloat16 *p, int64_t i) { retu
 __device__ __forceinline__ void st_io(float *p, int64_t i, float v) { p[i] = v; }
 __device__ __forceinline__ void st_io(__nv_bfloat16 *p, int64_t i, float v) { p[i] = __float2bfloat16_rn(v); }
 
+// 4 consecutive elements (16 bytes of fp32, 8 of bf16)
+__device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 ld4(const __nv_bfloat16 *p) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(p);
+    return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u), __uint_as_float(u.y << 16),
+                       __uint_as_float(u.y & 0xffff0000u));
+}
+__device__ __forceinline__ void st4(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
+__device__ __forceinline__ void st4(__nv_bfloat16 *p, float4 v) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<const uint32_t *>(&a);
+    u.y = *reinterpret_cast<const uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(p) = u;
+}
+__device__ __forceinline__ float4 mul4(float4 a, float4 b) { return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w); }
+__device__ __forceinline__ float4 rev4(float4 a) { return make_float4(a.w, a.z, a.y, a.x); }
+
 constexpr int NT = 256;
 
 unsigned grid_for(int64_t n) {
@@ -32,14 +50,42 @@ unsigned grid_for(int64_t n) {
     return (unsigned)(b < 1 ? 1 : (b > cap ? cap : b));
 }
 
+// Element-wise passes walk rows: block y strides over rows, threads over
+// the row in groups of 4 (L a multiple of 4) or singly.
+#define HY_ROWS_LOOP(rows)                                                        \
+    for (int64_t row = blockIdx.y; row < (rows); row += gridDim.y)
+
+dim3 rows_grid(int64_t rows, int L, bool vec) {
+    const int per_row = (vec ? L / 4 : L);
+    unsigned x = (unsigned)((per_row + NT - 1) / NT);
+    if (x < 1) x = 1;
+    int64_t y = (int64_t)148 * 64 / x;
+    if (y < 1) y = 1;
+    if (y > rows) y = rows;
+    if (y > 65535) y = 65535;
+    return dim3(x, (unsigned)y);
+}
+
 template <typename IO>
 __global__ void __launch_bounds__(NT) k_to_f32(const IO *src, float *dst, int64_t n) {
     for (int64_t i = blockIdx.x * (int64_t)NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT) dst[i] = ld_io(src, i);
 }
 
 template <typename IO>
+__global__ void __launch_bounds__(NT) k_to_f32_v(const IO *src, float *dst, int64_t n4) {
+    for (int64_t i = blockIdx.x * (int64_t)NT + threadIdx.x; i < n4; i += (int64_t)gridDim.x * NT)
+        st4(dst + 4 * i, ld4(src + 4 * i));
+}
+
+template <typename IO>
 __global__ void __launch_bounds__(NT) k_from_f32(const float *src, IO *dst, int64_t n) {
     for (int64_t i = blockIdx.x * (int64_t)NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT) st_io(dst, i, src[i]);
+}
+
+template <typename IO>
+__global__ void __launch_bounds__(NT) k_from_f32_v(const float *src, IO *dst, int64_t n4) {
+    for (int64_t i = blockIdx.x * (int64_t)NT + threadIdx.x; i < n4; i += (int64_t)gridDim.x * NT)
+        st4(dst + 4 * i, ld4(src + 4 * i));
 }
 
 // z = x ⊙ c
@@ -49,26 +95,47 @@ __global__ void __launch_bounds__(NT) k_gate(const IO *x, const float *c, float 
 }
 
 // dx = g ⊙ c; er[row][L-1-t] = g[row][t] x[row][t]
-template <typename IO>
+template <typename IO, bool VEC>
 __global__ void __launch_bounds__(NT) k_dx_e(const float *g, const float *c, const IO *x, IO *dx, float *er,
-                                             int64_t n, int L) {
-    for (int64_t i = blockIdx.x * (int64_t)NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT) {
-        const float gi = g[i];
-        st_io(dx, i, gi * c[i]);
-        const int64_t row = i / L, t = i - row * L;
-        er[row * L + (L - 1 - t)] = gi * ld_io(x, i);
+                                             int64_t rows, int L) {
+    HY_ROWS_LOOP(rows) {
+        const int64_t o = row * L;
+        if constexpr (VEC) {
+            for (int q = blockIdx.x * NT + threadIdx.x; q < L / 4; q += gridDim.x * NT) {
+                const int t = 4 * q;
+                const float4 gv = ld4(g + o + t);
+                st4(dx + o + t, mul4(gv, ld4(c + o + t)));
+                st4(er + o + (L - 4 - t), rev4(mul4(gv, ld4(x + o + t))));
+            }
+        } else {
+            for (int t = blockIdx.x * NT + threadIdx.x; t < L; t += gridDim.x * NT) {
+                const float gi = g[o + t];
+                st_io(dx, o + t, gi * c[o + t]);
+                er[o + (L - 1 - t)] = gi * ld_io(x, o + t);
+            }
+        }
     }
 }
 
 // g[row][t] <- r[row][L-1-t] + D[row % D] g[row][t] x[row][t]  (in place)
-template <typename IO>
-__global__ void __launch_bounds__(NT) k_next_g(const float *r, float *g, const IO *x, const float *Dk, int64_t n,
+template <typename IO, bool VEC>
+__global__ void __launch_bounds__(NT) k_next_g(const float *r, float *g, const IO *x, const float *Dk, int64_t rows,
                                                int D, int L) {
-    for (int64_t i = blockIdx.x * (int64_t)NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT) {
-        const int64_t row = i / L, t = i - row * L;
-        float v = r[row * L + (L - 1 - t)];
-        if (Dk) v = fmaf(__ldg(Dk + row % D), g[i] * ld_io(x, i), v);
-        g[i] = v;
+    HY_ROWS_LOOP(rows) {
+        const int64_t o = row * L;
+        const float dk = Dk ? __ldg(Dk + row % D) : 0.f;
+        if constexpr (VEC) {
+            for (int q = blockIdx.x * NT + threadIdx.x; q < L / 4; q += gridDim.x * NT) {
+                const int t = 4 * q;
+                const float4 rv = rev4(ld4(r + o + (L - 4 - t)));
+                const float4 e = mul4(ld4(g + o + t), ld4(x + o + t));
+                st4(g + o + t, make_float4(fmaf(dk, e.x, rv.x), fmaf(dk, e.y, rv.y), fmaf(dk, e.z, rv.z),
+                                           fmaf(dk, e.w, rv.w)));
+            }
+        } else {
+            for (int t = blockIdx.x * NT + threadIdx.x; t < L; t += gridDim.x * NT)
+                g[o + t] = fmaf(dk, g[o + t] * ld_io(x, o + t), r[o + (L - 1 - t)]);
+        }
     }
 }
 
@@ -117,13 +184,24 @@ __global__ void __launch_bounds__(NT) k_dD(const float *g, const IO *x, const fl
         }                                                  \
     } while (0)
 
+// Vector paths need 4 | n and row starts at a multiple of 4 elements; the
+// pointers are the library's own workspace or the caller's signals, whose
+// alignment the entry point checks (16-byte fp32 / 8-byte bf16 when 4 | L).
 hy_status bw_to_f32(const void *src, hy_dtype dt, float *dst, int64_t n, cudaStream_t s) {
-    HY_IO_DISPATCH(dt, T, k_to_f32<T><<<grid_for(n), NT, 0, s>>>(reinterpret_cast<const T *>(src), dst, n));
+    const bool vec = n % 4 == 0 && (uintptr_t)src % (4 * (dt == HY_BF16 ? 2 : 4)) == 0;
+    if (vec)
+        HY_IO_DISPATCH(dt, T, k_to_f32_v<T><<<grid_for(n / 4), NT, 0, s>>>(reinterpret_cast<const T *>(src), dst, n / 4));
+    else
+        HY_IO_DISPATCH(dt, T, k_to_f32<T><<<grid_for(n), NT, 0, s>>>(reinterpret_cast<const T *>(src), dst, n));
     return check_launch("backward: convert");
 }
 
 hy_status bw_from_f32(const float *src, hy_dtype dt, void *dst, int64_t n, cudaStream_t s) {
-    HY_IO_DISPATCH(dt, T, k_from_f32<T><<<grid_for(n), NT, 0, s>>>(src, reinterpret_cast<T *>(dst), n));
+    const bool vec = n % 4 == 0 && (uintptr_t)dst % (4 * (dt == HY_BF16 ? 2 : 4)) == 0;
+    if (vec)
+        HY_IO_DISPATCH(dt, T, k_from_f32_v<T><<<grid_for(n / 4), NT, 0, s>>>(src, reinterpret_cast<T *>(dst), n / 4));
+    else
+        HY_IO_DISPATCH(dt, T, k_from_f32<T><<<grid_for(n), NT, 0, s>>>(src, reinterpret_cast<T *>(dst), n));
     return check_launch("backward: convert");
 }
 
@@ -134,16 +212,27 @@ hy_status bw_gate(const void *x, hy_dtype dt, const float *c, float *z, int64_t 
 
 hy_status bw_dx_e(const float *g, const float *c, const void *x, hy_dtype dt, void *dx, float *er, int64_t rows, int L,
                   cudaStream_t s) {
-    const int64_t n = rows * L;
-    HY_IO_DISPATCH(dt, T, k_dx_e<T><<<grid_for(n), NT, 0, s>>>(g, c, reinterpret_cast<const T *>(x),
-                                                                reinterpret_cast<T *>(dx), er, n, L));
+    const size_t al = 4 * (dt == HY_BF16 ? 2 : 4);
+    const bool vec = L % 4 == 0 && (uintptr_t)x % al == 0 && (uintptr_t)dx % al == 0;
+    const dim3 grid = rows_grid(rows, L, vec);
+    if (vec)
+        HY_IO_DISPATCH(dt, T, k_dx_e<T, true><<<grid, NT, 0, s>>>(g, c, reinterpret_cast<const T *>(x),
+                                                                   reinterpret_cast<T *>(dx), er, rows, L));
+    else
+        HY_IO_DISPATCH(dt, T, k_dx_e<T, false><<<grid, NT, 0, s>>>(g, c, reinterpret_cast<const T *>(x),
+                                                                    reinterpret_cast<T *>(dx), er, rows, L));
     return check_launch("backward: dx");
 }
 
 hy_status bw_next_g(const float *r, float *g, const void *x, hy_dtype dt, const float *Dk, int64_t rows, int D, int L,
                     cudaStream_t s) {
-    const int64_t n = rows * L;
-    HY_IO_DISPATCH(dt, T, k_next_g<T><<<grid_for(n), NT, 0, s>>>(r, g, reinterpret_cast<const T *>(x), Dk, n, D, L));
+    const size_t al = 4 * (dt == HY_BF16 ? 2 : 4);
+    const bool vec = L % 4 == 0 && (uintptr_t)x % al == 0;
+    const dim3 grid = rows_grid(rows, L, vec);
+    if (vec)
+        HY_IO_DISPATCH(dt, T, k_next_g<T, true><<<grid, NT, 0, s>>>(r, g, reinterpret_cast<const T *>(x), Dk, rows, D, L));
+    else
+        HY_IO_DISPATCH(dt, T, k_next_g<T, false><<<grid, NT, 0, s>>>(r, g, reinterpret_cast<const T *>(x), Dk, rows, D, L));
     return check_launch("backward: next gradient");
 }
 

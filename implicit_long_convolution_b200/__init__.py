@@ -32,7 +32,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhyena_b2
 STATUS = {0: "HY_OK", 1: "HY_ERR_INVALID_ARG", 2: "HY_ERR_UNSUPPORTED", 3: "HY_ERR_WORKSPACE",
           4: "HY_ERR_CUDA", 5: "HY_ERR_TIMEOUT"}
 HY_F32, HY_BF16 = 0, 1
-HY_ACT_SILU, HY_ACT_IDENTITY = 0, 1
+HY_ACT_SILU, HY_ACT_IDENTITY, HY_ACT_SINE = 0, 1, 2
+HY_WIN_EXP, HY_WIN_GAUSS = 0, 1
 
 
 class HyenaLibraryMissing(RuntimeError):
@@ -54,6 +55,7 @@ class FilterDesc(ctypes.Structure):
         ("W", ctypes.POINTER(ctypes.c_void_p)), ("b", ctypes.POINTER(ctypes.c_void_p)),
         ("act", ctypes.c_int), ("film_gamma", ctypes.c_void_p), ("film_beta", ctypes.c_void_p),
         ("alpha", ctypes.c_void_p), ("n_sets", ctypes.c_int),
+        ("omega", ctypes.c_void_p), ("window", ctypes.c_int),
     ]
 
 
@@ -162,13 +164,13 @@ def spectrum_bins(L: int) -> int:
 def hyena_filter_gen(h_out, *, ndim: int, Ws: Sequence, bs: Sequence, alpha, n_freq: int,
                      L: int = 0, include_t: bool = True, grid: int = 0, circular: bool = False,
                      film_gamma=None, film_beta=None, n_sets: int = 1, act: int = HY_ACT_SILU,
-                     stream=None):
+                     omega=None, window: int = HY_WIN_EXP, stream=None):
     """Fill h_out (fp32, device) with implicit filters; see hyena.h."""
     widths = [int(Ws[0].shape[1])] + [int(w.shape[0]) for w in Ws]
     keep = (_ints(widths), _ptrs(Ws), _ptrs(bs))
     d = FilterDesc(ndim, L, grid, int(circular), n_freq, int(include_t), len(Ws),
                    keep[0], keep[1], keep[2], act, _ptr(film_gamma), _ptr(film_beta),
-                   _ptr(alpha), n_sets)
+                   _ptr(alpha), n_sets, _ptr(omega), window)
     _check(lib().hyena_filter_gen(ctypes.byref(d), _ptr(h_out), _stream(stream)))
     return h_out
 

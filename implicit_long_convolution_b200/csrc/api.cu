@@ -151,7 +151,9 @@ hy_status hyena_filter_gen(const hy_filter_desc *d, float *h, void *stream) {
     if (d->n_layers < 1 || d->n_layers > 4) return set_error(HY_ERR_UNSUPPORTED, "hyena_filter_gen: n_layers must be 1..4");
     if (!d->widths || !d->W || !d->b || !d->alpha) return set_error(HY_ERR_INVALID_ARG, "hyena_filter_gen: null parameter array");
     if (d->n_freq < 0 || d->n_sets < 1) return set_error(HY_ERR_INVALID_ARG, "hyena_filter_gen: bad n_freq or n_sets");
-    if (d->act != HY_ACT_SILU && d->act != HY_ACT_IDENTITY) return set_error(HY_ERR_INVALID_ARG, "hyena_filter_gen: bad activation");
+    if (d->act != HY_ACT_SILU && d->act != HY_ACT_IDENTITY && d->act != HY_ACT_SINE)
+        return set_error(HY_ERR_INVALID_ARG, "hyena_filter_gen: bad activation");
+    if (d->window != HY_WIN_EXP && d->window != HY_WIN_GAUSS) return set_error(HY_ERR_INVALID_ARG, "hyena_filter_gen: bad window");
     if ((d->film_gamma == nullptr) != (d->film_beta == nullptr))
         return set_error(HY_ERR_INVALID_ARG, "hyena_filter_gen: film_gamma and film_beta go together");
     if (d->film_gamma && d->n_layers < 2) return set_error(HY_ERR_INVALID_ARG, "hyena_filter_gen: FiLM needs a hidden layer");

@@ -35,7 +35,7 @@ constexpr int OT_MAX = 16 * CPT_L;
 constexpr int OTS = OT_MAX + 4; // wT row stride: = 4 (mod 32) keeps the staging stores conflict-free
 constexpr int MAXW = 132;       // max layer input width
 constexpr int MAXL = 4;
-constexpr int NPAR = 4;         // per-output parameter rows staged with a tile: bias, alpha, gamma, beta
+constexpr int NPAR = 5;         // per-output parameter rows staged with a tile: bias, alpha, gamma, beta, omega
 
 struct GenParams {
     int ndim;
@@ -49,6 +49,8 @@ struct GenParams {
     int act;
     const float *gamma, *beta;
     const float *alpha;
+    const float *om[MAXL];      // sine frequencies of hidden layer l's units, or NULL
+    int window;                 // HY_WIN_EXP / HY_WIN_GAUSS
     int64_t npos;               // positions per set (L or S^3)
     int ka;                     // max layer input width (activation rows)
     int wbuf;                   // floats per weight buffer
@@ -106,6 +108,7 @@ __device__ __forceinline__ void stage_tile(const GenParams &p, int l, int o0, in
             cpa4(par + 2 * OT_MAX + r, p.gamma + (int64_t)set * wout + o);
             cpa4(par + 3 * OT_MAX + r, p.beta + (int64_t)set * wout + o);
         }
+        if (!last && p.om[l]) cpa4(par + 4 * OT_MAX + r, p.om[l] + o);
     }
 }
 
@@ -282,12 +285,14 @@ __global__ void __launch_bounds__(NT, 2) filter_gen_kernel(const GenParams p) {
                 const float bo = par[r];
                 const float gm = film ? par[2 * OT_MAX + r] : 0.f;
                 const float bt = film ? par[3 * OT_MAX + r] : 0.f;
+                const float om = p.om[l] ? par[4 * OT_MAX + r] : 1.f;
                 float v[4];
 #pragma unroll
                 for (int a = 0; a < 4; ++a) {
                     float x = acc[a][c] + bo;
                     if (film) x = fmaf(1.f + gm, x, bt);
                     if (p.act == HY_ACT_SILU) x = silu(x);
+                    else if (p.act == HY_ACT_SINE) x = sinf(om * x);
                     v[a] = x;
                 }
                 *reinterpret_cast<float4 *>(nxt + o * P + 4 * tx) = make_float4(v[0], v[1], v[2], v[3]);
@@ -300,6 +305,7 @@ __global__ void __launch_bounds__(NT, 2) filter_gen_kernel(const GenParams p) {
 #pragma unroll
             for (int a = 0; a < 4; ++a) {
                 nrm[a] = s_norm[4 * tx + a];
+                if (p.window == HY_WIN_GAUSS) nrm[a] *= nrm[a];
                 ok[a] = s_valid[4 * tx + a] != 0;
             }
             const int64_t q0 = p0 + 4 * tx;
@@ -313,7 +319,7 @@ __global__ void __launch_bounds__(NT, 2) filter_gen_kernel(const GenParams p) {
                 const float al = par[OT_MAX + r] * kLog2e;      // e^{-a n} = 2^{-a log2(e) n}
                 float v[4];
 #pragma unroll
-                for (int a = 0; a < 4; ++a) v[a] = ok[a] ? (acc[a][c] + bo) * exp2f(-al * nrm[a]) : 0.f;
+                for (int a = 0; a < 4; ++a) v[a] = ok[a] ? (acc[a][c] + bo) * exp2f(-al * nrm[a]) : 0.f;   // nrm: n or n^2
                 float *dst = p.h + ((int64_t)set * nout + o) * p.npos + q0;
                 if (full) {
                     *reinterpret_cast<float4 *>(dst) = make_float4(v[0], v[1], v[2], v[3]);
@@ -364,6 +370,11 @@ hy_status launch_filter_gen(const hy_filter_desc &d, float *h, cudaStream_t s) {
         p.b[l] = d.b[l];
     }
     p.act = d.act;
+    for (int l = 0, off = 0; l < p.nl; ++l) {
+        p.om[l] = (d.act == HY_ACT_SINE && d.omega && l < p.nl - 1) ? d.omega + off : nullptr;
+        if (l < p.nl - 1) off += d.widths[l + 1];
+    }
+    p.window = d.window;
     p.gamma = d.film_gamma;
     p.beta = d.film_beta;
     p.alpha = d.alpha;

@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define HYENA_ABI_VERSION 1
+#define HYENA_ABI_VERSION 2
 
 typedef enum hy_status {
     HY_OK = 0,
@@ -57,7 +57,13 @@ typedef enum hy_status {
 
 typedef enum hy_dtype { HY_F32 = 0, HY_BF16 = 1 } hy_dtype;
 
-typedef enum hy_act { HY_ACT_SILU = 0, HY_ACT_IDENTITY = 1 } hy_act;
+/* Hidden activation: SiLU, identity, or sine sin(ω x) (the SIREN of [ND]
+ * 방법론, 커널 매개변수화, with per-unit frequencies ω). */
+typedef enum hy_act { HY_ACT_SILU = 0, HY_ACT_IDENTITY = 1, HY_ACT_SINE = 2 } hy_act;
+/* Window on the normalised distance n (t/L or |r|/g): exp(-α n) ([HN] step 2,
+ * w(t) = e^{-αt}) or the Gaussian exp(-α n²) ([ND] 커널 합성: 학습 가능한
+ * 가우시안 윈도우, α = 1/(2σ²)). */
+typedef enum hy_window { HY_WIN_EXP = 0, HY_WIN_GAUSS = 1 } hy_window;
 
 /* Interleaved single-precision complex (same bytes as float2 / complex64). */
 typedef struct hy_c32 { float re; float im; } hy_c32;
@@ -72,17 +78,21 @@ int64_t hyena_spectrum_bins(int64_t L);
 /* ------------------------------------------------------------------------
  * Filter generator  ([HN] step 2 and ImplicitFilter; [ES]; [ND] FiLM)
  *
- *   1-D:  h[s, o, t] = MLP(PE(t))[o] · exp(-alpha[o] · t / L)
+ *   1-D:  h[s, o, t] = MLP(PE(t))[o] · w_o(t / L)
  *         PE(t) = [t/L (if include_t), cos(2π j t/L) j=1..F, sin(2π j t/L) j=1..F]
- *   3-D:  h[s, o, p] = MLP_s(PE3(r(p)))[o] · exp(-alpha[o] · |r(p)| / g)
+ *   3-D:  h[s, o, p] = MLP_s(PE3(r(p)))[o] · w_o(|r(p)| / g)
  *         on the transform grid of edge S (S = 2g, or g when circular); r(p)
  *         is the signed offset of grid index p per axis (i < S/2 -> i, else
  *         i - S); PE3 = per axis (x, y, z): cos(π j r_a/g), sin(π j r_a/g),
  *         j = 1..F.  Non-circular kernels are zero outside |r_a| <= g - 1.
  *   MLP: layer l maps widths[l] -> widths[l+1], y = W_l x + b_l (W_l row-major
- *   out x in); every layer but the last is followed by `act`; when
+ *   out x in); every layer but the last is followed by `act` (for
+ *   HY_ACT_SINE: sin(omega[u] y) per hidden unit u, omega holding every
+ *   hidden layer's units in order, or 1 when omega is NULL); when
  *   film_gamma is set, the first hidden layer is modulated per filter set s
  *   before the activation: y <- (1 + gamma[s]) ⊙ y + beta[s].
+ *   w_o(n) = exp(-alpha[o] n) (window = HY_WIN_EXP) or exp(-alpha[o] n²)
+ *   (HY_WIN_GAUSS).
  * ---------------------------------------------------------------------- */
 typedef struct hy_filter_desc {
     int ndim;                /* 1 or 3 */
@@ -100,6 +110,8 @@ typedef struct hy_filter_desc {
     const float *film_beta;  /* device (n_sets, widths[1]) or NULL (with gamma) */
     const float *alpha;      /* device (widths[n_layers]); >= 0 */
     int n_sets;              /* filter sets s (1 unless FiLM-conditioned) */
+    const float *omega;      /* device (Σ hidden widths) sine frequencies, or NULL */
+    int window;              /* hy_window */
 } hy_filter_desc;
 
 /* Writes h (device, fp32): 1-D (n_sets, n_out, L); 3-D (n_sets, n_out, S, S, S). */

@@ -153,20 +153,37 @@ def _mlp_args(Ws, bs):
     return Ws, bs, widths, warr
 
 
-def filter_gen_1d(L, F, include_t, Ws, bs, alpha) -> np.ndarray:
-    """h[o, t] = MLP(PE(t))[o] * exp(-alpha_o t / L), float64, shape (n_out, L)."""
+ACT = {"silu": 0, "identity": 1, "sine": 2}
+WINDOW = {"exp": 0, "gauss": 1}
+
+
+def _omega_arg(omega, widths):
+    """Per-hidden-unit sine frequencies, all hidden layers concatenated."""
+    if omega is None:
+        return None, None
+    om = _f64(omega)
+    assert om.shape == (sum(widths[1:-1]),)
+    return om, _dp(om)
+
+
+def filter_gen_1d(L, F, include_t, Ws, bs, alpha, act="silu", omega=None, window="exp") -> np.ndarray:
+    """h[o, t] = MLP(PE(t))[o] * w_o(t/L), float64, shape (n_out, L); hidden
+    activation SiLU, identity or sin(omega x); window exp(-alpha_o n) or the
+    Gaussian exp(-alpha_o n^2)."""
     Ws, bs, widths, warr = _mlp_args(Ws, bs)
     alpha = _f64(alpha)
     nout = widths[-1]
     assert alpha.shape == (nout,)
+    om, omp = _omega_arg(omega, widths)
     h = np.empty((nout, L), np.float64)
     _load().orc_filter_gen_1d(ctypes.c_int64(L), ctypes.c_int(F), ctypes.c_int(int(include_t)),
                               ctypes.c_int(len(Ws)), warr, _ptr_array(Ws), _ptr_array(bs),
-                              _dp(alpha), _dp(h))
+                              _dp(alpha), ctypes.c_int(ACT[act]), omp, ctypes.c_int(WINDOW[window]), _dp(h))
     return h
 
 
-def filter_gen_3d_points(g, circular, F, Ws, bs, gamma, beta, alpha, idx) -> np.ndarray:
+def filter_gen_3d_points(g, circular, F, Ws, bs, gamma, beta, alpha, idx, act="silu", omega=None,
+                         window="exp") -> np.ndarray:
     """Kernel values at flat transform-grid indices idx: shape (len(idx), n_out)."""
     Ws, bs, widths, warr = _mlp_args(Ws, bs)
     alpha = _f64(alpha)
@@ -176,9 +193,11 @@ def filter_gen_3d_points(g, circular, F, Ws, bs, gamma, beta, alpha, idx) -> np.
     if gamma is not None:
         gamma = _f64(gamma); beta = _f64(beta)
         gp, bp = _dp(gamma), _dp(beta)
+    om, omp = _omega_arg(omega, widths)
     _load().orc_filter_gen_3d_points(ctypes.c_int(g), ctypes.c_int(int(circular)), ctypes.c_int(F),
                                      ctypes.c_int(len(Ws)), warr, _ptr_array(Ws), _ptr_array(bs),
-                                     gp, bp, _dp(alpha), ctypes.c_int64(idx.size), _ip(idx), _dp(out))
+                                     gp, bp, _dp(alpha), ctypes.c_int(ACT[act]), omp, ctypes.c_int(WINDOW[window]),
+                                     ctypes.c_int64(idx.size), _ip(idx), _dp(out))
     return out
 
 

@@ -87,12 +87,22 @@ static double orc_silu(double a) { return a / (1.0 + exp(-a)); }
  * y = W_l x + b_l with W_l row-major (out x in).  Hidden layers (all but the
  * last) optionally get FiLM on the first hidden layer, y <- (1+γ)⊙y + β
  * ([ND] FiLM conditioning of the kernel MLP), then SiLU ([HN] sketch).  */
+/* Hidden activation: 0 SiLU, 1 identity, 2 sine sin(ω x) (SIREN, [ND]
+ * 방법론: 좌표 기반 SIREN MLP; ω per hidden unit, 1 when omega is NULL). */
+static double orc_act(int act, double s, double w)
+{
+    if (act == 1) return s;
+    if (act == 2) return sin(w * s);
+    return orc_silu(s);
+}
+
 static void orc_mlp_point(int nl, const int *widths, const double *const *W,
                           const double *const *b, const double *film_gamma,
-                          const double *film_beta, const double *x, double *out,
-                          double *scratch_a, double *scratch_b)
+                          const double *film_beta, int act, const double *omega,
+                          const double *x, double *out, double *scratch_a, double *scratch_b)
 {
     const double *cur = x;
+    int64_t woff = 0;   /* offset of this hidden layer's frequencies in omega */
     for (int l = 0; l < nl; ++l) {
         int win = widths[l], wout = widths[l + 1];
         double *dst = (l == nl - 1) ? out : ((l & 1) ? scratch_b : scratch_a);
@@ -102,12 +112,21 @@ static void orc_mlp_point(int nl, const int *widths, const double *const *W,
             for (int i = 0; i < win; ++i) s += wr[i] * cur[i];
             if (l < nl - 1) {
                 if (l == 0 && film_gamma) s = (1.0 + film_gamma[o]) * s + film_beta[o];
-                s = orc_silu(s);
+                s = orc_act(act, s, omega ? omega[woff + o] : 1.0);
             }
             dst[o] = s;
         }
+        if (l < nl - 1) woff += wout;
         cur = dst;
     }
+}
+
+/* Window on the normalised distance n (t/L or |r|/g): 0 exponential
+ * exp(-α n) ([HN] w(t) = e^{-αt}), 1 Gaussian exp(-α n²) ([ND] 커널 합성:
+ * 학습 가능한 가우시안 윈도우, α = 1/(2σ²)). */
+static double orc_window(int window, double alpha, double n)
+{
+    return window == 1 ? exp(-alpha * n * n) : exp(-alpha * n);
 }
 
 static int orc_max_width(int nl, const int *widths)
@@ -123,7 +142,7 @@ static int orc_max_width(int nl, const int *widths)
  * h is row-major (n_out x L).  n_out = K·D for an operator with K filters. */
 void orc_filter_gen_1d(int64_t L, int F, int include_t, int nl, const int *widths,
                        const double *const *W, const double *const *b,
-                       const double *alpha, double *h)
+                       const double *alpha, int act, const double *omega, int window, double *h)
 {
     const int win = widths[0];
     const int nout = widths[nl];
@@ -143,9 +162,9 @@ void orc_filter_gen_1d(int64_t L, int F, int include_t, int nl, const int *width
                 pe[c + j - 1] = cos(2.0 * ORC_PI * (double)r / (double)L);
                 pe[c + F + j - 1] = sin(2.0 * ORC_PI * (double)r / (double)L);
             }
-            orc_mlp_point(nl, widths, W, b, NULL, NULL, pe, o, sa, sb);
+            orc_mlp_point(nl, widths, W, b, NULL, NULL, act, omega, pe, o, sa, sb);
             double tn = (double)t / (double)L;
-            for (int k = 0; k < nout; ++k) h[(int64_t)k * L + t] = o[k] * exp(-alpha[k] * tn);
+            for (int k = 0; k < nout; ++k) h[(int64_t)k * L + t] = o[k] * orc_window(window, alpha[k], tn);
         }
         free(pe); free(sa); free(sb); free(o);
     }
@@ -166,8 +185,8 @@ static int orc_signed_offset(int64_t i, int64_t S) { return (int)(i < S / 2 ? i 
 void orc_filter_gen_3d_points(int g, int circular, int F, int nl, const int *widths,
                               const double *const *W, const double *const *b,
                               const double *film_gamma, const double *film_beta,
-                              const double *alpha, int64_t npts, const int64_t *idx,
-                              double *out)
+                              const double *alpha, int act, const double *omega, int window,
+                              int64_t npts, const int64_t *idx, double *out)
 {
     const int64_t S = circular ? (int64_t)g : 2 * (int64_t)g;
     const int nout = widths[nl];
@@ -189,9 +208,9 @@ void orc_filter_gen_3d_points(int g, int circular, int F, int nl, const int *wid
             double *row = out + q * nout;
             if (!inside) { for (int k = 0; k < nout; ++k) row[k] = 0.0; continue; }
             orc_pe3d_point(g, F, r, pe);
-            orc_mlp_point(nl, widths, W, b, film_gamma, film_beta, pe, o, sa, sb);
+            orc_mlp_point(nl, widths, W, b, film_gamma, film_beta, act, omega, pe, o, sa, sb);
             double rn = sqrt((double)r[0] * r[0] + (double)r[1] * r[1] + (double)r[2] * r[2]) / (double)g;
-            for (int k = 0; k < nout; ++k) row[k] = o[k] * exp(-alpha[k] * rn);
+            for (int k = 0; k < nout; ++k) row[k] = o[k] * orc_window(window, alpha[k], rn);
         }
         free(pe); free(sa); free(sb); free(o);
     }

@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_strings(lib):
-    assert lib.hyena_abi_version() == 1
+    assert lib.hyena_abi_version() == 2
     assert lib.hyena_status_string(3) == b"HY_ERR_WORKSPACE"
     assert lib.hyena_spectrum_bins(8192) == 8193
     assert lib.hyena_spectrum_bins(1000) == 1025
@@ -108,6 +108,11 @@ def test_filter_and_nd_validation(lib):
     assert _err(lib, lib.hyena_filter_gen(ctypes.byref(d), FAKE * 2, None), "include_t + 2F") == 1
     d = hy.FilterDesc(3, 0, 48, 0, 4, 0, 2, (ctypes.c_int * 3)(24, 64, 8), W, W, 0, None, None, FAKE, 1)
     assert lib.hyena_filter_gen(ctypes.byref(d), FAKE * 2, None) == 2
+    # unknown activation or window
+    d = hy.FilterDesc(1, 1024, 0, 0, 8, 1, 2, (ctypes.c_int * 3)(17, 32, 16), W, W, 7, None, None, FAKE, 1)
+    assert _err(lib, lib.hyena_filter_gen(ctypes.byref(d), FAKE * 2, None), "activation") == 1
+    d = hy.FilterDesc(1, 1024, 0, 0, 8, 1, 2, (ctypes.c_int * 3)(17, 32, 16), W, W, 2, None, None, FAKE, 1, None, 5)
+    assert _err(lib, lib.hyena_filter_gen(ctypes.byref(d), FAKE * 2, None), "window") == 1
 
 
 def test_host_entry_validation_and_workspace(lib):

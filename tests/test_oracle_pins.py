@@ -489,3 +489,36 @@ def test_backward_samples_equal_full_backward():
     np.testing.assert_allclose(sx, dxs[0], rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(sh, dh[0], rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(sD, dD[0], rtol=1e-12, atol=1e-12)
+
+
+def test_filter_gen_sine_and_gaussian_window_closed_forms():
+    """SIREN hidden layers with frequency 0 output sin(0) = 0, so the filter
+    is the last bias under the window: b_o exp(-alpha_o n^2) for the Gaussian
+    window (n = t/L in 1-D, |r|/g in 3-D); the identity activation makes the
+    MLP one affine map of the encoding."""
+    rng = np.random.default_rng(23)
+    L, F, nout = 64, 4, 3
+    Ws = [rng.standard_normal((16, 9)), rng.standard_normal((8, 16)), rng.standard_normal((nout, 8))]
+    bs = [rng.standard_normal(16), rng.standard_normal(8), rng.standard_normal(nout)]
+    alpha = rng.uniform(0.5, 3.0, nout)
+    h = oracle.filter_gen_1d(L, F, True, Ws, bs, alpha, act="sine", omega=np.zeros(24), window="gauss")
+    n = np.arange(L) / L
+    np.testing.assert_allclose(h, bs[2][:, None] * np.exp(-alpha[:, None] * n[None] ** 2), rtol=1e-14, atol=1e-14)
+    g = 4
+    Ws3 = [rng.standard_normal((16, 6 * 2)), rng.standard_normal((nout, 16))]
+    bs3 = [rng.standard_normal(16), rng.standard_normal(nout)]
+    idx = np.arange((2 * g) ** 3)
+    pts = oracle.filter_gen_3d_points(g, False, 2, Ws3, bs3, rng.standard_normal(16) * 0.1,
+                                      rng.standard_normal(16) * 0.1, alpha, idx, act="sine",
+                                      omega=np.zeros(16), window="gauss")
+    S = 2 * g
+    off = lambda i: np.where(i < S // 2, i, i - S)
+    r = np.stack([off(idx // (S * S)), off((idx // S) % S), off(idx % S)], 1)
+    inside = np.all(np.abs(r) < g, 1)
+    rn2 = np.sum(r.astype(np.float64) ** 2, 1) / g ** 2
+    ref = np.where(inside[:, None], bs3[1][None] * np.exp(-alpha[None] * rn2[:, None]), 0.0)
+    np.testing.assert_allclose(pts, ref, rtol=1e-14, atol=1e-14)
+    lin = oracle.filter_gen_1d(L, F, True, Ws, bs, alpha, act="identity")
+    pe = oracle.pe1d(L, F, True)
+    aff = ((pe @ Ws[0].T + bs[0]) @ Ws[1].T + bs[1]) @ Ws[2].T + bs[2]
+    np.testing.assert_allclose(lin, aff.T * np.exp(-alpha[:, None] * n[None]), rtol=1e-11, atol=1e-11)

@@ -137,6 +137,35 @@ def test_nd_filter_gen_small_grids(g, circular, hidden, nout):
         check(got[b].reshape(nout, -1), ref.T, "f32", "3-D filters g%d circ%d set %d" % (g, circular, b))
 
 
+@pytest.mark.parametrize("circular", [False, True])
+def test_nd_filter_gen_siren_gaussian(circular):
+    """HyenaND kernel synthesis: SIREN hidden layers (sin of per-unit
+    frequencies, FiLM on the first) under the Gaussian window."""
+    g, F, nout = 8, 3, 20
+    rng = np.random.default_rng(31 + circular)
+    widths = [6 * F, 32, 24, nout]
+    Ws = [rng.uniform(-1, 1, (b, a)).astype(np.float32) / np.sqrt(a) for a, b in zip(widths[:-1], widths[1:])]
+    bs = [rng.uniform(-0.5, 0.5, b).astype(np.float32) for b in widths[1:]]
+    # frequencies kept where fp32 pre-activations still give ~1e-6 phase error (the
+    # map x -> sin(omega x) amplifies rounding by omega)
+    omega = np.concatenate([rng.uniform(1, 8, 32), rng.uniform(0.5, 2, 24)]).astype(np.float32)
+    alpha = rng.uniform(0.5, 4.0, nout).astype(np.float32)
+    gam = rng.normal(0, 0.1, (2, 32)).astype(np.float32)
+    bet = rng.normal(0, 0.1, (2, 32)).astype(np.float32)
+    S = g if circular else 2 * g
+    h = torch.empty((2, nout, S, S, S), device="cuda")
+    hy.hyena_filter_gen(h, ndim=3, grid=g, circular=circular, Ws=[f32_dev(a) for a in Ws], bs=[f32_dev(a) for a in bs],
+                        alpha=f32_dev(alpha), n_freq=F, film_gamma=f32_dev(gam), film_beta=f32_dev(bet), n_sets=2,
+                        act=hy.HY_ACT_SINE, omega=f32_dev(omega), window=hy.HY_WIN_GAUSS)
+    torch.cuda.synchronize()
+    got = to_np(h)
+    idx = np.arange(S ** 3)
+    for b in range(2):
+        ref = oracle.filter_gen_3d_points(g, circular, F, Ws, bs, gam[b], bet[b], alpha, idx, act="sine",
+                                          omega=omega, window="gauss")
+        check(got[b].reshape(nout, -1), ref.T, "f32", "SIREN/Gaussian 3-D filters circ%d set %d" % (circular, b))
+
+
 def test_c4_full_size():
     """Workload 4 at full size: per-sample FiLM filters on the 128^3 transform
     grid, their spectra and the gated convolution of B2 D128 64^3.  Four slabs

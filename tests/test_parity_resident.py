@@ -153,6 +153,25 @@ def test_filter_gen_1d_shapes(L, F, include_t, hidden, nout, offset):
         assert np.isnan(to_np(flat[:offset])).all()
 
 
+@pytest.mark.parametrize("act,window", [("sine", "gauss"), ("identity", "exp"), ("sine", "exp")])
+def test_filter_gen_1d_activations_and_windows(act, window):
+    rng = np.random.default_rng(41)
+    L, F, nout = 3000, 8, 150
+    widths = [1 + 2 * F, 48, 40, nout]
+    Ws, bs = _mlp(rng, widths)
+    omega = rng.uniform(0.5, 8, 88).astype(np.float32) if act == "sine" else None
+    alpha = rng.uniform(0.2, 5.0, nout).astype(np.float32)
+    h = torch.empty((nout, L), device="cuda")
+    codes = {"silu": hy.HY_ACT_SILU, "identity": hy.HY_ACT_IDENTITY, "sine": hy.HY_ACT_SINE}
+    hy.hyena_filter_gen(h, ndim=1, L=L, Ws=[f32_dev(a) for a in Ws], bs=[f32_dev(a) for a in bs],
+                        alpha=f32_dev(alpha), n_freq=F, include_t=True, act=codes[act],
+                        omega=f32_dev(omega) if omega is not None else None,
+                        window=hy.HY_WIN_GAUSS if window == "gauss" else hy.HY_WIN_EXP)
+    torch.cuda.synchronize()
+    ref = oracle.filter_gen_1d(L, F, True, Ws, bs, alpha, act=act, omega=omega, window=window)
+    check(to_np(h), ref, "f32", "filter_gen %s/%s" % (act, window))
+
+
 def test_c1_end_to_end():
     """Workload 1 exactly: MLP parameters -> filters -> spectra -> operator."""
     w = hw.make("c1")

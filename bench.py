@@ -674,6 +674,49 @@ def run_backward(args):
                        "step_bytes": step_bytes}}), flush=True)
 
 
+def run_decode(args):
+    """One streaming decode step of the spectral gate at the gate workload's
+    shape (B4 H32 Dh64, n = 32768, bf16 tokens): the prefix-FFT cache of all
+    8192 rows is read and written once per step.  GB/s = (cache read + write,
+    gate, the step's x, x2 and y) / time."""
+    import torch
+    import implicit_long_convolution_b200 as hy
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    B, Hh, Dh, n = 4, 32, 64, 32768
+    nb = n // 2 + 1
+    g = torch.randn((Hh, nb), dtype=torch.complex64, device=dev)
+    cache = torch.zeros((B, Hh, Dh, nb), dtype=torch.complex64, device=dev)
+    x = torch.randn((B, Hh, Dh), device=dev).to(torch.bfloat16)
+    x2 = torch.randn_like(x)
+    y = torch.empty_like(x)
+    stream = torch.cuda.current_stream(dev)
+    for p in range(max(3, args.warmup)):
+        hy.spectral_gate_decode(x, g, cache, y, pos=p, x2=x2)
+    steps = args.steps if args.steps > 0 else 100
+    torch.cuda.synchronize()
+    barrier(world)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        hy.spectral_gate_decode(x, g, cache, y, pos=(args.warmup + i) % n, x2=x2)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(t0.elapsed_time(t1), world) / steps
+    rows = B * Hh * Dh
+    step_bytes = 2 * rows * nb * 8 + Hh * nb * 8 + 3 * rows * 2
+    if rank == 0:
+        print(json.dumps({
+            "metric": "spectral gate streaming decode GB/s (prefix-FFT cache, B4 H32 Dh64 n32768, bf16 tokens)",
+            "value": round(world * step_bytes / (ms / 1e3) / 1e9, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32 math, bf16 I/O", "data": "synthetic",
+            "tokens_per_s": round(world * B / (ms / 1e3), 1),
+            "config": {"workload": "spectral gate decode step B4 H32 Dh64 n32768", "B": B, "H": Hh, "Dh": Dh,
+                       "n": n, "step_bytes": step_bytes}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -683,6 +726,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(DESCR), default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode", action="store_true",
+                    help="time one streaming decode step of the spectral gate (prefix-FFT cache) instead")
     ap.add_argument("--backward", action="store_true",
                     help="time the operator's backward pass on the order-2 operator workload instead")
     ap.add_argument("--projection", action="store_true",
@@ -704,6 +749,9 @@ def main():
         return
     if args.backward:
         run_backward(args)
+        return
+    if args.decode:
+        run_decode(args)
         return
     run_ours(args)
 

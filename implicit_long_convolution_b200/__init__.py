@@ -24,6 +24,7 @@ __all__ = [
     "nd_conv_workspace", "spectral_gate", "operator_host_workspace", "hyena_operator_host",
     "spectral_gate_host_workspace", "spectral_gate_host", "nd_conv_host_workspace", "hyena_nd_conv_host",
     "projection_workspace", "hyena_projection", "operator_backward_workspace", "hyena_operator_backward",
+    "spectral_gate_decode",
     "STATUS",
 ]
 
@@ -102,6 +103,7 @@ def lib():
         "hyena_operator_backward": (_I, [_I, _I, _I, _I, _I, _VP, ctypes.POINTER(_VP), ctypes.POINTER(_VP),
                                          ctypes.POINTER(_VP), _VP, _VP, ctypes.POINTER(_VP), ctypes.POINTER(_VP),
                                          ctypes.POINTER(_VP), _VP, _SZ, _VP]),
+        "spectral_gate_decode": (_I, [_I, _I, _I, _I, _I, _I64, _VP, _VP, _I64, _VP, _VP, _VP, _VP]),
         "hyena_projection_workspace": (_SZ, []),
         "hyena_projection": (_I, [_I, _I, _I, _I, _I, _I, _VP, _VP, _VP, ctypes.POINTER(_VP), _VP, _SZ, _VP]),
         "hyena_nd_conv_host_workspace": (_SZ, [_I, ctypes.POINTER(_I), _I, _I, _I]),
@@ -326,3 +328,14 @@ def hyena_operator_backward(v, xs: Sequence, Hs: Sequence, dy, dv, dxs: Sequence
         _ptr(dy), _ptr(dv), _ptrs(dxs), _ptrs(dhs) if dhs is not None else None,
         _ptrs(dDs) if dDs is not None else None, _ptr(ws), wsb, _stream(stream)))
     return dv
+
+
+def spectral_gate_decode(x, g, cache, y, *, pos: int, x2=None, g_batch_stride: int = 0, stream=None):
+    """One streaming step at position pos: x, x2, y are (B, H, Dh) device
+    tensors (the new token's values), cache the (B, H, Dh, n/2+1) complex64
+    prefix spectrum, updated in place (see hyena.h)."""
+    B, Hh, Dh = x.shape
+    n = 2 * (cache.shape[-1] - 1)
+    _check(lib().spectral_gate_decode(B, Hh, Dh, n, _dt(x), pos, _ptr(x), _ptr(g), g_batch_stride, _ptr(x2),
+                                      _ptr(cache), _ptr(y), _stream(stream)))
+    return y

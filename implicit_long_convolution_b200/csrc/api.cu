@@ -202,7 +202,8 @@ hy_status hyena_filter_spectrum(int64_t rows, int ndim, const int *dims, int cir
     if (ndim == 1) {
         const int64_t L = dims[0];
         if (L < 1) return set_error(HY_ERR_INVALID_ARG, "hyena_filter_spectrum: L must be >= 1");
-        if (overlap(h, (size_t)rows * L * 4, H, (size_t)rows * (L + 2) * 8))
+        const int64_t bins = circular ? L / 2 + 1 : spectrum_m(L) + 1;
+        if (overlap(h, (size_t)rows * L * 4, H, (size_t)rows * bins * 8))
             return set_error(HY_ERR_INVALID_ARG, "hyena_filter_spectrum: H aliases h");
         if (circular) {
             if (!is_pow2(L) || L < 32 || L > 32768)
@@ -784,4 +785,34 @@ extern "C" hy_status hyena_operator_backward(int order, int B, int D, int L, hy_
         if ((st = bw_next_g(r, g, x[k], dt, Dskip ? Dskip[k] : nullptr, R, D, L, s)) != HY_OK) return st;
     }
     return bw_from_f32(g, dt, dv, n, s);
+}
+
+extern "C" hy_status spectral_gate_decode(int B, int H, int Dh, int n, hy_dtype dt, int64_t pos, const void *x,
+                                          const hy_c32 *g, int64_t g_batch_stride, const void *x2, hy_c32 *cache,
+                                          void *y, void *stream) {
+    clear_error();
+    const char *who = "spectral_gate_decode";
+    if (B < 1 || H < 1 || Dh < 1) return set_error(HY_ERR_INVALID_ARG, "%s: B, H, Dh must be >= 1", who);
+    if (dt != HY_F32 && dt != HY_BF16) return set_error(HY_ERR_INVALID_ARG, "%s: unknown dtype", who);
+    if (!is_pow2(n) || n < 2 || n > (1 << 24))
+        return set_error(HY_ERR_UNSUPPORTED, "%s: n must be a power of two in [2, 2^24]", who);
+    if (pos < 0 || pos >= n) return set_error(HY_ERR_INVALID_ARG, "%s: pos %lld outside [0, %d)", who, (long long)pos, n);
+    if (!x || !g || !cache || !y) return set_error(HY_ERR_INVALID_ARG, "%s: null pointer", who);
+    if (g_batch_stride < 0) return set_error(HY_ERR_INVALID_ARG, "%s: negative gate stride", who);
+    if (!aligned(g, 8) || !aligned(cache, 8)) return set_error(HY_ERR_INVALID_ARG, "%s: g and cache must be 8-byte aligned", who);
+    const int64_t rows = (int64_t)B * H * Dh;
+    const size_t esz = dt_size(dt);
+    if (overlap(cache, (size_t)rows * (n / 2 + 1) * 8, y, (size_t)rows * esz) ||
+        overlap(x, (size_t)rows * esz, y, (size_t)rows * esz))
+        return set_error(HY_ERR_INVALID_ARG, "%s: y aliases an input", who);
+    GateDecodeArgs a{};
+    a.rows = rows;
+    a.n = n;
+    a.pos = pos;
+    a.dh = Dh;
+    a.heads = H;
+    a.g = reinterpret_cast<const float2 *>(g);
+    a.g_batch_stride = g_batch_stride;
+    a.cache = reinterpret_cast<float2 *>(cache);
+    return launch_gate_decode(a, dt, x, x2, y, (cudaStream_t)stream);
 }

@@ -54,6 +54,19 @@ hy_status bw_dh(const float *w, float *dh, int B, int D, int L, cudaStream_t s);
 hy_status bw_dD(const float *g, const void *x, hy_dtype dt, const float *z, float *dD, int B, int D, int L,
                 cudaStream_t s);
 
+// streaming decode of the spectral gate with a prefix-FFT cache (decode.cu)
+struct GateDecodeArgs {
+    int64_t rows;                  // B * H * Dh
+    int n;                         // transform length (power of two)
+    int64_t pos;                   // position of the new token, 0 <= pos < n
+    int64_t dh, heads;             // gate row of row r: (r / dh) % heads, sample r / (dh * heads)
+    const float2 *g;
+    int64_t g_batch_stride;        // complex elements; 0 = shared
+    float2 *cache;                 // rows x (n/2 + 1), updated in place
+};
+hy_status launch_gate_decode(const GateDecodeArgs &a, hy_dtype dt, const void *x, const void *x2, void *y,
+                             cudaStream_t s);
+
 // N-D path (ndconv.cu)
 struct NDArgs {
     int g[3];                      // grid

@@ -171,6 +171,28 @@ hy_status hyena_operator(int order, int B, int D, int L, hy_dtype dt, const void
                          void *stream);
 
 /* ------------------------------------------------------------------------
+ * Streaming decode step of the spectral gate with a prefix-FFT cache
+ * ([SP] 토큰 믹서 구성과 생성 지원: the cache plays the role of a KV-cache so
+ * that autoregressive generation does not recompute the FFT every step).
+ *
+ *   cache: device (B, H, Dh, n/2 + 1) complex, the spectrum of the prefix
+ *   seen so far, X_k = Σ_{m < pos} x[m] e^{-2πi k m / n}: all zeros before
+ *   the first token, or a prompt's spectrum from hyena_filter_spectrum
+ *   (ndim = 1, dims = {n}, circular = 1, each row the prompt padded with
+ *   zeros to n).  One call consumes the token at position pos (0 <= pos <
+ *   n): x, x2, y are device (B, H, Dh) values at that position (dt), g the
+ *   gate as in spectral_gate.
+ *     X_k += x e^{-2πi k pos / n}             (cache updated in place)
+ *     y = x2 · (1/n) Σ_{k=0}^{n/2} c_k Re(g_k X_k e^{2πi k pos / n}),
+ *   c_0 = c_{n/2} = 1, c_k = 2 otherwise: the output of spectral_gate at
+ *   pos for the sequence with every later position zero.  x2 may be NULL.
+ *   n a power of two in [2, 2^24]; O(n) work per row per step.
+ * ---------------------------------------------------------------------- */
+hy_status spectral_gate_decode(int B, int H, int Dh, int n, hy_dtype dt, int64_t pos,
+                               const void *x, const hy_c32 *g, int64_t g_batch_stride,
+                               const void *x2, hy_c32 *cache, void *y, void *stream);
+
+/* ------------------------------------------------------------------------
  * Backward pass of the operator  ([HN] 아키텍처 상세, step 3, differentiated;
  * the pages train the operator but print no gradient formulas -- these are
  * the derivatives of the recurrence above.)

@@ -55,6 +55,7 @@ PINS = {
     "projection": "identity weights give the transposed input, zero weights the bias, linearity",
     "hyena_backward": "central finite differences of the direct forward (hyena_rows) for every input",
     "hyena_backward_samples": "equals hyena_backward (order 2) at every index",
+    "prefix_gate_outputs": "composition of gate_kernel and circular_conv_samples (pinned); first output x2 kappa[0] x",
 }
 
 
@@ -397,6 +398,21 @@ def circular_conv_samples(kappa, x1, x2, ts) -> np.ndarray:
         xp = _dp(x2)
     _load().orc_circular_conv_samples(ctypes.c_int64(kappa.shape[0]), _dp(kappa), _dp(x1), xp,
                                       ctypes.c_int64(ts.size), _ip(ts), _dp(out))
+    return out
+
+
+def prefix_gate_outputs(g, x1, x2, T: int) -> np.ndarray:
+    """Streaming reading of the spectral gate ([SP] 토큰 믹서 구성과 생성 지원):
+    output n < T is the full gated circular convolution of the sequence whose
+    positions after n are zero, at position n.  g: n/2+1 bins; x1, x2:
+    length-n rows (x2 may be None).  Returns (T,)."""
+    kap = gate_kernel(g)
+    x1 = _f64(x1)
+    out = np.empty(T)
+    for n in range(T):
+        xp = x1.copy()
+        xp[n + 1:] = 0.0
+        out[n] = circular_conv_samples(kap, xp, None if x2 is None else _f64(x2), [n])[0]
     return out
 
 

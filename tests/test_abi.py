@@ -151,3 +151,19 @@ def test_binding_raises_named_errors(lib):
     with pytest.raises(hy.HyenaError) as ei:
         hy._check(lib.spectral_gate(1, 1, 1, 100, 1, FAKE, FAKE, 0, None, FAKE * 2, None))
     assert ei.value.status_name == "HY_ERR_UNSUPPORTED"
+
+
+def test_spectrum_alias_check_uses_the_exact_extent(lib):
+    """The aliasing check covers exactly the spectrum's bins: a circular
+    spectrum (L/2+1 bins) right after the filters is accepted up to the
+    launch (which fails without a GPU only after validation), one that
+    overlaps is rejected; a ragged causal spectrum is M+1 bins long."""
+    one = (ctypes.c_int * 1)(512)
+    h = 0x100000
+    # rows = 2, L = 512: h spans 4096 bytes; a spectrum starting there does not alias
+    st = lib.hyena_filter_spectrum(2, 1, one, 1, h, h + 2 * 512 * 4, None, 0, None)
+    assert st != 1 or b"aliases" not in lib.hyena_last_error()
+    assert _err(lib, lib.hyena_filter_spectrum(2, 1, one, 1, h, h + 2 * 512 * 4 - 8, None, 0, None), "aliases") == 1
+    # ragged causal L = 1000 -> 1025 bins per row: a spectrum ending inside h aliases
+    ragged = (ctypes.c_int * 1)(1000)
+    assert _err(lib, lib.hyena_filter_spectrum(1, 1, ragged, 0, h, h - 1025 * 8 + 8, None, 0, None), "aliases") == 1

@@ -522,3 +522,17 @@ def test_filter_gen_sine_and_gaussian_window_closed_forms():
     pe = oracle.pe1d(L, F, True)
     aff = ((pe @ Ws[0].T + bs[0]) @ Ws[1].T + bs[1]) @ Ws[2].T + bs[2]
     np.testing.assert_allclose(lin, aff.T * np.exp(-alpha[:, None] * n[None]), rtol=1e-11, atol=1e-11)
+
+
+def test_prefix_gate_outputs_first_step_and_full_prefix():
+    """Streaming gate: the first output is x2[0] kappa[0] x[0]; the last one
+    (whole sequence seen) equals the full circular convolution there."""
+    rng = np.random.default_rng(24)
+    n = 32
+    g = rng.standard_normal(n // 2 + 1) + 1j * rng.standard_normal(n // 2 + 1)
+    x1, x2 = rng.standard_normal((2, n))
+    out = oracle.prefix_gate_outputs(g, x1, x2, n)
+    kap = oracle.gate_kernel(g)
+    assert abs(out[0] - x2[0] * kap[0] * x1[0]) < 1e-12
+    full = oracle.circular_conv_samples(kap, x1, x2, [n - 1])[0]
+    assert abs(out[-1] - full) < 1e-12

@@ -26,6 +26,7 @@ def _need_gpu():
     (2, 3, 4, 64, 64, "f32"),      # every position, cache wraps to the full sequence
     (1, 2, 8, 1024, 200, "f32"),
     (2, 2, 3, 4096, 50, "bf16"),
+    (1, 1, 2, 32768, 40, "f32"),   # the largest gate length
 ])
 def test_decode_steps_vs_oracle(B, Hh, Dh, n, T, dtype):
     rng = np.random.default_rng(n + T)

@@ -10,7 +10,9 @@
 // gated prefix spectrum at the one new position (only the real part of the
 // product counts at DC and Nyquist, as in the spectral gate).  One CTA per
 // row; each step reads and writes the row's cache once: O(n) per token
-// instead of the O(n log n) of a full transform.
+// instead of the O(n log n) of a full transform.  A thread's bins are NT
+// apart, so its twiddles advance by the fixed rotation e^{2πi NT pos/n},
+// recomputed exactly every 8th bin.
 #include <cuda_bf16.h>
 
 #include "kernels.h"
@@ -36,19 +38,46 @@ __global__ void __launch_bounds__(NT) gate_decode_kernel(const GateDecodeArgs a,
         const float2 *G = a.g + (row / (a.dh * a.heads)) * a.g_batch_stride + ((row / a.dh) % a.heads) * (int64_t)nb;
         float2 *X = a.cache + row * (int64_t)nb;
         float acc = 0.f;
-        for (int k = threadIdx.x; k < nb; k += NT) {
-            const uint64_t m = ((uint64_t)k * (uint64_t)a.pos) & mask;       // k pos mod n, exact
-            float s, c;
-            sincospif((float)(2 * m) / (float)a.n, &s, &c);                 // W = e^{+2πi m/n} = (c, s)
-            float2 Xk = X[k];
-            Xk.x = fmaf(xv, c, Xk.x);                                        // + x conj(W)
-            Xk.y = fmaf(-xv, s, Xk.y);
-            X[k] = Xk;
-            const float2 gk = __ldg(G + k);
-            const float pr = gk.x * Xk.x - gk.y * Xk.y;                      // P = G X
-            const float pi = gk.x * Xk.y + gk.y * Xk.x;
-            const float w = (k == 0 || k == nb - 1) ? 1.f : 2.f;
-            acc = fmaf(w, pr * c - pi * s, acc);                             // c_k Re(P W)
+        // this thread's bins k, k + NT, ...: W^{(k + NT) pos} = W^{k pos} W^{NT pos};
+        // exact every 8th bin, the step rotation in between (a few ulp).
+        // Bins go in groups of U whose cache and gate loads are all issued
+        // before any of them is used.
+        constexpr int U = 4;
+        float s1, c1;
+        sincospif((float)(2 * (((uint64_t)NT * (uint64_t)a.pos) & mask)) / (float)a.n, &s1, &c1);
+        float s = 0.f, c = 1.f;
+        int j = 0;
+        for (int k0 = threadIdx.x; k0 < nb; k0 += U * NT) {
+            float2 Xk[U], gk[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int k = k0 + u * NT;
+                if (k < nb) {
+                    Xk[u] = X[k];
+                    gk[u] = __ldg(G + k);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u, ++j) {
+                const int k = k0 + u * NT;
+                if (k >= nb) break;
+                if ((j & 7) == 0) {
+                    const uint64_t m = ((uint64_t)k * (uint64_t)a.pos) & mask;   // k pos mod n, exact
+                    sincospif((float)(2 * m) / (float)a.n, &s, &c);             // W = e^{+2πi m/n} = (c, s)
+                } else {
+                    const float cn = c * c1 - s * s1;
+                    s = fmaf(s, c1, c * s1);
+                    c = cn;
+                }
+                float2 v = Xk[u];
+                v.x = fmaf(xv, c, v.x);                                          // + x conj(W)
+                v.y = fmaf(-xv, s, v.y);
+                X[k] = v;
+                const float pr = gk[u].x * v.x - gk[u].y * v.y;                  // P = G X
+                const float pi = gk[u].x * v.y + gk[u].y * v.x;
+                const float w = (k == 0 || k == nb - 1) ? 1.f : 2.f;
+                acc = fmaf(w, pr * c - pi * s, acc);                             // c_k Re(P W)
+            }
         }
         for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
         __shared__ float part[NT / 32];

@@ -42,7 +42,7 @@ __global__ void __launch_bounds__(NT) gate_decode_kernel(const GateDecodeArgs a,
         // exact every 8th bin, the step rotation in between (a few ulp).
         // Bins go in groups of U whose cache and gate loads are all issued
         // before any of them is used.
-        constexpr int U = 4;
+        constexpr int U = 8;
         float s1, c1;
         sincospif((float)(2 * (((uint64_t)NT * (uint64_t)a.pos) & mask)) / (float)a.n, &s1, &c1);
         float s = 0.f, c = 1.f;

@@ -446,6 +446,7 @@ def run_ours(args):
 
     cfg = {"workload": DESCR[name] + (" [D=%d profiling case]" % s["D"] if over else "")}
     cfg.update({k: v for k, v in s.items() if k in ("B", "D", "L", "order", "H", "Dh", "grid")})
+    cfg["io_dtype"] = s["dtype"]
     cfg.update({"step": ("filter_gen + filter_spectrum + convolution" if s["kind"] != "gate"
                          else "spectral_gate"),
                 "step_bytes": step_bytes, "conv_bytes": op_bytes,
@@ -464,7 +465,7 @@ def run_ours(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f32 math, %s I/O" % s["dtype"],
+        "dtype": "f32",
         "data": "synthetic (seeded N(0,1) signals, random-init filter MLP)",
         "config": cfg,
         "tokens_channels_per_s": round(world * steps * (hw.signal_bytes(s) // el) / sec, 1),
@@ -614,11 +615,12 @@ def run_projection(args):
             "metric": "input projection TFLOP/s (B8 L8192, 768 -> 2 x 768, bf16, channel-major outputs + bias)",
             "value": round(tf, 1), "unit": "TFLOP/s", "n_gpus": world, "steps": steps, "warmup": args.warmup,
             "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16 (fp32 accumulate)", "data": "synthetic",
+            "dtype": "bf16", "data": "synthetic",
             "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(tf / world / peak, 4) if peak else None, "traffic": None},
             "config": {"workload": "hyena input projection at the order-2 operator width",
-                       "B": B, "L": L, "C": C, "D": D, "n_out": n_out}}), flush=True)
+                       "B": B, "L": L, "C": C, "D": D, "n_out": n_out,
+                       "accumulate": "f32"}}), flush=True)
 
 
 def run_backward(args):
@@ -669,9 +671,9 @@ def run_backward(args):
             "metric": "Hyena op backward GB/s (order-2 operator B8 D768 L8192 bf16: dv, dx1, dh1, dD1)",
             "value": round(world * step_bytes / (ms / 1e3) / 1e9, 2), "unit": "GB/s", "n_gpus": world,
             "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32 math, bf16 I/O", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": "hyena order-2 operator backward B8 D768 L8192 bf16", "B": B, "D": D, "L": L,
-                       "step_bytes": step_bytes}}), flush=True)
+                       "io_dtype": "bf16", "step_bytes": step_bytes}}), flush=True)
 
 
 def run_decode(args):
@@ -711,10 +713,10 @@ def run_decode(args):
             "metric": "spectral gate streaming decode GB/s (prefix-FFT cache, B4 H32 Dh64 n32768, bf16 tokens)",
             "value": round(world * step_bytes / (ms / 1e3) / 1e9, 2), "unit": "GB/s", "n_gpus": world,
             "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32 math, bf16 I/O", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "tokens_per_s": round(world * B / (ms / 1e3), 1),
             "config": {"workload": "spectral gate decode step B4 H32 Dh64 n32768", "B": B, "H": Hh, "Dh": Dh,
-                       "n": n, "step_bytes": step_bytes}}), flush=True)
+                       "n": n, "io_dtype": "bf16", "step_bytes": step_bytes}}), flush=True)
 
 
 def main():

@@ -78,7 +78,7 @@ def workload_bytes(spec):
     return op, op
 
 
-CONV_SOURCES = ["common.cuh", "fft_core.cuh", "resident.cuh", "resident_launch.cuh", "resident.cu",
+CONV_SOURCES = ["bulk_copy.cuh", "common.cuh", "fft_core.cuh", "resident.cuh", "resident_launch.cuh", "resident.cu",
                 "resident_stream_bf16.cu", "resident_stream_f32.cu", "twiddle.cu", "twiddle.h"]
 
 
@@ -269,7 +269,10 @@ def setup_operator(w, dev, hy, torch):
         st.kernel = "multi-pass colpass/rowpass kernels (M=2^%d)" % (M.bit_length() - 1)
     else:
         op_l = 1
-        st.kernel = "resident_conv_kernel<M=2^%d>" % (M.bit_length() - 1)
+        # one order over power-of-two rows runs the persistent streaming kernel
+        stream = K == 1 and L == M and M >= 64
+        st.kernel = "%s<M=2^%d>" % ("resident_stream_kernel" if stream else "resident_conv_kernel",
+                                    M.bit_length() - 1)
     spec_l = 2 * -(-(K * D) // max(1, wsf // (12 * M))) if wsf else 1
     st.launches = 1 + spec_l + op_l
     return st
@@ -337,7 +340,7 @@ def setup_gate(w, dev, hy, torch):
     st.inputs = [(x, w.v), (x2, w.xs[0])]
     st.output = y
     st.launches = 1
-    st.kernel = "resident_conv_kernel<M=2^%d, circular>" % ((s["L"] // 2).bit_length() - 1)
+    st.kernel = "resident_stream_kernel<M=2^%d, circular>" % ((s["L"] // 2).bit_length() - 1)
     return st
 
 

@@ -24,7 +24,7 @@ __all__ = [
     "nd_conv_workspace", "spectral_gate", "operator_host_workspace", "hyena_operator_host",
     "spectral_gate_host_workspace", "spectral_gate_host", "nd_conv_host_workspace", "hyena_nd_conv_host",
     "projection_workspace", "hyena_projection", "operator_backward_workspace", "hyena_operator_backward",
-    "spectral_gate_decode",
+    "spectral_gate_decode", "device_faults", "selftest_bounded_wait",
     "STATUS",
 ]
 
@@ -35,6 +35,7 @@ STATUS = {0: "HY_OK", 1: "HY_ERR_INVALID_ARG", 2: "HY_ERR_UNSUPPORTED", 3: "HY_E
 HY_F32, HY_BF16 = 0, 1
 HY_ACT_SILU, HY_ACT_IDENTITY, HY_ACT_SINE = 0, 1, 2
 HY_WIN_EXP, HY_WIN_GAUSS = 0, 1
+HY_FAULT_STREAM_INPUT, HY_FAULT_STREAM_GATE, HY_FAULT_SELFTEST = 0x1, 0x2, 0x80000000
 
 
 class HyenaLibraryMissing(RuntimeError):
@@ -111,6 +112,8 @@ def lib():
                                     _VP, _SZ, _VP]),
         "spectral_gate_host_workspace": (_SZ, [_I, _I, _I, _I, _I]),
         "spectral_gate_host": (_I, [_I, _I, _I, _I, _I, _VP, _VP, _I64, _VP, _VP, _VP, _SZ, _VP]),
+        "hyena_device_faults": (_I, [ctypes.POINTER(ctypes.c_uint32), _I, _VP]),
+        "hyena_selftest_bounded_wait": (_I, [ctypes.c_uint32, _VP]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -339,3 +342,21 @@ def spectral_gate_decode(x, g, cache, y, *, pos: int, x2=None, g_batch_stride: i
     _check(lib().spectral_gate_decode(B, Hh, Dh, n, _dt(x), pos, _ptr(x), _ptr(g), g_batch_stride, _ptr(x2),
                                       _ptr(cache), _ptr(y), _stream(stream)))
     return y
+
+
+def device_faults(*, clear: bool = True, stream=None) -> int:
+    """The current device's fault word (HY_FAULT_* bits) once the work queued
+    on `stream` has finished; 0 when no bounded device wait gave up.  Unlike
+    the other calls this does not raise on HY_ERR_TIMEOUT: it returns the
+    bits (and resets them when `clear`)."""
+    v = ctypes.c_uint32(0)
+    st = lib().hyena_device_faults(ctypes.byref(v), int(clear), _stream(stream))
+    if st not in (0, 5):
+        _check(st)
+    return int(v.value)
+
+
+def selftest_bounded_wait(limit_us: int = 2000, *, stream=None):
+    """Launch the bounded-wait self-test: a wait that can never be satisfied
+    runs out after limit_us and records HY_FAULT_SELFTEST."""
+    _check(lib().hyena_selftest_bounded_wait(limit_us, _stream(stream)))

@@ -16,6 +16,7 @@
 // which makes every order a linear, causal convolution.  In the circular
 // variant (spectral gate) n = L and nothing is padded.
 #pragma once
+#include "bulk_copy.cuh"
 #include "fft_core.cuh"
 
 namespace hy {
@@ -44,6 +45,7 @@ struct ResidentParams {
     float scale;                 // 1 / (2n): folds the halving of split and the 1/n
     const float2 *tw_fft;
     const float2 *tw_split;
+    uint32_t *fault;             // device fault word (bounded waits), or NULL
 };
 
 // The skip term folds into the spectrum: h * u + D u = (h + D delta) * u, and
@@ -236,19 +238,15 @@ resident_conv_kernel(const ResidentParams p) {
 // ----------------------------------------------------------------------------
 // Streaming variant for one order (K = 1) with L = 2^LOG_M (causal) or
 // L = 2^(LOG_M+1) (circular) samples per row: a persistent CTA walks its rows
-// and overlaps HBM with the FFTs.  While row r is being transformed, cp.async
-// brings row r+1's input and row r's gate into shared memory (stage buffers
-// next to the FFT exchange buffer); the skip term rides on the spectrum (see
-// split_multiply_merge).  Without PF_GATE (when two stage buffers would not
-// fit) the gate is read from global memory in the epilogue.
+// and overlaps HBM with the FFTs.  While row r is being transformed, TMA bulk
+// copies bring row r+1's input and row r's gate into shared memory (stage
+// buffers next to the FFT exchange buffer), each landing on its own mbarrier;
+// the skip term rides on the spectrum (see split_multiply_merge).  Without
+// PF_GATE (when two stage buffers would not fit) the gate is read from
+// global memory in the epilogue.  Every wait is bounded: a copy that has not
+// landed within the limit records a fault bit, and the CTA stops at the next
+// row boundary (after waiting, again bounded, for its copies in flight).
 // ----------------------------------------------------------------------------
-__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
-    const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // float2 slots before the stage buffers (even, so they start 16-byte aligned)
 __host__ __device__ constexpr int stream_stage_offset(int m) { return ((spad_size(m) + 1) / 2) * 2; }
@@ -273,27 +271,36 @@ resident_stream_kernel(const ResidentParams p) {
     constexpr int T = M / P;
     constexpr int PIN = CIRC ? P : P / 2;
     constexpr int L = CIRC ? 2 * M : M;                  // samples per row
-    constexpr int CHUNKS = L * (int)sizeof(IO) / 16;     // 16-byte copies per row
+    constexpr uint32_t ROW_BYTES = (uint32_t)(L * sizeof(IO));
+    static_assert(ROW_BYTES % 16 == 0 && ROW_BYTES < (1u << 20), "bulk copy size");
     using IOT = IOTraits<IO>;
 
-    extern __shared__ float2 smem[];
+    extern __shared__ __align__(128) float2 smem[];   // stage buffers take 16-byte aligned bulk copies
     float2 *sbuf = smem;
     IO *in_st = reinterpret_cast<IO *>(smem + stream_stage_offset(M));   // 16-byte aligned
     IO *g_st = in_st + L;
+    __shared__ uint64_t bars[2];                         // [0]: input stage, [1]: gate stage
+    __shared__ int s_abort;
 
-    const int t = threadIdx.x;
     const IO *ubase = reinterpret_cast<const IO *>(p.u);
     const IO *gbase = reinterpret_cast<const IO *>(p.gate[0]);
     IO *ybase = reinterpret_cast<IO *>(p.y);
+    const bool gate_pf = PF_GATE && gbase != nullptr;
     auto row_of = [&](int64_t c) { return p.remap ? (c % p.B) * (int64_t)p.D + c / p.B : c; };
-    auto copy_row = [&](IO *dst, const IO *src) {
-        for (int i = t; i < CHUNKS; i += T)
-            cp_async16(reinterpret_cast<char *>(dst) + 16 * i, reinterpret_cast<const char *>(src) + 16 * i);
-    };
 
     int64_t c = blockIdx.x;
-    if (c < p.n_rows) copy_row(in_st, ubase + row_of(c) * L);
-    cp_async_commit();
+    if (threadIdx.x == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        mbar_init_fence();
+        s_abort = 0;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && c < p.n_rows) bulk_g2s(in_st, ubase + row_of(c) * L, ROW_BYTES, &bars[0]);
+    // waits taken on each barrier; every copy issued is waited on by the
+    // iteration that issued it (gate) or the next one (input), so at any
+    // exit of the loop these are also the copies issued
+    uint32_t w_in = 0, w_g = 0;
     for (; c < p.n_rows; c += gridDim.x) {
         // the thread index re-read per row (volatile) so the addresses derived
         // from it are formed inside the loop instead of held across it
@@ -302,8 +309,11 @@ resident_stream_kernel(const ResidentParams p) {
         const int64_t row = row_of(c);
         const int64_t ch = (row / p.sdiv) % p.smod;
         const int64_t smp = row / (p.sdiv * p.smod);
-        cp_async_wait<0>();
-        __syncthreads();
+        if (!mbar_wait(&bars[0], w_in & 1)) {
+            record_fault(p.fault, HY_FAULT_STREAM_INPUT);
+            s_abort = 1;
+        }
+        ++w_in;
         float2 x[P];
 #pragma unroll
         for (int m = 0; m < P; ++m) {
@@ -318,11 +328,13 @@ resident_stream_kernel(const ResidentParams p) {
                 }
             }
         }
-        __syncthreads();                                  // stage buffer free for the next row
-        if (PF_GATE && gbase) copy_row(g_st, gbase + row * L);
-        cp_async_commit();
-        if (c + gridDim.x < p.n_rows) copy_row(in_st, ubase + row_of(c + gridDim.x) * L);
-        cp_async_commit();
+        __syncthreads();                                  // stage buffers free for the next copies
+        if (s_abort) break;                               // uniform: read between two barriers
+        if (t == 0) {
+            fence_proxy_async_smem();
+            if (gate_pf) bulk_g2s(g_st, gbase + row * L, ROW_BYTES, &bars[1]);
+            if (c + gridDim.x < p.n_rows) bulk_g2s(in_st, ubase + row_of(c + gridDim.x) * L, ROW_BYTES, &bars[0]);
+        }
 
         block_fft<LOG_M, LOG_P, -1, !CIRC>(x, sbuf, t, p.tw_fft);
         const float dk = p.skip[0] ? ldv(p.skip[0] + ch) : 0.f;
@@ -330,9 +342,12 @@ resident_stream_kernel(const ResidentParams p) {
         split_multiply_merge<LOG_M, LOG_P>(x, sbuf, t, H, p.tw_split, dk);
         block_fft<LOG_M, LOG_P, +1, false>(x, sbuf, t, p.tw_fft);
 
-        if constexpr (PF_GATE) {
-            cp_async_wait<1>();                           // the gate of this row has landed
-            __syncthreads();
+        if (gate_pf) {
+            if (!mbar_wait(&bars[1], w_g & 1)) {          // the gate of this row has landed
+                record_fault(p.fault, HY_FAULT_STREAM_GATE);
+                s_abort = 1;                              // seen after the next row's first barrier
+            }
+            ++w_g;
         }
         IO *yout = ybase + row * (int64_t)L;
 #pragma unroll
@@ -341,7 +356,7 @@ resident_stream_kernel(const ResidentParams p) {
             float2 z = make_float2(x[m].x * p.scale, x[m].y * p.scale);
             if (gbase) {
                 float2 gv;
-                if constexpr (PF_GATE) {
+                if (gate_pf) {
                     if constexpr (sizeof(IO) == 2) {
                         const uint32_t b = *reinterpret_cast<const uint32_t *>(g_st + i0);
                         gv = make_float2(__uint_as_float(b << 16), __uint_as_float(b & 0xffff0000u));
@@ -356,7 +371,11 @@ resident_stream_kernel(const ResidentParams p) {
             IOT::store2(yout + i0, z);
         }
     }
-    cp_async_wait<0>();
+    // no copy may still be landing in shared memory when the CTA exits
+    if (threadIdx.x == 0) {
+        if (w_in && !mbar_wait(&bars[0], (w_in - 1) & 1)) record_fault(p.fault, HY_FAULT_STREAM_INPUT);
+        if (w_g && !mbar_wait(&bars[1], (w_g - 1) & 1)) record_fault(p.fault, HY_FAULT_STREAM_GATE);
+    }
 }
 
 // Filter spectrum rows: H[r, k] = Σ_t h[r, t] W_n^{kt}, k = 0..M, for rows of

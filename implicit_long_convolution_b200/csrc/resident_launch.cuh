@@ -46,7 +46,7 @@ hy_status dispatch_conv(int log_m, const ResidentParams &p, cudaStream_t s) {
     }
 }
 
-// ---- streaming (persistent, cp.async prefetch) variant
+// ---- streaming (persistent, TMA bulk-copy prefetch) variant
 int device_sm_count();
 
 template <int LOG_M, typename IO, bool CIRC>
@@ -58,6 +58,8 @@ hy_status launch_stream_t(ResidentParams p, cudaStream_t s) {
     p.tw_fft = tw_stages(LOG_M, LOG_P);
     p.tw_split = tw_split(LOG_M);
     if (!p.tw_fft || !p.tw_split) return set_error(HY_ERR_CUDA, "twiddle tables missing for M=2^%d", LOG_M);
+    p.fault = device_fault_word();
+    if (!p.fault) return set_error(HY_ERR_CUDA, "device fault word unavailable");
     const size_t smem = stream_smem_bytes(LOG_M, (int)sizeof(IO), CIRC, PF);
     auto kernel = resident_stream_kernel<LOG_M, IO, CIRC, PF>;
     hy_status st = set_smem_limit(kernel, smem, "stream conv smem attribute");

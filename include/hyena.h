@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define HYENA_ABI_VERSION 2
+#define HYENA_ABI_VERSION 3
 
 typedef enum hy_status {
     HY_OK = 0,
@@ -52,7 +52,7 @@ typedef enum hy_status {
     HY_ERR_UNSUPPORTED = 2,   /* a valid request outside what is built    */
     HY_ERR_WORKSPACE = 3,     /* workspace missing or too small           */
     HY_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed      */
-    HY_ERR_TIMEOUT = 5        /* reserved: a bounded device wait gave up   */
+    HY_ERR_TIMEOUT = 5        /* a bounded device wait gave up (hyena_device_faults) */
 } hy_status;
 
 typedef enum hy_dtype { HY_F32 = 0, HY_BF16 = 1 } hy_dtype;
@@ -354,6 +354,26 @@ hy_status spectral_gate_host(int B, int H, int Dh, int L, hy_dtype dt, const voi
 /* ------------------------------------------------------------------------
  * Library state and errors
  * ---------------------------------------------------------------------- */
+/* Device faults.  No kernel traps or waits without limit.  The streaming
+ * convolution (one order over 16-byte aligned power-of-two rows) stages rows
+ * with TMA bulk copies that complete on mbarriers; each wait gives up after
+ * about one second of %globaltimer, ORs a bit below into a per-device fault
+ * word (a static device variable; nothing is allocated) and the CTA returns
+ * at its next row boundary, after a bounded wait for its copies in flight.
+ * The outputs of such a launch are then undefined. */
+#define HY_FAULT_STREAM_INPUT 0x1u      /* a row's input copy did not land in time */
+#define HY_FAULT_STREAM_GATE 0x2u       /* a row's gate copy did not land in time  */
+#define HY_FAULT_SELFTEST 0x80000000u   /* hyena_selftest_bounded_wait ran out      */
+/* Reads the current device's fault word into *faults after the work queued on
+ * `stream` has finished (the call synchronises that stream); clear != 0 then
+ * resets it (queued on `stream`).  Returns HY_ERR_TIMEOUT when any bit was
+ * set, HY_OK when none, HY_ERR_INVALID_ARG for a null `faults`. */
+hy_status hyena_device_faults(uint32_t *faults, int clear, void *stream);
+/* Diagnostic for the failure path: launches one CTA whose wait on an
+ * mbarrier that can never complete runs out after limit_us microseconds
+ * (1..1000000); it records HY_FAULT_SELFTEST and returns, leaving the
+ * context usable.  Read the result with hyena_device_faults. */
+hy_status hyena_selftest_bounded_wait(uint32_t limit_us, void *stream);
 /* Uploads the constant twiddle tables to the current device.  Called
  * implicitly by the first call on each device; that first call blocks the
  * host briefly and must not be made while a stream is being captured.  */

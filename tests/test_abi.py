@@ -35,12 +35,21 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_strings(lib):
-    assert lib.hyena_abi_version() == 2
+    assert lib.hyena_abi_version() == 3
     assert lib.hyena_status_string(3) == b"HY_ERR_WORKSPACE"
     assert lib.hyena_spectrum_bins(8192) == 8193
     assert lib.hyena_spectrum_bins(1000) == 1025
     assert lib.hyena_spectrum_bins(1) == 17
     assert lib.hyena_spectrum_bins(0) == 0
+
+
+def test_fault_api_validation(lib):
+    # host-side checks only: a null output and an out-of-range limit are
+    # rejected before the device is touched
+    assert _err(lib, lib.hyena_device_faults(None, 1, None), "null output") == 1
+    assert _err(lib, lib.hyena_selftest_bounded_wait(0, None), "limit") == 1
+    assert _err(lib, lib.hyena_selftest_bounded_wait(2000000, None), "limit") == 1
+    assert lib.hyena_status_string(5) == b"HY_ERR_TIMEOUT"
 
 
 def _err(lib, status, substring):

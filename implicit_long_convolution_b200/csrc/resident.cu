@@ -45,7 +45,7 @@ hy_status launch_resident_conv(const ResidentParams &p, int log_m, hy_dtype dt, 
     if (p.n_rows > 0x7fffffffLL) return set_error(HY_ERR_UNSUPPORTED, "too many rows (%lld)", (long long)p.n_rows);
     const bool chain = p.K > 1;
     // one order over whole power-of-two rows, 16-byte aligned: the persistent
-    // streaming kernel (cp.async prefetch of inputs and gate)
+    // streaming kernel (TMA bulk-copy prefetch of inputs and gate)
     const int64_t full = circular ? (int64_t)2 << log_m : (int64_t)1 << log_m;
     const int esz = dt == HY_BF16 ? 2 : 4;
     const bool fits = stream_smem_bytes(log_m, esz, circular, false) <= (size_t)227 * 1024;

@@ -35,7 +35,7 @@ STATUS = {0: "HY_OK", 1: "HY_ERR_INVALID_ARG", 2: "HY_ERR_UNSUPPORTED", 3: "HY_E
 HY_F32, HY_BF16 = 0, 1
 HY_ACT_SILU, HY_ACT_IDENTITY, HY_ACT_SINE = 0, 1, 2
 HY_WIN_EXP, HY_WIN_GAUSS = 0, 1
-HY_FAULT_STREAM_INPUT, HY_FAULT_STREAM_GATE, HY_FAULT_FILTER_MMA, HY_FAULT_SELFTEST = 0x1, 0x2, 0x4, 0x80000000
+HY_FAULT_STREAM_INPUT, HY_FAULT_STREAM_GATE, HY_FAULT_SELFTEST = 0x1, 0x2, 0x80000000
 
 
 class HyenaLibraryMissing(RuntimeError):

@@ -360,12 +360,9 @@ hy_status spectral_gate_host(int B, int H, int Dh, int L, hy_dtype dt, const voi
  * about one second of %globaltimer, ORs a bit below into a per-device fault
  * word (a static device variable; nothing is allocated) and the CTA returns
  * at its next row boundary, after a bounded wait for its copies in flight.
- * The filter generator waits the same way for its tensor-core MMAs
- * (HY_FAULT_FILTER_MMA); it then skips its remaining tiles and frees its
- * tensor memory.  The outputs of such a launch are then undefined. */
+ * The outputs of such a launch are then undefined. */
 #define HY_FAULT_STREAM_INPUT 0x1u      /* a row's input copy did not land in time */
 #define HY_FAULT_STREAM_GATE 0x2u       /* a row's gate copy did not land in time  */
-#define HY_FAULT_FILTER_MMA 0x4u        /* filter generator: tensor-core MMAs did not complete in time */
 #define HY_FAULT_SELFTEST 0x80000000u   /* hyena_selftest_bounded_wait ran out      */
 /* Reads the current device's fault word into *faults after the work queued on
  * `stream` has finished (the call synchronises that stream); clear != 0 then

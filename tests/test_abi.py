@@ -43,6 +43,21 @@ def test_version_and_strings(lib):
     assert lib.hyena_spectrum_bins(0) == 0
 
 
+def test_header_constants_match_binding():
+    """Every enum value and fault bit the header defines that the binding
+    mirrors has the same value there (no GPU, no library call)."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    consts = {m.group(1): int(m.group(2)) for m in re.finditer(r"\b(HY_[A-Z0-9_]+)\s*=\s*(\d+)", src)}
+    consts.update({m.group(1): int(m.group(2), 16)
+                   for m in re.finditer(r"#define\s+(HY_FAULT_[A-Z_]+)\s+0x([0-9a-fA-F]+)u", src)})
+    mirrored = [k for k in consts if hasattr(hy, k)]
+    assert len(mirrored) >= 10, mirrored
+    for k in mirrored:
+        assert getattr(hy, k) == consts[k], k
+    for code, name in hy.STATUS.items():
+        assert consts[name] == code, name
+
+
 def test_fault_api_validation(lib):
     # host-side checks only: a null output and an out-of-range limit are
     # rejected before the device is touched

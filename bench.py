@@ -115,17 +115,74 @@ def measured_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
+    """SM clock and clock-event reasons sampled DURING the timed region.
+
+    Read-only NVML queries from a thread of this process every ~1 ms (so even
+    a timed region of a few milliseconds has samples); nvidia-smi at 100 ms
+    when NVML cannot be used.  Nothing is set on the GPU."""
     Q = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits (nvml.h): sw power cap, hw slowdown, sw / hw thermal
+    BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40}
 
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.thread = None
+        self.samples = []
+        self.stop_flag = False
+        self.f = None
+        self.nvml = None
+        self.handle = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = self._handle(pynvml, index)
+        except Exception:
+            self.nvml = None
+
+    @staticmethod
+    def _handle(pynvml, index):
+        """The NVML handle of CUDA device `index` (matched by UUID, so a
+        CUDA_VISIBLE_DEVICES remap is honoured)."""
+        try:
+            import torch
+            want = str(torch.cuda.get_device_properties(index).uuid).lower()
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                u = (u.decode() if isinstance(u, bytes) else u).lower()
+                if u.replace("gpu-", "") == want.replace("gpu-", ""):
+                    return h
+        except Exception:
+            pass
+        return pynvml.nvmlDeviceGetHandleByIndex(index)
+
+    def _poll(self):
+        nv, h = self.nvml, self.handle
+        reasons_fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        while not self.stop_flag:
+            try:
+                self.samples.append((time.time(), nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                     int(reasons_fn(h))))
+            except Exception:
+                pass
+            time.sleep(0.001)
 
     def start(self):
+        if self.nvml is not None:
+            import threading
+            try:
+                self.max_mhz = self.nvml.nvmlDeviceGetMaxClockInfo(self.handle, self.nvml.NVML_CLOCK_SM)
+            except Exception:
+                self.max_mhz = None
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
@@ -135,6 +192,16 @@ class ClockSampler:
             self.proc = None
 
     def stop(self, t_begin=None, t_end=None):
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join(5)
+            rows = [r for r in self.samples
+                    if t_begin is None or (t_begin - 0.002 <= r[0] <= t_end + 0.002)]
+            if not rows:
+                return None
+            reasons = sorted({n for r in rows for n, b in self.BITS.items() if r[2] & b})
+            return {"sm_mhz": statistics.median(r[1] for r in rows), "sm_max_mhz": self.max_mhz,
+                    "reasons": reasons, "samples": len(rows), "source": "nvml in-process, ~1 ms"}
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -165,7 +232,8 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows),
+                "source": "nvidia-smi, 100 ms"}
 
 
 def dist_setup():
@@ -207,6 +275,21 @@ def rank_seed(name, rank):
 def job_value(world, steps, step_bytes, max_ms):
     """Whole-job GB/s: the bytes of every rank's steps over the slowest rank's time."""
     return world * steps * step_bytes / (max_ms / 1e3) / 1e9
+
+
+def workload_config(name, s, world, over=None):
+    """The `config` object of a bench line (the same for both arms)."""
+    step_bytes, op_bytes = workload_bytes(s)
+    cfg = {"workload": DESCR[name] + (" [D=%d profiling case]" % s["D"] if over else "")}
+    cfg.update({k: v for k, v in s.items() if k in ("B", "D", "L", "order", "H", "Dh", "grid")})
+    cfg["io_dtype"] = s["dtype"]
+    cfg.update({"step": ("filter_gen + filter_spectrum + convolution" if s["kind"] != "gate"
+                         else "spectral_gate"),
+                "step_bytes": step_bytes, "conv_bytes": op_bytes,
+                "l2": ("inputs larger than L2 (%.0f MB streamed per step vs 126 MB); no flush" % (op_bytes / 1e6)
+                       if op_bytes > 126e6 else "inputs smaller than L2 (no flush): launch-bound case"),
+                "parallelism": "independent replicas x%d (no data-path collective)" % world})
+    return cfg
 
 
 # ------------------------------------------------------------------ setups
@@ -447,15 +530,7 @@ def run_ours(args):
     h2d = sum(hh.numel() * hh.element_size() for hh in hosts)
     d2h = out_h.numel() * out_h.element_size()
 
-    cfg = {"workload": DESCR[name] + (" [D=%d profiling case]" % s["D"] if over else "")}
-    cfg.update({k: v for k, v in s.items() if k in ("B", "D", "L", "order", "H", "Dh", "grid")})
-    cfg["io_dtype"] = s["dtype"]
-    cfg.update({"step": ("filter_gen + filter_spectrum + convolution" if s["kind"] != "gate"
-                         else "spectral_gate"),
-                "step_bytes": step_bytes, "conv_bytes": op_bytes,
-                "l2": ("inputs larger than L2 (%.0f MB streamed per step vs 126 MB); no flush" % (op_bytes / 1e6)
-                       if op_bytes > 126e6 else "inputs smaller than L2 (no flush): launch-bound case"),
-                "parallelism": "independent replicas x%d (no data-path collective)" % world})
+    cfg = workload_config(name, s, world, over)
     el = 2 if s["dtype"] == "bf16" else 4
     line = {
         "metric": "Hyena op GB/s (%s)" % cfg["workload"],
@@ -483,9 +558,8 @@ def run_ours(args):
         "gpu_launches": st.launches * steps,
         "clocks": ck,
     }
-    if (rank == 0 and world == 1 and not args.no_cpu_baseline and s["kind"] == "operator"
-            and s["L"] <= 16384):
-        line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -496,80 +570,168 @@ def run_ours(args):
 
 # ------------------------------------------------------------------ oracle arm
 
-def cpu_baseline(w, budget_s=12.0):
-    """The float64 oracle as it stands on a bounded sample of the workload:
-    the filter MLP for all L positions plus the direct O(L^2) gated chain on
-    as many rows as fit the time budget; the value scales the sample to one
-    whole step (rows are independent, so row time scales linearly)."""
-    import oracle
-    s = w.spec
-    B, D, L, K = s["B"], s["D"], s["L"], s["order"] - 1
-    step_bytes, _ = workload_bytes(s)
-    rows_total = B * D
-    t0 = time.perf_counter()
-    h64 = oracle.filter_gen_1d(L, s["F"], True, w.Ws, w.bs, w.alpha)
-    t_filter = time.perf_counter() - t0
-    cores = oracle.threads()
-    # growing batches of distinct random rows until the sample has used about
-    # the budget (the rate of a small batch is not a good predictor)
-    order = np.random.default_rng(0).permutation(rows_total)
-    done, t_rows, n = 0, 0.0, min(rows_total, max(cores, 8))
-    while done < rows_total:
-        batch = order[done:done + n]
+class CpuSample:
+    """One bounded sample of a workload, run by the float64 oracle (the
+    direct definitions) and by the naive float64 FFT reference.
+
+    `run_oracle()` / `run_fft()` each execute the sample once; `frac` is the
+    sample's share of the step's elements, so `frac * step_bytes` are the
+    compulsory bytes of the elements the sample produces and a rate is those
+    bytes over the measured time.  Nothing is extrapolated."""
+
+    def __init__(self, w):
+        import oracle
+        self.w = w
+        s = w.spec
+        kind = s["kind"]
+        self.step_bytes = workload_bytes(s)[0]
+        if kind == "operator":
+            B, D, L, K = s["B"], s["D"], s["L"], s["order"] - 1
+            rows_total = B * D
+            if L <= 16384:
+                # whole rows: the direct O(L^2) chain and the FFT route on the same rows
+                # (about one second of the direct chain on 16 cores at L = 8192)
+                n_rows = min(rows_total, max(16, (768 * 8192 ** 2) // (L * L)))
+                rows = np.random.default_rng(0).permutation(rows_total)[:n_rows]
+                self.frac = rows.size / rows_total
+                self.fft_frac = self.frac
+                self.desc = ("filter MLP on all %d positions + the direct O(L^2) float64 chain on %d of %d "
+                             "whole rows" % (L, rows.size, rows_total))
+                self.fft_desc = ("filter MLP on all %d positions + the naive radix-2 FFT chain (n = %d, "
+                                 "filter transform per row) on the same %d rows" % (L, 2 * (spectrum_bins(L) - 1),
+                                                                                     rows.size))
+                fft_rows = rows
+                T = L
+            else:
+                # long rows: the direct chain on a prefix (causal: a prefix needs input prefixes only);
+                # the FFT route needs whole rows
+                T = min(L, 32768)
+                rows = np.arange(min(rows_total, max(oracle.threads(), 16)))
+                fft_rows = np.arange(min(rows_total, 2))
+                self.frac = rows.size * T / (rows_total * L)
+                self.fft_frac = fft_rows.size / rows_total
+                self.desc = ("filter MLP on all %d positions + the direct O(T^2) float64 chain on the first "
+                             "T = %d samples of %d of %d rows (a longer prefix costs more per sample)"
+                             % (L, T, rows.size, rows_total))
+                self.fft_desc = ("filter MLP on all %d positions + the naive radix-2 FFT chain (n = %d) on %d of "
+                                 "%d whole rows" % (L, 2 * (spectrum_bins(L) - 1), fft_rows.size, rows_total))
+            v = w.v.f32
+            xs = [x.f32 for x in w.xs]
+
+            def filt():
+                return oracle.filter_gen_1d(L, s["F"], True, w.Ws, w.bs, w.alpha).reshape(K, D, L)
+
+            self.run_oracle = lambda: oracle.hyena_rows(v, xs, filt(), w.Dskip, rows=rows, T=T)
+            self.run_fft = lambda: oracle.fftref_hyena_rows(v, xs, filt(), w.Dskip, rows=fft_rows)
+        elif kind == "nd":
+            B, D, g = s["B"], s["D"], s["grid"][0]
+            S = 2 * g
+            nvox = g ** 3
+            pts = np.random.default_rng(0).permutation(nvox)[:min(nvox, 2048)]
+            b, d = 0, 0
+            self.frac = pts.size / (B * D * nvox)
+            self.fft_frac = 1 / (B * D)
+            self.desc = ("one slab's kernel from the filter MLP on the whole %d^3 transform grid (all %d channels "
+                         "of sample 0) + the direct N-D sum at %d of its %d voxels" % (S, D, pts.size, nvox))
+            self.fft_desc = ("the same kernel + the naive 3-D FFT route (1-D radix-2 FFTs along each axis of the "
+                             "%d^3 grid) on that whole slab" % S)
+
+            def kern():
+                return oracle.filter_gen_3d(g, False, s["F"], w.Ws, w.bs, w.film_gamma[b:b + 1],
+                                            w.film_beta[b:b + 1], w.alpha)
+
+            vs, x1 = w.v.f32[b, d], w.xs[0].f32[b, d]
+            self.run_oracle = lambda: oracle.nd_conv_points(kern()[d], vs, x1, 0.0, pts, False)
+            self.run_fft = lambda: oracle.fftref_nd_conv(kern()[d:d + 1], [0], vs[None], x1[None], False)
+        else:
+            B, H, Dh, L = s["B"], s["H"], s["Dh"], s["L"]
+            rows_total = B * H * Dh
+            head = 0
+            n_rows = max(oracle.threads(), 16)
+            x1 = w.v.f32.reshape(rows_total, L)
+            x2 = w.xs[0].f32.reshape(rows_total, L)
+            rows = np.arange(n_rows)                        # sample 0, head 0: channels 0..n_rows-1
+            fft_rows = np.arange(min(Dh * 4, rows_total))   # sample 0, heads 0..3
+            self.frac = rows.size / rows_total
+            self.fft_frac = fft_rows.size / rows_total
+            self.desc = ("the gate's circular kernel of one head by the direct inverse DFT + the direct O(L^2) "
+                         "circular convolution on %d of %d rows" % (rows.size, rows_total))
+            self.fft_desc = "the naive radix-2 FFT route on %d of %d rows" % (fft_rows.size, rows_total)
+
+            def oracle_run():
+                kap = oracle.gate_kernel(w.gate[head])
+                return oracle.circular_conv_rows(kap[None], np.zeros(rows.size, np.int64), x1[rows], x2[rows])
+
+            self.run_oracle = oracle_run
+            gidx = (fft_rows // Dh) % H
+            self.run_fft = lambda: oracle.fftref_gate_rows(w.gate, gidx, x1[fft_rows], x2[fft_rows])
+
+    def time(self, which):
+        fn = self.run_oracle if which == "oracle" else self.run_fft
         t0 = time.perf_counter()
-        oracle.hyena_rows(w.v.f32, [x.f32 for x in w.xs], h64.reshape(K, D, L), w.Dskip, rows=batch)
-        dt = time.perf_counter() - t0
-        done += batch.size
-        t_rows += dt
-        left = budget_s - t_filter - t_rows
-        if left <= 0:
-            break
-        per_row = dt / batch.size
-        n = int(min(rows_total - done, max(cores, min(8 * batch.size, left / per_row))))
-    rows = order[:done]
-    est_step = t_filter + t_rows * rows_total / rows.size
-    return {"value": round(step_bytes / est_step / 1e9, 6), "unit": "GB/s", "cores": cores,
-            "kind": "oracle",
-            "sample": "filter MLP on all %d positions + direct O(L^2) float64 chain on %d of %d rows "
-                      "(%.1f s); value scales the sample to one whole step" % (L, rows.size, rows_total,
-                                                                               t_filter + t_rows)}
+        fn()
+        return time.perf_counter() - t0
+
+    def rate(self, which, seconds):
+        frac = self.frac if which == "oracle" else self.fft_frac
+        return self.step_bytes * frac / seconds / 1e9
+
+
+def cpu_baseline(w):
+    """The float64 oracle as it stands, and the naive float64 FFT reference,
+    each timed once on a bounded sample of the workload on this host's
+    cores.  value = compulsory bytes of the sample's elements / time."""
+    import oracle
+    cs = CpuSample(w)
+    cores = oracle.threads()
+    t_o = cs.time("oracle")
+    t_f = cs.time("fft")
+    return {"value": round(cs.rate("oracle", t_o), 6), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": "%s (%.2f s); value = the compulsory bytes of the sampled elements / time" % (cs.desc, t_o),
+            "fft_reference": {"value": round(cs.rate("fft", t_f), 6), "unit": "GB/s", "cores": cores,
+                              "kind": "naive float64 FFT reference",
+                              "sample": "%s (%.2f s)" % (cs.fft_desc, t_f)}}
 
 
 def run_reference(args):
+    """The reference arm: the float64 oracle as it stands, on this host's
+    cores.  Every step runs the same bounded sample of the workload (see
+    CpuSample); ms_per_step is the measured time of one such step and value
+    the sample's compulsory bytes over it.  Under torchrun only rank 0 runs."""
+    import oracle
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     name = args.workload
     w = hw.make(name)
-    if w.spec["kind"] != "operator" or w.spec["L"] > 16384:
-        print(json.dumps({"impl": "reference", "unavailable":
-                          "the oracle arm is timed on the on-chip operator workloads (c1, c2) only"}))
-        return
-    budget = max(2.0, min(args.cpu_budget, 150.0 / max(1, args.steps + args.warmup)))
+    cs = CpuSample(w)
     for _ in range(args.warmup):
-        cpu_baseline(w, budget_s=budget)
-    vals = []
+        cs.time("oracle")
     t0 = time.perf_counter()
-    last = None
-    for _ in range(args.steps):
-        last = cpu_baseline(w, budget_s=budget)
-        vals.append(last["value"])
+    times = [cs.time("oracle") for _ in range(args.steps)]
     wall = time.perf_counter() - t0
-    step_bytes, _ = workload_bytes(w.spec)
-    value = statistics.median(vals)
+    t_f = cs.time("fft")
+    per_step = sum(times) / len(times)
+    value = cs.rate("oracle", per_step)
     s = w.spec
+    cores = oracle.threads()
     line = {
         "impl": "reference",
         "metric": "Hyena op GB/s (%s)" % DESCR[name],
-        "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(step_bytes / (value * 1e9) * 1e3, 3) if value > 0 else None,
+        "value": round(value, 6), "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(per_step * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) signals, random-init filter MLP)",
-        "config": {"workload": DESCR[name], "B": s["B"], "D": s["D"], "L": s["L"], "order": s["order"]},
-        "cpu_baseline": last,
-        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-        "wall_s": round(wall, 1),
+        "config": workload_config(name, s, world),
+        "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": "each step: %s; value = the compulsory bytes of the sampled elements "
+                                   "(%.4f of the step) / the measured step time" % (cs.desc, cs.frac),
+                         "fft_reference": {"value": round(cs.rate("fft", t_f), 6), "unit": "GB/s",
+                                           "cores": cores, "kind": "naive float64 FFT reference",
+                                           "sample": "%s (%.2f s, once)" % (cs.fft_desc, t_f)}},
+        "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": round(wall, 4),
     }
     print(json.dumps(line), flush=True)
 
@@ -729,7 +891,6 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(DESCR), default=DEFAULT_WORKLOAD)
-    ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode", action="store_true",
                     help="time one streaming decode step of the spectral gate (prefix-FFT cache) instead")

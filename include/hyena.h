@@ -367,7 +367,16 @@ hy_status spectral_gate_host(int B, int H, int Dh, int L, hy_dtype dt, const voi
 /* Reads the current device's fault word into *faults after the work queued on
  * `stream` has finished (the call synchronises that stream); clear != 0 then
  * resets it (queued on `stream`).  Returns HY_ERR_TIMEOUT when any bit was
- * set, HY_OK when none, HY_ERR_INVALID_ARG for a null `faults`. */
+ * set, HY_OK when none, HY_ERR_INVALID_ARG for a null `faults`.
+ *
+ * The word is one per device, shared by every stream, host thread and call
+ * that runs this library's kernels on the device.  The compute entry points
+ * return HY_OK once their kernels are launched, so a wait that gives up
+ * during those kernels shows up only here.  Synchronising `stream` does not
+ * wait for other streams: a bit may belong to another stream's work, and a
+ * clear resets the bits of every caller.  Read (and clear) the word only
+ * after all streams that ran the library's kernels on this device have been
+ * synchronised (cudaDeviceSynchronize), by one owner of that device. */
 hy_status hyena_device_faults(uint32_t *faults, int clear, void *stream);
 /* Diagnostic for the failure path: launches one CTA whose wait on an
  * mbarrier that can never complete runs out after limit_us microseconds

@@ -14,6 +14,10 @@ Two layers:
   ``numpy.fft`` in float64, used as a library step, for tensors too large for
   the direct sums.  They are trusted only where the tests have matched them
   against the direct definitions.
+* ``fft_reference.c`` (``fftref_*``): a naive float64 CPU FFT route (one
+  iterative radix-2 complex FFT, real rows as complex, the filter transform
+  recomputed per row) -- the plain CPU program the benchmark times beside the
+  direct oracle.  Pinned to the direct definitions like the ``fft_*`` ones.
 
 Pages cited (title, section):
   [HN] "Hyena: 암묵적 장거리 컨볼루션으로 어텐션을 완전 대체한 서브-이차 모델",
@@ -37,6 +41,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "hyena_oracle.c")
+_SRC_FFT = os.path.join(_HERE, "fft_reference.c")
 _BUILD = os.path.join(_HERE, "_build")
 _SO = os.path.join(_BUILD, "libhyena_oracle.so")
 
@@ -52,6 +57,8 @@ PINS = {
     "gate_kernel": "g=1 delta, shift gate, constant gate, numpy.fft.irfft",
     "circular_conv": "shift gate, Parseval, numpy.fft circular convolution",
     "fft_*": "matched against the direct functions above on sampled outputs",
+    "fftref_fft": "delta and constant closed forms, inverse(forward) = n x, direct DFT (dft_real_rows)",
+    "fftref_*": "equal to the direct hyena_rows, gate kernel + circular_conv_rows and nd_conv_points",
     "projection": "identity weights give the transposed input, zero weights the bias, linearity",
     "hyena_backward": "central finite differences of the direct forward (hyena_rows) for every input",
     "hyena_backward_samples": "equals hyena_backward (order 2) at every index",
@@ -60,14 +67,15 @@ PINS = {
 
 
 def build(force: bool = False) -> str:
-    """Compile hyena_oracle.c into oracle/_build/libhyena_oracle.so (gcc)."""
+    """Compile hyena_oracle.c and fft_reference.c into
+    oracle/_build/libhyena_oracle.so (gcc)."""
     os.makedirs(_BUILD, exist_ok=True)
     if (not force and os.path.exists(_SO)
-            and os.path.getmtime(_SO) >= os.path.getmtime(_SRC)):
+            and os.path.getmtime(_SO) >= max(os.path.getmtime(_SRC), os.path.getmtime(_SRC_FFT))):
         return _SO
     tmp = _SO + ".tmp.%d" % os.getpid()
     cmd = ["gcc", "-O2", "-ffp-contract=off", "-fopenmp", "-fPIC", "-shared",
-           _SRC, "-o", tmp, "-lm"]
+           _SRC, _SRC_FFT, "-o", tmp, "-lm"]
     subprocess.check_call(cmd)
     os.replace(tmp, _SO)
     return _SO
@@ -497,3 +505,73 @@ def fft_spectral_gate_rows(g_rows, x1, x2) -> np.ndarray:
     n = x1.shape[-1]
     y = np.fft.irfft(np.fft.rfft(x1, axis=-1) * np.asarray(g_rows, np.complex128), n=n, axis=-1)
     return y if x2 is None else _f64(x2) * y
+
+
+# --------------------------------------------------------------------------
+# naive float64 CPU FFT route (fft_reference.c): the baseline program timed
+# beside the direct oracle
+# --------------------------------------------------------------------------
+
+def fftref_fft(x, inverse: bool = False) -> np.ndarray:
+    """Unnormalised DFT of a complex vector (length a power of two) by the
+    naive radix-2 FFT: X[k] = sum_j x[j] exp(-+2 pi i jk/n)."""
+    x = np.asarray(x, np.complex128)
+    re = np.ascontiguousarray(x.real)
+    im = np.ascontiguousarray(x.imag)
+    _load().fref_fft(ctypes.c_int64(x.size), _dp(re), _dp(im), ctypes.c_int(1 if inverse else 0))
+    return re + 1j * im
+
+
+def fftref_hyena_rows(v, xs, h, Dskip, rows=None) -> np.ndarray:
+    """The order-(K+1) chain of hyena_rows through the naive FFT route
+    (zero-padded to transform_len(L), filter transform per row)."""
+    v = _f64(v)
+    B, D, L = v.shape
+    xs = [_f64(x) for x in xs]
+    K = len(xs)
+    h = _f64(h)
+    assert h.shape == (K, D, L)
+    if rows is None:
+        rows = np.arange(B * D, dtype=np.int64)
+    rows = np.ascontiguousarray(np.asarray(rows, np.int64))
+    y = np.empty((rows.size, L))
+    dsk = None
+    if Dskip is not None:
+        Dskip = _f64(Dskip)
+        dsk = _dp(Dskip)
+    _load().fref_hyena_rows(ctypes.c_int(K), ctypes.c_int64(D), ctypes.c_int64(L),
+                            ctypes.c_int64(transform_len(L)), _dp(v), _ptr_array(xs), _dp(h), dsk,
+                            ctypes.c_int64(rows.size), _ip(rows), _dp(y))
+    return y
+
+
+def fftref_gate_rows(g, gidx, x1, x2) -> np.ndarray:
+    """Spectral gate rows through the naive FFT route.  g: (nk, n/2+1)
+    complex; gidx: the g row of each x1 row; x1, x2: (nrows, n) (x2 may be None)."""
+    x1 = _f64(x1)
+    nrows, n = x1.shape
+    g = np.asarray(g, np.complex128)
+    gre, gim = np.ascontiguousarray(g.real), np.ascontiguousarray(g.imag)
+    gidx = np.ascontiguousarray(np.asarray(gidx, np.int64))
+    y = np.empty((nrows, n))
+    x2keep = _f64(x2) if x2 is not None else None
+    x2p = _dp(x2keep) if x2keep is not None else None
+    _load().fref_gate_rows(ctypes.c_int64(n), ctypes.c_int64(nrows), _dp(gre), _dp(gim), _ip(gidx),
+                           _dp(x1), x2p, _dp(y))
+    return y
+
+
+def fftref_nd_conv(Kern, kidx, v, x1, circular: bool = False) -> np.ndarray:
+    """Gated N-D convolution of slabs v (nslab, g0, g1, g2) through the naive
+    FFT route; Kern (nk, S0, S1, S2) on the transform grid, slab s using
+    Kern[kidx[s]]; x1 like v or None.  No skip term."""
+    v = _f64(v)
+    nslab = v.shape[0]
+    g = (ctypes.c_int * 3)(*v.shape[1:])
+    Kern = _f64(Kern)
+    kidx = np.ascontiguousarray(np.asarray(kidx, np.int64))
+    y = np.empty_like(v)
+    x1keep = _f64(x1) if x1 is not None else None
+    _load().fref_nd_conv(g, ctypes.c_int(1 if circular else 0), ctypes.c_int64(nslab), _dp(Kern), _ip(kidx),
+                         _dp(v), _dp(x1keep) if x1keep is not None else None, _dp(y))
+    return y

@@ -75,9 +75,29 @@ def test_reference_arm_only_rank0_prints(tmp_path):
     assert r.returncode == 0 and r.stdout.strip() == ""
     env = dict(os.environ, RANK="0", WORLD_SIZE="1")
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                        "--workload", "c1", "--steps", "1", "--warmup", "0", "--cpu-budget", "2"],
+                        "--workload", "c1", "--steps", "2", "--warmup", "0"],
                        capture_output=True, text=True, env=env, timeout=300)
     assert r.returncode == 0
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["cpu_baseline"]["fft_reference"]["value"] > 0
+    # the steps it reports are the steps it timed
+    assert line["steps"] == 2 and line["ms_per_step"] * line["steps"] <= 1e3 * line["wall_s"] * 1.05
+    sys.path.insert(0, ROOT)
+    import bench
+    import hyena_workloads as hw
+    assert line["config"] == bench.workload_config("c1", hw.make("c1", with_signals=False).spec, 1)
+
+
+@pytest.mark.parametrize("name,over", [("c3", dict(D=2, L=1 << 15)), ("c4", dict(D=2, grid=(8, 8, 8))),
+                                       ("c5", dict(H=2, Dh=4, L=64))])
+def test_cpu_samples_of_every_workload(name, over):
+    """The CPU baselines (direct oracle and naive FFT reference) run on a
+    bounded sample of every workload kind and report a positive rate."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import hyena_workloads as hw
+    w = hw.make(name, **over)
+    cb = bench.cpu_baseline(w)
+    assert cb["value"] > 0 and cb["fft_reference"]["value"] > 0 and cb["cores"] >= 1

@@ -408,6 +408,74 @@ def test_fft_spectrum_matches_direct():
     np.testing.assert_allclose(oracle.fft_spectrum(h), oracle.dft_real_rows(h, 128), atol=1e-11)
 
 
+# ---------------------------------------------------------------- naive CPU FFT reference
+
+def test_fftref_fft_closed_forms_and_direct_dft():
+    """The naive radix-2 FFT: a delta at s transforms to the phase ramp
+    e^{-2 pi i k s/n} (closed form), a constant c to n c at k = 0 and zeros
+    elsewhere, inverse(forward(x)) = n x, and a real row equals the direct
+    DFT of hyena_oracle.c (not numpy) on every bin."""
+    n = 64
+    k = np.arange(n)
+    for s in (0, 1, 5, 32, 63):
+        e = np.zeros(n, complex)
+        e[s] = 1.0
+        np.testing.assert_allclose(oracle.fftref_fft(e), np.exp(-2j * np.pi * k * s / n), atol=1e-14)
+        np.testing.assert_allclose(oracle.fftref_fft(e, inverse=True), np.exp(2j * np.pi * k * s / n), atol=1e-14)
+    c = np.full(n, 0.75 - 0.5j)
+    X = oracle.fftref_fft(c)
+    np.testing.assert_allclose(X[0], n * (0.75 - 0.5j), atol=1e-13)
+    np.testing.assert_allclose(X[1:], 0, atol=1e-13)
+    rng = np.random.default_rng(40)
+    x = rng.standard_normal(n) + 1j * rng.standard_normal(n)
+    np.testing.assert_allclose(oracle.fftref_fft(oracle.fftref_fft(x), inverse=True), n * x, atol=1e-12)
+    h = rng.standard_normal((3, 40))
+    for r in range(3):
+        pad = np.zeros(128, complex)
+        pad[:40] = h[r]
+        np.testing.assert_allclose(oracle.fftref_fft(pad)[:65], oracle.dft_real_rows(h[r:r + 1], 128)[0],
+                                   atol=1e-12)
+
+
+def test_fftref_hyena_rows_matches_direct():
+    rng = np.random.default_rng(41)
+    for (B, D, L, K) in [(2, 3, 100, 1), (1, 2, 64, 3), (1, 1, 1, 2)]:
+        v = rng.standard_normal((B, D, L))
+        xs = [rng.standard_normal((B, D, L)) for _ in range(K)]
+        h = rng.standard_normal((K, D, L)) * np.exp(-np.arange(L) / 30)
+        Dk = rng.standard_normal((K, D))
+        a = oracle.fftref_hyena_rows(v, xs, h, Dk)
+        b = oracle.hyena_rows(v, xs, h, Dk)
+        np.testing.assert_allclose(a, b, rtol=1e-10, atol=1e-11)
+    rows = np.array([4, 0])
+    a = oracle.fftref_hyena_rows(v, xs, h, None, rows=rows)
+    np.testing.assert_allclose(a, oracle.hyena_rows(v, xs, h, None, rows=rows), rtol=1e-10, atol=1e-11)
+
+
+def test_fftref_gate_and_nd_match_direct():
+    rng = np.random.default_rng(42)
+    n = 64
+    g = rng.standard_normal((2, n // 2 + 1)) + 1j * rng.standard_normal((2, n // 2 + 1))
+    x1, x2 = rng.standard_normal((2, 3, n))
+    gidx = np.array([1, 0, 1])
+    kap = np.stack([oracle.gate_kernel(gg) for gg in g])
+    np.testing.assert_allclose(oracle.fftref_gate_rows(g, gidx, x1, x2),
+                               oracle.circular_conv_rows(kap, gidx, x1, x2), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(oracle.fftref_gate_rows(g, gidx, x1, None),
+                               oracle.circular_conv_rows(kap, gidx, x1, None), rtol=1e-11, atol=1e-12)
+    gr = (4, 2, 8)
+    for circular in (False, True):
+        S = gr if circular else tuple(2 * a for a in gr)
+        Kern = rng.standard_normal((2,) + S)
+        v, x1 = rng.standard_normal((2, 3) + gr)
+        kidx = np.array([1, 1, 0])
+        a = oracle.fftref_nd_conv(Kern, kidx, v, x1, circular)
+        for s in range(3):
+            b = oracle.nd_conv_points(Kern[kidx[s]], v[s], x1[s], 0.0, np.arange(int(np.prod(gr))),
+                                      circular).reshape(gr)
+            np.testing.assert_allclose(a[s], b, rtol=1e-11, atol=1e-11)
+
+
 def test_projection_identity_zero_and_linearity():
     """Input projection: identity blocks return the input transposed to
     channel-major (times the block's scale), zero weights return the bias on

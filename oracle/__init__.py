@@ -60,6 +60,8 @@ PINS = {
     "fftref_fft": "delta and constant closed forms, inverse(forward) = n x, direct DFT (dft_real_rows)",
     "fftref_*": "equal to the direct hyena_rows, gate kernel + circular_conv_rows and nd_conv_points",
     "projection": "identity weights give the transposed input, zero weights the bias, linearity",
+    "register_film": "no logits -> plain mean, one-hot limit -> selection, shift invariance, stable at large "
+                     "logits, loop brute force, identity / zero FiLM maps",
     "hyena_backward": "central finite differences of the direct forward (hyena_rows) for every input",
     "hyena_backward_samples": "equals hyena_backward (order 2) at every index",
     "prefix_gate_outputs": "composition of gate_kernel and circular_conv_samples (pinned); first output x2 kappa[0] x",
@@ -139,6 +141,37 @@ def projection(x, W, bias, n_out: int) -> list:
     if bias is not None:
         full = full + np.asarray(bias, np.float64)[None, None, :]
     return [np.ascontiguousarray(full[:, :, k * D:(k + 1) * D].transpose(0, 2, 1)) for k in range(n_out)]
+
+
+# --------------------------------------------------------------------------
+# HyenaND input conditioning ([ND] 방법론: HyenaND, 레지스터 및 FiLM을 통한 입력
+# 의존적 커널): register activations -> z(x) by a softmax-weighted mean ->
+# FiLM parameters of the kernel MLP
+# --------------------------------------------------------------------------
+
+def register_film(reg, query, scores, W, b):
+    """z(x) and the FiLM parameters it drives, float64.
+
+    reg: (B, R, C) activations of the R register tokens of each sample.
+    Pooling logits l[b, r] = query . reg[b, r] (if query is given) + scores[b, r]
+    (if given); weights w[b] = softmax_r(l[b]); z[b] = sum_r w[b, r] reg[b, r].
+    The control variable drives FiLM through one linear map:
+    (gamma[b], beta[b]) = W z[b] + b, W of shape (2 H, C), gamma the first H
+    outputs and beta the next H.  Returns (gamma, beta, z, w)."""
+    reg = np.asarray(reg, np.float64)
+    B, R, C = reg.shape
+    logits = np.zeros((B, R))
+    if query is not None:
+        logits = logits + np.einsum("brc,c->br", reg, np.asarray(query, np.float64))
+    if scores is not None:
+        logits = logits + np.asarray(scores, np.float64)
+    m = logits.max(axis=1, keepdims=True)           # softmax with the maximum subtracted
+    e = np.exp(logits - m)
+    w = e / e.sum(axis=1, keepdims=True)
+    z = np.einsum("br,brc->bc", w, reg)
+    out = z @ np.asarray(W, np.float64).T + np.asarray(b, np.float64)[None, :]
+    H = out.shape[1] // 2
+    return out[:, :H], out[:, H:], z, w
 
 
 # --------------------------------------------------------------------------

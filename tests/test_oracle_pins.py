@@ -476,6 +476,62 @@ def test_fftref_gate_and_nd_match_direct():
             np.testing.assert_allclose(a[s], b, rtol=1e-11, atol=1e-11)
 
 
+# ---------------------------------------------------------------- HyenaND register conditioning
+
+def test_register_film_closed_forms():
+    """z(x) = softmax-weighted mean of the register activations
+    ([ND] 레지스터 및 FiLM): without logits it is the plain mean; a logit far
+    above the rest selects that register; adding a constant to every logit of
+    a sample changes nothing; logits of 1e4 stay finite (the maximum is
+    subtracted); the FiLM map with identity blocks returns z and with zero
+    weights the bias."""
+    rng = np.random.default_rng(50)
+    B, R, C, H = 3, 5, 6, 6
+    reg = rng.standard_normal((B, R, C))
+    I = np.eye(C)
+    W = np.concatenate([I, 2 * I])
+    b0 = np.zeros(2 * H)
+    g, be, z, w = oracle.register_film(reg, None, None, W, b0)
+    np.testing.assert_allclose(z, reg.mean(axis=1), rtol=0, atol=1e-15)
+    np.testing.assert_allclose(g, z, atol=1e-15)
+    np.testing.assert_allclose(be, 2 * z, atol=1e-15)
+    s = np.zeros((B, R))
+    s[np.arange(B), [4, 0, 2]] = 60.0
+    _, _, z1, _ = oracle.register_film(reg, None, s, W, b0)
+    np.testing.assert_allclose(z1, reg[np.arange(B), [4, 0, 2]], atol=1e-12)
+    s2 = rng.standard_normal((B, R))
+    _, _, za, _ = oracle.register_film(reg, None, s2, W, b0)
+    _, _, zb, _ = oracle.register_film(reg, None, s2 + rng.standard_normal((B, 1)) * 100, W, b0)
+    np.testing.assert_allclose(za, zb, rtol=1e-12, atol=1e-13)
+    _, _, zc, wc = oracle.register_film(reg, None, 1e4 * s2, W, b0)
+    assert np.all(np.isfinite(zc)) and np.allclose(wc.sum(axis=1), 1.0)
+    c = rng.standard_normal(2 * H)
+    g0, be0, _, _ = oracle.register_film(reg, rng.standard_normal(C), s2, np.zeros((2 * H, C)), c)
+    np.testing.assert_array_equal(g0, np.broadcast_to(c[:H], (B, H)))
+    np.testing.assert_array_equal(be0, np.broadcast_to(c[H:], (B, H)))
+
+
+def test_register_film_bruteforce_loops():
+    """Query logits and FiLM map against plain Python loops on a tiny case."""
+    rng = np.random.default_rng(51)
+    B, R, C, H = 2, 3, 4, 2
+    reg = rng.standard_normal((B, R, C))
+    q = rng.standard_normal(C)
+    sc = rng.standard_normal((B, R))
+    W = rng.standard_normal((2 * H, C))
+    bb = rng.standard_normal(2 * H)
+    g, be, z, w = oracle.register_film(reg, q, sc, W, bb)
+    for bi in range(B):
+        lg = [sum(q[c] * reg[bi, r, c] for c in range(C)) + sc[bi, r] for r in range(R)]
+        ex = [math.exp(v) for v in lg]
+        tot = sum(ex)
+        zz = [sum(ex[r] / tot * reg[bi, r, c] for r in range(R)) for c in range(C)]
+        out = [bb[o] + sum(W[o, c] * zz[c] for c in range(C)) for o in range(2 * H)]
+        np.testing.assert_allclose(z[bi], zz, rtol=1e-12)
+        np.testing.assert_allclose(g[bi], out[:H], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(be[bi], out[H:], rtol=1e-12, atol=1e-14)
+
+
 def test_projection_identity_zero_and_linearity():
     """Input projection: identity blocks return the input transposed to
     channel-major (times the block's scale), zero weights return the bias on

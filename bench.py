@@ -48,7 +48,7 @@ DESCR = {
     "c1": "hyena order-2 operator B1 D16 L1024 fp32 (filters 17->32->16)",
     "c2": "hyena order-2 operator B8 D768 L8192 bf16 (filters 65->64->64->768)",
     "c3": "hyena order-3 operator B1 D256 L1048576 fp32 (filters 17->64->512)",
-    "c4": "hyenaND order-2 3-D conv B2 D128 64^3 fp32 (FiLM filters 24->64->128 on 128^3)",
+    "c4": "hyenaND order-2 3-D conv B2 D128 64^3 fp32 (FiLM from 8 register tokens; filters 24->64->128 on 128^3)",
     "c5": "spectral gate B4 H32 Dh64 L32768 bf16",
 }
 
@@ -79,7 +79,8 @@ def workload_bytes(spec):
 
 
 CONV_SOURCES = ["bulk_copy.cuh", "common.cuh", "fft_core.cuh", "resident.cuh", "resident_launch.cuh", "resident.cu",
-                "resident_stream_bf16.cu", "resident_stream_f32.cu", "twiddle.cu", "twiddle.h"]
+                "resident_stream_bf16.cu", "resident_stream_f32.cu", "resident_tc.cu", "tcgen05.cuh", "twiddle.cu",
+                "twiddle.h"]
 
 
 def conv_sources_digest():
@@ -283,8 +284,9 @@ def workload_config(name, s, world, over=None):
     cfg = {"workload": DESCR[name] + (" [D=%d profiling case]" % s["D"] if over else "")}
     cfg.update({k: v for k, v in s.items() if k in ("B", "D", "L", "order", "H", "Dh", "grid")})
     cfg["io_dtype"] = s["dtype"]
-    cfg.update({"step": ("filter_gen + filter_spectrum + convolution" if s["kind"] != "gate"
-                         else "spectral_gate"),
+    cfg.update({"step": ("spectral_gate" if s["kind"] == "gate" else
+                         "register_film + filter_gen + filter_spectrum + convolution" if s.get("registers")
+                         else "filter_gen + filter_spectrum + convolution"),
                 "step_bytes": step_bytes, "conv_bytes": op_bytes,
                 "l2": ("inputs larger than L2 (%.0f MB streamed per step vs 126 MB); no flush" % (op_bytes / 1e6)
                        if op_bytes > 126e6 else "inputs smaller than L2 (no flush): launch-bound case"),
@@ -352,9 +354,12 @@ def setup_operator(w, dev, hy, torch):
         st.kernel = "multi-pass colpass/rowpass kernels (M=2^%d)" % (M.bit_length() - 1)
     else:
         op_l = 1
-        # one order over power-of-two rows runs the persistent streaming kernel
+        # one order over power-of-two rows runs a persistent streaming kernel;
+        # bf16 rows of 8192 take the one with tensor-core radix-32 stages
         stream = K == 1 and L == M and M >= 64
-        st.kernel = "%s<M=2^%d>" % ("resident_stream_kernel" if stream else "resident_conv_kernel",
+        tensor = stream and L == 8192 and s["dtype"] == "bf16" and os.environ.get("HYENA_FFT_ENGINE") == "tensor"
+        st.kernel = "%s<M=2^%d>" % ("resident_tc_kernel" if tensor else
+                                    "resident_stream_kernel" if stream else "resident_conv_kernel",
                                     M.bit_length() - 1)
     spec_l = 2 * -(-(K * D) // max(1, wsf // (12 * M))) if wsf else 1
     st.launches = 1 + spec_l + op_l
@@ -367,7 +372,16 @@ def setup_nd(w, dev, hy, torch):
     S = 2 * g
     f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dev)
     Ws, bs, alpha = [f32(a) for a in w.Ws], [f32(a) for a in w.bs], f32(w.alpha)
-    gm, bt = f32(w.film_gamma), f32(w.film_beta)
+    if w.reg is not None:
+        # input conditioning: z(x) from the register activations drives FiLM
+        H1 = s["hidden"][0]
+        gm = torch.empty((B, H1), device=dev)
+        bt = torch.empty((B, H1), device=dev)
+        reg, rq, fW, fb = f32(w.reg), f32(w.reg_query), f32(w.film_W), f32(w.film_b)
+        condition = lambda: hy.hyena_register_film(reg, fW, gm, bt, query=rq, b_film=fb)
+    else:
+        gm, bt = f32(w.film_gamma), f32(w.film_beta)
+        condition = lambda: None
     u, x1 = f32(w.v.f32), f32(w.xs[0].f32)
     y = torch.empty_like(u)
     h = torch.empty((B, D, S, S, S), device=dev)
@@ -378,6 +392,7 @@ def setup_nd(w, dev, hy, torch):
     st = Setup()
 
     def spectra():
+        condition()
         hy.hyena_filter_gen(h, ndim=3, grid=g, Ws=Ws, bs=bs, alpha=alpha, n_freq=s["F"],
                             film_gamma=gm, film_beta=bt, n_sets=B)
         hy.hyena_filter_spectrum(h, H, rows=B * D, ndim=3, dims=[g, g, g], ws=ws)
@@ -395,7 +410,7 @@ def setup_nd(w, dev, hy, torch):
     st.output = y
     per_c = g * S * (S // 2 + 1) * 8
     per_s = S * S * (S // 2 + 1) * 8
-    st.launches = (1 + 2 * -(-(B * D) // max(1, wsf // per_s))
+    st.launches = ((2 if w.reg is not None else 1) + 2 * -(-(B * D) // max(1, wsf // per_s))
                    + 3 * -(-(B * D) // max(1, wsc // per_c)))
     st.kernel = "nd_fwd_plane/nd_xpass/nd_inv_plane<S=%d>" % S
     return st
@@ -637,8 +652,11 @@ class CpuSample:
                              "%d^3 grid) on that whole slab" % S)
 
             def kern():
-                return oracle.filter_gen_3d(g, False, s["F"], w.Ws, w.bs, w.film_gamma[b:b + 1],
-                                            w.film_beta[b:b + 1], w.alpha)
+                if w.reg is not None:      # z(x) from the registers, then FiLM
+                    gm, bt, _, _ = oracle.register_film(w.reg[b:b + 1], w.reg_query, None, w.film_W, w.film_b)
+                else:
+                    gm, bt = w.film_gamma[b:b + 1], w.film_beta[b:b + 1]
+                return oracle.filter_gen_3d(g, False, s["F"], w.Ws, w.bs, gm, bt, w.alpha)
 
             vs, x1 = w.v.f32[b, d], w.xs[0].f32[b, d]
             self.run_oracle = lambda: oracle.nd_conv_points(kern()[d], vs, x1, 0.0, pts, False)
@@ -738,9 +756,9 @@ def run_reference(args):
 
 def run_projection(args):
     """The input projection at the operator workload's width (B8 L8192,
-    768 -> 2 x 768 channels, bf16): one bf16 GEMM per projection plus the
-    bias pass, timed with CUDA events; TFLOP/s against the measured bf16
-    GEMM peak (burst)."""
+    768 -> 2 x 768 channels, bf16): one launch of the library's tcgen05 GEMM
+    with the bias fused into its epilogue, timed with CUDA events; TFLOP/s
+    against the measured bf16 GEMM peak (burst)."""
     import torch
     import implicit_long_convolution_b200 as hy
     world, rank, local = dist_setup()
@@ -770,19 +788,20 @@ def run_projection(args):
     ms = max_over_ranks(t0.elapsed_time(t1), world) / steps
     flops = 2.0 * B * L * C * n_out * D
     tf = world * flops / (ms / 1e3) / 1e12
-    peak = None
+    peak, peak_kind = 1590.0, "fallback"
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         with open(path) as f:
-            peak = float(json.load(f)["bf16_tflops"])
+            peak, peak_kind = float(json.load(f)["bf16_tflops"]), "measured"
     if rank == 0:
         print(json.dumps({
             "metric": "input projection TFLOP/s (B8 L8192, 768 -> 2 x 768, bf16, channel-major outputs + bias)",
             "value": round(tf, 1), "unit": "TFLOP/s", "n_gpus": world, "steps": steps, "warmup": args.warmup,
             "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peak, "unit": "TFLOP/s",
-                         "frac": round(tf / world / peak, 4) if peak else None, "traffic": None},
+            "roofline": {"bound": "tensor", "kernel": "proj_tc_kernel", "achieved": round(tf / world, 1),
+                         "peak": peak, "unit": "TFLOP/s", "frac": round(tf / world / peak, 4),
+                         "peak_kind": peak_kind, "traffic": None},
             "config": {"workload": "hyena input projection at the order-2 operator width",
                        "B": B, "L": L, "C": C, "D": D, "n_out": n_out,
                        "accumulate": "f32"}}), flush=True)

@@ -20,7 +20,12 @@ overridden), drawn in this fixed order:
    rounded to complex64 (gate workload);
 5. the signals: v then x_1, x_2, ... (or x1 then x2 for the gate), N(0, 1)
    float32, rounded to bfloat16 (round-to-nearest-even) for bf16 workloads --
-   the rounded values are the inputs both sides see.
+   the rounded values are the inputs both sides see;
+6. (N-D workload with ``registers=R``) register activations (B, R, C) ~ N(0,1),
+   the pooling query ~ N(0, 1/C), the FiLM map W ~ U(+-0.1/sqrt(C)) of shape
+   (2 hidden0, C) and its bias ~ N(0, 0.01^2): the input conditioning that
+   replaces the drawn gamma/beta of step 4 when a test or the benchmark asks
+   for it.
 """
 from __future__ import annotations
 
@@ -43,8 +48,10 @@ WORKLOADS = {
     "c3": dict(kind="operator", order=3, dtype="f32", B=1, D=256, L=1 << 20, F=8, include_t=True,
                hidden=[64], alpha=(0.1, 2.0), skip=True),
     # order-2 gated 3-D global convolution: B2 D128 64^3 fp32, per-sample FiLM filters
+    # (conditioned on the input through 8 register tokens of width 64)
     "c4": dict(kind="nd", order=2, dtype="f32", B=2, D=128, grid=(64, 64, 64), F=4,
-               hidden=[64], alpha=(0.5, 3.0), skip=False, film=True, circular=False),
+               hidden=[64], alpha=(0.5, 3.0), skip=False, film=True, circular=False,
+               registers=8, register_width=64),
     # spectral-gating token mixer: B4 H32 Dh64 L32768 bf16
     "c5": dict(kind="gate", dtype="bf16", B=4, H=32, Dh=64, L=32768),
 }
@@ -87,6 +94,10 @@ class Workload:
     film_gamma: Optional[np.ndarray] = None  # (B, hidden0) float32
     film_beta: Optional[np.ndarray] = None
     gate: Optional[np.ndarray] = None    # (H, L/2+1) complex64
+    reg: Optional[np.ndarray] = None     # (B, R, C) register activations (N-D, registers=R)
+    reg_query: Optional[np.ndarray] = None
+    film_W: Optional[np.ndarray] = None  # (2 hidden0, C): z(x) -> (gamma, beta)
+    film_b: Optional[np.ndarray] = None
     v: Optional[Signal] = None
     xs: list = dataclasses.field(default_factory=list)
 
@@ -150,6 +161,15 @@ def make(name: str, seed: Optional[int] = None, with_signals: bool = True, **ove
             shape = (spec["B"], spec["D"]) + tuple(spec["grid"])
             w.v = _signal(rng, shape, spec["dtype"])
             w.xs = [_signal(rng, shape, spec["dtype"])]
+        if spec.get("registers"):
+            # input conditioning through register tokens (drawn after everything
+            # above, so the draws before stay the same): activations of R
+            # registers per sample, the pooling query, and the FiLM map of z(x)
+            R, C, H = spec["registers"], spec.get("register_width", 64), spec["hidden"][0]
+            w.reg = rng.standard_normal(size=(spec["B"], R, C)).astype(np.float32)
+            w.reg_query = (rng.standard_normal(size=(C,)) / math.sqrt(C)).astype(np.float32)
+            w.film_W = rng.uniform(-0.1 / math.sqrt(C), 0.1 / math.sqrt(C), size=(2 * H, C)).astype(np.float32)
+            w.film_b = (0.01 * rng.standard_normal(size=(2 * H,))).astype(np.float32)
         return w
     if kind == "gate":
         nb = spec["L"] // 2 + 1

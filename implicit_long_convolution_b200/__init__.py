@@ -24,7 +24,7 @@ __all__ = [
     "nd_conv_workspace", "spectral_gate", "operator_host_workspace", "hyena_operator_host",
     "spectral_gate_host_workspace", "spectral_gate_host", "nd_conv_host_workspace", "hyena_nd_conv_host",
     "projection_workspace", "hyena_projection", "operator_backward_workspace", "hyena_operator_backward",
-    "spectral_gate_decode", "device_faults", "selftest_bounded_wait",
+    "spectral_gate_decode", "device_faults", "selftest_bounded_wait", "hyena_register_film",
     "STATUS",
 ]
 
@@ -35,7 +35,8 @@ STATUS = {0: "HY_OK", 1: "HY_ERR_INVALID_ARG", 2: "HY_ERR_UNSUPPORTED", 3: "HY_E
 HY_F32, HY_BF16 = 0, 1
 HY_ACT_SILU, HY_ACT_IDENTITY, HY_ACT_SINE = 0, 1, 2
 HY_WIN_EXP, HY_WIN_GAUSS = 0, 1
-HY_FAULT_STREAM_INPUT, HY_FAULT_STREAM_GATE, HY_FAULT_SELFTEST = 0x1, 0x2, 0x80000000
+HY_FAULT_STREAM_INPUT, HY_FAULT_STREAM_GATE, HY_FAULT_PROJECTION, HY_FAULT_TC_CONV = 0x1, 0x2, 0x4, 0x8
+HY_FAULT_SELFTEST = 0x80000000
 
 
 class HyenaLibraryMissing(RuntimeError):
@@ -113,6 +114,7 @@ def lib():
         "spectral_gate_host_workspace": (_SZ, [_I, _I, _I, _I, _I]),
         "spectral_gate_host": (_I, [_I, _I, _I, _I, _I, _VP, _VP, _I64, _VP, _VP, _VP, _SZ, _VP]),
         "hyena_device_faults": (_I, [ctypes.POINTER(ctypes.c_uint32), _I, _VP]),
+        "hyena_register_film": (_I, [_I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
         "hyena_selftest_bounded_wait": (_I, [ctypes.c_uint32, _VP]),
     }
     for name, (res, args) in sig.items():
@@ -296,6 +298,17 @@ def hyena_nd_conv_host(u, H, y, *, H_batch_stride: int = 0, circular: bool = Fal
                                     H_batch_stride, _ptr(Dskip), _ptr(gate), _ptr(y), _ptr(ws), wsb,
                                     _stream(stream)))
     return y
+
+
+def hyena_register_film(reg, W_film, gamma, beta, *, query=None, scores=None, b_film=None, stream=None):
+    """z(x) = softmax-weighted mean of the register activations reg (B, R, C)
+    and the FiLM parameters (gamma, beta) = W_film z + b_film, each (B, H)
+    (device tensors; see hyena.h)."""
+    B, R, C = reg.shape
+    H = gamma.shape[1]
+    _check(lib().hyena_register_film(B, R, C, H, _ptr(reg), _ptr(query), _ptr(scores), _ptr(W_film),
+                                     _ptr(b_film), _ptr(gamma), _ptr(beta), _stream(stream)))
+    return gamma, beta
 
 
 def projection_workspace() -> int:

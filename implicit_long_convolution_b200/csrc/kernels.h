@@ -11,6 +11,16 @@ struct ResidentParams;
 
 hy_status launch_resident_conv(const ResidentParams &p, int log_m, hy_dtype dt, bool circular,
                                cudaStream_t s);
+// one order over bf16 rows of L = 8192 with the radix-32 FFT stages on the
+// tensor cores (resident_tc.cu)
+bool resident_tc_eligible(const ResidentParams &p, int log_m, hy_dtype dt, bool circular);
+hy_status launch_resident_tc(ResidentParams p, cudaStream_t s);
+// FFT engine for the transforms that have a tensor-core version: the fp32
+// SIMT kernel (faster, see the measurements) unless the environment
+// variable HYENA_FFT_ENGINE is "tensor" (read at every call, so both can be
+// run and compared in one process).
+bool fft_engine_tensor();
+int device_sm_count();
 hy_status launch_spectrum_1d(int64_t rows, int L, int log_m, bool circular, const float *h, float2 *H,
                              cudaStream_t s);
 

@@ -1,220 +1,398 @@
 // projection.cu -- input projection of the operator ([HN] 아키텍처 상세, step 1:
 // v, x_1, ..., x_{N-1} = split(W_proj · x), a learnable linear map of the
 // token activations), written straight into the channel-major (B, D, L)
-// layout the convolution reads.
+// layout the convolution reads, with the bias added in the epilogue.
 //
-// out_k[b, d, l] = bias[k D + d] + Σ_c W[k D + d, c] · x[b, l, c]
+//   out_k[b, d, l] = bias[k D + d] + Σ_c W[k D + d, c] · x[b, l, c]
 //
-// Per output k this is one batched GEMM.  In column-major terms the output of
-// sample b is the L x D matrix with leading dimension L, so
-//   out_k[b] (L x D) = x[b]^T (L x C, i.e. the row-major (L, C) block read
-//   transposed) · W_k^T (C x D, the row-major (D, C) block read as is)
-// and the transposed layout costs nothing.  The GEMM is cuBLASLt's (bf16
-// tensor cores with fp32 accumulation, or plain fp32 without TF32); the
-// library is loaded on first use, so entry points that do not project never
-// need it.  The bias is added by a streaming pass over the output (cuBLASLt
-// offers its bias epilogue only along the other dimension of this layout).
-#include <dlfcn.h>
+// For sample b this is the GEMM  Out[m, l] = Σ_c W[m, c] · x[b, l, c]  with
+// m = k D + d.  Both operands are K-major as they sit in memory (c is the
+// contiguous index of W's rows and of x's tokens), and row m of the result is
+// the contiguous row (b, d) of out_k -- so the transpose into the
+// channel-major layout is free: one thread of the epilogue owns one row m of
+// the tile and writes its sequence positions as 16-byte runs.
+//
+// bf16: a persistent, warp-specialised tcgen05 kernel, one CTA per SM.
+//   warp 0    TMA producer: 128 x 64 tiles of W and 256 x 64 tiles of x
+//             (128-byte swizzle) into a 4-stage shared-memory ring;
+//   warp 1    allocates 512 TMEM columns (two 128 x 256 fp32 accumulators)
+//             and issues the MMAs (M = 128, N = 256, K = 16, bf16 x bf16 ->
+//             fp32) from one thread; each stage is released to the
+//             producer by tcgen05.commit, each finished tile handed to the
+//             epilogue the same way;
+//   warps 2-5 epilogue: tcgen05.ld of the accumulator (one TMEM lane = one
+//             output row per thread), + bias in fp32, one rounding to bf16,
+//             vector stores; the other accumulator is being filled
+//             meanwhile.
+// Tiles run n-major (consecutive tiles share the x tile, W stays in L2).
+// Every wait is bounded: one that gives up records HY_FAULT_PROJECTION in the
+// device fault word and the CTA winds down (the producer waits for the
+// copies it issued, the MMA thread for its MMAs) before freeing TMEM.
+//
+// fp32: plain fp32 FMA arithmetic (no TF32), a tiled SIMT kernel with the
+// same fused bias and channel-major stores.
+#include <cuda.h>
+#include <cuda_bf16.h>
 #include <mutex>
 
-#include <cublasLt.h>
-#include <cuda_bf16.h>
-
+#include "common.cuh"
 #include "status.h"
+#include "tcgen05.cuh"
 
 namespace hy {
 
 namespace {
 
-struct LtApi {
-    bool loaded = false;
-    decltype(&cublasLtCreate) create = nullptr;
-    decltype(&cublasLtMatmulDescCreate) desc_create = nullptr;
-    decltype(&cublasLtMatmulDescDestroy) desc_destroy = nullptr;
-    decltype(&cublasLtMatmulDescSetAttribute) desc_set = nullptr;
-    decltype(&cublasLtMatrixLayoutCreate) layout_create = nullptr;
-    decltype(&cublasLtMatrixLayoutDestroy) layout_destroy = nullptr;
-    decltype(&cublasLtMatrixLayoutSetAttribute) layout_set = nullptr;
-    decltype(&cublasLtMatmulPreferenceCreate) pref_create = nullptr;
-    decltype(&cublasLtMatmulPreferenceDestroy) pref_destroy = nullptr;
-    decltype(&cublasLtMatmulPreferenceSetAttribute) pref_set = nullptr;
-    decltype(&cublasLtMatmulAlgoGetHeuristic) heuristic = nullptr;
-    decltype(&cublasLtMatmul) matmul = nullptr;
+constexpr int MAX_OUT = 9;
+
+// ---------------------------------------------------------------- bf16: tcgen05
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr uint32_t A_BYTES = BM * BK * 2;           // 16 KB
+constexpr uint32_t B_BYTES = BN * BK * 2;           // 32 KB
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr uint32_t ACC_COLS = BN;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr int NT_TC = 192;
+constexpr size_t TC_SMEM = (size_t)STAGES * STAGE_BYTES + 1024;   // + 1024-byte alignment slack
+constexpr uint32_t IDESC = tc::idesc_f16(BM, BN, true);
+
+struct ProjParams {
+    int M, L, C, D;
+    int tiles_m, tiles_l;       // tiles along m, along l per sample
+    int64_t n_tiles;
+    const float *bias;
+    void *out[MAX_OUT];
+    uint32_t *fault;
 };
 
-std::mutex g_lt_mu;
-LtApi g_lt;
-cublasLtHandle_t g_lt_handle[64] = {};
-
-hy_status load_lt() {
-    if (g_lt.loaded) return HY_OK;
-    void *h = dlopen("libcublasLt.so.12", RTLD_NOW | RTLD_GLOBAL);
-    if (!h) h = dlopen("libcublasLt.so", RTLD_NOW | RTLD_GLOBAL);
-    if (!h) return set_error(HY_ERR_UNSUPPORTED, "hyena_projection: cannot load libcublasLt (%s)", dlerror());
-#define HY_SYM(field, name)                                                                              \
-    g_lt.field = reinterpret_cast<decltype(g_lt.field)>(dlsym(h, #name));                               \
-    if (!g_lt.field) return set_error(HY_ERR_UNSUPPORTED, "hyena_projection: libcublasLt lacks " #name);
-    HY_SYM(create, cublasLtCreate)
-    HY_SYM(desc_create, cublasLtMatmulDescCreate)
-    HY_SYM(desc_destroy, cublasLtMatmulDescDestroy)
-    HY_SYM(desc_set, cublasLtMatmulDescSetAttribute)
-    HY_SYM(layout_create, cublasLtMatrixLayoutCreate)
-    HY_SYM(layout_destroy, cublasLtMatrixLayoutDestroy)
-    HY_SYM(layout_set, cublasLtMatrixLayoutSetAttribute)
-    HY_SYM(pref_create, cublasLtMatmulPreferenceCreate)
-    HY_SYM(pref_destroy, cublasLtMatmulPreferenceDestroy)
-    HY_SYM(pref_set, cublasLtMatmulPreferenceSetAttribute)
-    HY_SYM(heuristic, cublasLtMatmulAlgoGetHeuristic)
-    HY_SYM(matmul, cublasLtMatmul)
-#undef HY_SYM
-    g_lt.loaded = true;
-    return HY_OK;
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&h);
 }
 
-hy_status lt_handle(cublasLtHandle_t &out) {
-    std::lock_guard<std::mutex> lock(g_lt_mu);
-    hy_status st = load_lt();
-    if (st != HY_OK) return st;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return set_cuda_error("hyena_projection: cudaGetDevice", e);
-    if (dev < 0 || dev >= 64) return set_error(HY_ERR_UNSUPPORTED, "hyena_projection: device %d", dev);
-    if (!g_lt_handle[dev]) {
-        const cublasStatus_t s = g_lt.create(&g_lt_handle[dev]);
-        if (s != CUBLAS_STATUS_SUCCESS) {
-            g_lt_handle[dev] = nullptr;
-            return set_error(HY_ERR_CUDA, "hyena_projection: cublasLtCreate failed (%d)", (int)s);
+__global__ void __launch_bounds__(NT_TC, 1)
+proj_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, const ProjParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t full[STAGES], empty[STAGES], tfull[2], tempty[2], drain;
+    __shared__ uint32_t s_tmem;
+    __shared__ volatile int s_abort;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (warp == 1) tc::tmem_alloc(&s_tmem, TMEM_COLS);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
         }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 4);             // one arrival per epilogue warp
+        }
+        mbar_init(&drain, 1);
+        mbar_init_fence();
+        s_abort = 0;
     }
-    out = g_lt_handle[dev];
-    return HY_OK;
-}
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    const uint32_t tmem = s_tmem;
+    const int nk = (p.C + BK - 1) / BK;
+    auto give_up = [&]() {
+        record_fault(p.fault, HY_FAULT_PROJECTION);
+        s_abort = 1;
+    };
 
-// out[row, l] += bias[row % D] over rows = B * D rows of length L (row-major).
-// Streaming pass: with L a multiple of 8 every 16-byte chunk (8 bf16 or 4
-// fp32) lies in one row; each thread keeps UNROLL chunks in flight.
-template <typename T>
-__global__ void __launch_bounds__(256) add_bias_vec_kernel(T *out, const float *__restrict__ bias, int64_t chunks,
-                                                           int D, int L) {
-    constexpr int PER = 16 / sizeof(T);         // elements per chunk
-    constexpr int UNROLL = 4;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t c0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; c0 < chunks; c0 += stride * UNROLL) {
-        uint4 v[UNROLL];
-        float b[UNROLL];
-#pragma unroll
-        for (int u = 0; u < UNROLL; ++u) {
-            const int64_t c = c0 + u * stride;
-            if (c < chunks) {
-                v[u] = *reinterpret_cast<const uint4 *>(out + c * PER);
-                b[u] = __ldg(bias + ((c * PER) / L) % D);
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---- TMA producer
+            int s = 0;
+            uint32_t ph = 0;
+            uint32_t armed = 0, armed_ph = 0;      // per stage: a load was issued, and its phase parity
+            for (int64_t t = blockIdx.x; t < p.n_tiles && !s_abort; t += gridDim.x) {
+                const int mt = (int)(t % p.tiles_m);
+                const int64_t nt = t / p.tiles_m;
+                const int b = (int)(nt / p.tiles_l);
+                const int l0 = (int)(nt % p.tiles_l) * BN;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(&empty[s], ph ^ 1)) {
+                        give_up();
+                        break;
+                    }
+                    uint8_t *sa = smem + (size_t)s * STAGE_BYTES;
+                    tc::mbar_expect_tx(&full[s], STAGE_BYTES);
+                    tc::tma_load_2d(sa, &tmW, kb * BK, mt * BM, &full[s]);
+                    tc::tma_load_2d(sa + A_BYTES, &tmX, kb * BK, b * p.L + l0, &full[s]);
+                    armed |= 1u << s;
+                    armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                }
             }
+            // no copy may still be landing when the CTA exits
+            for (int q = 0; q < STAGES; ++q)
+                if ((armed >> q) & 1)
+                    if (!mbar_wait(&full[q], (armed_ph >> q) & 1)) record_fault(p.fault, HY_FAULT_PROJECTION);
         }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---- MMA issuer
+            int s = 0, acc = 0;
+            uint32_t ph = 0, aph = 0;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; t < p.n_tiles && ok && !s_abort; t += gridDim.x) {
+                if (!mbar_wait(&tempty[acc], aph ^ 1)) {
+                    give_up();
+                    break;
+                }
+                tc::fence_after();
+                const uint32_t d = tmem + (uint32_t)acc * ACC_COLS;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(&full[s], ph)) {
+                        give_up();
+                        ok = false;
+                        break;
+                    }
+                    tc::fence_after();
+                    const uint32_t sa = smem_u32(smem + (size_t)s * STAGE_BYTES);
+                    const uint64_t ad = tc::desc_k_sw128(sa), bd = tc::desc_k_sw128(sa + A_BYTES);
 #pragma unroll
-        for (int u = 0; u < UNROLL; ++u) {
-            const int64_t c = c0 + u * stride;
-            if (c >= chunks) continue;
-            if constexpr (sizeof(T) == 4) {
-                float4 f = *reinterpret_cast<float4 *>(&v[u]);
-                f.x += b[u]; f.y += b[u]; f.z += b[u]; f.w += b[u];
-                *reinterpret_cast<float4 *>(out + c * PER) = f;
-            } else {
-                __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&v[u]);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) h[q] = __floats2bfloat162_rn(__low2float(h[q]) + b[u], __high2float(h[q]) + b[u]);
-                *reinterpret_cast<uint4 *>(out + c * PER) = v[u];
+                    for (int k = 0; k < BK / 16; ++k)     // K step of 16 elements = 32 bytes = 2 descriptor units
+                        tc::mma_f16(d, ad + 2 * k, bd + 2 * k, IDESC, (kb | k) != 0);
+                    tc::commit(&empty[s]);                // the stage is free once these MMAs have read it
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                }
+                if (!ok) break;
+                tc::commit(&tfull[acc]);                  // the tile's accumulator is complete
+                if (++acc == 2) {
+                    acc = 0;
+                    aph ^= 1;
+                }
             }
+            // every MMA issued has finished before TMEM is freed
+            tc::commit(&drain);
+            if (!mbar_wait(&drain, 0)) record_fault(p.fault, HY_FAULT_PROJECTION);
         }
-    }
-}
-
-// any L: one element per thread and row
-template <typename T>
-__global__ void __launch_bounds__(256) add_bias_kernel(T *out, const float *__restrict__ bias, int64_t rows,
-                                                       int D, int L) {
-    const int64_t row = blockIdx.y * (int64_t)gridDim.z + blockIdx.z;
-    if (row >= rows) return;
-    const float b = __ldg(bias + row % D);
-    T *p = out + row * (int64_t)L;
-    for (int l = blockIdx.x * blockDim.x + threadIdx.x; l < L; l += gridDim.x * blockDim.x) {
-        if constexpr (sizeof(T) == 4) p[l] = p[l] + b;
-        else p[l] = __float2bfloat16_rn(__bfloat162float(p[l]) + b);
-    }
-}
-
-template <typename T>
-hy_status add_bias(T *out, const float *bias, int64_t rows, int D, int L, cudaStream_t s) {
-    if (L % 8 == 0) {
-        const int64_t chunks = rows * L / (16 / sizeof(T));
-        int sms = 148, dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        int64_t blocks = (chunks + 256 * 4 - 1) / (256 * 4);
-        if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
-        add_bias_vec_kernel<T><<<(unsigned)blocks, 256, 0, s>>>(out, bias, chunks, D, L);
     } else {
-        dim3 grid((unsigned)((L + 255) / 256 < 8 ? (L + 255) / 256 : 8), (unsigned)((rows + 65534) / 65535),
-                  (unsigned)(rows < 65535 ? rows : 65535));
-        add_bias_kernel<T><<<grid, 256, 0, s>>>(out, bias, rows, D, L);
+        // ---- epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        int acc = 0;
+        uint32_t aph = 0;
+        for (int64_t t = blockIdx.x; t < p.n_tiles && !s_abort; t += gridDim.x) {
+            // the warp takes one decision (tcgen05.ld below is warp-wide)
+            if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], aph))) {
+                give_up();
+                break;
+            }
+            tc::fence_after();
+            const int mt = (int)(t % p.tiles_m);
+            const int64_t nt = t / p.tiles_m;
+            const int b = (int)(nt / p.tiles_l);
+            const int l0 = (int)(nt % p.tiles_l) * BN;
+            const int m = mt * BM + row;
+            const bool valid = m < p.M;
+            const int ko = valid ? m / p.D : 0;
+            const int dd = valid ? m % p.D : 0;
+            const float bias = (valid && p.bias) ? __ldg(p.bias + m) : 0.f;
+            __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.out[ko]) + ((int64_t)b * p.D + dd) * p.L;
+            const bool vec = (p.L & 7) == 0;
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t v[32];
+                tc::tmem_ld32(tmem + (uint32_t)acc * ACC_COLS + (uint32_t)(c * 32) + ((uint32_t)(q * 32) << 16), v);
+                tc::tmem_wait_ld();
+                if (!valid) continue;
+                const int l = l0 + c * 32;
+                if (vec && l + 32 <= p.L) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + l);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        uint4 w;
+                        w.x = pack_bf16(__uint_as_float(v[8 * j + 0]) + bias, __uint_as_float(v[8 * j + 1]) + bias);
+                        w.y = pack_bf16(__uint_as_float(v[8 * j + 2]) + bias, __uint_as_float(v[8 * j + 3]) + bias);
+                        w.z = pack_bf16(__uint_as_float(v[8 * j + 4]) + bias, __uint_as_float(v[8 * j + 5]) + bias);
+                        w.w = pack_bf16(__uint_as_float(v[8 * j + 6]) + bias, __uint_as_float(v[8 * j + 7]) + bias);
+                        dst[j] = w;
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (l + j < p.L) orow[l + j] = __float2bfloat16_rn(__uint_as_float(v[j]) + bias);
+                }
+            }
+            tc::fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&tempty[acc]);
+            if (++acc == 2) {
+                acc = 0;
+                aph ^= 1;
+            }
+        }
     }
-    return check_launch("hyena_projection bias");
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    __syncwarp();
+    if (warp == 1) tc::tmem_free(tmem, TMEM_COLS);
 }
 
-// One batched GEMM per projection k: out_k[b] as the column-major L x D
-// matrix (ld L) = x[b] (stored C x L, read transposed) · W_k (stored C x D).
-hy_status project_gemm(cublasLtHandle_t lt, int B, int L, int C, int D, int n_out, hy_dtype dt, const void *x,
-                       const void *W, void *const *out, void *ws, cudaStream_t stream) {
-    const char *who = "hyena_projection";
-    const size_t esz = dt == HY_BF16 ? 2 : 4;
-    const cudaDataType_t ty = dt == HY_BF16 ? CUDA_R_16BF : CUDA_R_32F;
-    cublasLtMatmulDesc_t op = nullptr;
-    cublasLtMatrixLayout_t la = nullptr, lb = nullptr, ld = nullptr;
-    cublasLtMatmulPreference_t pref = nullptr;
-    auto cleanup = [&]() {
-        if (pref) g_lt.pref_destroy(pref);
-        if (la) g_lt.layout_destroy(la);
-        if (lb) g_lt.layout_destroy(lb);
-        if (ld) g_lt.layout_destroy(ld);
-        if (op) g_lt.desc_destroy(op);
-    };
-    auto fail = [&](const char *what, cublasStatus_t s) {
-        cleanup();
-        return set_error(HY_ERR_CUDA, "%s: %s failed (%d)", who, what, (int)s);
-    };
-    cublasStatus_t s = g_lt.desc_create(&op, CUBLAS_COMPUTE_32F, CUDA_R_32F);   // no TF32: plain fp32 or bf16 MMA
-    if (s != CUBLAS_STATUS_SUCCESS) return fail("cublasLtMatmulDescCreate", s);
-    const cublasOperation_t ta = CUBLAS_OP_T, tb = CUBLAS_OP_N;
-    g_lt.desc_set(op, CUBLASLT_MATMUL_DESC_TRANSA, &ta, sizeof(ta));
-    g_lt.desc_set(op, CUBLASLT_MATMUL_DESC_TRANSB, &tb, sizeof(tb));
-    if ((s = g_lt.layout_create(&la, ty, C, L, C)) != CUBLAS_STATUS_SUCCESS) return fail("layout A", s);
-    if ((s = g_lt.layout_create(&lb, ty, C, D, C)) != CUBLAS_STATUS_SUCCESS) return fail("layout B", s);
-    if ((s = g_lt.layout_create(&ld, ty, L, D, L)) != CUBLAS_STATUS_SUCCESS) return fail("layout D", s);
-    const int32_t batch = B;
-    const int64_t sa = (int64_t)L * C, sb = 0, sd = (int64_t)L * D;   // the weights are shared by the samples
-    g_lt.layout_set(la, CUBLASLT_MATRIX_LAYOUT_BATCH_COUNT, &batch, sizeof(batch));
-    g_lt.layout_set(la, CUBLASLT_MATRIX_LAYOUT_STRIDED_BATCH_OFFSET, &sa, sizeof(sa));
-    g_lt.layout_set(lb, CUBLASLT_MATRIX_LAYOUT_BATCH_COUNT, &batch, sizeof(batch));
-    g_lt.layout_set(lb, CUBLASLT_MATRIX_LAYOUT_STRIDED_BATCH_OFFSET, &sb, sizeof(sb));
-    g_lt.layout_set(ld, CUBLASLT_MATRIX_LAYOUT_BATCH_COUNT, &batch, sizeof(batch));
-    g_lt.layout_set(ld, CUBLASLT_MATRIX_LAYOUT_STRIDED_BATCH_OFFSET, &sd, sizeof(sd));
-    if ((s = g_lt.pref_create(&pref)) != CUBLAS_STATUS_SUCCESS) return fail("preference", s);
-    const size_t wsb = (size_t)32 << 20;
-    g_lt.pref_set(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &wsb, sizeof(wsb));
-    cublasLtMatmulHeuristicResult_t heur{};
-    int found = 0;
-    s = g_lt.heuristic(lt, op, la, lb, ld, ld, pref, 1, &heur, &found);
-    if (s != CUBLAS_STATUS_SUCCESS || found < 1) {
-        cleanup();
-        return set_error(HY_ERR_UNSUPPORTED, "%s: no cuBLASLt algorithm for this shape (%d)", who, (int)s);
+// ---------------------------------------------------------------- fp32: SIMT
+constexpr int FM = 128, FN = 128, FK = 16, NT_F = 256;
+
+__global__ void __launch_bounds__(NT_F) proj_f32_kernel(const float *__restrict__ x, const float *__restrict__ W,
+                                                        const ProjParams p, int B) {
+    __shared__ float As[FK][FM + 4];     // As[k][m] = W[m0 + m, k0 + k]
+    __shared__ float Bs[FK][FN + 4];     // Bs[k][l] = x[b, l0 + l, k0 + k]
+    const int tid = threadIdx.x;
+    const int tx = tid & 15, ty = tid >> 4;
+    const int m0 = blockIdx.x * FM;
+    const int l0 = blockIdx.y * FN;
+    const int b = blockIdx.z;
+    float acc[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    const float *xb = x + (int64_t)b * p.L * p.C;
+    for (int k0 = 0; k0 < p.C; k0 += FK) {
+        // 128 rows x 16 k of each operand: 8 elements per thread, k fastest
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int idx = tid + e * NT_F;
+            const int r = idx >> 4, k = idx & 15;
+            const int gm = m0 + r, gl = l0 + r, gk = k0 + k;
+            As[k][r] = (gm < p.M && gk < p.C) ? __ldg(W + (int64_t)gm * p.C + gk) : 0.f;
+            Bs[k][r] = (gl < p.L && gk < p.C) ? __ldg(xb + (int64_t)gl * p.C + gk) : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < FK; ++k) {
+            float a[8], bv[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) a[i] = As[k][ty * 8 + i];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                bv[j] = Bs[k][tx * 4 + j];
+                bv[4 + j] = Bs[k][64 + tx * 4 + j];
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], bv[j], acc[i][j]);
+        }
+        __syncthreads();
     }
-    const float one = 1.f, zero = 0.f;
-    for (int k = 0; k < n_out; ++k) {
-        const char *Wk = reinterpret_cast<const char *>(W) + (size_t)k * D * C * esz;
-        s = g_lt.matmul(lt, op, &one, x, la, Wk, lb, &zero, out[k], ld, out[k], ld, &heur.algo, ws, wsb, stream);
-        if (s != CUBLAS_STATUS_SUCCESS) return fail("cublasLtMatmul", s);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int m = m0 + ty * 8 + i;
+        if (m >= p.M) continue;
+        const float bias = p.bias ? __ldg(p.bias + m) : 0.f;
+        float *orow = reinterpret_cast<float *>(p.out[m / p.D]) + ((int64_t)b * p.D + m % p.D) * p.L;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int l = l0 + h * 64 + tx * 4;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (l + j < p.L) orow[l + j] = acc[i][4 * h + j] + bias;
+        }
     }
-    cleanup();
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::mutex g_mu;
+EncodeTiledFn g_encode = nullptr;
+bool g_attr_set[64] = {};
+
+hy_status encode_fn(EncodeTiledFn *out) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_encode) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        const cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+            return set_error(HY_ERR_CUDA, "hyena_projection: cuTensorMapEncodeTiled is not available");
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    *out = g_encode;
     return HY_OK;
+}
+
+// 2-D bf16 tensor map over `rows` rows of `cols` elements (row pitch cols*2
+// bytes), box of 64 elements x box_rows rows, 128-byte swizzle; reads past
+// the extent land as zeros.
+hy_status bf16_map(EncodeTiledFn enc, CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows,
+                   uint32_t box_rows) {
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return set_error(HY_ERR_CUDA, "hyena_projection: cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return HY_OK;
+}
+
+hy_status launch_tc(int B, int L, int C, int D, int n_out, const void *x, const void *W, const float *bias,
+                    void *const *out, cudaStream_t s) {
+    EncodeTiledFn enc;
+    hy_status st = encode_fn(&enc);
+    if (st != HY_OK) return st;
+    const int M = n_out * D;
+    CUtensorMap mw, mx;
+    if ((st = bf16_map(enc, &mw, W, (uint64_t)C, (uint64_t)M, BM)) != HY_OK) return st;
+    if ((st = bf16_map(enc, &mx, x, (uint64_t)C, (uint64_t)B * L, BN)) != HY_OK) return st;
+    ProjParams p{};
+    p.M = M;
+    p.L = L;
+    p.C = C;
+    p.D = D;
+    p.tiles_m = (M + BM - 1) / BM;
+    p.tiles_l = (L + BN - 1) / BN;
+    p.n_tiles = (int64_t)p.tiles_m * p.tiles_l * B;
+    p.bias = bias;
+    for (int k = 0; k < n_out; ++k) p.out[k] = out[k];
+    p.fault = device_fault_word();
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (dev >= 0 && dev < 64 && !g_attr_set[dev]) {
+            const cudaError_t e =
+                cudaFuncSetAttribute(proj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TC_SMEM);
+            if (e != cudaSuccess) return set_cuda_error("hyena_projection: shared memory attribute", e);
+            g_attr_set[dev] = true;
+        }
+    }
+    const int64_t grid = p.n_tiles < sms ? p.n_tiles : sms;
+    proj_tc_kernel<<<(unsigned)grid, NT_TC, TC_SMEM, s>>>(mw, mx, p);
+    return check_launch("hyena_projection (tcgen05 GEMM)");
+}
+
+hy_status launch_f32(int B, int L, int C, int D, int n_out, const float *x, const float *W, const float *bias,
+                     void *const *out, cudaStream_t s) {
+    ProjParams p{};
+    p.M = n_out * D;
+    p.L = L;
+    p.C = C;
+    p.D = D;
+    p.bias = bias;
+    for (int k = 0; k < n_out; ++k) p.out[k] = out[k];
+    if (B > 65535) return set_error(HY_ERR_UNSUPPORTED, "hyena_projection: fp32 path takes B <= 65535");
+    dim3 grid((unsigned)((p.M + FM - 1) / FM), (unsigned)((L + FN - 1) / FN), (unsigned)B);
+    proj_f32_kernel<<<grid, NT_F, 0, s>>>(x, W, p, B);
+    return check_launch("hyena_projection (fp32 GEMM)");
 }
 
 }  // namespace
@@ -223,14 +401,16 @@ hy_status project_gemm(cublasLtHandle_t lt, int B, int L, int C, int D, int n_ou
 
 using namespace hy;
 
-extern "C" size_t hyena_projection_workspace(void) { return (size_t)32 << 20; }
+extern "C" size_t hyena_projection_workspace(void) { return 0; }
 
 extern "C" hy_status hyena_projection(int B, int L, int C, int D, int n_out, hy_dtype dt, const void *x,
                                       const void *W, const float *bias, void *const *out, void *ws,
                                       size_t ws_bytes, void *stream) {
+    (void)ws;
+    (void)ws_bytes;
     clear_error();
     const char *who = "hyena_projection";
-    if (B < 1 || L < 1 || C < 1 || D < 1 || n_out < 1 || n_out > 9)
+    if (B < 1 || L < 1 || C < 1 || D < 1 || n_out < 1 || n_out > MAX_OUT)
         return set_error(HY_ERR_INVALID_ARG, "%s: B, L, C, D must be >= 1 and n_out in 1..9", who);
     if (dt != HY_F32 && dt != HY_BF16) return set_error(HY_ERR_INVALID_ARG, "%s: unknown dtype", who);
     if (!x || !W || !out) return set_error(HY_ERR_INVALID_ARG, "%s: null pointer", who);
@@ -241,24 +421,9 @@ extern "C" hy_status hyena_projection(int B, int L, int C, int D, int n_out, hy_
         return set_error(HY_ERR_INVALID_ARG, "%s: x and W must be 16-byte aligned with rows of a multiple of 16 bytes", who);
     for (int k = 0; k < n_out; ++k)
         if ((uintptr_t)out[k] % 16) return set_error(HY_ERR_INVALID_ARG, "%s: out[%d] misaligned", who, k);
-    if (!ws || ws_bytes < hyena_projection_workspace() || (uintptr_t)ws % 256)
-        return set_error(HY_ERR_WORKSPACE, "%s: needs %zu bytes of 256-byte aligned workspace", who,
-                         hyena_projection_workspace());
-    cublasLtHandle_t lt;
-    hy_status st = lt_handle(lt);
-    if (st != HY_OK) return st;
-    st = project_gemm(lt, B, L, C, D, n_out, dt, x, W, out, ws, (cudaStream_t)stream);
-    if (st != HY_OK) return st;
-    if (bias) {
-        const int64_t rows = (int64_t)B * D;
-        for (int k = 0; k < n_out; ++k) {
-            st = dt == HY_BF16
-                     ? add_bias(reinterpret_cast<__nv_bfloat16 *>(out[k]), bias + (size_t)k * D, rows, D, L,
-                                (cudaStream_t)stream)
-                     : add_bias(reinterpret_cast<float *>(out[k]), bias + (size_t)k * D, rows, D, L,
-                                (cudaStream_t)stream);
-            if (st != HY_OK) return st;
-        }
-    }
-    return HY_OK;
+    if ((int64_t)n_out * D > (int64_t)1 << 30 || (int64_t)B * L > ((int64_t)1 << 31) - 1)
+        return set_error(HY_ERR_UNSUPPORTED, "%s: n_out*D and B*L must stay below 2^30 and 2^31", who);
+    if (dt == HY_BF16) return launch_tc(B, L, C, D, n_out, x, W, bias, out, (cudaStream_t)stream);
+    return launch_f32(B, L, C, D, n_out, reinterpret_cast<const float *>(x), reinterpret_cast<const float *>(W), bias,
+                      out, (cudaStream_t)stream);
 }

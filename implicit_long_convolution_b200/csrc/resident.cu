@@ -1,5 +1,8 @@
 // resident.cu -- entry to the on-chip path: variant selection for the
 // FFT convolution and the 1-D filter-spectrum kernels.
+#include <cstdlib>
+#include <cstring>
+
 #include "resident_launch.cuh"
 
 namespace hy {
@@ -39,10 +42,16 @@ int device_sm_count() {
 
 static bool aligned16(const void *q) { return ((uintptr_t)q & 15u) == 0; }
 
+bool fft_engine_tensor() {
+    const char *e = std::getenv("HYENA_FFT_ENGINE");
+    return e && std::strcmp(e, "tensor") == 0;
+}
+
 hy_status launch_resident_conv(const ResidentParams &p, int log_m, hy_dtype dt, bool circular,
                                cudaStream_t s) {
     if (p.n_rows <= 0) return HY_OK;
     if (p.n_rows > 0x7fffffffLL) return set_error(HY_ERR_UNSUPPORTED, "too many rows (%lld)", (long long)p.n_rows);
+    if (resident_tc_eligible(p, log_m, dt, circular) && fft_engine_tensor()) return launch_resident_tc(p, s);
     const bool chain = p.K > 1;
     // one order over whole power-of-two rows, 16-byte aligned: the persistent
     // streaming kernel (TMA bulk-copy prefetch of inputs and gate)

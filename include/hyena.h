@@ -118,6 +118,29 @@ typedef struct hy_filter_desc {
 hy_status hyena_filter_gen(const hy_filter_desc *desc, float *h, void *stream);
 
 /* ------------------------------------------------------------------------
+ * HyenaND input conditioning  ([ND] 방법론: HyenaND, 레지스터 및 FiLM을 통한
+ * 입력 의존적 커널: R register tokens are processed with each sample; the
+ * control variable z(x) is the softmax-weighted mean of their activations
+ * and modulates the kernel MLP through FiLM)
+ *
+ *   l[b, r] = query · reg[b, r, :] (query != NULL) + scores[b, r] (scores != NULL)
+ *   w[b, :] = softmax_r(l[b, :]);   z[b, :] = Σ_r w[b, r] reg[b, r, :]
+ *   gamma[b, o] = b_film[o] + Σ_c W_film[o, c] z[b, c],         o < H
+ *   beta[b, o]  = b_film[H + o] + Σ_c W_film[H + o, c] z[b, c],  o < H
+ *
+ *   reg: device fp32 (B, R, C), the register activations; query: device
+ *   fp32 (C) or NULL; scores: device fp32 (B, R) or NULL (both NULL: the
+ *   plain mean); W_film: device fp32 (2H, C) row-major; b_film: device fp32
+ *   (2H) or NULL; gamma, beta: device fp32 (B, H) outputs -- the film_gamma
+ *   / film_beta of hyena_filter_gen with n_sets = B and H = widths[1].
+ *   R <= 1024, C <= 8192.  fp32 arithmetic; the softmax subtracts the
+ *   maximum logit.
+ * ---------------------------------------------------------------------- */
+hy_status hyena_register_film(int B, int R, int C, int H, const float *reg, const float *query,
+                              const float *scores, const float *W_film, const float *b_film,
+                              float *gamma, float *beta, void *stream);
+
+/* ------------------------------------------------------------------------
  * Filter spectrum  ([HN] fft_conv; [ES] FFT convolution; [ND] N-D FFT)
  *
  *   ndim = 1: dims[0] = L.  Each of `rows` filter rows h[r, 0..L) is
@@ -294,13 +317,15 @@ hy_status spectral_gate(int B, int H, int Dh, int L, hy_dtype dt, const void *x,
  *   row-major (the PyTorch Linear layout); bias: device fp32 (n_out·D) or
  *   NULL; out: host array of n_out device pointers, each (B, D, L) -- the
  *   channel-major layout hyena_operator reads, no transpose needed.
- *   x, W, out share dt.  bf16: tensor-core GEMM with fp32 accumulation,
- *   the product rounded to bf16, then the bias added (a second pass over
- *   the outputs) and rounded again; fp32: fp32 arithmetic (no TF32).  The GEMM is cuBLASLt's, loaded on the first
- *   call (HY_ERR_UNSUPPORTED if it cannot be loaded).
+ *   x, W, out share dt.  bf16: the library's tcgen05 tensor-core GEMM
+ *   (bf16 operands, fp32 accumulation in tensor memory); the bias is added
+ *   to the fp32 result in the kernel's epilogue and the sum is rounded to
+ *   bf16 once.  fp32: fp32 FMA arithmetic (no TF32), the same fused bias.
  *   x, W, out 16-byte aligned and C·sizeof(dt) a multiple of 16;
- *   ws: device workspace of hyena_projection_workspace() bytes, 256-byte
- *   aligned.
+ *   n_out·D < 2^30, B·L < 2^31.  No workspace is needed
+ *   (hyena_projection_workspace() returns 0; ws may be NULL).
+ *   A bounded wait of the GEMM that gives up sets HY_FAULT_PROJECTION
+ *   (see hyena_device_faults).
  * ---------------------------------------------------------------------- */
 size_t hyena_projection_workspace(void);
 hy_status hyena_projection(int B, int L, int C, int D, int n_out, hy_dtype dt, const void *x,
@@ -360,9 +385,14 @@ hy_status spectral_gate_host(int B, int H, int Dh, int L, hy_dtype dt, const voi
  * about one second of %globaltimer, ORs a bit below into a per-device fault
  * word (a static device variable; nothing is allocated) and the CTA returns
  * at its next row boundary, after a bounded wait for its copies in flight.
+ * The tensor-core kernels (projection GEMM, tensor-core convolution) bound
+ * their pipeline waits the same way and wait for their copies and MMAs in
+ * flight before they free tensor memory and return.
  * The outputs of such a launch are then undefined. */
 #define HY_FAULT_STREAM_INPUT 0x1u      /* a row's input copy did not land in time */
 #define HY_FAULT_STREAM_GATE 0x2u       /* a row's gate copy did not land in time  */
+#define HY_FAULT_PROJECTION 0x4u        /* a wait of the tensor-core projection GEMM ran out */
+#define HY_FAULT_TC_CONV 0x8u           /* a wait for the tensor-core convolution's MMAs ran out */
 #define HY_FAULT_SELFTEST 0x80000000u   /* hyena_selftest_bounded_wait ran out      */
 /* Reads the current device's fault word into *faults after the work queued on
  * `stream` has finished (the call synchronises that stream); clear != 0 then

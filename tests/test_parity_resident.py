@@ -191,10 +191,13 @@ def test_c1_end_to_end():
     check(to_np(y).reshape(B * D, L), ref, "f32", "c1 end-to-end")
 
 
-def test_c2_full_size():
+@pytest.mark.parametrize("engine", ["tensor", "simt"])
+def test_c2_full_size(engine, monkeypatch):
     """Workload 2 at full size (B8 D768 L8192, bf16 I/O) in the launch the
-    benchmark times: all rows against the FFT-route reference, 16 sampled rows
-    against the direct O(L^2) chain."""
+    benchmark times, with the radix-32 FFT stages on the fp32 SIMT pipes (the
+    default) and on the tensor cores: all rows against the FFT-route
+    reference, 16 sampled rows against the direct O(L^2) chain."""
+    monkeypatch.setenv("HYENA_FFT_ENGINE", engine)
     w = hw.make("c2")
     s = w.spec
     B, D, L = s["B"], s["D"], s["L"]
@@ -212,9 +215,9 @@ def test_c2_full_size():
     got = to_np(y).reshape(B * D, L)
     rows = np.random.default_rng(2).choice(B * D, 16, replace=False)
     ref_rows = oracle.hyena_rows(w.v.f32, [w.xs[0].f32], h64.reshape(1, D, L), w.Dskip, rows=rows)
-    check(got[rows], ref_rows, "bf16", "c2 sampled rows (direct)")
+    check(got[rows], ref_rows, "bf16", "c2 sampled rows (direct), %s engine" % engine)
     ref_all = oracle.fft_hyena_rows(w.v.f32, [w.xs[0].f32], h64.reshape(1, D, L), w.Dskip)
-    r = check(got, ref_all, "bf16", "c2 all rows (FFT route)")
+    r = check(got, ref_all, "bf16", "c2 all rows (FFT route), %s engine" % engine)
     assert r < 5e-3
     assert bf16_ulp_diff(y, ref_all.reshape(y.shape)) <= 2
 

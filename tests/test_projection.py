@@ -1,14 +1,16 @@
 """Input projection (v, x_1, ... = split(W_proj x), written channel-major)
-against the float64 oracle: ragged and odd sizes in bf16 (tensor cores) and
-fp32, with and without bias; the projection feeding the operator end to end;
-and the order-2 projection at the width of the operator workload (B8 L8192,
-768 -> 2 x 768) on sampled rows."""
+against the float64 oracle: ragged and odd sizes in bf16 (the tcgen05 GEMM:
+partial M, L and K tiles, several tiles per CTA) and fp32, with and without
+bias; bf16 outputs are the fp32 result plus bias rounded once (within one
+bf16 ulp of the float64 value); the projection feeding the operator end to
+end; and the order-2 projection at the width of the operator workload (B8
+L8192, 768 -> 2 x 768) on sampled rows."""
 import numpy as np
 import pytest
 
 import hyena_workloads as hw
 import oracle
-from _helpers import check, f32_dev, to_np
+from _helpers import bf16_ulp_diff, check, f32_dev, to_np
 
 pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
@@ -33,6 +35,7 @@ def _ws():
 @pytest.mark.parametrize("B,L,C,D,n_out,dtype,with_bias", [
     (2, 1000, 64, 48, 3, "bf16", True),
     (3, 257, 24, 40, 2, "bf16", False),
+    (4, 8000, 200, 100, 3, "bf16", True),
     (1, 513, 32, 16, 2, "f32", True),
     (2, 64, 8, 5, 4, "f32", False),
 ])
@@ -54,6 +57,9 @@ def test_projection_vs_oracle(B, L, C, D, n_out, dtype, with_bias):
     ref = oracle.projection(x, W, bias, n_out)
     for k in range(n_out):
         check(to_np(outs[k]), ref[k], dtype, "projection %s out %d" % (dtype, k))
+        if dtype == "bf16":
+            # one rounding of the fp32 accumulator plus bias
+            assert bf16_ulp_diff(outs[k], ref[k]) <= 1, "projection out %d: more than 1 bf16 ulp" % k
 
 
 def test_projection_then_operator():
@@ -96,3 +102,4 @@ def test_projection_operator_width_sampled():
         ref = oracle.projection(xs[b:b + 1, ls], Ws, bias, 2)
         for k in range(2):
             check(to_np(outs[k][b:b + 1, :, ls]), ref[k], "bf16", "projection B8 L8192 b%d out %d" % (b, k))
+            assert bf16_ulp_diff(outs[k][b:b + 1, :, ls].contiguous(), ref[k]) <= 1

@@ -73,6 +73,28 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
     return false;
 }
 
+// The same bounded wait for one thread that expects a long wait (tensor-core
+// work): each try_wait suspends the thread for up to kSleepHintNs or until
+// the phase completes, so the waiting warp issues almost nothing.
+constexpr uint32_t kSleepHintNs = 20000;
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
+    const uint32_t b = smem_u32(bar);
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 0; i < kWaitMaxPolls; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(b), "r"(parity), "r"(kSleepHintNs)
+            : "memory");
+        if (done) return true;
+        if (global_ns() - t0 > limit_ns) return false;
+    }
+    return false;
+}
+
 __device__ __forceinline__ void record_fault(uint32_t *word, uint32_t bit) {
     if (word) atomicOr(word, bit);
 }

@@ -393,6 +393,7 @@ hy_status spectral_gate_host(int B, int H, int Dh, int L, hy_dtype dt, const voi
 #define HY_FAULT_STREAM_GATE 0x2u       /* a row's gate copy did not land in time  */
 #define HY_FAULT_PROJECTION 0x4u        /* a wait of the tensor-core projection GEMM ran out */
 #define HY_FAULT_TC_CONV 0x8u           /* a wait for the tensor-core convolution's MMAs ran out */
+#define HY_FAULT_FILTER_MMA 0x10u       /* a wait for the filter generator's last-layer MMAs ran out */
 #define HY_FAULT_SELFTEST 0x80000000u   /* hyena_selftest_bounded_wait ran out      */
 /* Reads the current device's fault word into *faults after the work queued on
  * `stream` has finished (the call synchronises that stream); clear != 0 then

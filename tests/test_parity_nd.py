@@ -206,3 +206,27 @@ def test_c4_full_size():
         direct = oracle.nd_conv_points(kern, w.v.f32[b, d], w.xs[0].f32[b, d], 0.0, pts)
         check_part(got[b, d].ravel()[pts], direct, float(np.sqrt(np.mean(ref ** 2))), "f32",
                    "c4 slab b%d d%d voxels (direct)" % (b, d))
+
+
+def test_nd_filter_gen_resident_weights_film():
+    """3-D kernels on a 64^3 transform grid (g = 32), FiLM on two sets: the
+    persistent resident-weight filter kernel; sampled grid points of both
+    sets against the oracle (with the support mask)."""
+    g, F, nout = 32, 4, 12
+    rng = np.random.default_rng(3232)
+    widths = [6 * F, 32, nout]
+    Ws = [rng.uniform(-1, 1, (b, a)).astype(np.float32) / np.sqrt(a) for a, b in zip(widths[:-1], widths[1:])]
+    bs = [rng.uniform(-0.5, 0.5, b).astype(np.float32) for b in widths[1:]]
+    alpha = rng.uniform(0.5, 3.0, nout).astype(np.float32)
+    gam = rng.normal(0, 0.1, (2, 32)).astype(np.float32)
+    bet = rng.normal(0, 0.1, (2, 32)).astype(np.float32)
+    S = 2 * g
+    h = torch.empty((2, nout, S, S, S), device="cuda")
+    hy.hyena_filter_gen(h, ndim=3, grid=g, Ws=[f32_dev(a) for a in Ws], bs=[f32_dev(a) for a in bs],
+                        alpha=f32_dev(alpha), n_freq=F, film_gamma=f32_dev(gam), film_beta=f32_dev(bet), n_sets=2)
+    torch.cuda.synchronize()
+    got = to_np(h).reshape(2, nout, -1)
+    idx = np.random.default_rng(5).choice(S ** 3, 20000, replace=False)
+    for b in range(2):
+        ref = oracle.filter_gen_3d_points(g, False, F, Ws, bs, gam[b], bet[b], alpha, idx)
+        check(got[b][:, idx], ref.T, "f32", "resident-weight 3-D filters set %d" % b)

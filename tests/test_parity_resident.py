@@ -287,3 +287,32 @@ def test_c5_full_size():
                                        w.v.f32.reshape(R, L)[rows], w.xs[0].f32.reshape(R, L)[rows])
     check(got[rows], direct, "bf16", "c5 sampled rows (direct)")
     assert rel_l2(got, ref) < 5e-3
+
+
+@pytest.mark.parametrize("engine", ["simt", "tensor"])
+@pytest.mark.parametrize("act,hidden,nout", [("silu", [32, 24], 40), ("sine", [32, 24], 40),
+                                               ("silu", [96], 200), ("silu", [64], 512)])
+def test_filter_gen_resident_weights_many_tiles(act, hidden, nout, engine, monkeypatch):
+    """Enough positions for the persistent resident-weight filter kernel
+    (more than 8 position tiles per SM), its last layer on the FP32 pipes
+    (default) or on the tensor cores (HYENA_FILTER_ENGINE=tensor, fp16 hi/lo
+    operands): 1-D L = 2^17, one or two hidden layers, a last layer with K over
+    one 64-element atom and outputs over several 128-row tiles (512 outputs:
+    one CTA per SM, or the streaming kernel on the FP32 pipes); every position
+    and output against the oracle."""
+    monkeypatch.setenv("HYENA_FILTER_ENGINE", engine)
+    L, F = 1 << 17, 8
+    rng = np.random.default_rng(170 + (act == "sine") + nout)
+    widths = [1 + 2 * F] + hidden + [nout]
+    Ws = [rng.uniform(-1, 1, (b, a)).astype(np.float32) / np.sqrt(a) for a, b in zip(widths[:-1], widths[1:])]
+    bs = [rng.uniform(-0.5, 0.5, b).astype(np.float32) for b in widths[1:]]
+    alpha = rng.uniform(0.1, 2.0, widths[-1]).astype(np.float32)
+    omega = rng.uniform(1, 4, sum(hidden)).astype(np.float32) if act == "sine" else None
+    h = torch.empty((widths[-1], L), device="cuda")
+    hy.hyena_filter_gen(h, ndim=1, L=L, Ws=[f32_dev(a) for a in Ws], bs=[f32_dev(a) for a in bs],
+                        alpha=f32_dev(alpha), n_freq=F, include_t=True,
+                        act=hy.HY_ACT_SINE if act == "sine" else hy.HY_ACT_SILU,
+                        omega=f32_dev(omega) if omega is not None else None)
+    torch.cuda.synchronize()
+    ref = oracle.filter_gen_1d(L, F, True, Ws, bs, alpha, act=act, omega=omega)
+    check(to_np(h), ref, "f32", "resident-weight filters L=2^17 (%s, %s)" % (act, engine))

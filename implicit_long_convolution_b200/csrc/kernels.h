@@ -1,5 +1,6 @@
 // kernels.h -- internal launcher declarations (host side).
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -21,6 +22,13 @@ hy_status launch_resident_tc(ResidentParams p, cudaStream_t s);
 // run and compared in one process).
 bool fft_engine_tensor();
 int device_sm_count();
+
+// 2-D TMA tensor map over `outer` rows of `inner` elements (row pitch
+// row_bytes), box box_inner x box_outer, reads past the extent land as zeros
+// (tma_map.cu).  The map covers this GPU's memory only.
+hy_status tma_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
+                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle,
+                     const char *who);
 hy_status launch_spectrum_1d(int64_t rows, int L, int log_m, bool circular, const float *h, float2 *H,
                              cudaStream_t s);
 

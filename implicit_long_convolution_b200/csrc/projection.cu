@@ -36,6 +36,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "kernels.h"
 #include "status.h"
 #include "tcgen05.cuh"
 
@@ -305,53 +306,21 @@ __global__ void __launch_bounds__(NT_F) proj_f32_kernel(const float *__restrict_
 }
 
 // ---------------------------------------------------------------- host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
 std::mutex g_mu;
-EncodeTiledFn g_encode = nullptr;
 bool g_attr_set[64] = {};
-
-hy_status encode_fn(EncodeTiledFn *out) {
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_encode) {
-        void *fn = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        const cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
-        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
-            return set_error(HY_ERR_CUDA, "hyena_projection: cuTensorMapEncodeTiled is not available");
-        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
-    }
-    *out = g_encode;
-    return HY_OK;
-}
-
-// 2-D bf16 tensor map over `rows` rows of `cols` elements (row pitch cols*2
-// bytes), box of 64 elements x box_rows rows, 128-byte swizzle; reads past
-// the extent land as zeros.
-hy_status bf16_map(EncodeTiledFn enc, CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows,
-                   uint32_t box_rows) {
-    const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {cols * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
-                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return set_error(HY_ERR_CUDA, "hyena_projection: cuTensorMapEncodeTiled failed (%d)", (int)r);
-    return HY_OK;
-}
 
 hy_status launch_tc(int B, int L, int C, int D, int n_out, const void *x, const void *W, const float *bias,
                     void *const *out, cudaStream_t s) {
-    EncodeTiledFn enc;
-    hy_status st = encode_fn(&enc);
-    if (st != HY_OK) return st;
     const int M = n_out * D;
+    // W and x as 2-D bf16 arrays (rows of C elements), boxes of 64 x 128 and
+    // 64 x 256 with the 128-byte swizzle; reads past the extent land as zeros
     CUtensorMap mw, mx;
-    if ((st = bf16_map(enc, &mw, W, (uint64_t)C, (uint64_t)M, BM)) != HY_OK) return st;
-    if ((st = bf16_map(enc, &mx, x, (uint64_t)C, (uint64_t)B * L, BN)) != HY_OK) return st;
+    hy_status st = tma_map_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, (uint64_t)C, (uint64_t)M, (uint64_t)C * 2, BK,
+                              BM, CU_TENSOR_MAP_SWIZZLE_128B, "hyena_projection");
+    if (st != HY_OK) return st;
+    st = tma_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)C, (uint64_t)B * L, (uint64_t)C * 2, BK, BN,
+                    CU_TENSOR_MAP_SWIZZLE_128B, "hyena_projection");
+    if (st != HY_OK) return st;
     ProjParams p{};
     p.M = M;
     p.L = L;

@@ -349,7 +349,7 @@ def setup_operator(w, dev, hy, torch):
     st.output = y
     M = nb - 1
     if wso:
-        rows_chunk = max(1, wso // (12 * M))
+        rows_chunk = max(1, wso // (8 * M))
         op_l = -(-(B * D) // rows_chunk) * (1 + 2 * K)
         st.kernel = "multi-pass colpass/rowpass kernels (M=2^%d)" % (M.bit_length() - 1)
     else:
@@ -361,7 +361,7 @@ def setup_operator(w, dev, hy, torch):
         st.kernel = "%s<M=2^%d>" % ("resident_tc_kernel" if tensor else
                                     "resident_stream_kernel" if stream else "resident_conv_kernel",
                                     M.bit_length() - 1)
-    spec_l = 2 * -(-(K * D) // max(1, wsf // (12 * M))) if wsf else 1
+    spec_l = 2 * -(-(K * D) // max(1, wsf // (8 * M))) if wsf else 1
     st.launches = 1 + spec_l + op_l
     return st
 

@@ -37,6 +37,7 @@ HY_ACT_SILU, HY_ACT_IDENTITY, HY_ACT_SINE = 0, 1, 2
 HY_WIN_EXP, HY_WIN_GAUSS = 0, 1
 HY_FAULT_STREAM_INPUT, HY_FAULT_STREAM_GATE, HY_FAULT_PROJECTION, HY_FAULT_TC_CONV = 0x1, 0x2, 0x4, 0x8
 HY_FAULT_FILTER_MMA = 0x10
+HY_FAULT_MULTIPASS = 0x20
 HY_FAULT_SELFTEST = 0x80000000
 
 

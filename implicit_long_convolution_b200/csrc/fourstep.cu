@@ -17,18 +17,31 @@
 //                     the merge there, then the inverse row FFT and
 //                     W_M^{-n1 k2}.
 //   pass C (columns): inverse FFT over k2, first half of the outputs only,
-//                     then skip term and gate; when another order follows,
-//                     its pass A runs in the same kernel on the same columns.
+//                     then the gate; when another order follows, its pass A
+//                     runs in the same kernel on the same columns.
+//
+// The skip term D_k z_k is taken into the product: D_k z_k is the causal
+// convolution of z_k with D_k times a unit impulse, whose length-2M DFT is
+// D_k at every bin, so pass B multiplies by H_k + D_k instead of H_k and
+// nothing else of z_k has to be kept (the rounding of the skip term then
+// follows the FFT round trip, a few fp32 ulps of |D_k z_k|).
 //
 // Each column or row FFT (N1, N2 <= 1024) is done by one warp (block_fft with
-// warp synchronisation); columns are staged through shared memory so global
-// accesses stay coalesced.  Rows are processed in chunks whose intermediates
-// (8 bytes per complex point) stay resident in the 126 MB L2 between passes.
+// warp synchronisation).  A column pass moves its 8 columns x N2 rows of the
+// complex intermediate between global and shared memory as 2-D TMA tensor
+// tiles (rows of 64 bytes, 64-byte swizzle, loads completing on an mbarrier
+// with a bounded wait, stores as bulk tensor stores), so no thread spends
+// registers or instructions on the strided transfer and three CTAs fit on an
+// SM.  Rows are processed in chunks whose intermediates (8 bytes per complex
+// point) stay resident in the 126 MB L2 between passes.
+#include <cstdlib>
 #include <mutex>
 
+#include "../../include/hyena.h"
 #include "kernels.h"
 #include "fft_core.cuh"
 #include "status.h"
+#include "tcgen05.cuh"
 #include "twiddle.h"
 
 namespace hy {
@@ -46,6 +59,11 @@ __device__ __forceinline__ float2 tw2(const float2 *__restrict__ tab, int lo, ui
     const float2 b = __ldg(tab + (1u << lo) + (e >> lo));
     return cmul(a, b);
 }
+// The twiddles of a warp's 32 P points e = u (lane + 32 m) (u the same for
+// the whole warp) split as W^{u lane} W^{32 u m}: one gather per lane, and per
+// m a lookup whose address is the same in every lane (one sector instead of
+// up to 32 scattered ones).  Four table entries and three roundings per
+// twiddle instead of two and one.
 
 struct FsParams {
     int64_t row0;                 // first row of this chunk (flat b*D + d)
@@ -54,10 +72,9 @@ struct FsParams {
     int K, k;                     // orders, current order
     const void *u;                // z_0 rows (IO)
     const void *gate_k;           // x_k of the current order (pass C), IO
-    const float *skip_k;          // D_k (pass C)
+    const float *skip_k;          // D_k (pass B: added to every bin of H_k)
     const float2 *spec;           // H of the current order (pass B)
     float2 *buf;                  // ws: complex buffer, chunk_rows x M
-    float *stash;                 // ws: fp32 z_{k} of the chunk, chunk_rows x M
     void *y;                      // output (IO)
     float scale;                  // 1 / (2n)
     const float2 *tw_n1;          // block FFT tables (size N1, per-lane 2^(log N1 - 5))
@@ -68,14 +85,27 @@ struct FsParams {
     int lo_2m;
     float2 *Hout;                 // spectrum mode: output bins (rows x (M+1))
     int vec4;                     // rows of u, gates and y take 4-element vector accesses
+    uint32_t *fault;              // device fault word (a tile copy that did not land)
 };
+
+// Column tiles in shared memory.  The TMA tile of a column pass is N2 rows x
+// 64 bytes (8 complex columns) with the 64-byte swizzle: the 16-byte chunk j
+// of row r sits at chunk j ^ ((r >> 1) & 3).  It shares its space with the
+// warps' padded FFT exchange buffers (WARPS x spad_size(N2) complex), which
+// are larger; the space starts on a 1024-byte boundary.
+template <int LOG_N2>
+__host__ __device__ constexpr size_t colpass_smem_bytes() {
+    return 1024 + sizeof(float2) * (size_t)WARPS * spad_size(1 << LOG_N2);
+}
+constexpr int kTileBoxRows = 256;    // rows per TMA box (the box limit)
+__device__ __forceinline__ int tile_swz(int r, int c) { return 64 * r + ((((c >> 1) ^ (r >> 1)) & 3) << 4) + ((c & 1) << 3); }
 
 // ----------------------------------------------------------------------------
 // Column pass: A (forward), C (inverse + epilogue), or C followed by A.
 // Block (blockIdx.x = column block of 8, blockIdx.y = row in chunk).
 // ----------------------------------------------------------------------------
 template <int LOG_N1, int LOG_N2, typename IO, bool INV, bool FWD, bool SPEC_INPUT>
-__global__ void __launch_bounds__(NT) colpass_kernel(const FsParams p) {
+__global__ void __launch_bounds__(NT, 3) colpass_kernel(const FsParams p, const __grid_constant__ CUtensorMap bmap) {
     constexpr int N1 = 1 << LOG_N1;
     constexpr int N2 = 1 << LOG_N2;
     constexpr int M = N1 * N2;
@@ -84,13 +114,15 @@ __global__ void __launch_bounds__(NT) colpass_kernel(const FsParams p) {
     constexpr int CS = spad_size(N2);           // column stride in the tile
     using IOT = IOTraits<IO>;
 
-    extern __shared__ float2 tile[];            // WARPS columns x CS
+    constexpr int BR = N2 < kTileBoxRows ? N2 : kTileBoxRows;
+    extern __shared__ unsigned char smem_raw[];
+    __shared__ uint64_t tile_bar;
+    unsigned char *tb = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);   // TMA tile
+    float2 *tile = reinterpret_cast<float2 *>(tb);   // WARPS padded columns x CS (same space)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n1_0 = blockIdx.x * WARPS;
     const int64_t row = p.row0 + blockIdx.y;
     const int64_t rl = blockIdx.y;              // row within chunk
-    float2 *buf = p.buf + rl * (int64_t)M;
-    float *stash = p.stash + rl * (int64_t)M;
     const int L = p.L;
     float2 *col = tile + warp * CS;
     float2 x[P];
@@ -120,53 +152,54 @@ __global__ void __launch_bounds__(NT) colpass_kernel(const FsParams p) {
     };
     auto io1 = [](const IO *q) { return IOT::load(q); };
     auto io4 = [](const IO *q) { return IOT::load4(q); };
-    auto f1 = [](const float *q) { return __ldcg(q); };
-    auto f4 = [](const float *q) { return __ldcg(reinterpret_cast<const float4 *>(q)); };
     auto h1 = [](const float *q) { return ldv(q); };
     auto h4 = [](const float *q) { return ldv4(q); };
 
     if constexpr (INV) {
-        // ---- load all N2 rows of the 8 columns (coalesced float4 = 2 complex)
-        {
-            constexpr int EL = N2 * (WARPS / 2) / NT;
-            float4 v[EL];
-#pragma unroll
-            for (int i = 0; i < EL; ++i) {
-                const int e = tid + i * NT;
-                const int r = e / (WARPS / 2), c2 = (e % (WARPS / 2)) * 2;
-                v[i] = __ldcg(reinterpret_cast<const float4 *>(buf + n1_0 + c2 + (int64_t)N1 * r));
-            }
-#pragma unroll
-            for (int i = 0; i < EL; ++i) {
-                const int e = tid + i * NT;
-                const int r = e / (WARPS / 2), c2 = (e % (WARPS / 2)) * 2;
-                tile[c2 * CS + spad(r)] = make_float2(v[i].x, v[i].y);
-                tile[(c2 + 1) * CS + spad(r)] = make_float2(v[i].z, v[i].w);
-            }
+        // ---- all N2 rows of the 8 columns: one TMA tile (N2 / BR boxes of
+        //      16 floats x BR rows at x = 2 n1_0, y = rl N2 + b BR)
+        if (tid == 0) {
+            mbar_init(&tile_bar, 1);
+            mbar_init_fence();
         }
         __syncthreads();
-        load_own<LOG_N2, LP>(x, col, lane);
-        __syncwarp();
+        if (tid == 0) {
+            tc::mbar_expect_tx(&tile_bar, (uint32_t)N2 * 64u);
+#pragma unroll
+            for (int b = 0; b < N2 / BR; ++b)
+                tc::tma_load_2d(tb + b * BR * 64, &bmap, 2 * n1_0, (int)(rl * N2 + b * BR), &tile_bar);
+        }
+        const bool landed = mbar_wait(&tile_bar, 0);
+        // column `warp`, rows lane + 32 m: the swizzle term depends on the lane only
+        {
+            const unsigned char *src = tb + tile_swz(lane, warp);
+#pragma unroll
+            for (int m = 0; m < P; ++m) x[m] = *reinterpret_cast<const float2 *>(src + 2048 * m);
+        }
+        if (__syncthreads_or(!landed)) {
+            // the tile did not land in time: record it, give the copy one more
+            // bounded wait so it does not write into a later CTA's memory, stop
+            if (tid == 0) {
+                record_fault(p.fault, HY_FAULT_MULTIPASS);
+                mbar_wait(&tile_bar, 0);
+            }
+            return;
+        }
         block_fft<LOG_N2, LP, +1, false, SyncWarp>(x, col, lane, p.tw_n2, SyncWarp{});
         // keep the first half (n2 < N2/2): samples 2m, 2m+1 with m < M/2
 #pragma unroll
         for (int m = 0; m < P / 2; ++m) col[spad(lane + 32 * m)] = x[m];
-        // ---- epilogue inputs (gate, skip source), all requested up front
-        const float dk = p.skip_k ? __ldg(p.skip_k + row % p.D) : 0.f;
+        // ---- gate inputs, all requested up front
         const IO *g = reinterpret_cast<const IO *>(p.gate_k);
         const IO *grow = g ? g + row * (int64_t)L : nullptr;
-        const IO *uin = reinterpret_cast<const IO *>(p.u) + row * (int64_t)L;
         const bool vec = p.vec4 != 0;
-        float4 gv[EIT], pv[EIT];
+        float4 gv[EIT];
 #pragma unroll
         for (int i = 0; i < EIT; ++i) {
             int r, c2;
             group_of(i, r, c2);
             const int64_t s0 = 2 * ((int64_t)n1_0 + c2 + (int64_t)N1 * r);
             gv[i] = grow ? load_row4(grow, s0, vec, io1, io4) : make_float4(1.f, 1.f, 1.f, 1.f);
-            if (dk == 0.f) pv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-            else if (p.k == 0) pv[i] = load_row4(uin, s0, vec, io1, io4);
-            else pv[i] = load_row4(stash, s0, true, f1, f4);
         }
         __syncthreads();
         // ---- epilogue: 8 columns x N2/2 rows; each thread handles 2 complex
@@ -180,8 +213,8 @@ __global__ void __launch_bounds__(NT) colpass_kernel(const FsParams p) {
             const int64_t s0 = 2 * ((int64_t)n1_0 + c2 + (int64_t)N1 * r);   // first real sample
             const float2 a = tile[c2 * CS + spad(r)], b = tile[(c2 + 1) * CS + spad(r)];
             const float sc = p.scale;
-            float4 v = make_float4(gv[i].x * fmaf(dk, pv[i].x, a.x * sc), gv[i].y * fmaf(dk, pv[i].y, a.y * sc),
-                                   gv[i].z * fmaf(dk, pv[i].z, b.x * sc), gv[i].w * fmaf(dk, pv[i].w, b.y * sc));
+            float4 v = make_float4(gv[i].x * (a.x * sc), gv[i].y * (a.y * sc), gv[i].z * (b.x * sc),
+                                   gv[i].w * (b.y * sc));
             if (s0 + 0 >= L) v.x = 0.f;
             if (s0 + 1 >= L) v.y = 0.f;
             if (s0 + 2 >= L) v.z = 0.f;
@@ -197,14 +230,6 @@ __global__ void __launch_bounds__(NT) colpass_kernel(const FsParams p) {
                         if (s0 + q < L) IOT::store(yout + s0 + q, vv[q]);
                 }
             } else {
-                if (full) {
-                    __stcg(reinterpret_cast<float4 *>(stash + s0), v);
-                } else {
-                    const float vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        if (s0 + q < L) __stcg(stash + s0 + q, vv[q]);
-                }
                 tile[c2 * CS + spad(r)] = make_float2(v.x, v.y);
                 tile[(c2 + 1) * CS + spad(r)] = make_float2(v.z, v.w);
             }
@@ -245,18 +270,26 @@ __global__ void __launch_bounds__(NT) colpass_kernel(const FsParams p) {
         load_own<LOG_N2, LP>(x, col, lane);
         __syncwarp();
         block_fft<LOG_N2, LP, -1, true, SyncWarp>(x, col, lane, p.tw_n2, SyncWarp{});
+        // W_M^{n1 k2}, k2 = lane + 32 m
         const uint32_t n1 = n1_0 + warp;
+        const float2 tl = tw2(p.tw_m, p.lo_m, (n1 * (uint32_t)lane) & (M - 1));
 #pragma unroll
-        for (int m = 0; m < P; ++m) {
-            const uint32_t k2 = lane + 32 * m;
-            x[m] = cmul(x[m], tw2(p.tw_m, p.lo_m, (n1 * k2) & (M - 1)));
-            col[spad(k2)] = x[m];
-        }
+        for (int m = 0; m < P; ++m) x[m] = cmul(x[m], cmul(tl, tw2(p.tw_m, p.lo_m, (32u * n1 * (uint32_t)m) & (M - 1))));
+        // ---- back to the buffer as one TMA tile: every warp is done with its
+        //      exchange buffer before the tile overwrites them
         __syncthreads();
-        for (int e = tid; e < N2 * (WARPS / 2); e += NT) {
-            const int r = e / (WARPS / 2), c2 = (e % (WARPS / 2)) * 2;
-            const float2 a = tile[c2 * CS + spad(r)], b = tile[(c2 + 1) * CS + spad(r)];
-            __stcg(reinterpret_cast<float4 *>(buf + n1_0 + c2 + (int64_t)N1 * r), make_float4(a.x, a.y, b.x, b.y));
+        {
+            unsigned char *dst = tb + tile_swz(lane, warp);
+#pragma unroll
+            for (int m = 0; m < P; ++m) *reinterpret_cast<float2 *>(dst + 2048 * m) = x[m];
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+#pragma unroll
+            for (int b = 0; b < N2 / BR; ++b) tc::tma_store_2d(&bmap, tb + b * BR * 64, 2 * n1_0, (int)(rl * N2 + b * BR));
+            tc::bulk_commit();
+            tc::bulk_wait_all();
         }
     }
 }
@@ -330,6 +363,7 @@ __global__ void __launch_bounds__(NT, 2) rowpass_kernel(const FsParams p) {
 
     const int64_t d = row % p.D;
     const float2 *H = SPEC ? nullptr : p.spec + d * (int64_t)(M + 1);
+    const float dk = (!SPEC && p.skip_k) ? __ldg(p.skip_k + d) : 0.f;   // skip term: H_k + D_k
     float2 *Ho = SPEC ? p.Hout + row * (int64_t)(M + 1) : nullptr;
 
     // staging of batch b: [w][0][kk] = H[k], [w][1][kk] = H[M - k] with
@@ -365,7 +399,9 @@ __global__ void __launch_bounds__(NT, 2) rowpass_kernel(const FsParams p) {
     for (int m = 0; m < P; ++m) own[spad(lane + 32 * m)] = x[m];
     __syncthreads();
 
-    // ---- pairs of the owned bins k1 = lane + 32 m < N1/2 (m < P/2)
+    // ---- pairs of the owned bins k1 = lane + 32 m < N1/2 (m < P/2);
+    //      W_{2M}^{k2 + N2 k1} = W_{2M}^{k2 + N2 lane} W_{2M}^{32 N2 m}
+    const float2 wl = tw2(p.tw_2m, p.lo_2m, (uint32_t)k2 + (uint32_t)N2 * (uint32_t)lane);
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
         const float2 *hs = hstage + (b & 1) * (WARPS * 2 * BK);
@@ -384,12 +420,13 @@ __global__ void __launch_bounds__(NT, 2) rowpass_kernel(const FsParams p) {
             const int m = b * MB + mm;
             const int k1 = lane + 32 * m;
             const int pk1 = mode == SELF0 ? ((N1 - k1) & (N1 - 1)) : (N1 - 1 - k1);
-            const uint32_t k = (uint32_t)k2 + (uint32_t)N2 * k1;
             const float2 zk = x[m];
             float2 hk = make_float2(0.f, 0.f), hn = make_float2(0.f, 0.f);
             if constexpr (!SPEC) {
                 hk = hs[(2 * warp + 0) * BK + lane + 32 * mm];
                 hn = hs[(2 * warp + 1) * BK + lane + 32 * mm];
+                hk.x += dk;
+                hn.x += dk;
             }
             if (mode == SELF0 && k1 == 0) {
                 // DC (bin 0) and Nyquist (bin M): both real
@@ -406,7 +443,7 @@ __global__ void __launch_bounds__(NT, 2) rowpass_kernel(const FsParams p) {
             const float2 zn = oth[spad(pk1)];
             const float2 A = make_float2(zk.x + zn.x, zk.y - zn.y);
             const float2 Bv = make_float2(zk.x - zn.x, zk.y + zn.y);
-            const float2 w = tw2(p.tw_2m, p.lo_2m, k);                   // W_{2M}^k
+            const float2 w = cmul(wl, tw2(p.tw_2m, p.lo_2m, 32u * (uint32_t)N2 * (uint32_t)m));   // W_{2M}^k
             const float2 wB = cmul(Bv, w);
             const float2 C = make_float2(wB.y, -wB.x);
             const float2 Xk = cadd(A, C);                                 // 2 X[k]
@@ -443,7 +480,9 @@ __global__ void __launch_bounds__(NT, 2) rowpass_kernel(const FsParams p) {
     // self-paired element of row 0: bin M/2 (k1 = N1/2)
     if (mode == SELF0 && lane == 0) {
         constexpr int mh = (N1 / 2) / 32;
-        const float2 r = cmulc(x[mh], __ldg(H + M / 2));
+        float2 hm = __ldg(H + M / 2);
+        hm.x += dk;
+        const float2 r = cmulc(x[mh], hm);
         x[mh] = make_float2(4.f * r.x, 4.f * r.y);
     }
     __syncthreads();
@@ -457,16 +496,19 @@ __global__ void __launch_bounds__(NT, 2) rowpass_kernel(const FsParams p) {
     // ---- inverse FFT over k1 -> n1, times W_M^{-n1 k2}, back to the buffer
     block_fft<LOG_N1, LP, +1, false, SyncWarp>(x, own, lane, p.tw_n1, SyncWarp{});
     float2 *dst = buf + (int64_t)N1 * k2;
+    const float2 tl = tw2(p.tw_m, p.lo_m, ((uint32_t)k2 * (uint32_t)lane) & (M - 1));
 #pragma unroll
     for (int m = 0; m < P; ++m) {
-        const uint32_t n1 = lane + 32 * m;
-        __stcg(dst + n1, cmulc(x[m], tw2(p.tw_m, p.lo_m, (n1 * (uint32_t)k2) & (M - 1))));
+        const float2 t = cmul(tl, tw2(p.tw_m, p.lo_m, (32u * (uint32_t)k2 * (uint32_t)m) & (M - 1)));
+        __stcg(dst + lane + 32 * m, cmulc(x[m], t));
     }
 }
 
 int64_t chunk_rows_of(int64_t rows, int log_mc) {
-    const int64_t per_row = (int64_t)12 << log_mc;
-    int64_t c = ((int64_t)96 << 20) / per_row;
+    const int64_t per_row = (int64_t)8 << log_mc;
+    int64_t mb = 96;
+    if (const char *e = getenv("HYENA_CHUNK_MB")) mb = atoi(e);
+    int64_t c = (mb << 20) / per_row;
     if (c < 1) c = 1;
     return c < rows ? c : rows;
 }
@@ -486,7 +528,20 @@ hy_status smem_attr(Kern k, size_t bytes) {
         cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
         if (e != cudaSuccess) return set_cuda_error("multi-pass smem attribute", e);
     }
+    // the column passes run three CTAs per SM: all of shared memory is asked for
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return set_cuda_error("multi-pass carveout attribute", e);
     return HY_OK;
+}
+
+// Tensor map of the chunk's complex buffer as a 2-D fp32 array: rows_chunk x
+// N2 rows of 2 N1 floats (row pitch 8 N1 bytes), boxes of 16 floats (8
+// complex columns, 64 bytes) x min(N2, 256) rows, 64-byte swizzle.
+hy_status buf_map(CUtensorMap *m, const float2 *buf, int log_n1, int log_n2, int64_t rows_chunk) {
+    const uint64_t n1 = (uint64_t)1 << log_n1, n2 = (uint64_t)1 << log_n2;
+    return tma_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, buf, 2 * n1, (uint64_t)rows_chunk * n2, 8 * n1, 16,
+                      (uint32_t)(n2 < (uint64_t)kTileBoxRows ? n2 : (uint64_t)kTileBoxRows),
+                      CU_TENSOR_MAP_SWIZZLE_64B, "multi-pass column tiles");
 }
 
 template <int LOG_N1, int LOG_N2, typename IO>
@@ -502,7 +557,6 @@ hy_status run_conv(const LongConvArgs &a, cudaStream_t s) {
     p.u = a.u;
     p.y = a.y;
     p.buf = reinterpret_cast<float2 *>(a.ws);
-    p.stash = reinterpret_cast<float *>(reinterpret_cast<char *>(a.ws) + (size_t)cr * ((size_t)8 << LOG_MC));
     p.scale = (float)(1.0 / (4.0 * (double)((int64_t)1 << LOG_MC)));
     p.vec4 = vec4_rows(a, sizeof(IO));
     p.tw_n1 = tw_stages(LOG_N1, fs_log_p(LOG_N1));
@@ -512,13 +566,16 @@ hy_status run_conv(const LongConvArgs &a, cudaStream_t s) {
     p.lo_2m = (LOG_MC + 1) / 2;
     p.tw_2m = tw_pow2(LOG_MC + 1, p.lo_2m);
     if (!p.tw_n1 || !p.tw_n2 || !p.tw_m || !p.tw_2m) return set_error(HY_ERR_CUDA, "multi-pass twiddle tables missing");
-    const size_t smem_c = sizeof(float2) * WARPS * spad_size(N2);
+    p.fault = device_fault_word();
+    CUtensorMap bmap;
+    hy_status st = buf_map(&bmap, p.buf, LOG_N1, LOG_N2, cr);
+    if (st != HY_OK) return st;
+    const size_t smem_c = colpass_smem_bytes<LOG_N2>();
     const size_t smem_r = rowpass_smem_bytes<LOG_N1, false>();
     auto kA = colpass_kernel<LOG_N1, LOG_N2, IO, false, true, false>;
     auto kCA = colpass_kernel<LOG_N1, LOG_N2, IO, true, true, false>;
     auto kC = colpass_kernel<LOG_N1, LOG_N2, IO, true, false, false>;
     auto kB = rowpass_kernel<LOG_N1, LOG_N2, false>;
-    hy_status st;
     if ((st = smem_attr(kA, smem_c)) != HY_OK || (st = smem_attr(kCA, smem_c)) != HY_OK ||
         (st = smem_attr(kC, smem_c)) != HY_OK || (st = smem_attr(kB, smem_r)) != HY_OK)
         return st;
@@ -527,15 +584,15 @@ hy_status run_conv(const LongConvArgs &a, cudaStream_t s) {
         p.row0 = r0;
         dim3 gc(N1 / WARPS, (unsigned)nr), gr(N2 / 8, (unsigned)nr);
         p.k = 0;
-        kA<<<gc, NT, smem_c, s>>>(p);
+        kA<<<gc, NT, smem_c, s>>>(p, bmap);
         for (int k = 0; k < a.K; ++k) {
             p.k = k;
             p.spec = a.spec[k];
             p.gate_k = a.gate[k];
             p.skip_k = a.skip[k];
             kB<<<gr, NT, smem_r, s>>>(p);
-            if (k + 1 < a.K) kCA<<<gc, NT, smem_c, s>>>(p);
-            else kC<<<gc, NT, smem_c, s>>>(p);
+            if (k + 1 < a.K) kCA<<<gc, NT, smem_c, s>>>(p, bmap);
+            else kC<<<gc, NT, smem_c, s>>>(p, bmap);
         }
         if ((st = check_launch("multi-pass conv launch")) != HY_OK) return st;
     }
@@ -553,7 +610,6 @@ hy_status run_spectrum(int64_t rows, int64_t L, const float *h, float2 *H, void 
     p.K = 1;
     p.u = h;
     p.buf = reinterpret_cast<float2 *>(ws);
-    p.stash = nullptr;
     p.Hout = H;
     p.vec4 = L % 4 == 0 && (uintptr_t)h % 16 == 0;
     p.tw_n1 = tw_stages(LOG_N1, fs_log_p(LOG_N1));
@@ -563,16 +619,19 @@ hy_status run_spectrum(int64_t rows, int64_t L, const float *h, float2 *H, void 
     p.lo_2m = (LOG_MC + 1) / 2;
     p.tw_2m = tw_pow2(LOG_MC + 1, p.lo_2m);
     if (!p.tw_n1 || !p.tw_n2 || !p.tw_m || !p.tw_2m) return set_error(HY_ERR_CUDA, "multi-pass twiddle tables missing");
-    const size_t smem_c = sizeof(float2) * WARPS * spad_size(N2);
+    p.fault = device_fault_word();
+    CUtensorMap bmap;
+    hy_status st = buf_map(&bmap, p.buf, LOG_N1, LOG_N2, cr);
+    if (st != HY_OK) return st;
+    const size_t smem_c = colpass_smem_bytes<LOG_N2>();
     const size_t smem_r = rowpass_smem_bytes<LOG_N1, true>();
     auto kA = colpass_kernel<LOG_N1, LOG_N2, float, false, true, true>;
     auto kB = rowpass_kernel<LOG_N1, LOG_N2, true>;
-    hy_status st;
     if ((st = smem_attr(kA, smem_c)) != HY_OK || (st = smem_attr(kB, smem_r)) != HY_OK) return st;
     for (int64_t r0 = 0; r0 < rows; r0 += cr) {
         const int64_t nr = (rows - r0) < cr ? (rows - r0) : cr;
         p.row0 = r0;
-        kA<<<dim3(N1 / WARPS, (unsigned)nr), NT, smem_c, s>>>(p);
+        kA<<<dim3(N1 / WARPS, (unsigned)nr), NT, smem_c, s>>>(p, bmap);
         kB<<<dim3(N2 / 8, (unsigned)nr), NT, smem_r, s>>>(p);
         if ((st = check_launch("multi-pass spectrum launch")) != HY_OK) return st;
     }
@@ -583,12 +642,12 @@ hy_status run_spectrum(int64_t rows, int64_t L, const float *h, float2 *H, void 
 
 size_t long_conv_workspace(int64_t B, int64_t D, int log_mc, int) {
     if (log_mc < 15 || log_mc > 20) return 0;
-    return (size_t)chunk_rows_of(B * D, log_mc) * ((size_t)12 << log_mc);
+    return (size_t)chunk_rows_of(B * D, log_mc) * ((size_t)8 << log_mc);
 }
 
 size_t long_spectrum_workspace(int64_t rows, int log_mc) {
     if (log_mc < 15 || log_mc > 20) return 0;
-    return (size_t)chunk_rows_of(rows, log_mc) * ((size_t)12 << log_mc);
+    return (size_t)chunk_rows_of(rows, log_mc) * ((size_t)8 << log_mc);
 }
 
 hy_status launch_long_conv(const LongConvArgs &a, cudaStream_t s) {
@@ -660,7 +719,7 @@ hy_status run_conv_static(const LongConvArgs &a, void *scratch, cudaStream_t s) 
     constexpr int N1 = 1 << LOG_N1, N2 = 1 << LOG_N2;
     constexpr int LOG_MC = LOG_N1 + LOG_N2;
     const int64_t rows = a.B * a.D;
-    const size_t per_row = (size_t)12 << LOG_MC;
+    const size_t per_row = (size_t)8 << LOG_MC;
     int64_t cr = (int64_t)(kNoAllocScratchBytes / per_row);
     if (cr < 1)
         return set_error(HY_ERR_WORKSPACE, "hyena_operator_noalloc: one row needs %zu bytes, the static scratch holds %zu",
@@ -673,7 +732,6 @@ hy_status run_conv_static(const LongConvArgs &a, void *scratch, cudaStream_t s) 
     p.u = a.u;
     p.y = a.y;
     p.buf = reinterpret_cast<float2 *>(scratch);
-    p.stash = reinterpret_cast<float *>(reinterpret_cast<char *>(scratch) + (size_t)cr * ((size_t)8 << LOG_MC));
     p.scale = (float)(1.0 / (4.0 * (double)((int64_t)1 << LOG_MC)));
     p.vec4 = vec4_rows(a, sizeof(IO));
     p.tw_n1 = tw_stages(LOG_N1, fs_log_p(LOG_N1));
@@ -683,33 +741,35 @@ hy_status run_conv_static(const LongConvArgs &a, void *scratch, cudaStream_t s) 
     p.lo_2m = (LOG_MC + 1) / 2;
     p.tw_2m = tw_pow2(LOG_MC + 1, p.lo_2m);
     if (!p.tw_n1 || !p.tw_n2 || !p.tw_m || !p.tw_2m) return set_error(HY_ERR_CUDA, "multi-pass twiddle tables missing");
-    const size_t smem_c = sizeof(float2) * WARPS * spad_size(N2);
+    p.fault = device_fault_word();
+    CUtensorMap bmap;
+    hy_status st = buf_map(&bmap, p.buf, LOG_N1, LOG_N2, cr);
+    if (st != HY_OK) return st;
+    const size_t smem_c = colpass_smem_bytes<LOG_N2>();
     const size_t smem_r = rowpass_smem_bytes<LOG_N1, false>();
     auto kA = colpass_kernel<LOG_N1, LOG_N2, IO, false, true, false>;
     auto kCA = colpass_kernel<LOG_N1, LOG_N2, IO, true, true, false>;
     auto kC = colpass_kernel<LOG_N1, LOG_N2, IO, true, false, false>;
     auto kB = rowpass_kernel<LOG_N1, LOG_N2, false>;
-    hy_status st;
     if ((st = smem_attr(kA, smem_c)) != HY_OK || (st = smem_attr(kCA, smem_c)) != HY_OK ||
         (st = smem_attr(kC, smem_c)) != HY_OK || (st = smem_attr(kB, smem_r)) != HY_OK)
         return st;
     // Nothing in the scratch has to start at zero: pass A writes every complex
-    // point of a row before pass B reads it, and the fp32 stash is written by
-    // one order before the next order reads it.
+    // point of a row before pass B reads it.
     for (int64_t r0 = 0; r0 < rows; r0 += cr) {
         const int64_t nr = (rows - r0) < cr ? (rows - r0) : cr;
         p.row0 = r0;
         dim3 gc(N1 / WARPS, (unsigned)nr), gr(N2 / 8, (unsigned)nr);
         p.k = 0;
-        kA<<<gc, NT, smem_c, s>>>(p);
+        kA<<<gc, NT, smem_c, s>>>(p, bmap);
         for (int k = 0; k < a.K; ++k) {
             p.k = k;
             p.spec = a.spec[k];
             p.gate_k = a.gate[k];
             p.skip_k = a.skip[k];
             kB<<<gr, NT, smem_r, s>>>(p);
-            if (k + 1 < a.K) kCA<<<gc, NT, smem_c, s>>>(p);
-            else kC<<<gc, NT, smem_c, s>>>(p);
+            if (k + 1 < a.K) kCA<<<gc, NT, smem_c, s>>>(p, bmap);
+            else kC<<<gc, NT, smem_c, s>>>(p, bmap);
         }
         if ((st = check_launch("no-alloc multi-pass launch")) != HY_OK) return st;
     }

@@ -2,8 +2,8 @@
 // PTX: tensor-memory (TMEM) allocation, shared-memory matrix descriptors,
 // tcgen05.mma of kind::f16 (fp16 or bf16 operands, fp32 accumulator),
 // completion through tcgen05.commit on an mbarrier, tcgen05.ld of the
-// accumulator, and 2-D TMA tensor loads (no multicast; the tensor maps only
-// ever cover this GPU's own memory).
+// accumulator, and 2-D TMA tensor loads and stores (no multicast; the tensor
+// maps only ever cover this GPU's own memory).
 //
 // Conventions (PTX ISA, tcgen05 chapter):
 //   * An accumulator of an M = 128 MMA lives in TMEM lanes 0..127 (lane =
@@ -138,6 +138,18 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         ::"r"(smem_u32(dst)), "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
         : "memory");
 }
+// 2-D TMA tensor store from shared memory (bulk async-group completion).
+// The shared-memory writes it reads must be ordered before it with
+// fence.proxy.async.shared::cta and a CTA barrier.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];"
+                 ::"l"(map), "r"(smem_u32(src)), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until every committed bulk group of this thread has completed (its
+// global writes performed).
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                  : "memory");

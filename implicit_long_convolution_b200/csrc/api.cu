@@ -737,6 +737,18 @@ extern "C" hy_status hyena_operator_backward(int order, int B, int D, int L, hy_
         return set_error(HY_ERR_WORKSPACE, "%s: needs %zu workspace bytes, got %zu", who, lay.total, ws ? ws_bytes : (size_t)0);
     if (!aligned(ws, 256)) return set_error(HY_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", who);
     cudaStream_t s = (cudaStream_t)stream;
+    // order 2 over power-of-two rows that fit on chip: one fused kernel
+    // (both transforms of every row and the batch sums of dh and dD on chip)
+    {
+        const void *p16[5] = {v, x[0], dy, dv, dx[0]};
+        float *dh0 = dh ? dh[0] : nullptr;
+        float *dD0 = dD ? dD[0] : nullptr;
+        if (bw_fused_eligible(order, L, dt, p16, 5) && (!dh0 || aligned(dh0, 8))) {
+            hy_status st = prologue(s);
+            if (st != HY_OK) return st;
+            return launch_bw_fused(B, D, L, dt, v, x[0], dy, H[0], Dskip ? Dskip[0] : nullptr, dv, dx[0], dh0, dD0, s);
+        }
+    }
     char *base = reinterpret_cast<char *>(ws);
     auto buf = [&](size_t off) { return reinterpret_cast<float *>(base + off); };
     float *c[kMaxOrders], *z[kMaxOrders];

@@ -23,6 +23,13 @@ hy_status launch_resident_tc(ResidentParams p, cudaStream_t s);
 bool fft_engine_tensor();
 int device_sm_count();
 
+// Fused backward of the order-2 operator (bw_fused.cu): L a power of two in
+// [512, 8192] whose shared-memory plan fits, the ptrs16 16-byte aligned.
+bool bw_fused_eligible(int order, int L, hy_dtype dt, const void *const *ptrs16, int nptrs);
+hy_status launch_bw_fused(int B, int D, int L, hy_dtype dt, const void *v, const void *x1, const void *dy,
+                          const void *H, const float *Dsk, void *dv, void *dx1, float *dh, float *dD,
+                          cudaStream_t s);
+
 // 2-D TMA tensor map over `outer` rows of `inner` elements (row pitch
 // row_bytes), box box_inner x box_outer, reads past the extent land as zeros
 // (tma_map.cu).  The map covers this GPU's memory only.

@@ -243,7 +243,8 @@ resident_conv_kernel(const ResidentParams p) {
 // buffers next to the FFT exchange buffer), each landing on its own mbarrier;
 // the skip term rides on the spectrum (see split_multiply_merge).  Without
 // PF_GATE (when two stage buffers would not fit) the gate is read from
-// global memory in the epilogue.  Every wait is bounded: a copy that has not
+// global memory in the epilogue (an L2 bulk prefetch of the gate row at the
+// start of the row was measured slower at the 16384-point spectral gate).  Every wait is bounded: a copy that has not
 // landed within the limit records a fault bit, and the CTA stops at the next
 // row boundary (after waiting, again bounded, for its copies in flight).
 // ----------------------------------------------------------------------------

@@ -230,12 +230,20 @@ hy_status spectral_gate_decode(int B, int H, int Dh, int n, hy_dtype dt, int64_t
  *   Inputs as hyena_operator (v, x[k], H[k] = spectra of h_k, Dskip may be
  *   NULL) plus dy (dt, (B, D, L)).  Outputs: dv and dx[k] (dt, (B, D, L));
  *   dh[k] (fp32, (D, L)) and dD[k] (fp32, (D)) -- either array or any entry
- *   may be NULL to skip it.  All arithmetic fp32; the convolutions are the
- *   forward path's (the sums over t >= s are causal convolutions of the
- *   time-reversed e_k).  Deterministic (no atomics).
+ *   may be NULL to skip it.  All arithmetic fp32.  Order 2 with L a power
+ *   of two in [512, 8192] (and v, x, dy, dv, dx 16-byte aligned, dh 8-byte
+ *   aligned) runs one fused kernel: per row both forward transforms, the two
+ *   products and inverse transforms on chip, the sums over t >= s taken as
+ *   correlations (spectra times conjugate spectra), dh and dD summed per
+ *   channel on chip; a channel's rows are shared by at most two CTAs, which
+ *   add their partial sums onto the zeroed dh / dD (two fp32 terms onto zero
+ *   commute, so the result is deterministic).  Otherwise the convolutions
+ *   are the forward path's (the sums over t >= s as causal convolutions of
+ *   the time-reversed e_k) with fp32 intermediates in the workspace;
+ *   deterministic (no atomics).
  *   ws: device workspace of hyena_operator_backward_workspace() bytes,
  *   256-byte aligned (fp32 intermediates: 2K + 4 signals and the per-row
- *   spectra of e_k).
+ *   spectra of e_k; the fused path does not touch it).
  * ---------------------------------------------------------------------- */
 size_t hyena_operator_backward_workspace(int order, int B, int D, int L, hy_dtype dt);
 hy_status hyena_operator_backward(int order, int B, int D, int L, hy_dtype dt, const void *v,

@@ -1,8 +1,9 @@
 """Backward pass of the operator against the float64 oracle (explicit
 adjoint matrices, pinned to finite differences of the direct forward):
-orders 2 and 3, fp32 and bf16 I/O, ragged lengths, with and without the
+orders 2 to 4, fp32 and bf16 I/O, ragged lengths, with and without the
 skip term, gradients of the inputs, the gates, the filters and D; one
-multi-pass length."""
+multi-pass length; the fused order-2 kernel (power-of-two rows) at small
+sizes in full and at the 8192-sample width on sampled indices."""
 import numpy as np
 import pytest
 
@@ -36,6 +37,11 @@ def _spectra(h32):
     (1, 4, 777, 3, "f32", False),
     (3, 2, 2048, 2, "bf16", True),
     (1, 2, 300, 4, "f32", True),
+    # order 2 over power-of-two rows: the fused per-channel kernel
+    (4, 3, 512, 2, "f32", True),
+    (2, 3, 1024, 2, "bf16", False),
+    (5, 2, 2048, 2, "f32", True),
+    (1, 1, 4096, 2, "f32", True),
 ])
 def test_backward_vs_oracle(B, D, L, order, dtype, skip):
     K = order - 1
@@ -124,3 +130,104 @@ def test_backward_multipass_length_sampled():
     check_part(gdx[..., ts], sx, rms(gdx), "f32", "dx L=20000")
     check_part(gdh[:, ts], sh, rms(gdh), "f32", "dh L=20000")
     check(to_np(dD[0]), sD, "f32", "dD L=20000")
+
+
+def test_backward_fused_width_8192_sampled():
+    """Order 2, bf16, L = 8192 (the fused kernel at the widest row it takes,
+    with eight samples per channel summed into dh and dD): direct sums at 40
+    indices and lags of every row, dD in full."""
+    from _helpers import check_part
+    B, D, L = 8, 6, 8192
+    rng = np.random.default_rng(11)
+    t = np.arange(L)
+    h = (rng.standard_normal((1, D, L)) * np.exp(-rng.uniform(0.5, 3.0, (1, D, 1)) * t / L)).astype(np.float32)
+    Dk = rng.standard_normal((1, D)).astype(np.float32)
+    sig = lambda: hw.Signal(rng.standard_normal((B, D, L)).astype(np.float32))
+    v, x1, dy = sig(), sig(), sig()
+    for s_ in (v, x1, dy):
+        s_.bf16 = hw.bf16_round(s_.f32)
+        s_.f32 = hw.bf16_to_f32(s_.bf16)
+    Hs = _spectra(h)
+    vd, xd, dyd = (to_dev(a, "bf16") for a in (v, x1, dy))
+    dv = torch.empty_like(vd)
+    dx = [torch.empty_like(vd)]
+    dh = [torch.empty((D, L), device="cuda")]
+    dD = [torch.empty(D, device="cuda")]
+    ws = torch.empty(hy.operator_backward_workspace(2, B, D, L, hy.HY_BF16), dtype=torch.uint8, device="cuda")
+    hy.hyena_operator_backward(vd, [xd], Hs, dyd, dv, dx, Dskips=[f32_dev(Dk[0])], dhs=dh, dDs=dD, ws=ws)
+    torch.cuda.synchronize()
+    ts = np.unique(np.concatenate([[0, 1, L // 2, L - 2, L - 1], rng.choice(L, 35, replace=False)]))
+    sv, sx, sh, sD = oracle.hyena_backward_samples(v.f32, x1.f32, h[0], Dk[0], dy.f32, ts)
+    gdv, gdx, gdh = to_np(dv), to_np(dx[0]), to_np(dh[0])
+    rms = lambda a: float(np.sqrt(np.mean(a.astype(np.float64) ** 2)))
+    check_part(gdv[..., ts], sv, rms(gdv), "bf16", "dv L=8192")
+    check_part(gdx[..., ts], sx, rms(gdx), "bf16", "dx L=8192")
+    check_part(gdh[:, ts], sh, rms(gdh), "f32", "dh L=8192")
+    check(to_np(dD[0]), sD, "f32", "dD L=8192")
+
+
+def test_backward_fused_optional_outputs_and_reuse():
+    """Order 2 on the fused kernel: dh and dD may each be omitted without
+    changing dv and dx, a repeated call is bit-identical (no atomics), and
+    with dh alone its lag-0 value is dD."""
+    B, D, L = 3, 4, 1024
+    rng = np.random.default_rng(5)
+    h = (rng.standard_normal((1, D, L)) * 0.05).astype(np.float32)
+    Hs = _spectra(h)
+    v, x1, dy = (f32_dev(rng.standard_normal((B, D, L)).astype(np.float32)) for _ in range(3))
+    Dk = [f32_dev(rng.standard_normal(D).astype(np.float32))]
+    ws = torch.empty(hy.operator_backward_workspace(2, B, D, L, hy.HY_F32), dtype=torch.uint8, device="cuda")
+    outs = []
+    for extra in ({"dhs": [torch.empty((D, L), device="cuda")], "dDs": [torch.empty(D, device="cuda")]},
+                  {"dhs": [torch.empty((D, L), device="cuda")]}, {"dDs": [torch.empty(D, device="cuda")]}, {},
+                  {"dhs": [torch.empty((D, L), device="cuda")], "dDs": [torch.empty(D, device="cuda")]}):
+        dv = torch.empty_like(v)
+        dx = [torch.empty_like(v)]
+        hy.hyena_operator_backward(v, [x1], Hs, dy, dv, dx, Dskips=Dk, ws=ws, **extra)
+        torch.cuda.synchronize()
+        outs.append((dv.clone(), dx[0].clone(), extra))
+    for dv, dx, _ in outs[1:]:
+        assert torch.equal(dv, outs[0][0]) and torch.equal(dx, outs[0][1])
+    a, b = outs[0][2], outs[4][2]
+    assert torch.equal(a["dhs"][0], b["dhs"][0]) and torch.equal(a["dDs"][0], b["dDs"][0])
+    assert torch.equal(outs[1][2]["dhs"][0], a["dhs"][0])
+    assert torch.equal(outs[2][2]["dDs"][0], a["dDs"][0])
+    lag0 = to_np(a["dhs"][0])[:, 0].astype(np.float64)
+    dd = to_np(a["dDs"][0]).astype(np.float64)
+    assert np.max(np.abs(lag0 - dd)) <= 1e-4 * np.sqrt(np.mean(dd ** 2))
+
+
+def test_backward_fused_channels_shared_by_two_ctas():
+    """Order 2, fp32, L = 8192 with more channels than CTAs (600 rows over
+    the SMs): a channel's rows are split between two CTAs whose partial dh and
+    dD meet in the output; checked against direct sums at sampled indices and
+    lags of every channel, dD in full, and a repeated call bit for bit."""
+    from _helpers import check_part
+    B, D, L = 3, 200, 8192
+    rng = np.random.default_rng(21)
+    t = np.arange(L)
+    h = (rng.standard_normal((1, D, L)) * np.exp(-rng.uniform(0.5, 3.0, (1, D, 1)) * t / L)).astype(np.float32)
+    Dk = rng.standard_normal((1, D)).astype(np.float32)
+    v, x1, dy = (rng.standard_normal((B, D, L)).astype(np.float32) for _ in range(3))
+    Hs = _spectra(h)
+    ws = torch.empty(hy.operator_backward_workspace(2, B, D, L, hy.HY_F32), dtype=torch.uint8, device="cuda")
+    res = []
+    for _ in range(2):
+        dv = torch.empty((B, D, L), device="cuda")
+        dx = [torch.empty_like(dv)]
+        dh = [torch.empty((D, L), device="cuda")]
+        dD = [torch.empty(D, device="cuda")]
+        hy.hyena_operator_backward(f32_dev(v), [f32_dev(x1)], Hs, f32_dev(dy), dv, dx, Dskips=[f32_dev(Dk[0])],
+                                   dhs=dh, dDs=dD, ws=ws)
+        torch.cuda.synchronize()
+        res.append((dv, dx[0], dh[0], dD[0]))
+    for a, b in zip(res[0], res[1]):
+        assert torch.equal(a, b)
+    ts = np.unique(np.concatenate([[0, 1, L - 1], rng.choice(L, 9, replace=False)]))
+    sv, sx, sh, sD = oracle.hyena_backward_samples(v, x1, h[0], Dk[0], dy, ts)
+    gdv, gdx, gdh = (to_np(a) for a in res[0][:3])
+    rms = lambda a: float(np.sqrt(np.mean(a.astype(np.float64) ** 2)))
+    check_part(gdv[..., ts], sv, rms(gdv), "f32", "dv")
+    check_part(gdx[..., ts], sx, rms(gdx), "f32", "dx")
+    check_part(gdh[:, ts], sh, rms(gdh), "f32", "dh")
+    check(to_np(res[0][3]), sD, "f32", "dD")

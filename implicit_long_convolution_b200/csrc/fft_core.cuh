@@ -115,39 +115,43 @@ __host__ __device__ constexpr int plan_tw_total(int log_m, int log_p) {
     return plan_tw_offset(log_m, log_p, plan_stages(log_m, log_p));
 }
 
-// Shared-memory slot of complex element e: one pad slot every 32 elements
-// keeps the stride-R writes of the first stage conflict-free.
-__device__ __forceinline__ int spad(int e) { return e + (e >> 5); }
+// Shared-memory slot of complex element e: one pad slot every 2^SH elements
+// keeps the stride-R writes of the first stage conflict-free.  SH = 5 (a pad
+// every 32) is the default of the row kernels, whose FFTs span whole warps;
+// FFTs of 8 or 16 threads (several per warp) take SH = 3 or 4.
+template <int SH>
+__device__ __forceinline__ int spadx(int e) { return e + (e >> SH); }
+__device__ __forceinline__ int spad(int e) { return spadx<5>(e); }
 __host__ __device__ constexpr int spad_size(int m) { return m + (m >> 5) + 1; }
 
 // x[m] = element t + m*T of a padded shared buffer (linear addressing when
-// T is a multiple of 32).
-template <int LOG_M, int LOG_P>
+// T is a multiple of 2^SH).
+template <int LOG_M, int LOG_P, int SH = 5>
 __device__ __forceinline__ void load_own(float2 (&x)[1 << LOG_P], const float2 *sbuf, int t) {
     constexpr int P = 1 << LOG_P;
     constexpr int T = (1 << LOG_M) / P;
-    if constexpr (T % 32 == 0) {
-        const float2 *src = sbuf + spad(t);
-        constexpr int STEP = T + T / 32;
+    if constexpr (T % (1 << SH) == 0) {
+        const float2 *src = sbuf + spadx<SH>(t);
+        constexpr int STEP = T + (T >> SH);
 #pragma unroll
         for (int m = 0; m < P; ++m) x[m] = src[m * STEP];
     } else {
 #pragma unroll
-        for (int m = 0; m < P; ++m) x[m] = sbuf[spad(t + m * T)];
+        for (int m = 0; m < P; ++m) x[m] = sbuf[spadx<SH>(t + m * T)];
     }
 }
-template <int LOG_M, int LOG_P>
+template <int LOG_M, int LOG_P, int SH = 5>
 __device__ __forceinline__ void store_own(const float2 (&x)[1 << LOG_P], float2 *sbuf, int t) {
     constexpr int P = 1 << LOG_P;
     constexpr int T = (1 << LOG_M) / P;
-    if constexpr (T % 32 == 0) {
-        float2 *dst = sbuf + spad(t);
-        constexpr int STEP = T + T / 32;
+    if constexpr (T % (1 << SH) == 0) {
+        float2 *dst = sbuf + spadx<SH>(t);
+        constexpr int STEP = T + (T >> SH);
 #pragma unroll
         for (int m = 0; m < P; ++m) dst[m * STEP] = x[m];
     } else {
 #pragma unroll
-        for (int m = 0; m < P; ++m) sbuf[spad(t + m * T)] = x[m];
+        for (int m = 0; m < P; ++m) sbuf[spadx<SH>(t + m * T)] = x[m];
     }
 }
 // Padded slot of the thread's own element t + m*T.
@@ -201,7 +205,7 @@ __device__ __forceinline__ void wide_last_stage(float2 (&x)[P], float2 (&y)[NB][
 // in registers (natural order); otherwise written to sbuf and read back.
 // tw: this stage's table, layout [(r-1) * p + k] = W_{pR}^{k r} (forward).
 // ----------------------------------------------------------------------------
-template <int LOG_M, int LOG_P, int S, int DIR, bool UPPER_ZERO, typename Sync>
+template <int LOG_M, int LOG_P, int S, int DIR, bool UPPER_ZERO, typename Sync, int SH = 5>
 __device__ __forceinline__ void fft_stage(float2 (&x)[1 << LOG_P], float2 *sbuf, int t,
                                           const float2 *__restrict__ tw, Sync sync) {
     constexpr int M = 1 << LOG_M;
@@ -247,40 +251,41 @@ __device__ __forceinline__ void fft_stage(float2 (&x)[1 << LOG_P], float2 *sbuf,
             const int i = t + q * T;
             const int k = i & (PS - 1);
             const int base = (i - k) * R + k;
-            if constexpr (PS % 32 == 0 || (PS == 1 && R <= 32)) {
+            if constexpr (PS % (1 << SH) == 0 || (PS == 1 && R <= (1 << SH))) {
                 // padded address is linear in r here: one base, constant steps
-                float2 *dst = sbuf + spad(base);
-                constexpr int STEP = PS + PS / 32;
+                float2 *dst = sbuf + spadx<SH>(base);
+                constexpr int STEP = PS + (PS >> SH);
 #pragma unroll
                 for (int r = 0; r < R; ++r) dst[r * STEP] = y[q][bitrev(r, LR)];
             } else {
 #pragma unroll
-                for (int r = 0; r < R; ++r) sbuf[spad(base + r * PS)] = y[q][bitrev(r, LR)];
+                for (int r = 0; r < R; ++r) sbuf[spadx<SH>(base + r * PS)] = y[q][bitrev(r, LR)];
             }
         }
         sync();
-        load_own<LOG_M, LOG_P>(x, sbuf, t);
+        load_own<LOG_M, LOG_P, SH>(x, sbuf, t);
         sync();
     }
 }
 
-template <int LOG_M, int LOG_P, int S, int DIR, bool UPPER_ZERO, typename Sync>
+template <int LOG_M, int LOG_P, int S, int DIR, bool UPPER_ZERO, typename Sync, int SH>
 __device__ __forceinline__ void fft_stages_from(float2 (&x)[1 << LOG_P], float2 *sbuf, int t,
                                                 const float2 *__restrict__ tw, Sync sync) {
     constexpr int NS = plan_stages(LOG_M, LOG_P);
     if constexpr (S < NS) {
-        fft_stage<LOG_M, LOG_P, S, DIR, (S == 0) && UPPER_ZERO>(x, sbuf, t, tw + plan_tw_offset(LOG_M, LOG_P, S), sync);
-        fft_stages_from<LOG_M, LOG_P, S + 1, DIR, UPPER_ZERO>(x, sbuf, t, tw, sync);
+        fft_stage<LOG_M, LOG_P, S, DIR, (S == 0) && UPPER_ZERO, Sync, SH>(x, sbuf, t,
+                                                                           tw + plan_tw_offset(LOG_M, LOG_P, S), sync);
+        fft_stages_from<LOG_M, LOG_P, S + 1, DIR, UPPER_ZERO, Sync, SH>(x, sbuf, t, tw, sync);
     }
 }
 
 // Full complex FFT of size 2^LOG_M (unnormalised).  DIR = -1: forward
 // (e^{-2πi/M}); +1: inverse.  UPPER_ZERO: elements M/2..M-1 of the input are
-// zero (zero-padded rows) and are not read.
-template <int LOG_M, int LOG_P, int DIR, bool UPPER_ZERO = false, typename Sync = SyncBlock>
+// zero (zero-padded rows) and are not read.  SH: the padding of sbuf (spadx).
+template <int LOG_M, int LOG_P, int DIR, bool UPPER_ZERO = false, typename Sync = SyncBlock, int SH = 5>
 __device__ __forceinline__ void block_fft(float2 (&x)[1 << LOG_P], float2 *sbuf, int t,
                                           const float2 *__restrict__ tw, Sync sync = Sync{}) {
-    fft_stages_from<LOG_M, LOG_P, 0, DIR, UPPER_ZERO>(x, sbuf, t, tw, sync);
+    fft_stages_from<LOG_M, LOG_P, 0, DIR, UPPER_ZERO, Sync, SH>(x, sbuf, t, tw, sync);
 }
 
 }  // namespace hy

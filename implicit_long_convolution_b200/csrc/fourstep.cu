@@ -34,7 +34,6 @@
 // registers or instructions on the strided transfer and three CTAs fit on an
 // SM.  Rows are processed in chunks whose intermediates (8 bytes per complex
 // point) stay resident in the 126 MB L2 between passes.
-#include <cstdlib>
 #include <mutex>
 
 #include "../../include/hyena.h"
@@ -504,11 +503,13 @@ __global__ void __launch_bounds__(NT, 2) rowpass_kernel(const FsParams p) {
     }
 }
 
+// Rows per chunk: the complex buffer of a chunk (8 bytes per point) is kept
+// near 96 MB.  At M = 2^20, 64 and 96 MB chunks measured the same and 32 MB
+// ones slower, although only the smaller chunks keep the buffer in L2 between
+// passes: the passes are latency-bound, and short launches lose to their tail.
 int64_t chunk_rows_of(int64_t rows, int log_mc) {
     const int64_t per_row = (int64_t)8 << log_mc;
-    int64_t mb = 96;
-    if (const char *e = getenv("HYENA_CHUNK_MB")) mb = atoi(e);
-    int64_t c = (mb << 20) / per_row;
+    int64_t c = ((int64_t)96 << 20) / per_row;
     if (c < 1) c = 1;
     return c < rows ? c : rows;
 }

@@ -56,6 +56,10 @@ __device__ __forceinline__ float2 wsplit(const float2 *tab, int k, int half) {
 }
 
 // One small FFT per group of T = N/P threads; group g, lane t within group.
+// Its exchange buffer pads one slot every 2^SH elements and groups follow
+// each other every N + N/2^SH slots: with several groups in a warp this makes
+// the stride-8 writes of the first stage and the reads back conflict-free
+// (up to 64 points) or nearly so (128).
 template <int LOG_N>
 struct Grp {
     static constexpr int N = 1 << LOG_N;
@@ -63,6 +67,8 @@ struct Grp {
     static constexpr int P = 1 << LP;
     static constexpr int T = N / P;
     static constexpr int G = NT / T;
+    static constexpr int SH = LOG_N <= 6 ? 3 : 4;
+    static constexpr int BUF = N + (N >> SH);       // exchange buffer of a group
 };
 
 // ---------------------------------------------------------------------------
@@ -89,7 +95,7 @@ __global__ void __launch_bounds__(NT) nd_fwd_plane(const NdParams p) {
     // ---- row pass: real FFT along z of rows j < gI
     {
         const int g = tid / R::T, t = tid % R::T;
-        float2 *xb = gbuf + g * spad_size(R::N);
+        float2 *xb = gbuf + g * R::BUF;
         // the next round's row is requested before this round's FFT
         auto load_row = [&](int j, float2 (&v)[R::P]) {
 #pragma unroll
@@ -108,15 +114,15 @@ __global__ void __launch_bounds__(NT) nd_fwd_plane(const NdParams p) {
 #pragma unroll
             for (int m = 0; m < R::P; ++m) x[m] = xn[m];
             if (j0 + R::G < gI) load_row(j + R::G, xn);
-            block_fft<LOG_S - 1, R::LP, -1, PAD, SyncWarp>(x, xb, t, p.tw_r, SyncWarp{});
-            store_own<LOG_S - 1, R::LP>(x, xb, t);
+            block_fft<LOG_S - 1, R::LP, -1, PAD, SyncWarp, R::SH>(x, xb, t, p.tw_r, SyncWarp{});
+            store_own<LOG_S - 1, R::LP, R::SH>(x, xb, t);
             __syncwarp();
             // split: bins k = t + m*T (k < H2) and the Nyquist bin H2
 #pragma unroll
             for (int m = 0; m < R::P; ++m) {
                 const int k = t + m * R::T;
                 const float2 zk = x[m];
-                const float2 zn = xb[spad((H2 - k) & (H2 - 1))];
+                const float2 zn = xb[spadx<R::SH>((H2 - k) & (H2 - 1))];
                 const float2 A = make_float2(zk.x + zn.x, zk.y - zn.y);
                 const float2 Bv = make_float2(zk.x - zn.x, zk.y + zn.y);
                 const float2 wB = cmul(Bv, wsplit(p.tw_split, k, H2));
@@ -131,7 +137,7 @@ __global__ void __launch_bounds__(NT) nd_fwd_plane(const NdParams p) {
     // ---- column pass: FFT along y of each bin column (inputs j < gI)
     {
         const int g = tid / C::T, t = tid % C::T;
-        float2 *xb = gbuf + g * spad_size(C::N);
+        float2 *xb = gbuf + g * C::BUF;
         for (int k0 = 0; k0 < NB; k0 += C::G) {
             const int k = k0 + g;
             const bool act = k < NB;
@@ -141,7 +147,7 @@ __global__ void __launch_bounds__(NT) nd_fwd_plane(const NdParams p) {
                 const int j = t + m * C::T;
                 x[m] = (act && j < gI) ? tile[j * NB + k] : make_float2(0.f, 0.f);
             }
-            block_fft<LOG_S, C::LP, -1, PAD, SyncWarp>(x, xb, t, p.tw_c, SyncWarp{});
+            block_fft<LOG_S, C::LP, -1, PAD, SyncWarp, C::SH>(x, xb, t, p.tw_c, SyncWarp{});
             __syncwarp();
             if (act) {
 #pragma unroll
@@ -189,7 +195,7 @@ __global__ void __launch_bounds__(NT) nd_xpass(const NdParams p) {
     extern __shared__ float2 sm[];
     float2 *tile = sm;                                  // gI rows (x) x NB
     float2 *gbuf = sm + gI * NB;
-    float2 *hst = gbuf + NT / C::T * spad_size(C::N);   // conv: 2 x [S][HS]
+    float2 *hst = gbuf + NT / C::T * C::BUF;   // conv: 2 x [S][HS]
     const int tid = threadIdx.x;
     const int64_t sl = blockIdx.y;                      // slab within chunk
     const int64_t slab = p.slab0 + sl;
@@ -216,7 +222,7 @@ __global__ void __launch_bounds__(NT) nd_xpass(const NdParams p) {
     nd_wait<0>();
     __syncthreads();
     const int g = tid / C::T, t = tid % C::T;
-    float2 *xb = gbuf + g * spad_size(C::N);
+    float2 *xb = gbuf + g * C::BUF;
 #pragma unroll 1
     for (int r = 0; r < NR; ++r) {
         const int k = r * G + g;
@@ -237,7 +243,7 @@ __global__ void __launch_bounds__(NT) nd_xpass(const NdParams p) {
             const int ii = t + m * C::T;
             x[m] = (act && ii < gI) ? tile[ii * NB + k] : make_float2(0.f, 0.f);
         }
-        block_fft<LOG_S, C::LP, -1, PAD, SyncWarp>(x, xb, t, p.tw_c, SyncWarp{});
+        block_fft<LOG_S, C::LP, -1, PAD, SyncWarp, C::SH>(x, xb, t, p.tw_c, SyncWarp{});
         if constexpr (SPEC) {
             // back into column k of the tile (gI = S here); the z split
             // carries a factor 2 (folded into the conv scale)
@@ -257,7 +263,7 @@ __global__ void __launch_bounds__(NT) nd_xpass(const NdParams p) {
                 x[m] = cmul(x[m], act ? hb[kx * HS] : make_float2(0.f, 0.f));
             }
             __syncwarp();
-            block_fft<LOG_S, C::LP, +1, false, SyncWarp>(x, xb, t, p.tw_c, SyncWarp{});
+            block_fft<LOG_S, C::LP, +1, false, SyncWarp, C::SH>(x, xb, t, p.tw_c, SyncWarp{});
             __syncwarp();
             if (act) {
 #pragma unroll
@@ -310,14 +316,14 @@ __global__ void __launch_bounds__(NT) nd_inv_plane(const NdParams p) {
     // ---- inverse along y (k1 -> j), keep j < gI
     {
         const int g = tid / C::T, t = tid % C::T;
-        float2 *xb = gbuf + g * spad_size(C::N);
+        float2 *xb = gbuf + g * C::BUF;
         for (int k0 = 0; k0 < NB; k0 += C::G) {
             const int k = k0 + g;
             const bool act = k < NB;
             float2 x[C::P];
 #pragma unroll
             for (int m = 0; m < C::P; ++m) x[m] = act ? tile[(t + m * C::T) * NB + k] : make_float2(0.f, 0.f);
-            block_fft<LOG_S, C::LP, +1, false, SyncWarp>(x, xb, t, p.tw_c, SyncWarp{});
+            block_fft<LOG_S, C::LP, +1, false, SyncWarp, C::SH>(x, xb, t, p.tw_c, SyncWarp{});
             __syncwarp();
             if (act) {
 #pragma unroll
@@ -335,7 +341,7 @@ __global__ void __launch_bounds__(NT) nd_inv_plane(const NdParams p) {
     const int64_t pbase = (slab * gI + i) * (int64_t)gI * gI;
     {
         const int g = tid / R::T, t = tid % R::T;
-        float2 *xb = gbuf + g * spad_size(R::N);
+        float2 *xb = gbuf + g * R::BUF;
         for (int j0 = 0; j0 < gI; j0 += R::G) {
             const int j = j0 + g;
             const bool act = j < gI;
@@ -364,7 +370,7 @@ __global__ void __launch_bounds__(NT) nd_inv_plane(const NdParams p) {
                 const float2 cB = cmulc(Bv, wsplit(p.tw_split, k, H2));     // W^-k B
                 x[m] = make_float2(A.x - cB.y, A.y + cB.x);                // A + i W^-k B
             }
-            block_fft<LOG_S - 1, R::LP, +1, false, SyncWarp>(x, xb, t, p.tw_r, SyncWarp{});
+            block_fft<LOG_S - 1, R::LP, +1, false, SyncWarp, R::SH>(x, xb, t, p.tw_r, SyncWarp{});
             if (act) {
 #pragma unroll
                 for (int m = 0; m < R::P; ++m) {
@@ -406,10 +412,10 @@ hy_status nd_smem(Kern k, size_t bytes) {
 
 template <int LOG_S>
 size_t gbuf_elems() {
-    return (size_t)NT / Grp<LOG_S>::T * spad_size(Grp<LOG_S>::N) >
-                   (size_t)NT / Grp<LOG_S - 1>::T * spad_size(Grp<LOG_S - 1>::N)
-               ? (size_t)NT / Grp<LOG_S>::T * spad_size(Grp<LOG_S>::N)
-               : (size_t)NT / Grp<LOG_S - 1>::T * spad_size(Grp<LOG_S - 1>::N);
+    return (size_t)NT / Grp<LOG_S>::T * Grp<LOG_S>::BUF >
+                   (size_t)NT / Grp<LOG_S - 1>::T * Grp<LOG_S - 1>::BUF
+               ? (size_t)NT / Grp<LOG_S>::T * Grp<LOG_S>::BUF
+               : (size_t)NT / Grp<LOG_S - 1>::T * Grp<LOG_S - 1>::BUF;
 }
 
 template <int LOG_S, bool PAD>
@@ -424,7 +430,7 @@ hy_status run_nd(const NDArgs &a, NdParams p, cudaStream_t s, bool spec, int64_t
     const int64_t per_slab = (int64_t)gI * S * NB * 8;
     const int64_t cs = nd_chunk(slabs, per_slab);
     const size_t sm1 = sizeof(float2) * ((size_t)S * NB + gbuf_elems<LOG_S>());
-    const size_t sm2 = sizeof(float2) * ((size_t)gI * NB + (size_t)NT / Grp<LOG_S>::T * spad_size(Grp<LOG_S>::N));
+    const size_t sm2 = sizeof(float2) * ((size_t)gI * NB + (size_t)NT / Grp<LOG_S>::T * Grp<LOG_S>::BUF);
     const size_t sm2c = sm2 + sizeof(float2) * 2 * (size_t)S * xpass_hstride<LOG_S>();
     auto k1 = nd_fwd_plane<LOG_S, PAD>;
     auto k2c = nd_xpass<LOG_S, PAD, false>;

@@ -313,6 +313,12 @@ __global__ void __launch_bounds__(NT, 3) colpass_kernel(const FsParams p, const 
 enum { PAIR = 0, SELF0 = 1, SELFH = 2 };
 
 __host__ __device__ constexpr int rp_batches(int log_n1) { return (1 << log_n1) / 64 >= 4 ? 4 : (1 << log_n1) / 64; }
+// Staging rows are BK + 2 complex apart: the four lanes that copy the bins of
+// four neighbouring rows at one k1 then land 8 banks apart instead of on
+// one bank (the cp.async writes were 96% of the pass's bank conflicts).
+__host__ __device__ constexpr int rp_stage_stride(int log_n1) {
+    return (1 << log_n1) / 2 / rp_batches(log_n1) + 2;
+}
 
 __device__ __forceinline__ void cpa8(void *smem, const void *g) {
     const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
@@ -324,9 +330,9 @@ __device__ __forceinline__ void cpa_wait() { asm volatile("cp.async.wait_group %
 
 template <int LOG_N1, bool SPEC>
 __host__ __device__ constexpr size_t rowpass_smem_bytes() {
-    // row buffers, then (conv) two staging buffers of [8 rows][k, M-k][N1/2 / batches]
+    // row buffers, then (conv) two staging buffers of [8 rows][k, M-k][N1/2 / batches + 2]
     return sizeof(float2) * ((size_t)WARPS * spad_size(1 << LOG_N1) +
-                             (SPEC ? 0 : (size_t)2 * WARPS * 2 * ((1 << LOG_N1) / 2 / rp_batches(LOG_N1))));
+                             (SPEC ? 0 : (size_t)2 * WARPS * 2 * rp_stage_stride(LOG_N1)));
 }
 
 template <int LOG_N1, int LOG_N2, bool SPEC>
@@ -340,9 +346,10 @@ __global__ void __launch_bounds__(NT, 2) rowpass_kernel(const FsParams p) {
     constexpr int NB = rp_batches(LOG_N1);    // staging batches over the owned k1 < N1/2
     constexpr int MB = P / 2 / NB;            // m values per batch
     constexpr int BK = 32 * MB;               // k1 values per batch
+    constexpr int HS = rp_stage_stride(LOG_N1);   // staging row stride (BK + 2)
     static_assert(NB >= 1 && MB >= 1 && MB * NB * 2 == P, "row pass batching");
     extern __shared__ float2 rows_s[];        // WARPS rows x RS, then the staging buffers
-    float2 *hstage = rows_s + WARPS * RS;     // [2 buffers][8 rows][k, M-k][BK]
+    float2 *hstage = rows_s + WARPS * RS;     // [2 buffers][8 rows][k, M-k][HS]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = blockIdx.x;
     const int64_t row = p.row0 + blockIdx.y;
@@ -376,10 +383,10 @@ __global__ void __launch_bounds__(NT, 2) rowpass_kernel(const FsParams p) {
             const int kk = skk + i * (NT / 4);
             if (kk < BK) {
                 const uint32_t off = (uint32_t)N2 * (uint32_t)(b * BK + i * (NT / 4));
-                cpa8(dst + (2 * sj + 0) * BK + kk, H + (k_lo + off));
-                cpa8(dst + (2 * sj + 1) * BK + kk, H + (M - (k_lo + off)));
-                cpa8(dst + (2 * (4 + sj) + 0) * BK + kk, H + (k_hi + off));
-                cpa8(dst + (2 * (4 + sj) + 1) * BK + kk, H + (M - (k_hi + off)));
+                cpa8(dst + (2 * sj + 0) * HS + kk, H + (k_lo + off));
+                cpa8(dst + (2 * sj + 1) * HS + kk, H + (M - (k_lo + off)));
+                cpa8(dst + (2 * (4 + sj) + 0) * HS + kk, H + (k_hi + off));
+                cpa8(dst + (2 * (4 + sj) + 1) * HS + kk, H + (M - (k_hi + off)));
             }
         }
     };
@@ -403,10 +410,10 @@ __global__ void __launch_bounds__(NT, 2) rowpass_kernel(const FsParams p) {
     const float2 wl = tw2(p.tw_2m, p.lo_2m, (uint32_t)k2 + (uint32_t)N2 * (uint32_t)lane);
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
-        const float2 *hs = hstage + (b & 1) * (WARPS * 2 * BK);
+        const float2 *hs = hstage + (b & 1) * (WARPS * 2 * HS);
         if constexpr (!SPEC) {
             if (b + 1 < NB) {
-                stage(b + 1, hstage + ((b + 1) & 1) * (WARPS * 2 * BK));
+                stage(b + 1, hstage + ((b + 1) & 1) * (WARPS * 2 * HS));
                 cpa_commit();
                 cpa_wait<1>();
             } else {
@@ -422,8 +429,8 @@ __global__ void __launch_bounds__(NT, 2) rowpass_kernel(const FsParams p) {
             const float2 zk = x[m];
             float2 hk = make_float2(0.f, 0.f), hn = make_float2(0.f, 0.f);
             if constexpr (!SPEC) {
-                hk = hs[(2 * warp + 0) * BK + lane + 32 * mm];
-                hn = hs[(2 * warp + 1) * BK + lane + 32 * mm];
+                hk = hs[(2 * warp + 0) * HS + lane + 32 * mm];
+                hn = hs[(2 * warp + 1) * HS + lane + 32 * mm];
                 hk.x += dk;
                 hn.x += dk;
             }

@@ -19,7 +19,9 @@
 // copied with cp.async while the current one is computed (two buffers).
 // Hidden outputs get bias, FiLM and the activation and stay in shared
 // memory; last-layer outputs get bias and the decay window and go straight
-// to HBM as float4 row segments.
+// to HBM as float4 row segments.  With many positions per filter set the
+// weights stay resident in persistent CTAs, and the last layer runs on the
+// tensor cores (filter_gen_tc_kernel) where its shape allows.
 #include <cuda_fp16.h>
 #include <cstdlib>
 #include <cstring>
@@ -66,11 +68,11 @@ struct GenParams {
     int r_w[MAXL], r_ws[MAXL];  // wT_l[k][o] at r_w[l] + k * r_ws[l] + o
     int r_b[MAXL], r_om[MAXL];  // biases, sine frequencies (or -1)
     int r_g, r_be, r_al;        // FiLM gamma / beta of the CTA's set (or -1), decay rates
-    // tensor-core last layer (resident kernel): operands after the resident region
+    // tensor-core last layer: operands after the resident region
     int t_kpad;                 // last-layer K rounded up to 16
     int t_katoms;               // 64-element K atoms
-    int t_nmt;                  // 128-output M tiles
-    uint32_t t_cols;            // TMEM columns (64 per M tile, power of two >= 32)
+    int t_npad;                 // outputs rounded up to 16 (MMA N, in chunks of <= 256)
+    uint32_t t_cols;            // TMEM columns (power of two >= max(32, t_npad))
     uint32_t *fault;            // device fault word
 };
 
@@ -369,19 +371,6 @@ __global__ void __launch_bounds__(NT, 2) filter_gen_kernel(const GenParams p) {
     }
 }
 
-// ---- tensor-core last layer: fp16 hi/lo operands in the K-major
-// 128-byte-swizzled layout (64 K elements per 128-byte row, 8-row atoms)
-constexpr int TC_A_ATOM = 128 * 128;   // bytes of one K atom of a 128-row A tile
-constexpr int TC_B_ATOM = P * 128;     // bytes of one K atom of the 64-row B tile
-
-__device__ __forceinline__ uint32_t fg_sw128(int r, int k) {
-    return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((((k & 63) >> 3) ^ (r & 7)) << 4) + (k & 7) * 2);
-}
-__device__ __forceinline__ void fp16_split(float x, __half &hi, __half &lo) {
-    hi = __float2half_rn(x);
-    lo = __float2half_rn(x - __half2float(hi));
-}
-
 // ----------------------------------------------------------------------------
 // Resident-weight variant, for many position tiles per filter set: every
 // layer's weights (transposed: wT_l[k][o]) and per-output parameters (bias,
@@ -390,57 +379,18 @@ __device__ __forceinline__ void fp16_split(float x, __half &hi, __half &lo) {
 // blockIdx.x + gridDim.x, ... of set blockIdx.y.  The arithmetic per tile is
 // the streaming kernel's (same tile GEMMs, same epilogues).
 // ----------------------------------------------------------------------------
-template <bool TC>
-__global__ void __launch_bounds__(NT, 2) filter_gen_resident_kernel(const GenParams p, int64_t res_floats) {
-    extern __shared__ __align__(16) float sm[];
-    float *actA = sm;                          // [ka][P]
-    float *actB = actA + p.ka * P;             // [ka][P]
-    float *res = actB + p.ka * P;              // resident weights and parameters
-    __shared__ float s_norm[P];
-    __shared__ int s_valid[P];
-    // tensor-core operands (1024-byte aligned): A hi, A lo (last-layer W), B hi, B lo (its inputs)
-    uint8_t *tcb = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(res + res_floats) + 1023) & ~uintptr_t(1023));
-    const int a_part = p.t_nmt * p.t_katoms * TC_A_ATOM, b_part = p.t_katoms * TC_B_ATOM;
-    uint8_t *a_hi = tcb, *a_lo = tcb + a_part, *b_hi = tcb + 2 * a_part, *b_lo = b_hi + b_part;
-    __shared__ uint32_t s_tmem;
-    __shared__ uint64_t s_bar;
-    __shared__ int s_abort;
 
+// Loads the resident region (hidden layers and, unless `skip_last`, the last
+// layer's transposed weights; every layer's bias and sine frequencies; the
+// set's FiLM rows; the decay rates times log2 e).
+__device__ void load_resident(const GenParams &p, float *res, int set, bool skip_last) {
     const int tid = threadIdx.x;
-    const int tx = tid & 15, ty = tid >> 4;
-    const int set = blockIdx.y;
     const int nl = p.nl;
-    const int nout = p.widths[nl];
-    const int64_t nblk = (p.npos + P - 1) / P;
-
-    if (TC) {
-        if ((tid >> 5) == 0) tc::tmem_alloc(&s_tmem, p.t_cols);
-        if (tid == 0) {
-            mbar_init(&s_bar, 1);
-            mbar_init_fence();
-            s_abort = 0;
-        }
-        // A: last-layer weights, rows = outputs (zero past nout), K = inputs (zero past K)
-        const int K = p.widths[nl - 1];
-        const float *W = p.W[nl - 1];
-        const int rows = p.t_nmt * 128;
-        for (int idx = tid; idx < rows * p.t_kpad; idx += NT) {
-            const int o = idx / p.t_kpad, k = idx - o * p.t_kpad;
-            const float v = (o < nout && k < K) ? __ldg(W + (int64_t)o * K + k) : 0.f;
-            __half hi, lo;
-            fp16_split(v, hi, lo);
-            const uint32_t off = (uint32_t)((o >> 7) * p.t_katoms * TC_A_ATOM + (k >> 6) * TC_A_ATOM) + fg_sw128(o & 127, k);
-            *reinterpret_cast<__half *>(a_hi + off) = hi;
-            *reinterpret_cast<__half *>(a_lo + off) = lo;
-        }
-        // B: the K padding stays zero (the hidden epilogue writes k < K only)
-        for (int idx = tid; idx < 2 * b_part / 16; idx += NT) reinterpret_cast<uint4 *>(b_hi)[idx] = make_uint4(0, 0, 0, 0);
-    }
     for (int l = 0; l < nl; ++l) {
         const int win = p.widths[l], wout = p.widths[l + 1];
         const float *W = p.W[l];
         float *wT = res + p.r_w[l];
-        if (!(TC && l == nl - 1))
+        if (!(skip_last && l == nl - 1))
             for (int idx = tid; idx < win * wout; idx += NT) {    // W row-major (out x in): reads along k
                 const int o = idx / win, k = idx - o * win;
                 wT[k * p.r_ws[l] + o] = __ldg(W + idx);
@@ -454,185 +404,310 @@ __global__ void __launch_bounds__(NT, 2) filter_gen_resident_kernel(const GenPar
             }
         }
     }
-    for (int o = tid; o < nout; o += NT) res[p.r_al + o] = __ldg(p.alpha + o) * kLog2e;   // e^{-a n} = 2^{-a log2(e) n}
+    for (int o = tid; o < p.widths[nl]; o += NT) res[p.r_al + o] = __ldg(p.alpha + o) * kLog2e;   // e^{-a n} = 2^{-a log2(e) n}
+}
 
-    if (TC) {
-        fence_proxy_async_smem();              // the A operand is read by the tensor cores
-        tc::fence_before();
+// Positional encoding and hidden layers of the P positions from p0 with the
+// resident weights; returns the buffer holding the last hidden layer's
+// outputs ([width][P]; the encoding itself when there is no hidden layer).
+// Ends with a CTA barrier.
+__device__ float *resident_hidden(const GenParams &p, const float *res, int64_t p0, float *actA, float *actB,
+                                  float *s_norm, int *s_valid) {
+    const int tid = threadIdx.x;
+    const int tx = tid & 15, ty = tid >> 4;
+    encode_positions(p, p0, actA, actB, s_norm, s_valid);
+    __syncthreads();
+    float *cur = actA, *nxt = actB;
+    for (int l = 0; l < p.nl - 1; ++l) {
+        const int K = p.widths[l];
+        const float *wT = res + p.r_w[l];
+        const int wout = p.widths[l + 1];
+        const bool film = (l == 0) && p.r_g >= 0;
+        for (int o0 = 0; o0 < wout; o0 += 16 * CPT_H) {
+            float acc[4][CPT_H];
+            tile_gemm<CPT_H>(cur, wT + o0, K, tx, ty, acc, p.r_ws[l]);
+#pragma unroll
+            for (int c = 0; c < CPT_H; ++c) {
+                const int o = o0 + CPT_H * ty + c;
+                if (o >= wout) continue;
+                const float bo = res[p.r_b[l] + o];
+                const float gm = film ? res[p.r_g + o] : 0.f;
+                const float bt2 = film ? res[p.r_be + o] : 0.f;
+                const float om = p.r_om[l] >= 0 ? res[p.r_om[l] + o] : 1.f;
+                float v[4];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    float x = acc[a][c] + bo;
+                    if (film) x = fmaf(1.f + gm, x, bt2);
+                    if (p.act == HY_ACT_SILU) x = silu(x);
+                    else if (p.act == HY_ACT_SINE) x = sinf(om * x);
+                    v[a] = x;
+                }
+                *reinterpret_cast<float4 *>(nxt + o * P + 4 * tx) = make_float4(v[0], v[1], v[2], v[3]);
+            }
+        }
+        __syncthreads();
+        float *t2 = cur;
+        cur = nxt;
+        nxt = t2;
     }
-    uint32_t tc_phase = 0;
+    return cur;
+}
+
+__global__ void __launch_bounds__(NT, 2) filter_gen_resident_kernel(const GenParams p) {
+    extern __shared__ __align__(16) float sm[];
+    float *actA = sm;                          // [ka][P]
+    float *actB = actA + p.ka * P;             // [ka][P]
+    float *res = actB + p.ka * P;              // resident weights and parameters
+    __shared__ float s_norm[P];
+    __shared__ int s_valid[P];
+
+    const int tid = threadIdx.x;
+    const int tx = tid & 15, ty = tid >> 4;
+    const int set = blockIdx.y;
+    const int nl = p.nl;
+    const int nout = p.widths[nl];
+    const int64_t nblk = (p.npos + P - 1) / P;
+    load_resident(p, res, set, false);
+    const int l = nl - 1;
+    const int K = p.widths[l];
+    const float *wT = res + p.r_w[l];
     for (int64_t bt = blockIdx.x; bt < nblk; bt += gridDim.x) {
         const int64_t p0 = bt * P;
         __syncthreads();                       // resident region written / previous tile's reads done
-        if (TC) {
-            tc::fence_after();
-            if (s_abort) break;                // uniform: read between two barriers
+        const float *cur = resident_hidden(p, res, p0, actA, actB, s_norm, s_valid);
+        float nrm[4];
+        bool ok[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            nrm[a] = s_norm[4 * tx + a];
+            if (p.window == HY_WIN_GAUSS) nrm[a] *= nrm[a];
+            ok[a] = s_valid[4 * tx + a] != 0;
         }
-        encode_positions(p, p0, actA, actB, s_norm, s_valid);
-        __syncthreads();
-        float *cur = actA, *nxt = actB;
-        for (int l = 0; l < nl; ++l) {
-            const int K = p.widths[l];
-            const float *wT = res + p.r_w[l];
-            if (l < nl - 1) {
-                const int wout = p.widths[l + 1];
-                const bool film = (l == 0) && p.r_g >= 0;
-                for (int o0 = 0; o0 < wout; o0 += 16 * CPT_H) {
-                    float acc[4][CPT_H];
-                    tile_gemm<CPT_H>(cur, wT + o0, K, tx, ty, acc, p.r_ws[l]);
+        const int64_t q0 = p0 + 4 * tx;
+        const bool full = p.vec_out && q0 + 3 < p.npos;
+        for (int o0 = 0; o0 < nout; o0 += 16 * CPT_L) {
+            float acc[4][CPT_L];
+            tile_gemm<CPT_L>(cur, wT + o0, K, tx, ty, acc, p.r_ws[l]);
 #pragma unroll
-                    for (int c = 0; c < CPT_H; ++c) {
-                        const int o = o0 + CPT_H * ty + c;
-                        if (o >= wout) continue;
-                        const float bo = res[p.r_b[l] + o];
-                        const float gm = film ? res[p.r_g + o] : 0.f;
-                        const float bt2 = film ? res[p.r_be + o] : 0.f;
-                        const float om = p.r_om[l] >= 0 ? res[p.r_om[l] + o] : 1.f;
-                        float v[4];
+            for (int c = 0; c < CPT_L; ++c) {
+                const int o = o0 + CPT_L * ty + c;
+                if (o >= nout) continue;
+                const float bo = res[p.r_b[l] + o];
+                const float al = res[p.r_al + o];
+                float v[4];
 #pragma unroll
-                        for (int a = 0; a < 4; ++a) {
-                            float x = acc[a][c] + bo;
-                            if (film) x = fmaf(1.f + gm, x, bt2);
-                            if (p.act == HY_ACT_SILU) x = silu(x);
-                            else if (p.act == HY_ACT_SINE) x = sinf(om * x);
-                            v[a] = x;
-                        }
-                        if (TC && l == nl - 2) {
-                            // inputs of the tensor-core last layer: B[pos][k = o], fp16 hi and lo
+                for (int a = 0; a < 4; ++a) v[a] = ok[a] ? (acc[a][c] + bo) * exp2f(-al * nrm[a]) : 0.f;
+                float *dst = p.h + ((int64_t)set * nout + o) * p.npos + q0;
+                if (full) {
+                    *reinterpret_cast<float4 *>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+                } else {
 #pragma unroll
-                            for (int a = 0; a < 4; ++a) {
-                                __half hi, lo;
-                                fp16_split(v[a], hi, lo);
-                                const int pos = 4 * tx + a;
-                                const uint32_t off = (uint32_t)((o >> 6) * TC_B_ATOM) + fg_sw128(pos, o);
-                                *reinterpret_cast<__half *>(b_hi + off) = hi;
-                                *reinterpret_cast<__half *>(b_lo + off) = lo;
-                            }
-                        } else {
-                            *reinterpret_cast<float4 *>(nxt + o * P + 4 * tx) = make_float4(v[0], v[1], v[2], v[3]);
-                        }
-                    }
-                }
-                if (TC && l == nl - 2) fence_proxy_async_smem();   // the B operand is read by the tensor cores
-                __syncthreads();
-                float *t2 = cur;
-                cur = nxt;
-                nxt = t2;
-            } else if (TC) {
-                // D[o][pos] = Σ_k W[o][k] act[pos][k] on the tensor cores: hi·hi + hi·lo + lo·hi
-                if (tid == 0) {
-                    tc::fence_after();
-                    constexpr uint32_t IDESC = tc::idesc_f16(128, P, false);
-                    for (int mt = 0; mt < p.t_nmt; ++mt) {
-                        bool first = true;
-                        for (int term = 0; term < 3; ++term) {
-                            const uint8_t *A = (term == 2 ? a_lo : a_hi) + mt * p.t_katoms * TC_A_ATOM;
-                            const uint8_t *Bm = term == 1 ? b_lo : b_hi;
-                            for (int ks = 0; ks < p.t_kpad / 16; ++ks) {
-                                const uint64_t ad = tc::desc_k_sw128(smem_u32(A + (ks >> 2) * TC_A_ATOM)) + 2 * (ks & 3);
-                                const uint64_t bd = tc::desc_k_sw128(smem_u32(Bm + (ks >> 2) * TC_B_ATOM)) + 2 * (ks & 3);
-                                tc::mma_f16(s_tmem + 64u * mt, ad, bd, IDESC, first ? 0u : 1u);
-                                first = false;
-                            }
-                        }
-                    }
-                    tc::commit(&s_bar);
-                    if (!mbar_wait_sleep(&s_bar, tc_phase)) {
-                        record_fault(p.fault, HY_FAULT_FILTER_MMA);
-                        s_abort = 1;
-                    }
-                }
-                tc_phase ^= 1;
-                __syncthreads();
-                tc::fence_after();
-                // epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 (outputs) and
-                // positions 32 (w / 4) .. + 31 of each M tile
-                const int warp = tid >> 5, lane = tid & 31;
-                const int q = warp & 3, hc = warp >> 2;
-                for (int mt = 0; mt < p.t_nmt; ++mt) {
-                    __syncwarp();                      // tcgen05.ld is warp-wide
-                    uint32_t v[32];
-                    tc::tmem_ld32(s_tmem + ((uint32_t)(32 * q) << 16) + 64u * mt + 32u * hc, v);
-                    tc::tmem_wait_ld();
-                    const int o = 128 * mt + 32 * q + lane;
-                    if (o >= nout) continue;
-                    const float bo = res[p.r_b[l] + o];
-                    const float al = res[p.r_al + o];
-                    const int64_t q0 = p0 + 32 * hc;
-                    float *dst = p.h + ((int64_t)set * nout + o) * p.npos + q0;
-                    float w[32];
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        float nr = s_norm[32 * hc + j];
-                        if (p.window == HY_WIN_GAUSS) nr *= nr;
-                        w[j] = s_valid[32 * hc + j] ? (__uint_as_float(v[j]) + bo) * exp2f(-al * nr) : 0.f;
-                    }
-                    if (p.vec_out && q0 + 31 < p.npos) {
-#pragma unroll
-                        for (int j = 0; j < 32; j += 4)
-                            *reinterpret_cast<float4 *>(dst + j) = make_float4(w[j], w[j + 1], w[j + 2], w[j + 3]);
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (q0 + j < p.npos) dst[j] = w[j];
-                    }
-                }
-                tc::fence_before();
-            } else {
-                float nrm[4];
-                bool ok[4];
-#pragma unroll
-                for (int a = 0; a < 4; ++a) {
-                    nrm[a] = s_norm[4 * tx + a];
-                    if (p.window == HY_WIN_GAUSS) nrm[a] *= nrm[a];
-                    ok[a] = s_valid[4 * tx + a] != 0;
-                }
-                const int64_t q0 = p0 + 4 * tx;
-                const bool full = p.vec_out && q0 + 3 < p.npos;
-                for (int o0 = 0; o0 < nout; o0 += 16 * CPT_L) {
-                    float acc[4][CPT_L];
-                    tile_gemm<CPT_L>(cur, wT + o0, K, tx, ty, acc, p.r_ws[l]);
-#pragma unroll
-                    for (int c = 0; c < CPT_L; ++c) {
-                        const int o = o0 + CPT_L * ty + c;
-                        if (o >= nout) continue;
-                        const float bo = res[p.r_b[l] + o];
-                        const float al = res[p.r_al + o];
-                        float v[4];
-#pragma unroll
-                        for (int a = 0; a < 4; ++a) v[a] = ok[a] ? (acc[a][c] + bo) * exp2f(-al * nrm[a]) : 0.f;
-                        float *dst = p.h + ((int64_t)set * nout + o) * p.npos + q0;
-                        if (full) {
-                            *reinterpret_cast<float4 *>(dst) = make_float4(v[0], v[1], v[2], v[3]);
-                        } else {
-#pragma unroll
-                            for (int a = 0; a < 4; ++a)
-                                if (q0 + a < p.npos) dst[a] = v[a];
-                        }
-                    }
+                    for (int a = 0; a < 4; ++a)
+                        if (q0 + a < p.npos) dst[a] = v[a];
                 }
             }
         }
     }
-    if (TC) {
-        // no MMA may still be running when TMEM is freed (all were waited on;
-        // this covers one whose wait gave up)
-        if (tid == 0) {
-            tc::commit(&s_bar);
-            if (!mbar_wait_sleep(&s_bar, tc_phase)) record_fault(p.fault, HY_FAULT_FILTER_MMA);
-        }
-        tc::fence_before();
-        __syncthreads();
-        tc::fence_after();
-        __syncwarp();
-        if ((tid >> 5) == 0) tc::tmem_free(s_tmem, p.t_cols);
-    }
 }
 
-// The tensor-core last layer is opt-in (HYENA_FILTER_ENGINE=tensor).
-bool tensor_last_layer_enabled() {
+// ----------------------------------------------------------------------------
+// Tensor-core last layer (the dense contraction: 85-97% of the MACs).  A tile
+// is TP = 128 positions of one set, the M of one tcgen05 MMA:
+//   D[pos][o] = sum_k act[pos][k] W[o][k]
+// with both operands K-major in the 128-byte-swizzled layout: A = the last
+// hidden layer's outputs of the tile (rows = positions), B = the last layer's
+// weights (rows = outputs), held for the whole kernel.  Each operand is split
+// into fp16 hi + lo (|x - hi - lo| <= 2^-22 |x|) and the three products
+// hi.hi + hi.lo + lo.hi accumulate in fp32 in tensor memory: 128 lanes (the
+// positions) x the padded outputs.  The hidden layers run on the FP32 pipes
+// (resident weights, two halves of 64 positions); their fp32 outputs are
+// packed into A as 16-byte chunks (one position row per thread, swizzled, so
+// the stores do not conflict).  The epilogue reads a row per thread from
+// tensor memory -- all outputs of one position -- adds the bias, applies the
+// decay window and stores: at each output the 32 lanes of a warp write 32
+// consecutive positions, one 128-byte segment.  One thread issues the MMAs
+// and waits for them (bounded, HY_FAULT_FILTER_MMA).
+// ----------------------------------------------------------------------------
+constexpr int TP = 2 * P;                 // positions per tensor-core tile
+constexpr int TC_ROW = 128;               // bytes per operand row and K atom (64 fp16)
+
+// Byte offset of 16-byte chunk c (k = 8c .. 8c+7 within the atom) of row r in
+// a K-major 128-byte-swizzled atom column (8-row groups 1024 bytes apart).
+__device__ __forceinline__ uint32_t sw128_chunk(int r, int c) {
+    return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
+}
+__device__ __forceinline__ void split_h2(float a, float b, uint32_t &hi, uint32_t &lo) {
+    const __half2 h = __floats2half2_rn(a, b);
+    const float2 hf = __half22float2(h);
+    const __half2 l = __floats2half2_rn(a - hf.x, b - hf.y);
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
+__global__ void __launch_bounds__(NT, 2) filter_gen_tc_kernel(const GenParams p, int64_t res_floats) {
+    extern __shared__ __align__(16) float sm[];
+    float *actA = sm;                          // [ka][P]
+    float *actB = actA + p.ka * P;             // [ka][P]
+    float *res = actB + p.ka * P;              // resident hidden weights and parameters
+    // operands (1024-byte aligned): A hi, A lo ([katoms][TP rows][128 B]), B hi, B lo ([katoms][npad rows][128 B])
+    uint8_t *tcb = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(res + res_floats) + 1023) & ~uintptr_t(1023));
+    const int katoms = p.t_katoms, npad = p.t_npad;
+    const int a_part = katoms * TP * TC_ROW, b_part = katoms * npad * TC_ROW;
+    uint8_t *a_hi = tcb, *a_lo = tcb + a_part, *b_hi = tcb + 2 * a_part, *b_lo = b_hi + b_part;
+    __shared__ float s_norm[TP];
+    __shared__ int s_valid[TP];
+    __shared__ uint32_t s_tmem;
+    __shared__ uint64_t s_bar;
+    __shared__ int s_abort;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int set = blockIdx.y;
+    const int nl = p.nl;
+    const int nout = p.widths[nl];
+    const int K = p.widths[nl - 1];
+    const int kchunks = p.t_kpad / 8;          // 16-byte chunks of a row
+    const int64_t ntiles = (p.npos + TP - 1) / TP;
+
+    if (warp == 0) tc::tmem_alloc(&s_tmem, p.t_cols);
+    if (tid == 0) {
+        mbar_init(&s_bar, 1);
+        mbar_init_fence();
+        s_abort = 0;
+    }
+    load_resident(p, res, set, true);
+    // B: the last layer's weights, rows o < npad (zero past nout), K padded with zeros
+    {
+        const float *W = p.W[nl - 1];
+        for (int idx = tid; idx < npad * kchunks; idx += NT) {
+            const int o = idx / kchunks, c = idx - o * kchunks;
+            float v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int k = 8 * c + j;
+                v[j] = (o < nout && k < K) ? __ldg(W + (int64_t)o * K + k) : 0.f;
+            }
+            uint4 hi, lo;
+            split_h2(v[0], v[1], hi.x, lo.x);
+            split_h2(v[2], v[3], hi.y, lo.y);
+            split_h2(v[4], v[5], hi.z, lo.z);
+            split_h2(v[6], v[7], hi.w, lo.w);
+            const uint32_t off = (uint32_t)((c >> 3) * npad * TC_ROW) + sw128_chunk(o, c & 7);
+            *reinterpret_cast<uint4 *>(b_hi + off) = hi;
+            *reinterpret_cast<uint4 *>(b_lo + off) = lo;
+        }
+    }
+    fence_proxy_async_smem();                  // B is read by the tensor cores
+    tc::fence_before();
+    uint32_t phase = 0;
+    for (int64_t bt = blockIdx.x; bt < ntiles; bt += gridDim.x) {
+        __syncthreads();                       // operands / TMEM of the previous tile released
+        tc::fence_after();
+        if (s_abort) break;                    // uniform: read between two barriers
+        // ---- hidden layers of the two halves, packed into A
+        for (int half = 0; half < 2; ++half) {
+            const int64_t p0 = bt * TP + half * P;
+            const float *cur = resident_hidden(p, res, p0, actA, actB, s_norm + half * P, s_valid + half * P);
+            for (int idx = tid; idx < P * kchunks; idx += NT) {
+                const int r = idx & (P - 1), c = idx / P;
+                float v[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int k = 8 * c + j;
+                    v[j] = k < K ? cur[k * P + r] : 0.f;
+                }
+                uint4 hi, lo;
+                split_h2(v[0], v[1], hi.x, lo.x);
+                split_h2(v[2], v[3], hi.y, lo.y);
+                split_h2(v[4], v[5], hi.z, lo.z);
+                split_h2(v[6], v[7], hi.w, lo.w);
+                const int row = half * P + r;
+                const uint32_t off = (uint32_t)((c >> 3) * TP * TC_ROW) + sw128_chunk(row, c & 7);
+                *reinterpret_cast<uint4 *>(a_hi + off) = hi;
+                *reinterpret_cast<uint4 *>(a_lo + off) = lo;
+            }
+            __syncthreads();                   // cur is overwritten by the next half
+        }
+        fence_proxy_async_smem();              // A is read by the tensor cores
+        __syncthreads();
+        // ---- D = A B^T in up to two N chunks of <= 256 outputs: hi.hi + hi.lo + lo.hi
+        if (tid == 0) {
+            tc::fence_after();
+            for (int n0 = 0; n0 < npad; n0 += 256) {
+                const int nc = npad - n0 < 256 ? npad - n0 : 256;
+                const uint32_t idesc = tc::idesc_f16(128, nc, false);
+                bool first = true;
+                for (int term = 0; term < 3; ++term) {
+                    const uint8_t *A = term == 2 ? a_lo : a_hi;
+                    const uint8_t *Bm = (term == 1 ? b_lo : b_hi) + n0 * TC_ROW;
+                    for (int ks = 0; ks < p.t_kpad / 16; ++ks) {
+                        const uint64_t ad = tc::desc_k_sw128(smem_u32(A + (ks >> 2) * TP * TC_ROW)) + 2 * (ks & 3);
+                        const uint64_t bd = tc::desc_k_sw128(smem_u32(Bm + (ks >> 2) * npad * TC_ROW)) + 2 * (ks & 3);
+                        tc::mma_f16(s_tmem + (uint32_t)n0, ad, bd, idesc, first ? 0u : 1u);
+                        first = false;
+                    }
+                }
+            }
+            tc::commit(&s_bar);
+            if (!mbar_wait_sleep(&s_bar, phase)) {
+                record_fault(p.fault, HY_FAULT_FILTER_MMA);
+                s_abort = 1;
+            }
+        }
+        phase ^= 1;
+        __syncthreads();
+        tc::fence_after();
+        // ---- epilogue: warp w takes positions 32 (w % 4) + lane (TMEM lanes)
+        //      and every other 16-column chunk from w / 4
+        {
+            const int q = warp & 3;
+            const int pos = 32 * q + lane;
+            const int64_t qq = bt * TP + pos;
+            float nr = s_norm[pos];
+            if (p.window == HY_WIN_GAUSS) nr *= nr;
+            const bool ok = s_valid[pos] != 0;
+            const bool in = qq < p.npos;
+            const float *bias = res + p.r_b[nl - 1];
+            const float *al = res + p.r_al;
+            const float nrn = ok ? -nr : 0.f;
+            for (int c0 = 16 * (warp >> 2); c0 < npad; c0 += 32) {
+                __syncwarp();                  // tcgen05.ld is warp-wide
+                uint32_t v[16];
+                tc::tmem_ld16(s_tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+                tc::tmem_wait_ld();
+                float *dst = p.h + ((int64_t)set * nout + c0) * p.npos + qq;
+#pragma unroll
+                for (int j = 0; j < 16; ++j, dst += p.npos) {
+                    if (c0 + j < nout && in) {
+                        const float y = (__uint_as_float(v[j]) + bias[c0 + j]) * exp2f(al[c0 + j] * nrn);
+                        *dst = ok ? y : 0.f;
+                    }
+                }
+            }
+        }
+        tc::fence_before();
+    }
+    // no MMA may still be running when TMEM is freed (all were waited on;
+    // this covers one whose wait gave up)
+    if (tid == 0) {
+        tc::commit(&s_bar);
+        if (!mbar_wait_sleep(&s_bar, phase)) record_fault(p.fault, HY_FAULT_FILTER_MMA);
+    }
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    __syncwarp();
+    if (warp == 0) tc::tmem_free(s_tmem, p.t_cols);
+}
+
+// Engine of the last layer: HYENA_FILTER_ENGINE=simt keeps it on the FP32
+// pipes, =tensor asks for the tensor cores; unset, the tensor cores take it
+// wherever the kernel applies.
+int filter_engine() {
     const char *e = std::getenv("HYENA_FILTER_ENGINE");
-    return e && std::strcmp(e, "tensor") == 0;
+    if (e && std::strcmp(e, "simt") == 0) return 0;
+    if (e && std::strcmp(e, "tensor") == 0) return 2;
+    return 1;
 }
 
 // Float layout of the resident region; returns its size in floats.  Each
@@ -704,45 +779,69 @@ hy_status launch_filter_gen(const hy_filter_desc &d, float *h, cudaStream_t s) {
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     }
-    // Many position tiles per set, weights that fit in shared memory: keep
-    // them resident in persistent CTAs instead of staging them per tile; the
-    // last layer runs on the tensor cores when it has a hidden layer before it
-    // and K <= 128 (its operands follow the resident region).
+    // Tensor-core last layer: a hidden layer before it, K <= 128, at most 512
+    // outputs, at least one 128-position tile per SM.
     {
         GenParams q = p;
         const int Klast = q.widths[q.nl - 1];
         const int nlast = q.widths[q.nl];
-        // (the tensor-core last layer is built and tested but slower than the
-        // FP32 pipes here: its fp16 operand stores conflict in shared memory)
-        const bool tc = tensor_last_layer_enabled() && q.nl >= 2 && Klast <= 128 && nlast <= 512;
-        const int64_t rfl = resident_layout(q, tc);
-        size_t tc_bytes = 0;
-        if (tc) {
+        const int64_t ntiles = (q.npos + TP - 1) / TP;
+        if (filter_engine() > 0 && q.nl >= 2 && Klast <= 128 && nlast <= 512 && ntiles * d.n_sets >= sms) {
+            const int64_t rfl = resident_layout(q, true);
             q.t_kpad = (Klast + 15) & ~15;
             q.t_katoms = (q.t_kpad + 63) / 64;
-            q.t_nmt = (nlast + 127) / 128;
-            q.t_cols = q.t_nmt <= 1 ? 64u : (q.t_nmt <= 2 ? 128u : 256u);
+            q.t_npad = (nlast + 15) & ~15;
+            q.t_cols = 32;
+            while ((int)q.t_cols < q.t_npad) q.t_cols <<= 1;
             q.fault = device_fault_word();
             if (!q.fault) return set_error(HY_ERR_CUDA, "device fault word unavailable");
-            tc_bytes = 1024 + (size_t)2 * q.t_nmt * q.t_katoms * TC_A_ATOM + (size_t)2 * q.t_katoms * TC_B_ATOM;
+            size_t smem = sizeof(float) * ((size_t)2 * q.ka * P + (size_t)rfl) + 1024 +
+                          (size_t)2 * q.t_katoms * TP * TC_ROW + (size_t)2 * q.t_katoms * q.t_npad * TC_ROW;
+            // the CTAs that share an SM must fit its 512 TMEM columns: ask for
+            // enough shared memory that no more of them can be resident
+            const int fit = 512 / (int)q.t_cols;
+            const size_t floor_smem = (size_t)233472 / (size_t)(fit + 1) + 1024;
+            if (fit < 8 && smem < floor_smem) smem = floor_smem;
+            if (smem <= (size_t)227 * 1024) {
+                cudaError_t e = cudaFuncSetAttribute(filter_gen_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     (int)smem);
+                if (e != cudaSuccess) return set_cuda_error("filter_gen tensor-core smem attribute", e);
+                e = cudaFuncSetAttribute(filter_gen_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         (int)cudaSharedmemCarveoutMaxShared);
+                if (e != cudaSuccess) return set_cuda_error("filter_gen carve-out attribute", e);
+                // CTAs per SM from the shared memory they take (two at most: the
+                // launch bounds give each thread 128 registers)
+                int per_sm = (int)((size_t)233472 / (smem + 1024));
+                if (per_sm > 2) per_sm = 2;
+                if (per_sm > fit) per_sm = fit;
+                if (per_sm < 1) per_sm = 1;
+                int64_t per_set = ((int64_t)per_sm * sms + d.n_sets - 1) / d.n_sets;
+                if (per_set > ntiles) per_set = ntiles;
+                dim3 grid((unsigned)per_set, (unsigned)d.n_sets, 1);
+                filter_gen_tc_kernel<<<grid, NT, smem, s>>>(q, rfl);
+                return check_launch("filter_gen (tensor-core last layer) launch");
+            }
         }
-        const size_t rsmem = sizeof(float) * ((size_t)2 * q.ka * P + (size_t)rfl) + tc_bytes;
-        // FP32-pipe last layer: only with two CTAs per SM (with one, the FP32
-        // pipes idle at every barrier and the streaming kernel's two CTAs per
-        // SM are faster).  Tensor-core last layer: one CTA per SM is enough.
-        const bool two = rsmem <= (size_t)113 * 1024;
-        if (nblk * d.n_sets >= (int64_t)8 * sms && (two || (tc && rsmem <= (size_t)227 * 1024))) {
-            auto kernel = tc ? filter_gen_resident_kernel<true> : filter_gen_resident_kernel<false>;
-            cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem);
+    }
+    // Many position tiles per set, weights that fit in shared memory: keep
+    // them resident in persistent CTAs instead of staging them per tile (only
+    // with two CTAs per SM: with one, the FP32 pipes idle at every barrier and
+    // the streaming kernel's two CTAs per SM are faster).
+    {
+        GenParams q = p;
+        const int64_t rfl = resident_layout(q, false);
+        const size_t rsmem = sizeof(float) * ((size_t)2 * q.ka * P + (size_t)rfl);
+        if (nblk * d.n_sets >= (int64_t)8 * sms && rsmem <= (size_t)113 * 1024) {
+            cudaError_t e = cudaFuncSetAttribute(filter_gen_resident_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)rsmem);
             if (e != cudaSuccess) return set_cuda_error("filter_gen resident smem attribute", e);
-            e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+            e = cudaFuncSetAttribute(filter_gen_resident_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                                      (int)cudaSharedmemCarveoutMaxShared);
             if (e != cudaSuccess) return set_cuda_error("filter_gen carve-out attribute", e);
-            // two CTAs per SM when they fit (TMEM <= 256 columns each), else one
-            int64_t per_set = ((int64_t)(two ? 2 : 1) * sms + d.n_sets - 1) / d.n_sets;
+            int64_t per_set = ((int64_t)2 * sms + d.n_sets - 1) / d.n_sets;
             if (per_set > nblk) per_set = nblk;
             dim3 grid((unsigned)per_set, (unsigned)d.n_sets, 1);
-            kernel<<<grid, NT, rsmem, s>>>(q, rfl);
+            filter_gen_resident_kernel<<<grid, NT, rsmem, s>>>(q);
             return check_launch("filter_gen (resident weights) launch");
         }
     }

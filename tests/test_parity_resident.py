@@ -293,13 +293,14 @@ def test_c5_full_size():
 @pytest.mark.parametrize("act,hidden,nout", [("silu", [32, 24], 40), ("sine", [32, 24], 40),
                                                ("silu", [96], 200), ("silu", [64], 512)])
 def test_filter_gen_resident_weights_many_tiles(act, hidden, nout, engine, monkeypatch):
-    """Enough positions for the persistent resident-weight filter kernel
-    (more than 8 position tiles per SM), its last layer on the FP32 pipes
-    (default) or on the tensor cores (HYENA_FILTER_ENGINE=tensor, fp16 hi/lo
-    operands): 1-D L = 2^17, one or two hidden layers, a last layer with K over
-    one 64-element atom and outputs over several 128-row tiles (512 outputs:
-    one CTA per SM, or the streaming kernel on the FP32 pipes); every position
-    and output against the oracle."""
+    """Enough positions for the persistent filter kernels: the last layer on
+    the tensor cores (the default where it applies: 128-position tiles as the
+    MMA M, fp16 hi/lo operands, fp32 accumulation) or, with
+    HYENA_FILTER_ENGINE=simt, on the FP32 pipes with resident weights (or the
+    streaming kernel when they do not fit two CTAs per SM): 1-D L = 2^17, one
+    or two hidden layers, a last layer with K of 24, 64 or 96 (padded to 16,
+    one or two 64-element atoms) and 40, 200 or 512 outputs (padded to 16, one
+    or two MMA N chunks); every position and output against the oracle."""
     monkeypatch.setenv("HYENA_FILTER_ENGINE", engine)
     L, F = 1 << 17, 8
     rng = np.random.default_rng(170 + (act == "sine") + nout)

@@ -71,7 +71,8 @@ struct GenParams {
     // tensor-core last layer: operands after the resident region
     int t_kpad;                 // last-layer K rounded up to 16
     int t_katoms;               // 64-element K atoms
-    int t_npad;                 // outputs rounded up to 16 (MMA N, in chunks of <= 256)
+    int t_npad;                 // outputs of a CTA's slice rounded up to 16 (MMA N, in chunks of <= 256)
+    int t_slice;                // outputs per grid-z slice (all of them, or 256 when split)
     uint32_t t_cols;            // TMEM columns (power of two >= max(32, t_npad))
     uint32_t *fault;            // device fault word
 };
@@ -565,6 +566,8 @@ __global__ void __launch_bounds__(NT, 2) filter_gen_tc_kernel(const GenParams p,
     const int set = blockIdx.y;
     const int nl = p.nl;
     const int nout = p.widths[nl];
+    const int obase = blockIdx.z * p.t_slice;  // this CTA's outputs: obase .. obase + t_slice - 1
+    const int oend = min(nout, obase + p.t_slice);
     const int K = p.widths[nl - 1];
     const int kchunks = p.t_kpad / 8;          // 16-byte chunks of a row
     const int64_t ntiles = (p.npos + TP - 1) / TP;
@@ -576,7 +579,8 @@ __global__ void __launch_bounds__(NT, 2) filter_gen_tc_kernel(const GenParams p,
         s_abort = 0;
     }
     load_resident(p, res, set, true);
-    // B: the last layer's weights, rows o < npad (zero past nout), K padded with zeros
+    // B: the last layer's weights of the slice, rows obase + o for o < npad
+    // (zero past the slice), K padded with zeros
     {
         const float *W = p.W[nl - 1];
         for (int idx = tid; idx < npad * kchunks; idx += NT) {
@@ -585,7 +589,7 @@ __global__ void __launch_bounds__(NT, 2) filter_gen_tc_kernel(const GenParams p,
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int k = 8 * c + j;
-                v[j] = (o < nout && k < K) ? __ldg(W + (int64_t)o * K + k) : 0.f;
+                v[j] = (obase + o < oend && k < K) ? __ldg(W + (int64_t)(obase + o) * K + k) : 0.f;
             }
             uint4 hi, lo;
             split_h2(v[0], v[1], hi.x, lo.x);
@@ -675,11 +679,12 @@ __global__ void __launch_bounds__(NT, 2) filter_gen_tc_kernel(const GenParams p,
                 uint32_t v[16];
                 tc::tmem_ld16(s_tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
                 tc::tmem_wait_ld();
-                float *dst = p.h + ((int64_t)set * nout + c0) * p.npos + qq;
+                const int ob = obase + c0;
+                float *dst = p.h + ((int64_t)set * nout + ob) * p.npos + qq;
 #pragma unroll
                 for (int j = 0; j < 16; ++j, dst += p.npos) {
-                    if (c0 + j < nout && in) {
-                        const float y = (__uint_as_float(v[j]) + bias[c0 + j]) * exp2f(al[c0 + j] * nrn);
+                    if (ob + j < oend && in) {
+                        const float y = (__uint_as_float(v[j]) + bias[ob + j]) * exp2f(al[ob + j] * nrn);
                         *dst = ok ? y : 0.f;
                     }
                 }
@@ -779,18 +784,24 @@ hy_status launch_filter_gen(const hy_filter_desc &d, float *h, cudaStream_t s) {
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     }
-    // Tensor-core last layer: a hidden layer before it, K <= 128, at most 512
-    // outputs, at least one 128-position tile per SM.
+    // Tensor-core last layer: a hidden layer before it, K <= 128, at least one
+    // (128-position tile, output slice) pair per SM.
     {
         GenParams q = p;
         const int Klast = q.widths[q.nl - 1];
         const int nlast = q.widths[q.nl];
         const int64_t ntiles = (q.npos + TP - 1) / TP;
-        if (filter_engine() > 0 && q.nl >= 2 && Klast <= 128 && nlast <= 512 && ntiles * d.n_sets >= sms) {
+        // more than 512 outputs: split over grid z in slices of 256 (each
+        // slice recomputes the hidden layers).  With fewer position tiles than
+        // SMs the FP32-pipe kernels stay: slicing the 768 outputs of an
+        // 8192-position filter set over 64 tiles measured 2x slower than them.
+        q.t_slice = nlast > 512 ? 256 : nlast;
+        const int nslices = (nlast + q.t_slice - 1) / q.t_slice;
+        if (filter_engine() > 0 && q.nl >= 2 && Klast <= 128 && nslices <= 64 && ntiles * d.n_sets >= sms) {
             const int64_t rfl = resident_layout(q, true);
             q.t_kpad = (Klast + 15) & ~15;
             q.t_katoms = (q.t_kpad + 63) / 64;
-            q.t_npad = (nlast + 15) & ~15;
+            q.t_npad = (q.t_slice + 15) & ~15;
             q.t_cols = 32;
             while ((int)q.t_cols < q.t_npad) q.t_cols <<= 1;
             q.fault = device_fault_word();
@@ -815,9 +826,9 @@ hy_status launch_filter_gen(const hy_filter_desc &d, float *h, cudaStream_t s) {
                 if (per_sm > 2) per_sm = 2;
                 if (per_sm > fit) per_sm = fit;
                 if (per_sm < 1) per_sm = 1;
-                int64_t per_set = ((int64_t)per_sm * sms + d.n_sets - 1) / d.n_sets;
+                int64_t per_set = ((int64_t)per_sm * sms + (int64_t)d.n_sets * nslices - 1) / ((int64_t)d.n_sets * nslices);
                 if (per_set > ntiles) per_set = ntiles;
-                dim3 grid((unsigned)per_set, (unsigned)d.n_sets, 1);
+                dim3 grid((unsigned)per_set, (unsigned)d.n_sets, (unsigned)nslices);
                 filter_gen_tc_kernel<<<grid, NT, smem, s>>>(q, rfl);
                 return check_launch("filter_gen (tensor-core last layer) launch");
             }

@@ -109,7 +109,14 @@ def test_fftconv_gate_skip_variants_and_guard_bands():
         check(to_np(y).reshape(B * D, L), conv, "f32", "fftconv gate=%s skip=%s" % (g is not None, s is not None))
 
 
-def test_filter_gen_1d_vs_oracle():
+@pytest.mark.parametrize("engine", ["default", "simt"])
+def test_filter_gen_1d_vs_oracle(engine, monkeypatch):
+    """The filters of workloads 1-3 (c3 at L = 4096) with the default engine
+    choice and with HYENA_FILTER_ENGINE=simt (FP32-pipe kernels); these
+    lengths have too few position tiles for the tensor-core last layer, so
+    both run the streaming kernel."""
+    if engine == "simt":
+        monkeypatch.setenv("HYENA_FILTER_ENGINE", "simt")
     for name, L in [("c1", 1024), ("c2", 8192), ("c3", 4096)]:
         w = hw.make(name, with_signals=False, L=L)
         spec = w.spec
@@ -317,3 +324,26 @@ def test_filter_gen_resident_weights_many_tiles(act, hidden, nout, engine, monke
     torch.cuda.synchronize()
     ref = oracle.filter_gen_1d(L, F, True, Ws, bs, alpha, act=act, omega=omega)
     check(to_np(h), ref, "f32", "resident-weight filters L=2^17 (%s, %s)" % (act, engine))
+
+
+@pytest.mark.parametrize("engine", ["default", "simt"])
+def test_filter_gen_output_slices(engine, monkeypatch):
+    """More than 512 outputs with enough positions: the tensor-core last layer
+    splits them over grid z in 256-output slices (600 = 256 + 256 + 88, the
+    last slice padded to 96 MMA columns); L = 2^16, every position and output
+    against the oracle.  "simt" runs the FP32-pipe kernels on the same
+    filters."""
+    if engine == "simt":
+        monkeypatch.setenv("HYENA_FILTER_ENGINE", "simt")
+    L, F = 1 << 16, 8
+    rng = np.random.default_rng(600)
+    widths = [1 + 2 * F, 64, 600]
+    Ws = [rng.uniform(-1, 1, (b, a)).astype(np.float32) / np.sqrt(a) for a, b in zip(widths[:-1], widths[1:])]
+    bs = [rng.uniform(-0.5, 0.5, b).astype(np.float32) for b in widths[1:]]
+    alpha = rng.uniform(0.1, 2.0, widths[-1]).astype(np.float32)
+    h = torch.empty((widths[-1], L), device="cuda")
+    hy.hyena_filter_gen(h, ndim=1, L=L, Ws=[f32_dev(a) for a in Ws], bs=[f32_dev(a) for a in bs],
+                        alpha=f32_dev(alpha), n_freq=F, include_t=True)
+    torch.cuda.synchronize()
+    ref = oracle.filter_gen_1d(L, F, True, Ws, bs, alpha)
+    check(to_np(h), ref, "f32", "filters with 600 outputs (%s)" % engine)

@@ -267,7 +267,7 @@ hy_status hyena_operator_backward(int order, int B, int D, int L, hy_dtype dt, c
  * Sequences with hyena_spectrum_bins(L) - 1 <= 16384 run on chip as in
  * hyena_operator (no workspace at all).  Longer ones keep their intermediates
  * in one static device array of 32 MiB that the library reserves on every
- * GPU that loads it, until the process exits; one row needs 12 bytes per
+ * GPU that loads it, until the process exits; one row needs 8 bytes per
  * complex point, so L <= 1,048,576 (longer is rejected with
  * HY_ERR_WORKSPACE or HY_ERR_UNSUPPORTED).  The call allocates nothing and
  * calls no allocating routine.

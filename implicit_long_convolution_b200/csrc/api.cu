@@ -402,10 +402,10 @@ extern "C" hy_status hyena_operator_noalloc(int order, int B, int D, int L, hy_d
         return run_chain(K, B, D, L, dt, v, x, H, Dskip, y, const_cast<void *>(no_ws), 0,
                          (cudaStream_t)stream, who);
     }
-    // one row's intermediates (12 bytes per complex point) must fit the scratch
-    if ((size_t)12 * (size_t)M > noalloc_scratch_bytes())
+    // one row's intermediates (8 bytes per complex point) must fit the scratch
+    if ((size_t)8 * (size_t)M > noalloc_scratch_bytes())
         return set_error(HY_ERR_WORKSPACE, "%s: L=%d needs %zu scratch bytes per row; the static scratch holds %zu",
-                         who, L, (size_t)12 * (size_t)M, noalloc_scratch_bytes());
+                         who, L, (size_t)8 * (size_t)M, noalloc_scratch_bytes());
     if (log_m > 20) return set_error(HY_ERR_UNSUPPORTED, "%s: L=%d is beyond the supported length", who, L);
     hy_status st = prologue((cudaStream_t)stream);
     if (st != HY_OK) return st;

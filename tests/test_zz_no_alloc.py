@@ -92,8 +92,9 @@ def test_noalloc_short_sequences_and_limits():
     ref = _with_workspace(v, xs, Hs, dsk)
     torch.cuda.synchronize()
     check(to_np(y).reshape(6, -1), to_np(ref).reshape(6, -1), "bf16", "no-alloc on chip")
-    # longer than one row of the static scratch: rejected before any launch
-    L = 1 << 22
+    # longer than one row of the static scratch (8 bytes per complex point of
+    # the 2L transform, 64 MiB here): rejected before any launch
+    L = 1 << 23
     x = torch.empty((1, 1, L), device="cuda")
     H = torch.empty((1, hy.spectrum_bins(L)), dtype=torch.complex64, device="cuda")
     with pytest.raises(hy.HyenaError) as ei:

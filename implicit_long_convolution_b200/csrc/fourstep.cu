@@ -34,6 +34,7 @@
 // registers or instructions on the strided transfer and three CTAs fit on an
 // SM.  Rows are processed in chunks whose intermediates (8 bytes per complex
 // point) stay resident in the 126 MB L2 between passes.
+#include <cstring>
 #include <mutex>
 
 #include "../../include/hyena.h"
@@ -84,6 +85,7 @@ struct FsParams {
     int lo_2m;
     float2 *Hout;                 // spectrum mode: output bins (rows x (M+1))
     int vec4;                     // rows of u, gates and y take 4-element vector accesses
+    int in_tma;                   // pass A reads its input tile through imap (fp32 rows of M samples)
     uint32_t *fault;              // device fault word (a tile copy that did not land)
 };
 
@@ -104,7 +106,8 @@ __device__ __forceinline__ int tile_swz(int r, int c) { return 64 * r + ((((c >>
 // Block (blockIdx.x = column block of 8, blockIdx.y = row in chunk).
 // ----------------------------------------------------------------------------
 template <int LOG_N1, int LOG_N2, typename IO, bool INV, bool FWD, bool SPEC_INPUT>
-__global__ void __launch_bounds__(NT, 3) colpass_kernel(const FsParams p, const __grid_constant__ CUtensorMap bmap) {
+__global__ void __launch_bounds__(NT, 3) colpass_kernel(const FsParams p, const __grid_constant__ CUtensorMap bmap,
+                                                        const __grid_constant__ CUtensorMap imap) {
     constexpr int N1 = 1 << LOG_N1;
     constexpr int N2 = 1 << LOG_N2;
     constexpr int M = N1 * N2;
@@ -235,6 +238,36 @@ __global__ void __launch_bounds__(NT, 3) colpass_kernel(const FsParams p, const 
         }
         if (last || !FWD) return;
         __syncthreads();
+    } else if (p.in_tma) {
+        // ---- first order, fp32 rows of exactly M samples: the 8 columns'
+        //      N2/2 nonzero rows as one TMA tile of the input viewed as rows
+        //      of 2 N1 floats (y = row N2/2 + b BR), read straight into x
+        constexpr int BRI = (N2 / 2) < kTileBoxRows ? (N2 / 2) : kTileBoxRows;
+        if (tid == 0) {
+            mbar_init(&tile_bar, 1);
+            mbar_init_fence();
+        }
+        __syncthreads();
+        if (tid == 0) {
+            tc::mbar_expect_tx(&tile_bar, (uint32_t)(N2 / 2) * 64u);
+#pragma unroll
+            for (int b = 0; b < (N2 / 2) / BRI; ++b)
+                tc::tma_load_2d(tb + b * BRI * 64, &imap, 2 * n1_0, (int)(row * (N2 / 2) + b * BRI), &tile_bar);
+        }
+        const bool landed = mbar_wait(&tile_bar, 0);
+        {
+            const unsigned char *src = tb + tile_swz(lane, warp);
+#pragma unroll
+            for (int m = 0; m < P; ++m)
+                x[m] = m < P / 2 ? *reinterpret_cast<const float2 *>(src + 2048 * m) : make_float2(0.f, 0.f);
+        }
+        if (__syncthreads_or(!landed)) {
+            if (tid == 0) {
+                record_fault(p.fault, HY_FAULT_MULTIPASS);
+                mbar_wait(&tile_bar, 0);
+            }
+            return;
+        }
     } else {
         // ---- first order: packed input rows n2 < N2/2 of the 8 columns
         float4 v[EIT];
@@ -266,8 +299,10 @@ __global__ void __launch_bounds__(NT, 3) colpass_kernel(const FsParams p, const 
     }
     if constexpr (FWD) {
         // ---- forward column FFT (upper half zero) and W_M^{n1 k2}
-        load_own<LOG_N2, LP>(x, col, lane);
-        __syncwarp();
+        if (INV || !p.in_tma) {
+            load_own<LOG_N2, LP>(x, col, lane);
+            __syncwarp();
+        }
         block_fft<LOG_N2, LP, -1, true, SyncWarp>(x, col, lane, p.tw_n2, SyncWarp{});
         // W_M^{n1 k2}, k2 = lane + 32 m
         const uint32_t n1 = n1_0 + warp;
@@ -542,6 +577,22 @@ hy_status smem_attr(Kern k, size_t bytes) {
     return HY_OK;
 }
 
+// Tensor map of fp32 input rows of exactly M = N1 N2 samples seen as a 2-D
+// array of rows x N2/2 rows of 2 N1 floats (pass A's input tiles); p->in_tma
+// says whether it applies (length, 16-byte alignment).
+hy_status input_map(CUtensorMap *m, int *in_tma, const void *in, int64_t rows, int64_t L, int log_n1, int log_n2) {
+    const uint64_t n1 = (uint64_t)1 << log_n1, n2 = (uint64_t)1 << log_n2;
+    *in_tma = 0;
+    memset(m, 0, sizeof(*m));
+    if (L != (int64_t)(n1 * n2) || ((uintptr_t)in & 15) != 0) return HY_OK;
+    const uint64_t half = n2 / 2;
+    hy_status st = tma_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, in, 2 * n1, (uint64_t)rows * half, 8 * n1, 16,
+                              (uint32_t)(half < (uint64_t)kTileBoxRows ? half : (uint64_t)kTileBoxRows),
+                              CU_TENSOR_MAP_SWIZZLE_64B, "multi-pass input tiles");
+    if (st == HY_OK) *in_tma = 1;
+    return st;
+}
+
 // Tensor map of the chunk's complex buffer as a 2-D fp32 array: rows_chunk x
 // N2 rows of 2 N1 floats (row pitch 8 N1 bytes), boxes of 16 floats (8
 // complex columns, 64 bytes) x min(N2, 256) rows, 64-byte swizzle.
@@ -575,9 +626,15 @@ hy_status run_conv(const LongConvArgs &a, cudaStream_t s) {
     p.tw_2m = tw_pow2(LOG_MC + 1, p.lo_2m);
     if (!p.tw_n1 || !p.tw_n2 || !p.tw_m || !p.tw_2m) return set_error(HY_ERR_CUDA, "multi-pass twiddle tables missing");
     p.fault = device_fault_word();
-    CUtensorMap bmap;
+    CUtensorMap bmap, imap;
     hy_status st = buf_map(&bmap, p.buf, LOG_N1, LOG_N2, cr);
     if (st != HY_OK) return st;
+    if (sizeof(IO) == 4) {
+        if ((st = input_map(&imap, &p.in_tma, a.u, rows, a.L, LOG_N1, LOG_N2)) != HY_OK) return st;
+    } else {
+        memset(&imap, 0, sizeof(imap));
+        p.in_tma = 0;
+    }
     const size_t smem_c = colpass_smem_bytes<LOG_N2>();
     const size_t smem_r = rowpass_smem_bytes<LOG_N1, false>();
     auto kA = colpass_kernel<LOG_N1, LOG_N2, IO, false, true, false>;
@@ -592,15 +649,15 @@ hy_status run_conv(const LongConvArgs &a, cudaStream_t s) {
         p.row0 = r0;
         dim3 gc(N1 / WARPS, (unsigned)nr), gr(N2 / 8, (unsigned)nr);
         p.k = 0;
-        kA<<<gc, NT, smem_c, s>>>(p, bmap);
+        kA<<<gc, NT, smem_c, s>>>(p, bmap, imap);
         for (int k = 0; k < a.K; ++k) {
             p.k = k;
             p.spec = a.spec[k];
             p.gate_k = a.gate[k];
             p.skip_k = a.skip[k];
             kB<<<gr, NT, smem_r, s>>>(p);
-            if (k + 1 < a.K) kCA<<<gc, NT, smem_c, s>>>(p, bmap);
-            else kC<<<gc, NT, smem_c, s>>>(p, bmap);
+            if (k + 1 < a.K) kCA<<<gc, NT, smem_c, s>>>(p, bmap, imap);
+            else kC<<<gc, NT, smem_c, s>>>(p, bmap, imap);
         }
         if ((st = check_launch("multi-pass conv launch")) != HY_OK) return st;
     }
@@ -628,9 +685,10 @@ hy_status run_spectrum(int64_t rows, int64_t L, const float *h, float2 *H, void 
     p.tw_2m = tw_pow2(LOG_MC + 1, p.lo_2m);
     if (!p.tw_n1 || !p.tw_n2 || !p.tw_m || !p.tw_2m) return set_error(HY_ERR_CUDA, "multi-pass twiddle tables missing");
     p.fault = device_fault_word();
-    CUtensorMap bmap;
+    CUtensorMap bmap, imap;
     hy_status st = buf_map(&bmap, p.buf, LOG_N1, LOG_N2, cr);
     if (st != HY_OK) return st;
+    if ((st = input_map(&imap, &p.in_tma, h, rows, L, LOG_N1, LOG_N2)) != HY_OK) return st;
     const size_t smem_c = colpass_smem_bytes<LOG_N2>();
     const size_t smem_r = rowpass_smem_bytes<LOG_N1, true>();
     auto kA = colpass_kernel<LOG_N1, LOG_N2, float, false, true, true>;
@@ -639,7 +697,7 @@ hy_status run_spectrum(int64_t rows, int64_t L, const float *h, float2 *H, void 
     for (int64_t r0 = 0; r0 < rows; r0 += cr) {
         const int64_t nr = (rows - r0) < cr ? (rows - r0) : cr;
         p.row0 = r0;
-        kA<<<dim3(N1 / WARPS, (unsigned)nr), NT, smem_c, s>>>(p, bmap);
+        kA<<<dim3(N1 / WARPS, (unsigned)nr), NT, smem_c, s>>>(p, bmap, imap);
         kB<<<dim3(N2 / 8, (unsigned)nr), NT, smem_r, s>>>(p);
         if ((st = check_launch("multi-pass spectrum launch")) != HY_OK) return st;
     }
@@ -750,9 +808,15 @@ hy_status run_conv_static(const LongConvArgs &a, void *scratch, cudaStream_t s) 
     p.tw_2m = tw_pow2(LOG_MC + 1, p.lo_2m);
     if (!p.tw_n1 || !p.tw_n2 || !p.tw_m || !p.tw_2m) return set_error(HY_ERR_CUDA, "multi-pass twiddle tables missing");
     p.fault = device_fault_word();
-    CUtensorMap bmap;
+    CUtensorMap bmap, imap;
     hy_status st = buf_map(&bmap, p.buf, LOG_N1, LOG_N2, cr);
     if (st != HY_OK) return st;
+    if (sizeof(IO) == 4) {
+        if ((st = input_map(&imap, &p.in_tma, a.u, rows, a.L, LOG_N1, LOG_N2)) != HY_OK) return st;
+    } else {
+        memset(&imap, 0, sizeof(imap));
+        p.in_tma = 0;
+    }
     const size_t smem_c = colpass_smem_bytes<LOG_N2>();
     const size_t smem_r = rowpass_smem_bytes<LOG_N1, false>();
     auto kA = colpass_kernel<LOG_N1, LOG_N2, IO, false, true, false>;
@@ -769,15 +833,15 @@ hy_status run_conv_static(const LongConvArgs &a, void *scratch, cudaStream_t s) 
         p.row0 = r0;
         dim3 gc(N1 / WARPS, (unsigned)nr), gr(N2 / 8, (unsigned)nr);
         p.k = 0;
-        kA<<<gc, NT, smem_c, s>>>(p, bmap);
+        kA<<<gc, NT, smem_c, s>>>(p, bmap, imap);
         for (int k = 0; k < a.K; ++k) {
             p.k = k;
             p.spec = a.spec[k];
             p.gate_k = a.gate[k];
             p.skip_k = a.skip[k];
             kB<<<gr, NT, smem_r, s>>>(p);
-            if (k + 1 < a.K) kCA<<<gc, NT, smem_c, s>>>(p, bmap);
-            else kC<<<gc, NT, smem_c, s>>>(p, bmap);
+            if (k + 1 < a.K) kCA<<<gc, NT, smem_c, s>>>(p, bmap, imap);
+            else kC<<<gc, NT, smem_c, s>>>(p, bmap, imap);
         }
         if ((st = check_launch("no-alloc multi-pass launch")) != HY_OK) return st;
     }

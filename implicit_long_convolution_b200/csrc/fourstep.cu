@@ -86,6 +86,7 @@ struct FsParams {
     float2 *Hout;                 // spectrum mode: output bins (rows x (M+1))
     int vec4;                     // rows of u, gates and y take 4-element vector accesses
     int in_tma;                   // pass A reads its input tile through imap (fp32 rows of M samples)
+    int gate_pf;                  // pass C: imap is the gate's map; its tile is prefetched into L2
     uint32_t *fault;              // device fault word (a tile copy that did not land)
 };
 
@@ -170,6 +171,12 @@ __global__ void __launch_bounds__(NT, 3) colpass_kernel(const FsParams p, const 
 #pragma unroll
             for (int b = 0; b < N2 / BR; ++b)
                 tc::tma_load_2d(tb + b * BR * 64, &bmap, 2 * n1_0, (int)(rl * N2 + b * BR), &tile_bar);
+            if (p.gate_pf) {
+                // the gate tile of the epilogue (the same 8 columns' N2/2 rows) into L2
+                constexpr int BRI = (N2 / 2) < kTileBoxRows ? (N2 / 2) : kTileBoxRows;
+#pragma unroll
+                for (int b = 0; b < (N2 / 2) / BRI; ++b) tc::tma_prefetch_l2_2d(&imap, 2 * n1_0, (int)(row * (N2 / 2) + b * BRI));
+            }
         }
         const bool landed = mbar_wait(&tile_bar, 0);
         // column `warp`, rows lane + 32 m: the swizzle term depends on the lane only
@@ -629,12 +636,22 @@ hy_status run_conv(const LongConvArgs &a, cudaStream_t s) {
     CUtensorMap bmap, imap;
     hy_status st = buf_map(&bmap, p.buf, LOG_N1, LOG_N2, cr);
     if (st != HY_OK) return st;
+    // gates of the pass C epilogues: same geometry as the input, prefetched into L2
+    CUtensorMap gmap[8];
+    int gpf[8] = {0};
     if (sizeof(IO) == 4) {
         if ((st = input_map(&imap, &p.in_tma, a.u, rows, a.L, LOG_N1, LOG_N2)) != HY_OK) return st;
+        for (int k = 0; k < a.K; ++k) {
+            memset(&gmap[k], 0, sizeof(gmap[k]));
+            if (a.gate[k] && (st = input_map(&gmap[k], &gpf[k], a.gate[k], rows, a.L, LOG_N1, LOG_N2)) != HY_OK)
+                return st;
+        }
     } else {
         memset(&imap, 0, sizeof(imap));
         p.in_tma = 0;
+        for (int k = 0; k < a.K; ++k) memset(&gmap[k], 0, sizeof(gmap[k]));
     }
+    p.gate_pf = 0;
     const size_t smem_c = colpass_smem_bytes<LOG_N2>();
     const size_t smem_r = rowpass_smem_bytes<LOG_N1, false>();
     auto kA = colpass_kernel<LOG_N1, LOG_N2, IO, false, true, false>;
@@ -656,8 +673,10 @@ hy_status run_conv(const LongConvArgs &a, cudaStream_t s) {
             p.gate_k = a.gate[k];
             p.skip_k = a.skip[k];
             kB<<<gr, NT, smem_r, s>>>(p);
-            if (k + 1 < a.K) kCA<<<gc, NT, smem_c, s>>>(p, bmap, imap);
-            else kC<<<gc, NT, smem_c, s>>>(p, bmap, imap);
+            p.gate_pf = gpf[k];
+            if (k + 1 < a.K) kCA<<<gc, NT, smem_c, s>>>(p, bmap, gmap[k]);
+            else kC<<<gc, NT, smem_c, s>>>(p, bmap, gmap[k]);
+            p.gate_pf = 0;
         }
         if ((st = check_launch("multi-pass conv launch")) != HY_OK) return st;
     }
@@ -811,12 +830,22 @@ hy_status run_conv_static(const LongConvArgs &a, void *scratch, cudaStream_t s) 
     CUtensorMap bmap, imap;
     hy_status st = buf_map(&bmap, p.buf, LOG_N1, LOG_N2, cr);
     if (st != HY_OK) return st;
+    // gates of the pass C epilogues: same geometry as the input, prefetched into L2
+    CUtensorMap gmap[8];
+    int gpf[8] = {0};
     if (sizeof(IO) == 4) {
         if ((st = input_map(&imap, &p.in_tma, a.u, rows, a.L, LOG_N1, LOG_N2)) != HY_OK) return st;
+        for (int k = 0; k < a.K; ++k) {
+            memset(&gmap[k], 0, sizeof(gmap[k]));
+            if (a.gate[k] && (st = input_map(&gmap[k], &gpf[k], a.gate[k], rows, a.L, LOG_N1, LOG_N2)) != HY_OK)
+                return st;
+        }
     } else {
         memset(&imap, 0, sizeof(imap));
         p.in_tma = 0;
+        for (int k = 0; k < a.K; ++k) memset(&gmap[k], 0, sizeof(gmap[k]));
     }
+    p.gate_pf = 0;
     const size_t smem_c = colpass_smem_bytes<LOG_N2>();
     const size_t smem_r = rowpass_smem_bytes<LOG_N1, false>();
     auto kA = colpass_kernel<LOG_N1, LOG_N2, IO, false, true, false>;
@@ -840,8 +869,10 @@ hy_status run_conv_static(const LongConvArgs &a, void *scratch, cudaStream_t s) 
             p.gate_k = a.gate[k];
             p.skip_k = a.skip[k];
             kB<<<gr, NT, smem_r, s>>>(p);
-            if (k + 1 < a.K) kCA<<<gc, NT, smem_c, s>>>(p, bmap, imap);
-            else kC<<<gc, NT, smem_c, s>>>(p, bmap, imap);
+            p.gate_pf = gpf[k];
+            if (k + 1 < a.K) kCA<<<gc, NT, smem_c, s>>>(p, bmap, gmap[k]);
+            else kC<<<gc, NT, smem_c, s>>>(p, bmap, gmap[k]);
+            p.gate_pf = 0;
         }
         if ((st = check_launch("no-alloc multi-pass launch")) != HY_OK) return st;
     }

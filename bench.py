@@ -78,9 +78,10 @@ def workload_bytes(spec):
     return op, op
 
 
+# sources of the default (SIMT) on-chip convolution kernels; the opt-in
+# tensor-core engine (resident_tc.cu, tcgen05.cuh) is not part of them
 CONV_SOURCES = ["bulk_copy.cuh", "common.cuh", "fft_core.cuh", "resident.cuh", "resident_launch.cuh", "resident.cu",
-                "resident_stream_bf16.cu", "resident_stream_f32.cu", "resident_tc.cu", "tcgen05.cuh", "twiddle.cu",
-                "twiddle.h"]
+                "resident_stream_bf16.cu", "resident_stream_f32.cu", "twiddle.cu", "twiddle.h"]
 
 
 def conv_sources_digest():

@@ -567,8 +567,7 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "kernel": st.kernel,
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
-                     "traffic": recorded_traffic(name) if s["kind"] == "operator" and "resident" in st.kernel
-                     else None},
+                     "traffic": recorded_traffic(name) if "resident_stream" in st.kernel else None},
         "e2e": {"value": round(world * step_bytes / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": st.launches * steps,

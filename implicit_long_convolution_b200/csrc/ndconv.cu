@@ -30,6 +30,10 @@ namespace {
 constexpr int NT = 256;
 
 __host__ __device__ constexpr int nd_log_p(int log_n) { return log_n < 3 ? log_n : 3; }
+// The column transforms of the plane kernels (F1, F3) at 128 points take 16
+// points per thread: one exchange instead of two (the x pass keeps 8, its
+// staging of the kernel spectrum would not fit beside the wider groups).
+__host__ __device__ constexpr int nd_col_log_p(int log_n) { return log_n >= 7 ? 4 : nd_log_p(log_n); }
 
 struct NdParams {
     int64_t slab0;              // first slab of the chunk (b*D + d)
@@ -45,6 +49,7 @@ struct NdParams {
     float scale;
     const float2 *tw_r;         // row FFT (S/2 points) stage tables
     const float2 *tw_c;         // column FFT (S points) stage tables
+    const float2 *tw_cp;        // the plane kernels' column FFT (nd_col_log_p) stage tables
     const float2 *tw_split;     // W_S^k, k <= S/4
 };
 
@@ -60,10 +65,10 @@ __device__ __forceinline__ float2 wsplit(const float2 *tab, int k, int half) {
 // each other every N + N/2^SH slots: with several groups in a warp this makes
 // the stride-8 writes of the first stage and the reads back conflict-free
 // (up to 64 points) or nearly so (128).
-template <int LOG_N>
+template <int LOG_N, int LOG_P = nd_log_p(LOG_N)>
 struct Grp {
     static constexpr int N = 1 << LOG_N;
-    static constexpr int LP = nd_log_p(LOG_N);
+    static constexpr int LP = LOG_P;
     static constexpr int P = 1 << LP;
     static constexpr int T = N / P;
     static constexpr int G = NT / T;
@@ -134,24 +139,27 @@ __global__ void __launch_bounds__(NT) nd_fwd_plane(const NdParams p) {
         }
     }
     __syncthreads();
-    // ---- column pass: FFT along y of each bin column (inputs j < gI)
+    // ---- column pass: FFT along y of each bin column (inputs j < gI); a
+    //      warp whose groups all fall past the last column skips the round
     {
-        const int g = tid / C::T, t = tid % C::T;
-        float2 *xb = gbuf + g * C::BUF;
-        for (int k0 = 0; k0 < NB; k0 += C::G) {
+        using CP = Grp<LOG_S, nd_col_log_p(LOG_S)>;
+        const int g = tid / CP::T, t = tid % CP::T;
+        float2 *xb = gbuf + g * CP::BUF;
+        for (int k0 = 0; k0 < NB; k0 += CP::G) {
+            if (k0 + (tid >> 5) * (32 / CP::T) >= NB) continue;   // warp-uniform
             const int k = k0 + g;
             const bool act = k < NB;
-            float2 x[C::P];
+            float2 x[CP::P];
 #pragma unroll
-            for (int m = 0; m < C::P; ++m) {
-                const int j = t + m * C::T;
+            for (int m = 0; m < CP::P; ++m) {
+                const int j = t + m * CP::T;
                 x[m] = (act && j < gI) ? tile[j * NB + k] : make_float2(0.f, 0.f);
             }
-            block_fft<LOG_S, C::LP, -1, PAD, SyncWarp, C::SH>(x, xb, t, p.tw_c, SyncWarp{});
+            block_fft<LOG_S, CP::LP, -1, PAD, SyncWarp, CP::SH>(x, xb, t, p.tw_cp, SyncWarp{});
             __syncwarp();
             if (act) {
 #pragma unroll
-                for (int m = 0; m < C::P; ++m) tile[(t + m * C::T) * NB + k] = x[m];
+                for (int m = 0; m < CP::P; ++m) tile[(t + m * CP::T) * NB + k] = x[m];
             }
         }
     }
@@ -315,20 +323,22 @@ __global__ void __launch_bounds__(NT) nd_inv_plane(const NdParams p) {
     __syncthreads();
     // ---- inverse along y (k1 -> j), keep j < gI
     {
-        const int g = tid / C::T, t = tid % C::T;
-        float2 *xb = gbuf + g * C::BUF;
-        for (int k0 = 0; k0 < NB; k0 += C::G) {
+        using CP = Grp<LOG_S, nd_col_log_p(LOG_S)>;
+        const int g = tid / CP::T, t = tid % CP::T;
+        float2 *xb = gbuf + g * CP::BUF;
+        for (int k0 = 0; k0 < NB; k0 += CP::G) {
+            if (k0 + (tid >> 5) * (32 / CP::T) >= NB) continue;   // warp-uniform
             const int k = k0 + g;
             const bool act = k < NB;
-            float2 x[C::P];
+            float2 x[CP::P];
 #pragma unroll
-            for (int m = 0; m < C::P; ++m) x[m] = act ? tile[(t + m * C::T) * NB + k] : make_float2(0.f, 0.f);
-            block_fft<LOG_S, C::LP, +1, false, SyncWarp, C::SH>(x, xb, t, p.tw_c, SyncWarp{});
+            for (int m = 0; m < CP::P; ++m) x[m] = act ? tile[(t + m * CP::T) * NB + k] : make_float2(0.f, 0.f);
+            block_fft<LOG_S, CP::LP, +1, false, SyncWarp, CP::SH>(x, xb, t, p.tw_cp, SyncWarp{});
             __syncwarp();
             if (act) {
 #pragma unroll
-                for (int m = 0; m < C::P; ++m) {
-                    const int j = t + m * C::T;
+                for (int m = 0; m < CP::P; ++m) {
+                    const int j = t + m * CP::T;
                     if (j < gI) tile[j * NB + k] = x[m];
                 }
             }
@@ -415,10 +425,13 @@ hy_status nd_smem(Kern k, size_t bytes) {
 
 template <int LOG_S>
 size_t gbuf_elems() {
-    return (size_t)NT / Grp<LOG_S>::T * Grp<LOG_S>::BUF >
-                   (size_t)NT / Grp<LOG_S - 1>::T * Grp<LOG_S - 1>::BUF
-               ? (size_t)NT / Grp<LOG_S>::T * Grp<LOG_S>::BUF
-               : (size_t)NT / Grp<LOG_S - 1>::T * Grp<LOG_S - 1>::BUF;
+    using CP = Grp<LOG_S, nd_col_log_p(LOG_S)>;
+    size_t m = (size_t)NT / Grp<LOG_S>::T * Grp<LOG_S>::BUF;
+    const size_t r = (size_t)NT / Grp<LOG_S - 1>::T * Grp<LOG_S - 1>::BUF;
+    const size_t c = (size_t)NT / CP::T * CP::BUF;
+    if (r > m) m = r;
+    if (c > m) m = c;
+    return m;
 }
 
 template <int LOG_S, bool PAD>
@@ -428,8 +441,9 @@ hy_status run_nd(const NDArgs &a, NdParams p, cudaStream_t s, bool spec, int64_t
     constexpr int gI = PAD ? S / 2 : S;
     p.tw_r = tw_stages(LOG_S - 1, nd_log_p(LOG_S - 1));
     p.tw_c = tw_stages(LOG_S, nd_log_p(LOG_S));
+    p.tw_cp = tw_stages(LOG_S, nd_col_log_p(LOG_S));
     p.tw_split = tw_split(LOG_S - 1);
-    if (!p.tw_r || !p.tw_c || !p.tw_split) return set_error(HY_ERR_CUDA, "N-D twiddle tables missing");
+    if (!p.tw_r || !p.tw_c || !p.tw_cp || !p.tw_split) return set_error(HY_ERR_CUDA, "N-D twiddle tables missing");
     const int64_t per_slab = (int64_t)gI * S * NB * 8;
     const int64_t cs = nd_chunk(slabs, per_slab);
     const size_t sm1 = sizeof(float2) * ((size_t)S * NB + gbuf_elems<LOG_S>());

@@ -73,6 +73,7 @@ struct GenParams {
     int t_katoms;               // 64-element K atoms
     int t_npad;                 // outputs of a CTA's slice rounded up to 16 (MMA N, in chunks of <= 256)
     int t_slice;                // outputs per grid-z slice (all of them, or 256 when split)
+    int t_hpad;                 // hidden units rounded up to 16 (both layers on the tensor cores)
     uint32_t t_cols;            // TMEM columns (power of two >= max(32, t_npad))
     uint32_t *fault;            // device fault word
 };
@@ -705,12 +706,329 @@ __global__ void __launch_bounds__(NT, 2) filter_gen_tc_kernel(const GenParams p,
     if (warp == 0) tc::tmem_free(s_tmem, p.t_cols);
 }
 
-// Engine of the last layer: HYENA_FILTER_ENGINE=simt keeps it on the FP32
-// pipes, =tensor asks for the tensor cores; unset, the tensor cores take it
-// wherever the kernel applies.
+// ----------------------------------------------------------------------------
+// Both layers on the tensor cores, for MLPs with one hidden layer (input
+// width <= 63, hidden width <= 64).  A tile is 128 positions of one set (the
+// MMA M; warps w and w + 4 share TMEM lanes 32 (w % 4) .. + 31, one position
+// per thread).  Each thread writes its position's encoding straight into the
+// first operand row (fp16 hi/lo, K-major, 128-byte swizzle), with the columns
+// permuted so that the cos and sin of one frequency sit side by side (one
+// phase gives both) and a constant-1 column after them.  The first-layer
+// weights are held with the set's FiLM scale (1 + gamma), the sine
+// frequencies and the bias folded in (the bias as the weight of the constant
+// column), so the first MMA leaves the activation's argument itself in
+// tensor memory.  Each thread reads half of its row back, applies the
+// activation and writes the second operand row over the first; the second
+// MMA gives the outputs of the CTA's slice (the output bias folded in the
+// same way when the hidden width leaves a free column), and the epilogue
+// adds the decay window and stores as filter_gen_tc_kernel's does.
+// ----------------------------------------------------------------------------
+constexpr uint32_t TC2_OUT_COL = 128;     // TMEM column of the output accumulator
+
+// PTX approximate 2^x and 1/x (one MUFU operation each; subnormal results flush to zero)
+__device__ __forceinline__ float ex2_fast(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp_fast(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Encoding feature (its index in the positional encoding's own order) held
+// in operand column k: pairs (cos, sin) of each frequency first, then t/L
+// (1-D with include_t); -1 for the constant-1 column, -2 for a zero column.
+__device__ __forceinline__ int tc2_feature_of_column(const GenParams &p, int k, int npairs) {
+    if (k < 2 * npairs) {
+        const int pp = k >> 1, s = k & 1;
+        if (p.ndim == 1) return p.include_t + s * p.F + pp;
+        const int axis = pp / p.F, jm = pp - axis * p.F;
+        return axis * 2 * p.F + s * p.F + jm;
+    }
+    if (p.ndim == 1 && p.include_t && k == 2 * npairs) return 0;
+    return k == p.widths[0] ? -1 : -2;
+}
+
+__global__ void __launch_bounds__(NT, 2) filter_gen_tc2_kernel(const GenParams p) {
+    extern __shared__ __align__(16) unsigned char sm2_raw[];
+    uint8_t *tcb = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sm2_raw) + 1023) & ~uintptr_t(1023));
+    const int kpad = p.t_kpad, hpad = p.t_hpad, npad = p.t_npad;
+    // A hi/lo: 128 position rows (the encodings, then the hidden outputs);
+    // B0 hi/lo: hpad unit rows; B1 hi/lo: npad output rows of the slice
+    uint8_t *a_hi = tcb, *a_lo = tcb + TP * TC_ROW;
+    uint8_t *b0_hi = a_lo + TP * TC_ROW, *b0_lo = b0_hi + hpad * TC_ROW;
+    uint8_t *b1_hi = b0_lo + hpad * TC_ROW, *b1_lo = b1_hi + npad * TC_ROW;
+    float *bias1 = reinterpret_cast<float *>(b1_lo + npad * TC_ROW);   // output bias (0 when folded)
+    float *al1 = bias1 + npad;                                         // decay rate x log2 e
+    int *pdesc = reinterpret_cast<int *>(al1 + npad);                  // 3-D pair: axis | j << 2
+    float2 *phase = reinterpret_cast<float2 *>(pdesc + 32);            // 3-D: (cos, sin)(pi m / g)
+    __shared__ uint32_t s_tmem;
+    __shared__ uint64_t s_bar;
+    __shared__ int s_abort;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int set = blockIdx.y;
+    const int K0 = p.widths[0], H = p.widths[1], nout = p.widths[2];
+    const int npairs = p.ndim == 1 ? p.F : 3 * p.F;
+    const int obase = blockIdx.z * p.t_slice;
+    const int oend = min(nout, obase + p.t_slice);
+    const int64_t ntiles = (p.npos + TP - 1) / TP;
+    const bool film = p.gamma != nullptr;
+    const bool fold_b1 = H < hpad;
+
+    if (warp == 0) tc::tmem_alloc(&s_tmem, p.t_cols);
+    if (tid == 0) {
+        mbar_init(&s_bar, 1);
+        mbar_init_fence();
+        s_abort = 0;
+    }
+    auto put_row = [&](uint8_t *hi, uint8_t *lo, int r, int c, const float (&v)[8]) {
+        uint4 h4, l4;
+        split_h2(v[0], v[1], h4.x, l4.x);
+        split_h2(v[2], v[3], h4.y, l4.y);
+        split_h2(v[4], v[5], h4.z, l4.z);
+        split_h2(v[6], v[7], h4.w, l4.w);
+        const uint32_t off = sw128_chunk(r, c);
+        *reinterpret_cast<uint4 *>(hi + off) = h4;
+        *reinterpret_cast<uint4 *>(lo + off) = l4;
+    };
+    // B0: row u = (1 + gamma_u) omega_u W0[u][feature(k)]; the constant
+    // column omega_u ((1 + gamma_u) b0_u + beta_u); zero rows past H
+    for (int idx = tid; idx < hpad * (kpad / 8); idx += NT) {
+        const int u = idx / (kpad / 8), c = idx - u * (kpad / 8);
+        float v[8];
+        float sc = 0.f, bias = 0.f;
+        if (u < H) {
+            const float gm = film ? 1.f + __ldg(p.gamma + (int64_t)set * H + u) : 1.f;
+            const float bt = film ? __ldg(p.beta + (int64_t)set * H + u) : 0.f;
+            const float om = p.om[0] ? __ldg(p.om[0] + u) : 1.f;
+            sc = gm * om;
+            bias = om * fmaf(gm, __ldg(p.b[0] + u), bt);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int f = tc2_feature_of_column(p, 8 * c + j, npairs);
+            v[j] = u >= H ? 0.f : (f >= 0 ? sc * __ldg(p.W[0] + (int64_t)u * K0 + f) : (f == -1 ? bias : 0.f));
+        }
+        put_row(b0_hi, b0_lo, u, c, v);
+    }
+    // B1: row o = W1[obase + o][k] for k < H, the output bias in column H
+    // when it is free; zero rows past the slice
+    for (int idx = tid; idx < npad * (hpad / 8); idx += NT) {
+        const int o = idx / (hpad / 8), c = idx - o * (hpad / 8);
+        const bool live = obase + o < oend;
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int k = 8 * c + j;
+            v[j] = !live ? 0.f
+                         : (k < H ? __ldg(p.W[1] + (int64_t)(obase + o) * H + k)
+                                  : (k == H ? __ldg(p.b[1] + obase + o) : 0.f));
+        }
+        put_row(b1_hi, b1_lo, o, c, v);
+    }
+    for (int o = tid; o < npad; o += NT) {
+        const bool live = obase + o < oend;
+        bias1[o] = (live && !fold_b1) ? __ldg(p.b[1] + obase + o) : 0.f;
+        al1[o] = live ? __ldg(p.alpha + obase + o) * kLog2e : 0.f;
+    }
+    if (p.ndim == 3) {
+        for (int pp = tid; pp < npairs; pp += NT) pdesc[pp] = (pp / p.F) | ((pp % p.F + 1) << 2);
+        for (int m = tid; m < 2 * p.g; m += NT) {
+            float sn, cs;
+            sincospif((float)m / (float)p.g, &sn, &cs);
+            phase[m] = make_float2(cs, sn);
+        }
+    }
+    fence_proxy_async_smem();                  // B0 and B1 are read by the tensor cores
+    tc::fence_before();
+    const uint32_t idesc0 = tc::idesc_f16(128, hpad, false);
+    const uint32_t idesc1 = tc::idesc_f16(128, npad, false);
+    uint32_t phase_bit = 0;
+    // D[tmem + dcol] = A B^T with hi.hi + hi.lo + lo.hi; thread 0 issues and waits
+    auto run_mma = [&](const uint8_t *Bhi, const uint8_t *Blo, uint32_t idesc, uint32_t dcol, int ksteps) {
+        if (tid == 0) {
+            tc::fence_after();
+            bool first = true;
+            for (int term = 0; term < 3; ++term) {
+                const uint64_t ad = tc::desc_k_sw128(smem_u32(term == 2 ? a_lo : a_hi));
+                const uint64_t bd = tc::desc_k_sw128(smem_u32(term == 1 ? Blo : Bhi));
+                for (int ks = 0; ks < ksteps; ++ks) {
+                    tc::mma_f16(s_tmem + dcol, ad + 2 * ks, bd + 2 * ks, idesc, first ? 0u : 1u);
+                    first = false;
+                }
+            }
+            tc::commit(&s_bar);
+            if (!mbar_wait_sleep(&s_bar, phase_bit)) {
+                record_fault(p.fault, HY_FAULT_FILTER_MMA);
+                s_abort = 1;
+            }
+        }
+        phase_bit ^= 1;
+        __syncthreads();
+        tc::fence_after();
+    };
+    const int q4 = warp & 3, hc = warp >> 2;
+    const int pos = 32 * q4 + lane;            // this thread's position in the tile (its TMEM lane)
+    const uint32_t trow = s_tmem + ((uint32_t)(32 * q4) << 16);
+    const bool narrow = p.L * (int64_t)(p.F + 1) < (1LL << 31) && p.L <= (1 << 24);
+    const bool pow2 = (p.L & (p.L - 1)) == 0;
+    const float Lf = (float)p.L, invL = 1.f / Lf;   // exact when L is a power of two
+    for (int64_t bt = blockIdx.x; bt < ntiles; bt += gridDim.x) {
+        __syncthreads();                       // operands / TMEM of the previous tile released
+        tc::fence_after();
+        if (s_abort) break;                    // uniform: read between two barriers
+        const int64_t qq = bt * TP + pos;
+        const bool in = qq < p.npos;
+        // ---- window argument and validity of the position; its signed
+        //      offsets (3-D) for the encoding
+        int r0 = 0, r1 = 0, r2 = 0;
+        float nrm;
+        bool valid = in;
+        if (p.ndim == 3) {
+            const int S = p.S, ls = p.log_s;
+            r0 = signed_off((int)(qq >> (2 * ls)) & (S - 1), S);
+            r1 = signed_off((int)(qq >> ls) & (S - 1), S);
+            r2 = signed_off((int)qq & (S - 1), S);
+            valid = in && (p.circular || ((abs(r0) < p.g) && (abs(r1) < p.g) && (abs(r2) < p.g)));
+            nrm = sqrtf((float)(r0 * r0 + r1 * r1 + r2 * r2)) / (float)p.g;
+        } else {
+            nrm = narrow ? __fdiv_rn((float)qq, Lf) : (float)((double)qq / (double)p.L);
+        }
+        // ---- encoding into A: the two warps of a lane quadrant take
+        //      alternate 16-byte chunks (4 column pairs) of the row
+        for (int c = hc; c < kpad / 8; c += 2) {
+            float v[8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int pp = 4 * c + q;
+                float cs, sn;
+                if (pp < npairs) {
+                    if (p.ndim == 3) {
+                        const int d = pdesc[pp];
+                        const int ax = d & 3;
+                        const int rv = ax == 0 ? r0 : (ax == 1 ? r1 : r2);
+                        const float2 ph = phase[((d >> 2) * rv) & (2 * p.g - 1)];   // angle pi j r / g
+                        cs = ph.x;
+                        sn = ph.y;
+                    } else {
+                        const int j = pp + 1;
+                        float arg;
+                        if (narrow) {
+                            const unsigned jt = (unsigned)(j * (int)qq);
+                            arg = pow2 ? (float)(2u * (jt & (unsigned)(p.L - 1))) * invL
+                                       : __fdiv_rn((float)(2u * (jt % (unsigned)p.L)), Lf);
+                        } else {
+                            const int64_t r = ((int64_t)j * qq) % p.L;
+                            arg = (float)(2.0 * (double)r / (double)p.L);
+                        }
+                        sincospif(arg, &sn, &cs);        // angle 2 pi (j t mod L) / L
+                    }
+                } else {
+                    const int k = 2 * pp;
+                    const int kt = (p.ndim == 1 && p.include_t) ? 2 * npairs : -1;
+                    cs = k == kt ? nrm : (k == K0 ? 1.f : 0.f);
+                    sn = k + 1 == kt ? nrm : (k + 1 == K0 ? 1.f : 0.f);
+                }
+                v[2 * q] = cs;
+                v[2 * q + 1] = sn;
+            }
+            put_row(a_hi, a_lo, pos, c, v);
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        // ---- first layer: the activation's argument per unit, TMEM columns 0 .. hpad-1
+        run_mma(b0_hi, b0_lo, idesc0, 0u, kpad / 16);
+        if (s_abort) break;                    // uniform: set before run_mma's barrier
+        // ---- activation of this warp's half of the units, written over A
+        {
+            const int ub = hc * (hpad / 2), ue = ub + hpad / 2;
+            uint32_t x[4][8];
+#pragma unroll
+            for (int g8 = 0; g8 < 4; ++g8)
+                if (ub + 8 * g8 < ue) tc::tmem_ld8(trow + (uint32_t)(ub + 8 * g8), x[g8]);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int g8 = 0; g8 < 4; ++g8) {
+                const int u0 = ub + 8 * g8;
+                if (u0 >= ue) break;
+                float a[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    float xv = __uint_as_float(x[g8][j]);
+                    if (p.act == HY_ACT_SILU) xv = xv * rcp_fast(1.f + ex2_fast(-kLog2e * xv));
+                    else if (p.act == HY_ACT_SINE) xv = sinf(xv);
+                    a[j] = xv;
+                }
+                if (fold_b1 && u0 == (H & ~7)) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        if (u0 + j == H) a[j] = 1.f;   // the constant column of the output bias
+                }
+                put_row(a_hi, a_lo, pos, u0 / 8, a);
+            }
+        }
+        tc::fence_before();
+        fence_proxy_async_smem();
+        __syncthreads();
+        // ---- last layer: the slice's outputs, TMEM columns 128 ..
+        run_mma(b1_hi, b1_lo, idesc1, TC2_OUT_COL, hpad / 16);
+        {
+            float nr = nrm;
+            if (p.window == HY_WIN_GAUSS) nr *= nr;
+            const float nrn = valid ? -nr : 0.f;
+            for (int c0 = 16 * hc; c0 < npad; c0 += 32) {
+                __syncwarp();                  // tcgen05.ld is warp-wide
+                uint32_t v[16];
+                tc::tmem_ld16(trow + TC2_OUT_COL + (uint32_t)c0, v);
+                tc::tmem_wait_ld();
+                float y[16];
+#pragma unroll
+                for (int j4 = 0; j4 < 4; ++j4) {
+                    const float4 a4 = *reinterpret_cast<const float4 *>(al1 + c0 + 4 * j4);
+                    const float4 b4 = *reinterpret_cast<const float4 *>(bias1 + c0 + 4 * j4);
+                    y[4 * j4 + 0] = (__uint_as_float(v[4 * j4 + 0]) + b4.x) * ex2_fast(a4.x * nrn);
+                    y[4 * j4 + 1] = (__uint_as_float(v[4 * j4 + 1]) + b4.y) * ex2_fast(a4.y * nrn);
+                    y[4 * j4 + 2] = (__uint_as_float(v[4 * j4 + 2]) + b4.z) * ex2_fast(a4.z * nrn);
+                    y[4 * j4 + 3] = (__uint_as_float(v[4 * j4 + 3]) + b4.w) * ex2_fast(a4.w * nrn);
+                }
+                const int ob = obase + c0;
+                float *dst = p.h + ((int64_t)set * nout + ob) * p.npos + qq;
+                if (in && ob + 16 <= oend) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j, dst += p.npos) *dst = valid ? y[j] : 0.f;
+                } else if (in) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j, dst += p.npos)
+                        if (ob + j < oend) *dst = valid ? y[j] : 0.f;
+                }
+            }
+        }
+        tc::fence_before();
+    }
+    // no MMA may still be running when TMEM is freed (all were waited on;
+    // this covers one whose wait gave up)
+    if (tid == 0) {
+        tc::commit(&s_bar);
+        if (!mbar_wait_sleep(&s_bar, phase_bit)) record_fault(p.fault, HY_FAULT_FILTER_MMA);
+    }
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    __syncwarp();
+    if (warp == 0) tc::tmem_free(s_tmem, p.t_cols);
+}
+
+// Engine of the layers: HYENA_FILTER_ENGINE=simt keeps them on the FP32
+// pipes, =tensor_last puts only the last layer on the tensor cores, =tensor
+// (or unset) both layers of a one-hidden-layer MLP where that kernel applies,
+// else the last layer.
 int filter_engine() {
     const char *e = std::getenv("HYENA_FILTER_ENGINE");
     if (e && std::strcmp(e, "simt") == 0) return 0;
+    if (e && std::strcmp(e, "tensor_last") == 0) return 3;
     if (e && std::strcmp(e, "tensor") == 0) return 2;
     return 1;
 }
@@ -783,6 +1101,50 @@ hy_status launch_filter_gen(const hy_filter_desc &d, float *h, cudaStream_t s) {
         int dev = 0;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    // Both layers on the tensor cores: one hidden layer, input width <= 63
+    // (a free column for the bias), hidden width <= 64, output slices of
+    // <= 128 (two CTAs of 256 TMEM columns per SM), at least one 128-position
+    // tile per SM.
+    {
+        GenParams q = p;
+        const int nlast = q.widths[q.nl];
+        const int64_t ntiles = (q.npos + TP - 1) / TP;
+        const int eng = filter_engine();
+        if ((eng == 1 || eng == 2) && q.nl == 2 && q.widths[0] <= 63 && q.widths[1] <= 64 &&
+            ntiles * d.n_sets >= sms) {
+            q.t_slice = nlast > 128 ? 128 : nlast;
+            const int nslices = (nlast + q.t_slice - 1) / q.t_slice;
+            q.t_kpad = (q.widths[0] + 1 + 15) & ~15;
+            q.t_hpad = (q.widths[1] + 15) & ~15;
+            q.t_npad = (q.t_slice + 15) & ~15;
+            q.t_cols = 32;
+            while ((int)q.t_cols < (int)TC2_OUT_COL + q.t_npad) q.t_cols <<= 1;
+            q.fault = device_fault_word();
+            if (!q.fault) return set_error(HY_ERR_CUDA, "device fault word unavailable");
+            size_t smem = 1024 + (size_t)2 * TC_ROW * (TP + q.t_hpad + q.t_npad) +
+                          sizeof(float) * (2 * (size_t)q.t_npad + 32) + (q.ndim == 3 ? (size_t)16 * q.g : 0);
+            const int fit = 512 / (int)q.t_cols;
+            const size_t floor_smem = (size_t)233472 / (size_t)(fit + 1) + 1024;
+            if (fit < 8 && smem < floor_smem) smem = floor_smem;
+            if (nslices <= 65535 && smem <= (size_t)227 * 1024) {
+                cudaError_t e = cudaFuncSetAttribute(filter_gen_tc2_kernel,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+                if (e != cudaSuccess) return set_cuda_error("filter_gen two-layer smem attribute", e);
+                e = cudaFuncSetAttribute(filter_gen_tc2_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         (int)cudaSharedmemCarveoutMaxShared);
+                if (e != cudaSuccess) return set_cuda_error("filter_gen carve-out attribute", e);
+                int per_sm = (int)((size_t)233472 / (smem + 1024));
+                if (per_sm > 2) per_sm = 2;
+                if (per_sm > fit) per_sm = fit;
+                if (per_sm < 1) per_sm = 1;
+                int64_t per_set = ((int64_t)per_sm * sms + (int64_t)d.n_sets * nslices - 1) / ((int64_t)d.n_sets * nslices);
+                if (per_set > ntiles) per_set = ntiles;
+                dim3 grid((unsigned)per_set, (unsigned)d.n_sets, (unsigned)nslices);
+                filter_gen_tc2_kernel<<<grid, NT, smem, s>>>(q);
+                return check_launch("filter_gen (two tensor-core layers) launch");
+            }
+        }
     }
     // Tensor-core last layer: a hidden layer before it, K <= 128, at least one
     // (128-position tile, output slice) pair per SM.

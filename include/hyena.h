@@ -115,12 +115,14 @@ typedef struct hy_filter_desc {
 } hy_filter_desc;
 
 /* Writes h (device, fp32): 1-D (n_sets, n_out, L); 3-D (n_sets, n_out, S, S, S).
- * With at least one hidden layer of width <= 128 and at least one
- * 128-position tile per SM, the last layer runs on the tensor cores: its
- * inputs and weights are split into fp16 hi + lo (relative error <= 2^-22,
- * fp32 accumulation), which assumes their magnitudes stay below 65504 (the
- * encodings here are bounded and the hidden units O(1)); the environment
- * variable HYENA_FILTER_ENGINE=simt keeps every layer on the FP32 pipes. */
+ * With at least one 128-position tile per SM the layers run on the tensor
+ * cores: both of them for one hidden layer with input and hidden widths
+ * <= 64, else the last one (after at least one hidden layer of width <= 128).
+ * Their inputs and weights are split into fp16 hi + lo (relative error
+ * <= 2^-22, fp32 accumulation), which assumes their magnitudes stay below
+ * 65504 (the encodings here are bounded and the hidden units O(1)).  The
+ * environment variable HYENA_FILTER_ENGINE=simt keeps every layer on the FP32
+ * pipes; =tensor_last puts only the last layer on the tensor cores. */
 hy_status hyena_filter_gen(const hy_filter_desc *desc, float *h, void *stream);
 
 /* ------------------------------------------------------------------------

@@ -137,6 +137,42 @@ def test_nd_filter_gen_small_grids(g, circular, hidden, nout):
         check(got[b].reshape(nout, -1), ref.T, "f32", "3-D filters g%d circ%d set %d" % (g, circular, b))
 
 
+@pytest.mark.parametrize("engine", ["tensor", "tensor_last", "simt"])
+@pytest.mark.parametrize("act,hidden,nout", [("silu", 64, 130), ("sine", 40, 24)])
+def test_nd_filter_gen_tensor_core_grid(act, hidden, nout, engine, monkeypatch):
+    """A grid with enough 128-position tiles for the tensor-core filter
+    kernels (g = 16: 32^3 positions per set, two FiLM sets): both layers on
+    the tensor cores (the default for one hidden layer of <= 64 units: the
+    3-D encoding of each position written into the first MMA operand), the
+    last layer alone, and the FP32 pipes; 130 outputs take two output slices
+    (128 + 2), the SIREN case the Gaussian window.  Every voxel and output
+    against the oracle."""
+    monkeypatch.setenv("HYENA_FILTER_ENGINE", engine)
+    g, F = 16, 3
+    rng = np.random.default_rng(1600 + nout)
+    widths = [6 * F, hidden, nout]
+    Ws = [rng.uniform(-1, 1, (b, a)).astype(np.float32) / np.sqrt(a) for a, b in zip(widths[:-1], widths[1:])]
+    bs = [rng.uniform(-0.5, 0.5, b).astype(np.float32) for b in widths[1:]]
+    alpha = rng.uniform(0.5, 3.0, nout).astype(np.float32)
+    gam = rng.normal(0, 0.1, (2, hidden)).astype(np.float32)
+    bet = rng.normal(0, 0.1, (2, hidden)).astype(np.float32)
+    sine = act == "sine"
+    omega = rng.uniform(1, 4, hidden).astype(np.float32) if sine else None
+    S = 2 * g
+    h = torch.empty((2, nout, S, S, S), device="cuda")
+    hy.hyena_filter_gen(h, ndim=3, grid=g, Ws=[f32_dev(a) for a in Ws], bs=[f32_dev(a) for a in bs],
+                        alpha=f32_dev(alpha), n_freq=F, film_gamma=f32_dev(gam), film_beta=f32_dev(bet), n_sets=2,
+                        act=hy.HY_ACT_SINE if sine else hy.HY_ACT_SILU,
+                        omega=f32_dev(omega) if sine else None, window=hy.HY_WIN_GAUSS if sine else hy.HY_WIN_EXP)
+    torch.cuda.synchronize()
+    got = to_np(h)
+    idx = np.arange(S ** 3)
+    for b in range(2):
+        kw = dict(act="sine", omega=omega, window="gauss") if sine else {}
+        ref = oracle.filter_gen_3d_points(g, False, F, Ws, bs, gam[b], bet[b], alpha, idx, **kw)
+        check(got[b].reshape(nout, -1), ref.T, "f32", "3-D filters g16 %s %s set %d" % (act, engine, b))
+
+
 @pytest.mark.parametrize("circular", [False, True])
 def test_nd_filter_gen_siren_gaussian(circular):
     """HyenaND kernel synthesis: SIREN hidden layers (sin of per-unit

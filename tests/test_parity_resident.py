@@ -296,18 +296,23 @@ def test_c5_full_size():
     assert rel_l2(got, ref) < 5e-3
 
 
-@pytest.mark.parametrize("engine", ["simt", "tensor"])
+@pytest.mark.parametrize("engine", ["simt", "tensor", "tensor_last"])
 @pytest.mark.parametrize("act,hidden,nout", [("silu", [32, 24], 40), ("sine", [32, 24], 40),
-                                               ("silu", [96], 200), ("silu", [64], 512)])
+                                               ("silu", [96], 200), ("silu", [64], 512),
+                                               ("sine", [64], 40), ("silu", [40], 200)])
 def test_filter_gen_resident_weights_many_tiles(act, hidden, nout, engine, monkeypatch):
-    """Enough positions for the persistent filter kernels: the last layer on
-    the tensor cores (the default where it applies: 128-position tiles as the
-    MMA M, fp16 hi/lo operands, fp32 accumulation) or, with
-    HYENA_FILTER_ENGINE=simt, on the FP32 pipes with resident weights (or the
+    """Enough positions for the persistent filter kernels: with one hidden
+    layer of <= 64 units both layers on the tensor cores (the default; the
+    encoding written straight into the first MMA operand, hidden units read
+    back from tensor memory, output slices of <= 128), else the last layer
+    alone (HYENA_FILTER_ENGINE=tensor_last forces that kernel: 128-position
+    tiles as the MMA M, fp16 hi/lo operands, fp32 accumulation) or, with
+    HYENA_FILTER_ENGINE=simt, the FP32 pipes with resident weights (or the
     streaming kernel when they do not fit two CTAs per SM): 1-D L = 2^17, one
-    or two hidden layers, a last layer with K of 24, 64 or 96 (padded to 16,
-    one or two 64-element atoms) and 40, 200 or 512 outputs (padded to 16, one
-    or two MMA N chunks); every position and output against the oracle."""
+    or two hidden layers of 24 to 96 units (padded to 16, one or two 64-element
+    atoms) and 40, 200 or 512 outputs (one MMA N chunk or several, one output
+    slice or several, the last one ragged); every position and output against
+    the oracle."""
     monkeypatch.setenv("HYENA_FILTER_ENGINE", engine)
     L, F = 1 << 17, 8
     rng = np.random.default_rng(170 + (act == "sine") + nout)
@@ -326,15 +331,16 @@ def test_filter_gen_resident_weights_many_tiles(act, hidden, nout, engine, monke
     check(to_np(h), ref, "f32", "resident-weight filters L=2^17 (%s, %s)" % (act, engine))
 
 
-@pytest.mark.parametrize("engine", ["default", "simt"])
+@pytest.mark.parametrize("engine", ["default", "simt", "tensor_last"])
 def test_filter_gen_output_slices(engine, monkeypatch):
-    """More than 512 outputs with enough positions: the tensor-core last layer
-    splits them over grid z in 256-output slices (600 = 256 + 256 + 88, the
-    last slice padded to 96 MMA columns); L = 2^16, every position and output
-    against the oracle.  "simt" runs the FP32-pipe kernels on the same
-    filters."""
-    if engine == "simt":
-        monkeypatch.setenv("HYENA_FILTER_ENGINE", "simt")
+    """600 outputs with enough positions, split over grid z: by default both
+    layers on the tensor cores in 128-output slices (4 x 128 + 88), with
+    HYENA_FILTER_ENGINE=tensor_last the last layer alone in 256-output slices
+    (256 + 256 + 88, the last slice padded to 96 MMA columns); L = 2^16, every
+    position and output against the oracle.  "simt" runs the FP32-pipe
+    kernels on the same filters."""
+    if engine != "default":
+        monkeypatch.setenv("HYENA_FILTER_ENGINE", engine)
     L, F = 1 << 16, 8
     rng = np.random.default_rng(600)
     widths = [1 + 2 * F, 64, 600]

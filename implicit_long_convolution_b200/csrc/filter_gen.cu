@@ -751,6 +751,9 @@ __device__ __forceinline__ int tc2_feature_of_column(const GenParams &p, int k, 
     return k == p.widths[0] ? -1 : -2;
 }
 
+// NDIM (1 or 3) and ACT (hy_act) are template parameters: each instance
+// holds only its own encoding and activation code.
+template <int NDIM, int ACT>
 __global__ void __launch_bounds__(NT, 2) filter_gen_tc2_kernel(const GenParams p) {
     extern __shared__ __align__(16) unsigned char sm2_raw[];
     uint8_t *tcb = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sm2_raw) + 1023) & ~uintptr_t(1023));
@@ -771,7 +774,7 @@ __global__ void __launch_bounds__(NT, 2) filter_gen_tc2_kernel(const GenParams p
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int set = blockIdx.y;
     const int K0 = p.widths[0], H = p.widths[1], nout = p.widths[2];
-    const int npairs = p.ndim == 1 ? p.F : 3 * p.F;
+    const int npairs = NDIM == 1 ? p.F : 3 * p.F;
     const int obase = blockIdx.z * p.t_slice;
     const int oend = min(nout, obase + p.t_slice);
     const int64_t ntiles = (p.npos + TP - 1) / TP;
@@ -834,7 +837,7 @@ __global__ void __launch_bounds__(NT, 2) filter_gen_tc2_kernel(const GenParams p
         bias1[o] = (live && !fold_b1) ? __ldg(p.b[1] + obase + o) : 0.f;
         al1[o] = live ? __ldg(p.alpha + obase + o) * kLog2e : 0.f;
     }
-    if (p.ndim == 3) {
+    if constexpr (NDIM == 3) {
         for (int pp = tid; pp < npairs; pp += NT) pdesc[pp] = (pp / p.F) | ((pp % p.F + 1) << 2);
         for (int m = tid; m < 2 * p.g; m += NT) {
             float sn, cs;
@@ -887,7 +890,7 @@ __global__ void __launch_bounds__(NT, 2) filter_gen_tc2_kernel(const GenParams p
         int r0 = 0, r1 = 0, r2 = 0;
         float nrm;
         bool valid = in;
-        if (p.ndim == 3) {
+        if constexpr (NDIM == 3) {
             const int S = p.S, ls = p.log_s;
             r0 = signed_off((int)(qq >> (2 * ls)) & (S - 1), S);
             r1 = signed_off((int)(qq >> ls) & (S - 1), S);
@@ -906,7 +909,7 @@ __global__ void __launch_bounds__(NT, 2) filter_gen_tc2_kernel(const GenParams p
                 const int pp = 4 * c + q;
                 float cs, sn;
                 if (pp < npairs) {
-                    if (p.ndim == 3) {
+                    if constexpr (NDIM == 3) {
                         const int d = pdesc[pp];
                         const int ax = d & 3;
                         const int rv = ax == 0 ? r0 : (ax == 1 ? r1 : r2);
@@ -928,7 +931,7 @@ __global__ void __launch_bounds__(NT, 2) filter_gen_tc2_kernel(const GenParams p
                     }
                 } else {
                     const int k = 2 * pp;
-                    const int kt = (p.ndim == 1 && p.include_t) ? 2 * npairs : -1;
+                    const int kt = (NDIM == 1 && p.include_t) ? 2 * npairs : -1;
                     cs = k == kt ? nrm : (k == K0 ? 1.f : 0.f);
                     sn = k + 1 == kt ? nrm : (k + 1 == K0 ? 1.f : 0.f);
                 }
@@ -958,8 +961,8 @@ __global__ void __launch_bounds__(NT, 2) filter_gen_tc2_kernel(const GenParams p
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     float xv = __uint_as_float(x[g8][j]);
-                    if (p.act == HY_ACT_SILU) xv = xv * rcp_fast(1.f + ex2_fast(-kLog2e * xv));
-                    else if (p.act == HY_ACT_SINE) xv = sinf(xv);
+                    if constexpr (ACT == HY_ACT_SILU) xv = xv * rcp_fast(1.f + ex2_fast(-kLog2e * xv));
+                    else if constexpr (ACT == HY_ACT_SINE) xv = sinf(xv);
                     a[j] = xv;
                 }
                 if (fold_b1 && u0 == (H & ~7)) {
@@ -1128,10 +1131,18 @@ hy_status launch_filter_gen(const hy_filter_desc &d, float *h, cudaStream_t s) {
             const size_t floor_smem = (size_t)233472 / (size_t)(fit + 1) + 1024;
             if (fit < 8 && smem < floor_smem) smem = floor_smem;
             if (nslices <= 65535 && smem <= (size_t)227 * 1024) {
-                cudaError_t e = cudaFuncSetAttribute(filter_gen_tc2_kernel,
-                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+                void (*kern)(const GenParams) = nullptr;
+                if (q.ndim == 1)
+                    kern = q.act == HY_ACT_SILU ? filter_gen_tc2_kernel<1, HY_ACT_SILU>
+                         : q.act == HY_ACT_SINE ? filter_gen_tc2_kernel<1, HY_ACT_SINE>
+                                                : filter_gen_tc2_kernel<1, HY_ACT_IDENTITY>;
+                else
+                    kern = q.act == HY_ACT_SILU ? filter_gen_tc2_kernel<3, HY_ACT_SILU>
+                         : q.act == HY_ACT_SINE ? filter_gen_tc2_kernel<3, HY_ACT_SINE>
+                                                : filter_gen_tc2_kernel<3, HY_ACT_IDENTITY>;
+                cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
                 if (e != cudaSuccess) return set_cuda_error("filter_gen two-layer smem attribute", e);
-                e = cudaFuncSetAttribute(filter_gen_tc2_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                                          (int)cudaSharedmemCarveoutMaxShared);
                 if (e != cudaSuccess) return set_cuda_error("filter_gen carve-out attribute", e);
                 int per_sm = (int)((size_t)233472 / (smem + 1024));
@@ -1141,7 +1152,7 @@ hy_status launch_filter_gen(const hy_filter_desc &d, float *h, cudaStream_t s) {
                 int64_t per_set = ((int64_t)per_sm * sms + (int64_t)d.n_sets * nslices - 1) / ((int64_t)d.n_sets * nslices);
                 if (per_set > ntiles) per_set = ntiles;
                 dim3 grid((unsigned)per_set, (unsigned)d.n_sets, (unsigned)nslices);
-                filter_gen_tc2_kernel<<<grid, NT, smem, s>>>(q);
+                kern<<<grid, NT, smem, s>>>(q);
                 return check_launch("filter_gen (two tensor-core layers) launch");
             }
         }

@@ -751,9 +751,11 @@ __device__ __forceinline__ int tc2_feature_of_column(const GenParams &p, int k, 
     return k == p.widths[0] ? -1 : -2;
 }
 
-// NDIM (1 or 3) and ACT (hy_act) are template parameters: each instance
-// holds only its own encoding and activation code.
-template <int NDIM, int ACT>
+// NDIM (1 or 3) and ACT (hy_act) are template parameters, and FAST1D marks
+// a 1-D length that is a power of two with every j t below 2^31 (the phase
+// is then a mask and the angle an exact scaling): each instance holds only
+// its own encoding and activation code.
+template <int NDIM, int ACT, bool FAST1D>
 __global__ void __launch_bounds__(NT, 2) filter_gen_tc2_kernel(const GenParams p) {
     extern __shared__ __align__(16) unsigned char sm2_raw[];
     uint8_t *tcb = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sm2_raw) + 1023) & ~uintptr_t(1023));
@@ -877,7 +879,6 @@ __global__ void __launch_bounds__(NT, 2) filter_gen_tc2_kernel(const GenParams p
     const int pos = 32 * q4 + lane;            // this thread's position in the tile (its TMEM lane)
     const uint32_t trow = s_tmem + ((uint32_t)(32 * q4) << 16);
     const bool narrow = p.L * (int64_t)(p.F + 1) < (1LL << 31) && p.L <= (1 << 24);
-    const bool pow2 = (p.L & (p.L - 1)) == 0;
     const float Lf = (float)p.L, invL = 1.f / Lf;   // exact when L is a power of two
     for (int64_t bt = blockIdx.x; bt < ntiles; bt += gridDim.x) {
         __syncthreads();                       // operands / TMEM of the previous tile released
@@ -898,7 +899,8 @@ __global__ void __launch_bounds__(NT, 2) filter_gen_tc2_kernel(const GenParams p
             valid = in && (p.circular || ((abs(r0) < p.g) && (abs(r1) < p.g) && (abs(r2) < p.g)));
             nrm = sqrtf((float)(r0 * r0 + r1 * r1 + r2 * r2)) / (float)p.g;
         } else {
-            nrm = narrow ? __fdiv_rn((float)qq, Lf) : (float)((double)qq / (double)p.L);
+            if constexpr (FAST1D) nrm = (float)qq * invL;
+            else nrm = narrow ? __fdiv_rn((float)qq, Lf) : (float)((double)qq / (double)p.L);
         }
         // ---- encoding into A: the two warps of a lane quadrant take
         //      alternate 16-byte chunks (4 column pairs) of the row
@@ -919,10 +921,12 @@ __global__ void __launch_bounds__(NT, 2) filter_gen_tc2_kernel(const GenParams p
                     } else {
                         const int j = pp + 1;
                         float arg;
-                        if (narrow) {
+                        if constexpr (FAST1D) {
                             const unsigned jt = (unsigned)(j * (int)qq);
-                            arg = pow2 ? (float)(2u * (jt & (unsigned)(p.L - 1))) * invL
-                                       : __fdiv_rn((float)(2u * (jt % (unsigned)p.L)), Lf);
+                            arg = (float)(2u * (jt & (unsigned)(p.L - 1))) * invL;
+                        } else if (narrow) {
+                            const unsigned jt = (unsigned)(j * (int)qq);
+                            arg = __fdiv_rn((float)(2u * (jt % (unsigned)p.L)), Lf);
                         } else {
                             const int64_t r = ((int64_t)j * qq) % p.L;
                             arg = (float)(2.0 * (double)r / (double)p.L);
@@ -1132,14 +1136,19 @@ hy_status launch_filter_gen(const hy_filter_desc &d, float *h, cudaStream_t s) {
             if (fit < 8 && smem < floor_smem) smem = floor_smem;
             if (nslices <= 65535 && smem <= (size_t)227 * 1024) {
                 void (*kern)(const GenParams) = nullptr;
-                if (q.ndim == 1)
-                    kern = q.act == HY_ACT_SILU ? filter_gen_tc2_kernel<1, HY_ACT_SILU>
-                         : q.act == HY_ACT_SINE ? filter_gen_tc2_kernel<1, HY_ACT_SINE>
-                                                : filter_gen_tc2_kernel<1, HY_ACT_IDENTITY>;
+                const bool fast1d = q.L * (int64_t)(q.F + 1) < (1LL << 31) && q.L <= (1 << 24) && (q.L & (q.L - 1)) == 0;
+                if (q.ndim == 3)
+                    kern = q.act == HY_ACT_SILU ? filter_gen_tc2_kernel<3, HY_ACT_SILU, false>
+                         : q.act == HY_ACT_SINE ? filter_gen_tc2_kernel<3, HY_ACT_SINE, false>
+                                                : filter_gen_tc2_kernel<3, HY_ACT_IDENTITY, false>;
+                else if (fast1d)
+                    kern = q.act == HY_ACT_SILU ? filter_gen_tc2_kernel<1, HY_ACT_SILU, true>
+                         : q.act == HY_ACT_SINE ? filter_gen_tc2_kernel<1, HY_ACT_SINE, true>
+                                                : filter_gen_tc2_kernel<1, HY_ACT_IDENTITY, true>;
                 else
-                    kern = q.act == HY_ACT_SILU ? filter_gen_tc2_kernel<3, HY_ACT_SILU>
-                         : q.act == HY_ACT_SINE ? filter_gen_tc2_kernel<3, HY_ACT_SINE>
-                                                : filter_gen_tc2_kernel<3, HY_ACT_IDENTITY>;
+                    kern = q.act == HY_ACT_SILU ? filter_gen_tc2_kernel<1, HY_ACT_SILU, false>
+                         : q.act == HY_ACT_SINE ? filter_gen_tc2_kernel<1, HY_ACT_SINE, false>
+                                                : filter_gen_tc2_kernel<1, HY_ACT_IDENTITY, false>;
                 cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
                 if (e != cudaSuccess) return set_cuda_error("filter_gen two-layer smem attribute", e);
                 e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,

@@ -331,6 +331,29 @@ def test_filter_gen_resident_weights_many_tiles(act, hidden, nout, engine, monke
     check(to_np(h), ref, "f32", "resident-weight filters L=2^17 (%s, %s)" % (act, engine))
 
 
+@pytest.mark.parametrize("act", ["silu", "sine"])
+def test_filter_gen_two_layers_length_not_power_of_two(act):
+    """Both layers on the tensor cores with L = 3 * 2^14 (the encoding's
+    phase j t mod L by an integer remainder rather than a mask), a ragged
+    last tile of positions and 72 outputs; every position and output against
+    the oracle."""
+    L, F = 3 * (1 << 14) + 77, 6
+    rng = np.random.default_rng(4915 + (act == "sine"))
+    widths = [1 + 2 * F, 48, 72]
+    Ws = [rng.uniform(-1, 1, (b, a)).astype(np.float32) / np.sqrt(a) for a, b in zip(widths[:-1], widths[1:])]
+    bs = [rng.uniform(-0.5, 0.5, b).astype(np.float32) for b in widths[1:]]
+    alpha = rng.uniform(0.1, 2.0, widths[-1]).astype(np.float32)
+    omega = rng.uniform(1, 4, widths[1]).astype(np.float32) if act == "sine" else None
+    h = torch.empty((widths[-1], L), device="cuda")
+    hy.hyena_filter_gen(h, ndim=1, L=L, Ws=[f32_dev(a) for a in Ws], bs=[f32_dev(a) for a in bs],
+                        alpha=f32_dev(alpha), n_freq=F, include_t=True,
+                        act=hy.HY_ACT_SINE if act == "sine" else hy.HY_ACT_SILU,
+                        omega=f32_dev(omega) if omega is not None else None)
+    torch.cuda.synchronize()
+    ref = oracle.filter_gen_1d(L, F, True, Ws, bs, alpha, act=act, omega=omega)
+    check(to_np(h), ref, "f32", "two-layer filters L=%d (%s)" % (L, act))
+
+
 @pytest.mark.parametrize("engine", ["default", "simt", "tensor_last"])
 def test_filter_gen_output_slices(engine, monkeypatch):
     """600 outputs with enough positions, split over grid z: by default both

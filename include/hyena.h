@@ -401,16 +401,17 @@ hy_status spectral_gate_host(int B, int H, int Dh, int L, hy_dtype dt, const voi
  * about one second of %globaltimer, ORs a bit below into a per-device fault
  * word (a static device variable; nothing is allocated) and the CTA returns
  * at its next row boundary, after a bounded wait for its copies in flight.
- * The tensor-core kernels (projection GEMM, tensor-core convolution) bound
- * their pipeline waits the same way and wait for their copies and MMAs in
- * flight before they free tensor memory and return; so do the column passes
- * of the multi-pass convolution, which load their tiles with TMA.
+ * The tensor-core kernels (projection GEMM, tensor-core convolution, filter
+ * generator) bound their pipeline waits the same way and wait for their
+ * copies and MMAs in flight before they free tensor memory and return; so do
+ * the column passes of the multi-pass convolution, which load their tiles
+ * with TMA.
  * The outputs of such a launch are then undefined. */
 #define HY_FAULT_STREAM_INPUT 0x1u      /* a row's input copy did not land in time */
 #define HY_FAULT_STREAM_GATE 0x2u       /* a row's gate copy did not land in time  */
 #define HY_FAULT_PROJECTION 0x4u        /* a wait of the tensor-core projection GEMM ran out */
 #define HY_FAULT_TC_CONV 0x8u           /* a wait for the tensor-core convolution's MMAs ran out */
-#define HY_FAULT_FILTER_MMA 0x10u       /* a wait for the filter generator's last-layer MMAs ran out */
+#define HY_FAULT_FILTER_MMA 0x10u       /* a wait for the filter generator's MMAs ran out */
 #define HY_FAULT_MULTIPASS 0x20u        /* a column tile of the multi-pass convolution did not land in time */
 #define HY_FAULT_SELFTEST 0x80000000u   /* hyena_selftest_bounded_wait ran out      */
 /* Reads the current device's fault word into *faults after the work queued on

@@ -349,9 +349,12 @@ def setup_operator(w, dev, hy, torch):
     st.inputs = [(v, w.v)] + list(zip(xs, w.xs))
     st.output = y
     M = nb - 1
+    # multi-pass chunks: ~104 MB of 8-byte points per chunk (the workspace
+    # holds two chunk buffers when there is more than one chunk)
+    def chunk_rows(rows):
+        return max(1, min(rows, (104 << 20) // (8 * M)))
     if wso:
-        rows_chunk = max(1, wso // (8 * M))
-        op_l = -(-(B * D) // rows_chunk) * (1 + 2 * K)
+        op_l = -(-(B * D) // chunk_rows(B * D)) * (1 + 2 * K)
         st.kernel = "multi-pass colpass/rowpass kernels (M=2^%d)" % (M.bit_length() - 1)
     else:
         op_l = 1
@@ -362,7 +365,7 @@ def setup_operator(w, dev, hy, torch):
         st.kernel = "%s<M=2^%d>" % ("resident_tc_kernel" if tensor else
                                     "resident_stream_kernel" if stream else "resident_conv_kernel",
                                     M.bit_length() - 1)
-    spec_l = 2 * -(-(K * D) // max(1, wsf // (8 * M))) if wsf else 1
+    spec_l = 2 * -(-(K * D) // chunk_rows(K * D)) if wsf else 1
     st.launches = 1 + spec_l + op_l
     return st
 

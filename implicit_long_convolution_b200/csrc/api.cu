@@ -106,7 +106,7 @@ hy_status run_chain(int K, int B, int D, int L, hy_dtype dt, const void *v, cons
     a.y = y;
     a.ws = ws;
     a.ws_bytes = ws_bytes;
-    const size_t need = long_conv_workspace(B, D, log_m, K);
+    const size_t need = long_conv_workspace_min(B, D, log_m);
     if (need == 0) return set_error(HY_ERR_UNSUPPORTED, "%s: L=%d is beyond the supported length", who, L);
     if (!ws || ws_bytes < need)
         return set_error(HY_ERR_WORKSPACE, "%s: needs %zu workspace bytes, got %zu", who, need, ws ? ws_bytes : (size_t)0);
@@ -218,7 +218,7 @@ hy_status hyena_filter_spectrum(int64_t rows, int ndim, const int *dims, int cir
             if (st != HY_OK) return st;
             return launch_spectrum_1d(rows, (int)L, log_m, false, h, reinterpret_cast<float2 *>(H), s);
         }
-        const size_t need = long_spectrum_workspace(rows, log_m);
+        const size_t need = long_spectrum_workspace_min(rows, log_m);
         if (need == 0) return set_error(HY_ERR_UNSUPPORTED, "hyena_filter_spectrum: L=%lld beyond the supported length", (long long)L);
         if (!ws || ws_bytes < need)
             return set_error(HY_ERR_WORKSPACE, "hyena_filter_spectrum: needs %zu workspace bytes", need);

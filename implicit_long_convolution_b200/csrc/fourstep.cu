@@ -565,6 +565,80 @@ int64_t chunk_rows_of(int64_t rows, int log_mc) {
     return c < rows ? c : rows;
 }
 
+// Chunk pipelines.  With more than one chunk and a workspace of two chunk
+// buffers, consecutive chunks alternate between the caller's stream and a
+// second stream of the library's (one per device, created on first use and
+// kept), each chunk in its own buffer: the passes of one chunk then run in
+// the tail waves of the other's instead of after them (the passes are
+// latency-bound; a chunk's last wave leaves most SMs idle).  The second
+// stream joins the caller's by events, so the call stays ordered on the
+// caller's stream and can be captured into a graph.  Calls from several host
+// threads on one device take turns on the second stream.
+constexpr int kMaxLanes = 2;
+struct ChunkLanes {
+    cudaStream_t s2 = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+    std::mutex mu;
+};
+ChunkLanes *chunk_lanes_of_device() {
+    constexpr int kMaxDevices = 64;
+    static ChunkLanes lanes[kMaxDevices];
+    static std::once_flag once[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    ChunkLanes *l = &lanes[dev];
+    std::call_once(once[dev], [l] {
+        if (cudaStreamCreateWithFlags(&l->s2, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&l->fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&l->join, cudaEventDisableTiming) != cudaSuccess) {
+            cudaGetLastError();
+            l->s2 = nullptr;
+        }
+    });
+    return l->s2 ? l : nullptr;
+}
+
+// Lanes for `rows` rows in chunks of `cr` with `ws_bytes` of workspace.
+int chunk_lanes(int64_t rows, int64_t cr, int log_mc, size_t ws_bytes) {
+    const size_t chunk_bytes = (size_t)cr * ((size_t)8 << log_mc);
+    return (rows > cr && ws_bytes >= (size_t)kMaxLanes * chunk_bytes) ? kMaxLanes : 1;
+}
+
+// Forks the second stream off `s` (holding the device's lanes while the call
+// launches) or, with one lane, does nothing; `stream_of(ci)` then names chunk
+// ci's stream, and join() puts the caller's stream behind the second one.
+struct LaneScope {
+    ChunkLanes *l = nullptr;
+    cudaStream_t s = nullptr;
+    std::unique_lock<std::mutex> lock;
+    hy_status open(int lanes, cudaStream_t caller) {
+        s = caller;
+        if (lanes < 2) return HY_OK;
+        l = chunk_lanes_of_device();
+        if (!l) return HY_OK;                  // no second stream: one lane
+        lock = std::unique_lock<std::mutex>(l->mu);
+        cudaError_t e = cudaEventRecord(l->fork, caller);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(l->s2, l->fork, 0);
+        if (e != cudaSuccess) {
+            lock.unlock();
+            l = nullptr;
+            return set_cuda_error("multi-pass stream fork", e);
+        }
+        return HY_OK;
+    }
+    int lanes() const { return l ? 2 : 1; }
+    cudaStream_t stream_of(int ci) const { return (l && (ci & 1)) ? l->s2 : s; }
+    hy_status join() {
+        if (!l) return HY_OK;
+        cudaError_t e = cudaEventRecord(l->join, l->s2);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s, l->join, 0);
+        lock.unlock();
+        l = nullptr;
+        return e == cudaSuccess ? HY_OK : set_cuda_error("multi-pass stream join", e);
+    }
+    ~LaneScope() { join(); }
+};
+
 // Every row start of u, the gates and y is aligned for 4-element vectors.
 bool vec4_rows(const LongConvArgs &a, size_t el) {
     const uintptr_t al = 4 * el;
@@ -635,9 +709,13 @@ hy_status run_conv(const LongConvArgs &a, cudaStream_t s) {
     p.tw_2m = tw_pow2(LOG_MC + 1, p.lo_2m);
     if (!p.tw_n1 || !p.tw_n2 || !p.tw_m || !p.tw_2m) return set_error(HY_ERR_CUDA, "multi-pass twiddle tables missing");
     p.fault = device_fault_word();
-    CUtensorMap bmap, imap;
-    hy_status st = buf_map(&bmap, p.buf, LOG_N1, LOG_N2, cr);
-    if (st != HY_OK) return st;
+    const size_t chunk_el = (size_t)cr << LOG_MC;           // complex points of one chunk buffer
+    const int want = chunk_lanes(rows, cr, LOG_MC, a.ws_bytes);
+    float2 *bufs[kMaxLanes] = {p.buf, want > 1 ? p.buf + chunk_el : p.buf};
+    CUtensorMap bmap[kMaxLanes], imap;
+    hy_status st;
+    for (int l = 0; l < want; ++l)
+        if ((st = buf_map(&bmap[l], bufs[l], LOG_N1, LOG_N2, cr)) != HY_OK) return st;
     // gates of the pass C epilogues: same geometry as the input, prefetched into L2
     CUtensorMap gmap[8];
     int gpf[8] = {0};
@@ -663,30 +741,37 @@ hy_status run_conv(const LongConvArgs &a, cudaStream_t s) {
     if ((st = smem_attr(kA, smem_c)) != HY_OK || (st = smem_attr(kCA, smem_c)) != HY_OK ||
         (st = smem_attr(kC, smem_c)) != HY_OK || (st = smem_attr(kB, smem_r)) != HY_OK)
         return st;
-    for (int64_t r0 = 0; r0 < rows; r0 += cr) {
+    LaneScope lanes;
+    if ((st = lanes.open(want, s)) != HY_OK) return st;
+    int ci = 0;
+    for (int64_t r0 = 0; r0 < rows; r0 += cr, ++ci) {
         const int64_t nr = (rows - r0) < cr ? (rows - r0) : cr;
+        const int ln = lanes.lanes() > 1 ? (ci & 1) : 0;
+        const cudaStream_t cs = lanes.stream_of(ci);
+        p.buf = bufs[ln];
         p.row0 = r0;
         dim3 gc(N1 / WARPS, (unsigned)nr), gr(N2 / 8, (unsigned)nr);
         p.k = 0;
-        kA<<<gc, NT, smem_c, s>>>(p, bmap, imap);
+        kA<<<gc, NT, smem_c, cs>>>(p, bmap[ln], imap);
         for (int k = 0; k < a.K; ++k) {
             p.k = k;
             p.spec = a.spec[k];
             p.gate_k = a.gate[k];
             p.skip_k = a.skip[k];
-            kB<<<gr, NT, smem_r, s>>>(p);
+            kB<<<gr, NT, smem_r, cs>>>(p);
             p.gate_pf = gpf[k];
-            if (k + 1 < a.K) kCA<<<gc, NT, smem_c, s>>>(p, bmap, gmap[k]);
-            else kC<<<gc, NT, smem_c, s>>>(p, bmap, gmap[k]);
+            if (k + 1 < a.K) kCA<<<gc, NT, smem_c, cs>>>(p, bmap[ln], gmap[k]);
+            else kC<<<gc, NT, smem_c, cs>>>(p, bmap[ln], gmap[k]);
             p.gate_pf = 0;
         }
         if ((st = check_launch("multi-pass conv launch")) != HY_OK) return st;
     }
-    return HY_OK;
+    return lanes.join();
 }
 
 template <int LOG_N1, int LOG_N2>
-hy_status run_spectrum(int64_t rows, int64_t L, const float *h, float2 *H, void *ws, cudaStream_t s) {
+hy_status run_spectrum(int64_t rows, int64_t L, const float *h, float2 *H, void *ws, size_t ws_bytes,
+                       cudaStream_t s) {
     constexpr int N1 = 1 << LOG_N1, N2 = 1 << LOG_N2;
     constexpr int LOG_MC = LOG_N1 + LOG_N2;
     const int64_t cr = chunk_rows_of(rows, LOG_MC);
@@ -706,36 +791,50 @@ hy_status run_spectrum(int64_t rows, int64_t L, const float *h, float2 *H, void 
     p.tw_2m = tw_pow2(LOG_MC + 1, p.lo_2m);
     if (!p.tw_n1 || !p.tw_n2 || !p.tw_m || !p.tw_2m) return set_error(HY_ERR_CUDA, "multi-pass twiddle tables missing");
     p.fault = device_fault_word();
-    CUtensorMap bmap, imap;
-    hy_status st = buf_map(&bmap, p.buf, LOG_N1, LOG_N2, cr);
-    if (st != HY_OK) return st;
+    const size_t chunk_el = (size_t)cr << LOG_MC;
+    const int want = chunk_lanes(rows, cr, LOG_MC, ws_bytes);
+    float2 *bufs[kMaxLanes] = {p.buf, want > 1 ? p.buf + chunk_el : p.buf};
+    CUtensorMap bmap[kMaxLanes], imap;
+    hy_status st;
+    for (int l = 0; l < want; ++l)
+        if ((st = buf_map(&bmap[l], bufs[l], LOG_N1, LOG_N2, cr)) != HY_OK) return st;
     if ((st = input_map(&imap, &p.in_tma, h, rows, L, LOG_N1, LOG_N2)) != HY_OK) return st;
     const size_t smem_c = colpass_smem_bytes<LOG_N2>();
     const size_t smem_r = rowpass_smem_bytes<LOG_N1, true>();
     auto kA = colpass_kernel<LOG_N1, LOG_N2, float, false, true, true>;
     auto kB = rowpass_kernel<LOG_N1, LOG_N2, true>;
     if ((st = smem_attr(kA, smem_c)) != HY_OK || (st = smem_attr(kB, smem_r)) != HY_OK) return st;
-    for (int64_t r0 = 0; r0 < rows; r0 += cr) {
+    LaneScope lanes;
+    if ((st = lanes.open(want, s)) != HY_OK) return st;
+    int ci = 0;
+    for (int64_t r0 = 0; r0 < rows; r0 += cr, ++ci) {
         const int64_t nr = (rows - r0) < cr ? (rows - r0) : cr;
+        const int ln = lanes.lanes() > 1 ? (ci & 1) : 0;
+        const cudaStream_t cs = lanes.stream_of(ci);
+        p.buf = bufs[ln];
         p.row0 = r0;
-        kA<<<dim3(N1 / WARPS, (unsigned)nr), NT, smem_c, s>>>(p, bmap, imap);
-        kB<<<dim3(N2 / 8, (unsigned)nr), NT, smem_r, s>>>(p);
+        kA<<<dim3(N1 / WARPS, (unsigned)nr), NT, smem_c, cs>>>(p, bmap[ln], imap);
+        kB<<<dim3(N2 / 8, (unsigned)nr), NT, smem_r, cs>>>(p);
         if ((st = check_launch("multi-pass spectrum launch")) != HY_OK) return st;
     }
-    return HY_OK;
+    return lanes.join();
 }
 
 }  // namespace
 
-size_t long_conv_workspace(int64_t B, int64_t D, int log_mc, int) {
+// Workspace: one chunk buffer at least; two (the recommended size the
+// queries return) when there is more than one chunk.
+size_t long_workspace_of(int64_t rows, int log_mc, bool minimum) {
     if (log_mc < 15 || log_mc > 20) return 0;
-    return (size_t)chunk_rows_of(B * D, log_mc) * ((size_t)8 << log_mc);
+    const int64_t cr = chunk_rows_of(rows, log_mc);
+    const size_t one = (size_t)cr * ((size_t)8 << log_mc);
+    return (minimum || rows <= cr) ? one : (size_t)kMaxLanes * one;
 }
 
-size_t long_spectrum_workspace(int64_t rows, int log_mc) {
-    if (log_mc < 15 || log_mc > 20) return 0;
-    return (size_t)chunk_rows_of(rows, log_mc) * ((size_t)8 << log_mc);
-}
+size_t long_conv_workspace(int64_t B, int64_t D, int log_mc, int) { return long_workspace_of(B * D, log_mc, false); }
+size_t long_conv_workspace_min(int64_t B, int64_t D, int log_mc) { return long_workspace_of(B * D, log_mc, true); }
+size_t long_spectrum_workspace(int64_t rows, int log_mc) { return long_workspace_of(rows, log_mc, false); }
+size_t long_spectrum_workspace_min(int64_t rows, int log_mc) { return long_workspace_of(rows, log_mc, true); }
 
 hy_status launch_long_conv(const LongConvArgs &a, cudaStream_t s) {
     const bool bf = a.dt == HY_BF16;
@@ -750,10 +849,9 @@ hy_status launch_long_conv(const LongConvArgs &a, cudaStream_t s) {
 
 hy_status launch_long_spectrum(int64_t rows, int64_t L, int log_mc, const float *h, float2 *H, void *ws,
                                size_t ws_bytes, cudaStream_t s) {
-    (void)ws_bytes;
     switch (log_mc) {
 #define HY_LS(LM, N1L, N2L) \
-    case LM: return run_spectrum<N1L, N2L>(rows, L, h, H, ws, s);
+    case LM: return run_spectrum<N1L, N2L>(rows, L, h, H, ws, ws_bytes, s);
         HY_LS(15, 7, 8) HY_LS(16, 8, 8) HY_LS(17, 8, 9) HY_LS(18, 9, 9) HY_LS(19, 9, 10) HY_LS(20, 10, 10)
 #undef HY_LS
         default: return set_error(HY_ERR_UNSUPPORTED, "multi-pass length 2^%d not built", log_mc);

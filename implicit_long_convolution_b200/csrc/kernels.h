@@ -56,9 +56,14 @@ struct LongConvArgs {
     void *ws;
     size_t ws_bytes;
 };
+// Workspace of the multi-pass path: the recommended size (two chunk buffers
+// when there is more than one chunk: the chunks then alternate between two
+// streams) and the minimum (one chunk buffer: one stream).
 size_t long_conv_workspace(int64_t B, int64_t D, int log_mc, int K);
+size_t long_conv_workspace_min(int64_t B, int64_t D, int log_mc);
 hy_status launch_long_conv(const LongConvArgs &a, cudaStream_t s);
 size_t long_spectrum_workspace(int64_t rows, int log_mc);
+size_t long_spectrum_workspace_min(int64_t rows, int log_mc);
 hy_status launch_long_spectrum(int64_t rows, int64_t L, int log_mc, const float *h, float2 *H, void *ws,
                                size_t ws_bytes, cudaStream_t s);
 

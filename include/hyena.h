@@ -159,8 +159,14 @@ hy_status hyena_register_film(int B, int R, int C, int H, const float *reg, cons
  *   ndim = 3: dims = (g0, g1, g2) unpadded grid; rows are kernels on the
  *             transform grid S_a = 2 g_a (or g_a when circular), row-major;
  *             H[r] = rFFT3(h[r]) with shape (S0, S1, S2/2 + 1).
- *   ws: device workspace of at least hyena_filter_spectrum_workspace() bytes
- *   (may be NULL when that is 0).
+ *   ws: device workspace of hyena_filter_spectrum_workspace() bytes (may be
+ *   NULL when that is 0).  For rows longer than the on-chip transform that
+ *   size holds two chunk buffers when the rows take more than one chunk: the
+ *   chunks then alternate between `stream` and a second stream the library
+ *   creates once per device, joined back to `stream` by events (the call
+ *   stays ordered on `stream` and can be captured into a graph; calls from
+ *   several host threads take turns on the second stream).  Any workspace
+ *   of at least one chunk buffer is accepted and runs on `stream` alone.
  * ---------------------------------------------------------------------- */
 size_t hyena_filter_spectrum_workspace(int64_t rows, int ndim, const int *dims, int circular);
 hy_status hyena_filter_spectrum(int64_t rows, int ndim, const int *dims, int circular,
@@ -193,7 +199,10 @@ hy_status hyena_fftconv(int B, int D, int L, hy_dtype dt, const void *u, const h
  *   any entry, may be NULL for no skip).  Intermediate z_k stay fp32.
  *   Sequences with hyena_spectrum_bins(L) - 1 <= 16384 run on chip in one
  *   launch with no workspace; longer ones use the multi-pass path, which
- *   needs hyena_operator_workspace() bytes of device workspace.
+ *   takes hyena_operator_workspace() bytes of device workspace: two chunk
+ *   buffers of ~104 MB when the rows take more than one chunk, run as two
+ *   chunk pipelines on `stream` and a second stream of the library's, as
+ *   for hyena_filter_spectrum; one chunk buffer is the minimum accepted.
  * ---------------------------------------------------------------------- */
 size_t hyena_operator_workspace(int order, int B, int D, int L, hy_dtype dt);
 hy_status hyena_operator(int order, int B, int D, int L, hy_dtype dt, const void *v,

@@ -48,6 +48,54 @@ def _run(v, xs, Hs, dsk, L, B, D, order, code):
     return y
 
 
+def test_two_chunk_pipelines_match_one():
+    """More rows than one ~104 MB chunk holds (L = 2^15: 416 rows per chunk;
+    1000 rows = 3 chunks, the last one ragged): with the recommended
+    workspace (two chunk buffers) consecutive chunks alternate between the
+    caller's stream and the library's second stream; with the minimum (one
+    chunk buffer) they all run on the caller's stream.  The spectra and the
+    order-3 operator outputs of the two runs are equal bit for bit, sampled
+    rows of each chunk match the float64 oracle, and the outputs are ordered
+    on the caller's stream (read right after its synchronisation)."""
+    B, D, L, order = 2, 500, 1 << 15, 3
+    K = order - 1
+    rows = B * D
+    rng = np.random.default_rng(2015)
+    h32 = _filters(rng, K, D, L)
+    nb = hy.spectrum_bins(L)
+    hd = f32_dev(h32.reshape(K * D, L))
+    full = hy.filter_spectrum_workspace(K * D, 1, [L])
+    one = (416 * 8) << 15
+    assert full == 2 * one
+    Hs_ = []
+    for wsb in (full, one):
+        H = torch.empty((K * D, nb), dtype=torch.complex64, device="cuda")
+        ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+        hy.hyena_filter_spectrum(hd, H, rows=K * D, ndim=1, dims=[L], ws=ws)
+        torch.cuda.current_stream().synchronize()
+        Hs_.append(H)
+    assert torch.equal(torch.view_as_real(Hs_[0]), torch.view_as_real(Hs_[1]))
+    H = Hs_[0]
+    Hs = [H[k * D:(k + 1) * D] for k in range(K)]
+    v = torch.randn(B, D, L, device="cuda")
+    xs = [torch.randn(B, D, L, device="cuda") for _ in range(K)]
+    dsk = [f32_dev(rng.standard_normal(D).astype(np.float32)) for _ in range(K)]
+    wfull = hy.operator_workspace(order, B, D, L, 0)
+    assert wfull == 2 * one
+    ys = []
+    for wsb in (wfull, one):
+        y = torch.empty_like(v)
+        ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+        hy.hyena_operator(v, xs, Hs, y, Dskips=dsk, ws=ws)
+        torch.cuda.current_stream().synchronize()
+        ys.append(y)
+    assert torch.equal(ys[0], ys[1])
+    pick = np.array([0, 415, 416, 500, 831, 832, 999])      # rows of each chunk, both lanes
+    Dsk = np.stack([to_np(dk) for dk in dsk])
+    ref = oracle.fft_hyena_rows(to_np(v), [to_np(x) for x in xs], h32.astype(np.float64), Dsk, rows=pick)
+    check(to_np(ys[0]).reshape(rows, L)[pick], ref, "f32", "two-lane operator sampled rows")
+
+
 LONG = [
     # B, D, L, order, dtype, skip
     (1, 2, 20000, 2, "f32", True),

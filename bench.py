@@ -414,8 +414,11 @@ def setup_nd(w, dev, hy, torch):
     st.output = y
     per_c = g * S * (S // 2 + 1) * 8
     per_s = S * S * (S // 2 + 1) * 8
-    st.launches = ((2 if w.reg is not None else 1) + 2 * -(-(B * D) // max(1, wsf // per_s))
-                   + 3 * -(-(B * D) // max(1, wsc // per_c)))
+    # 3-D chunks: ~80 MB of transform planes (the workspace holds two chunk
+    # buffers when there is more than one chunk)
+    def chunks(per):
+        return -(-(B * D) // max(1, min(B * D, (80 << 20) // per)))
+    st.launches = (2 if w.reg is not None else 1) + 2 * chunks(per_s) + 3 * chunks(per_c)
     st.kernel = "nd_fwd_plane/nd_xpass/nd_inv_plane<S=%d>" % S
     return st
 

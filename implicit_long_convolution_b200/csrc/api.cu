@@ -235,7 +235,7 @@ hy_status hyena_filter_spectrum(int64_t rows, int ndim, const int *dims, int cir
             S[a] = circular ? dims[a] : 2 * dims[a];
             if (S[a] > 128) return set_error(HY_ERR_UNSUPPORTED, "hyena_filter_spectrum: transform edge %d > 128", S[a]);
         }
-        const size_t need = nd_spectrum_workspace(rows, S);
+        const size_t need = nd_spectrum_workspace(rows, S, true);
         if (need > 0 && (!ws || ws_bytes < need))
             return set_error(HY_ERR_WORKSPACE, "hyena_filter_spectrum: needs %zu workspace bytes", need);
         hy_status st = prologue(s);
@@ -312,7 +312,7 @@ hy_status hyena_nd_conv(int ndim, const int *dims, int B, int D, int circular, c
     a.y = y;
     a.ws = ws;
     a.ws_bytes = ws_bytes;
-    const size_t need = nd_conv_workspace(a.g, a.circular, B, D);
+    const size_t need = nd_conv_workspace(a.g, a.circular, B, D, true);
     if (need > 0 && (!ws || ws_bytes < need))
         return set_error(HY_ERR_WORKSPACE, "hyena_nd_conv: needs %zu workspace bytes, got %zu", need, ws ? ws_bytes : (size_t)0);
     if (ws && !aligned(ws, 256)) return set_error(HY_ERR_INVALID_ARG, "hyena_nd_conv: workspace must be 256-byte aligned");

@@ -38,6 +38,7 @@
 #include <mutex>
 
 #include "../../include/hyena.h"
+#include "chunk_lanes.h"
 #include "kernels.h"
 #include "fft_core.cuh"
 #include "status.h"
@@ -565,79 +566,6 @@ int64_t chunk_rows_of(int64_t rows, int log_mc) {
     return c < rows ? c : rows;
 }
 
-// Chunk pipelines.  With more than one chunk and a workspace of two chunk
-// buffers, consecutive chunks alternate between the caller's stream and a
-// second stream of the library's (one per device, created on first use and
-// kept), each chunk in its own buffer: the passes of one chunk then run in
-// the tail waves of the other's instead of after them (the passes are
-// latency-bound; a chunk's last wave leaves most SMs idle).  The second
-// stream joins the caller's by events, so the call stays ordered on the
-// caller's stream and can be captured into a graph.  Calls from several host
-// threads on one device take turns on the second stream.
-constexpr int kMaxLanes = 2;
-struct ChunkLanes {
-    cudaStream_t s2 = nullptr;
-    cudaEvent_t fork = nullptr, join = nullptr;
-    std::mutex mu;
-};
-ChunkLanes *chunk_lanes_of_device() {
-    constexpr int kMaxDevices = 64;
-    static ChunkLanes lanes[kMaxDevices];
-    static std::once_flag once[kMaxDevices];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    ChunkLanes *l = &lanes[dev];
-    std::call_once(once[dev], [l] {
-        if (cudaStreamCreateWithFlags(&l->s2, cudaStreamNonBlocking) != cudaSuccess ||
-            cudaEventCreateWithFlags(&l->fork, cudaEventDisableTiming) != cudaSuccess ||
-            cudaEventCreateWithFlags(&l->join, cudaEventDisableTiming) != cudaSuccess) {
-            cudaGetLastError();
-            l->s2 = nullptr;
-        }
-    });
-    return l->s2 ? l : nullptr;
-}
-
-// Lanes for `rows` rows in chunks of `cr` with `ws_bytes` of workspace.
-int chunk_lanes(int64_t rows, int64_t cr, int log_mc, size_t ws_bytes) {
-    const size_t chunk_bytes = (size_t)cr * ((size_t)8 << log_mc);
-    return (rows > cr && ws_bytes >= (size_t)kMaxLanes * chunk_bytes) ? kMaxLanes : 1;
-}
-
-// Forks the second stream off `s` (holding the device's lanes while the call
-// launches) or, with one lane, does nothing; `stream_of(ci)` then names chunk
-// ci's stream, and join() puts the caller's stream behind the second one.
-struct LaneScope {
-    ChunkLanes *l = nullptr;
-    cudaStream_t s = nullptr;
-    std::unique_lock<std::mutex> lock;
-    hy_status open(int lanes, cudaStream_t caller) {
-        s = caller;
-        if (lanes < 2) return HY_OK;
-        l = chunk_lanes_of_device();
-        if (!l) return HY_OK;                  // no second stream: one lane
-        lock = std::unique_lock<std::mutex>(l->mu);
-        cudaError_t e = cudaEventRecord(l->fork, caller);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(l->s2, l->fork, 0);
-        if (e != cudaSuccess) {
-            lock.unlock();
-            l = nullptr;
-            return set_cuda_error("multi-pass stream fork", e);
-        }
-        return HY_OK;
-    }
-    int lanes() const { return l ? 2 : 1; }
-    cudaStream_t stream_of(int ci) const { return (l && (ci & 1)) ? l->s2 : s; }
-    hy_status join() {
-        if (!l) return HY_OK;
-        cudaError_t e = cudaEventRecord(l->join, l->s2);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(s, l->join, 0);
-        lock.unlock();
-        l = nullptr;
-        return e == cudaSuccess ? HY_OK : set_cuda_error("multi-pass stream join", e);
-    }
-    ~LaneScope() { join(); }
-};
 
 // Every row start of u, the gates and y is aligned for 4-element vectors.
 bool vec4_rows(const LongConvArgs &a, size_t el) {
@@ -710,7 +638,7 @@ hy_status run_conv(const LongConvArgs &a, cudaStream_t s) {
     if (!p.tw_n1 || !p.tw_n2 || !p.tw_m || !p.tw_2m) return set_error(HY_ERR_CUDA, "multi-pass twiddle tables missing");
     p.fault = device_fault_word();
     const size_t chunk_el = (size_t)cr << LOG_MC;           // complex points of one chunk buffer
-    const int want = chunk_lanes(rows, cr, LOG_MC, a.ws_bytes);
+    const int want = chunk_lanes(rows, cr, (size_t)8 << LOG_MC, a.ws_bytes);
     float2 *bufs[kMaxLanes] = {p.buf, want > 1 ? p.buf + chunk_el : p.buf};
     CUtensorMap bmap[kMaxLanes], imap;
     hy_status st;
@@ -792,7 +720,7 @@ hy_status run_spectrum(int64_t rows, int64_t L, const float *h, float2 *H, void 
     if (!p.tw_n1 || !p.tw_n2 || !p.tw_m || !p.tw_2m) return set_error(HY_ERR_CUDA, "multi-pass twiddle tables missing");
     p.fault = device_fault_word();
     const size_t chunk_el = (size_t)cr << LOG_MC;
-    const int want = chunk_lanes(rows, cr, LOG_MC, ws_bytes);
+    const int want = chunk_lanes(rows, cr, (size_t)8 << LOG_MC, ws_bytes);
     float2 *bufs[kMaxLanes] = {p.buf, want > 1 ? p.buf + chunk_el : p.buf};
     CUtensorMap bmap[kMaxLanes], imap;
     hy_status st;
@@ -821,6 +749,26 @@ hy_status run_spectrum(int64_t rows, int64_t L, const float *h, float2 *H, void 
 }
 
 }  // namespace
+
+// The device's second stream and events for the chunk pipelines
+// (chunk_lanes.h), made on first use and kept for the process.
+ChunkLanes *chunk_lanes_of_device() {
+    constexpr int kMaxDevices = 64;
+    static ChunkLanes lanes[kMaxDevices];
+    static std::once_flag once[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    ChunkLanes *l = &lanes[dev];
+    std::call_once(once[dev], [l] {
+        if (cudaStreamCreateWithFlags(&l->s2, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&l->fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&l->join, cudaEventDisableTiming) != cudaSuccess) {
+            cudaGetLastError();
+            l->s2 = nullptr;
+        }
+    });
+    return l->s2 ? l : nullptr;
+}
 
 // Workspace: one chunk buffer at least; two (the recommended size the
 // queries return) when there is more than one chunk.

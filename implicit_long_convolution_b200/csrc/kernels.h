@@ -112,9 +112,11 @@ struct NDArgs {
     void *ws;
     size_t ws_bytes;
 };
-size_t nd_conv_workspace(const int g[3], int circular, int64_t B, int64_t D);
+// Workspace of the 3-D passes: the recommended size (two chunk buffers when
+// there is more than one chunk) or, with `minimum`, one chunk buffer.
+size_t nd_conv_workspace(const int g[3], int circular, int64_t B, int64_t D, bool minimum = false);
 hy_status launch_nd_conv(const NDArgs &a, cudaStream_t s);
-size_t nd_spectrum_workspace(int64_t rows, const int S[3]);
+size_t nd_spectrum_workspace(int64_t rows, const int S[3], bool minimum = false);
 hy_status launch_nd_spectrum(int64_t rows, const int S[3], const float *h, float2 *H, void *ws,
                              size_t ws_bytes, cudaStream_t s);
 

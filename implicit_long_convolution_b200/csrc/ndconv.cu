@@ -18,6 +18,7 @@
 // done by a group of S/16 or S/32 threads (8 points per thread) with warp
 // synchronisation; planes stay in shared memory; slabs are processed in
 // chunks whose workspace stays in L2 between the passes.
+#include "chunk_lanes.h"
 #include "kernels.h"
 #include "fft_core.cuh"
 #include "status.h"
@@ -435,7 +436,7 @@ size_t gbuf_elems() {
 }
 
 template <int LOG_S, bool PAD>
-hy_status run_nd(const NDArgs &a, NdParams p, cudaStream_t s, bool spec, int64_t slabs) {
+hy_status run_nd(const NDArgs &a, NdParams p, cudaStream_t s, bool spec, int64_t slabs, size_t ws_bytes) {
     constexpr int S = 1 << LOG_S;
     constexpr int NB = S / 2 + 1;
     constexpr int gI = PAD ? S / 2 : S;
@@ -458,19 +459,27 @@ hy_status run_nd(const NDArgs &a, NdParams p, cudaStream_t s, bool spec, int64_t
         (st = nd_smem(k2s, sm2)) != HY_OK || (st = nd_smem(k3, sm1)) != HY_OK)
         return st;
     (void)a;
-    for (int64_t s0 = 0; s0 < slabs; s0 += cs) {
+    // chunks alternate between two streams and two workspace buffers when
+    // the workspace holds two (chunk_lanes.h)
+    float2 *const ws0 = p.ws;
+    LaneScope lanes;
+    if ((st = lanes.open(chunk_lanes(slabs, cs, (size_t)per_slab, ws_bytes), s)) != HY_OK) return st;
+    int ci = 0;
+    for (int64_t s0 = 0; s0 < slabs; s0 += cs, ++ci) {
         const int64_t ns = (slabs - s0) < cs ? (slabs - s0) : cs;
+        const cudaStream_t st_ = lanes.stream_of(ci);
+        p.ws = ws0 + (lanes.lanes() > 1 && (ci & 1) ? cs * (per_slab / 8) : 0);
         p.slab0 = s0;
-        k1<<<dim3(gI, (unsigned)ns), NT, sm1, s>>>(p);
+        k1<<<dim3(gI, (unsigned)ns), NT, sm1, st_>>>(p);
         if (spec) {
-            k2s<<<dim3(S, (unsigned)ns), NT, sm2, s>>>(p);
+            k2s<<<dim3(S, (unsigned)ns), NT, sm2, st_>>>(p);
         } else {
-            k2c<<<dim3(S, (unsigned)ns), NT, sm2c, s>>>(p);
-            k3<<<dim3(gI, (unsigned)ns), NT, sm1, s>>>(p);
+            k2c<<<dim3(S, (unsigned)ns), NT, sm2c, st_>>>(p);
+            k3<<<dim3(gI, (unsigned)ns), NT, sm1, st_>>>(p);
         }
         if ((st = check_launch("N-D launch")) != HY_OK) return st;
     }
-    return HY_OK;
+    return lanes.join();
 }
 
 bool cube(const int g[3]) { return g[0] == g[1] && g[1] == g[2]; }
@@ -482,11 +491,19 @@ int ilog2i(int x) {
 
 }  // namespace
 
-size_t nd_conv_workspace(const int g[3], int circular, int64_t B, int64_t D) {
+// Workspace: one chunk buffer at least; two (the recommended size the
+// queries return) when there is more than one chunk (chunk_lanes.h).
+size_t nd_workspace_of(int64_t slabs, int64_t per, bool minimum) {
+    const int64_t cs = nd_chunk(slabs, per);
+    const size_t one = (size_t)(cs * per);
+    return (minimum || slabs <= cs) ? one : (size_t)kMaxLanes * one;
+}
+
+size_t nd_conv_workspace(const int g[3], int circular, int64_t B, int64_t D, bool minimum) {
     if (!cube(g)) return 0;
     const int64_t S = circular ? g[0] : 2 * g[0];
     const int64_t per = (int64_t)g[0] * S * (S / 2 + 1) * 8;
-    return (size_t)(nd_chunk(B * D, per) * per);
+    return nd_workspace_of(B * D, per, minimum);
 }
 
 hy_status launch_nd_conv(const NDArgs &a, cudaStream_t s) {
@@ -506,20 +523,20 @@ hy_status launch_nd_conv(const NDArgs &a, cudaStream_t s) {
     const bool pad = !a.circular;
     switch (ilog2i(S)) {
 #define HY_ND(LS) \
-    case LS: return pad ? run_nd<LS, true>(a, p, s, false, slabs) : run_nd<LS, false>(a, p, s, false, slabs);
+    case LS: return pad ? run_nd<LS, true>(a, p, s, false, slabs, a.ws_bytes) : run_nd<LS, false>(a, p, s, false, slabs, a.ws_bytes);
         HY_ND(3) HY_ND(4) HY_ND(5) HY_ND(6) HY_ND(7)
 #undef HY_ND
         default: return set_error(HY_ERR_UNSUPPORTED, "hyena_nd_conv: transform edge %d not built", S);
     }
 }
 
-size_t nd_spectrum_workspace(int64_t rows, const int S[3]) {
+size_t nd_spectrum_workspace(int64_t rows, const int S[3], bool minimum) {
     if (!(S[0] == S[1] && S[1] == S[2])) return 0;
     const int64_t per = (int64_t)S[0] * S[0] * (S[0] / 2 + 1) * 8;
-    return (size_t)(nd_chunk(rows, per) * per);
+    return nd_workspace_of(rows, per, minimum);
 }
 
-hy_status launch_nd_spectrum(int64_t rows, const int S[3], const float *h, float2 *H, void *ws, size_t,
+hy_status launch_nd_spectrum(int64_t rows, const int S[3], const float *h, float2 *H, void *ws, size_t ws_bytes,
                              cudaStream_t s) {
     if (!(S[0] == S[1] && S[1] == S[2]))
         return set_error(HY_ERR_UNSUPPORTED, "hyena_filter_spectrum: only cubic grids are built");
@@ -531,7 +548,7 @@ hy_status launch_nd_spectrum(int64_t rows, const int S[3], const float *h, float
     NDArgs a{};
     switch (ilog2i(S[0])) {
 #define HY_NS(LS) \
-    case LS: return run_nd<LS, false>(a, p, s, true, rows);
+    case LS: return run_nd<LS, false>(a, p, s, true, rows, ws_bytes);
         HY_NS(3) HY_NS(4) HY_NS(5) HY_NS(6) HY_NS(7)
 #undef HY_NS
         default: return set_error(HY_ERR_UNSUPPORTED, "hyena_filter_spectrum: transform edge %d not built", S[0]);

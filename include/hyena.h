@@ -311,6 +311,10 @@ hy_status hyena_operator_noalloc(int order, int B, int D, int L, hy_dtype dt, co
  *   (S0, S1, S2/2 + 1) per (sample, channel), sample b at H + b·H_batch_stride
  *   (in hy_c32 units; 0 = shared across samples), channel d at
  *   + d·S0·S1·(S2/2+1).  gate / Dskip may be NULL.
+ *   ws: hyena_nd_conv_workspace() bytes: slabs run in chunks of ~80 MB of
+ *   transform planes, two chunk buffers when there is more than one chunk
+ *   (two chunk pipelines on `stream` and the library's second stream, as
+ *   for hyena_filter_spectrum); one chunk buffer is the minimum accepted.
  * ---------------------------------------------------------------------- */
 size_t hyena_nd_conv_workspace(int ndim, const int *dims, int B, int D, int circular);
 hy_status hyena_nd_conv(int ndim, const int *dims, int B, int D, int circular, const float *u,

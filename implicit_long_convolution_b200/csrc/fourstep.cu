@@ -639,11 +639,13 @@ hy_status run_conv(const LongConvArgs &a, cudaStream_t s) {
     p.fault = device_fault_word();
     const size_t chunk_el = (size_t)cr << LOG_MC;           // complex points of one chunk buffer
     const int want = chunk_lanes(rows, cr, (size_t)8 << LOG_MC, a.ws_bytes);
-    float2 *bufs[kMaxLanes] = {p.buf, want > 1 ? p.buf + chunk_el : p.buf};
+    float2 *bufs[kMaxLanes];
     CUtensorMap bmap[kMaxLanes], imap;
     hy_status st;
-    for (int l = 0; l < want; ++l)
+    for (int l = 0; l < want; ++l) {
+        bufs[l] = p.buf + (size_t)l * chunk_el;
         if ((st = buf_map(&bmap[l], bufs[l], LOG_N1, LOG_N2, cr)) != HY_OK) return st;
+    }
     // gates of the pass C epilogues: same geometry as the input, prefetched into L2
     CUtensorMap gmap[8];
     int gpf[8] = {0};
@@ -674,7 +676,7 @@ hy_status run_conv(const LongConvArgs &a, cudaStream_t s) {
     int ci = 0;
     for (int64_t r0 = 0; r0 < rows; r0 += cr, ++ci) {
         const int64_t nr = (rows - r0) < cr ? (rows - r0) : cr;
-        const int ln = lanes.lanes() > 1 ? (ci & 1) : 0;
+        const int ln = lanes.lane_of(ci);
         const cudaStream_t cs = lanes.stream_of(ci);
         p.buf = bufs[ln];
         p.row0 = r0;
@@ -721,11 +723,13 @@ hy_status run_spectrum(int64_t rows, int64_t L, const float *h, float2 *H, void 
     p.fault = device_fault_word();
     const size_t chunk_el = (size_t)cr << LOG_MC;
     const int want = chunk_lanes(rows, cr, (size_t)8 << LOG_MC, ws_bytes);
-    float2 *bufs[kMaxLanes] = {p.buf, want > 1 ? p.buf + chunk_el : p.buf};
+    float2 *bufs[kMaxLanes];
     CUtensorMap bmap[kMaxLanes], imap;
     hy_status st;
-    for (int l = 0; l < want; ++l)
+    for (int l = 0; l < want; ++l) {
+        bufs[l] = p.buf + (size_t)l * chunk_el;
         if ((st = buf_map(&bmap[l], bufs[l], LOG_N1, LOG_N2, cr)) != HY_OK) return st;
+    }
     if ((st = input_map(&imap, &p.in_tma, h, rows, L, LOG_N1, LOG_N2)) != HY_OK) return st;
     const size_t smem_c = colpass_smem_bytes<LOG_N2>();
     const size_t smem_r = rowpass_smem_bytes<LOG_N1, true>();
@@ -737,7 +741,7 @@ hy_status run_spectrum(int64_t rows, int64_t L, const float *h, float2 *H, void 
     int ci = 0;
     for (int64_t r0 = 0; r0 < rows; r0 += cr, ++ci) {
         const int64_t nr = (rows - r0) < cr ? (rows - r0) : cr;
-        const int ln = lanes.lanes() > 1 ? (ci & 1) : 0;
+        const int ln = lanes.lane_of(ci);
         const cudaStream_t cs = lanes.stream_of(ci);
         p.buf = bufs[ln];
         p.row0 = r0;
@@ -759,24 +763,24 @@ ChunkLanes *chunk_lanes_of_device() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
     ChunkLanes *l = &lanes[dev];
-    std::call_once(once[dev], [l] {
-        if (cudaStreamCreateWithFlags(&l->s2, cudaStreamNonBlocking) != cudaSuccess ||
-            cudaEventCreateWithFlags(&l->fork, cudaEventDisableTiming) != cudaSuccess ||
-            cudaEventCreateWithFlags(&l->join, cudaEventDisableTiming) != cudaSuccess) {
-            cudaGetLastError();
-            l->s2 = nullptr;
-        }
+    static bool ok[kMaxDevices];
+    std::call_once(once[dev], [l, dev] {
+        bool good = cudaEventCreateWithFlags(&l->fork, cudaEventDisableTiming) == cudaSuccess;
+        for (int i = 0; good && i + 1 < kMaxLanes; ++i)
+            good = cudaStreamCreateWithFlags(&l->extra[i], cudaStreamNonBlocking) == cudaSuccess &&
+                   cudaEventCreateWithFlags(&l->join[i], cudaEventDisableTiming) == cudaSuccess;
+        if (!good) cudaGetLastError();
+        ok[dev] = good;
     });
-    return l->s2 ? l : nullptr;
+    return ok[dev] ? l : nullptr;
 }
 
-// Workspace: one chunk buffer at least; two (the recommended size the
-// queries return) when there is more than one chunk.
+// Workspace: one chunk buffer at least; the queries return one per lane
+// that can be busy (chunk_lanes.h).
 size_t long_workspace_of(int64_t rows, int log_mc, bool minimum) {
     if (log_mc < 15 || log_mc > 20) return 0;
     const int64_t cr = chunk_rows_of(rows, log_mc);
-    const size_t one = (size_t)cr * ((size_t)8 << log_mc);
-    return (minimum || rows <= cr) ? one : (size_t)kMaxLanes * one;
+    return minimum ? (size_t)cr * ((size_t)8 << log_mc) : chunk_workspace(rows, cr, (size_t)8 << log_mc);
 }
 
 size_t long_conv_workspace(int64_t B, int64_t D, int log_mc, int) { return long_workspace_of(B * D, log_mc, false); }

@@ -468,7 +468,7 @@ hy_status run_nd(const NDArgs &a, NdParams p, cudaStream_t s, bool spec, int64_t
     for (int64_t s0 = 0; s0 < slabs; s0 += cs, ++ci) {
         const int64_t ns = (slabs - s0) < cs ? (slabs - s0) : cs;
         const cudaStream_t st_ = lanes.stream_of(ci);
-        p.ws = ws0 + (lanes.lanes() > 1 && (ci & 1) ? cs * (per_slab / 8) : 0);
+        p.ws = ws0 + (int64_t)lanes.lane_of(ci) * cs * (per_slab / 8);
         p.slab0 = s0;
         k1<<<dim3(gI, (unsigned)ns), NT, sm1, st_>>>(p);
         if (spec) {
@@ -491,12 +491,11 @@ int ilog2i(int x) {
 
 }  // namespace
 
-// Workspace: one chunk buffer at least; two (the recommended size the
-// queries return) when there is more than one chunk (chunk_lanes.h).
+// Workspace: one chunk buffer at least; the queries return one per lane
+// that can be busy (chunk_lanes.h).
 size_t nd_workspace_of(int64_t slabs, int64_t per, bool minimum) {
     const int64_t cs = nd_chunk(slabs, per);
-    const size_t one = (size_t)(cs * per);
-    return (minimum || slabs <= cs) ? one : (size_t)kMaxLanes * one;
+    return minimum ? (size_t)(cs * per) : chunk_workspace(slabs, cs, (size_t)per);
 }
 
 size_t nd_conv_workspace(const int g[3], int circular, int64_t B, int64_t D, bool minimum) {

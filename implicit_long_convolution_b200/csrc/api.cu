@@ -3,6 +3,7 @@
 #include <cstdint>
 #include <cstring>
 
+#include "chunk_lanes.h"
 #include "kernels.h"
 #include "host_pipeline.h"
 #include "resident.cuh"
@@ -36,7 +37,11 @@ bool overlap(const void *a, size_t na, const void *b, size_t nb) {
 
 hy_status prologue(cudaStream_t) {
     clear_error();
-    return tw_ensure_device();
+    hy_status st = tw_ensure_device();
+    // the chunk pipelines' second stream is made here, with the first call
+    // on the device (before any capture), not inside a captured call
+    if (st == HY_OK) chunk_lanes_of_device();
+    return st;
 }
 
 // Shared body of hyena_fftconv / hyena_operator (1-D, causal).
@@ -135,8 +140,7 @@ const char *hyena_status_string(hy_status s) {
 }
 
 hy_status hyena_init(void) {
-    clear_error();
-    return tw_ensure_device();
+    return prologue(nullptr);
 }
 
 int64_t hyena_spectrum_bins(int64_t L) {

@@ -446,9 +446,10 @@ hy_status hyena_device_faults(uint32_t *faults, int clear, void *stream);
  * (1..1000000); it records HY_FAULT_SELFTEST and returns, leaving the
  * context usable.  Read the result with hyena_device_faults. */
 hy_status hyena_selftest_bounded_wait(uint32_t limit_us, void *stream);
-/* Uploads the constant twiddle tables to the current device.  Called
- * implicitly by the first call on each device; that first call blocks the
- * host briefly and must not be made while a stream is being captured.  */
+/* Uploads the constant twiddle tables to the current device and creates the
+ * stream and events of the chunk pipelines there.  Called implicitly by the
+ * first call on each device; that first call blocks the host briefly and
+ * must not be made while a stream is being captured.  */
 hy_status hyena_init(void);
 /* Message for the last non-OK status returned on this host thread. */
 const char *hyena_last_error(void);

@@ -96,6 +96,42 @@ def test_two_chunk_pipelines_match_one():
     check(to_np(ys[0]).reshape(rows, L)[pick], ref, "f32", "two-lane operator sampled rows")
 
 
+def test_two_chunk_pipelines_in_a_cuda_graph():
+    """The multi-pass operator with two chunk pipelines (L = 2^15, 1000 rows:
+    three chunks) captured into a CUDA graph on a side stream: the second
+    stream forks off the captured stream and joins it by events, so the
+    capture holds both chunk sequences; two replays give the eager result
+    bit for bit."""
+    B, D, L, order = 2, 500, 1 << 15, 2
+    rng = np.random.default_rng(3215)
+    h32 = _filters(rng, 1, D, L)
+    Hs, _ = _spectra(h32)
+    v = torch.randn(B, D, L, device="cuda")
+    xs = [torch.randn(B, D, L, device="cuda")]
+    wsb = hy.operator_workspace(order, B, D, L, 0)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    y_eager = torch.empty_like(v)
+    hy.hyena_operator(v, xs, Hs, y_eager, ws=ws)
+    torch.cuda.synchronize()
+    y = torch.zeros_like(v)
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        hy.hyena_operator(v, xs, Hs, y, ws=ws)          # warm-up on the capture stream
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    y.zero_()
+    with torch.cuda.graph(g):
+        hy.hyena_operator(v, xs, Hs, y, ws=ws)
+    for _ in range(2):
+        y.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(y, y_eager)
+    del g
+
+
 LONG = [
     # B, D, L, order, dtype, skip
     (1, 2, 20000, 2, "f32", True),

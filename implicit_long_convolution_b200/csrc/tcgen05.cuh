@@ -2,8 +2,8 @@
 // PTX: tensor-memory (TMEM) allocation, shared-memory matrix descriptors,
 // tcgen05.mma of kind::f16 (fp16 or bf16 operands, fp32 accumulator),
 // completion through tcgen05.commit on an mbarrier, tcgen05.ld of the
-// accumulator, and 2-D TMA tensor loads and stores (no multicast; the tensor
-// maps only ever cover this GPU's own memory).
+// accumulator, and 2-D TMA tensor loads and stores (each load fills one
+// CTA's shared memory; the tensor maps only ever cover this GPU's own memory).
 //
 // Conventions (PTX ISA, tcgen05 chapter):
 //   * An accumulator of an M = 128 MMA lives in TMEM lanes 0..127 (lane =

@@ -1,7 +1,7 @@
 // tma_map.cu -- host side of the TMA tensor maps: cuTensorMapEncodeTiled
 // from the driver, looked up once through the runtime (the library does not
 // link the driver library itself).  The maps only ever describe this GPU's
-// own memory; no load that uses them multicasts.
+// own memory, and every load through them fills one CTA's shared memory.
 #include <mutex>
 
 #include "kernels.h"

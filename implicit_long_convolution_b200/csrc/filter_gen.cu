@@ -74,6 +74,8 @@ struct GenParams {
     int t_npad;                 // outputs of a CTA's slice rounded up to 16 (MMA N, in chunks of <= 256)
     int t_slice;                // outputs per grid-z slice (all of them, or 256 when split)
     int t_hpad;                 // hidden units rounded up to 16 (both layers on the tensor cores)
+    int t_h2pad;                // second hidden layer's units rounded up to 16 (three layers)
+    int t_nslices;              // output slices of t_slice outputs (three layers)
     uint32_t t_cols;            // TMEM columns (power of two >= max(32, t_npad))
     uint32_t *fault;            // device fault word
 };
@@ -1028,6 +1030,332 @@ __global__ void __launch_bounds__(NT, 2) filter_gen_tc2_kernel(const GenParams p
     if (warp == 0) tc::tmem_free(s_tmem, p.t_cols);
 }
 
+// ----------------------------------------------------------------------------
+// All three layers on the tensor cores (two hidden layers of <= 64 units,
+// input width <= 127), for filter sets with fewer 128-position tiles than
+// SMs and many outputs: workload 2's 768 outputs over 8192 positions are 64
+// tiles, too few to spread one tile per CTA over the SMs in one pass of the
+// outputs.  A CTA takes one tile and the output slices blockIdx.z,
+// + gridDim.z, ... (128 outputs each): it encodes the tile into the first
+// operand (fp16 hi/lo, up to two 64-column atoms; columns as in
+// filter_gen_tc2_kernel), runs the first layer (FiLM, sine frequencies and
+// bias folded into the held weights), activates into the operand, runs the
+// second layer (sine frequencies folded, bias added before the
+// activation), activates again, and then for each slice loads the slice's
+// last-layer weights, runs the last layer and stores with the decay window.
+// The hidden layers are computed once per tile and CTA.
+// ----------------------------------------------------------------------------
+template <int NDIM, int ACT, bool FAST1D>
+__global__ void __launch_bounds__(NT, 1) filter_gen_tc3_kernel(const GenParams p) {
+    extern __shared__ __align__(16) unsigned char sm3_raw[];
+    uint8_t *tcb = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sm3_raw) + 1023) & ~uintptr_t(1023));
+    const int kpad = p.t_kpad, h1p = p.t_hpad, h2p = p.t_h2pad, npad = p.t_npad;
+    const int ka = (kpad + 63) / 64;           // 64-column atoms of the first operand
+    // A hi/lo: ka atoms of 128 position rows; B0: ka atoms of h1p rows; B1:
+    // h2p rows; B2: npad rows of the current slice
+    uint8_t *a_hi = tcb, *a_lo = a_hi + ka * TP * TC_ROW;
+    uint8_t *b0_hi = a_lo + ka * TP * TC_ROW, *b0_lo = b0_hi + ka * h1p * TC_ROW;
+    uint8_t *b1_hi = b0_lo + ka * h1p * TC_ROW, *b1_lo = b1_hi + h2p * TC_ROW;
+    uint8_t *b2_hi = b1_lo + h2p * TC_ROW, *b2_lo = b2_hi + npad * TC_ROW;
+    float *bias1 = reinterpret_cast<float *>(b2_lo + npad * TC_ROW);   // second hidden layer: omega b
+    float *bias2 = bias1 + 64;                                         // slice's output bias
+    float *al2 = bias2 + npad;                                         // slice's decay rate x log2 e
+    int *pdesc = reinterpret_cast<int *>(al2 + npad);                  // 3-D pair: axis | j << 2
+    float2 *phase = reinterpret_cast<float2 *>(pdesc + 64);            // 3-D: (cos, sin)(pi m / g)
+    __shared__ uint32_t s_tmem;
+    __shared__ uint64_t s_bar;
+    __shared__ int s_abort;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int set = blockIdx.y;
+    const int K0 = p.widths[0], H1 = p.widths[1], H2 = p.widths[2], nout = p.widths[3];
+    const int npairs = NDIM == 1 ? p.F : 3 * p.F;
+    const int64_t ntiles = (p.npos + TP - 1) / TP;
+    const bool film = p.gamma != nullptr;
+
+    if (warp == 0) tc::tmem_alloc(&s_tmem, p.t_cols);
+    if (tid == 0) {
+        mbar_init(&s_bar, 1);
+        mbar_init_fence();
+        s_abort = 0;
+    }
+    // 16-byte chunk c (8 columns) of row r of an operand of `rows` rows
+    auto put_row = [&](uint8_t *hi, uint8_t *lo, int rows, int r, int c, const float (&v)[8]) {
+        uint4 h4, l4;
+        split_h2(v[0], v[1], h4.x, l4.x);
+        split_h2(v[2], v[3], h4.y, l4.y);
+        split_h2(v[4], v[5], h4.z, l4.z);
+        split_h2(v[6], v[7], h4.w, l4.w);
+        const uint32_t off = (uint32_t)((c >> 3) * rows * TC_ROW) + sw128_chunk(r, c & 7);
+        *reinterpret_cast<uint4 *>(hi + off) = h4;
+        *reinterpret_cast<uint4 *>(lo + off) = l4;
+    };
+    // B0: row u = (1 + gamma_u) omega_u W0[u][feature(k)]; the constant
+    // column omega_u ((1 + gamma_u) b0_u + beta_u); zero rows past H1
+    for (int idx = tid; idx < h1p * (kpad / 8); idx += NT) {
+        const int u = idx / (kpad / 8), c = idx - u * (kpad / 8);
+        float v[8];
+        float sc = 0.f, bias = 0.f;
+        if (u < H1) {
+            const float gm = film ? 1.f + __ldg(p.gamma + (int64_t)set * H1 + u) : 1.f;
+            const float bt = film ? __ldg(p.beta + (int64_t)set * H1 + u) : 0.f;
+            const float om = p.om[0] ? __ldg(p.om[0] + u) : 1.f;
+            sc = gm * om;
+            bias = om * fmaf(gm, __ldg(p.b[0] + u), bt);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int f = tc2_feature_of_column(p, 8 * c + j, npairs);
+            v[j] = u >= H1 ? 0.f : (f >= 0 ? sc * __ldg(p.W[0] + (int64_t)u * K0 + f) : (f == -1 ? bias : 0.f));
+        }
+        put_row(b0_hi, b0_lo, h1p, u, c, v);
+    }
+    // B1: row u = omega_u W1[u][k] (k < H1); its bias omega_u b1_u is added
+    // before the activation
+    for (int idx = tid; idx < h2p * (h1p / 8); idx += NT) {
+        const int u = idx / (h1p / 8), c = idx - u * (h1p / 8);
+        const float om = (u < H2 && p.om[1]) ? __ldg(p.om[1] + u) : 1.f;
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int k = 8 * c + j;
+            v[j] = (u < H2 && k < H1) ? om * __ldg(p.W[1] + (int64_t)u * H1 + k) : 0.f;
+        }
+        put_row(b1_hi, b1_lo, h2p, u, c, v);
+    }
+    for (int u = tid; u < 64; u += NT) {
+        const float om = (u < H2 && p.om[1]) ? __ldg(p.om[1] + u) : 1.f;
+        bias1[u] = u < H2 ? om * __ldg(p.b[1] + u) : 0.f;
+    }
+    if constexpr (NDIM == 3) {
+        for (int pp = tid; pp < npairs; pp += NT) pdesc[pp] = (pp / p.F) | ((pp % p.F + 1) << 2);
+        for (int m = tid; m < 2 * p.g; m += NT) {
+            float sn, cs;
+            sincospif((float)m / (float)p.g, &sn, &cs);
+            phase[m] = make_float2(cs, sn);
+        }
+    }
+    // B2 and the per-output rows of slice sl
+    auto load_slice = [&](int sl) {
+        const int obase = sl * p.t_slice, oend = min(nout, obase + p.t_slice);
+        for (int idx = tid; idx < npad * (h2p / 8); idx += NT) {
+            const int o = idx / (h2p / 8), c = idx - o * (h2p / 8);
+            const bool live = obase + o < oend;
+            float v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int k = 8 * c + j;
+                v[j] = (live && k < H2) ? __ldg(p.W[2] + (int64_t)(obase + o) * H2 + k) : 0.f;
+            }
+            put_row(b2_hi, b2_lo, npad, o, c, v);
+        }
+        for (int o = tid; o < npad; o += NT) {
+            const bool live = obase + o < oend;
+            bias2[o] = live ? __ldg(p.b[2] + obase + o) : 0.f;
+            al2[o] = live ? __ldg(p.alpha + obase + o) * kLog2e : 0.f;
+        }
+    };
+    fence_proxy_async_smem();                  // B0 and B1 are read by the tensor cores
+    tc::fence_before();
+    uint32_t phase_bit = 0;
+    // D[tmem + dcol] = A B^T over ksteps of 16 columns (atoms of 4 steps;
+    // A atoms TP rows apart, B atoms b_rows rows apart): hi.hi + hi.lo + lo.hi
+    auto run_mma = [&](const uint8_t *Bhi, const uint8_t *Blo, int b_rows, uint32_t idesc, uint32_t dcol,
+                       int ksteps) {
+        if (tid == 0) {
+            tc::fence_after();
+            bool first = true;
+            for (int term = 0; term < 3; ++term) {
+                const uint8_t *A = term == 2 ? a_lo : a_hi;
+                const uint8_t *Bm = term == 1 ? Blo : Bhi;
+                for (int ks = 0; ks < ksteps; ++ks) {
+                    const uint64_t ad = tc::desc_k_sw128(smem_u32(A + (ks >> 2) * TP * TC_ROW)) + 2 * (ks & 3);
+                    const uint64_t bd = tc::desc_k_sw128(smem_u32(Bm + (ks >> 2) * b_rows * TC_ROW)) + 2 * (ks & 3);
+                    tc::mma_f16(s_tmem + dcol, ad, bd, idesc, first ? 0u : 1u);
+                    first = false;
+                }
+            }
+            tc::commit(&s_bar);
+            if (!mbar_wait_sleep(&s_bar, phase_bit)) {
+                record_fault(p.fault, HY_FAULT_FILTER_MMA);
+                s_abort = 1;
+            }
+        }
+        phase_bit ^= 1;
+        __syncthreads();
+        tc::fence_after();
+    };
+    // activation of this warp's half of the units of TMEM columns dcol ..
+    // (plus bias[u] when given) into chunk columns of the first operand
+    auto activate = [&](uint32_t trow, uint32_t dcol, int hp, int Hn, const float *bias, int pos, int hc) {
+        const int ub = hc * (hp / 2), ue = ub + hp / 2;
+        uint32_t x[4][8];
+#pragma unroll
+        for (int g8 = 0; g8 < 4; ++g8)
+            if (ub + 8 * g8 < ue) tc::tmem_ld8(trow + dcol + (uint32_t)(ub + 8 * g8), x[g8]);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int g8 = 0; g8 < 4; ++g8) {
+            const int u0 = ub + 8 * g8;
+            if (u0 >= ue) break;
+            float a[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float xv = __uint_as_float(x[g8][j]);
+                if (bias) xv += bias[u0 + j];
+                if constexpr (ACT == HY_ACT_SILU) xv = xv * rcp_fast(1.f + ex2_fast(-kLog2e * xv));
+                else if constexpr (ACT == HY_ACT_SINE) xv = sinf(xv);
+                a[j] = u0 + j < Hn ? xv : 0.f;
+            }
+            put_row(a_hi, a_lo, TP, pos, u0 / 8, a);
+        }
+    };
+    const uint32_t idesc0 = tc::idesc_f16(128, h1p, false);
+    const uint32_t idesc1 = tc::idesc_f16(128, h2p, false);
+    const uint32_t idesc2 = tc::idesc_f16(128, npad, false);
+    constexpr uint32_t D1_COL = 64, D2_COL = 128;
+    const int q4 = warp & 3, hc = warp >> 2;
+    const int pos = 32 * q4 + lane;            // this thread's position in the tile (its TMEM lane)
+    const uint32_t trow = s_tmem + ((uint32_t)(32 * q4) << 16);
+    const bool narrow = p.L * (int64_t)(p.F + 1) < (1LL << 31) && p.L <= (1 << 24);
+    const float Lf = (float)p.L, invL = 1.f / Lf;   // exact when L is a power of two
+    int cur_slice = -1;
+    for (int64_t bt = blockIdx.x; bt < ntiles; bt += gridDim.x) {
+        __syncthreads();                       // operands / TMEM of the previous tile released
+        tc::fence_after();
+        if (s_abort) break;                    // uniform: read between two barriers
+        const int64_t qq = bt * TP + pos;
+        const bool in = qq < p.npos;
+        int r0 = 0, r1 = 0, r2 = 0;
+        float nrm;
+        bool valid = in;
+        if constexpr (NDIM == 3) {
+            const int S = p.S, ls = p.log_s;
+            r0 = signed_off((int)(qq >> (2 * ls)) & (S - 1), S);
+            r1 = signed_off((int)(qq >> ls) & (S - 1), S);
+            r2 = signed_off((int)qq & (S - 1), S);
+            valid = in && (p.circular || ((abs(r0) < p.g) && (abs(r1) < p.g) && (abs(r2) < p.g)));
+            nrm = sqrtf((float)(r0 * r0 + r1 * r1 + r2 * r2)) / (float)p.g;
+        } else {
+            if constexpr (FAST1D) nrm = (float)qq * invL;
+            else nrm = narrow ? __fdiv_rn((float)qq, Lf) : (float)((double)qq / (double)p.L);
+        }
+        // ---- encoding into A (up to two atoms): the two warps of a lane
+        //      quadrant take alternate 16-byte chunks
+        for (int c = hc; c < kpad / 8; c += 2) {
+            float v[8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int pp = 4 * c + q;
+                float cs, sn;
+                if (pp < npairs) {
+                    if constexpr (NDIM == 3) {
+                        const int d = pdesc[pp];
+                        const int ax = d & 3;
+                        const int rv = ax == 0 ? r0 : (ax == 1 ? r1 : r2);
+                        const float2 ph = phase[((d >> 2) * rv) & (2 * p.g - 1)];
+                        cs = ph.x;
+                        sn = ph.y;
+                    } else {
+                        const int j = pp + 1;
+                        float arg;
+                        if constexpr (FAST1D) {
+                            const unsigned jt = (unsigned)(j * (int)qq);
+                            arg = (float)(2u * (jt & (unsigned)(p.L - 1))) * invL;
+                        } else if (narrow) {
+                            const unsigned jt = (unsigned)(j * (int)qq);
+                            arg = __fdiv_rn((float)(2u * (jt % (unsigned)p.L)), Lf);
+                        } else {
+                            const int64_t r = ((int64_t)j * qq) % p.L;
+                            arg = (float)(2.0 * (double)r / (double)p.L);
+                        }
+                        sincospif(arg, &sn, &cs);    // angle 2 pi (j t mod L) / L
+                    }
+                } else {
+                    const int kc = 2 * pp;
+                    const int kt = (NDIM == 1 && p.include_t) ? 2 * npairs : -1;
+                    cs = kc == kt ? nrm : (kc == K0 ? 1.f : 0.f);
+                    sn = kc + 1 == kt ? nrm : (kc + 1 == K0 ? 1.f : 0.f);
+                }
+                v[2 * q] = cs;
+                v[2 * q + 1] = sn;
+            }
+            put_row(a_hi, a_lo, TP, pos, c, v);
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        // ---- first hidden layer (its argument: biases and FiLM folded)
+        run_mma(b0_hi, b0_lo, h1p, idesc0, 0u, kpad / 16);
+        if (s_abort) break;
+        activate(trow, 0u, h1p, H1, nullptr, pos, hc);
+        tc::fence_before();
+        fence_proxy_async_smem();
+        __syncthreads();
+        // ---- second hidden layer
+        run_mma(b1_hi, b1_lo, h2p, idesc1, D1_COL, h1p / 16);
+        if (s_abort) break;
+        activate(trow, D1_COL, h2p, H2, bias1, pos, hc);
+        tc::fence_before();
+        fence_proxy_async_smem();
+        // ---- the output slices of this CTA
+        for (int sl = blockIdx.z; sl < p.t_nslices; sl += gridDim.z) {
+            const int obase = sl * p.t_slice;
+            const int oend = min(nout, obase + p.t_slice);
+            __syncthreads();                   // A written; the last MMA and TMEM reads done
+            if (sl != cur_slice) {
+                load_slice(sl);
+                cur_slice = sl;
+                fence_proxy_async_smem();
+                __syncthreads();
+            }
+            run_mma(b2_hi, b2_lo, npad, idesc2, D2_COL, h2p / 16);
+            if (s_abort) break;
+            float nr = nrm;
+            if (p.window == HY_WIN_GAUSS) nr *= nr;
+            const float nrn = valid ? -nr : 0.f;
+            for (int c0 = 16 * hc; c0 < npad; c0 += 32) {
+                __syncwarp();                  // tcgen05.ld is warp-wide
+                uint32_t v[16];
+                tc::tmem_ld16(trow + D2_COL + (uint32_t)c0, v);
+                tc::tmem_wait_ld();
+                float y[16];
+#pragma unroll
+                for (int j4 = 0; j4 < 4; ++j4) {
+                    const float4 a4 = *reinterpret_cast<const float4 *>(al2 + c0 + 4 * j4);
+                    const float4 b4 = *reinterpret_cast<const float4 *>(bias2 + c0 + 4 * j4);
+                    y[4 * j4 + 0] = (__uint_as_float(v[4 * j4 + 0]) + b4.x) * ex2_fast(a4.x * nrn);
+                    y[4 * j4 + 1] = (__uint_as_float(v[4 * j4 + 1]) + b4.y) * ex2_fast(a4.y * nrn);
+                    y[4 * j4 + 2] = (__uint_as_float(v[4 * j4 + 2]) + b4.z) * ex2_fast(a4.z * nrn);
+                    y[4 * j4 + 3] = (__uint_as_float(v[4 * j4 + 3]) + b4.w) * ex2_fast(a4.w * nrn);
+                }
+                const int ob = obase + c0;
+                float *dst = p.h + ((int64_t)set * nout + ob) * p.npos + qq;
+                if (in && ob + 16 <= oend) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j, dst += p.npos) *dst = valid ? y[j] : 0.f;
+                } else if (in) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j, dst += p.npos)
+                        if (ob + j < oend) *dst = valid ? y[j] : 0.f;
+                }
+            }
+            tc::fence_before();
+        }
+        if (s_abort) break;
+    }
+    // no MMA may still be running when TMEM is freed (all were waited on;
+    // this covers one whose wait gave up)
+    if (tid == 0) {
+        tc::commit(&s_bar);
+        if (!mbar_wait_sleep(&s_bar, phase_bit)) record_fault(p.fault, HY_FAULT_FILTER_MMA);
+    }
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    __syncwarp();
+    if (warp == 0) tc::tmem_free(s_tmem, p.t_cols);
+}
+
 // Engine of the layers: HYENA_FILTER_ENGINE=simt keeps them on the FP32
 // pipes, =tensor_last puts only the last layer on the tensor cores, =tensor
 // (or unset) both layers of a one-hidden-layer MLP where that kernel applies,
@@ -1163,6 +1491,59 @@ hy_status launch_filter_gen(const hy_filter_desc &d, float *h, cudaStream_t s) {
                 dim3 grid((unsigned)per_set, (unsigned)d.n_sets, (unsigned)nslices);
                 kern<<<grid, NT, smem, s>>>(q);
                 return check_launch("filter_gen (two tensor-core layers) launch");
+            }
+        }
+    }
+    // All three layers on the tensor cores: two hidden layers of <= 64 units,
+    // input width <= 127, fewer 128-position tiles than SMs and at least 256
+    // outputs.  One CTA per (tile, set, slice group): grid z splits the
+    // 128-output slices so that the CTAs about fill the SMs.
+    {
+        GenParams q = p;
+        const int64_t ntiles = (q.npos + TP - 1) / TP;
+        const int eng = filter_engine();
+        if ((eng == 1 || eng == 2) && q.nl == 3 && q.widths[0] <= 127 && q.widths[1] <= 64 && q.widths[2] <= 64 &&
+            q.widths[3] >= 256 && ntiles * d.n_sets < sms) {
+            const int nout = q.widths[3];
+            q.t_slice = 128;
+            q.t_nslices = (nout + 127) / 128;
+            int zsplit = (int)(sms / (ntiles * d.n_sets));
+            if (zsplit < 1) zsplit = 1;
+            if (zsplit > q.t_nslices) zsplit = q.t_nslices;
+            q.t_kpad = (q.widths[0] + 1 + 15) & ~15;
+            q.t_hpad = (q.widths[1] + 15) & ~15;
+            q.t_h2pad = (q.widths[2] + 15) & ~15;
+            q.t_npad = 128;
+            q.t_cols = 256;
+            q.fault = device_fault_word();
+            if (!q.fault) return set_error(HY_ERR_CUDA, "device fault word unavailable");
+            const int ka = (q.t_kpad + 63) / 64;
+            const size_t smem = 1024 + (size_t)2 * TC_ROW * (ka * TP + ka * q.t_hpad + q.t_h2pad + q.t_npad) +
+                                sizeof(float) * (64 + 2 * (size_t)q.t_npad) + sizeof(int) * 64 +
+                                (q.ndim == 3 ? (size_t)16 * q.g : 0);
+            if (smem <= (size_t)227 * 1024) {
+                void (*kern)(const GenParams) = nullptr;
+                const bool fast1d = q.L * (int64_t)(q.F + 1) < (1LL << 31) && q.L <= (1 << 24) && (q.L & (q.L - 1)) == 0;
+                if (q.ndim == 3)
+                    kern = q.act == HY_ACT_SILU ? filter_gen_tc3_kernel<3, HY_ACT_SILU, false>
+                         : q.act == HY_ACT_SINE ? filter_gen_tc3_kernel<3, HY_ACT_SINE, false>
+                                                : filter_gen_tc3_kernel<3, HY_ACT_IDENTITY, false>;
+                else if (fast1d)
+                    kern = q.act == HY_ACT_SILU ? filter_gen_tc3_kernel<1, HY_ACT_SILU, true>
+                         : q.act == HY_ACT_SINE ? filter_gen_tc3_kernel<1, HY_ACT_SINE, true>
+                                                : filter_gen_tc3_kernel<1, HY_ACT_IDENTITY, true>;
+                else
+                    kern = q.act == HY_ACT_SILU ? filter_gen_tc3_kernel<1, HY_ACT_SILU, false>
+                         : q.act == HY_ACT_SINE ? filter_gen_tc3_kernel<1, HY_ACT_SINE, false>
+                                                : filter_gen_tc3_kernel<1, HY_ACT_IDENTITY, false>;
+                cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+                if (e != cudaSuccess) return set_cuda_error("filter_gen three-layer smem attribute", e);
+                e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         (int)cudaSharedmemCarveoutMaxShared);
+                if (e != cudaSuccess) return set_cuda_error("filter_gen carve-out attribute", e);
+                dim3 grid((unsigned)ntiles, (unsigned)d.n_sets, (unsigned)zsplit);
+                kern<<<grid, NT, smem, s>>>(q);
+                return check_launch("filter_gen (three tensor-core layers) launch");
             }
         }
     }

@@ -220,6 +220,31 @@ def test_nd_filter_gen_tensor_core_grid(act, hidden, nout, engine, monkeypatch):
         check(got[b].reshape(nout, -1), ref.T, "f32", "3-D filters g16 %s %s set %d" % (act, engine, b))
 
 
+def test_nd_filter_gen_three_layers_few_tiles():
+    """3-D filters with two hidden layers and 300 outputs on a small grid
+    (g = 8: 16^3 positions = 32 tiles per set, two FiLM sets): all three
+    layers on the tensor cores with grid z = 2 over the 3 output slices (the
+    last one 44 wide); every voxel and output against the oracle."""
+    g, F, nout = 8, 3, 300
+    rng = np.random.default_rng(8300)
+    widths = [6 * F, 64, 32, nout]
+    Ws = [rng.uniform(-1, 1, (b, a)).astype(np.float32) / np.sqrt(a) for a, b in zip(widths[:-1], widths[1:])]
+    bs = [rng.uniform(-0.5, 0.5, b).astype(np.float32) for b in widths[1:]]
+    alpha = rng.uniform(0.5, 3.0, nout).astype(np.float32)
+    gam = rng.normal(0, 0.1, (2, 64)).astype(np.float32)
+    bet = rng.normal(0, 0.1, (2, 64)).astype(np.float32)
+    S = 2 * g
+    h = torch.empty((2, nout, S, S, S), device="cuda")
+    hy.hyena_filter_gen(h, ndim=3, grid=g, Ws=[f32_dev(a) for a in Ws], bs=[f32_dev(a) for a in bs],
+                        alpha=f32_dev(alpha), n_freq=F, film_gamma=f32_dev(gam), film_beta=f32_dev(bet), n_sets=2)
+    torch.cuda.synchronize()
+    got = to_np(h)
+    idx = np.arange(S ** 3)
+    for b in range(2):
+        ref = oracle.filter_gen_3d_points(g, False, F, Ws, bs, gam[b], bet[b], alpha, idx)
+        check(got[b].reshape(nout, -1), ref.T, "f32", "three-layer 3-D filters set %d" % b)
+
+
 @pytest.mark.parametrize("circular", [False, True])
 def test_nd_filter_gen_siren_gaussian(circular):
     """HyenaND kernel synthesis: SIREN hidden layers (sin of per-unit

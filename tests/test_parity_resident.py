@@ -112,9 +112,10 @@ def test_fftconv_gate_skip_variants_and_guard_bands():
 @pytest.mark.parametrize("engine", ["default", "simt"])
 def test_filter_gen_1d_vs_oracle(engine, monkeypatch):
     """The filters of workloads 1-3 (c3 at L = 4096) with the default engine
-    choice and with HYENA_FILTER_ENGINE=simt (FP32-pipe kernels); these
-    lengths have too few position tiles for the tensor-core last layer, so
-    both run the streaming kernel."""
+    choice and with HYENA_FILTER_ENGINE=simt (FP32-pipe kernels).  These
+    lengths have fewer 128-position tiles than SMs: by default workload 2's
+    three layers and 768 outputs run all on the tensor cores (one CTA per
+    tile and slice group); the others run the streaming kernel."""
     if engine == "simt":
         monkeypatch.setenv("HYENA_FILTER_ENGINE", "simt")
     for name, L in [("c1", 1024), ("c2", 8192), ("c3", 4096)]:
@@ -352,6 +353,31 @@ def test_filter_gen_two_layers_length_not_power_of_two(act):
     torch.cuda.synchronize()
     ref = oracle.filter_gen_1d(L, F, True, Ws, bs, alpha, act=act, omega=omega)
     check(to_np(h), ref, "f32", "two-layer filters L=%d (%s)" % (L, act))
+
+
+@pytest.mark.parametrize("act", ["silu", "sine"])
+def test_filter_gen_three_layers_few_tiles(act):
+    """Two hidden layers and many outputs over fewer 128-position tiles than
+    SMs (L = 5000: 40 tiles; 600 outputs): all three layers on the tensor
+    cores, each CTA one tile and a group of 128-output slices (grid z = 3:
+    slices 0, 3 / 1, 4 / 2, the last one ragged at 88 outputs); an 81-wide
+    encoding (two 64-column operand atoms), hidden widths 48 and 40 (padded
+    to 48), SiLU or SIREN; every position and output against the oracle."""
+    L, F = 5000, 40
+    rng = np.random.default_rng(5003 + (act == "sine"))
+    widths = [1 + 2 * F, 48, 40, 600]
+    Ws = [rng.uniform(-1, 1, (b, a)).astype(np.float32) / np.sqrt(a) for a, b in zip(widths[:-1], widths[1:])]
+    bs = [rng.uniform(-0.5, 0.5, b).astype(np.float32) for b in widths[1:]]
+    alpha = rng.uniform(0.1, 2.0, widths[-1]).astype(np.float32)
+    omega = rng.uniform(1, 3, 48 + 40).astype(np.float32) if act == "sine" else None
+    h = torch.empty((widths[-1], L), device="cuda")
+    hy.hyena_filter_gen(h, ndim=1, L=L, Ws=[f32_dev(a) for a in Ws], bs=[f32_dev(a) for a in bs],
+                        alpha=f32_dev(alpha), n_freq=F, include_t=True,
+                        act=hy.HY_ACT_SINE if act == "sine" else hy.HY_ACT_SILU,
+                        omega=f32_dev(omega) if omega is not None else None)
+    torch.cuda.synchronize()
+    ref = oracle.filter_gen_1d(L, F, True, Ws, bs, alpha, act=act, omega=omega)
+    check(to_np(h), ref, "f32", "three-layer filters L=5000 (%s)" % act)
 
 
 @pytest.mark.parametrize("engine", ["default", "simt", "tensor_last"])

@@ -116,8 +116,12 @@ typedef struct hy_filter_desc {
 
 /* Writes h (device, fp32): 1-D (n_sets, n_out, L); 3-D (n_sets, n_out, S, S, S).
  * With at least one 128-position tile per SM the layers run on the tensor
- * cores: both of them for one hidden layer with input and hidden widths
- * <= 64, else the last one (after at least one hidden layer of width <= 128).
+ * cores: both of them for one hidden layer with input width <= 63 and hidden
+ * width <= 64, else the last one (after at least one hidden layer of width
+ * <= 128).  With fewer tiles, two hidden layers of <= 64 units, an input
+ * width <= 127 and at least 256 outputs, all three layers do (one CTA per
+ * tile and group of 128-output slices); other small cases stay on the FP32
+ * pipes.
  * Their inputs and weights are split into fp16 hi + lo (relative error
  * <= 2^-22, fp32 accumulation), which assumes their magnitudes stay below
  * 65504 (the encodings here are bounded and the hidden units O(1)).  The

@@ -171,6 +171,41 @@ def test_host_entry_validation_and_workspace(lib):
                 "workspace") == 3
 
 
+def test_chunk_pipeline_workspaces(lib):
+    """The workspace queries of the chunked paths return one chunk buffer per
+    chunk pipeline that can be busy: two when the rows (slabs) take more than
+    one chunk, else one chunk of exactly the rows; the calls accept one chunk
+    buffer as the minimum (checked on the host: a byte less is refused)."""
+    MB = 1 << 20
+    row = 8 << 20                                    # L = 2^20: M = 2^20 complex points of 8 bytes
+    cr = (104 * MB) // row                           # 13 rows per chunk
+    assert cr == 13
+    assert lib.hyena_operator_workspace(3, 1, 256, 1 << 20, 0) == 2 * cr * row
+    assert lib.hyena_operator_workspace(3, 1, 14, 1 << 20, 0) == 2 * cr * row
+    assert lib.hyena_operator_workspace(3, 1, 13, 1 << 20, 0) == cr * row
+    assert lib.hyena_operator_workspace(2, 1, 5, 1 << 20, 1) == 5 * row
+    one = (ctypes.c_int * 1)(1 << 20)
+    assert lib.hyena_filter_spectrum_workspace(512, 1, one, 0) == 2 * cr * row
+    assert lib.hyena_filter_spectrum_workspace(13, 1, one, 0) == cr * row
+    dims = (ctypes.c_int * 3)(64, 64, 64)
+    per_c = 64 * 128 * 65 * 8                        # one slab's planes of the 3-D convolution
+    cs = (80 * MB) // per_c                          # 19 slabs per chunk
+    assert lib.hyena_nd_conv_workspace(3, dims, 1, 40, 0) == 2 * cs * per_c
+    assert lib.hyena_nd_conv_workspace(3, dims, 2, 19, 0) == 2 * cs * per_c
+    assert lib.hyena_nd_conv_workspace(3, dims, 1, 19, 0) == cs * per_c
+    assert lib.hyena_nd_conv_workspace(3, dims, 1, 5, 0) == 5 * per_c
+    per_s = 128 * 128 * 65 * 8                       # one 128^3 kernel's planes of the 3-D spectrum
+    assert lib.hyena_filter_spectrum_workspace(40, 3, dims, 0) == 2 * ((80 * MB) // per_s) * per_s
+    assert lib.hyena_filter_spectrum_workspace(9, 3, dims, 0) == 9 * per_s
+    # the minimum accepted: one chunk buffer (a byte less is a workspace error)
+    far = 1 << 40                                    # fake device addresses far apart (no overlap)
+    X2 = (ctypes.c_void_p * 2)(2 * far, 3 * far)
+    H2 = (ctypes.c_void_p * 2)(5 * far, 6 * far)
+    st = lib.hyena_operator(3, 1, 14, 1 << 20, 0, ctypes.c_void_p(far), X2, H2, None, ctypes.c_void_p(4 * far),
+                            ctypes.c_void_p(7 * far), ctypes.c_size_t(cr * row - 1), None)
+    assert _err(lib, st, "workspace") == 3
+
+
 def test_binding_raises_named_errors(lib):
     with pytest.raises(hy.HyenaError) as ei:
         hy._check(lib.spectral_gate(1, 1, 1, 100, 1, FAKE, FAKE, 0, None, FAKE * 2, None))

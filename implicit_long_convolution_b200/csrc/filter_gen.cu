@@ -20,8 +20,11 @@
 // Hidden outputs get bias, FiLM and the activation and stay in shared
 // memory; last-layer outputs get bias and the decay window and go straight
 // to HBM as float4 row segments.  With many positions per filter set the
-// weights stay resident in persistent CTAs, and the last layer runs on the
-// tensor cores (filter_gen_tc_kernel) where its shape allows.
+// weights stay resident in persistent CTAs, and the layers run on the
+// tensor cores where their shapes allow: every layer of a one-hidden-layer
+// MLP (filter_gen_tc2_kernel), every layer of a two-hidden-layer MLP over
+// few positions with many outputs (filter_gen_tc3_kernel), else the last
+// layer (filter_gen_tc_kernel).
 #include <cuda_fp16.h>
 #include <cstdlib>
 #include <cstring>
